@@ -1,0 +1,503 @@
+"""Pins for the CPU oracle (no GPU).
+
+Each test checks the oracle against something other than itself: brute force over
+every code of a format, closed forms, invariants, hand-worked fixtures under
+tests/golden/, or an independent library routine (torch's float8 cast, numpy's
+float64 matmul). A plausible slip in the oracle (a dropped term, a wrong sign or
+index, a transposed operand, a wrong tie rule) fails at least one of them.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from mtp_speculative_draft_lm_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+# ---------------------------------------------------------------- helpers (test-side)
+
+def e4m3_table():
+    """All 256 E4M3FN code values decoded by torch (independent of the oracle)."""
+    t = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).float().numpy()
+    return t.astype(np.float64)
+
+
+E2M1_MAG = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def brute_encode(v, mags, sat_code, sign_bit):
+    """Nearest magnitude by linear search over every code, ties to the even code."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    d = np.abs(a[:, None] - mags[None, :])
+    best = d.min(axis=1, keepdims=True)
+    cand = d == best
+    # among equal distances prefer the even code (lowest set bit clear)
+    even = cand & (np.arange(mags.size)[None, :] % 2 == 0)
+    pick = np.where(even.any(axis=1), even.argmax(axis=1), cand.argmax(axis=1))
+    pick = np.where(a >= mags[sat_code], sat_code, pick)
+    sign = np.signbit(v).astype(np.int64) * sign_bit
+    return (pick | sign).astype(np.uint8)
+
+
+def all_bf16_values():
+    bits = np.arange(65536, dtype=np.uint32)
+    f = (bits << 16).view(np.float32).astype(np.float64)
+    return f[~np.isnan(f)]
+
+
+def midpoints_with_neighbours(mags):
+    mids = (mags[1:] + mags[:-1]) / 2
+    f32 = mids.astype(np.float32)
+    up = np.nextafter(f32, np.float32(np.inf)).astype(np.float64)
+    dn = np.nextafter(f32, np.float32(-np.inf)).astype(np.float64)
+    v = np.concatenate([mids, up, dn])
+    return np.concatenate([v, -v])
+
+
+def bf16(a):
+    return torch.tensor(np.asarray(a, dtype=np.float32)).to(torch.bfloat16)
+
+
+def u16(t):
+    return synth.as_u16(t)
+
+
+# ---------------------------------------------------------------- formats
+
+def test_e4m3_decode_matches_torch(orc):
+    ref = e4m3_table()
+    got = orc.e4m3_value(np.arange(256))
+    finite = ~np.isnan(ref)
+    assert np.array_equal(np.isnan(got), ~finite)
+    assert np.array_equal(got[finite], ref[finite])
+    assert orc.e4m3_value([0x7E])[0] == 448.0
+    assert orc.e4m3_value([0x01])[0] == 2.0 ** -9
+
+
+def test_e4m3_encode_bruteforce_all_bf16_and_midpoints(orc):
+    mags = e4m3_table()[:127]  # codes 0x00..0x7E, increasing
+    assert np.all(np.diff(mags) > 0)
+    v = np.concatenate([all_bf16_values(), midpoints_with_neighbours(mags),
+                        [np.inf, -np.inf, 1e30, -1e30]])
+    got = orc.e4m3_encode(v)
+    ref = brute_encode(v, mags, 0x7E, 0x80)
+    bad = np.nonzero(got != ref)[0]
+    assert bad.size == 0, (v[bad[:5]], got[bad[:5]], ref[bad[:5]])
+
+
+def test_e4m3_encode_matches_torch_cast(orc):
+    g = torch.Generator().manual_seed(7)
+    x = torch.randn(200000, generator=g) * torch.exp2(torch.randint(-14, 9, (200000,),
+                                                                    generator=g).float())
+    x = x[x.abs() < 464]
+    ref = x.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = orc.e4m3_encode(x.double().numpy())
+    assert np.array_equal(got, ref)
+
+
+def test_e4m3_sign_and_saturation(orc):
+    assert orc.e4m3_encode([-1e-12])[0] == 0x80
+    assert orc.e4m3_encode([-0.0])[0] == 0x80
+    assert orc.e4m3_encode([0.0])[0] == 0x00
+    assert orc.e4m3_encode([448.0])[0] == 0x7E
+    assert orc.e4m3_encode([1e9])[0] == 0x7E
+    assert orc.e4m3_encode([-1e9])[0] == 0xFE
+    # never the NaN pattern for finite input
+    v = np.linspace(-1000, 1000, 100001)
+    assert not np.any((orc.e4m3_encode(v) & 0x7F) == 0x7F)
+
+
+def test_e2m1_encode_bruteforce_dense_grid(orc):
+    grid = np.arange(-8 * 4096, 8 * 4096 + 1) / 4096.0
+    v = np.concatenate([grid, midpoints_with_neighbours(E2M1_MAG)])
+    got = orc.e2m1_encode(v)
+    ref = brute_encode(v, E2M1_MAG, 7, 8)
+    bad = np.nonzero(got != ref)[0]
+    assert bad.size == 0, (v[bad[:5]], got[bad[:5]], ref[bad[:5]])
+
+
+def test_e2m1_tie_table(orc):
+    # worked special cases: each midpoint goes to the even code
+    ties = {0.25: 0.0, 0.75: 1.0, 1.25: 1.0, 1.75: 2.0, 2.5: 2.0, 3.5: 4.0, 5.0: 4.0}
+    for v, want in ties.items():
+        code = orc.e2m1_encode([v])[0]
+        assert orc.e2m1_value([code])[0] == want, v
+        assert orc.e2m1_value([orc.e2m1_encode([-v])[0]])[0] == -want
+    assert orc.e2m1_encode([-0.1])[0] == 0x8
+    assert orc.e2m1_encode([100.0])[0] == 0x7
+    assert list(orc.e2m1_value(np.arange(8))) == list(E2M1_MAG)
+
+
+def test_bf16_rounding(orc):
+    g = torch.Generator().manual_seed(3)
+    x = torch.randn(100000, generator=g) * 100
+    ref = x.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(orc.f64_to_bf16(x.double().numpy()), ref)
+    # single rounding from the real value: just above a bf16 midpoint rounds up,
+    # although an fp32 intermediate would have made it an exact tie (-> even, down)
+    assert orc.f64_to_bf16([1 + 2 ** -8 + 2 ** -30])[0] == 0x3F81
+    assert orc.f64_to_bf16([1 + 2 ** -8])[0] == 0x3F80  # exact tie -> even
+    assert orc.f64_to_bf16([-0.0])[0] == 0x8000
+
+
+# ---------------------------------------------------------------- RMSNorm
+
+def test_rmsnorm_constant_vector_is_the_weight(orc):
+    h = 96
+    w = u16(synth.normal_bf16(synth._gen(1), (h,), 0.1, 1.0))
+    for c in (0.5, 3.0, -2.0):
+        x = u16(bf16(np.full(h, c)))
+        y = orc.rmsnorm(x, w, 0.0)
+        want = w if c > 0 else (w ^ 0x8000)
+        assert np.array_equal(y, want)
+
+
+def test_rmsnorm_one_hot_and_scale_invariance(orc):
+    h = 64  # sqrt(h) = 8, a power of two: exact
+    w = u16(synth.normal_bf16(synth._gen(2), (h,), 0.1, 1.0))
+    x = np.zeros(h, np.float32)
+    x[17] = 0.37
+    y = orc.rmsnorm(u16(bf16(x)), w, 0.0)
+    wf = orc.bf16_to_f64(w)
+    assert orc.bf16_to_f64(y)[17] == wf[17] * 8.0
+    assert np.all(orc.bf16_to_f64(y)[np.arange(h) != 17] == 0)
+    xr = u16(synth.normal_bf16(synth._gen(3), (h,), 1.0))
+    x4 = orc.f64_to_bf16(orc.bf16_to_f64(xr) * 4.0)
+    assert np.array_equal(orc.rmsnorm(xr, w, 0.0), orc.rmsnorm(x4, w, 0.0))
+
+
+def test_rmsnorm_unit_rms_and_library(orc):
+    h = 512
+    ones = u16(bf16(np.ones(h)))
+    x = u16(synth.normal_bf16(synth._gen(4), (h,), 3.0))
+    y = orc.bf16_to_f64(orc.rmsnorm(x, ones, 0.0))
+    assert abs(np.mean(y * y) - 1.0) < 2 ** -7
+    xf = orc.bf16_to_f64(x)
+    eps = 1e-6
+    ref = xf / (np.linalg.norm(xf) / math.sqrt(h) * math.sqrt(1 + eps * h / np.dot(xf, xf)))
+    assert np.allclose(y, ref, rtol=2 ** -8, atol=0)
+    assert np.all(orc.rmsnorm(np.zeros(h, np.uint16), ones, 1e-6) == 0)
+
+
+# ---------------------------------------------------------------- combiner
+
+def tiny(h=32, vocab=50, M=3, seed=11):
+    d = synth.tiny_draft(seed=seed, vocab=vocab, h=h, M=M)
+    return {k: (u16(v) if isinstance(v, torch.Tensor) and v.dtype == torch.bfloat16 else v)
+            for k, v in d.items()}
+
+
+def test_combine_one_hot_selects_fc_column(orc):
+    d = tiny()
+    h = d["h"]
+    j = 5
+    w_ne = np.zeros(h, np.float32)
+    w_ne[j] = 1.0
+    embed = d["embed"].copy()
+    embed[3] = u16(bf16(np.full(h, 0.25)))
+    y, concat, flags = orc.combine(embed, [3], d["hidden"][:1], u16(bf16(w_ne)),
+                                   np.zeros(h, np.uint16), 0.0, d["fc"])
+    assert flags == 0
+    assert np.array_equal(y[0], d["fc"][:, j])
+    assert np.all(orc.bf16_to_f64(concat[0, h:]) == 0)
+
+
+def test_combine_embedding_half_only_and_order(orc):
+    d = tiny()
+    h = d["h"]
+    y, concat, _ = orc.combine(d["embed"], d["tokens"], d["hidden"], d["w_norm_embed"],
+                               np.zeros(h, np.uint16), d["eps"], d["fc"])
+    for m in range(d["hidden"].shape[0]):
+        ne = orc.rmsnorm(d["embed"][d["tokens"][m]], d["w_norm_embed"], d["eps"])
+        assert np.array_equal(concat[m, :h], ne)
+        ref = orc.bf16_to_f64(d["fc"])[:, :h] @ orc.bf16_to_f64(ne)
+        assert np.array_equal(y[m], orc.f64_to_bf16(ref))
+
+
+def test_combine_full_matches_numpy(orc):
+    d = tiny(h=4, vocab=9, M=2)
+    y, concat, _ = orc.combine(d["embed"], d["tokens"], d["hidden"], d["w_norm_embed"],
+                               d["w_norm_hidden"], d["eps"], d["fc"])
+    for m in range(2):
+        nh = orc.rmsnorm(d["hidden"][m], d["w_norm_hidden"], d["eps"])
+        assert np.array_equal(concat[m, 4:], nh)
+        ref = orc.bf16_to_f64(d["fc"]) @ orc.bf16_to_f64(concat[m])
+        assert np.array_equal(y[m], orc.f64_to_bf16(ref))
+
+
+def test_combine_bad_token_flags_and_zeroes(orc):
+    d = tiny()
+    y, concat, flags = orc.combine(d["embed"], [d["vocab"]], d["hidden"][:1],
+                                   d["w_norm_embed"], d["w_norm_hidden"], d["eps"], d["fc"])
+    assert flags & orc.FLAG_BAD_TOKEN
+    assert np.all(orc.bf16_to_f64(concat[0, : d["h"]]) == 0)
+
+
+# ---------------------------------------------------------------- lm_head + argmax
+
+def quantized(orc, W, fmt):
+    if fmt == orc.FMT_BF16:
+        return dict(data=W)
+    if fmt == orc.FMT_FP8_ROW:
+        c, s = orc.quantize_fp8(W)
+        return dict(data=c, row_scale=s)
+    c, b, g = orc.quantize_nvfp4(W)
+    return dict(data=c, block_scale=b, global_scale=g)
+
+
+def independent_dequant(orc, fmt, q, k):
+    """Dequantize with torch's float8 decode and a literal E2M1 table."""
+    if fmt == orc.FMT_BF16:
+        return orc.bf16_to_f64(q["data"])
+    t8 = e4m3_table()
+    if fmt == orc.FMT_FP8_ROW:
+        return t8[q["data"]] * q["row_scale"].astype(np.float64)[:, None]
+    lo = q["data"] & 0xF
+    hi = q["data"] >> 4
+    codes = np.stack([lo, hi], axis=2).reshape(q["data"].shape[0], k)
+    mag = E2M1_MAG[codes & 7] * np.where(codes & 8, -1.0, 1.0)
+    sc = np.repeat(t8[q["block_scale"]], 16, axis=1)
+    return mag * sc * np.float64(np.float32(q["global_scale"]))
+
+
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+def test_lm_head_one_hot_selects_entries(orc, fmt):
+    N, K = 37, 64
+    W = u16(synth.normal_bf16(synth._gen(21), (N, K), 0.02))
+    q = quantized(orc, W, fmt)
+    deq = independent_dequant(orc, fmt, q, K)
+    for j in (0, 17, K - 1):
+        x = np.zeros(K, np.float32)
+        x[j] = 1.0
+        logits, _, _, _ = orc.lm_head_argmax(fmt, q["data"], K, u16(bf16(x)),
+                                             row_scale=q.get("row_scale"),
+                                             block_scale=q.get("block_scale"),
+                                             global_scale=q.get("global_scale", 0.0))
+        assert np.array_equal(logits[0], deq[:, j])
+
+
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+def test_lm_head_matches_numpy_matmul(orc, fmt):
+    N, K, M = 37, 32, 3
+    W = u16(synth.normal_bf16(synth._gen(22), (N, K), 0.02))
+    x = u16(synth.normal_bf16(synth._gen(23), (M, K), 1.0))
+    q = quantized(orc, W, fmt)
+    logits, idx, val, flags = orc.lm_head_argmax(fmt, q["data"], K, x,
+                                                 row_scale=q.get("row_scale"),
+                                                 block_scale=q.get("block_scale"),
+                                                 global_scale=q.get("global_scale", 0.0))
+    ref = orc.bf16_to_f64(x) @ independent_dequant(orc, fmt, q, K).T
+    assert np.allclose(logits, ref, rtol=1e-13, atol=1e-15)
+    assert np.array_equal(idx, ref.argmax(axis=1)) and flags == 0
+    assert np.array_equal(val, ref.max(axis=1))
+
+
+def test_lm_head_n_eff_limits_rows(orc):
+    d = synth.head_table(31, 200, 64, 2)
+    W, x = u16(d["W"]), u16(d["x"])
+    full, _, _, _ = orc.lm_head_argmax(0, W, 64, x)
+    part, idx, _, _ = orc.lm_head_argmax(0, W, 64, x, n_eff=150)
+    assert part.shape == (2, 150)
+    assert np.array_equal(part, full[:, :150])
+    assert np.array_equal(idx, full[:, :150].argmax(axis=1))
+
+
+def test_argmax_planted_and_masked_decoy(orc):
+    d = synth.head_table(41, 3000, 128, 4, mask_keep=0.1)
+    W, x = u16(d["W"]), u16(d["x"])
+    logits, idx, val, flags = orc.lm_head_argmax(0, W, 128, x)
+    assert np.array_equal(idx, d["top"]) and flags == 0
+    words = d["mask"].shape[1]
+    mlog, midx, mval, mflags = orc.lm_head_argmax(0, W, 128, x, mask=d["mask"],
+                                                  mask_words=words, mask_stride_words=words)
+    assert np.array_equal(midx, d["second"]) and mflags == 0
+    for m in range(4):
+        assert mlog[m, d["top"][m]] > mval[m]  # the decoy is larger but masked
+        allowed = d["allowed"][m]
+        assert mval[m] == logits[m][allowed].max()
+        srt = np.sort(logits[m])
+        assert srt[-1] - srt[-2] >= 0.5  # planted gap
+
+
+def test_argmax_ties_lowest_index_and_empty_mask(orc):
+    d = synth.head_table(51, 100, 64, 1)
+    W = u16(d["W"]).copy()
+    top = int(d["top"][0])
+    dup = [3, top, 60] if top > 3 else [top, 70, 80]
+    for r in dup:
+        W[r] = W[top]
+    _, idx, _, _ = orc.lm_head_argmax(0, W, 64, u16(d["x"]))
+    assert idx[0] == min(dup)
+    # all tokens masked -> index 0, value -inf, flag
+    mask = np.zeros((1, 4), np.int32)
+    _, idx, val, flags = orc.lm_head_argmax(0, W, 64, u16(d["x"]), mask=mask, mask_words=4)
+    assert idx[0] == 0 and val[0] == -np.inf and flags & orc.FLAG_EMPTY_MASK
+    # words past the mask length disallow: only tokens 0..31 are reachable
+    mask = np.full((1, 1), -1, np.int32)
+    logits, idx, _, _ = orc.lm_head_argmax(0, W, 64, u16(d["x"]), mask=mask, mask_words=1)
+    assert idx[0] == int(np.argmax(logits[0, :32]))
+    # a shared mask (stride 0) applies to every row
+    d2 = synth.head_table(52, 100, 64, 3)
+    mask = synth.pack_mask(np.arange(100)[None, :] % 2 == 1)
+    logits, idx, _, _ = orc.lm_head_argmax(0, u16(d2["W"]), 64, u16(d2["x"]), mask=mask,
+                                           mask_words=mask.shape[1], mask_stride_words=0)
+    for m in range(3):
+        assert idx[m] == 1 + 2 * int(np.argmax(logits[m, 1::2]))
+
+
+def test_argmax_negative_zero_equals_zero(orc):
+    i, v, f = orc.argmax_masked(np.array([-0.0, 0.0, -1.0]))
+    assert i == 0 and f == 0
+    i, v, f = orc.argmax_masked(np.array([-1.0, 0.0, -0.0]))
+    assert i == 1
+
+
+# ---------------------------------------------------------------- quantizers
+
+def test_fp8_quantizer_matches_torch_and_bounds(orc):
+    W = u16(synth.normal_bf16(synth._gen(61), (64, 256), 0.02))
+    W[5] = 0  # zero row
+    codes, scale = orc.quantize_fp8(W)
+    Wt = torch.tensor(W.view(np.int16)).view(torch.bfloat16).float()
+    a = Wt.abs().amax(dim=1)
+    s = a / 448.0
+    assert np.array_equal(scale, s.numpy())
+    nz = a > 0
+    ref = (Wt[nz] / s[nz, None]).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(codes[nz.numpy()], ref)
+    assert scale[5] == 0 and np.all(codes[5] == 0)
+    # the absmax element of every row encodes to +-448
+    wf = orc.bf16_to_f64(W)
+    for r in np.nonzero(nz.numpy())[0]:
+        j = int(np.argmax(np.abs(wf[r])))
+        assert codes[r, j] in (0x7E, 0xFE)
+    # round trip: relative 2^-4 for normals, absolute 2^-10 * s below
+    deq = e4m3_table()[codes] * scale.astype(np.float64)[:, None]
+    q = np.abs(wf) / np.where(scale > 0, scale, 1)[:, None]
+    bound = np.where(q >= 2 ** -6, 2 ** -4 * np.abs(wf), 2 ** -10 * scale[:, None])
+    assert np.all(np.abs(deq - wf) <= bound + 1e-30)
+
+
+def load_golden_nvfp4():
+    vals = {}
+    with open(os.path.join(GOLDEN, "nvfp4_block.txt")) as f:
+        for line in f:
+            if line.startswith("#") or ":" not in line:
+                continue
+            key, rest = line.split(":", 1)
+            vals[key.strip()] = rest.split()
+    return vals
+
+
+def test_nvfp4_golden_block(orc):
+    gold = load_golden_nvfp4()
+    w = u16(bf16([float(v) for v in gold["values"]]))[None, :]
+    codes, bscale, g = orc.quantize_nvfp4(w)
+    assert g == float(gold["global_scale"][0])
+    assert list(bscale[0]) == [int(v, 16) for v in gold["block_scales"]]
+    assert list(codes[0]) == [int(v, 16) for v in gold["codes"]]
+
+
+def test_nvfp4_quantizer_bounds(orc):
+    W = u16(synth.normal_bf16(synth._gen(71), (48, 320), 0.02))
+    codes, bscale, g = orc.quantize_nvfp4(W)
+    wf = orc.bf16_to_f64(W)
+    A = np.abs(wf).max()
+    assert g == np.float32(np.float32(A) / np.float32(2688.0))
+    t8 = e4m3_table()
+    assert np.all(bscale <= 0x7E)  # positive, finite, <= 448
+    blocks = np.abs(wf).reshape(48, 20, 16).max(axis=2)
+    r, b = np.unravel_index(np.argmax(blocks), blocks.shape)
+    assert bscale[r, b] == 0x7E  # the block holding the global max gets 448
+    S = (t8[bscale].astype(np.float32) * np.float32(g)).astype(np.float64)
+    deq = independent_dequant(orc, 2, dict(data=codes, block_scale=bscale, global_scale=g), 320)
+    Sx = np.repeat(S, 16, axis=1)
+    a = np.abs(wf) / Sx
+    step = np.where(a <= 2, 0.25, np.where(a <= 4, 0.5, 1.0)) * Sx
+    bound = step + np.maximum(0.0, np.abs(wf) - 6 * Sx)
+    assert np.all(np.abs(deq - wf) <= bound * (1 + 1e-6))
+    z, zb, zg = orc.quantize_nvfp4(np.zeros((2, 32), np.uint16))
+    assert zg == 1.0 and np.all(zb == 0) and np.all(z == 0)
+
+
+# ---------------------------------------------------------------- RoPE / slots / KV
+
+def test_rope_identities(orc):
+    rng = np.random.default_rng(5)
+    k = rng.standard_normal(128)
+    assert np.array_equal(orc.rope_neox(k, 0, 1e6), k)
+    r = orc.rope_neox(k, 1234, 1e6)
+    assert np.allclose(k[:64] ** 2 + k[64:] ** 2, r[:64] ** 2 + r[64:] ** 2, rtol=1e-12)
+    one = orc.rope_neox(k, 1, 1e6)
+    rot = np.array([[math.cos(1), -math.sin(1)], [math.sin(1), math.cos(1)]])
+    assert np.allclose(rot @ np.array([k[0], k[64]]), [one[0], one[64]], rtol=1e-15)
+    assert np.allclose(orc.rope_neox(orc.rope_neox(k, 300, 1e6), 77, 1e6),
+                       orc.rope_neox(k, 377, 1e6), rtol=1e-9, atol=1e-12)
+    # the last pair turns slowest: theta = pos * base^(-126/128)
+    th = 1000 * 1e6 ** (-126 / 128)
+    r = orc.rope_neox(k, 1000, 1e6)
+    assert np.isclose(r[63], k[63] * math.cos(th) - k[127] * math.sin(th), rtol=1e-12)
+
+
+def test_slot_golden_cases(orc):
+    with open(os.path.join(GOLDEN, "slot_cases.txt")) as f:
+        rows = [l.split() for l in f if l.strip() and not l.startswith("#")]
+    assert len(rows) >= 8
+    for bt, nb, p, want in rows:
+        table = [int(v) for v in bt.split(",")]
+        assert orc.slot(table, 16, int(nb), int(p)) == int(want), (bt, p)
+
+
+def test_kv_encode_matches_torch(orc):
+    v = u16(synth.normal_bf16(synth._gen(81), (4096,), 3.0))
+    vt = torch.tensor(v.view(np.int16)).view(torch.bfloat16).float()
+    assert np.array_equal(orc.kv_encode(v, 1.0), vt.to(torch.float8_e4m3fn).view(torch.uint8).numpy())
+    assert np.array_equal(orc.kv_encode(v, 0.5), (vt / 0.5).to(torch.float8_e4m3fn).view(torch.uint8).numpy())
+
+
+def test_prefill_rows_stagewise(orc):
+    d = synth.prefill_inputs(seed=91, R=40, vocab=64, h=64, nkv=2, hd=32)
+    U = {k: (u16(v) if isinstance(v, torch.Tensor) and v.dtype == torch.bfloat16 else
+             (v.numpy() if isinstance(v, torch.Tensor) else v)) for k, v in d.items()}
+    rows = np.array([0, 7, 16, 39])
+    out = orc.prefill_rows(U["embed"], U["tokens"], U["hidden"], U["w_norm_embed"],
+                           U["w_norm_hidden"], U["eps"], U["fc"], U["wk"], U["wv"], 2, 32,
+                           U["rope_base"], U["rope_pos"], 0, U["block_table"], 16,
+                           U["num_blocks"], 1.0, 1.0, rows)
+    assert out["flags"] == 0
+    for i, r in enumerate(rows):
+        y, _, _ = orc.combine(U["embed"], U["tokens"][r:r + 1], U["hidden"][r:r + 1],
+                              U["w_norm_embed"], U["w_norm_hidden"], U["eps"], U["fc"])
+        assert np.array_equal(out["y"][i], y[0])
+        yf = orc.bf16_to_f64(y[0])
+        k = orc.f64_to_bf16(orc.bf16_to_f64(U["wk"]) @ yf)
+        v = orc.f64_to_bf16(orc.bf16_to_f64(U["wv"]) @ yf)
+        assert np.array_equal(out["v"][i], v)
+        for hh in range(2):
+            kr = orc.f64_to_bf16(orc.rope_neox(orc.bf16_to_f64(k[hh * 32:(hh + 1) * 32]),
+                                               U["rope_pos"][r], U["rope_base"]))
+            assert np.array_equal(out["k_rot"][i, hh * 32:(hh + 1) * 32], kr)
+        assert np.array_equal(out["k_codes"][i], orc.kv_encode(out["k_rot"][i], 1.0))
+        assert np.array_equal(out["v_codes"][i], orc.kv_encode(v, 1.0))
+        assert out["slot"][i] == orc.slot(U["block_table"], 16, U["num_blocks"], r)
+    # a cache row past the block table is flagged and not given a slot
+    bad = orc.prefill_rows(U["embed"], U["tokens"], U["hidden"], U["w_norm_embed"],
+                           U["w_norm_hidden"], U["eps"], U["fc"], U["wk"], U["wv"], 2, 32,
+                           U["rope_base"], U["rope_pos"], 10_000, U["block_table"], 16,
+                           U["num_blocks"], 1.0, 1.0, rows[:1])
+    assert bad["flags"] & orc.FLAG_BAD_SLOT and bad["slot"][0] == -1
+
+
+def test_head_table_planted_gap_full_size(orc):
+    """The benchmark's BF16 table (154,880 x 4,096): the planted row wins by >= 0.5."""
+    cfg = synth.BF16_HEAD
+    d = synth.head_table(cfg["seed"], cfg["N"], cfg["K"], 1)
+    logits, idx, val, _ = orc.lm_head_argmax(0, u16(d["W"]), cfg["K"], u16(d["x"]))
+    assert idx[0] == d["top"][0]
+    srt = np.sort(logits[0])
+    assert srt[-1] - srt[-2] >= 0.5
