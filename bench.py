@@ -1,0 +1,443 @@
+#!/usr/bin/env python
+"""Benchmark of the draft lm_head sweep + argmax (µs per draft, HBM GB/s, roofline).
+
+One step = one draft's lm_head sweep fused with argmax (mtp_lm_head_argmax) over the
+154,880 x 4,096 BF16 draft head at M = 1 (the table size of the GLM draft head on the
+metrale_model_arch/glm5next_mtp_head/init.rs page). The table is 1.27 GB, ten times
+the 126 MB L2, so every step streams it from HBM; no flush is needed. FP8 and NVFP4
+sweeps at M = 1 are measured the same way and reported under "rows".
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--full]
+
+N > 1 (under torchrun): every rank sweeps its own replica (the sweep has no
+exchange step on one table), timed on the device, max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "lm_head+argmax µs/draft and HBM GB/s (fraction of B200 peak) at M=1"
+FALLBACK_HBM_GBS = 6650.0
+
+# DRAM traffic per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum) and
+# the sha256 of sweep.cu when it was captured; reported as null once the source changed.
+NCU_TRAFFIC = {}
+
+
+def sweep_source_hash() -> str:
+    p = os.path.join(ROOT, "mtp_speculative_draft_lm_b200", "csrc", "sweep.cu")
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, torch_dev):
+        import torch
+
+        self.proc = None
+        self.sel = []
+        try:
+            pr = torch.cuda.get_device_properties(torch_dev)
+            self.sel = ["-i", f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"]
+        except Exception:
+            self.sel = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", *self.sel, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(args):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def build_table(fmt: str, dev):
+    """Seeded synthetic table for one format (quantized on the device)."""
+    import torch
+
+    from mtp_speculative_draft_lm_b200 import api, synth
+
+    cfg = {"bf16": synth.BF16_HEAD, "fp8": synth.FP8_HEAD, "nvfp4": synth.NVFP4_HEAD}[fmt]
+    d = synth.head_table(cfg["seed"], cfg["N"], cfg["K"], max(cfg["Ms"]),
+                         mask_keep=cfg.get("mask_keep"))
+    w = d["W"].to(dev)
+    qinfo = None
+    if fmt == "bf16":
+        table = api.bf16_table(w)
+    else:
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        table = api.quantize_fp8(w) if fmt == "fp8" else api.quantize_nvfp4(w)
+        e.record()
+        torch.cuda.synchronize()
+        ms = s.elapsed_time(e)
+        rd = w.numel() * 2
+        wr = table.nbytes()
+        qinfo = {"ms": ms, "GB/s": (rd * (2 if fmt == "nvfp4" else 1) + wr) / ms / 1e6,
+                 "note": "includes first-call setup" }
+        del w
+    return cfg, d, table, qinfo
+
+
+def time_sweep(head, x, steps, warmup, world, stream):
+    """Device time of `steps` back-to-back sweeps; per-launch event pairs."""
+    import torch
+
+    M = x.shape[0]
+    dev = x.device
+    idx = torch.empty((M,), dtype=torch.int32, device=dev)
+    val = torch.empty((M,), dtype=torch.float32, device=dev)
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            head(x, idx, val, stream=stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for s, e in ev:
+            s.record(stream)
+            head(x, idx, val, stream=stream)
+            e.record(stream)
+        t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    total_ms = t0.elapsed_time(t1)
+    per = [s.elapsed_time(e) for s, e in ev]
+    return total_ms / steps, statistics.mean(per), idx.cpu().numpy(), per
+
+
+def time_e2e(head, x_host, steps, warmup, world, stream):
+    """Same metric end to end: pinned-host input -> H2D -> sweep -> D2H of the result."""
+    import torch
+
+    M, K = x_host.shape
+    dev = torch.device("cuda", torch.cuda.current_device())
+    x_dev = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    idx = torch.empty((M,), dtype=torch.int32, device=dev)
+    val = torch.empty((M,), dtype=torch.float32, device=dev)
+    idx_h = torch.empty((M,), dtype=torch.int32).pin_memory()
+    val_h = torch.empty((M,), dtype=torch.float32).pin_memory()
+
+    def step():
+        x_dev.copy_(x_host, non_blocking=True)
+        head(x_dev, idx, val, stream=stream)
+        idx_h.copy_(idx, non_blocking=True)
+        val_h.copy_(val, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            step()
+    torch.cuda.synchronize()
+    barrier(world)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for _ in range(steps):
+            step()
+        t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    return t0.elapsed_time(t1) / steps, M * K * 2, M * 8, idx_h.numpy().copy()
+
+
+def cpu_baseline(fmt_table, d, cfg, budget_s=12.0):
+    """The oracle, as it stands, on the same table at M = 1 (all of its rows)."""
+    import numpy as np
+
+    import oracle
+    from mtp_speculative_draft_lm_b200 import synth
+
+    W = synth.as_u16(d["W"])
+    x = synth.as_u16(d["x"][:1])
+    nbytes = W.nbytes + x.nbytes + 8
+    times = []
+    t_start = time.perf_counter()
+    while True:
+        t = time.perf_counter()
+        _, idx, _, _ = oracle.lm_head_argmax(0, W, cfg["K"], x, want_logits=False)
+        times.append(time.perf_counter() - t)
+        if time.perf_counter() - t_start > budget_s or len(times) >= 20:
+            break
+    assert idx[0] == d["top"][0]
+    med = statistics.median(times)
+    return {"value": nbytes / med / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"full {cfg['N']}x{cfg['K']} bf16 table, M=1, {len(times)} runs, median "
+                      f"{med * 1e3:.1f} ms/draft (fp64 accumulation, OpenMP over rows)"}
+
+
+def run_reference(args):
+    """--impl reference: the CPU oracle on bounded row samples of the same workload."""
+    import numpy as np
+
+    import oracle
+    from mtp_speculative_draft_lm_b200 import synth
+
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    cfg = synth.BF16_HEAD
+    d = synth.head_table(cfg["seed"], cfg["N"], cfg["K"], 1)
+    W = synth.as_u16(d["W"])
+    x = synth.as_u16(d["x"][:1])
+    K = cfg["K"]
+    # size one step's row sample so that warmup + steps stay within about a minute
+    rows = 1024
+    t = time.perf_counter()
+    oracle.lm_head_argmax(0, W[:rows], K, x, want_logits=False)
+    per_row = (time.perf_counter() - t) / rows
+    total = args.steps + args.warmup
+    rows = int(max(16, min(cfg["N"], 60.0 / total / max(per_row, 1e-9))))
+    starts = [(i * rows) % (cfg["N"] - rows + 1) for i in range(total)]
+    for i in range(args.warmup):
+        oracle.lm_head_argmax(0, W[starts[i]: starts[i] + rows], K, x, want_logits=False)
+    t0 = time.perf_counter()
+    for i in range(args.warmup, total):
+        oracle.lm_head_argmax(0, W[starts[i]: starts[i] + rows], K, x, want_logits=False)
+    dt = (time.perf_counter() - t0) / args.steps
+    nbytes = rows * K * 2 + x.nbytes + 8
+    value = nbytes / dt / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"bf16 lm_head sweep + argmax, table [{cfg['N']}, {K}], M=1",
+                   "sample_rows_per_step": rows},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"{rows} of {cfg['N']} table rows per step (cycling), M=1"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--full", action="store_true", help="also M>1 and masked rows")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--formats", default="bf16,fp8,nvfp4")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import numpy as np
+    import torch
+
+    from mtp_speculative_draft_lm_b200 import api
+
+    world, rank, local = dist_setup(args)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.Stream(device=dev)
+    peak, peak_src = measured_peaks()
+    rows = {}
+    main_line = None
+    cpu_base = None
+    for fmt in args.formats.split(","):
+        cfg, d, table, qinfo = build_table(fmt, dev)
+        head = api.LmHead(table)
+        Ms = cfg["Ms"] if args.full else (1,)
+        for M in Ms:
+            x = d["x"][:M].to(dev)
+            clocks = ClockSampler(dev)
+            clocks.start()
+            ms_step, ms_kernel, idx, per = time_sweep(head, x, args.steps, args.warmup, world,
+                                                       stream)
+            clk = clocks.stop()
+            ok = bool(np.array_equal(idx, d["top"][:M]))
+            ms_max = max_over_ranks(ms_step, world)
+            kern_max = max_over_ranks(ms_kernel, world)
+            nbytes = head.bytes_per_call(M)
+            e2e_ms, h2d, d2h, e2e_idx = time_e2e(head, d["x"][:M].contiguous().pin_memory(),
+                                                  max(100, args.steps // 10), args.warmup,
+                                                  world, stream)
+            e2e_max = max_over_ranks(e2e_ms, world)
+            rec = {
+                "us_per_draft": ms_max * 1e3,
+                "kernel_us": kern_max * 1e3,
+                "GB/s": nbytes * world / (ms_max * 1e-3) / 1e9,
+                "kernel_GB/s": nbytes / (kern_max * 1e-3) / 1e9,
+                "frac_of_peak": nbytes / (kern_max * 1e-3) / 1e9 / peak,
+                "bytes_per_step": nbytes,
+                "e2e_us": e2e_max * 1e3,
+                "argmax_ok": ok and bool(np.array_equal(e2e_idx, d["top"][:M])),
+                "clocks": clk,
+                "p10_p90_kernel_us": [float(np.percentile(per, 10)) * 1e3,
+                                      float(np.percentile(per, 90)) * 1e3],
+            }
+            if qinfo and M == Ms[0]:
+                rec["quantizer"] = qinfo
+            rows[f"{fmt}_M{M}"] = rec
+            if fmt == "bf16" and M == 1:
+                main_line = (rec, nbytes, ms_max, kern_max, e2e_max, h2d, d2h, clk, cfg)
+        if "mask" in d and args.full:
+            words = d["mask"].shape[1]
+            m = torch.from_numpy(d["mask"][:1].reshape(-1)).to(dev)
+            x = d["x"][:1].to(dev)
+            idx = torch.empty((1,), dtype=torch.int32, device=dev)
+            for _ in range(args.warmup):
+                head(x, idx, None, mask=m, mask_words=words, mask_stride_words=words,
+                     stream=stream)
+            torch.cuda.synchronize()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                s.record(stream)
+                for _ in range(args.steps):
+                    head(x, idx, None, mask=m, mask_words=words, mask_stride_words=words,
+                         stream=stream)
+                e.record(stream)
+            torch.cuda.synchronize()
+            rows[f"{fmt}_M1_masked"] = {"us_per_draft": s.elapsed_time(e) / args.steps * 1e3,
+                                        "argmax_ok": int(idx.item()) == int(d["second"][0])}
+        if fmt == "bf16" and rank == 0 and world == 1 and not args.no_cpu:
+            cpu_base = cpu_baseline(table, d, cfg)
+        del head, table, d
+        torch.cuda.empty_cache()
+
+    if rank == 0 and main_line is not None:
+        rec, nbytes, ms_max, kern_max, e2e_max, h2d, d2h, clk, cfg = main_line
+        achieved = nbytes / (kern_max * 1e-3) / 1e9
+        tr = NCU_TRAFFIC.get("bf16_M1")
+        traffic = tr[0] if tr and tr[1] == sweep_source_hash() else None
+        line = {
+            "metric": METRIC,
+            "value": nbytes * world / (ms_max * 1e-3) / 1e9,
+            "unit": "GB/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_max,
+            "us_per_draft": ms_max * 1e3,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic: seeded N(0, 0.02) bf16 table with planted maximum rows",
+            "config": {"workload": f"bf16 lm_head sweep + argmax, table [{cfg['N']}, {cfg['K']}], M=1",
+                       "table_bytes": cfg["N"] * cfg["K"] * 2, "M": 1,
+                       "l2": "table (1.27 GB) larger than L2 (126 MB): no flush",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{peak_src} hbm_gbs (copy)",
+                         "kernel": "sweep_kernel<bf16, M<=8, argmax>"},
+            "cpu_baseline": cpu_base,
+            "e2e": {"value": nbytes * world / (e2e_max * 1e-3) / 1e9, "unit": "GB/s",
+                    "us_per_draft": e2e_max * 1e3, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps,
+            "clocks": clk,
+            "rows": rows,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,197 @@
+/*
+ * mtp.h -- C ABI of the B200 (sm_100a) multi-token-prediction draft-head library.
+ *
+ * The library implements the weight-streaming hot path of a single-layer MTP draft
+ * head, as described by these pages (cited below by title and section):
+ *   [mtp_head.rs] spark_model/layers/mtp_head.rs -- MtpHead docs, MtpQuantization,
+ *                 ProjectionWeight, the gemv dispatch, quantize_proj, the drafter-
+ *                 prefill docs and MtpPrefillScratch;
+ *   [new.rs]      metrale_model_layers/layers/mtp_head/new.rs -- MtpHead::new (the
+ *                 quantizer kernels, the KV-pool config, the prefill scratch);
+ *   [init.rs]     metrale_model_arch/glm5next_mtp_head/init.rs -- the vocab-sharded
+ *                 draft lm_head over [vocab, hidden] rows packed at K, FP8 shard;
+ *   [v4_mtp.rs]   metrale_model_arch/deepseek_v4_mtp.rs -- module docs "One draft",
+ *                 forward_one steps 1-7, argmax_grammar_masked.
+ *
+ * Conventions for every entry point:
+ *  - Pointers marked (device) are CUDA device memory owned by the caller; the
+ *    library never allocates, frees or retains them and keeps no state between
+ *    calls (except the workspace contract of the functions that take one).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *    All work is enqueued asynchronously on it; results are valid once the stream
+ *    reaches that point.
+ *  - bf16 values are passed as their uint16_t bit patterns.
+ *  - Arguments are validated on the host before anything is launched. A call that
+ *    returns non-zero has enqueued nothing (MTP_ERR_CUDA: a launch failed; earlier
+ *    kernels of the same call may have been enqueued).
+ *  - Data-dependent problems found on the device (a token id outside the table, a
+ *    cache row with no block, a mask that allows nothing) never trap: the kernel
+ *    ORs an MTP_DEVFLAG_* bit into *dev_err (when dev_err is not NULL) and carries
+ *    on with the documented fallback. Read it after the stream synchronises.
+ *  - Functions are re-entrant; calls that share a workspace must not overlap in time.
+ */
+#ifndef MTP_H
+#define MTP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MTP_ABI_VERSION 1
+
+typedef enum {
+    MTP_OK = 0,
+    MTP_ERR_INVALID_ARG = 1, /* null / misaligned pointer, bad size or stride */
+    MTP_ERR_UNSUPPORTED = 2, /* valid but outside what the kernels handle (shape, M) */
+    MTP_ERR_WORKSPACE = 3,   /* workspace missing or smaller than the *_ws_bytes size */
+    MTP_ERR_CUDA = 4,        /* a CUDA launch or API call failed */
+    MTP_WARN_EMPTY_MASK = 5  /* mtp_devflags_status(): a mask allowed no token */
+} mtp_status;
+
+/* Bits a kernel ORs into the caller's device error word. */
+#define MTP_DEVFLAG_BAD_TOKEN 1  /* token id outside [0, vocab): its row read as zeros */
+#define MTP_DEVFLAG_EMPTY_MASK 2 /* a row's mask allowed nothing: idx 0, value -inf */
+#define MTP_DEVFLAG_BAD_SLOT 4   /* a cache row had no valid block: row not written */
+
+/* Weight formats ([mtp_head.rs] MtpQuantization and ProjectionWeight: Bf16, Fp8,
+ * Nvfp4). */
+typedef enum {
+    MTP_FMT_BF16 = 0,    /* data: bf16 [n, k] */
+    MTP_FMT_FP8_ROW = 1, /* data: E4M3FN codes [n, k]; row_scale: f32 [n] */
+    MTP_FMT_NVFP4 = 2    /* data: E2M1 codes [n, k/2] (element 2j = low nibble of byte
+                            j); block_scale: E4M3FN [n, k/16]; global_scale: f32[1] */
+} mtp_format;
+
+/* A [n, k] weight table in one of the formats, rows packed at k (no row stride:
+ * [init.rs] notes the draft-head GEMV assumes rows packed at K). All pointers are
+ * device pointers; the unused ones must be NULL. dequant(W)[r, j] is the bf16
+ * value, e4m3(code) * row_scale[r], or e2m1(code) * e4m3(block_scale[r, j/16]) *
+ * global_scale[0]. */
+typedef struct {
+    int32_t fmt;
+    int32_t reserved; /* must be 0 */
+    int64_t n;
+    int64_t k;
+    const void* data;
+    const float* row_scale;
+    const uint8_t* block_scale;
+    const float* global_scale;
+} mtp_weight;
+
+/* ---------------------------------------------------------------------------------
+ * mtp_quantize_fp8 -- BF16 -> FP8 E4M3 with one fp32 scale per row.
+ * Source: [new.rs] MtpHead::new looks up the BF16 -> FP8 quantizer; [mtp_head.rs]
+ * quantize_proj calls it for MtpQuantization::Fp8; [init.rs] quantizes the draft
+ * head's rows to FP8. Rule (fp32, round to nearest even): a = max_j |w[r, j]|,
+ * row_scale[r] = a / 448, codes[r, j] = e4m3_satfinite(w[r, j] / row_scale[r]); an
+ * all-zero row gets scale 0 and codes 0.
+ *   w          (device) bf16 [n, k], 16-byte aligned
+ *   codes      (device) u8 [n, k], 16-byte aligned, written
+ *   row_scale  (device) f32 [n], written
+ * Requires n >= 1, k >= 16, k % 16 == 0.
+ * ------------------------------------------------------------------------------ */
+mtp_status mtp_quantize_fp8(const uint16_t* w, int64_t n, int64_t k, uint8_t* codes,
+                            float* row_scale, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * mtp_quantize_nvfp4 -- BF16 -> NVFP4 in two passes.
+ * Source: [new.rs] MtpHead::new looks up the global-absmax pass and the BF16 -> NVFP4
+ * pass; [mtp_head.rs] quantize_proj uses them for MtpQuantization::Nvfp4; the
+ * per-row size is k/2 code bytes (the MtpHead::new lm-head size log). Rule (fp32,
+ * round to nearest even): A = max|w|, g = A / 2688 (1 if A == 0); per block b of
+ * 16 consecutive k: B = max|w_b|, sb = e4m3_satfinite((B / 6) / g),
+ * S = e4m3(sb) * g, code = e2m1_satfinite(w / S) (0 when S == 0).
+ *   w            (device) bf16 [n, k], 16-byte aligned
+ *   codes        (device) u8 [n, k/2] written (two codes per byte, element 2j low)
+ *   block_scale  (device) u8 [n, k/16] written
+ *   global_scale (device) f32 [1] written (g)
+ *   ws           (device) >= mtp_quantize_nvfp4_ws_bytes(n, k) bytes, 16-byte
+ *                aligned, ALL ZERO before the first call; each call leaves it zero.
+ * Requires n >= 1, k >= 32, k % 32 == 0.
+ * ------------------------------------------------------------------------------ */
+size_t mtp_quantize_nvfp4_ws_bytes(int64_t n, int64_t k);
+mtp_status mtp_quantize_nvfp4(const uint16_t* w, int64_t n, int64_t k, uint8_t* codes,
+                              uint8_t* block_scale, float* global_scale, void* ws,
+                              size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * mtp_combine -- the draft's embed+hidden combiner for M rows.
+ * Source: [v4_mtp.rs] forward_one steps 1-2 (embedding row copy; two RMSNorms with
+ * plain weights w * x_normed; e_proj / h_proj combiner) and [mtp_head.rs] module
+ * docs (embed+hidden concat -> fc), with fc [h, 2h] as quantized in [new.rs].
+ *   e = embed[token_ids[m]];  ne = bf16(e / sqrt(mean(e^2) + eps) * w_norm_embed)
+ *   nh = bf16(x / sqrt(mean(x^2) + eps) * w_norm_hidden),  x = hidden[m]
+ *   out[m] = bf16(fc . [ne || nh])           (embedding half first)
+ *   embed         (device) bf16 [vocab, h]
+ *   token_ids     (device) i32 [M]; an id outside [0, vocab) reads as a zero row and
+ *                 sets MTP_DEVFLAG_BAD_TOKEN
+ *   hidden        (device) bf16 [M, h]
+ *   w_norm_embed, w_norm_hidden (device) bf16 [h]
+ *   fc            weight with n == h, k == 2h (MTP_FMT_BF16, MTP_FMT_FP8_ROW or
+ *                 MTP_FMT_NVFP4)
+ *   out           (device) bf16 [M, h], written
+ *   dev_err       (device) i32 [1] or NULL
+ * Requires 1 <= M <= 16, h % 16 == 0 (fc's k must meet its format's k rule), all
+ * device pointers 16-byte aligned except token_ids / dev_err (4-byte).
+ * ------------------------------------------------------------------------------ */
+mtp_status mtp_combine(const uint16_t* embed, int64_t vocab, const int32_t* token_ids,
+                       const uint16_t* hidden, int32_t M, int32_t h,
+                       const uint16_t* w_norm_embed, const uint16_t* w_norm_hidden,
+                       float eps, const mtp_weight* fc, uint16_t* out, int32_t* dev_err,
+                       void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * mtp_lm_head_argmax -- the draft lm_head sweep fused with a (masked) argmax.
+ * Source: [v4_mtp.rs] forward_one steps 6-7 (lm_head GEMV over the first v rows,
+ * v = the effective vocab, then argmax, grammar-masked when a bitmask is given) and
+ * argmax_grammar_masked (token t allowed iff word t/32 exists and bit t%32 is set;
+ * lowest index wins ties; nothing allowed -> token 0); [init.rs] the sweep over
+ * [vocab, hidden] rows, "most of the drafter's time".
+ *   l[m, r] = sum_j dequant(head)[r, j] * x[m, j]   (fp32 accumulation), r < n_eff
+ *   out_idx[m] = lowest allowed r with the largest l[m, r]; the argmax is taken on
+ *   the fp32 logit. No token allowed -> out_idx 0, out_val -inf, MTP_DEVFLAG_EMPTY_MASK.
+ *   head          weight [n, k]; n_eff <= n rows are swept (the effective vocab)
+ *   x             (device) bf16 [M, k], 16-byte aligned
+ *   mask          (device) i32 words or NULL; row m's mask starts at
+ *                 mask + m * mask_stride_words (stride 0: one mask for all rows) and
+ *                 has mask_words words (tokens past 32 * mask_words are disallowed)
+ *   out_idx       (device) i32 [M], written
+ *   out_val       (device) f32 [M] or NULL: the winning logit
+ *   out_logits    (device) bf16 [M, n_eff] or NULL: bf16(l), masked tokens -inf
+ *   dev_err       (device) i32 [1] or NULL
+ *   ws            (device) >= mtp_lm_head_ws_bytes(head, n_eff, M) bytes, 16-byte
+ *                 aligned, ALL ZERO before the first call; each call leaves its
+ *                 counter zero again.
+ * Requires 1 <= M <= 16, 1 <= n_eff <= n; k % 8 (BF16), k % 16 (FP8), k % 32 (NVFP4);
+ * the staged inputs (M * k * 2 bytes) must fit in shared memory (MTP_ERR_UNSUPPORTED
+ * otherwise).
+ * ------------------------------------------------------------------------------ */
+size_t mtp_lm_head_ws_bytes(const mtp_weight* head, int64_t n_eff, int32_t M);
+mtp_status mtp_lm_head_argmax(const mtp_weight* head, int64_t n_eff, const uint16_t* x,
+                              int32_t M, const int32_t* mask, int64_t mask_words,
+                              int64_t mask_stride_words, int32_t* out_idx, float* out_val,
+                              uint16_t* out_logits, int32_t* dev_err, void* ws,
+                              size_t ws_bytes, void* stream);
+
+/* Maps a device error word read back by the caller to a status: MTP_OK, or
+ * MTP_WARN_EMPTY_MASK when only the empty-mask bit is set, else MTP_ERR_INVALID_ARG. */
+mtp_status mtp_devflags_status(int32_t dev_err_value);
+
+/* ---------------------------------------------------------------------------------
+ * Exhaustive-check entry points: the device E4M3 / E2M1 encoders used by the
+ * quantizers and the KV write, one f32 in -> one code out (E2M1 in the low nibble).
+ *   in (device) f32 [n]; out (device) u8 [n]
+ * ------------------------------------------------------------------------------ */
+mtp_status mtp_debug_encode_e4m3(const float* in, int64_t n, uint8_t* out, void* stream);
+mtp_status mtp_debug_encode_e2m1(const float* in, int64_t n, uint8_t* out, void* stream);
+
+const char* mtp_status_str(mtp_status s);
+int32_t mtp_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MTP_H */

@@ -1,0 +1,182 @@
+"""ctypes binding of ``libmtp.so`` (include/mtp.h): argument marshalling only.
+
+Every function here has the C entry point's name and arguments. Pointer arguments
+accept a torch tensor (its ``data_ptr()``), a plain integer address, or None for
+NULL; ``stream`` defaults to torch's current CUDA stream. A non-zero status raises
+:class:`MtpError`. There is no fallback: if the library is missing, loading it
+raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libmtp.so")
+
+MTP_OK = 0
+MTP_ERR_INVALID_ARG = 1
+MTP_ERR_UNSUPPORTED = 2
+MTP_ERR_WORKSPACE = 3
+MTP_ERR_CUDA = 4
+MTP_WARN_EMPTY_MASK = 5
+
+MTP_DEVFLAG_BAD_TOKEN = 1
+MTP_DEVFLAG_EMPTY_MASK = 2
+MTP_DEVFLAG_BAD_SLOT = 4
+
+MTP_FMT_BF16 = 0
+MTP_FMT_FP8_ROW = 1
+MTP_FMT_NVFP4 = 2
+
+#: every symbol include/mtp.h declares
+EXPORTS = (
+    "mtp_abi_version", "mtp_status_str", "mtp_devflags_status",
+    "mtp_quantize_fp8", "mtp_quantize_nvfp4_ws_bytes", "mtp_quantize_nvfp4",
+    "mtp_combine", "mtp_lm_head_ws_bytes", "mtp_lm_head_argmax",
+    "mtp_debug_encode_e4m3", "mtp_debug_encode_e2m1",
+)
+
+
+class MtpError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: status {status} ({status_str(status)})")
+
+
+class mtp_weight(C.Structure):
+    _fields_ = [("fmt", C.c_int32), ("reserved", C.c_int32), ("n", C.c_int64),
+                ("k", C.c_int64), ("data", C.c_void_p), ("row_scale", C.c_void_p),
+                ("block_scale", C.c_void_p), ("global_scale", C.c_void_p)]
+
+
+_P = C.c_void_p
+_I32 = C.c_int32
+_I64 = C.c_int64
+_SZ = C.c_size_t
+_W = C.POINTER(mtp_weight)
+
+_SIGS = {
+    "mtp_abi_version": (_I32, []),
+    "mtp_status_str": (C.c_char_p, [C.c_int]),
+    "mtp_devflags_status": (C.c_int, [_I32]),
+    "mtp_quantize_fp8": (C.c_int, [_P, _I64, _I64, _P, _P, _P]),
+    "mtp_quantize_nvfp4_ws_bytes": (_SZ, [_I64, _I64]),
+    "mtp_quantize_nvfp4": (C.c_int, [_P, _I64, _I64, _P, _P, _P, _P, _SZ, _P]),
+    "mtp_combine": (C.c_int, [_P, _I64, _P, _P, _I32, _I32, _P, _P, C.c_float, _W, _P, _P,
+                              _P]),
+    "mtp_lm_head_ws_bytes": (_SZ, [_W, _I64, _I32]),
+    "mtp_lm_head_argmax": (C.c_int, [_W, _I64, _P, _I32, _P, _I64, _I64, _P, _P, _P, _P,
+                                     _P, _SZ, _P]),
+    "mtp_debug_encode_e4m3": (C.c_int, [_P, _I64, _P, _P]),
+    "mtp_debug_encode_e2m1": (C.c_int, [_P, _I64, _P, _P]),
+}
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> C.CDLL:
+    """Load libmtp.so (raises OSError if it is missing: there is no fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise OSError(f"{path} not found: build it with mtp_speculative_draft_lm_b200.build")
+        lib = C.CDLL(path)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(lib, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    if isinstance(a, int):
+        return a
+    return a.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        import torch
+
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(st: int, where: str):
+    if st != MTP_OK:
+        raise MtpError(st, where)
+
+
+def status_str(st: int) -> str:
+    return load().mtp_status_str(st).decode()
+
+
+def weight(fmt: int, n: int, k: int, data, row_scale=None, block_scale=None,
+           global_scale=None) -> mtp_weight:
+    return mtp_weight(int(fmt), 0, int(n), int(k), _ptr(data), _ptr(row_scale),
+                      _ptr(block_scale), _ptr(global_scale))
+
+
+def mtp_abi_version() -> int:
+    return load().mtp_abi_version()
+
+
+def mtp_devflags_status(value: int) -> int:
+    return load().mtp_devflags_status(int(value))
+
+
+def mtp_quantize_fp8(w, n, k, codes, row_scale, stream=None):
+    _check(load().mtp_quantize_fp8(_ptr(w), n, k, _ptr(codes), _ptr(row_scale),
+                                   _stream(stream)), "mtp_quantize_fp8")
+
+
+def mtp_quantize_nvfp4_ws_bytes(n, k) -> int:
+    return load().mtp_quantize_nvfp4_ws_bytes(n, k)
+
+
+def mtp_quantize_nvfp4(w, n, k, codes, block_scale, global_scale, ws, ws_bytes, stream=None):
+    _check(load().mtp_quantize_nvfp4(_ptr(w), n, k, _ptr(codes), _ptr(block_scale),
+                                     _ptr(global_scale), _ptr(ws), ws_bytes, _stream(stream)),
+           "mtp_quantize_nvfp4")
+
+
+def mtp_combine(embed, vocab, token_ids, hidden, M, h, w_norm_embed, w_norm_hidden, eps, fc,
+                out, dev_err=None, stream=None):
+    _check(load().mtp_combine(_ptr(embed), vocab, _ptr(token_ids), _ptr(hidden), M, h,
+                              _ptr(w_norm_embed), _ptr(w_norm_hidden), float(eps),
+                              C.byref(fc) if fc is not None else None, _ptr(out),
+                              _ptr(dev_err), _stream(stream)), "mtp_combine")
+
+
+def mtp_lm_head_ws_bytes(head, n_eff, M) -> int:
+    return load().mtp_lm_head_ws_bytes(C.byref(head), n_eff, M)
+
+
+def mtp_lm_head_argmax(head, n_eff, x, M, mask, mask_words, mask_stride_words, out_idx,
+                       out_val, out_logits, dev_err, ws, ws_bytes, stream=None):
+    _check(load().mtp_lm_head_argmax(C.byref(head) if head is not None else None, n_eff,
+                                     _ptr(x), M, _ptr(mask), mask_words, mask_stride_words,
+                                     _ptr(out_idx), _ptr(out_val), _ptr(out_logits),
+                                     _ptr(dev_err), _ptr(ws), ws_bytes, _stream(stream)),
+           "mtp_lm_head_argmax")
+
+
+def mtp_debug_encode_e4m3(inp, n, out, stream=None):
+    _check(load().mtp_debug_encode_e4m3(_ptr(inp), n, _ptr(out), _stream(stream)),
+           "mtp_debug_encode_e4m3")
+
+
+def mtp_debug_encode_e2m1(inp, n, out, stream=None):
+    _check(load().mtp_debug_encode_e2m1(_ptr(inp), n, _ptr(out), _stream(stream)),
+           "mtp_debug_encode_e2m1")
+
+
+def raw_status(name: str, *args) -> int:
+    """Call an entry point and return its status without raising (for error tests)."""
+    return getattr(load(), name)(*args)

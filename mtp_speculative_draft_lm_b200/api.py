@@ -1,0 +1,110 @@
+"""Torch-facing helpers over the C ABI: they allocate device buffers with torch
+(memory and streams are torch's job here) and call the ``mtp_*`` entry points.
+No arithmetic of the method happens in Python."""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import torch
+
+from . import _lib as L
+
+
+def _u16(t: torch.Tensor) -> torch.Tensor:
+    assert t.dtype in (torch.bfloat16, torch.int16, torch.uint16)
+    return t
+
+
+@dataclass
+class Table:
+    """A [n, k] weight table on the device in one of the three formats."""
+    fmt: int
+    n: int
+    k: int
+    data: torch.Tensor
+    row_scale: torch.Tensor | None = None
+    block_scale: torch.Tensor | None = None
+    global_scale: torch.Tensor | None = None
+    desc: L.mtp_weight = field(init=False)
+
+    def __post_init__(self):
+        self.desc = L.weight(self.fmt, self.n, self.k, self.data, self.row_scale,
+                             self.block_scale, self.global_scale)
+
+    def nbytes(self) -> int:
+        b = self.data.numel() * self.data.element_size()
+        for t in (self.row_scale, self.block_scale, self.global_scale):
+            if t is not None:
+                b += t.numel() * t.element_size()
+        return b
+
+
+def bf16_table(w: torch.Tensor) -> Table:
+    n, k = w.shape
+    return Table(L.MTP_FMT_BF16, n, k, _u16(w.contiguous()))
+
+
+def quantize_fp8(w: torch.Tensor, stream=None) -> Table:
+    n, k = w.shape
+    codes = torch.empty((n, k), dtype=torch.uint8, device=w.device)
+    scale = torch.empty((n,), dtype=torch.float32, device=w.device)
+    L.mtp_quantize_fp8(w, n, k, codes, scale, stream)
+    return Table(L.MTP_FMT_FP8_ROW, n, k, codes, row_scale=scale)
+
+
+def quantize_nvfp4(w: torch.Tensor, ws: torch.Tensor | None = None, stream=None) -> Table:
+    n, k = w.shape
+    codes = torch.empty((n, k // 2), dtype=torch.uint8, device=w.device)
+    bscale = torch.empty((n, k // 16), dtype=torch.uint8, device=w.device)
+    g = torch.empty((1,), dtype=torch.float32, device=w.device)
+    nbytes = L.mtp_quantize_nvfp4_ws_bytes(n, k)
+    if ws is None:
+        ws = torch.zeros((nbytes,), dtype=torch.uint8, device=w.device)
+    L.mtp_quantize_nvfp4(w, n, k, codes, bscale, g, ws, ws.numel(), stream)
+    return Table(L.MTP_FMT_NVFP4, n, k, codes, block_scale=bscale, global_scale=g)
+
+
+class LmHead:
+    """The fused sweep + argmax over a table, with its zeroed workspace."""
+
+    def __init__(self, table: Table, n_eff: int | None = None, max_m: int = 16):
+        self.table = table
+        self.n_eff = table.n if n_eff is None else int(n_eff)
+        dev = table.data.device
+        nbytes = L.mtp_lm_head_ws_bytes(table.desc, self.n_eff, max_m)
+        self.ws = torch.zeros((nbytes,), dtype=torch.uint8, device=dev)
+        self.dev_err = torch.zeros((1,), dtype=torch.int32, device=dev)
+
+    def bytes_per_call(self, M: int, mask_words: int = 0) -> int:
+        """Algorithmic bytes of one unmasked sweep: the swept table rows, the inputs,
+        the mask words and the outputs."""
+        t = self.table
+        frac = self.n_eff / t.n
+        return int(t.nbytes() * frac) + M * t.k * 2 + mask_words * 4 * (1 if M else 0) + M * 8
+
+    def __call__(self, x: torch.Tensor, out_idx: torch.Tensor, out_val=None, out_logits=None,
+                 mask=None, mask_words=0, mask_stride_words=0, stream=None):
+        M = x.shape[0]
+        L.mtp_lm_head_argmax(self.table.desc, self.n_eff, x, M, mask, mask_words,
+                             mask_stride_words, out_idx, out_val, out_logits, self.dev_err,
+                             self.ws, self.ws.numel(), stream)
+
+    def argmax(self, x: torch.Tensor, mask=None, mask_words=0, mask_stride_words=0,
+               logits=False, stream=None):
+        M = x.shape[0]
+        dev = x.device
+        idx = torch.empty((M,), dtype=torch.int32, device=dev)
+        val = torch.empty((M,), dtype=torch.float32, device=dev)
+        lg = torch.empty((M, self.n_eff), dtype=torch.bfloat16, device=dev) if logits else None
+        self(x, idx, val, lg, mask, mask_words, mask_stride_words, stream)
+        return idx, val, lg
+
+
+def combine(embed, token_ids, hidden, w_norm_embed, w_norm_hidden, eps, fc: Table,
+            out=None, dev_err=None, stream=None):
+    M, h = hidden.shape
+    if out is None:
+        out = torch.empty((M, h), dtype=torch.bfloat16, device=hidden.device)
+    L.mtp_combine(embed, embed.shape[0], token_ids, hidden, M, h, w_norm_embed, w_norm_hidden,
+                  eps, fc.desc, out, dev_err, stream)
+    return out

@@ -1,0 +1,203 @@
+// C ABI (include/mtp.h): host-side argument validation, then the kernel launches.
+// Nothing here computes the method; every arithmetic step runs in the kernels.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/mtp.h"
+#include "kernels.h"
+
+namespace {
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+mtp_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return MTP_OK;
+    if (e == cudaErrorInvalidValue) return MTP_ERR_UNSUPPORTED;
+    return MTP_ERR_CUDA;
+}
+
+// Checks a weight descriptor: format, sizes, pointer presence and alignment.
+mtp_status check_weight(const mtp_weight* w) {
+    if (!w || w->reserved != 0 || w->n < 1 || w->k < 1 || !w->data) return MTP_ERR_INVALID_ARG;
+    if (!aligned(w->data, 16)) return MTP_ERR_INVALID_ARG;
+    switch (w->fmt) {
+        case MTP_FMT_BF16:
+            if (w->k % 8 || w->row_scale || w->block_scale || w->global_scale)
+                return MTP_ERR_INVALID_ARG;
+            return MTP_OK;
+        case MTP_FMT_FP8_ROW:
+            if (w->k % 16 || !w->row_scale || w->block_scale || w->global_scale)
+                return MTP_ERR_INVALID_ARG;
+            if (!aligned(w->row_scale, 4)) return MTP_ERR_INVALID_ARG;
+            return MTP_OK;
+        case MTP_FMT_NVFP4:
+            if (w->k % 32 || w->row_scale || !w->block_scale || !w->global_scale)
+                return MTP_ERR_INVALID_ARG;
+            if (!aligned(w->block_scale, 2) || !aligned(w->global_scale, 4))
+                return MTP_ERR_INVALID_ARG;
+            return MTP_OK;
+        default:
+            return MTP_ERR_INVALID_ARG;
+    }
+}
+
+int64_t row_bytes(const mtp_weight* w) {
+    return w->fmt == MTP_FMT_BF16 ? w->k * 2 : w->fmt == MTP_FMT_FP8_ROW ? w->k : w->k / 2;
+}
+
+constexpr size_t kTicketBytes = 256;
+constexpr size_t kPartialBytes = 8;  // {float value, int32 index}
+constexpr int kMaxM = 16;
+
+}  // namespace
+
+extern "C" {
+
+int32_t mtp_abi_version(void) { return MTP_ABI_VERSION; }
+
+const char* mtp_status_str(mtp_status s) {
+    switch (s) {
+        case MTP_OK: return "ok";
+        case MTP_ERR_INVALID_ARG: return "invalid argument";
+        case MTP_ERR_UNSUPPORTED: return "unsupported shape or size";
+        case MTP_ERR_WORKSPACE: return "workspace missing or too small";
+        case MTP_ERR_CUDA: return "CUDA error";
+        case MTP_WARN_EMPTY_MASK: return "a grammar mask allowed no token";
+    }
+    return "unknown status";
+}
+
+mtp_status mtp_devflags_status(int32_t v) {
+    if (v == 0) return MTP_OK;
+    if (v == MTP_DEVFLAG_EMPTY_MASK) return MTP_WARN_EMPTY_MASK;
+    return MTP_ERR_INVALID_ARG;
+}
+
+mtp_status mtp_quantize_fp8(const uint16_t* w, int64_t n, int64_t k, uint8_t* codes,
+                            float* row_scale, void* stream) {
+    if (!w || !codes || !row_scale || n < 1 || k < 16 || k % 16) return MTP_ERR_INVALID_ARG;
+    if (!aligned(w, 16) || !aligned(codes, 16) || !aligned(row_scale, 4))
+        return MTP_ERR_INVALID_ARG;
+    return from_cuda(mtp::quant_fp8_launch(w, n, k, codes, row_scale, as_stream(stream)));
+}
+
+size_t mtp_quantize_nvfp4_ws_bytes(int64_t n, int64_t k) {
+    (void)n;
+    (void)k;
+    return kTicketBytes + sizeof(float) * (size_t)mtp::quant_nvfp4_max_grid();
+}
+
+mtp_status mtp_quantize_nvfp4(const uint16_t* w, int64_t n, int64_t k, uint8_t* codes,
+                              uint8_t* block_scale, float* global_scale, void* ws,
+                              size_t ws_bytes, void* stream) {
+    if (!w || !codes || !block_scale || !global_scale || n < 1 || k < 32 || k % 32)
+        return MTP_ERR_INVALID_ARG;
+    if (!aligned(w, 16) || !aligned(codes, 16) || !aligned(global_scale, 4))
+        return MTP_ERR_INVALID_ARG;
+    if (!ws || !aligned(ws, 16) || ws_bytes < mtp_quantize_nvfp4_ws_bytes(n, k))
+        return MTP_ERR_WORKSPACE;
+    return from_cuda(mtp::quant_nvfp4_launch(w, n, k, codes, block_scale, global_scale,
+                                             static_cast<uint32_t*>(ws), as_stream(stream)));
+}
+
+mtp_status mtp_combine(const uint16_t* embed, int64_t vocab, const int32_t* token_ids,
+                       const uint16_t* hidden, int32_t M, int32_t h,
+                       const uint16_t* w_norm_embed, const uint16_t* w_norm_hidden,
+                       float eps, const mtp_weight* fc, uint16_t* out, int32_t* dev_err,
+                       void* stream) {
+    if (!embed || !token_ids || !hidden || !w_norm_embed || !w_norm_hidden || !out)
+        return MTP_ERR_INVALID_ARG;
+    if (vocab < 1 || h < 16 || h % 16 || !(eps >= 0.f)) return MTP_ERR_INVALID_ARG;
+    if (M < 1 || M > kMaxM) return MTP_ERR_UNSUPPORTED;
+    mtp_status st = check_weight(fc);
+    if (st != MTP_OK) return st;
+    if (fc->n != h || fc->k != 2 * (int64_t)h) return MTP_ERR_INVALID_ARG;
+    if (!aligned(embed, 16) || !aligned(hidden, 16) || !aligned(out, 16) ||
+        !aligned(w_norm_embed, 4) || !aligned(w_norm_hidden, 4) || !aligned(token_ids, 4) ||
+        !aligned(dev_err, 4))
+        return MTP_ERR_INVALID_ARG;
+    if (mtp::sweep_smem_bytes(M, fc->k, fc->fmt, nullptr) > 227 * 1024) return MTP_ERR_UNSUPPORTED;
+    mtp::SweepParams p{};
+    p.w = static_cast<const uint8_t*>(fc->data);
+    p.row_scale = fc->row_scale;
+    p.block_scale = fc->block_scale;
+    p.global_scale = fc->global_scale;
+    p.n = fc->n;
+    p.k = fc->k;
+    p.row_bytes = row_bytes(fc);
+    p.M = M;
+    p.embed = embed;
+    p.vocab = vocab;
+    p.tokens = token_ids;
+    p.hidden = hidden;
+    p.w_norm_embed = w_norm_embed;
+    p.w_norm_hidden = w_norm_hidden;
+    p.eps = eps;
+    p.h = h;
+    p.out_y = out;
+    p.dev_err = dev_err;
+    p.num_tiles = (fc->n + 15) / 16;
+    return from_cuda(mtp::sweep_launch(p, fc->fmt, 1, as_stream(stream), nullptr));
+}
+
+size_t mtp_lm_head_ws_bytes(const mtp_weight* head, int64_t n_eff, int32_t M) {
+    (void)head;
+    (void)n_eff;
+    (void)M;
+    return kTicketBytes + kPartialBytes * 16 * (size_t)mtp::sweep_max_grid();
+}
+
+mtp_status mtp_lm_head_argmax(const mtp_weight* head, int64_t n_eff, const uint16_t* x,
+                              int32_t M, const int32_t* mask, int64_t mask_words,
+                              int64_t mask_stride_words, int32_t* out_idx, float* out_val,
+                              uint16_t* out_logits, int32_t* dev_err, void* ws,
+                              size_t ws_bytes, void* stream) {
+    mtp_status st = check_weight(head);
+    if (st != MTP_OK) return st;
+    if (!x || !out_idx || n_eff < 1 || n_eff > head->n) return MTP_ERR_INVALID_ARG;
+    if (n_eff > (int64_t)INT32_MAX) return MTP_ERR_UNSUPPORTED;
+    if (M < 1 || M > kMaxM) return MTP_ERR_UNSUPPORTED;
+    if (mask && (mask_words < 1 || mask_stride_words < 0)) return MTP_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(out_idx, 4) || !aligned(out_val, 4) ||
+        !aligned(out_logits, 2) || !aligned(dev_err, 4) || !aligned(mask, 4))
+        return MTP_ERR_INVALID_ARG;
+    if (!ws || !aligned(ws, 16) || ws_bytes < mtp_lm_head_ws_bytes(head, n_eff, M))
+        return MTP_ERR_WORKSPACE;
+    if (mtp::sweep_smem_bytes(M, head->k, head->fmt, nullptr) > 227 * 1024)
+        return MTP_ERR_UNSUPPORTED;
+    mtp::SweepParams p{};
+    p.w = static_cast<const uint8_t*>(head->data);
+    p.row_scale = head->row_scale;
+    p.block_scale = head->block_scale;
+    p.global_scale = head->global_scale;
+    p.n = n_eff;
+    p.k = head->k;
+    p.row_bytes = row_bytes(head);
+    p.M = M;
+    p.x = x;
+    p.mask = mask;
+    p.mask_words = mask ? mask_words : 0;
+    p.mask_stride = mask ? mask_stride_words : 0;
+    p.out_idx = out_idx;
+    p.out_val = out_val;
+    p.out_logits = out_logits;
+    p.dev_err = dev_err;
+    p.ticket = static_cast<uint32_t*>(ws);
+    p.partials = static_cast<uint8_t*>(ws) + kTicketBytes;
+    p.num_tiles = (n_eff + 15) / 16;
+    return from_cuda(mtp::sweep_launch(p, head->fmt, 0, as_stream(stream), nullptr));
+}
+
+mtp_status mtp_debug_encode_e4m3(const float* in, int64_t n, uint8_t* out, void* stream) {
+    if (!in || !out || n < 1 || !aligned(in, 4)) return MTP_ERR_INVALID_ARG;
+    return from_cuda(mtp::debug_encode_launch(in, n, out, 0, as_stream(stream)));
+}
+
+mtp_status mtp_debug_encode_e2m1(const float* in, int64_t n, uint8_t* out, void* stream) {
+    if (!in || !out || n < 1 || !aligned(in, 4)) return MTP_ERR_INVALID_ARG;
+    return from_cuda(mtp::debug_encode_launch(in, n, out, 1, as_stream(stream)));
+}
+
+}  // extern "C"

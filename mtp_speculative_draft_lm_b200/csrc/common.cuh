@@ -1,0 +1,145 @@
+// Device helpers shared by the draft-head kernels (sm_100a only).
+//
+// Number formats: bf16 is the top half of an fp32; E4M3 is OCP E4M3FN (largest
+// finite 448, no infinities); E2M1 is OCP FP4 ({0,.5,1,1.5,2,3,4,6} and sign).
+// Conversions to the narrow formats use the hardware's round-to-nearest-even,
+// saturating ("satfinite") converts; conversions from them are exact.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#ifndef __CUDACC_RTC__
+#include <cstddef>
+#endif
+
+namespace mtp {
+
+// ---------------------------------------------------------------- bf16 / fp32 bits
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+__device__ __forceinline__ float bf16_to_f32(uint16_t v) { return __uint_as_float((uint32_t)v << 16); }
+
+// fp32 -> bf16, round to nearest even (hardware convert).
+__device__ __forceinline__ uint16_t f32_to_bf16(float f) {
+    uint16_t r;
+    asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(f));
+    return r;
+}
+
+// fp32 -> f16, round to nearest even.
+__device__ __forceinline__ uint16_t f32_to_f16(float f) {
+    uint16_t r;
+    asm("cvt.rn.f16.f32 %0, %1;" : "=h"(r) : "f"(f));
+    return r;
+}
+
+// ---------------------------------------------------------------- narrow formats
+// Two fp32 -> two E4M3 codes; `lo` lands in bits 0..7, `hi` in bits 8..15.
+__device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Two fp32 -> two E2M1 codes in one byte; `lo` in bits 0..3, `hi` in bits 4..7.
+__device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 q;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q, %1, %2;\n\t"
+        "cvt.u32.u8 %0, q;\n\t}"
+        : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Exact decode of one E4M3 code to fp32 (used off the hot path).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
+    uint32_t h2;
+    uint16_t c = (uint16_t)(code & 0xFF);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(c));
+    float f;
+    asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.f32.f16 %0, lo;\n\t}"
+        : "=f"(f) : "r"(h2));
+    return f;
+}
+
+// Two E4M3 codes (bits 0..7 and 8..15) -> f16x2 (low half from bits 0..7). Exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
+    return r;
+}
+
+// Eight E2M1 codes packed in a word (element 2j in the low nibble of byte j) ->
+// four f16x2 registers, element order preserved (low half = lower element). Exact.
+__device__ __forceinline__ void e2m1x8_to_f16x2x4(uint32_t w, uint32_t (&o)[4]) {
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3]) : "r"(w));
+}
+
+// Packed f16x2 multiply (round to nearest). Used only where the product is exact.
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// ---------------------------------------------------------------- tensor-core MMA
+// D[16x8] += A[16x16] * B[16x8], fp32 accumulate. Fragment layout (lane = 4g + c):
+//   A: a0 = (row g,   k 2c..2c+1), a1 = (row g+8, k 2c..2c+1),
+//      a2 = (row g,   k 2c+8..+9), a3 = (row g+8, k 2c+8..+9)
+//   B: b0 = (k 2c..2c+1, col g),   b1 = (k 2c+8..+9, col g)
+//   D: d0,d1 = (row g, cols 2c, 2c+1), d2,d3 = (row g+8, cols 2c, 2c+1)
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
+                                              uint32_t a2, uint32_t a3, uint32_t b0,
+                                              uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// ---------------------------------------------------------------- memory
+// Streaming 16-byte load: read once, do not keep in L1.
+__device__ __forceinline__ uint4 ldg_stream(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t ldg_u16(const void* p) {
+    unsigned short r;
+    asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(r) : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ uint4 lds128(const void* p) {
+    return *reinterpret_cast<const uint4*>(p);
+}
+
+// Device error word bits (a copy of the public MTP_DEVFLAG_* values).
+enum : int32_t { DEVFLAG_BAD_TOKEN = 1, DEVFLAG_EMPTY_MASK = 2, DEVFLAG_BAD_SLOT = 4,
+                 DEVFLAG_TIMEOUT = 8 };
+
+__device__ __forceinline__ void raise_flag(int32_t* dev_err, int32_t f) {
+    if (dev_err) atomicOr(dev_err, f);
+}
+
+}  // namespace mtp

@@ -1,0 +1,73 @@
+// Internal launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mtp {
+
+// One draft-head GEMV sweep over rows [0, n) of a [*, k] table, with x staged per CTA.
+// mode 0: fused argmax (+ optional logits); mode 1: combiner (x built from the
+// embedding row and target hidden, output y = bf16(W . c)).
+struct SweepParams {
+    const uint8_t* w;            // table bytes, rows packed at `row_bytes`
+    const float* row_scale;      // FP8: f32[n]
+    const uint8_t* block_scale;  // NVFP4: e4m3[n, k/16]
+    const float* global_scale;   // NVFP4: f32[1] on the device
+    int64_t n;                   // rows swept
+    int64_t k;                   // reduction length (table columns)
+    int64_t row_bytes;
+    int32_t M;                   // input rows (1..16)
+    int32_t kpad;                // staged-x row stride in elements
+    // mode 0 input
+    const uint16_t* x;           // bf16 [M, k]
+    // mode 1 inputs (k == 2h)
+    const uint16_t* embed;
+    int64_t vocab;
+    const int32_t* tokens;       // [M]
+    const uint16_t* hidden;      // bf16 [M, h]
+    const uint16_t* w_norm_embed;
+    const uint16_t* w_norm_hidden;
+    float eps;
+    int32_t h;
+    // grammar mask (mode 0)
+    const int32_t* mask;
+    int64_t mask_words;
+    int64_t mask_stride;
+    // outputs
+    int32_t* out_idx;
+    float* out_val;
+    uint16_t* out_logits;        // bf16 [M, n] or null
+    uint16_t* out_y;             // mode 1: bf16 [M, n]
+    int32_t* dev_err;
+    // workspace (mode 0)
+    uint32_t* ticket;
+    void* partials;
+    int64_t num_tiles;
+};
+
+struct SweepLaunch {
+    int grid;
+    int smem_bytes;
+};
+
+// Picks the kernel instance and grid; returns cudaErrorInvalidValue if the staged
+// input does not fit in shared memory.
+cudaError_t sweep_launch(const SweepParams& p, int fmt, int mode, cudaStream_t s,
+                         SweepLaunch* info);
+size_t sweep_smem_bytes(int M, int64_t k, int fmt, int* kpad_out);
+int sweep_max_grid();
+
+// Quantizers.
+cudaError_t quant_fp8_launch(const uint16_t* w, int64_t n, int64_t k, uint8_t* codes,
+                             float* row_scale, cudaStream_t s);
+cudaError_t quant_nvfp4_launch(const uint16_t* w, int64_t n, int64_t k, uint8_t* codes,
+                               uint8_t* block_scale, float* global_scale, uint32_t* ws,
+                               cudaStream_t s);
+int quant_nvfp4_max_grid();
+
+// Encoders exposed for exhaustive checks.
+cudaError_t debug_encode_launch(const float* in, int64_t n, uint8_t* out, int which,
+                                cudaStream_t s);
+
+}  // namespace mtp

@@ -1,0 +1,143 @@
+"""The C ABI without a GPU: the library loads, exports every symbol include/mtp.h
+declares, and rejects bad arguments on the host before any CUDA call."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from mtp_speculative_draft_lm_b200 import _lib as L
+from mtp_speculative_draft_lm_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return L.load()
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(mtp_\w+)\s*\(", text))
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(L.EXPORTS) == names
+
+
+def test_version_and_status_strings(lib):
+    assert L.mtp_abi_version() == 1
+    for s in range(6):
+        assert L.status_str(s)
+    assert L.mtp_devflags_status(0) == L.MTP_OK
+    assert L.mtp_devflags_status(L.MTP_DEVFLAG_EMPTY_MASK) == L.MTP_WARN_EMPTY_MASK
+    assert L.mtp_devflags_status(L.MTP_DEVFLAG_BAD_TOKEN) == L.MTP_ERR_INVALID_ARG
+
+
+# Fake 256-byte-aligned addresses: every call below fails validation first, so they
+# are never dereferenced and no CUDA call is made.
+A = 0x10000
+B2 = 0x20000
+OUT = 0x30000
+
+
+def st(name, *args):
+    return L.raw_status(name, *args)
+
+
+def test_quantize_fp8_rejects(lib):
+    assert st("mtp_quantize_fp8", None, 4, 32, OUT, OUT, None) == L.MTP_ERR_INVALID_ARG
+    assert st("mtp_quantize_fp8", A, 4, 24, OUT, OUT, None) == L.MTP_ERR_INVALID_ARG  # k % 16
+    assert st("mtp_quantize_fp8", A, 0, 32, OUT, OUT, None) == L.MTP_ERR_INVALID_ARG
+    assert st("mtp_quantize_fp8", A + 2, 4, 32, OUT, OUT, None) == L.MTP_ERR_INVALID_ARG
+
+
+def test_quantize_nvfp4_rejects(lib):
+    ws_need = L.mtp_quantize_nvfp4_ws_bytes(4, 64)
+    assert ws_need >= 256
+    assert st("mtp_quantize_nvfp4", A, 4, 48, OUT, OUT, OUT, B2, ws_need, None) == \
+        L.MTP_ERR_INVALID_ARG  # k % 32
+    assert st("mtp_quantize_nvfp4", A, 4, 64, OUT, OUT, OUT, None, ws_need, None) == \
+        L.MTP_ERR_WORKSPACE
+    assert st("mtp_quantize_nvfp4", A, 4, 64, OUT, OUT, OUT, B2, ws_need - 1, None) == \
+        L.MTP_ERR_WORKSPACE
+
+
+def weight(fmt=L.MTP_FMT_BF16, n=100, k=64, data=A, rs=None, bs=None, gs=None):
+    return L.mtp_weight(fmt, 0, n, k, data, rs, bs, gs)
+
+
+def lm(head, n_eff=100, x=B2, M=1, mask=None, mw=0, ms=0, idx=OUT, ws=0x40000, wsb=None):
+    if wsb is None:
+        wsb = L.mtp_lm_head_ws_bytes(head, n_eff, M)
+    return st("mtp_lm_head_argmax", C.byref(head), n_eff, x, M, mask, mw, ms, idx, None, None,
+              None, ws, wsb, None)
+
+
+def test_lm_head_rejects(lib):
+    assert st("mtp_lm_head_argmax", None, 1, B2, 1, None, 0, 0, OUT, None, None, None,
+              0x40000, 1 << 20, None) == L.MTP_ERR_INVALID_ARG
+    assert lm(weight(k=60)) == L.MTP_ERR_INVALID_ARG             # bf16 k % 8
+    assert lm(weight(fmt=1, k=40, rs=OUT)) == L.MTP_ERR_INVALID_ARG  # fp8 k % 16
+    assert lm(weight(fmt=1, k=64)) == L.MTP_ERR_INVALID_ARG       # fp8 needs row scales
+    assert lm(weight(fmt=2, k=48, bs=OUT, gs=OUT)) == L.MTP_ERR_INVALID_ARG  # nvfp4 k % 32
+    assert lm(weight(fmt=2, k=64, bs=OUT)) == L.MTP_ERR_INVALID_ARG  # no global scale
+    assert lm(weight(fmt=0, k=64, rs=OUT)) == L.MTP_ERR_INVALID_ARG  # stray pointer
+    assert lm(weight(fmt=7)) == L.MTP_ERR_INVALID_ARG
+    assert lm(weight(data=A + 8)) == L.MTP_ERR_INVALID_ARG        # 16-byte alignment
+    assert lm(weight(), n_eff=101) == L.MTP_ERR_INVALID_ARG       # n_eff > n
+    assert lm(weight(), n_eff=0) == L.MTP_ERR_INVALID_ARG
+    assert lm(weight(), M=0) == L.MTP_ERR_UNSUPPORTED
+    assert lm(weight(), M=17) == L.MTP_ERR_UNSUPPORTED
+    assert lm(weight(), x=B2 + 4) == L.MTP_ERR_INVALID_ARG
+    assert lm(weight(), mask=OUT, mw=0) == L.MTP_ERR_INVALID_ARG
+    assert lm(weight(), ws=None) == L.MTP_ERR_WORKSPACE
+    assert lm(weight(), wsb=16) == L.MTP_ERR_WORKSPACE
+    # staged inputs larger than shared memory
+    assert lm(weight(n=100, k=16384), M=16) == L.MTP_ERR_UNSUPPORTED
+    w = weight()
+    w.reserved = 1
+    assert lm(w) == L.MTP_ERR_INVALID_ARG
+
+
+def test_combine_rejects(lib):
+    fc = weight(n=32, k=64)
+    args = [A, 50, B2, B2, 1, 32, OUT, OUT, 1e-6, C.byref(fc), OUT, None, None]
+    bad = list(args)
+    bad[0] = None
+    assert st("mtp_combine", *bad) == L.MTP_ERR_INVALID_ARG
+    bad = list(args)
+    bad[4] = 17
+    assert st("mtp_combine", *bad) == L.MTP_ERR_UNSUPPORTED
+    bad = list(args)
+    bad[5] = 24  # h % 16
+    assert st("mtp_combine", *bad) == L.MTP_ERR_INVALID_ARG
+    fc2 = weight(n=32, k=32)  # fc must be [h, 2h]
+    bad = list(args)
+    bad[9] = C.byref(fc2)
+    assert st("mtp_combine", *bad) == L.MTP_ERR_INVALID_ARG
+    bad = list(args)
+    bad[8] = -1.0
+    assert st("mtp_combine", *bad) == L.MTP_ERR_INVALID_ARG
+
+
+def test_debug_encoders_reject(lib):
+    assert st("mtp_debug_encode_e4m3", None, 4, OUT, None) == L.MTP_ERR_INVALID_ARG
+    assert st("mtp_debug_encode_e2m1", A, 0, OUT, None) == L.MTP_ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    monkeypatch.setattr(L, "_lib", None)
+    with pytest.raises(OSError):
+        L.load(str(tmp_path / "none.so"))

@@ -1,0 +1,97 @@
+"""The combiner (embedding row, two RMSNorms, concat, fc) and the tiny end-to-end
+draft step (hidden 256, vocab 4096) on the GPU against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+from helpers import assert_argmax, assert_close, bf16_bits_to_f64, to_dev, to_dev_u16, u16_of
+from mtp_speculative_draft_lm_b200 import _lib as L
+from mtp_speculative_draft_lm_b200 import api, synth
+
+pytestmark = pytest.mark.gpu
+
+
+def draft(M, seed=synth.TINY["seed"], h=synth.TINY["h"], vocab=synth.TINY["vocab"]):
+    d = synth.tiny_draft(seed=seed, vocab=vocab, h=h, M=M)
+    return {k: (synth.as_u16(v) if isinstance(v, torch.Tensor) and v.dtype == torch.bfloat16
+                else v) for k, v in d.items()}
+
+
+def gpu_combine(d, fc_table=None, tokens=None):
+    fc = fc_table or api.bf16_table(to_dev_u16(d["fc"]))
+    err = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    tok = to_dev(np.asarray(d["tokens"] if tokens is None else tokens, np.int32))
+    y = api.combine(to_dev_u16(d["embed"]), tok, to_dev_u16(d["hidden"]),
+                    to_dev_u16(d["w_norm_embed"]), to_dev_u16(d["w_norm_hidden"]), d["eps"], fc,
+                    dev_err=err)
+    torch.cuda.synchronize()
+    return u16_of(y), int(err.item())
+
+
+@pytest.mark.parametrize("M", [1, 2, 5, 8, 16])
+def test_combine_matches_oracle(orc, M):
+    d = draft(M)
+    y, err = gpu_combine(d)
+    ref, _, flags = orc.combine(d["embed"], d["tokens"].numpy(), d["hidden"], d["w_norm_embed"],
+                                d["w_norm_hidden"], d["eps"], d["fc"])
+    assert err == 0 and flags == 0
+    assert_close(bf16_bits_to_f64(y), bf16_bits_to_f64(ref), "y")
+    # bf16 outputs: all but a handful identical, none more than one bf16 ulp apart
+    diff = np.abs(y.astype(np.int32) - ref.astype(np.int32))
+    assert diff.max() <= 1 and (diff > 0).mean() < 0.02
+
+
+@pytest.mark.parametrize("h", [16, 512, 1024])
+def test_combine_other_widths(orc, h):
+    d = draft(3, seed=5, h=h, vocab=300)
+    y, _ = gpu_combine(d)
+    ref, _, _ = orc.combine(d["embed"], d["tokens"].numpy(), d["hidden"], d["w_norm_embed"],
+                            d["w_norm_hidden"], d["eps"], d["fc"])
+    assert_close(bf16_bits_to_f64(y), bf16_bits_to_f64(ref), "y")
+
+
+def test_combine_bad_token_flag(orc):
+    d = draft(2)
+    toks = np.array([d["vocab"] + 5, 3], np.int32)
+    y, err = gpu_combine(d, tokens=toks)
+    assert err & L.MTP_DEVFLAG_BAD_TOKEN
+    ref, _, flags = orc.combine(d["embed"], toks, d["hidden"], d["w_norm_embed"],
+                                d["w_norm_hidden"], d["eps"], d["fc"])
+    assert flags & 1
+    assert_close(bf16_bits_to_f64(y), bf16_bits_to_f64(ref), "y")
+
+
+@pytest.mark.parametrize("fmt", [1, 2])
+def test_combine_quantized_fc(orc, fmt):
+    d = draft(4, seed=6)
+    h = d["h"]
+    if fmt == 1:
+        c, s = orc.quantize_fp8(d["fc"])
+        fc = api.Table(1, h, 2 * h, to_dev(c), row_scale=to_dev(s))
+        deq = orc.dequant(1, c, 2 * h, row_scale=s)
+    else:
+        c, b, g = orc.quantize_nvfp4(d["fc"])
+        fc = api.Table(2, h, 2 * h, to_dev(c), block_scale=to_dev(b),
+                       global_scale=torch.tensor([g], dtype=torch.float32, device="cuda"))
+        deq = orc.dequant(2, c, 2 * h, block_scale=b, global_scale=g)
+    y, _ = gpu_combine(d, fc_table=fc)
+    _, concat, _ = orc.combine(d["embed"], d["tokens"].numpy(), d["hidden"], d["w_norm_embed"],
+                               d["w_norm_hidden"], d["eps"], d["fc"])
+    ref = orc.f64_to_bf16(bf16_bits_to_f64(concat) @ deq.T)
+    assert_close(bf16_bits_to_f64(y), bf16_bits_to_f64(ref), "y")
+
+
+@pytest.mark.parametrize("M", [1, 4])
+def test_tiny_draft_end_to_end(orc, M):
+    """combine -> lm_head sweep -> argmax on the hidden-256 / vocab-4096 draft."""
+    d = draft(M)
+    y, _ = gpu_combine(d)
+    head = api.LmHead(api.bf16_table(to_dev_u16(d["lm_head"])))
+    idx, val, lg = head.argmax(to_dev_u16(y), logits=True)
+    torch.cuda.synchronize()
+    ref_y, _, _ = orc.combine(d["embed"], d["tokens"].numpy(), d["hidden"], d["w_norm_embed"],
+                              d["w_norm_hidden"], d["eps"], d["fc"])
+    ref_l, ref_i, ref_v, _ = orc.lm_head_argmax(0, d["lm_head"], d["h"], ref_y)
+    for m in range(M):
+        assert_argmax(int(idx[m].item()), ref_l[m])
+        assert_close(bf16_bits_to_f64(u16_of(lg)[m]), ref_l[m], "logits")
