@@ -141,13 +141,15 @@ def max_over_ranks(v: float, world: int) -> float:
     return float(t.item())
 
 
-def build_table(fmt: str, dev):
+def build_table(fmt: str, dev, rows: int = 0):
     """Seeded synthetic table for one format (quantized on the device)."""
     import torch
 
     from mtp_speculative_draft_lm_b200 import api, synth
 
-    cfg = {"bf16": synth.BF16_HEAD, "fp8": synth.FP8_HEAD, "nvfp4": synth.NVFP4_HEAD}[fmt]
+    cfg = dict({"bf16": synth.BF16_HEAD, "fp8": synth.FP8_HEAD, "nvfp4": synth.NVFP4_HEAD}[fmt])
+    if rows:
+        cfg["N"] = rows
     d = synth.head_table(cfg["seed"], cfg["N"], cfg["K"], max(cfg["Ms"]),
                          mask_keep=cfg.get("mask_keep"))
     w = d["W"].to(dev)
@@ -318,6 +320,8 @@ def main():
     ap.add_argument("--full", action="store_true", help="also M>1 and masked rows")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--formats", default="bf16,fp8,nvfp4")
+    ap.add_argument("--rows", type=int, default=0,
+                    help="sweep a smaller table of this many rows (profiling cases)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     if args.impl == "reference":
@@ -336,7 +340,7 @@ def main():
     main_line = None
     cpu_base = None
     for fmt in args.formats.split(","):
-        cfg, d, table, qinfo = build_table(fmt, dev)
+        cfg, d, table, qinfo = build_table(fmt, dev, args.rows)
         head = api.LmHead(table)
         Ms = cfg["Ms"] if args.full else (1,)
         for M in Ms:

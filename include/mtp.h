@@ -55,6 +55,8 @@ typedef enum {
 #define MTP_DEVFLAG_BAD_TOKEN 1  /* token id outside [0, vocab): its row read as zeros */
 #define MTP_DEVFLAG_EMPTY_MASK 2 /* a row's mask allowed nothing: idx 0, value -inf */
 #define MTP_DEVFLAG_BAD_SLOT 4   /* a cache row had no valid block: row not written */
+#define MTP_DEVFLAG_TIMEOUT 8    /* an internal pipeline wait ran out (about 1 s): the
+                                    call's outputs are not valid */
 
 /* Weight formats ([mtp_head.rs] MtpQuantization and ProjectionWeight: Bf16, Fp8,
  * Nvfp4). */
@@ -62,14 +64,16 @@ typedef enum {
     MTP_FMT_BF16 = 0,    /* data: bf16 [n, k] */
     MTP_FMT_FP8_ROW = 1, /* data: E4M3FN codes [n, k]; row_scale: f32 [n] */
     MTP_FMT_NVFP4 = 2    /* data: E2M1 codes [n, k/2] (element 2j = low nibble of byte
-                            j); block_scale: E4M3FN [n, k/16]; global_scale: f32[1] */
+                            j); block_scale: E4M3FN [n, pitch] with
+                            pitch = mtp_nvfp4_scale_pitch(k) (k/16 rounded up to a
+                            multiple of 16; padding bytes zero); global_scale: f32[1] */
 } mtp_format;
 
 /* A [n, k] weight table in one of the formats, rows packed at k (no row stride:
  * [init.rs] notes the draft-head GEMV assumes rows packed at K). All pointers are
- * device pointers; the unused ones must be NULL. dequant(W)[r, j] is the bf16
- * value, e4m3(code) * row_scale[r], or e2m1(code) * e4m3(block_scale[r, j/16]) *
- * global_scale[0]. */
+ * device pointers (data and block_scale 16-byte aligned); the unused ones must be
+ * NULL. dequant(W)[r, j] is the bf16 value, e4m3(code) * row_scale[r], or
+ * e2m1(code) * e4m3(block_scale[r * pitch + j/16]) * global_scale[0]. */
 typedef struct {
     int32_t fmt;
     int32_t reserved; /* must be 0 */
@@ -80,6 +84,10 @@ typedef struct {
     const uint8_t* block_scale;
     const float* global_scale;
 } mtp_weight;
+
+/* Row pitch in bytes of an NVFP4 block-scale table: k/16 rounded up to a multiple
+ * of 16, so that every row starts 16-byte aligned. */
+int64_t mtp_nvfp4_scale_pitch(int64_t k);
 
 /* ---------------------------------------------------------------------------------
  * mtp_quantize_fp8 -- BF16 -> FP8 E4M3 with one fp32 scale per row.
@@ -106,7 +114,8 @@ mtp_status mtp_quantize_fp8(const uint16_t* w, int64_t n, int64_t k, uint8_t* co
  * S = e4m3(sb) * g, code = e2m1_satfinite(w / S) (0 when S == 0).
  *   w            (device) bf16 [n, k], 16-byte aligned
  *   codes        (device) u8 [n, k/2] written (two codes per byte, element 2j low)
- *   block_scale  (device) u8 [n, k/16] written
+ *   block_scale  (device) u8 [n, mtp_nvfp4_scale_pitch(k)] written (16-byte aligned;
+ *                the padding after the k/16 scales of each row is written as 0)
  *   global_scale (device) f32 [1] written (g)
  *   ws           (device) >= mtp_quantize_nvfp4_ws_bytes(n, k) bytes, 16-byte
  *                aligned, ALL ZERO before the first call; each call leaves it zero.
@@ -134,8 +143,9 @@ mtp_status mtp_quantize_nvfp4(const uint16_t* w, int64_t n, int64_t k, uint8_t* 
  *                 MTP_FMT_NVFP4)
  *   out           (device) bf16 [M, h], written
  *   dev_err       (device) i32 [1] or NULL
- * Requires 1 <= M <= 16, h % 16 == 0 (fc's k must meet its format's k rule), all
- * device pointers 16-byte aligned except token_ids / dev_err (4-byte).
+ * Requires 1 <= M <= 16, h % 16 == 0, fc rows a multiple of 128 bytes (2h % 64 for
+ * BF16, % 128 for FP8, % 256 for NVFP4), all device pointers 16-byte aligned except
+ * token_ids / dev_err (4-byte).
  * ------------------------------------------------------------------------------ */
 mtp_status mtp_combine(const uint16_t* embed, int64_t vocab, const int32_t* token_ids,
                        const uint16_t* hidden, int32_t M, int32_t h,
@@ -165,9 +175,10 @@ mtp_status mtp_combine(const uint16_t* embed, int64_t vocab, const int32_t* toke
  *   ws            (device) >= mtp_lm_head_ws_bytes(head, n_eff, M) bytes, 16-byte
  *                 aligned, ALL ZERO before the first call; each call leaves its
  *                 counter zero again.
- * Requires 1 <= M <= 16, 1 <= n_eff <= n; k % 8 (BF16), k % 16 (FP8), k % 32 (NVFP4);
- * the staged inputs (M * k * 2 bytes) must fit in shared memory (MTP_ERR_UNSUPPORTED
- * otherwise).
+ * Requires 1 <= M <= 16, 1 <= n_eff <= n; table rows a multiple of 128 bytes (k % 64
+ * for BF16, % 128 for FP8, % 256 for NVFP4; the sweep streams 128-byte segments) and
+ * the staged inputs (M * k * 2 bytes) small enough to leave shared memory for the
+ * stream (MTP_ERR_UNSUPPORTED otherwise).
  * ------------------------------------------------------------------------------ */
 size_t mtp_lm_head_ws_bytes(const mtp_weight* head, int64_t n_eff, int32_t M);
 mtp_status mtp_lm_head_argmax(const mtp_weight* head, int64_t n_eff, const uint16_t* x,

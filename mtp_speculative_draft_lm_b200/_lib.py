@@ -24,6 +24,7 @@ MTP_WARN_EMPTY_MASK = 5
 MTP_DEVFLAG_BAD_TOKEN = 1
 MTP_DEVFLAG_EMPTY_MASK = 2
 MTP_DEVFLAG_BAD_SLOT = 4
+MTP_DEVFLAG_TIMEOUT = 8
 
 MTP_FMT_BF16 = 0
 MTP_FMT_FP8_ROW = 1
@@ -34,7 +35,7 @@ EXPORTS = (
     "mtp_abi_version", "mtp_status_str", "mtp_devflags_status",
     "mtp_quantize_fp8", "mtp_quantize_nvfp4_ws_bytes", "mtp_quantize_nvfp4",
     "mtp_combine", "mtp_lm_head_ws_bytes", "mtp_lm_head_argmax",
-    "mtp_debug_encode_e4m3", "mtp_debug_encode_e2m1",
+    "mtp_debug_encode_e4m3", "mtp_debug_encode_e2m1", "mtp_nvfp4_scale_pitch",
 )
 
 
@@ -62,6 +63,7 @@ _SIGS = {
     "mtp_devflags_status": (C.c_int, [_I32]),
     "mtp_quantize_fp8": (C.c_int, [_P, _I64, _I64, _P, _P, _P]),
     "mtp_quantize_nvfp4_ws_bytes": (_SZ, [_I64, _I64]),
+    "mtp_nvfp4_scale_pitch": (_I64, [_I64]),
     "mtp_quantize_nvfp4": (C.c_int, [_P, _I64, _I64, _P, _P, _P, _P, _SZ, _P]),
     "mtp_combine": (C.c_int, [_P, _I64, _P, _P, _I32, _I32, _P, _P, C.c_float, _W, _P, _P,
                               _P]),
@@ -134,6 +136,10 @@ def mtp_devflags_status(value: int) -> int:
 def mtp_quantize_fp8(w, n, k, codes, row_scale, stream=None):
     _check(load().mtp_quantize_fp8(_ptr(w), n, k, _ptr(codes), _ptr(row_scale),
                                    _stream(stream)), "mtp_quantize_fp8")
+
+
+def mtp_nvfp4_scale_pitch(k) -> int:
+    return load().mtp_nvfp4_scale_pitch(k)
 
 
 def mtp_quantize_nvfp4_ws_bytes(n, k) -> int:

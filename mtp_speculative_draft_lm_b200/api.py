@@ -55,7 +55,7 @@ def quantize_fp8(w: torch.Tensor, stream=None) -> Table:
 def quantize_nvfp4(w: torch.Tensor, ws: torch.Tensor | None = None, stream=None) -> Table:
     n, k = w.shape
     codes = torch.empty((n, k // 2), dtype=torch.uint8, device=w.device)
-    bscale = torch.empty((n, k // 16), dtype=torch.uint8, device=w.device)
+    bscale = torch.empty((n, L.mtp_nvfp4_scale_pitch(k)), dtype=torch.uint8, device=w.device)
     g = torch.empty((1,), dtype=torch.float32, device=w.device)
     nbytes = L.mtp_quantize_nvfp4_ws_bytes(n, k)
     if ws is None:

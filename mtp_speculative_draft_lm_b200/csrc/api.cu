@@ -35,13 +35,19 @@ mtp_status check_weight(const mtp_weight* w) {
         case MTP_FMT_NVFP4:
             if (w->k % 32 || w->row_scale || !w->block_scale || !w->global_scale)
                 return MTP_ERR_INVALID_ARG;
-            if (!aligned(w->block_scale, 2) || !aligned(w->global_scale, 4))
+            if (!aligned(w->block_scale, 16) || !aligned(w->global_scale, 4))
                 return MTP_ERR_INVALID_ARG;
             return MTP_OK;
         default:
             return MTP_ERR_INVALID_ARG;
     }
 }
+
+}  // namespace
+
+extern "C" int64_t mtp_nvfp4_scale_pitch(int64_t k) { return mtp::nvfp4_scale_pitch(k); }
+
+namespace {
 
 int64_t row_bytes(const mtp_weight* w) {
     return w->fmt == MTP_FMT_BF16 ? w->k * 2 : w->fmt == MTP_FMT_FP8_ROW ? w->k : w->k / 2;
@@ -94,7 +100,8 @@ mtp_status mtp_quantize_nvfp4(const uint16_t* w, int64_t n, int64_t k, uint8_t* 
                               size_t ws_bytes, void* stream) {
     if (!w || !codes || !block_scale || !global_scale || n < 1 || k < 32 || k % 32)
         return MTP_ERR_INVALID_ARG;
-    if (!aligned(w, 16) || !aligned(codes, 16) || !aligned(global_scale, 4))
+    if (!aligned(w, 16) || !aligned(codes, 16) || !aligned(block_scale, 16) ||
+        !aligned(global_scale, 4))
         return MTP_ERR_INVALID_ARG;
     if (!ws || !aligned(ws, 16) || ws_bytes < mtp_quantize_nvfp4_ws_bytes(n, k))
         return MTP_ERR_WORKSPACE;
@@ -114,6 +121,7 @@ mtp_status mtp_combine(const uint16_t* embed, int64_t vocab, const int32_t* toke
     mtp_status st = check_weight(fc);
     if (st != MTP_OK) return st;
     if (fc->n != h || fc->k != 2 * (int64_t)h) return MTP_ERR_INVALID_ARG;
+    if (row_bytes(fc) % 128) return MTP_ERR_UNSUPPORTED;
     if (!aligned(embed, 16) || !aligned(hidden, 16) || !aligned(out, 16) ||
         !aligned(w_norm_embed, 4) || !aligned(w_norm_hidden, 4) || !aligned(token_ids, 4) ||
         !aligned(dev_err, 4))
@@ -139,6 +147,7 @@ mtp_status mtp_combine(const uint16_t* embed, int64_t vocab, const int32_t* toke
     p.out_y = out;
     p.dev_err = dev_err;
     p.num_tiles = (fc->n + 15) / 16;
+    p.scale_pitch = mtp::nvfp4_scale_pitch(fc->k);
     return from_cuda(mtp::sweep_launch(p, fc->fmt, 1, as_stream(stream), nullptr));
 }
 
@@ -157,7 +166,7 @@ mtp_status mtp_lm_head_argmax(const mtp_weight* head, int64_t n_eff, const uint1
     mtp_status st = check_weight(head);
     if (st != MTP_OK) return st;
     if (!x || !out_idx || n_eff < 1 || n_eff > head->n) return MTP_ERR_INVALID_ARG;
-    if (n_eff > (int64_t)INT32_MAX) return MTP_ERR_UNSUPPORTED;
+    if (n_eff > (int64_t)INT32_MAX || row_bytes(head) % 128) return MTP_ERR_UNSUPPORTED;
     if (M < 1 || M > kMaxM) return MTP_ERR_UNSUPPORTED;
     if (mask && (mask_words < 1 || mask_stride_words < 0)) return MTP_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(out_idx, 4) || !aligned(out_val, 4) ||
@@ -187,6 +196,7 @@ mtp_status mtp_lm_head_argmax(const mtp_weight* head, int64_t n_eff, const uint1
     p.ticket = static_cast<uint32_t*>(ws);
     p.partials = static_cast<uint8_t*>(ws) + kTicketBytes;
     p.num_tiles = (n_eff + 15) / 16;
+    p.scale_pitch = mtp::nvfp4_scale_pitch(head->k);
     return from_cuda(mtp::sweep_launch(p, head->fmt, 0, as_stream(stream), nullptr));
 }
 

@@ -44,6 +44,9 @@ struct SweepParams {
     uint32_t* ticket;
     void* partials;
     int64_t num_tiles;
+    int64_t scale_pitch;         // NVFP4: bytes between block-scale rows
+    int32_t stages;              // ring depth (set by the launcher)
+    int32_t stage_bytes;
 };
 
 struct SweepLaunch {
@@ -65,6 +68,7 @@ cudaError_t quant_nvfp4_launch(const uint16_t* w, int64_t n, int64_t k, uint8_t*
                                uint8_t* block_scale, float* global_scale, uint32_t* ws,
                                cudaStream_t s);
 int quant_nvfp4_max_grid();
+int64_t nvfp4_scale_pitch(int64_t k);
 
 // Encoders exposed for exhaustive checks.
 cudaError_t debug_encode_launch(const float* in, int64_t n, uint8_t* out, int which,

@@ -9,6 +9,8 @@
 //   NVFP4:        A = max|W|, g = A / 2688 (1 when A == 0); per 16-block:
 //                 B = max|W_b|, sb = e4m3((B / 6) / g), S = e4m3(sb) * g,
 //                 q = e2m1(W / S) (0 when S == 0); element 2j in the low nibble.
+//                 Block-scale rows are padded with zeros to a multiple of 16 bytes so that
+//                 every row starts 16-byte aligned (the sweep streams them with TMA).
 //
 // E4M3/E2M1 encodes use the hardware satfinite converts (round to nearest even,
 // saturating); the exhaustive checks compare them with the CPU oracle.
@@ -102,15 +104,18 @@ __global__ void __launch_bounds__(kQThreads) nvfp4_absmax_kernel(const uint16_t*
     }
 }
 
-// Pass 2: one thread per 16-element block.
+// Pass 2: one thread per 16-element block. Block-scale rows are `pitch` bytes long
+// (k/16 rounded up to 16); the padding bytes are written as zero.
 __global__ void __launch_bounds__(kQThreads) nvfp4_encode_kernel(const uint16_t* __restrict__ w,
-                                                                 int64_t blocks,
+                                                                 int64_t n, int64_t nb,
+                                                                 int64_t pitch,
                                                                  uint8_t* __restrict__ codes,
                                                                  uint8_t* __restrict__ bscale,
                                                                  const float* global_scale) {
     const float g = *global_scale;
-    for (int64_t b = (int64_t)blockIdx.x * kQThreads + threadIdx.x; b < blocks;
-         b += (int64_t)gridDim.x * kQThreads) {
+    const int64_t blocks = n * nb;
+    const int64_t stride = (int64_t)gridDim.x * kQThreads;
+    for (int64_t b = (int64_t)blockIdx.x * kQThreads + threadIdx.x; b < blocks; b += stride) {
         const uint4 v0 = ldg_stream(w + b * 16);
         const uint4 v1 = ldg_stream(w + b * 16 + 8);
         const float B = fmaxf(absmax8(v0), absmax8(v1));
@@ -129,7 +134,15 @@ __global__ void __launch_bounds__(kQThreads) nvfp4_encode_kernel(const uint16_t*
             q.y = bytes[4] | (bytes[5] << 8) | (bytes[6] << 16) | (bytes[7] << 24);
         }
         *reinterpret_cast<uint2*>(codes + b * 8) = q;
-        bscale[b] = (uint8_t)sb;
+        const int64_t r = b / nb;
+        bscale[r * pitch + (b - r * nb)] = (uint8_t)sb;
+    }
+    const int64_t pad = pitch - nb;
+    if (pad > 0) {
+        for (int64_t i = (int64_t)blockIdx.x * kQThreads + threadIdx.x; i < n * pad; i += stride) {
+            const int64_t r = i / pad;
+            bscale[r * pitch + nb + (i - r * pad)] = 0;
+        }
     }
 }
 
@@ -152,6 +165,8 @@ int sm_count() {
 }  // namespace
 
 int quant_nvfp4_max_grid() { return kAbsmaxMaxGrid; }
+
+int64_t nvfp4_scale_pitch(int64_t k) { return ((k / 16 + 15) / 16) * 16; }
 
 cudaError_t quant_fp8_launch(const uint16_t* w, int64_t n, int64_t k, uint8_t* codes,
                              float* row_scale, cudaStream_t s) {
@@ -177,8 +192,8 @@ cudaError_t quant_nvfp4_launch(const uint16_t* w, int64_t n, int64_t k, uint8_t*
     int64_t g2 = (blocks + kQThreads - 1) / kQThreads;
     const int64_t cap2 = (int64_t)sm_count() * 8;
     if (g2 > cap2) g2 = cap2;
-    nvfp4_encode_kernel<<<(int)g2, kQThreads, 0, s>>>(w, blocks, codes, block_scale,
-                                                        global_scale);
+    nvfp4_encode_kernel<<<(int)g2, kQThreads, 0, s>>>(w, n, k / 16, nvfp4_scale_pitch(k), codes,
+                                                        block_scale, global_scale);
     return cudaGetLastError();
 }
 

@@ -8,23 +8,34 @@
 // with deq(W) the BF16 value, an E4M3 code (row scale s_n) or an E2M1 code times its
 // E4M3 block scale (global scale s_n = g).
 //
-// Design (B200): the sweep is HBM-bound, so the whole table is streamed exactly once
-// with 16-byte non-allocating loads, many in flight per thread. A CTA of 8 warps owns
-// a contiguous range of 16-row tiles; the 8 warps split K (slab s of 4 lanes x 16 B
-// goes to warp s % 8). Each warp turns its slab into tensor-core MMAs with the table
-// rows as the 16-row A operand and the inputs as the 8-column B operand (swap-AB),
-// so dequantization needs one convert per 2 codes and no FP32 FMA work; codes are
-// decoded exactly into f16 (E4M3, and E2M1 times the E4M3 block scale, are exact in
-// f16) and x is staged once per CTA in shared memory (bf16 for BF16 tables; f16
-// scaled by a per-row power of two for quantized tables, undone in fp32 at the end).
-// Per tile the 8 warp partials are summed in a fixed order (deterministic, the same
-// for every M), scaled, masked and folded into a running (max, lowest index) per
-// input row. Each CTA writes its partial; the last CTA to finish (an atomic ticket,
-// no waiting) reduces them in CTA order and resets the ticket to zero.
+// Design (B200, HBM-bound): one persistent CTA per SM owns a contiguous range of
+// 16-row tiles. A producer warp streams the table through a shared-memory ring with
+// one TMA tensor copy per stage -- 16 rows x 1 KB of codes, written with the 128-byte
+// swizzle (plus a 16 x 128-byte copy of the NVFP4 block scales) -- completing on an
+// mbarrier. Large single copies matter: the TMA unit's per-copy cost caps a ring fed
+// by 1 KB row copies at about half of HBM bandwidth, while 16 KB tensor boxes stream
+// at the copy peak. Out-of-range rows and K tails arrive as zeros (tensor-map bounds).
+// Eight consumer warps split each stage's K range (16 slabs of 4 lanes x 16 B; warp w
+// takes slabs w and w+8), decode the codes exactly into f16/bf16 fragments and run
+// tensor-core MMAs with 16 table rows as the A operand and up to 16 inputs as the B
+// operand (swap-AB). MMA row g reads table row s(g) of the tile, a fixed permutation
+// that, with the swizzle, makes every shared-memory read conflict-free. E4M3 codes and
+// E2M1 codes times their E4M3 block scale are exact in f16; x is staged once per CTA
+// (bf16 for BF16 tables; f16 scaled by a per-row power of two for quantized tables,
+// undone in fp32), so the only roundings are the fp32 accumulation. Per tile the eight
+// warp partials are summed in a fixed order (deterministic and independent of M),
+// scaled, masked and folded into a running (max, lowest index) per input row. Tiles
+// whose 16 rows are all masked out for every input are neither loaded nor computed.
+// Each CTA writes its partial; the last CTA to finish (atomic ticket, no waiting)
+// reduces them in CTA order and re-zeroes the ticket. Every mbarrier wait is bounded:
+// a wait that runs out sets an abort flag and MTP_DEVFLAG_TIMEOUT, and the kernel runs
+// to its end.
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 #include <climits>
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -32,20 +43,59 @@
 namespace mtp {
 namespace {
 
-constexpr int kWarps = 8;
-constexpr int kThreads = kWarps * 32;
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kThreads = kConsumers + 32;  // + one producer warp
 constexpr int kTileRows = 16;
 constexpr int kMaxGrid = 1024;
+constexpr int kMaxStages = 12;
+constexpr int kStageRowBytes = 1024;                  // code bytes of one row per stage
+constexpr int kCodeStageBytes = kTileRows * kStageRowBytes;
+constexpr int kScaleStageBytes = kTileRows * 128;     // NVFP4: 128 scale bytes per row
+constexpr int kSmemLimit = 227 * 1024;
 
 struct Partial {
     float v;
     int32_t i;
 };
 
-template <int FMT> struct FmtTraits;
-template <> struct FmtTraits<0> { static constexpr int V = 8;  static constexpr int D = 8; };
-template <> struct FmtTraits<1> { static constexpr int V = 16; static constexpr int D = 6; };
-template <> struct FmtTraits<2> { static constexpr int V = 32; static constexpr int D = 4; };
+// V: K elements per 16-byte piece; KC: K elements per stage (1 KB of codes per row)
+template <int FMT> struct Fmt;
+template <> struct Fmt<0> { static constexpr int V = 8;  static constexpr int KC = 512; };
+template <> struct Fmt<1> { static constexpr int V = 16; static constexpr int KC = 1024; };
+template <> struct Fmt<2> { static constexpr int V = 32; static constexpr int KC = 2048; };
+
+__host__ __device__ inline int stage_bytes_for(int fmt) {
+    return fmt == 2 ? kCodeStageBytes + kScaleStageBytes : kCodeStageBytes;  // multiples of 1 KB
+}
+
+// MMA row g of a tile reads table row s(g) (a bijection on 0..15 with s(g+8) = s(g)+8).
+__device__ __forceinline__ int tile_row(int g) { return (g & 8) | ((g & 1) << 2) | ((g >> 1) & 3); }
+
+// Byte offset of logical byte b of row r inside a stage written by a 128-byte-swizzled
+// box of 128-byte segments: 16-byte chunk bits [4:6] are XORed with bits [7:9].
+__device__ __forceinline__ uint32_t swz(uint32_t logical) {
+    return logical ^ (((logical >> 7) & 7u) << 4);
+}
+
+// 3-D / 2-D TMA tensor loads into this CTA's shared memory (no multicast).
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
 
 __device__ __forceinline__ bool mask_allows(const SweepParams& p, int m, int64_t row) {
     if (!p.mask) return true;
@@ -63,44 +113,43 @@ __device__ __forceinline__ bool row_needed(const SweepParams& p, int64_t row) {
     return false;
 }
 
-__device__ __forceinline__ float block_sum(float v, float* scratch) {
+// Reductions over the 256 consumer threads (named barrier 1).
+__device__ __forceinline__ float consumer_sum(float v, float* scratch) {
     for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    __syncthreads();
+    named_sync(1, kConsumers);
     if (lane == 0) scratch[warp] = v;
-    __syncthreads();
+    named_sync(1, kConsumers);
     float t = 0.f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) t += scratch[w];
+    for (int w = 0; w < kConsumerWarps; ++w) t += scratch[w];
     return t;
 }
 
-__device__ __forceinline__ float block_max(float v, float* scratch) {
+__device__ __forceinline__ float consumer_max(float v, float* scratch) {
     for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    __syncthreads();
+    named_sync(1, kConsumers);
     if (lane == 0) scratch[warp] = v;
-    __syncthreads();
+    named_sync(1, kConsumers);
     float t = 0.f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) t = fmaxf(t, scratch[w]);
+    for (int w = 0; w < kConsumerWarps; ++w) t = fmaxf(t, scratch[w]);
     return t;
 }
 
-// Stage x (bf16) into xs[m][0..Kp): a copy (mode 0) or the combiner's concat
-// [bf16(rms(e) w_e) || bf16(rms(hidden) w_h)] (mode 1). Columns K..Kp are zero.
+// Stage x (bf16) into xs[m][0..K): a copy (mode 0) or the combiner's concat
+// [bf16(rms(e) w_e) || bf16(rms(hidden) w_h)] (mode 1).
 template <int MODE>
-__device__ void stage_bf16(const SweepParams& p, uint16_t* xs, int Kp, float* scratch) {
+__device__ void stage_bf16(const SweepParams& p, uint16_t* xs, float* scratch) {
     const int tid = threadIdx.x;
     const int64_t K = p.k;
     if (MODE == 0) {
-        const int vecs = Kp / 8;
-        for (int i = tid; i < p.M * vecs; i += kThreads) {
+        const int vecs = (int)(K / 8);
+        for (int i = tid; i < p.M * vecs; i += kConsumers) {
             int m = i / vecs, v = i - m * vecs;
-            int64_t k0 = (int64_t)v * 8;
-            uint4 val = make_uint4(0, 0, 0, 0);
-            if (k0 < K) val = *reinterpret_cast<const uint4*>(p.x + (int64_t)m * K + k0);
-            *reinterpret_cast<uint4*>(xs + (int64_t)m * p.kpad + k0) = val;
+            uint4 val = *reinterpret_cast<const uint4*>(p.x + (int64_t)m * K + (int64_t)v * 8);
+            *reinterpret_cast<uint4*>(xs + (int64_t)m * p.kpad + (int64_t)v * 8) = val;
         }
     } else {
         const int h = p.h;
@@ -111,144 +160,284 @@ __device__ void stage_bf16(const SweepParams& p, uint16_t* xs, int Kp, float* sc
             const uint16_t* e = bad ? nullptr : p.embed + tok * h;
             const uint16_t* hx = p.hidden + (int64_t)m * h;
             float se = 0.f, sx = 0.f;
-            for (int j = tid; j < h; j += kThreads) {
+            for (int j = tid; j < h; j += kConsumers) {
                 float ev = e ? bf16_to_f32(e[j]) : 0.f;
                 float xv = bf16_to_f32(hx[j]);
                 se += ev * ev;
                 sx += xv * xv;
             }
-            se = block_sum(se, scratch);
-            sx = block_sum(sx, scratch + kWarps);
+            se = consumer_sum(se, scratch);
+            sx = consumer_sum(sx, scratch + kConsumerWarps);
             float inv_e = 1.0f / sqrtf(se / (float)h + p.eps);
             float inv_x = 1.0f / sqrtf(sx / (float)h + p.eps);
             uint16_t* row = xs + (int64_t)m * p.kpad;
-            for (int j = tid; j < h; j += kThreads) {
+            for (int j = tid; j < h; j += kConsumers) {
                 float ev = e ? bf16_to_f32(e[j]) : 0.f;
                 row[j] = f32_to_bf16(ev * inv_e * bf16_to_f32(p.w_norm_embed[j]));
                 row[h + j] = f32_to_bf16(bf16_to_f32(hx[j]) * inv_x *
                                          bf16_to_f32(p.w_norm_hidden[j]));
             }
-            for (int j = (int)K + tid; j < Kp; j += kThreads) row[j] = 0;
         }
     }
-    __syncthreads();
+    named_sync(1, kConsumers);
 }
 
 // Quantized tables: rescale each staged row by 2^e_m (largest |x| lands in
 // [2^14, 2^15)) and convert it in place to f16. Exact for every element within
 // 2^29 of the row maximum; the power of two is undone on the fp32 logit.
-__device__ void stage_to_f16(const SweepParams& p, uint16_t* xs, int Kp, int* xexp,
-                             float* scratch) {
+__device__ void stage_to_f16(const SweepParams& p, uint16_t* xs, int* xexp, float* scratch) {
     const int tid = threadIdx.x;
+    const int K = (int)p.k;
     for (int m = 0; m < p.M; ++m) {
         uint16_t* row = xs + (int64_t)m * p.kpad;
         float a = 0.f;
-        for (int j = tid; j < Kp; j += kThreads) a = fmaxf(a, fabsf(bf16_to_f32(row[j])));
-        a = block_max(a, scratch);
+        for (int j = tid; j < K; j += kConsumers) a = fmaxf(a, fabsf(bf16_to_f32(row[j])));
+        a = consumer_max(a, scratch);
         int ex = 0;
         if (a > 0.f) frexpf(a, &ex);
         int e = (a > 0.f) ? 15 - ex : 0;
         if (tid == 0) xexp[m] = e;
-        for (int j = tid; j < Kp; j += kThreads)
+        for (int j = tid; j < K; j += kConsumers)
             row[j] = f32_to_f16(ldexpf(bf16_to_f32(row[j]), e));
-        __syncthreads();
+        named_sync(1, kConsumers);
     }
 }
 
+__device__ __forceinline__ bool tile_needed(const SweepParams& p, int64_t tile, int lane) {
+    const bool need = lane < kTileRows && row_needed(p, tile * kTileRows + lane);
+    return __ballot_sync(0xffffffffu, need) != 0u;
+}
+
 template <int FMT, int NT, int MODE>
-__global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) sweep_kernel(const SweepParams p) {
-    constexpr int V = FmtTraits<FMT>::V;
-    constexpr int D = FmtTraits<FMT>::D;
-    constexpr int SLAB = 4 * V;           // elements of one row covered by one slab
+__global__ void __launch_bounds__(kThreads, 1)
+    sweep_kernel(const __grid_constant__ SweepParams p, const __grid_constant__ CUtensorMap map_codes,
+                 const __grid_constant__ CUtensorMap map_scales) {
+    constexpr int V = Fmt<FMT>::V;
+    constexpr int KC = Fmt<FMT>::KC;
+    constexpr int SLAB = 4 * V;  // K elements of one slab (4 lanes x 16 bytes)
     constexpr int RED_COLS = 8 * NT;
 
-    extern __shared__ __align__(16) uint8_t smem[];
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g = lane >> 2, c = lane & 3;
-    const int64_t K = p.k;
-    const int S = (int)((K + SLAB - 1) / SLAB);
-    const int Kp = S * SLAB;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + kMaxStages;
+    int* misc = reinterpret_cast<int*>(empty + kMaxStages);  // [0] abort [1] last [2..17] xexp
+    volatile int* abort_flag = misc;
+    int* xexp = misc + 2;
+    float* red = reinterpret_cast<float*>(misc + 32);  // [2][8][16][RED_COLS]
+    float* scratch = red + 2 * kConsumerWarps * kTileRows * RED_COLS;  // [32]
+    uint16_t* xs = reinterpret_cast<uint16_t*>(scratch + 32);
+    // the ring starts on a 1 KB boundary of the shared window (the 128-byte swizzle atom)
+    const uint32_t head_end = smem_u32(xs) + (uint32_t)p.M * (uint32_t)p.kpad * 2u;
+    uint8_t* ring = smem + (((head_end + 1023u) & ~1023u) - smem_u32(smem));
 
-    uint16_t* xs = reinterpret_cast<uint16_t*>(smem);
-    size_t xs_bytes = ((size_t)p.M * p.kpad * 2 + 15) & ~(size_t)15;
-    float* red = reinterpret_cast<float*>(smem + xs_bytes);          // [2][8][16][RED_COLS]
-    float* scratch = red + 2 * kWarps * kTileRows * RED_COLS;        // [2*8]
-    int* xexp = reinterpret_cast<int*>(scratch + 2 * kWarps);        // [16]
-    int* last_flag = xexp + 16;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t K = p.k;
+    const int S = p.stages;
+    const int stage_bytes = p.stage_bytes;
+    const int NC = (int)((K + KC - 1) / KC);  // stages per tile
 
     const int64_t T = p.num_tiles;
     const int64_t t_begin = (T * blockIdx.x) / gridDim.x;
     const int64_t t_end = (T * (blockIdx.x + 1)) / gridDim.x;
 
-    stage_bf16<MODE>(p, xs, Kp, scratch);
-    if (FMT != 0) stage_to_f16(p, xs, Kp, xexp, scratch);
-
-    const int Sw = (S > warp) ? (S - warp + kWarps - 1) / kWarps : 0;
-    const int64_t total = (t_end - t_begin) * (int64_t)Sw;
-
-    // rows of this lane inside a tile
-    const int M = p.M;
-    const bool xg0 = g < M;                 // B column g of n-tile 0 is a real input row
-    const bool xg1 = NT > 1 && (8 + g) < M; // ... of n-tile 1
-
-    // load stream
-    int64_t lt = t_begin;
-    int ls = warp;
-    bool need0 = false, need1 = false;
-    if (total > 0) {
-        need0 = row_needed(p, lt * kTileRows + g);
-        need1 = row_needed(p, lt * kTileRows + g + 8);
-    }
-    uint4 ra[D], rb[D];
-    uint32_t rsc[D];
-
-    auto issue = [&](int d) {
-        const int64_t r0 = lt * kTileRows + g;
-        const int64_t e0 = (int64_t)ls * SLAB + c * V;
-        const bool kin = e0 < K;
-        const uint8_t* base = p.w + (int64_t)ls * 64 + c * 16;
-        ra[d] = (need0 && kin) ? ldg_stream(base + r0 * p.row_bytes) : make_uint4(0, 0, 0, 0);
-        rb[d] = (need1 && kin) ? ldg_stream(base + (r0 + 8) * p.row_bytes) : make_uint4(0, 0, 0, 0);
-        if (FMT == 2) {
-            const int64_t kb = K >> 4;
-            const uint8_t* sb = p.block_scale + (int64_t)ls * 8 + 2 * c;
-            uint32_t s0 = (need0 && kin) ? ldg_u16(sb + r0 * kb) : 0u;
-            uint32_t s1 = (need1 && kin) ? ldg_u16(sb + (r0 + 8) * kb) : 0u;
-            rsc[d] = s0 | (s1 << 16);
+    if (tid == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
         }
-        ls += kWarps;
-        if (ls >= S) {
-            ls = warp;
-            ++lt;
-            if (lt < t_end) {
-                need0 = row_needed(p, lt * kTileRows + g);
-                need1 = row_needed(p, lt * kTileRows + g + 8);
+        misc[0] = 0;
+        mbar_fence_init();
+    }
+    __syncthreads();
+
+    // ------------------------------------------------------------ producer warp
+    if (warp == kConsumerWarps) {
+        int slot = 0;
+        uint32_t phase = 0;
+        int64_t issued = 0;
+        const uint32_t tx = kCodeStageBytes + (FMT == 2 ? kScaleStageBytes : 0);
+        bool stop = false;
+        for (int64_t tile = t_begin; tile < t_end && !stop; ++tile) {
+            if (!tile_needed(p, tile, lane)) continue;
+            for (int ch = 0; ch < NC; ++ch) {
+                if (!mbar_wait_bounded(&empty[slot], phase ^ 1u, abort_flag)) {
+                    stop = true;
+                    break;
+                }
+                if (lane == 0) {
+                    uint8_t* dst = ring + (size_t)slot * stage_bytes;
+                    mbar_arrive_expect_tx(&full[slot], tx);
+                    tma_load_3d(dst, &map_codes, 0, (int)(tile * kTileRows), ch * (kStageRowBytes / 128),
+                                &full[slot]);
+                    if (FMT == 2)
+                        tma_load_2d(dst + kCodeStageBytes, &map_scales, ch * 128, (int)(tile * kTileRows),
+                                    &full[slot]);
+                }
+                __syncwarp();
+                ++issued;
+                if (++slot == S) {
+                    slot = 0;
+                    phase ^= 1u;
+                }
             }
         }
-    };
+        // leave no copy in flight: wait for the last stages issued (bounded)
+        for (int64_t j = issued > S ? issued - S : 0; j < issued; ++j)
+            if (!mbar_wait_bounded(&full[j % S], (uint32_t)((j / S) & 1), nullptr)) break;
+        return;
+    }
 
-    float acc[NT][4];
-#pragma unroll
-    for (int t = 0; t < NT; ++t)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[t][i] = 0.f;
+    // ------------------------------------------------------------ consumer warps
+    const int g = lane >> 2, c = lane & 3;
+    const int M = p.M;
+    stage_bf16<MODE>(p, xs, scratch);
+    if (FMT != 0) stage_to_f16(p, xs, xexp, scratch);
 
-    // running best (reducer threads with row 0)
+    const bool xg0 = g < M;
+    const bool xg1 = NT > 1 && (8 + g) < M;
+    const int r0 = tile_row(g);  // table rows r0 and r0 + 8 of the tile feed MMA rows g, g+8
+
+    // one accumulator set per slab of a stage: two independent MMA chains per warp
+    float accs[2][NT][4];
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int t = 0; t < NT; ++t)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) accs[j][t][i] = 0.f;
+
     float best_v = -INFINITY;
     int32_t best_i = INT_MAX;
     const int red_threads = kTileRows * RED_COLS;
     const int rrow = tid & 15, rcol = tid >> 4;
-
     int buf = 0;
-    int64_t ct = t_begin;
-    int cs = warp;
+    int slot = 0;
+    uint32_t phase = 0;
 
-    auto reduce_tile = [&](int64_t tile, int b) {
+    for (int64_t tile = t_begin; tile < t_end; ++tile) {
+        if (!tile_needed(p, tile, lane)) {  // warp-uniform, same rule as the producer
+            // every row of the tile is masked out for every input: logits are -inf
+            if (MODE == 0 && p.out_logits && tid < red_threads) {
+                const int64_t row = tile * kTileRows + rrow;
+                if (row < p.n && rcol < M) p.out_logits[(int64_t)rcol * p.n + row] = 0xFF80u;
+            }
+            continue;
+        }
+        for (int ch = 0; ch < NC; ++ch) {
+            mbar_wait_bounded(&full[slot], phase, abort_flag);
+            const uint8_t* st = ring + (size_t)slot * stage_bytes;
+            const int64_t kc0 = (int64_t)ch * KC;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                float(&acc)[NT][4] = accs[j];
+                const int sl = warp + kConsumerWarps * j;
+                const int64_t s0 = kc0 + (int64_t)sl * SLAB;
+                if (s0 >= K) continue;  // warp-uniform: slab past the end of K
+                const int64_t e0 = s0 + c * V;
+                const bool kin = e0 < K;  // beyond K the stage holds zeros
+                const uint32_t b = (uint32_t)(sl * 64 + c * 16);  // logical byte in the row chunk
+                const uint32_t la = (b >> 7) * 2048u + (uint32_t)r0 * 128u + (b & 127u);
+                const uint4 ra = lds128(st + swz(la));
+                const uint4 rb = lds128(st + swz(la + 8u * 128u));
+                const uint16_t* x0 = xs + (int64_t)g * p.kpad + e0;
+                const uint16_t* x1 = xs + (int64_t)(8 + g) * p.kpad + e0;
+                const bool l0 = xg0 && kin, l1 = xg1 && kin;
+                if (FMT == 0) {
+                    uint4 xa = l0 ? lds128(x0) : make_uint4(0, 0, 0, 0);
+                    mma_bf16_16816(acc[0], ra.x, rb.x, ra.y, rb.y, xa.x, xa.y);
+                    mma_bf16_16816(acc[0], ra.z, rb.z, ra.w, rb.w, xa.z, xa.w);
+                    if (NT > 1) {
+                        uint4 xb = l1 ? lds128(x1) : make_uint4(0, 0, 0, 0);
+                        mma_bf16_16816(acc[NT - 1], ra.x, rb.x, ra.y, rb.y, xb.x, xb.y);
+                        mma_bf16_16816(acc[NT - 1], ra.z, rb.z, ra.w, rb.w, xb.z, xb.w);
+                    }
+                } else if (FMT == 1) {
+                    const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w};
+                    const uint32_t wb[4] = {rb.x, rb.y, rb.z, rb.w};
+                    const uint4 xa0 = l0 ? lds128(x0) : make_uint4(0, 0, 0, 0);
+                    const uint4 xa1 = l0 ? lds128(x0 + 8) : make_uint4(0, 0, 0, 0);
+                    const uint32_t xa[8] = {xa0.x, xa0.y, xa0.z, xa0.w, xa1.x, xa1.y, xa1.z, xa1.w};
+                    uint32_t xb[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+                    if (NT > 1) {
+                        const uint4 xb0 = l1 ? lds128(x1) : make_uint4(0, 0, 0, 0);
+                        const uint4 xb1 = l1 ? lds128(x1 + 8) : make_uint4(0, 0, 0, 0);
+                        xb[0] = xb0.x; xb[1] = xb0.y; xb[2] = xb0.z; xb[3] = xb0.w;
+                        xb[4] = xb1.x; xb[5] = xb1.y; xb[6] = xb1.z; xb[7] = xb1.w;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t a0 = e4m3x2_to_f16x2((uint16_t)(wa[i] & 0xFFFFu));
+                        const uint32_t a2 = e4m3x2_to_f16x2((uint16_t)(wa[i] >> 16));
+                        const uint32_t a1 = e4m3x2_to_f16x2((uint16_t)(wb[i] & 0xFFFFu));
+                        const uint32_t a3 = e4m3x2_to_f16x2((uint16_t)(wb[i] >> 16));
+                        mma_f16_16816(acc[0], a0, a1, a2, a3, xa[2 * i], xa[2 * i + 1]);
+                        if (NT > 1)
+                            mma_f16_16816(acc[NT - 1], a0, a1, a2, a3, xb[2 * i], xb[2 * i + 1]);
+                    }
+                } else {
+                    const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w};
+                    const uint32_t wb[4] = {rb.x, rb.y, rb.z, rb.w};
+                    // block scales of rows r0 / r0+8: blocks 2c (words 0,1) and 2c+1 (words 2,3)
+                    const uint8_t* sp = st + kCodeStageBytes;
+                    const uint32_t sbyte = (uint32_t)(sl * 8 + 2 * c);
+                    const uint16_t s0v = *reinterpret_cast<const uint16_t*>(sp + swz((uint32_t)r0 * 128u + sbyte));
+                    const uint16_t s1v =
+                        *reinterpret_cast<const uint16_t*>(sp + swz((uint32_t)(r0 + 8) * 128u + sbyte));
+                    const uint32_t sa = e4m3x2_to_f16x2(s0v);
+                    const uint32_t sb = e4m3x2_to_f16x2(s1v);
+                    const uint32_t sa_lo = __byte_perm(sa, 0, 0x1010), sa_hi = __byte_perm(sa, 0, 0x3232);
+                    const uint32_t sb_lo = __byte_perm(sb, 0, 0x1010), sb_hi = __byte_perm(sb, 0, 0x3232);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        uint32_t qa[4], qb[4];
+                        e2m1x8_to_f16x2x4(wa[i], qa);
+                        e2m1x8_to_f16x2x4(wb[i], qb);
+                        const uint32_t s_a = i < 2 ? sa_lo : sa_hi;
+                        const uint32_t s_b = i < 2 ? sb_lo : sb_hi;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            qa[q] = hmul2(qa[q], s_a);
+                            qb[q] = hmul2(qb[q], s_b);
+                        }
+                        const uint4 xv = l0 ? lds128(x0 + 8 * i) : make_uint4(0, 0, 0, 0);
+                        mma_f16_16816(acc[0], qa[0], qb[0], qa[1], qb[1], xv.x, xv.y);
+                        mma_f16_16816(acc[0], qa[2], qb[2], qa[3], qb[3], xv.z, xv.w);
+                        if (NT > 1) {
+                            const uint4 xw = l1 ? lds128(x1 + 8 * i) : make_uint4(0, 0, 0, 0);
+                            mma_f16_16816(acc[NT - 1], qa[0], qb[0], qa[1], qb[1], xw.x, xw.y);
+                            mma_f16_16816(acc[NT - 1], qa[2], qb[2], qa[3], qb[3], xw.z, xw.w);
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[slot]);
+            if (++slot == S) {
+                slot = 0;
+                phase ^= 1u;
+            }
+        }
+
+        // ---- tile done: cross-warp sum (fixed order), scale, mask, running argmax
+        {
+            float* rp = red + (size_t)buf * kConsumerWarps * kTileRows * RED_COLS +
+                        warp * kTileRows * RED_COLS;
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                rp[r0 * RED_COLS + t * 8 + 2 * c] = accs[0][t][0] + accs[1][t][0];
+                rp[r0 * RED_COLS + t * 8 + 2 * c + 1] = accs[0][t][1] + accs[1][t][1];
+                rp[(r0 + 8) * RED_COLS + t * 8 + 2 * c] = accs[0][t][2] + accs[1][t][2];
+                rp[(r0 + 8) * RED_COLS + t * 8 + 2 * c + 1] = accs[0][t][3] + accs[1][t][3];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) accs[0][t][i] = accs[1][t][i] = 0.f;
+            }
+        }
+        named_sync(1, kConsumers);
         if (tid < red_threads) {
-            const float* rp = red + (size_t)b * kWarps * kTileRows * RED_COLS;
+            const float* rb = red + (size_t)buf * kConsumerWarps * kTileRows * RED_COLS;
             float a = 0.f;
 #pragma unroll
-            for (int w = 0; w < kWarps; ++w) a += rp[(w * kTileRows + rrow) * RED_COLS + rcol];
+            for (int w = 0; w < kConsumerWarps; ++w) a += rb[(w * kTileRows + rrow) * RED_COLS + rcol];
             const int64_t row = tile * kTileRows + rrow;
             const bool valid = row < p.n && rcol < M;
             float l = a;
@@ -265,9 +454,12 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) sweep_kernel(const 
                 int32_t i = ok ? (int32_t)row : INT_MAX;
 #pragma unroll
                 for (int o = 8; o; o >>= 1) {
-                    float ov = __shfl_xor_sync(0xffffffffu, v, o);
-                    int32_t oi = __shfl_xor_sync(0xffffffffu, i, o);
-                    if (ov > v || (ov == v && oi < i)) { v = ov; i = oi; }
+                    const float ov = __shfl_xor_sync(0xffffffffu, v, o);
+                    const int32_t oi = __shfl_xor_sync(0xffffffffu, i, o);
+                    if (ov > v || (ov == v && oi < i)) {
+                        v = ov;
+                        i = oi;
+                    }
                 }
                 if (rrow == 0 && (v > best_v || (v == best_v && i < best_i))) {
                     best_v = v;
@@ -275,139 +467,35 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) sweep_kernel(const 
                 }
             }
         }
-    };
-
-    auto flush_tile = [&]() {
-        float* rp = red + (size_t)buf * kWarps * kTileRows * RED_COLS + warp * kTileRows * RED_COLS;
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-            rp[g * RED_COLS + t * 8 + 2 * c] = acc[t][0];
-            rp[g * RED_COLS + t * 8 + 2 * c + 1] = acc[t][1];
-            rp[(g + 8) * RED_COLS + t * 8 + 2 * c] = acc[t][2];
-            rp[(g + 8) * RED_COLS + t * 8 + 2 * c + 1] = acc[t][3];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[t][i] = 0.f;
-        }
-        __syncthreads();
-        reduce_tile(ct, buf);
         buf ^= 1;
-    };
-
-    auto consume = [&](int d) {
-        const uint16_t* x0 = xs + (int64_t)g * p.kpad + cs * SLAB + c * V;
-        const uint16_t* x1 = xs + (int64_t)(8 + g) * p.kpad + cs * SLAB + c * V;
-        if (FMT == 0) {
-            uint4 xa = xg0 ? lds128(x0) : make_uint4(0, 0, 0, 0);
-            mma_bf16_16816(acc[0], ra[d].x, rb[d].x, ra[d].y, rb[d].y, xa.x, xa.y);
-            mma_bf16_16816(acc[0], ra[d].z, rb[d].z, ra[d].w, rb[d].w, xa.z, xa.w);
-            if (NT > 1) {
-                uint4 xb = xg1 ? lds128(x1) : make_uint4(0, 0, 0, 0);
-                mma_bf16_16816(acc[NT - 1], ra[d].x, rb[d].x, ra[d].y, rb[d].y, xb.x, xb.y);
-                mma_bf16_16816(acc[NT - 1], ra[d].z, rb[d].z, ra[d].w, rb[d].w, xb.z, xb.w);
-            }
-        } else if (FMT == 1) {
-            uint32_t wa[4] = {ra[d].x, ra[d].y, ra[d].z, ra[d].w};
-            uint32_t wb[4] = {rb[d].x, rb[d].y, rb[d].z, rb[d].w};
-            uint4 xa0 = xg0 ? lds128(x0) : make_uint4(0, 0, 0, 0);
-            uint4 xa1 = xg0 ? lds128(x0 + 8) : make_uint4(0, 0, 0, 0);
-            uint32_t xa[8] = {xa0.x, xa0.y, xa0.z, xa0.w, xa1.x, xa1.y, xa1.z, xa1.w};
-            uint32_t xb[8];
-            if (NT > 1) {
-                uint4 xb0 = xg1 ? lds128(x1) : make_uint4(0, 0, 0, 0);
-                uint4 xb1 = xg1 ? lds128(x1 + 8) : make_uint4(0, 0, 0, 0);
-                xb[0] = xb0.x; xb[1] = xb0.y; xb[2] = xb0.z; xb[3] = xb0.w;
-                xb[4] = xb1.x; xb[5] = xb1.y; xb[6] = xb1.z; xb[7] = xb1.w;
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                uint32_t a0 = e4m3x2_to_f16x2((uint16_t)(wa[i] & 0xFFFFu));
-                uint32_t a2 = e4m3x2_to_f16x2((uint16_t)(wa[i] >> 16));
-                uint32_t a1 = e4m3x2_to_f16x2((uint16_t)(wb[i] & 0xFFFFu));
-                uint32_t a3 = e4m3x2_to_f16x2((uint16_t)(wb[i] >> 16));
-                mma_f16_16816(acc[0], a0, a1, a2, a3, xa[2 * i], xa[2 * i + 1]);
-                if (NT > 1) mma_f16_16816(acc[NT - 1], a0, a1, a2, a3, xb[2 * i], xb[2 * i + 1]);
-            }
-        } else {
-            uint32_t wa[4] = {ra[d].x, ra[d].y, ra[d].z, ra[d].w};
-            uint32_t wb[4] = {rb[d].x, rb[d].y, rb[d].z, rb[d].w};
-            // block scales: rows g / g+8, blocks 2c (words 0,1) and 2c+1 (words 2,3)
-            uint32_t sa = e4m3x2_to_f16x2((uint16_t)(rsc[d] & 0xFFFFu));
-            uint32_t sb = e4m3x2_to_f16x2((uint16_t)(rsc[d] >> 16));
-            const uint32_t sa_lo = __byte_perm(sa, 0, 0x1010), sa_hi = __byte_perm(sa, 0, 0x3232);
-            const uint32_t sb_lo = __byte_perm(sb, 0, 0x1010), sb_hi = __byte_perm(sb, 0, 0x3232);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                uint32_t qa[4], qb[4];
-                e2m1x8_to_f16x2x4(wa[i], qa);
-                e2m1x8_to_f16x2x4(wb[i], qb);
-                const uint32_t s_a = i < 2 ? sa_lo : sa_hi;
-                const uint32_t s_b = i < 2 ? sb_lo : sb_hi;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    qa[j] = hmul2(qa[j], s_a);
-                    qb[j] = hmul2(qb[j], s_b);
-                }
-                // x words for elements 8i .. 8i+7 of this lane's 32
-                uint4 xv = xg0 ? lds128(x0 + 8 * i) : make_uint4(0, 0, 0, 0);
-                mma_f16_16816(acc[0], qa[0], qb[0], qa[1], qb[1], xv.x, xv.y);
-                mma_f16_16816(acc[0], qa[2], qb[2], qa[3], qb[3], xv.z, xv.w);
-                if (NT > 1) {
-                    uint4 xw = xg1 ? lds128(x1 + 8 * i) : make_uint4(0, 0, 0, 0);
-                    mma_f16_16816(acc[NT - 1], qa[0], qb[0], qa[1], qb[1], xw.x, xw.y);
-                    mma_f16_16816(acc[NT - 1], qa[2], qb[2], qa[3], qb[3], xw.z, xw.w);
-                }
-            }
-        }
-    };
-
-    if (Sw > 0) {
-#pragma unroll
-        for (int d = 0; d < D; ++d)
-            if (d < total) issue(d);
-        for (int64_t j0 = 0; j0 < total; j0 += D) {
-#pragma unroll
-            for (int d = 0; d < D; ++d) {
-                if (j0 + d < total) {
-                    consume(d);
-                    if (j0 + d + D < total) issue(d);
-                    cs += kWarps;
-                    if (cs >= S) {
-                        flush_tile();
-                        cs = warp;
-                        ++ct;
-                    }
-                }
-            }
-        }
-    } else {
-        // this warp owns no slab of K: it still takes part in every tile's barrier
-        for (; ct < t_end; ++ct) flush_tile();
     }
 
+    if (*abort_flag) raise_flag(p.dev_err, DEVFLAG_TIMEOUT);
     if (MODE == 1) return;
 
     Partial* parts = reinterpret_cast<Partial*>(p.partials);
-    if (tid < red_threads && rrow == 0 && rcol < M) {
+    if (tid < red_threads && rrow == 0 && rcol < M)
         parts[(int64_t)blockIdx.x * 16 + rcol] = Partial{best_v, best_i};
-    }
-    __syncthreads();
+    named_sync(1, kConsumers);
     if (tid == 0) {
         __threadfence();
-        unsigned int ticket = atomicAdd(p.ticket, 1u);
-        *last_flag = (ticket == gridDim.x - 1) ? 1 : 0;
+        const unsigned int ticket = atomicAdd(p.ticket, 1u);
+        misc[1] = (ticket == gridDim.x - 1) ? 1 : 0;
     }
-    __syncthreads();
-    if (*last_flag == 0) return;
+    named_sync(1, kConsumers);
+    if (misc[1] == 0) return;
     __threadfence();
     if (tid < M) {
         float bv = -INFINITY;
         int32_t bi = INT_MAX;
         for (int b = 0; b < (int)gridDim.x; ++b) {
-            Partial q;
             const Partial* src = parts + (int64_t)b * 16 + tid;
-            q.v = __ldcg(&src->v);
-            q.i = __ldcg(&src->i);
-            if (q.v > bv || (q.v == bv && q.i < bi)) { bv = q.v; bi = q.i; }
+            const float qv = __ldcg(&src->v);
+            const int32_t qi = __ldcg(&src->i);
+            if (qv > bv || (qv == bv && qi < bi)) {
+                bv = qv;
+                bi = qi;
+            }
         }
         if (bi == INT_MAX) {
             bi = 0;
@@ -420,33 +508,112 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) sweep_kernel(const 
     if (tid == 0) *p.ticket = 0u;  // leave the workspace ready for the next call
 }
 
+struct Geometry {
+    int kpad;
+    int stage_bytes;
+    int stages;
+    size_t smem;
+};
+
+Geometry geometry(int M, int64_t k, int fmt) {
+    Geometry g{};
+    g.kpad = (int)(k + 8);  // 16-byte skew between staged rows
+    const int NT = M > 8 ? 2 : 1;
+    size_t head = (size_t)2 * kMaxStages * 8 + 32 * sizeof(int) +
+                  (size_t)2 * kConsumerWarps * kTileRows * 8 * NT * sizeof(float) +
+                  32 * sizeof(float) + (size_t)M * g.kpad * 2;
+    head = ((head + 1023) & ~(size_t)1023) + 1024;  // 1 KB-aligned ring, plus slack
+    g.stage_bytes = stage_bytes_for(fmt);
+    long avail = (long)kSmemLimit - (long)head;
+    int stages = avail > 0 ? (int)(avail / g.stage_bytes) : 0;
+    if (stages > kMaxStages) stages = kMaxStages;
+    g.stages = stages;
+    g.smem = head + (size_t)stages * g.stage_bytes;
+    return g;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+// Codes: a 3-D view (byte within a 128-byte segment, row, segment) so that one box of
+// 128 B x 16 rows x 8 segments is a stage, with rows inside the 128-byte swizzle atom.
+// Rows >= rows and segments past the row read as zeros.
+cudaError_t make_code_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return cudaErrorNotSupported;
+    cuuint64_t dims[3] = {128, (cuuint64_t)rows, (cuuint64_t)(row_bytes / 128)};
+    cuuint64_t strides[2] = {(cuuint64_t)row_bytes, 128};
+    cuuint32_t box[3] = {128, kTileRows, kStageRowBytes / 128};
+    cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
+                    box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// NVFP4 block scales: [rows, pitch] bytes, boxes of 128 B x 16 rows, 128-byte swizzle.
+cudaError_t make_scale_map(CUtensorMap* m, const void* base, int64_t rows, int64_t pitch) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return cudaErrorNotSupported;
+    cuuint64_t dims[2] = {(cuuint64_t)pitch, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)pitch};
+    cuuint32_t box[2] = {128, kTileRows};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                    box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 template <int FMT, int NT, int MODE>
 cudaError_t launch_one(const SweepParams& p, cudaStream_t s, SweepLaunch* info) {
     auto kern = sweep_kernel<FMT, NT, MODE>;
-    int kpad = 0;
-    size_t smem = sweep_smem_bytes(p.M, p.k, FMT, &kpad);
-    if (smem > 227 * 1024) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    const Geometry geo = geometry(p.M, p.k, FMT);
+    if (geo.stages < 2) return cudaErrorInvalidValue;
+    CUtensorMap map_codes, map_scales;
+    cudaError_t e = make_code_map(&map_codes, p.w, p.n, p.row_bytes);
     if (e != cudaSuccess) return e;
-    int dev = 0, sms = 0, per_sm = 0;
+    if (FMT == 2) {
+        if ((e = make_scale_map(&map_scales, p.block_scale, p.n, p.scale_pitch)) != cudaSuccess)
+            return e;
+    } else {
+        map_scales = map_codes;  // unused
+    }
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)geo.smem)) != cudaSuccess)
+        return e;
+    int dev = 0, sms = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
         return e;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem)) !=
-        cudaSuccess)
-        return e;
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    int64_t grid = (int64_t)sms * per_sm;
+    int64_t grid = sms;
     if (grid > p.num_tiles) grid = p.num_tiles;
     if (grid > kMaxGrid) grid = kMaxGrid;
     if (grid < 1) grid = 1;
     SweepParams q = p;
-    q.kpad = kpad;
-    kern<<<(int)grid, kThreads, smem, s>>>(q);
+    q.kpad = geo.kpad;
+    q.stages = geo.stages;
+    q.stage_bytes = geo.stage_bytes;
+    kern<<<(int)grid, kThreads, geo.smem, s>>>(q, map_codes, map_scales);
     if (info) {
         info->grid = (int)grid;
-        info->smem_bytes = (int)smem;
+        info->smem_bytes = (int)geo.smem;
     }
     return cudaGetLastError();
 }
@@ -454,15 +621,9 @@ cudaError_t launch_one(const SweepParams& p, cudaStream_t s, SweepLaunch* info) 
 }  // namespace
 
 size_t sweep_smem_bytes(int M, int64_t k, int fmt, int* kpad_out) {
-    const int V = fmt == 0 ? 8 : fmt == 1 ? 16 : 32;
-    const int64_t slab = 4 * V;
-    const int64_t Kp = ((k + slab - 1) / slab) * slab;
-    const int64_t kpad = Kp + 8;  // 16-byte skew between staged rows
-    if (kpad_out) *kpad_out = (int)kpad;
-    const int NT = M > 8 ? 2 : 1;
-    size_t xs = ((size_t)M * kpad * 2 + 15) & ~(size_t)15;
-    size_t red = (size_t)2 * kWarps * kTileRows * 8 * NT * sizeof(float);
-    return xs + red + 2 * kWarps * sizeof(float) + 17 * sizeof(int) + 16;
+    const Geometry g = geometry(M, k, fmt);
+    if (kpad_out) *kpad_out = g.kpad;
+    return g.stages >= 2 ? g.smem : (size_t)kSmemLimit + 1;
 }
 
 int sweep_max_grid() { return kMaxGrid; }

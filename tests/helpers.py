@@ -64,3 +64,13 @@ def allowed_from_mask(mask_row: np.ndarray, n: int, mask_words: int) -> np.ndarr
     m = min(n, bits.size)
     out[:m] = bits[:m]
     return out
+
+
+def pad_scales(bscale: np.ndarray, k: int) -> np.ndarray:
+    """[n, k/16] NVFP4 block scales -> the library's [n, pitch] layout (rows padded
+    with zeros to a multiple of 16 bytes)."""
+    n = bscale.shape[0]
+    pitch = ((k // 16 + 15) // 16) * 16
+    out = np.zeros((n, pitch), dtype=np.uint8)
+    out[:, : k // 16] = bscale
+    return out

@@ -104,6 +104,10 @@ def test_lm_head_rejects(lib):
     assert lm(weight(), mask=OUT, mw=0) == L.MTP_ERR_INVALID_ARG
     assert lm(weight(), ws=None) == L.MTP_ERR_WORKSPACE
     assert lm(weight(), wsb=16) == L.MTP_ERR_WORKSPACE
+    # table rows must be a multiple of 128 bytes (the sweep streams 128-byte segments)
+    assert lm(weight(k=40)) == L.MTP_ERR_UNSUPPORTED
+    assert lm(weight(fmt=1, k=80, rs=OUT)) == L.MTP_ERR_UNSUPPORTED
+    assert lm(weight(fmt=2, k=224, bs=OUT, gs=OUT)) == L.MTP_ERR_UNSUPPORTED
     # staged inputs larger than shared memory
     assert lm(weight(n=100, k=16384), M=16) == L.MTP_ERR_UNSUPPORTED
     w = weight()
@@ -119,6 +123,11 @@ def test_combine_rejects(lib):
     assert st("mtp_combine", *bad) == L.MTP_ERR_INVALID_ARG
     bad = list(args)
     bad[4] = 17
+    assert st("mtp_combine", *bad) == L.MTP_ERR_UNSUPPORTED
+    bad = list(args)
+    bad[5] = 48
+    fc48 = weight(n=48, k=96)  # 192-byte fc rows: not a multiple of 128
+    bad[9] = C.byref(fc48)
     assert st("mtp_combine", *bad) == L.MTP_ERR_UNSUPPORTED
     bad = list(args)
     bad[5] = 24  # h % 16

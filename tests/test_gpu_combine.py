@@ -4,7 +4,8 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import assert_argmax, assert_close, bf16_bits_to_f64, to_dev, to_dev_u16, u16_of
+from helpers import (assert_argmax, assert_close, bf16_bits_to_f64, pad_scales, to_dev,
+                     to_dev_u16, u16_of)
 from mtp_speculative_draft_lm_b200 import _lib as L
 from mtp_speculative_draft_lm_b200 import api, synth
 
@@ -41,7 +42,7 @@ def test_combine_matches_oracle(orc, M):
     assert diff.max() <= 1 and (diff > 0).mean() < 0.02
 
 
-@pytest.mark.parametrize("h", [16, 512, 1024])
+@pytest.mark.parametrize("h", [32, 512, 1024])
 def test_combine_other_widths(orc, h):
     d = draft(3, seed=5, h=h, vocab=300)
     y, _ = gpu_combine(d)
@@ -71,7 +72,7 @@ def test_combine_quantized_fc(orc, fmt):
         deq = orc.dequant(1, c, 2 * h, row_scale=s)
     else:
         c, b, g = orc.quantize_nvfp4(d["fc"])
-        fc = api.Table(2, h, 2 * h, to_dev(c), block_scale=to_dev(b),
+        fc = api.Table(2, h, 2 * h, to_dev(c), block_scale=to_dev(pad_scales(b, 2 * h)),
                        global_scale=torch.tensor([g], dtype=torch.float32, device="cuda"))
         deq = orc.dequant(2, c, 2 * h, block_scale=b, global_scale=g)
     y, _ = gpu_combine(d, fc_table=fc)

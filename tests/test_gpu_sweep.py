@@ -9,7 +9,7 @@ import pytest
 import torch
 
 from helpers import (allowed_from_mask, assert_argmax, assert_close, bf16_bits_to_f64,
-                     to_dev, to_dev_u16, u16_of)
+                     pad_scales, to_dev, to_dev_u16, u16_of)
 from mtp_speculative_draft_lm_b200 import _lib as L
 from mtp_speculative_draft_lm_b200 import api, synth
 
@@ -31,7 +31,7 @@ def device_table(q, fmt, n, k):
         return api.Table(0, n, k, to_dev_u16(q["data"]))
     if fmt == 1:
         return api.Table(1, n, k, to_dev(q["data"]), row_scale=to_dev(q["row_scale"]))
-    return api.Table(2, n, k, to_dev(q["data"]), block_scale=to_dev(q["block_scale"]),
+    return api.Table(2, n, k, to_dev(q["data"]), block_scale=to_dev(pad_scales(q["block_scale"], k)),
                      global_scale=torch.tensor([q["global_scale"]], dtype=torch.float32,
                                                device="cuda"))
 
@@ -81,9 +81,9 @@ def check(orc, fmt, q, k, x_u16, got, n_eff=None, mask=None, mask_words=0, strid
     assert (flags & L.MTP_DEVFLAG_EMPTY_MASK) == (ref_f & 2)
 
 
-SHAPES = {0: [(1000, 256), (1000, 4096), (4133, 512)],
-          1: [(1000, 64), (1000, 4096), (517, 1040)],
-          2: [(1000, 128), (1000, 5120), (517, 1056)]}
+SHAPES = {0: [(1000, 256), (1000, 4096), (4133, 576)],
+          1: [(1000, 128), (1000, 4096), (517, 1152)],
+          2: [(1000, 256), (1000, 5120), (517, 1280)]}
 
 
 @pytest.mark.parametrize("fmt", [0, 1, 2])
