@@ -15,17 +15,19 @@
 // mbarrier. Large single copies matter: the TMA unit's per-copy cost caps a ring fed
 // by 1 KB row copies at about half of HBM bandwidth, while 16 KB tensor boxes stream
 // at the copy peak. Out-of-range rows and K tails arrive as zeros (tensor-map bounds).
-// Eight consumer warps split each stage's K range (16 slabs of 4 lanes x 16 B; warp w
-// takes slabs w and w+8), decode the codes exactly into f16/bf16 fragments and run
+// Sixteen compute warps (eight when M > 8) split each stage's K range into 16 slabs of
+// 4 lanes x 16 B, decode the codes exactly into f16/bf16 fragments and run
 // tensor-core MMAs with 16 table rows as the A operand and up to 16 inputs as the B
 // operand (swap-AB). MMA row g reads table row s(g) of the tile, a fixed permutation
 // that, with the swizzle, makes every shared-memory read conflict-free. E4M3 codes and
 // E2M1 codes times their E4M3 block scale are exact in f16; x is staged once per CTA
 // (bf16 for BF16 tables; f16 scaled by a per-row power of two for quantized tables,
-// undone in fp32), so the only roundings are the fp32 accumulation. Per tile the eight
-// warp partials are summed in a fixed order (deterministic and independent of M),
-// scaled, masked and folded into a running (max, lowest index) per input row. Tiles
-// whose 16 rows are all masked out for every input are neither loaded nor computed.
+// undone in fp32), so the only roundings are the fp32 accumulation. At the end of a
+// tile each compute warp hands its partial to a reducer warp through a double-buffered
+// shared slot (mbarrier hand-off, no CTA-wide barrier on the streaming path). The
+// reducer sums the partials in a fixed warp order (deterministic and independent of
+// M), scales, masks and folds them into a running (max, lowest index) per input row.
+// Tiles whose 16 rows are masked out for every input are neither loaded nor computed.
 // Each CTA writes its partial; the last CTA to finish (atomic ticket, no waiting)
 // reduces them in CTA order and re-zeroes the ticket. Every mbarrier wait is bounded:
 // a wait that runs out sets an abort flag and MTP_DEVFLAG_TIMEOUT, and the kernel runs
@@ -43,16 +45,24 @@
 namespace mtp {
 namespace {
 
-constexpr int kConsumerWarps = 8;
-constexpr int kConsumers = kConsumerWarps * 32;
-constexpr int kThreads = kConsumers + 32;  // + one producer warp
 constexpr int kTileRows = 16;
+constexpr int kSlabs = 16;  // slabs of 4 lanes x 16 bytes per stage row chunk
 constexpr int kMaxGrid = 1024;
 constexpr int kMaxStages = 12;
 constexpr int kStageRowBytes = 1024;                  // code bytes of one row per stage
 constexpr int kCodeStageBytes = kTileRows * kStageRowBytes;
 constexpr int kScaleStageBytes = kTileRows * 128;     // NVFP4: 128 scale bytes per row
 constexpr int kSmemLimit = 227 * 1024;
+
+// Warp roles: CW compute warps, then one reducer warp, then one producer warp.
+// M <= 8 uses 16 compute warps (one slab each per stage); M > 8 uses 8 (two slabs
+// each), which leaves shared memory for the larger staged input.
+template <int NT> struct Roles {
+    static constexpr int CW = NT == 1 ? 16 : 8;
+    static constexpr int SPW = kSlabs / CW;  // slabs per compute warp per stage
+    static constexpr int THREADS = (CW + 2) * 32;
+    static constexpr int RED_COLS = 8 * NT;
+};
 
 struct Partial {
     float v;
@@ -72,8 +82,8 @@ __host__ __device__ inline int stage_bytes_for(int fmt) {
 // MMA row g of a tile reads table row s(g) (a bijection on 0..15 with s(g+8) = s(g)+8).
 __device__ __forceinline__ int tile_row(int g) { return (g & 8) | ((g & 1) << 2) | ((g >> 1) & 3); }
 
-// Byte offset of logical byte b of row r inside a stage written by a 128-byte-swizzled
-// box of 128-byte segments: 16-byte chunk bits [4:6] are XORed with bits [7:9].
+// Byte offset of a logical byte inside a stage written by a 128-byte-swizzled box of
+// 128-byte segments: 16-byte chunk bits [4:6] are XORed with bits [7:9].
 __device__ __forceinline__ uint32_t swz(uint32_t logical) {
     return logical ^ (((logical >> 7) & 7u) << 4);
 }
@@ -113,40 +123,49 @@ __device__ __forceinline__ bool row_needed(const SweepParams& p, int64_t row) {
     return false;
 }
 
-// Reductions over the 256 consumer threads (named barrier 1).
-__device__ __forceinline__ float consumer_sum(float v, float* scratch) {
+// True when some row of the tile is allowed for some input (whole warp calls it).
+__device__ __forceinline__ bool tile_needed(const SweepParams& p, int64_t tile, int lane) {
+    const bool need = lane < kTileRows && row_needed(p, tile * kTileRows + lane);
+    return __ballot_sync(0xffffffffu, need) != 0u;
+}
+
+// Reductions over the CW compute warps (named barrier 1).
+template <int CW>
+__device__ __forceinline__ float compute_sum(float v, float* scratch) {
     for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    named_sync(1, kConsumers);
+    named_sync(1, CW * 32);
     if (lane == 0) scratch[warp] = v;
-    named_sync(1, kConsumers);
+    named_sync(1, CW * 32);
     float t = 0.f;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) t += scratch[w];
+    for (int w = 0; w < CW; ++w) t += scratch[w];
     return t;
 }
 
-__device__ __forceinline__ float consumer_max(float v, float* scratch) {
+template <int CW>
+__device__ __forceinline__ float compute_max(float v, float* scratch) {
     for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    named_sync(1, kConsumers);
+    named_sync(1, CW * 32);
     if (lane == 0) scratch[warp] = v;
-    named_sync(1, kConsumers);
+    named_sync(1, CW * 32);
     float t = 0.f;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) t = fmaxf(t, scratch[w]);
+    for (int w = 0; w < CW; ++w) t = fmaxf(t, scratch[w]);
     return t;
 }
 
 // Stage x (bf16) into xs[m][0..K): a copy (mode 0) or the combiner's concat
-// [bf16(rms(e) w_e) || bf16(rms(hidden) w_h)] (mode 1).
-template <int MODE>
+// [bf16(rms(e) w_e) || bf16(rms(hidden) w_h)] (mode 1). Compute warps only.
+template <int MODE, int CW>
 __device__ void stage_bf16(const SweepParams& p, uint16_t* xs, float* scratch) {
+    constexpr int NTH = CW * 32;
     const int tid = threadIdx.x;
     const int64_t K = p.k;
     if (MODE == 0) {
         const int vecs = (int)(K / 8);
-        for (int i = tid; i < p.M * vecs; i += kConsumers) {
+        for (int i = tid; i < p.M * vecs; i += NTH) {
             int m = i / vecs, v = i - m * vecs;
             uint4 val = *reinterpret_cast<const uint4*>(p.x + (int64_t)m * K + (int64_t)v * 8);
             *reinterpret_cast<uint4*>(xs + (int64_t)m * p.kpad + (int64_t)v * 8) = val;
@@ -160,18 +179,18 @@ __device__ void stage_bf16(const SweepParams& p, uint16_t* xs, float* scratch) {
             const uint16_t* e = bad ? nullptr : p.embed + tok * h;
             const uint16_t* hx = p.hidden + (int64_t)m * h;
             float se = 0.f, sx = 0.f;
-            for (int j = tid; j < h; j += kConsumers) {
+            for (int j = tid; j < h; j += NTH) {
                 float ev = e ? bf16_to_f32(e[j]) : 0.f;
                 float xv = bf16_to_f32(hx[j]);
                 se += ev * ev;
                 sx += xv * xv;
             }
-            se = consumer_sum(se, scratch);
-            sx = consumer_sum(sx, scratch + kConsumerWarps);
+            se = compute_sum<CW>(se, scratch);
+            sx = compute_sum<CW>(sx, scratch + CW);
             float inv_e = 1.0f / sqrtf(se / (float)h + p.eps);
             float inv_x = 1.0f / sqrtf(sx / (float)h + p.eps);
             uint16_t* row = xs + (int64_t)m * p.kpad;
-            for (int j = tid; j < h; j += kConsumers) {
+            for (int j = tid; j < h; j += NTH) {
                 float ev = e ? bf16_to_f32(e[j]) : 0.f;
                 row[j] = f32_to_bf16(ev * inv_e * bf16_to_f32(p.w_norm_embed[j]));
                 row[h + j] = f32_to_bf16(bf16_to_f32(hx[j]) * inv_x *
@@ -179,52 +198,135 @@ __device__ void stage_bf16(const SweepParams& p, uint16_t* xs, float* scratch) {
             }
         }
     }
-    named_sync(1, kConsumers);
+    named_sync(1, NTH);
 }
 
 // Quantized tables: rescale each staged row by 2^e_m (largest |x| lands in
 // [2^14, 2^15)) and convert it in place to f16. Exact for every element within
 // 2^29 of the row maximum; the power of two is undone on the fp32 logit.
+template <int CW>
 __device__ void stage_to_f16(const SweepParams& p, uint16_t* xs, int* xexp, float* scratch) {
+    constexpr int NTH = CW * 32;
     const int tid = threadIdx.x;
     const int K = (int)p.k;
     for (int m = 0; m < p.M; ++m) {
         uint16_t* row = xs + (int64_t)m * p.kpad;
         float a = 0.f;
-        for (int j = tid; j < K; j += kConsumers) a = fmaxf(a, fabsf(bf16_to_f32(row[j])));
-        a = consumer_max(a, scratch);
+        for (int j = tid; j < K; j += NTH) a = fmaxf(a, fabsf(bf16_to_f32(row[j])));
+        a = compute_max<CW>(a, scratch);
         int ex = 0;
         if (a > 0.f) frexpf(a, &ex);
         int e = (a > 0.f) ? 15 - ex : 0;
         if (tid == 0) xexp[m] = e;
-        for (int j = tid; j < K; j += kConsumers)
+        for (int j = tid; j < K; j += NTH)
             row[j] = f32_to_f16(ldexpf(bf16_to_f32(row[j]), e));
-        named_sync(1, kConsumers);
+        named_sync(1, NTH);
     }
 }
 
-__device__ __forceinline__ bool tile_needed(const SweepParams& p, int64_t tile, int lane) {
-    const bool need = lane < kTileRows && row_needed(p, tile * kTileRows + lane);
-    return __ballot_sync(0xffffffffu, need) != 0u;
+// One slab (4 lanes x 16 B of rows r0 and r0 + 8, K elements [e0, e0 + V) for lane c)
+// into the MMA accumulators; accumulator set (mma index & 1) alternates to split the
+// dependence chain.
+template <int FMT, int NT>
+__device__ __forceinline__ void slab_mma(float (&acc)[2][NT][4], const uint8_t* st, int sl,
+                                         int r0, int c, const uint16_t* x0, const uint16_t* x1,
+                                         bool l0, bool l1) {
+    const uint32_t b = (uint32_t)(sl * 64 + c * 16);  // logical byte in the row chunk
+    const uint32_t la = (b >> 7) * 2048u + (uint32_t)r0 * 128u + (b & 127u);
+    const uint4 ra = lds128(st + swz(la));
+    const uint4 rb = lds128(st + swz(la + 8u * 128u));
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    if (FMT == 0) {
+        const uint4 xa = l0 ? lds128(x0) : z;
+        mma_bf16_16816(acc[0][0], ra.x, rb.x, ra.y, rb.y, xa.x, xa.y);
+        mma_bf16_16816(acc[1][0], ra.z, rb.z, ra.w, rb.w, xa.z, xa.w);
+        if (NT > 1) {
+            const uint4 xb = l1 ? lds128(x1) : z;
+            mma_bf16_16816(acc[0][NT - 1], ra.x, rb.x, ra.y, rb.y, xb.x, xb.y);
+            mma_bf16_16816(acc[1][NT - 1], ra.z, rb.z, ra.w, rb.w, xb.z, xb.w);
+        }
+    } else if (FMT == 1) {
+        const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w};
+        const uint32_t wb[4] = {rb.x, rb.y, rb.z, rb.w};
+        const uint4 xa0 = l0 ? lds128(x0) : z;
+        const uint4 xa1 = l0 ? lds128(x0 + 8) : z;
+        const uint32_t xa[8] = {xa0.x, xa0.y, xa0.z, xa0.w, xa1.x, xa1.y, xa1.z, xa1.w};
+        uint32_t xb[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        if (NT > 1) {
+            const uint4 xb0 = l1 ? lds128(x1) : z;
+            const uint4 xb1 = l1 ? lds128(x1 + 8) : z;
+            xb[0] = xb0.x; xb[1] = xb0.y; xb[2] = xb0.z; xb[3] = xb0.w;
+            xb[4] = xb1.x; xb[5] = xb1.y; xb[6] = xb1.z; xb[7] = xb1.w;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t a0 = e4m3x2_to_f16x2((uint16_t)(wa[i] & 0xFFFFu));
+            const uint32_t a2 = e4m3x2_to_f16x2((uint16_t)(wa[i] >> 16));
+            const uint32_t a1 = e4m3x2_to_f16x2((uint16_t)(wb[i] & 0xFFFFu));
+            const uint32_t a3 = e4m3x2_to_f16x2((uint16_t)(wb[i] >> 16));
+            mma_f16_16816(acc[i & 1][0], a0, a1, a2, a3, xa[2 * i], xa[2 * i + 1]);
+            if (NT > 1) mma_f16_16816(acc[i & 1][NT - 1], a0, a1, a2, a3, xb[2 * i], xb[2 * i + 1]);
+        }
+    } else {
+        const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w};
+        const uint32_t wb[4] = {rb.x, rb.y, rb.z, rb.w};
+        // block scales of rows r0 / r0+8: blocks 2c (words 0,1) and 2c+1 (words 2,3)
+        const uint8_t* sp = st + kCodeStageBytes;
+        const uint32_t sbyte = (uint32_t)(sl * 8 + 2 * c);
+        const uint16_t s0v = *reinterpret_cast<const uint16_t*>(sp + swz((uint32_t)r0 * 128u + sbyte));
+        const uint16_t s1v =
+            *reinterpret_cast<const uint16_t*>(sp + swz((uint32_t)(r0 + 8) * 128u + sbyte));
+        const uint32_t sa = e4m3x2_to_f16x2(s0v);
+        const uint32_t sb = e4m3x2_to_f16x2(s1v);
+        const uint32_t sa_lo = __byte_perm(sa, 0, 0x1010), sa_hi = __byte_perm(sa, 0, 0x3232);
+        const uint32_t sb_lo = __byte_perm(sb, 0, 0x1010), sb_hi = __byte_perm(sb, 0, 0x3232);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            uint32_t qa[4], qb[4];
+            e2m1x8_to_f16x2x4(wa[i], qa);
+            e2m1x8_to_f16x2x4(wb[i], qb);
+            const uint32_t s_a = i < 2 ? sa_lo : sa_hi;
+            const uint32_t s_b = i < 2 ? sb_lo : sb_hi;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                qa[q] = hmul2(qa[q], s_a);
+                qb[q] = hmul2(qb[q], s_b);
+            }
+            const uint4 xv = l0 ? lds128(x0 + 8 * i) : z;
+            mma_f16_16816(acc[0][0], qa[0], qb[0], qa[1], qb[1], xv.x, xv.y);
+            mma_f16_16816(acc[1][0], qa[2], qb[2], qa[3], qb[3], xv.z, xv.w);
+            if (NT > 1) {
+                const uint4 xw = l1 ? lds128(x1 + 8 * i) : z;
+                mma_f16_16816(acc[0][NT - 1], qa[0], qb[0], qa[1], qb[1], xw.x, xw.y);
+                mma_f16_16816(acc[1][NT - 1], qa[2], qb[2], qa[3], qb[3], xw.z, xw.w);
+            }
+        }
+    }
 }
 
 template <int FMT, int NT, int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
     sweep_kernel(const __grid_constant__ SweepParams p, const __grid_constant__ CUtensorMap map_codes,
                  const __grid_constant__ CUtensorMap map_scales) {
     constexpr int V = Fmt<FMT>::V;
     constexpr int KC = Fmt<FMT>::KC;
-    constexpr int SLAB = 4 * V;  // K elements of one slab (4 lanes x 16 bytes)
-    constexpr int RED_COLS = 8 * NT;
+    constexpr int SLAB = 4 * V;  // K elements of one slab
+    constexpr int CW = Roles<NT>::CW;
+    constexpr int SPW = Roles<NT>::SPW;
+    constexpr int RED_COLS = Roles<NT>::RED_COLS;
+    constexpr int RED_WARP_FLOATS = kTileRows * RED_COLS;
+    constexpr int REDUCER = CW, PRODUCER = CW + 1;
 
     extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + kMaxStages;
-    int* misc = reinterpret_cast<int*>(empty + kMaxStages);  // [0] abort [1] last [2..17] xexp
+    uint64_t* red_full = empty + kMaxStages;  // [2]
+    uint64_t* red_empty = red_full + 2;       // [2]
+    int* misc = reinterpret_cast<int*>(red_empty + 2);  // [0] abort [2..17] xexp
     volatile int* abort_flag = misc;
     int* xexp = misc + 2;
-    float* red = reinterpret_cast<float*>(misc + 32);  // [2][8][16][RED_COLS]
-    float* scratch = red + 2 * kConsumerWarps * kTileRows * RED_COLS;  // [32]
+    float* red = reinterpret_cast<float*>(misc + 32);  // [2][CW][16][RED_COLS]
+    float* scratch = red + 2 * CW * RED_WARP_FLOATS;   // [32]
     uint16_t* xs = reinterpret_cast<uint16_t*>(scratch + 32);
     // the ring starts on a 1 KB boundary of the shared window (the 128-byte swizzle atom)
     const uint32_t head_end = smem_u32(xs) + (uint32_t)p.M * (uint32_t)p.kpad * 2u;
@@ -235,6 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int S = p.stages;
     const int stage_bytes = p.stage_bytes;
     const int NC = (int)((K + KC - 1) / KC);  // stages per tile
+    const int M = p.M;
 
     const int64_t T = p.num_tiles;
     const int64_t t_begin = (T * blockIdx.x) / gridDim.x;
@@ -243,7 +346,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kConsumerWarps);
+            mbar_init(&empty[s], CW);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&red_full[b], CW);
+            mbar_init(&red_empty[b], 1);
         }
         misc[0] = 0;
         mbar_fence_init();
@@ -251,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
 
     // ------------------------------------------------------------ producer warp
-    if (warp == kConsumerWarps) {
+    if (warp == PRODUCER) {
         int slot = 0;
         uint32_t phase = 0;
         int64_t issued = 0;
@@ -267,11 +374,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) {
                     uint8_t* dst = ring + (size_t)slot * stage_bytes;
                     mbar_arrive_expect_tx(&full[slot], tx);
-                    tma_load_3d(dst, &map_codes, 0, (int)(tile * kTileRows), ch * (kStageRowBytes / 128),
-                                &full[slot]);
+                    tma_load_3d(dst, &map_codes, 0, (int)(tile * kTileRows),
+                                ch * (kStageRowBytes / 128), &full[slot]);
                     if (FMT == 2)
-                        tma_load_2d(dst + kCodeStageBytes, &map_scales, ch * 128, (int)(tile * kTileRows),
-                                    &full[slot]);
+                        tma_load_2d(dst + kCodeStageBytes, &map_scales, ch * 128,
+                                    (int)(tile * kTileRows), &full[slot]);
                 }
                 __syncwarp();
                 ++issued;
@@ -287,128 +394,161 @@ __global__ void __launch_bounds__(kThreads, 1)
         return;
     }
 
-    // ------------------------------------------------------------ consumer warps
+    // ------------------------------------------------------------ reducer warp
+    if (warp == REDUCER) {
+        // lane holds items (row = lane & 15, col = 2q + (lane >> 4)) for q < RED_COLS/2
+        constexpr int Q = RED_COLS / 2;
+        float best_v[Q];
+        int32_t best_i[Q];
+#pragma unroll
+        for (int q = 0; q < Q; ++q) {
+            best_v[q] = -INFINITY;
+            best_i[q] = INT_MAX;
+        }
+        const int rrow = lane & 15;
+        int buf = 0;
+        uint32_t fph = 0u;  // bit b: phase parity of red_full[b]
+        for (int64_t tile = t_begin; tile < t_end; ++tile) {
+            const int64_t row = tile * kTileRows + rrow;
+            if (!tile_needed(p, tile, lane)) {
+                // every row is masked out for every input: logits -inf, nothing to fold
+                if (MODE == 0 && p.out_logits && row < p.n)
+                    for (int col = lane >> 4; col < M; col += 2)
+                        p.out_logits[(int64_t)col * p.n + row] = 0xFF80u;
+                continue;
+            }
+            mbar_wait_bounded(&red_full[buf], (fph >> buf) & 1u, abort_flag);
+            fph ^= 1u << buf;
+            const float* rb = red + (size_t)buf * CW * RED_WARP_FLOATS;
+#pragma unroll
+            for (int q = 0; q < Q; ++q) {
+                const int col = 2 * q + (lane >> 4);
+                if (2 * q >= M) break;  // warp-uniform
+                float a = 0.f;
+                if (CW == 16) {
+#pragma unroll
+                    for (int w = 0; w < 8; ++w)
+                        a += rb[w * RED_WARP_FLOATS + rrow * RED_COLS + col] +
+                             rb[(w + 8) * RED_WARP_FLOATS + rrow * RED_COLS + col];
+                } else {
+#pragma unroll
+                    for (int w = 0; w < CW; ++w) a += rb[w * RED_WARP_FLOATS + rrow * RED_COLS + col];
+                }
+                const bool valid = row < p.n && col < M;
+                float l = a;
+                if (FMT != 0 && valid) l = ldexpf(a, -xexp[col]);
+                if (FMT == 1 && valid) l *= __ldg(p.row_scale + row);
+                if (FMT == 2 && valid) l *= __ldg(p.global_scale);
+                if (MODE == 1) {
+                    if (valid) p.out_y[(int64_t)col * p.n + row] = f32_to_bf16(l);
+                } else {
+                    const bool ok = valid && mask_allows(p, col, row);
+                    if (valid && p.out_logits)
+                        p.out_logits[(int64_t)col * p.n + row] = ok ? f32_to_bf16(l) : (uint16_t)0xFF80u;
+                    float v = ok ? l : -INFINITY;
+                    int32_t i = ok ? (int32_t)row : INT_MAX;
+#pragma unroll
+                    for (int o = 8; o; o >>= 1) {
+                        const float ov = __shfl_xor_sync(0xffffffffu, v, o);
+                        const int32_t oi = __shfl_xor_sync(0xffffffffu, i, o);
+                        if (ov > v || (ov == v && oi < i)) {
+                            v = ov;
+                            i = oi;
+                        }
+                    }
+                    if (v > best_v[q] || (v == best_v[q] && i < best_i[q])) {
+                        best_v[q] = v;
+                        best_i[q] = i;
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&red_empty[buf]);
+            buf ^= 1;
+        }
+        if (*abort_flag) raise_flag(p.dev_err, DEVFLAG_TIMEOUT);
+        if (MODE == 1) return;
+
+        Partial* parts = reinterpret_cast<Partial*>(p.partials);
+#pragma unroll
+        for (int q = 0; q < Q; ++q) {
+            const int col = 2 * q + (lane >> 4);
+            if (rrow == 0 && col < M) parts[(int64_t)blockIdx.x * 16 + col] = Partial{best_v[q], best_i[q]};
+        }
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
+            __threadfence();
+            last = atomicAdd(p.ticket, 1u) == gridDim.x - 1;
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (!last) return;
+        __threadfence();
+        if (lane < M) {
+            float bv = -INFINITY;
+            int32_t bi = INT_MAX;
+            for (int b = 0; b < (int)gridDim.x; ++b) {
+                const Partial* src = parts + (int64_t)b * 16 + lane;
+                const float qv = __ldcg(&src->v);
+                const int32_t qi = __ldcg(&src->i);
+                if (qv > bv || (qv == bv && qi < bi)) {
+                    bv = qv;
+                    bi = qi;
+                }
+            }
+            if (bi == INT_MAX) {
+                bi = 0;
+                bv = -INFINITY;
+                raise_flag(p.dev_err, DEVFLAG_EMPTY_MASK);
+            }
+            p.out_idx[lane] = bi;
+            if (p.out_val) p.out_val[lane] = bv;
+        }
+        __syncwarp();
+        if (lane == 0) *p.ticket = 0u;  // leave the workspace ready for the next call
+        return;
+    }
+
+    // ------------------------------------------------------------ compute warps
     const int g = lane >> 2, c = lane & 3;
-    const int M = p.M;
-    stage_bf16<MODE>(p, xs, scratch);
-    if (FMT != 0) stage_to_f16(p, xs, xexp, scratch);
+    stage_bf16<MODE, CW>(p, xs, scratch);
+    if (FMT != 0) stage_to_f16<CW>(p, xs, xexp, scratch);
 
     const bool xg0 = g < M;
     const bool xg1 = NT > 1 && (8 + g) < M;
     const int r0 = tile_row(g);  // table rows r0 and r0 + 8 of the tile feed MMA rows g, g+8
 
-    // one accumulator set per slab of a stage: two independent MMA chains per warp
-    float accs[2][NT][4];
+    // an accumulator pair per slab this warp owns (SPW slabs)
+    float acc[SPW][2][NT][4];
 #pragma unroll
-    for (int j = 0; j < 2; ++j)
+    for (int j = 0; j < SPW; ++j)
 #pragma unroll
-        for (int t = 0; t < NT; ++t)
+        for (int a = 0; a < 2; ++a)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) accs[j][t][i] = 0.f;
+            for (int t = 0; t < NT; ++t)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[j][a][t][i] = 0.f;
 
-    float best_v = -INFINITY;
-    int32_t best_i = INT_MAX;
-    const int red_threads = kTileRows * RED_COLS;
-    const int rrow = tid & 15, rcol = tid >> 4;
     int buf = 0;
+    uint32_t eph = 0u;  // bit b: phase parity of red_empty[b]
     int slot = 0;
     uint32_t phase = 0;
 
     for (int64_t tile = t_begin; tile < t_end; ++tile) {
-        if (!tile_needed(p, tile, lane)) {  // warp-uniform, same rule as the producer
-            // every row of the tile is masked out for every input: logits are -inf
-            if (MODE == 0 && p.out_logits && tid < red_threads) {
-                const int64_t row = tile * kTileRows + rrow;
-                if (row < p.n && rcol < M) p.out_logits[(int64_t)rcol * p.n + row] = 0xFF80u;
-            }
-            continue;
-        }
+        if (!tile_needed(p, tile, lane)) continue;  // warp-uniform, same rule as the producer
         for (int ch = 0; ch < NC; ++ch) {
             mbar_wait_bounded(&full[slot], phase, abort_flag);
             const uint8_t* st = ring + (size_t)slot * stage_bytes;
             const int64_t kc0 = (int64_t)ch * KC;
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                float(&acc)[NT][4] = accs[j];
-                const int sl = warp + kConsumerWarps * j;
+            for (int j = 0; j < SPW; ++j) {
+                const int sl = warp + CW * j;
                 const int64_t s0 = kc0 + (int64_t)sl * SLAB;
                 if (s0 >= K) continue;  // warp-uniform: slab past the end of K
                 const int64_t e0 = s0 + c * V;
                 const bool kin = e0 < K;  // beyond K the stage holds zeros
-                const uint32_t b = (uint32_t)(sl * 64 + c * 16);  // logical byte in the row chunk
-                const uint32_t la = (b >> 7) * 2048u + (uint32_t)r0 * 128u + (b & 127u);
-                const uint4 ra = lds128(st + swz(la));
-                const uint4 rb = lds128(st + swz(la + 8u * 128u));
-                const uint16_t* x0 = xs + (int64_t)g * p.kpad + e0;
-                const uint16_t* x1 = xs + (int64_t)(8 + g) * p.kpad + e0;
-                const bool l0 = xg0 && kin, l1 = xg1 && kin;
-                if (FMT == 0) {
-                    uint4 xa = l0 ? lds128(x0) : make_uint4(0, 0, 0, 0);
-                    mma_bf16_16816(acc[0], ra.x, rb.x, ra.y, rb.y, xa.x, xa.y);
-                    mma_bf16_16816(acc[0], ra.z, rb.z, ra.w, rb.w, xa.z, xa.w);
-                    if (NT > 1) {
-                        uint4 xb = l1 ? lds128(x1) : make_uint4(0, 0, 0, 0);
-                        mma_bf16_16816(acc[NT - 1], ra.x, rb.x, ra.y, rb.y, xb.x, xb.y);
-                        mma_bf16_16816(acc[NT - 1], ra.z, rb.z, ra.w, rb.w, xb.z, xb.w);
-                    }
-                } else if (FMT == 1) {
-                    const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w};
-                    const uint32_t wb[4] = {rb.x, rb.y, rb.z, rb.w};
-                    const uint4 xa0 = l0 ? lds128(x0) : make_uint4(0, 0, 0, 0);
-                    const uint4 xa1 = l0 ? lds128(x0 + 8) : make_uint4(0, 0, 0, 0);
-                    const uint32_t xa[8] = {xa0.x, xa0.y, xa0.z, xa0.w, xa1.x, xa1.y, xa1.z, xa1.w};
-                    uint32_t xb[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-                    if (NT > 1) {
-                        const uint4 xb0 = l1 ? lds128(x1) : make_uint4(0, 0, 0, 0);
-                        const uint4 xb1 = l1 ? lds128(x1 + 8) : make_uint4(0, 0, 0, 0);
-                        xb[0] = xb0.x; xb[1] = xb0.y; xb[2] = xb0.z; xb[3] = xb0.w;
-                        xb[4] = xb1.x; xb[5] = xb1.y; xb[6] = xb1.z; xb[7] = xb1.w;
-                    }
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const uint32_t a0 = e4m3x2_to_f16x2((uint16_t)(wa[i] & 0xFFFFu));
-                        const uint32_t a2 = e4m3x2_to_f16x2((uint16_t)(wa[i] >> 16));
-                        const uint32_t a1 = e4m3x2_to_f16x2((uint16_t)(wb[i] & 0xFFFFu));
-                        const uint32_t a3 = e4m3x2_to_f16x2((uint16_t)(wb[i] >> 16));
-                        mma_f16_16816(acc[0], a0, a1, a2, a3, xa[2 * i], xa[2 * i + 1]);
-                        if (NT > 1)
-                            mma_f16_16816(acc[NT - 1], a0, a1, a2, a3, xb[2 * i], xb[2 * i + 1]);
-                    }
-                } else {
-                    const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w};
-                    const uint32_t wb[4] = {rb.x, rb.y, rb.z, rb.w};
-                    // block scales of rows r0 / r0+8: blocks 2c (words 0,1) and 2c+1 (words 2,3)
-                    const uint8_t* sp = st + kCodeStageBytes;
-                    const uint32_t sbyte = (uint32_t)(sl * 8 + 2 * c);
-                    const uint16_t s0v = *reinterpret_cast<const uint16_t*>(sp + swz((uint32_t)r0 * 128u + sbyte));
-                    const uint16_t s1v =
-                        *reinterpret_cast<const uint16_t*>(sp + swz((uint32_t)(r0 + 8) * 128u + sbyte));
-                    const uint32_t sa = e4m3x2_to_f16x2(s0v);
-                    const uint32_t sb = e4m3x2_to_f16x2(s1v);
-                    const uint32_t sa_lo = __byte_perm(sa, 0, 0x1010), sa_hi = __byte_perm(sa, 0, 0x3232);
-                    const uint32_t sb_lo = __byte_perm(sb, 0, 0x1010), sb_hi = __byte_perm(sb, 0, 0x3232);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        uint32_t qa[4], qb[4];
-                        e2m1x8_to_f16x2x4(wa[i], qa);
-                        e2m1x8_to_f16x2x4(wb[i], qb);
-                        const uint32_t s_a = i < 2 ? sa_lo : sa_hi;
-                        const uint32_t s_b = i < 2 ? sb_lo : sb_hi;
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            qa[q] = hmul2(qa[q], s_a);
-                            qb[q] = hmul2(qb[q], s_b);
-                        }
-                        const uint4 xv = l0 ? lds128(x0 + 8 * i) : make_uint4(0, 0, 0, 0);
-                        mma_f16_16816(acc[0], qa[0], qb[0], qa[1], qb[1], xv.x, xv.y);
-                        mma_f16_16816(acc[0], qa[2], qb[2], qa[3], qb[3], xv.z, xv.w);
-                        if (NT > 1) {
-                            const uint4 xw = l1 ? lds128(x1 + 8 * i) : make_uint4(0, 0, 0, 0);
-                            mma_f16_16816(acc[NT - 1], qa[0], qb[0], qa[1], qb[1], xw.x, xw.y);
-                            mma_f16_16816(acc[NT - 1], qa[2], qb[2], qa[3], qb[3], xw.z, xw.w);
-                        }
-                    }
-                }
+                slab_mma<FMT, NT>(acc[j], st, sl, r0, c, xs + (int64_t)g * p.kpad + e0,
+                                  xs + (int64_t)(8 + g) * p.kpad + e0, xg0 && kin, xg1 && kin);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[slot]);
@@ -417,95 +557,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                 phase ^= 1u;
             }
         }
-
-        // ---- tile done: cross-warp sum (fixed order), scale, mask, running argmax
-        {
-            float* rp = red + (size_t)buf * kConsumerWarps * kTileRows * RED_COLS +
-                        warp * kTileRows * RED_COLS;
+        // hand this warp's partial of the tile to the reducer (double-buffered). The
+        // summation order is fixed whatever the warp count: a slab's partial is
+        // acc[0] + acc[1]; slabs w and w + 8 are added first (here when one warp owns
+        // both, by the reducer otherwise), then the eight pair sums in order of w.
+        mbar_wait_bounded(&red_empty[buf], ((eph >> buf) & 1u) ^ 1u, abort_flag);
+        eph ^= 1u << buf;
+        float* rp = red + (size_t)buf * CW * RED_WARP_FLOATS + warp * RED_WARP_FLOATS;
 #pragma unroll
-            for (int t = 0; t < NT; ++t) {
-                rp[r0 * RED_COLS + t * 8 + 2 * c] = accs[0][t][0] + accs[1][t][0];
-                rp[r0 * RED_COLS + t * 8 + 2 * c + 1] = accs[0][t][1] + accs[1][t][1];
-                rp[(r0 + 8) * RED_COLS + t * 8 + 2 * c] = accs[0][t][2] + accs[1][t][2];
-                rp[(r0 + 8) * RED_COLS + t * 8 + 2 * c + 1] = accs[0][t][3] + accs[1][t][3];
+        for (int t = 0; t < NT; ++t) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) accs[0][t][i] = accs[1][t][i] = 0.f;
+            for (int i = 0; i < 4; ++i) {
+                float v = acc[0][0][t][i] + acc[0][1][t][i];
+                if (SPW == 2) v = v + (acc[SPW - 1][0][t][i] + acc[SPW - 1][1][t][i]);
+                const int row = (i < 2 ? r0 : r0 + 8);
+                rp[row * RED_COLS + t * 8 + 2 * c + (i & 1)] = v;
+#pragma unroll
+                for (int j = 0; j < SPW; ++j) acc[j][0][t][i] = acc[j][1][t][i] = 0.f;
             }
         }
-        named_sync(1, kConsumers);
-        if (tid < red_threads) {
-            const float* rb = red + (size_t)buf * kConsumerWarps * kTileRows * RED_COLS;
-            float a = 0.f;
-#pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) a += rb[(w * kTileRows + rrow) * RED_COLS + rcol];
-            const int64_t row = tile * kTileRows + rrow;
-            const bool valid = row < p.n && rcol < M;
-            float l = a;
-            if (FMT != 0 && valid) l = ldexpf(a, -xexp[rcol]);
-            if (FMT == 1 && valid) l *= __ldg(p.row_scale + row);
-            if (FMT == 2 && valid) l *= __ldg(p.global_scale);
-            if (MODE == 1) {
-                if (valid) p.out_y[(int64_t)rcol * p.n + row] = f32_to_bf16(l);
-            } else {
-                const bool ok = valid && mask_allows(p, rcol, row);
-                if (valid && p.out_logits)
-                    p.out_logits[(int64_t)rcol * p.n + row] = ok ? f32_to_bf16(l) : (uint16_t)0xFF80u;
-                float v = ok ? l : -INFINITY;
-                int32_t i = ok ? (int32_t)row : INT_MAX;
-#pragma unroll
-                for (int o = 8; o; o >>= 1) {
-                    const float ov = __shfl_xor_sync(0xffffffffu, v, o);
-                    const int32_t oi = __shfl_xor_sync(0xffffffffu, i, o);
-                    if (ov > v || (ov == v && oi < i)) {
-                        v = ov;
-                        i = oi;
-                    }
-                }
-                if (rrow == 0 && (v > best_v || (v == best_v && i < best_i))) {
-                    best_v = v;
-                    best_i = i;
-                }
-            }
-        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&red_full[buf]);
         buf ^= 1;
     }
-
-    if (*abort_flag) raise_flag(p.dev_err, DEVFLAG_TIMEOUT);
-    if (MODE == 1) return;
-
-    Partial* parts = reinterpret_cast<Partial*>(p.partials);
-    if (tid < red_threads && rrow == 0 && rcol < M)
-        parts[(int64_t)blockIdx.x * 16 + rcol] = Partial{best_v, best_i};
-    named_sync(1, kConsumers);
-    if (tid == 0) {
-        __threadfence();
-        const unsigned int ticket = atomicAdd(p.ticket, 1u);
-        misc[1] = (ticket == gridDim.x - 1) ? 1 : 0;
-    }
-    named_sync(1, kConsumers);
-    if (misc[1] == 0) return;
-    __threadfence();
-    if (tid < M) {
-        float bv = -INFINITY;
-        int32_t bi = INT_MAX;
-        for (int b = 0; b < (int)gridDim.x; ++b) {
-            const Partial* src = parts + (int64_t)b * 16 + tid;
-            const float qv = __ldcg(&src->v);
-            const int32_t qi = __ldcg(&src->i);
-            if (qv > bv || (qv == bv && qi < bi)) {
-                bv = qv;
-                bi = qi;
-            }
-        }
-        if (bi == INT_MAX) {
-            bi = 0;
-            bv = -INFINITY;
-            raise_flag(p.dev_err, DEVFLAG_EMPTY_MASK);
-        }
-        p.out_idx[tid] = bi;
-        if (p.out_val) p.out_val[tid] = bv;
-    }
-    if (tid == 0) *p.ticket = 0u;  // leave the workspace ready for the next call
 }
 
 struct Geometry {
@@ -519,9 +593,10 @@ Geometry geometry(int M, int64_t k, int fmt) {
     Geometry g{};
     g.kpad = (int)(k + 8);  // 16-byte skew between staged rows
     const int NT = M > 8 ? 2 : 1;
-    size_t head = (size_t)2 * kMaxStages * 8 + 32 * sizeof(int) +
-                  (size_t)2 * kConsumerWarps * kTileRows * 8 * NT * sizeof(float) +
-                  32 * sizeof(float) + (size_t)M * g.kpad * 2;
+    const int CW = NT == 1 ? Roles<1>::CW : Roles<2>::CW;
+    size_t head = (size_t)(2 * kMaxStages + 4) * 8 + 32 * sizeof(int) +
+                  (size_t)2 * CW * kTileRows * 8 * NT * sizeof(float) + 32 * sizeof(float) +
+                  (size_t)M * g.kpad * 2;
     head = ((head + 1023) & ~(size_t)1023) + 1024;  // 1 KB-aligned ring, plus slack
     g.stage_bytes = stage_bytes_for(fmt);
     long avail = (long)kSmemLimit - (long)head;
@@ -610,7 +685,7 @@ cudaError_t launch_one(const SweepParams& p, cudaStream_t s, SweepLaunch* info) 
     q.kpad = geo.kpad;
     q.stages = geo.stages;
     q.stage_bytes = geo.stage_bytes;
-    kern<<<(int)grid, kThreads, geo.smem, s>>>(q, map_codes, map_scales);
+    kern<<<(int)grid, Roles<NT>::THREADS, geo.smem, s>>>(q, map_codes, map_scales);
     if (info) {
         info->grid = (int)grid;
         info->smem_bytes = (int)geo.smem;
