@@ -47,6 +47,8 @@ struct SweepParams {
     int64_t scale_pitch;         // NVFP4: bytes between block-scale rows
     int32_t stages;              // ring depth (set by the launcher)
     int32_t stage_bytes;
+    int32_t segs;                // 128-byte row segments per stage
+    int32_t stages_per_tile;
 };
 
 struct SweepLaunch {

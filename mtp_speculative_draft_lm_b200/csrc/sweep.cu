@@ -46,20 +46,16 @@ namespace mtp {
 namespace {
 
 constexpr int kTileRows = 16;
-constexpr int kSlabs = 16;  // slabs of 4 lanes x 16 bytes per stage row chunk
 constexpr int kMaxGrid = 1024;
 constexpr int kMaxStages = 12;
-constexpr int kStageRowBytes = 1024;                  // code bytes of one row per stage
-constexpr int kCodeStageBytes = kTileRows * kStageRowBytes;
-constexpr int kScaleStageBytes = kTileRows * 128;     // NVFP4: 128 scale bytes per row
+constexpr int kMaxSegs = 16;  // 128-byte segments of a row per stage (box of 16 rows x 2 KB)
 constexpr int kSmemLimit = 227 * 1024;
 
 // Warp roles: CW compute warps, then one reducer warp, then one producer warp.
-// M <= 8 uses 16 compute warps (one slab each per stage); M > 8 uses 8 (two slabs
-// each), which leaves shared memory for the larger staged input.
+// M <= 8 uses 16 compute warps; M > 8 uses 8, which leaves shared memory for the
+// larger staged input.
 template <int NT> struct Roles {
     static constexpr int CW = NT == 1 ? 16 : 8;
-    static constexpr int SPW = kSlabs / CW;  // slabs per compute warp per stage
     static constexpr int THREADS = (CW + 2) * 32;
     static constexpr int RED_COLS = 8 * NT;
 };
@@ -69,14 +65,19 @@ struct Partial {
     int32_t i;
 };
 
-// V: K elements per 16-byte piece; KC: K elements per stage (1 KB of codes per row)
+// V: K elements per 16-byte piece of codes. A slab is 64 bytes of one row (4 lanes x
+// 16 B, 4V elements); a stage holds `segs` 128-byte segments (2 * segs slabs) of each
+// of the tile's 16 rows, plus for NVFP4 the matching 16 * segs block-scale bytes.
 template <int FMT> struct Fmt;
-template <> struct Fmt<0> { static constexpr int V = 8;  static constexpr int KC = 512; };
-template <> struct Fmt<1> { static constexpr int V = 16; static constexpr int KC = 1024; };
-template <> struct Fmt<2> { static constexpr int V = 32; static constexpr int KC = 2048; };
+template <> struct Fmt<0> { static constexpr int V = 8; };
+template <> struct Fmt<1> { static constexpr int V = 16; };
+template <> struct Fmt<2> { static constexpr int V = 32; };
 
-__host__ __device__ inline int stage_bytes_for(int fmt) {
-    return fmt == 2 ? kCodeStageBytes + kScaleStageBytes : kCodeStageBytes;  // multiples of 1 KB
+__host__ __device__ inline int code_stage_bytes(int segs) { return kTileRows * 128 * segs; }
+__host__ __device__ inline int scale_stage_bytes(int segs) { return kTileRows * 16 * segs; }
+__host__ __device__ inline int stage_bytes_for(int fmt, int segs) {
+    int b = code_stage_bytes(segs) + (fmt == 2 ? scale_stage_bytes(segs) : 0);
+    return (b + 1023) & ~1023;
 }
 
 // MMA row g of a tile reads table row s(g) (a bijection on 0..15 with s(g+8) = s(g)+8).
@@ -230,7 +231,7 @@ __device__ void stage_to_f16(const SweepParams& p, uint16_t* xs, int* xexp, floa
 template <int FMT, int NT>
 __device__ __forceinline__ void slab_mma(float (&acc)[2][NT][4], const uint8_t* st, int sl,
                                          int r0, int c, const uint16_t* x0, const uint16_t* x1,
-                                         bool l0, bool l1) {
+                                         bool l0, bool l1, int segs) {
     const uint32_t b = (uint32_t)(sl * 64 + c * 16);  // logical byte in the row chunk
     const uint32_t la = (b >> 7) * 2048u + (uint32_t)r0 * 128u + (b & 127u);
     const uint4 ra = lds128(st + swz(la));
@@ -270,12 +271,13 @@ __device__ __forceinline__ void slab_mma(float (&acc)[2][NT][4], const uint8_t* 
     } else {
         const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w};
         const uint32_t wb[4] = {rb.x, rb.y, rb.z, rb.w};
-        // block scales of rows r0 / r0+8: blocks 2c (words 0,1) and 2c+1 (words 2,3)
-        const uint8_t* sp = st + kCodeStageBytes;
+        // block scales of rows r0 / r0+8: blocks 2c (words 0,1) and 2c+1 (words 2,3);
+        // the stage's scales are [16 rows][16 * segs bytes], unswizzled
+        const uint8_t* sp = st + code_stage_bytes(segs);
+        const uint32_t spitch = 16u * (uint32_t)segs;
         const uint32_t sbyte = (uint32_t)(sl * 8 + 2 * c);
-        const uint16_t s0v = *reinterpret_cast<const uint16_t*>(sp + swz((uint32_t)r0 * 128u + sbyte));
-        const uint16_t s1v =
-            *reinterpret_cast<const uint16_t*>(sp + swz((uint32_t)(r0 + 8) * 128u + sbyte));
+        const uint16_t s0v = *reinterpret_cast<const uint16_t*>(sp + (uint32_t)r0 * spitch + sbyte);
+        const uint16_t s1v = *reinterpret_cast<const uint16_t*>(sp + (uint32_t)(r0 + 8) * spitch + sbyte);
         const uint32_t sa = e4m3x2_to_f16x2(s0v);
         const uint32_t sb = e4m3x2_to_f16x2(s1v);
         const uint32_t sa_lo = __byte_perm(sa, 0, 0x1010), sa_hi = __byte_perm(sa, 0, 0x3232);
@@ -309,10 +311,8 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
     sweep_kernel(const __grid_constant__ SweepParams p, const __grid_constant__ CUtensorMap map_codes,
                  const __grid_constant__ CUtensorMap map_scales) {
     constexpr int V = Fmt<FMT>::V;
-    constexpr int KC = Fmt<FMT>::KC;
     constexpr int SLAB = 4 * V;  // K elements of one slab
     constexpr int CW = Roles<NT>::CW;
-    constexpr int SPW = Roles<NT>::SPW;
     constexpr int RED_COLS = Roles<NT>::RED_COLS;
     constexpr int RED_WARP_FLOATS = kTileRows * RED_COLS;
     constexpr int REDUCER = CW, PRODUCER = CW + 1;
@@ -336,7 +336,9 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
     const int64_t K = p.k;
     const int S = p.stages;
     const int stage_bytes = p.stage_bytes;
-    const int NC = (int)((K + KC - 1) / KC);  // stages per tile
+    const int segs = p.segs;                   // 128-byte segments per row per stage
+    const int slabs_per_stage = 2 * segs;
+    const int NC = p.stages_per_tile;          // ceil(row segments / segs)
     const int M = p.M;
 
     const int64_t T = p.num_tiles;
@@ -362,7 +364,7 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
         int slot = 0;
         uint32_t phase = 0;
         int64_t issued = 0;
-        const uint32_t tx = kCodeStageBytes + (FMT == 2 ? kScaleStageBytes : 0);
+        const uint32_t tx = code_stage_bytes(segs) + (FMT == 2 ? scale_stage_bytes(segs) : 0);
         bool stop = false;
         for (int64_t tile = t_begin; tile < t_end && !stop; ++tile) {
             if (!tile_needed(p, tile, lane)) continue;
@@ -374,10 +376,9 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
                 if (lane == 0) {
                     uint8_t* dst = ring + (size_t)slot * stage_bytes;
                     mbar_arrive_expect_tx(&full[slot], tx);
-                    tma_load_3d(dst, &map_codes, 0, (int)(tile * kTileRows),
-                                ch * (kStageRowBytes / 128), &full[slot]);
+                    tma_load_3d(dst, &map_codes, 0, (int)(tile * kTileRows), ch * segs, &full[slot]);
                     if (FMT == 2)
-                        tma_load_2d(dst + kCodeStageBytes, &map_scales, ch * 128,
+                        tma_load_2d(dst + code_stage_bytes(segs), &map_scales, ch * 16 * segs,
                                     (int)(tile * kTileRows), &full[slot]);
                 }
                 __syncwarp();
@@ -484,25 +485,50 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
         last = __shfl_sync(0xffffffffu, last, 0);
         if (!last) return;
         __threadfence();
-        if (lane < M) {
+        // the last CTA folds every CTA's partial: lane l reads CTAs l, l + 32, ...
+        // (independent loads in flight together), then a shuffle reduction; ties go
+        // to the lowest row index, so the result does not depend on the order
+        const int G = (int)gridDim.x;
+        for (int m = 0; m < M; ++m) {
             float bv = -INFINITY;
             int32_t bi = INT_MAX;
-            for (int b = 0; b < (int)gridDim.x; ++b) {
-                const Partial* src = parts + (int64_t)b * 16 + lane;
-                const float qv = __ldcg(&src->v);
-                const int32_t qi = __ldcg(&src->i);
-                if (qv > bv || (qv == bv && qi < bi)) {
-                    bv = qv;
-                    bi = qi;
+            float qv[kMaxGrid / 32];
+            int32_t qi[kMaxGrid / 32];
+#pragma unroll
+            for (int j = 0; j < kMaxGrid / 32; ++j) {
+                const int b = lane + 32 * j;
+                qv[j] = -INFINITY;
+                qi[j] = INT_MAX;
+                if (b < G) {
+                    const Partial* src = parts + (int64_t)b * 16 + m;
+                    qv[j] = __ldcg(&src->v);
+                    qi[j] = __ldcg(&src->i);
                 }
             }
-            if (bi == INT_MAX) {
-                bi = 0;
-                bv = -INFINITY;
-                raise_flag(p.dev_err, DEVFLAG_EMPTY_MASK);
+#pragma unroll
+            for (int j = 0; j < kMaxGrid / 32; ++j)
+                if (qv[j] > bv || (qv[j] == bv && qi[j] < bi)) {
+                    bv = qv[j];
+                    bi = qi[j];
+                }
+#pragma unroll
+            for (int o = 16; o; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                const int32_t oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                if (ov > bv || (ov == bv && oi < bi)) {
+                    bv = ov;
+                    bi = oi;
+                }
             }
-            p.out_idx[lane] = bi;
-            if (p.out_val) p.out_val[lane] = bv;
+            if (lane == 0) {
+                if (bi == INT_MAX) {
+                    bi = 0;
+                    bv = -INFINITY;
+                    raise_flag(p.dev_err, DEVFLAG_EMPTY_MASK);
+                }
+                p.out_idx[m] = bi;
+                if (p.out_val) p.out_val[m] = bv;
+            }
         }
         __syncwarp();
         if (lane == 0) *p.ticket = 0u;  // leave the workspace ready for the next call
@@ -518,10 +544,14 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
     const bool xg1 = NT > 1 && (8 + g) < M;
     const int r0 = tile_row(g);  // table rows r0 and r0 + 8 of the tile feed MMA rows g, g+8
 
-    // an accumulator pair per slab this warp owns (SPW slabs)
-    float acc[SPW][2][NT][4];
+    // Accumulation chains follow the absolute slab index a (64-byte column block of
+    // the row): chain a % 16 takes slabs in increasing a. With 16 compute warps warp w
+    // owns chain w; with 8, warp w owns chains w and w + 8. The same chains, summed
+    // in the same order, whatever M, the warp count or the stage geometry.
+    constexpr int CH = CW == 16 ? 1 : 2;
+    float acc[CH][2][NT][4];
 #pragma unroll
-    for (int j = 0; j < SPW; ++j)
+    for (int j = 0; j < CH; ++j)
 #pragma unroll
         for (int a = 0; a < 2; ++a)
 #pragma unroll
@@ -539,16 +569,20 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
         for (int ch = 0; ch < NC; ++ch) {
             mbar_wait_bounded(&full[slot], phase, abort_flag);
             const uint8_t* st = ring + (size_t)slot * stage_bytes;
-            const int64_t kc0 = (int64_t)ch * KC;
-#pragma unroll
-            for (int j = 0; j < SPW; ++j) {
-                const int sl = warp + CW * j;
-                const int64_t s0 = kc0 + (int64_t)sl * SLAB;
-                if (s0 >= K) continue;  // warp-uniform: slab past the end of K
+            const int a0 = ch * slabs_per_stage;  // absolute slab index of the stage's first slab
+            // this warp's slabs in the stage: a = a0 + l with a % CW == warp
+            for (int l = (warp - a0 % CW + CW) % CW; l < slabs_per_stage; l += CW) {
+                const int a = a0 + l;
+                const int64_t s0 = (int64_t)a * SLAB;
+                if (s0 >= K) break;  // warp-uniform: past the end of K
                 const int64_t e0 = s0 + c * V;
                 const bool kin = e0 < K;  // beyond K the stage holds zeros
-                slab_mma<FMT, NT>(acc[j], st, sl, r0, c, xs + (int64_t)g * p.kpad + e0,
-                                  xs + (int64_t)(8 + g) * p.kpad + e0, xg0 && kin, xg1 && kin);
+                const uint16_t* x0 = xs + (int64_t)g * p.kpad + e0;
+                const uint16_t* x1 = xs + (int64_t)(8 + g) * p.kpad + e0;
+                if (CH == 2 && ((a >> 3) & 1))
+                    slab_mma<FMT, NT>(acc[CH - 1], st, l, r0, c, x0, x1, xg0 && kin, xg1 && kin, segs);
+                else
+                    slab_mma<FMT, NT>(acc[0], st, l, r0, c, x0, x1, xg0 && kin, xg1 && kin, segs);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[slot]);
@@ -558,9 +592,9 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
             }
         }
         // hand this warp's partial of the tile to the reducer (double-buffered). The
-        // summation order is fixed whatever the warp count: a slab's partial is
-        // acc[0] + acc[1]; slabs w and w + 8 are added first (here when one warp owns
-        // both, by the reducer otherwise), then the eight pair sums in order of w.
+        // summation order is fixed: a chain's partial is acc[0] + acc[1]; chains w and
+        // w + 8 are added first (here when one warp owns both, by the reducer
+        // otherwise), then the eight pair sums in order of w.
         mbar_wait_bounded(&red_empty[buf], ((eph >> buf) & 1u) ^ 1u, abort_flag);
         eph ^= 1u << buf;
         float* rp = red + (size_t)buf * CW * RED_WARP_FLOATS + warp * RED_WARP_FLOATS;
@@ -569,11 +603,11 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 float v = acc[0][0][t][i] + acc[0][1][t][i];
-                if (SPW == 2) v = v + (acc[SPW - 1][0][t][i] + acc[SPW - 1][1][t][i]);
+                if (CH == 2) v = v + (acc[CH - 1][0][t][i] + acc[CH - 1][1][t][i]);
                 const int row = (i < 2 ? r0 : r0 + 8);
                 rp[row * RED_COLS + t * 8 + 2 * c + (i & 1)] = v;
 #pragma unroll
-                for (int j = 0; j < SPW; ++j) acc[j][0][t][i] = acc[j][1][t][i] = 0.f;
+                for (int j = 0; j < CH; ++j) acc[j][0][t][i] = acc[j][1][t][i] = 0.f;
             }
         }
         __syncwarp();
@@ -584,6 +618,8 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
 
 struct Geometry {
     int kpad;
+    int segs;             // 128-byte segments per row per stage
+    int stages_per_tile;  // ceil(row segments / segs)
     int stage_bytes;
     int stages;
     size_t smem;
@@ -598,12 +634,28 @@ Geometry geometry(int M, int64_t k, int fmt) {
                   (size_t)2 * CW * kTileRows * 8 * NT * sizeof(float) + 32 * sizeof(float) +
                   (size_t)M * g.kpad * 2;
     head = ((head + 1023) & ~(size_t)1023) + 1024;  // 1 KB-aligned ring, plus slack
-    g.stage_bytes = stage_bytes_for(fmt);
-    long avail = (long)kSmemLimit - (long)head;
-    int stages = avail > 0 ? (int)(avail / g.stage_bytes) : 0;
-    if (stages > kMaxStages) stages = kMaxStages;
-    g.stages = stages;
-    g.smem = head + (size_t)stages * g.stage_bytes;
+    const int64_t row_bytes = fmt == 0 ? k * 2 : fmt == 1 ? k : k / 2;
+    const int row_segs = (int)(row_bytes / 128);
+    const long avail = (long)kSmemLimit - (long)head;
+    // the widest stage (up to 16 segments) that still leaves a ring of >= 4 stages,
+    // else >= 2; segments are spread evenly over the stages of a row
+    for (int want = 4; want >= 2 && g.stages < 2; want /= 2) {
+        for (int max_segs = kMaxSegs; max_segs >= 1; max_segs /= 2) {
+            const int nc = (row_segs + max_segs - 1) / max_segs;
+            const int segs = (row_segs + nc - 1) / nc;
+            const int sb = stage_bytes_for(fmt, segs);
+            int stages = avail > 0 ? (int)(avail / sb) : 0;
+            if (stages > kMaxStages) stages = kMaxStages;
+            if (stages >= want) {
+                g.segs = segs;
+                g.stages_per_tile = nc;
+                g.stage_bytes = sb;
+                g.stages = stages;
+                break;
+            }
+        }
+    }
+    g.smem = head + (size_t)g.stages * g.stage_bytes;
     return g;
 }
 
@@ -629,12 +681,13 @@ EncodeTiledFn encode_tiled() {
 // Codes: a 3-D view (byte within a 128-byte segment, row, segment) so that one box of
 // 128 B x 16 rows x 8 segments is a stage, with rows inside the 128-byte swizzle atom.
 // Rows >= rows and segments past the row read as zeros.
-cudaError_t make_code_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes) {
+cudaError_t make_code_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes,
+                          int segs) {
     EncodeTiledFn fn = encode_tiled();
     if (!fn) return cudaErrorNotSupported;
     cuuint64_t dims[3] = {128, (cuuint64_t)rows, (cuuint64_t)(row_bytes / 128)};
     cuuint64_t strides[2] = {(cuuint64_t)row_bytes, 128};
-    cuuint32_t box[3] = {128, kTileRows, kStageRowBytes / 128};
+    cuuint32_t box[3] = {128, kTileRows, (cuuint32_t)segs};
     cuuint32_t es[3] = {1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
                     box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -642,16 +695,17 @@ cudaError_t make_code_map(CUtensorMap* m, const void* base, int64_t rows, int64_
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// NVFP4 block scales: [rows, pitch] bytes, boxes of 128 B x 16 rows, 128-byte swizzle.
-cudaError_t make_scale_map(CUtensorMap* m, const void* base, int64_t rows, int64_t pitch) {
+// NVFP4 block scales: [rows, pitch] bytes, boxes of 16 * segs bytes x 16 rows.
+cudaError_t make_scale_map(CUtensorMap* m, const void* base, int64_t rows, int64_t pitch,
+                           int segs) {
     EncodeTiledFn fn = encode_tiled();
     if (!fn) return cudaErrorNotSupported;
     cuuint64_t dims[2] = {(cuuint64_t)pitch, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)pitch};
-    cuuint32_t box[2] = {128, kTileRows};
+    cuuint32_t box[2] = {(cuuint32_t)(16 * segs), kTileRows};
     cuuint32_t es[2] = {1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
-                    box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
@@ -662,10 +716,11 @@ cudaError_t launch_one(const SweepParams& p, cudaStream_t s, SweepLaunch* info) 
     const Geometry geo = geometry(p.M, p.k, FMT);
     if (geo.stages < 2) return cudaErrorInvalidValue;
     CUtensorMap map_codes, map_scales;
-    cudaError_t e = make_code_map(&map_codes, p.w, p.n, p.row_bytes);
+    cudaError_t e = make_code_map(&map_codes, p.w, p.n, p.row_bytes, geo.segs);
     if (e != cudaSuccess) return e;
     if (FMT == 2) {
-        if ((e = make_scale_map(&map_scales, p.block_scale, p.n, p.scale_pitch)) != cudaSuccess)
+        if ((e = make_scale_map(&map_scales, p.block_scale, p.n, p.scale_pitch, geo.segs)) !=
+            cudaSuccess)
             return e;
     } else {
         map_scales = map_codes;  // unused
@@ -685,6 +740,8 @@ cudaError_t launch_one(const SweepParams& p, cudaStream_t s, SweepLaunch* info) 
     q.kpad = geo.kpad;
     q.stages = geo.stages;
     q.stage_bytes = geo.stage_bytes;
+    q.segs = geo.segs;
+    q.stages_per_tile = geo.stages_per_tile;
     kern<<<(int)grid, Roles<NT>::THREADS, geo.smem, s>>>(q, map_codes, map_scales);
     if (info) {
         info->grid = (int)grid;
