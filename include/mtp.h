@@ -187,6 +187,28 @@ mtp_status mtp_lm_head_argmax(const mtp_weight* head, int64_t n_eff, const uint1
                               uint16_t* out_logits, int32_t* dev_err, void* ws,
                               size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------------
+ * mtp_lm_head_argmax_noalloc -- mtp_lm_head_argmax without a workspace argument.
+ * The pages have no counterpart: this entry point exists for callers that cannot
+ * allocate device memory when they run a draft (a plugin inside another framework's
+ * memory pool, an engine that reserves all free memory for its KV cache at start-up,
+ * code that must not risk the device synchronisation cudaMalloc/cudaFree can cause).
+ * Inputs and outputs are the caller's, exactly as for mtp_lm_head_argmax; the scratch
+ * is a static device array inside the library, mtp_noalloc_scratch_bytes() bytes
+ * (131,328) held on every GPU that loads the library until the process exits.
+ *  - The first call made with a device current looks up that array's device address
+ *    and zeroes its counter (synchronously); make it before any stream capture.
+ *  - All calls on a device share the array: calls that overlap on the GPU race and
+ *    must be serialised by the caller. Each call leaves the counter zero again.
+ *  - Returns MTP_ERR_WORKSPACE if a call would need more scratch than the array holds;
+ *    it never allocates.
+ * ------------------------------------------------------------------------------ */
+size_t mtp_noalloc_scratch_bytes(void);
+mtp_status mtp_lm_head_argmax_noalloc(const mtp_weight* head, int64_t n_eff, const uint16_t* x,
+                                      int32_t M, const int32_t* mask, int64_t mask_words,
+                                      int64_t mask_stride_words, int32_t* out_idx, float* out_val,
+                                      uint16_t* out_logits, int32_t* dev_err, void* stream);
+
 /* Maps a device error word read back by the caller to a status: MTP_OK, or
  * MTP_WARN_EMPTY_MASK when only the empty-mask bit is set, else MTP_ERR_INVALID_ARG. */
 mtp_status mtp_devflags_status(int32_t dev_err_value);

@@ -36,6 +36,7 @@ EXPORTS = (
     "mtp_quantize_fp8", "mtp_quantize_nvfp4_ws_bytes", "mtp_quantize_nvfp4",
     "mtp_combine", "mtp_lm_head_ws_bytes", "mtp_lm_head_argmax",
     "mtp_debug_encode_e4m3", "mtp_debug_encode_e2m1", "mtp_nvfp4_scale_pitch",
+    "mtp_noalloc_scratch_bytes", "mtp_lm_head_argmax_noalloc",
 )
 
 
@@ -70,6 +71,9 @@ _SIGS = {
     "mtp_lm_head_ws_bytes": (_SZ, [_W, _I64, _I32]),
     "mtp_lm_head_argmax": (C.c_int, [_W, _I64, _P, _I32, _P, _I64, _I64, _P, _P, _P, _P,
                                      _P, _SZ, _P]),
+    "mtp_noalloc_scratch_bytes": (_SZ, []),
+    "mtp_lm_head_argmax_noalloc": (C.c_int, [_W, _I64, _P, _I32, _P, _I64, _I64, _P, _P, _P,
+                                             _P, _P]),
     "mtp_debug_encode_e4m3": (C.c_int, [_P, _I64, _P, _P]),
     "mtp_debug_encode_e2m1": (C.c_int, [_P, _I64, _P, _P]),
 }
@@ -171,6 +175,19 @@ def mtp_lm_head_argmax(head, n_eff, x, M, mask, mask_words, mask_stride_words, o
                                      _ptr(out_idx), _ptr(out_val), _ptr(out_logits),
                                      _ptr(dev_err), _ptr(ws), ws_bytes, _stream(stream)),
            "mtp_lm_head_argmax")
+
+
+def mtp_noalloc_scratch_bytes() -> int:
+    return load().mtp_noalloc_scratch_bytes()
+
+
+def mtp_lm_head_argmax_noalloc(head, n_eff, x, M, mask, mask_words, mask_stride_words, out_idx,
+                               out_val, out_logits, dev_err, stream=None):
+    _check(load().mtp_lm_head_argmax_noalloc(C.byref(head) if head is not None else None, n_eff,
+                                             _ptr(x), M, _ptr(mask), mask_words,
+                                             mask_stride_words, _ptr(out_idx), _ptr(out_val),
+                                             _ptr(out_logits), _ptr(dev_err), _stream(stream)),
+           "mtp_lm_head_argmax_noalloc")
 
 
 def mtp_debug_encode_e4m3(inp, n, out, stream=None):

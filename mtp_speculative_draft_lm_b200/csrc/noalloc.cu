@@ -1,0 +1,75 @@
+// mtp_lm_head_argmax_noalloc: the fused lm_head sweep + argmax without a caller
+// workspace, for callers that cannot allocate device memory.
+//
+// Some callers cannot call cudaMalloc at the point where they run a draft: a plugin
+// that lives inside another framework's memory pool and may not allocate behind its
+// back, an engine that reserves all free device memory for its KV cache at start-up
+// and treats any later allocation as an error, or code that must not risk the device
+// synchronisation that cudaMalloc/cudaFree can cause. They still pass their own
+// inputs and outputs; only the sweep's scratch (the CTA partials and the last-CTA
+// counter) comes from here.
+//
+// The scratch is the file-scope device array below: every GPU that loads this library
+// holds it (kScratchBytes) until the process exits, and every call on that GPU shares
+// it. In host code `g_sweep_scratch` names a host-side stand-in, not device memory, so
+// the kernel is given the address that cudaGetSymbolAddress returns for the current
+// device. That set-up runs on the first call made with each device current (it also
+// zeroes the counter once, with a synchronous cudaMemset); make that first call
+// before any stream capture. Afterwards each call leaves the counter at zero again.
+// Calls that overlap on the GPU (two streams, or two host threads) share the array
+// and race: serialise them. Nothing here allocates: no cudaMalloc, no cudaFree.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "../../include/mtp.h"
+#include "kernels.h"
+
+namespace {
+
+constexpr size_t kTicketBytes = 256;
+constexpr size_t kScratchBytes = kTicketBytes + 8 * 16 * 1024;  // counter + 1024 CTAs x 16 rows
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) uint8_t g_sweep_scratch[kScratchBytes];
+
+std::mutex g_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// The device address of g_sweep_scratch on the current device (set up once per device).
+mtp_status scratch_for_current_device(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MTP_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!g_scratch_ptr[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_sweep_scratch) != cudaSuccess || !ptr) return MTP_ERR_CUDA;
+        if (cudaMemset(ptr, 0, kTicketBytes) != cudaSuccess) return MTP_ERR_CUDA;
+        g_scratch_ptr[dev] = ptr;
+    }
+    *out = g_scratch_ptr[dev];
+    return MTP_OK;
+}
+
+}  // namespace
+
+extern "C" size_t mtp_noalloc_scratch_bytes(void) { return kScratchBytes; }
+
+extern "C" mtp_status mtp_lm_head_argmax_noalloc(const mtp_weight* head, int64_t n_eff,
+                                                 const uint16_t* x, int32_t M,
+                                                 const int32_t* mask, int64_t mask_words,
+                                                 int64_t mask_stride_words, int32_t* out_idx,
+                                                 float* out_val, uint16_t* out_logits,
+                                                 int32_t* dev_err, void* stream) {
+    if (head && mtp_lm_head_ws_bytes(head, n_eff, M) > kScratchBytes) return MTP_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    // argument checks first, so that a rejected call never triggers the set-up
+    mtp_status st = mtp_lm_head_argmax(head, n_eff, x, M, mask, mask_words, mask_stride_words,
+                                       out_idx, out_val, out_logits, dev_err, nullptr,
+                                       kScratchBytes, nullptr);
+    if (st != MTP_ERR_WORKSPACE) return st == MTP_OK ? MTP_ERR_CUDA : st;
+    if ((st = scratch_for_current_device(&scratch)) != MTP_OK) return st;
+    return mtp_lm_head_argmax(head, n_eff, x, M, mask, mask_words, mask_stride_words, out_idx,
+                              out_val, out_logits, dev_err, scratch, kScratchBytes, stream);
+}
