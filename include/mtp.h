@@ -188,6 +188,59 @@ mtp_status mtp_lm_head_argmax(const mtp_weight* head, int64_t n_eff, const uint1
                               size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------
+ * mtp_prefill_kv -- the drafter-context prefill: the drafter's K/V cache rows for R
+ * prompt rows, written as E4M3 codes into a paged cache.
+ * Source: [mtp_head.rs] drafter-prefill docs (the drafter's K/V for prompt row i are a
+ * pure function of (embed(token_{i+1}), target_hidden_i): fc + k/v projections + norms +
+ * RoPE + cache write, no attention) and MtpPrefillScratch (chunked rows, bf16 buffers);
+ * [new.rs] KV config (block size 16, FP8 cache with unit K/V scales); [v4_mtp.rs]
+ * forward_one step 4 (block = block_table[pos / bs], slot = block * bs + pos % bs).
+ * Per row r (all intermediate activations rounded to bf16):
+ *   c = [rms(embed[token_ids[r]]) w_norm_embed || rms(hidden[r]) w_norm_hidden]
+ *   y = fc . c;  k = wk . y;  v = wv . y;  k' = NeoX RoPE over each head of hd at
+ *   position rope_pos[r] (theta_j = pos * rope_base^(-2j/hd));
+ *   p = cache_start + r;  slot = block_table[p / block_size] * block_size + p % block_size
+ *   k_cache[(slot * nkv + head) * hd + d] = e4m3_satfinite(k'[head, d] / k_scale), same
+ *   for v with v_scale. A row whose block is missing (p / block_size >= n_table) or out of
+ *   range is not written and sets MTP_DEVFLAG_BAD_SLOT; a bad token id reads as a zero
+ *   embedding row and sets MTP_DEVFLAG_BAD_TOKEN.
+ *   embed (device) bf16 [vocab, h]; token_ids, rope_pos (device) i32 [R];
+ *   hidden (device) bf16 [R, h]; w_norm_* (device) bf16 [h]; fc (device) bf16 [h, 2h];
+ *   wk, wv (device) bf16 [nkv * hd, h]; block_table (device) i32 [n_table];
+ *   k_cache, v_cache (device) u8 [num_blocks, block_size, nkv, hd], written in place;
+ *   ws (device) >= mtp_prefill_ws_bytes(min(chunk_rows, R), h, nkv, hd) bytes, 1 KB
+ *   aligned (per chunk: the concat rows, fc output and a RoPE table).
+ * Rows run in chunks of chunk_rows (the GEMMs' M). Requires h % 256 == 0,
+ * hd in {64, 128, 256}, nkv * hd % 256 == 0, k_scale, v_scale > 0.
+ * ------------------------------------------------------------------------------ */
+size_t mtp_prefill_ws_bytes(int64_t chunk_rows, int32_t h, int32_t nkv, int32_t hd);
+mtp_status mtp_prefill_kv(const uint16_t* embed, int64_t vocab, const int32_t* token_ids,
+                          const uint16_t* hidden, int64_t R, int32_t h,
+                          const uint16_t* w_norm_embed, const uint16_t* w_norm_hidden, float eps,
+                          const uint16_t* fc, const uint16_t* wk, const uint16_t* wv, int32_t nkv,
+                          int32_t hd, float rope_base, const int32_t* rope_pos,
+                          int64_t cache_start, const int32_t* block_table, int64_t n_table,
+                          int32_t block_size, uint8_t* k_cache, uint8_t* v_cache,
+                          int64_t num_blocks, float k_scale, float v_scale, int64_t chunk_rows,
+                          void* ws, size_t ws_bytes, int32_t* dev_err, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * Stage checks of the prefill, each through the code the prefill itself runs:
+ * mtp_debug_gemm_bf16: C = bf16(A . B^T), A bf16 [M, K], B bf16 [N, K], C bf16 [M, N]
+ *   (the tcgen05 GEMM); requires N % 256 == 0, K % 64 == 0, 16-byte aligned pointers.
+ * mtp_debug_kv_write: already-rotated bf16 k'[R, nkv*hd] and v[R, nkv*hd] -> E4M3 codes
+ *   at the paged slots of cache rows cache_start + r (the GEMM epilogue's encode and
+ *   slot code).
+ * ------------------------------------------------------------------------------ */
+mtp_status mtp_debug_gemm_bf16(const uint16_t* A, const uint16_t* B, uint16_t* C, int32_t M,
+                               int32_t N, int32_t K, void* stream);
+mtp_status mtp_debug_kv_write(const uint16_t* k_rot, const uint16_t* v, int64_t R, int32_t nkv,
+                              int32_t hd, int64_t cache_start, const int32_t* block_table,
+                              int64_t n_table, int32_t block_size, int64_t num_blocks,
+                              uint8_t* k_cache, uint8_t* v_cache, float k_scale, float v_scale,
+                              int32_t* dev_err, void* stream);
+
+/* ---------------------------------------------------------------------------------
  * mtp_lm_head_argmax_noalloc -- mtp_lm_head_argmax without a workspace argument.
  * The pages have no counterpart: this entry point exists for callers that cannot
  * allocate device memory when they run a draft (a plugin inside another framework's

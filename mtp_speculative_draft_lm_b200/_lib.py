@@ -37,6 +37,7 @@ EXPORTS = (
     "mtp_combine", "mtp_lm_head_ws_bytes", "mtp_lm_head_argmax",
     "mtp_debug_encode_e4m3", "mtp_debug_encode_e2m1", "mtp_nvfp4_scale_pitch",
     "mtp_noalloc_scratch_bytes", "mtp_lm_head_argmax_noalloc",
+    "mtp_prefill_ws_bytes", "mtp_prefill_kv", "mtp_debug_gemm_bf16", "mtp_debug_kv_write",
 )
 
 
@@ -71,6 +72,13 @@ _SIGS = {
     "mtp_lm_head_ws_bytes": (_SZ, [_W, _I64, _I32]),
     "mtp_lm_head_argmax": (C.c_int, [_W, _I64, _P, _I32, _P, _I64, _I64, _P, _P, _P, _P,
                                      _P, _SZ, _P]),
+    "mtp_prefill_ws_bytes": (_SZ, [_I64, _I32, _I32, _I32]),
+    "mtp_prefill_kv": (C.c_int, [_P, _I64, _P, _P, _I64, _I32, _P, _P, C.c_float, _P, _P, _P,
+                                 _I32, _I32, C.c_float, _P, _I64, _P, _I64, _I32, _P, _P, _I64,
+                                 C.c_float, C.c_float, _I64, _P, _SZ, _P, _P]),
+    "mtp_debug_gemm_bf16": (C.c_int, [_P, _P, _P, _I32, _I32, _I32, _P]),
+    "mtp_debug_kv_write": (C.c_int, [_P, _P, _I64, _I32, _I32, _I64, _P, _I64, _I32, _I64, _P,
+                                     _P, C.c_float, C.c_float, _P, _P]),
     "mtp_noalloc_scratch_bytes": (_SZ, []),
     "mtp_lm_head_argmax_noalloc": (C.c_int, [_W, _I64, _P, _I32, _P, _I64, _I64, _P, _P, _P,
                                              _P, _P]),
@@ -175,6 +183,36 @@ def mtp_lm_head_argmax(head, n_eff, x, M, mask, mask_words, mask_stride_words, o
                                      _ptr(out_idx), _ptr(out_val), _ptr(out_logits),
                                      _ptr(dev_err), _ptr(ws), ws_bytes, _stream(stream)),
            "mtp_lm_head_argmax")
+
+
+def mtp_prefill_ws_bytes(chunk_rows, h, nkv, hd) -> int:
+    return load().mtp_prefill_ws_bytes(chunk_rows, h, nkv, hd)
+
+
+def mtp_prefill_kv(embed, vocab, token_ids, hidden, R, h, w_norm_embed, w_norm_hidden, eps, fc,
+                   wk, wv, nkv, hd, rope_base, rope_pos, cache_start, block_table, n_table,
+                   block_size, k_cache, v_cache, num_blocks, k_scale, v_scale, chunk_rows, ws,
+                   ws_bytes, dev_err=None, stream=None):
+    _check(load().mtp_prefill_kv(_ptr(embed), vocab, _ptr(token_ids), _ptr(hidden), R, h,
+                                 _ptr(w_norm_embed), _ptr(w_norm_hidden), float(eps), _ptr(fc),
+                                 _ptr(wk), _ptr(wv), nkv, hd, float(rope_base), _ptr(rope_pos),
+                                 cache_start, _ptr(block_table), n_table, block_size,
+                                 _ptr(k_cache), _ptr(v_cache), num_blocks, float(k_scale),
+                                 float(v_scale), chunk_rows, _ptr(ws), ws_bytes, _ptr(dev_err),
+                                 _stream(stream)), "mtp_prefill_kv")
+
+
+def mtp_debug_gemm_bf16(A, B, Cout, M, N, K, stream=None):
+    _check(load().mtp_debug_gemm_bf16(_ptr(A), _ptr(B), _ptr(Cout), M, N, K, _stream(stream)),
+           "mtp_debug_gemm_bf16")
+
+
+def mtp_debug_kv_write(k_rot, v, R, nkv, hd, cache_start, block_table, n_table, block_size,
+                       num_blocks, k_cache, v_cache, k_scale, v_scale, dev_err=None, stream=None):
+    _check(load().mtp_debug_kv_write(_ptr(k_rot), _ptr(v), R, nkv, hd, cache_start,
+                                     _ptr(block_table), n_table, block_size, num_blocks,
+                                     _ptr(k_cache), _ptr(v_cache), float(k_scale), float(v_scale),
+                                     _ptr(dev_err), _stream(stream)), "mtp_debug_kv_write")
 
 
 def mtp_noalloc_scratch_bytes() -> int:

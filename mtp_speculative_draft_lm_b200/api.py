@@ -108,3 +108,22 @@ def combine(embed, token_ids, hidden, w_norm_embed, w_norm_hidden, eps, fc: Tabl
     L.mtp_combine(embed, embed.shape[0], token_ids, hidden, M, h, w_norm_embed, w_norm_hidden,
                   eps, fc.desc, out, dev_err, stream)
     return out
+
+
+def prefill_kv(inputs: dict, k_cache: torch.Tensor, v_cache: torch.Tensor, chunk_rows: int = 2048,
+               ws: torch.Tensor | None = None, dev_err: torch.Tensor | None = None, stream=None):
+    """Drafter-context prefill over device tensors named as in synth.prefill_inputs."""
+    d = inputs
+    R, h = d["hidden"].shape
+    nkv, hd = int(d["nkv"]), int(d["hd"])
+    chunk = min(int(chunk_rows), R)
+    nbytes = L.mtp_prefill_ws_bytes(chunk, h, nkv, hd)
+    if ws is None:
+        ws = torch.empty((nbytes,), dtype=torch.uint8, device=k_cache.device)
+    L.mtp_prefill_kv(d["embed"], d["embed"].shape[0], d["tokens"], d["hidden"], R, h,
+                     d["w_norm_embed"], d["w_norm_hidden"], d["eps"], d["fc"], d["wk"], d["wv"],
+                     nkv, hd, d["rope_base"], d["rope_pos"], int(d["cache_start"]),
+                     d["block_table"], d["block_table"].numel(), int(d["block_size"]), k_cache,
+                     v_cache, k_cache.shape[0], d["k_scale"], d["v_scale"], chunk, ws, ws.numel(),
+                     dev_err, stream)
+    return ws

@@ -200,6 +200,98 @@ mtp_status mtp_lm_head_argmax(const mtp_weight* head, int64_t n_eff, const uint1
     return from_cuda(mtp::sweep_launch(p, head->fmt, 0, as_stream(stream), nullptr));
 }
 
+size_t mtp_prefill_ws_bytes(int64_t chunk_rows, int32_t h, int32_t nkv, int32_t hd) {
+    if (chunk_rows < 1 || h < 1 || nkv < 1 || hd < 2) return 0;
+    return mtp::prefill_ws_bytes(chunk_rows, h, nkv, hd);
+}
+
+static bool finite_pos(float v) { return v > 0.f && v < 3.0e38f; }
+
+mtp_status mtp_prefill_kv(const uint16_t* embed, int64_t vocab, const int32_t* token_ids,
+                          const uint16_t* hidden, int64_t R, int32_t h,
+                          const uint16_t* w_norm_embed, const uint16_t* w_norm_hidden, float eps,
+                          const uint16_t* fc, const uint16_t* wk, const uint16_t* wv, int32_t nkv,
+                          int32_t hd, float rope_base, const int32_t* rope_pos,
+                          int64_t cache_start, const int32_t* block_table, int64_t n_table,
+                          int32_t block_size, uint8_t* k_cache, uint8_t* v_cache,
+                          int64_t num_blocks, float k_scale, float v_scale, int64_t chunk_rows,
+                          void* ws, size_t ws_bytes, int32_t* dev_err, void* stream) {
+    if (!embed || !token_ids || !hidden || !w_norm_embed || !w_norm_hidden || !fc || !wk ||
+        !wv || !rope_pos || !block_table || !k_cache || !v_cache)
+        return MTP_ERR_INVALID_ARG;
+    if (vocab < 1 || R < 1 || h < 1 || nkv < 1 || hd < 2 || block_size < 1 || n_table < 1 ||
+        num_blocks < 1 || chunk_rows < 1 || !(eps >= 0.f) || !finite_pos(k_scale) ||
+        !finite_pos(v_scale) || !(rope_base > 0.f) || cache_start < 0)
+        return MTP_ERR_INVALID_ARG;
+    const int tn = mtp::gemm_tile_n();
+    if (h % tn || (hd != 64 && hd != 128 && hd != 256) || ((int64_t)nkv * hd) % tn ||
+        chunk_rows > (int64_t)1 << 30)
+        return MTP_ERR_UNSUPPORTED;
+    if (!aligned(embed, 16) || !aligned(hidden, 16) || !aligned(fc, 16) || !aligned(wk, 16) ||
+        !aligned(wv, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(w_norm_embed, 2) || !aligned(w_norm_hidden, 2) || !aligned(token_ids, 4) ||
+        !aligned(rope_pos, 4) || !aligned(block_table, 4) || !aligned(dev_err, 4))
+        return MTP_ERR_INVALID_ARG;
+    const int64_t chunk = chunk_rows < R ? chunk_rows : R;
+    if (!ws || !aligned(ws, 1024) || ws_bytes < mtp::prefill_ws_bytes(chunk, h, nkv, hd))
+        return MTP_ERR_WORKSPACE;
+    mtp::PrefillArgs a{};
+    a.embed = embed;
+    a.vocab = vocab;
+    a.tokens = token_ids;
+    a.hidden = hidden;
+    a.R = R;
+    a.h = h;
+    a.w_norm_embed = w_norm_embed;
+    a.w_norm_hidden = w_norm_hidden;
+    a.eps = eps;
+    a.fc = fc;
+    a.wk = wk;
+    a.wv = wv;
+    a.nkv = nkv;
+    a.hd = hd;
+    a.rope_base = (double)rope_base;
+    a.rope_pos = rope_pos;
+    a.cache_start = cache_start;
+    a.block_table = block_table;
+    a.n_table = n_table;
+    a.block_size = block_size;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.num_blocks = num_blocks;
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
+    a.chunk_rows = chunk;
+    a.ws = ws;
+    a.dev_err = dev_err;
+    return from_cuda(mtp::prefill_launch(a, as_stream(stream)));
+}
+
+mtp_status mtp_debug_gemm_bf16(const uint16_t* A, const uint16_t* B, uint16_t* C, int32_t M,
+                               int32_t N, int32_t K, void* stream) {
+    if (!A || !B || !C || M < 1 || N < 1 || K < 1) return MTP_ERR_INVALID_ARG;
+    if (N % mtp::gemm_tile_n() || K % mtp::gemm_tile_k()) return MTP_ERR_UNSUPPORTED;
+    if (!aligned(A, 16) || !aligned(B, 16) || !aligned(C, 16)) return MTP_ERR_INVALID_ARG;
+    return from_cuda(mtp::gemm_bf16_launch(A, B, C, M, N, K, nullptr, as_stream(stream)));
+}
+
+mtp_status mtp_debug_kv_write(const uint16_t* k_rot, const uint16_t* v, int64_t R, int32_t nkv,
+                              int32_t hd, int64_t cache_start, const int32_t* block_table,
+                              int64_t n_table, int32_t block_size, int64_t num_blocks,
+                              uint8_t* k_cache, uint8_t* v_cache, float k_scale, float v_scale,
+                              int32_t* dev_err, void* stream) {
+    if (!k_rot || !v || !block_table || !k_cache || !v_cache || R < 1 || nkv < 1 || hd < 32 ||
+        hd % 32 || block_size < 1 || n_table < 1 || num_blocks < 1 || cache_start < 0 ||
+        !finite_pos(k_scale) || !finite_pos(v_scale))
+        return MTP_ERR_INVALID_ARG;
+    if (!aligned(k_rot, 16) || !aligned(v, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(block_table, 4) || !aligned(dev_err, 4))
+        return MTP_ERR_INVALID_ARG;
+    return from_cuda(mtp::kv_write_launch(k_rot, v, R, nkv, hd, cache_start, block_table, n_table,
+                                          block_size, num_blocks, k_cache, v_cache, k_scale,
+                                          v_scale, dev_err, as_stream(stream)));
+}
+
 mtp_status mtp_debug_encode_e4m3(const float* in, int64_t n, uint8_t* out, void* stream) {
     if (!in || !out || n < 1 || !aligned(in, 4)) return MTP_ERR_INVALID_ARG;
     return from_cuda(mtp::debug_encode_launch(in, n, out, 0, as_stream(stream)));

@@ -72,6 +72,46 @@ cudaError_t quant_nvfp4_launch(const uint16_t* w, int64_t n, int64_t k, uint8_t*
 int quant_nvfp4_max_grid();
 int64_t nvfp4_scale_pitch(int64_t k);
 
+// Drafter-context prefill (prefill.cu).
+struct PrefillArgs {
+    const uint16_t* embed;
+    int64_t vocab;
+    const int32_t* tokens;
+    const uint16_t* hidden;
+    int64_t R;
+    int32_t h;
+    const uint16_t* w_norm_embed;
+    const uint16_t* w_norm_hidden;
+    float eps;
+    const uint16_t* fc;
+    const uint16_t* wk;
+    const uint16_t* wv;
+    int32_t nkv, hd;
+    double rope_base;
+    const int32_t* rope_pos;
+    int64_t cache_start;
+    const int32_t* block_table;
+    int64_t n_table;
+    int32_t block_size;
+    uint8_t* k_cache;
+    uint8_t* v_cache;
+    int64_t num_blocks;
+    float k_scale, v_scale;
+    int64_t chunk_rows;
+    void* ws;
+    int32_t* dev_err;
+};
+size_t prefill_ws_bytes(int64_t chunk_rows, int32_t h, int32_t nkv, int32_t hd);
+cudaError_t prefill_launch(const PrefillArgs& a, cudaStream_t s);
+cudaError_t gemm_bf16_launch(const uint16_t* A, const uint16_t* B, uint16_t* C, int M, int N,
+                             int K, int32_t* dev_err, cudaStream_t s);
+cudaError_t kv_write_launch(const uint16_t* k_rot, const uint16_t* v, int64_t R, int nkv, int hd,
+                            int64_t cache_start, const int32_t* block_table, int64_t n_table,
+                            int block_size, int64_t num_blocks, uint8_t* k_cache, uint8_t* v_cache,
+                            float k_scale, float v_scale, int32_t* dev_err, cudaStream_t s);
+int gemm_tile_n();
+int gemm_tile_k();
+
 // Encoders exposed for exhaustive checks.
 cudaError_t debug_encode_launch(const float* in, int64_t n, uint8_t* out, int which,
                                 cudaStream_t s);

@@ -150,3 +150,39 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(L, "_lib", None)
     with pytest.raises(OSError):
         L.load(str(tmp_path / "none.so"))
+
+
+def prefill_args(**kw):
+    a = dict(embed=A, vocab=100, tok=B2, hidden=A, R=10, h=256, wne=OUT, wnh=OUT, eps=1e-6,
+             fc=A, wk=A, wv=A, nkv=2, hd=128, base=1e6, pos=B2, start=0, table=B2, n_table=4,
+             bs=16, kc=OUT, vc=OUT, nb=4, ks=1.0, vs=1.0, chunk=8, ws=0x100000, wsb=None,
+             err=None)
+    a.update(kw)
+    if a["wsb"] is None:
+        a["wsb"] = L.mtp_prefill_ws_bytes(min(a["chunk"], a["R"]), a["h"], a["nkv"], a["hd"])
+    return [a[k] for k in ("embed", "vocab", "tok", "hidden", "R", "h", "wne", "wnh", "eps",
+                           "fc", "wk", "wv", "nkv", "hd", "base", "pos", "start", "table",
+                           "n_table", "bs", "kc", "vc", "nb", "ks", "vs", "chunk", "ws", "wsb",
+                           "err")] + [None]
+
+
+def test_prefill_rejects(lib):
+    assert L.mtp_prefill_ws_bytes(2048, 5120, 8, 128) >= 2048 * 5120 * 6
+    assert st("mtp_prefill_kv", *prefill_args(embed=None)) == L.MTP_ERR_INVALID_ARG
+    assert st("mtp_prefill_kv", *prefill_args(R=0)) == L.MTP_ERR_INVALID_ARG
+    assert st("mtp_prefill_kv", *prefill_args(ks=0.0)) == L.MTP_ERR_INVALID_ARG
+    assert st("mtp_prefill_kv", *prefill_args(h=320)) == L.MTP_ERR_UNSUPPORTED   # h % 256
+    assert st("mtp_prefill_kv", *prefill_args(hd=96)) == L.MTP_ERR_UNSUPPORTED
+    assert st("mtp_prefill_kv", *prefill_args(nkv=1)) == L.MTP_ERR_UNSUPPORTED  # nkv*hd % 256
+    assert st("mtp_prefill_kv", *prefill_args(hidden=A + 8)) == L.MTP_ERR_INVALID_ARG
+    assert st("mtp_prefill_kv", *prefill_args(ws=None)) == L.MTP_ERR_WORKSPACE
+    assert st("mtp_prefill_kv", *prefill_args(ws=0x100000 + 512)) == L.MTP_ERR_WORKSPACE
+    assert st("mtp_prefill_kv", *prefill_args(wsb=1024)) == L.MTP_ERR_WORKSPACE
+
+
+def test_gemm_and_kv_stage_reject(lib):
+    assert st("mtp_debug_gemm_bf16", A, B2, OUT, 128, 100, 64, None) == L.MTP_ERR_UNSUPPORTED
+    assert st("mtp_debug_gemm_bf16", A, B2, OUT, 128, 256, 48, None) == L.MTP_ERR_UNSUPPORTED
+    assert st("mtp_debug_gemm_bf16", None, B2, OUT, 128, 256, 64, None) == L.MTP_ERR_INVALID_ARG
+    assert st("mtp_debug_kv_write", A, B2, 10, 2, 100, 0, B2, 4, 16, 4, OUT, OUT, 1.0, 1.0,
+              None, None) == L.MTP_ERR_INVALID_ARG  # hd % 32

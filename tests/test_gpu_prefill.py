@@ -1,0 +1,189 @@
+"""The drafter-context prefill on the GPU against the oracle.
+
+Stage by stage: the tcgen05 GEMM (one-hot rows select B rows exactly; random operands
+within 2e-2 + 1e-2|ref|), the E4M3 encode + paged scatter given the same bf16 k'/v
+(bit-exact codes and slots, every other cache byte untouched), then the whole prefill
+on a small multi-chunk prompt (every row) and on the benchmark prompt (32,768 rows,
+hidden 5,120, chunks of 2,048; sampled rows spread over all chunks).
+
+End to end the codes are not bit-exact by construction: the GPU accumulates the two
+projections in fp32 and the oracle in fp64, so bf16(y) and bf16(k) can differ by an
+ulp, which the RoPE rotation and the E4M3 rounding can expose. The criterion is the
+activation tolerance carried through: RoPE rotates each pair (k_j, k_{j+hd/2}) without
+changing its norm, so a k' value may differ from the oracle's by 2e-2 + 1e-2 x the pair
+norm, plus one E4M3 step of the final rounding (where the rotation nearly cancels, a
+tiny k' inherits the absolute error of inputs near the pair norm); a v value by
+2e-2 + 1e-2 |v| plus one step. At least 98% of codes are identical; slots are exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+from helpers import assert_close, bf16_bits_to_f64, to_dev, to_dev_u16, u16_of
+from mtp_speculative_draft_lm_b200 import _lib as L
+from mtp_speculative_draft_lm_b200 import api, synth
+
+pytestmark = pytest.mark.gpu
+
+SENTINEL = 0x7F  # E4M3 NaN: never produced by a saturating encode
+
+
+def gemm(A, B):
+    M, K = A.shape
+    N = B.shape[0]
+    C = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    L.mtp_debug_gemm_bf16(to_dev_u16(A), to_dev_u16(B), C, M, N, K)
+    torch.cuda.synchronize()
+    return u16_of(C)
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (300, 512, 640), (1000, 1024, 4096)])
+def test_gemm_matches_numpy(orc, M, N, K):
+    A = synth.as_u16(synth.normal_bf16(synth._gen(M + N), (M, K), 1.0))
+    B = synth.as_u16(synth.normal_bf16(synth._gen(K + 3), (N, K), 0.02))
+    C = gemm(A, B)
+    ref = orc.bf16_to_f64(A) @ orc.bf16_to_f64(B).T
+    assert_close(bf16_bits_to_f64(C), ref, "C")
+
+
+def test_gemm_one_hot_rows_are_exact(orc):
+    M, N, K = 256, 512, 1024
+    B = synth.as_u16(synth.normal_bf16(synth._gen(5), (N, K), 1.0))
+    A = np.zeros((M, K), np.uint16)
+    cols = (np.arange(M) * 37) % K
+    A[np.arange(M), cols] = 0x3F80  # 1.0
+    C = gemm(A, B)
+    assert np.array_equal(C, B[:, cols].T)
+
+
+def kv_ordinal(c):
+    c = np.asarray(c, np.int32)
+    return np.where(c & 0x80, -(c & 0x7F), c & 0x7F)
+
+
+def new_caches(num_blocks, bs, nkv, hd):
+    k = torch.full((num_blocks, bs, nkv, hd), SENTINEL, dtype=torch.uint8, device="cuda")
+    v = torch.full((num_blocks, bs, nkv, hd), SENTINEL, dtype=torch.uint8, device="cuda")
+    return k, v
+
+
+def test_kv_write_stage_bit_exact(orc):
+    R, nkv, hd, bs = 200, 2, 128, 16
+    nb = R // bs + 3
+    table = torch.randperm(nb, generator=synth._gen(4)).to(torch.int32)
+    k_rot = synth.as_u16(synth.normal_bf16(synth._gen(6), (R, nkv * hd), 2.0))
+    v = synth.as_u16(synth.normal_bf16(synth._gen(7), (R, nkv * hd), 2.0))
+    for start, ks, vs in ((0, 1.0, 1.0), (5, 0.5, 2.0)):
+        kc, vc = new_caches(nb, bs, nkv, hd)
+        err = torch.zeros((1,), dtype=torch.int32, device="cuda")
+        L.mtp_debug_kv_write(to_dev_u16(k_rot), to_dev_u16(v), R, nkv, hd, start,
+                             table.cuda(), nb, bs, nb, kc, vc, ks, vs, err)
+        torch.cuda.synchronize()
+        kc = kc.cpu().numpy().reshape(-1, nkv * hd)
+        vc = vc.cpu().numpy().reshape(-1, nkv * hd)
+        written = np.zeros(kc.shape[0], bool)
+        for r in range(R):
+            slot = orc.slot(table.numpy(), bs, nb, start + r)
+            if slot < 0:
+                continue
+            written[slot] = True
+            assert np.array_equal(kc[slot], orc.kv_encode(k_rot[r], ks)), r
+            assert np.array_equal(vc[slot], orc.kv_encode(v[r], vs)), r
+        assert np.all(kc[~written] == SENTINEL) and np.all(vc[~written] == SENTINEL)
+        expect_bad = any(orc.slot(table.numpy(), bs, nb, start + r) < 0 for r in range(R))
+        assert bool(err.item() & L.MTP_DEVFLAG_BAD_SLOT) == expect_bad
+
+
+def run_prefill(d, chunk, extra_blocks_cache=0):
+    dev = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    nb = int(d["num_blocks"]) + extra_blocks_cache
+    kc, vc = new_caches(nb, d["block_size"], d["nkv"], d["hd"])
+    err = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    api.prefill_kv(dev, kc, vc, chunk_rows=chunk, dev_err=err)
+    torch.cuda.synchronize()
+    return kc.cpu().numpy(), vc.cpu().numpy(), int(err.item())
+
+
+def oracle_rows(orc, d, rows):
+    U = {k: (synth.as_u16(v) if isinstance(v, torch.Tensor) and v.dtype == torch.bfloat16 else
+             (v.numpy() if isinstance(v, torch.Tensor) else v)) for k, v in d.items()}
+    return orc.prefill_rows(U["embed"], U["tokens"], U["hidden"], U["w_norm_embed"],
+                            U["w_norm_hidden"], U["eps"], U["fc"], U["wk"], U["wv"], d["nkv"],
+                            d["hd"], d["rope_base"], U["rope_pos"], d["cache_start"],
+                            U["block_table"], d["block_size"], d["num_blocks"], d["k_scale"],
+                            d["v_scale"], rows)
+
+
+def e4m3_step(v):
+    """Spacing of E4M3 values at |v| (2^-9 below the smallest normal)."""
+    a = np.abs(np.asarray(v, np.float64))
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -6)))
+    return np.where(a < 2.0 ** -6, 2.0 ** -9, 2.0 ** (e - 3))
+
+
+def check_rows(orc, d, kc, vc, rows, min_exact=0.98):
+    ref = oracle_rows(orc, d, rows)
+    nkv, hd = d["nkv"], d["hd"]
+    kc = kc.reshape(-1, nkv * hd)
+    vc = vc.reshape(-1, nkv * hd)
+    exact = total = 0
+    for i, r in enumerate(rows):
+        slot = ref["slot"][i]
+        assert slot >= 0
+        kr = bf16_bits_to_f64(ref["k_rot"][i]).reshape(nkv, 2, hd // 2)
+        pair = np.sqrt((kr ** 2).sum(axis=1, keepdims=True))
+        k_scale = np.broadcast_to(pair, kr.shape).reshape(-1) / d["k_scale"]
+        v_scale = np.abs(bf16_bits_to_f64(ref["v"][i])) / d["v_scale"]
+        for got, want, sc in ((kc[slot], ref["k_codes"][i], k_scale),
+                              (vc[slot], ref["v_codes"][i], v_scale)):
+            gv, wv = orc.e4m3_value(got), orc.e4m3_value(want)
+            lim = np.maximum(e4m3_step(gv), e4m3_step(wv)) + 2e-2 + 1e-2 * sc
+            bad = np.abs(gv - wv) > lim
+            assert not bad.any(), (r, np.nonzero(bad)[0][:5], got[bad][:5], want[bad][:5])
+            exact += int((got == want).sum())
+            total += got.size
+    assert exact / total >= min_exact, exact / total
+
+
+def test_prefill_small_multi_chunk(orc):
+    d = synth.prefill_inputs(seed=77, R=300, vocab=500, h=256, nkv=2, hd=128)
+    kc, vc, err = run_prefill(d, chunk=128)
+    assert err == 0
+    check_rows(orc, d, kc, vc, np.arange(300))
+    # every cache row that no prompt row maps to keeps the sentinel
+    slots = {orc.slot(d["block_table"].numpy(), 16, d["num_blocks"], r) for r in range(300)}
+    flat = kc.reshape(-1, 256)
+    untouched = [s for s in range(flat.shape[0]) if s not in slots]
+    assert np.all(flat[untouched] == SENTINEL)
+
+
+def test_prefill_other_heads_and_positions(orc):
+    d = synth.prefill_inputs(seed=78, R=70, vocab=300, h=512, nkv=4, hd=64)
+    d["rope_pos"] = torch.arange(1000, 1070, dtype=torch.int32)
+    d["cache_start"] = 5
+    d["num_blocks"] = int(d["num_blocks"]) + 1
+    d["block_table"] = torch.randperm(d["num_blocks"], generator=synth._gen(3)).to(torch.int32)
+    kc, vc, err = run_prefill(d, chunk=64)
+    assert err == 0
+    check_rows(orc, d, kc, vc, np.arange(70))
+
+
+def test_prefill_bad_slot_and_token_flags(orc):
+    d = synth.prefill_inputs(seed=79, R=40, vocab=100, h=256, nkv=2, hd=128)
+    d["tokens"] = d["tokens"].clone()
+    d["tokens"][3] = 1000
+    d["block_table"] = d["block_table"][:2].clone()  # rows 32.. have no block
+    kc, vc, err = run_prefill(d, chunk=64)
+    assert err & L.MTP_DEVFLAG_BAD_SLOT and err & L.MTP_DEVFLAG_BAD_TOKEN
+    check_rows(orc, d, kc, vc, np.arange(32))
+
+
+def test_prefill_full_prompt_sampled_rows(orc):
+    d = synth.prefill_inputs()
+    kc, vc, err = run_prefill(d, chunk=synth.PREFILL["chunk"])
+    assert err == 0
+    rng = np.random.default_rng(5)
+    rows = np.unique(np.concatenate([
+        [0, 1, 2047, 2048, 32767],
+        rng.choice(d["R"], 59, replace=False)]))
+    check_rows(orc, d, kc, vc, rows)
