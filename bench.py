@@ -32,13 +32,19 @@ FALLBACK_HBM_GBS = 6650.0
 
 # DRAM traffic per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum) and
 # the sha256 of sweep.cu when it was captured; reported as null once the source changed.
-NCU_TRAFFIC = {}
+# bf16_M1: the 40,000-row capture (profiles/sweep_kernel_bf16_40k_rows.md) read
+# 327,776,000 B and wrote 3,560,192 B; reads scale with the rows swept, so a full
+# 154,880-row launch reads 327,776,000 x 154,880 / 40,000 B (writes kept unscaled).
+NCU_TRAFFIC = {"bf16_M1": (1272708864, "ddf3fbe92253daf5")}
 
 
 def sweep_source_hash() -> str:
     p = os.path.join(ROOT, "mtp_speculative_draft_lm_b200", "csrc", "sweep.cu")
     with open(p, "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+FALLBACK_TFLOPS_SUSTAINED = 1400.0
 
 
 def measured_peaks():
@@ -48,6 +54,15 @@ def measured_peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_tflops():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d.get("bf16_tflops_sustained", d.get("bf16_tflops"))), "measured"
+    return FALLBACK_TFLOPS_SUSTAINED, "fallback"
 
 
 class ClockSampler:
@@ -157,17 +172,34 @@ def build_table(fmt: str, dev, rows: int = 0):
     if fmt == "bf16":
         table = api.bf16_table(w)
     else:
+        from mtp_speculative_draft_lm_b200 import _lib as L
+
+        table = api.quantize_fp8(w) if fmt == "fp8" else api.quantize_nvfp4(w)
+        n, k = w.shape
+        if fmt == "fp8":
+            def quant():
+                L.mtp_quantize_fp8(w, n, k, table.data, table.row_scale)
+        else:
+            ws = torch.zeros((L.mtp_quantize_nvfp4_ws_bytes(n, k),), dtype=torch.uint8, device=dev)
+
+            def quant():
+                L.mtp_quantize_nvfp4(w, n, k, table.data, table.block_scale, table.global_scale,
+                                     ws, ws.numel())
+        quant()
         torch.cuda.synchronize()
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 5
         s.record()
-        table = api.quantize_fp8(w) if fmt == "fp8" else api.quantize_nvfp4(w)
+        for _ in range(reps):
+            quant()
         e.record()
         torch.cuda.synchronize()
-        ms = s.elapsed_time(e)
+        ms = s.elapsed_time(e) / reps
         rd = w.numel() * 2
         wr = table.nbytes()
+        # NVFP4 reads the table twice (global absmax pass, then the encode pass)
         qinfo = {"ms": ms, "GB/s": (rd * (2 if fmt == "nvfp4" else 1) + wr) / ms / 1e6,
-                 "note": "includes first-call setup" }
+                 "bytes": rd * (2 if fmt == "nvfp4" else 1) + wr}
         del w
     return cfg, d, table, qinfo
 
@@ -236,6 +268,68 @@ def time_e2e(head, x_host, steps, warmup, world, stream):
     torch.cuda.synchronize()
     barrier(world)
     return t0.elapsed_time(t1) / steps, M * K * 2, M * 8, idx_h.numpy().copy()
+
+
+def bench_tiny_draft(dev, steps, warmup):
+    """The tiny draft step (hidden 256, vocab 4096): combiner + lm_head sweep + argmax,
+    M = 1; everything is L2-resident, so this is latency (reported warm)."""
+    import torch
+
+    from mtp_speculative_draft_lm_b200 import api, synth
+
+    d = synth.tiny_draft(M=1)
+    dd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    fc = api.bf16_table(dd["fc"])
+    head = api.LmHead(api.bf16_table(dd["lm_head"]))
+    y = torch.empty((1, d["h"]), dtype=torch.bfloat16, device=dev)
+    idx = torch.empty((1,), dtype=torch.int32, device=dev)
+
+    def step():
+        api.combine(dd["embed"], dd["tokens"], dd["hidden"], dd["w_norm_embed"],
+                    dd["w_norm_hidden"], d["eps"], fc, out=y)
+        head(y, idx)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    return {"us_per_draft": s.elapsed_time(e) / steps * 1e3, "launches_per_draft": 2,
+            "note": "hidden 256, vocab 4096, M=1, warm (L2-resident)"}
+
+
+def bench_prefill(dev, reps, tflops_peak, peak_src, rows=0):
+    """Drafter-context prefill: 32,768 prompt rows, hidden 5,120, chunks of 2,048."""
+    import torch
+
+    from mtp_speculative_draft_lm_b200 import api, synth
+
+    d = synth.prefill_inputs(R=rows, vocab=4096) if rows else synth.prefill_inputs()
+    dd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    kc = torch.zeros((d["num_blocks"], d["block_size"], d["nkv"], d["hd"]), dtype=torch.uint8,
+                     device=dev)
+    vc = torch.zeros_like(kc)
+    ws = api.prefill_kv(dd, kc, vc, chunk_rows=synth.PREFILL["chunk"])
+    for _ in range(2):
+        api.prefill_kv(dd, kc, vc, chunk_rows=synth.PREFILL["chunk"], ws=ws)
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(reps):
+        api.prefill_kv(dd, kc, vc, chunk_rows=synth.PREFILL["chunk"], ws=ws)
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / reps
+    R, h, kvd = d["R"], d["h"], d["nkv"] * d["hd"]
+    flops = 2.0 * R * (2 * h) * h + 2.0 * R * h * (2 * kvd)
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"ms": ms, "TFLOP/s": tf, "frac_of_peak": tf / tflops_peak,
+            "peak_source": f"{peak_src} bf16_tflops_sustained", "flops": flops,
+            "rows": R, "hidden": h, "chunk": synth.PREFILL["chunk"]}
 
 
 def cpu_baseline(fmt_table, d, cfg, budget_s=12.0):
@@ -322,6 +416,11 @@ def main():
     ap.add_argument("--formats", default="bf16,fp8,nvfp4")
     ap.add_argument("--rows", type=int, default=0,
                     help="sweep a smaller table of this many rows (profiling cases)")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the tiny-draft and prefill rows")
+    ap.add_argument("--only", default="", help="profiling: run only 'prefill' or 'tiny'")
+    ap.add_argument("--prefill-rows", type=int, default=0,
+                    help="profiling: prefill prompt rows (default: the 32,768-row workload)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     if args.impl == "reference":
@@ -336,6 +435,14 @@ def main():
     dev = torch.device("cuda", local)
     stream = torch.cuda.Stream(device=dev)
     peak, peak_src = measured_peaks()
+    if args.only:
+        tpk, tsrc = measured_tflops()
+        if args.only == "prefill":
+            out = bench_prefill(dev, 2, tpk, tsrc, args.prefill_rows)
+        else:
+            out = bench_tiny_draft(dev, args.steps, args.warmup)
+        print(json.dumps({"only": args.only, **out}), flush=True)
+        return 0
     rows = {}
     main_line = None
     cpu_base = None
@@ -398,6 +505,12 @@ def main():
         if fmt == "bf16" and rank == 0 and world == 1 and not args.no_cpu:
             cpu_base = cpu_baseline(table, d, cfg)
         del head, table, d
+        torch.cuda.empty_cache()
+
+    if world == 1 and not args.no_extra and not args.rows:
+        rows["tiny_draft_M1"] = bench_tiny_draft(dev, max(200, args.steps // 10), args.warmup)
+        tpk, tsrc = measured_tflops()
+        rows["prefill_32k"] = bench_prefill(dev, 5, tpk, tsrc)
         torch.cuda.empty_cache()
 
     if rank == 0 and main_line is not None:
