@@ -48,7 +48,7 @@ namespace {
 constexpr int kTileRows = 16;
 constexpr int kMaxGrid = 1024;
 constexpr int kMaxStages = 12;
-constexpr int kMaxSegs = 16;  // 128-byte segments of a row per stage (box of 16 rows x 2 KB)
+constexpr int kMaxSegs = 32;  // 128-byte segments of a row per stage (box of 16 rows x 4 KB)
 constexpr int kSmemLimit = 227 * 1024;
 
 // Warp roles: CW compute warps, then one reducer warp, then one producer warp.
@@ -378,7 +378,7 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
                     mbar_arrive_expect_tx(&full[slot], tx);
                     tma_load_3d(dst, &map_codes, 0, (int)(tile * kTileRows), ch * segs, &full[slot]);
                     if (FMT == 2)
-                        tma_load_2d(dst + code_stage_bytes(segs), &map_scales, ch * 16 * segs,
+                        tma_load_2d(dst + code_stage_bytes(segs), &map_scales, ch * 8 * segs,
                                     (int)(tile * kTileRows), &full[slot]);
                 }
                 __syncwarp();
@@ -637,9 +637,9 @@ Geometry geometry(int M, int64_t k, int fmt) {
     const int64_t row_bytes = fmt == 0 ? k * 2 : fmt == 1 ? k : k / 2;
     const int row_segs = (int)(row_bytes / 128);
     const long avail = (long)kSmemLimit - (long)head;
-    // the widest stage (up to 16 segments) that still leaves a ring of >= 4 stages,
+    // the widest stage (up to 32 segments) that still leaves a ring of >= 3 stages,
     // else >= 2; segments are spread evenly over the stages of a row
-    for (int want = 4; want >= 2 && g.stages < 2; want /= 2) {
+    for (int want = 3; want >= 2 && g.stages < 2; --want) {
         for (int max_segs = kMaxSegs; max_segs >= 1; max_segs /= 2) {
             const int nc = (row_segs + max_segs - 1) / max_segs;
             const int segs = (row_segs + nc - 1) / nc;
@@ -695,16 +695,17 @@ cudaError_t make_code_map(CUtensorMap* m, const void* base, int64_t rows, int64_
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// NVFP4 block scales: [rows, pitch] bytes, boxes of 16 * segs bytes x 16 rows.
+// NVFP4 block scales: [rows, pitch] bytes viewed as 16-bit elements, boxes of
+// 16 * segs bytes x 16 rows (up to 512 bytes per row: two scale bytes per element).
 cudaError_t make_scale_map(CUtensorMap* m, const void* base, int64_t rows, int64_t pitch,
                            int segs) {
     EncodeTiledFn fn = encode_tiled();
     if (!fn) return cudaErrorNotSupported;
-    cuuint64_t dims[2] = {(cuuint64_t)pitch, (cuuint64_t)rows};
+    cuuint64_t dims[2] = {(cuuint64_t)(pitch / 2), (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)pitch};
-    cuuint32_t box[2] = {(cuuint32_t)(16 * segs), kTileRows};
+    cuuint32_t box[2] = {(cuuint32_t)(8 * segs), kTileRows};
     cuuint32_t es[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides,
                     box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
