@@ -182,20 +182,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Like mbar_try_wait, but the thread may sleep in hardware for up to `ns` nanoseconds
+// waiting for the phase (no issue slots spent spinning).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
 // About one second at the B200's clock: a wait this long means the pipeline is broken.
 constexpr long long kWaitLimitCycles = 2000000000LL;
 
-// Waits for `bar` to complete the phase with `parity`. Gives up after
-// kWaitLimitCycles -- or at once when *abort is already set -- sets *abort and
-// returns false; the caller then runs on without the data so that every thread
-// still reaches the end of the kernel. With abort == nullptr only the time limit
+// Waits for `bar` to complete the phase with `parity`, sleeping in hardware between
+// checks. Gives up after kWaitLimitCycles -- or at once when *abort is already set --
+// sets *abort and returns false; the caller then runs on without the data so that every
+// thread still reaches the end of the kernel. With abort == nullptr only the time limit
 // applies (used to drain copies in flight at exit).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   volatile int* abort) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity, 2000u)) return true;
         if (abort && *abort) return false;
         if (clock64() - t0 > kWaitLimitCycles) {
             if (abort) *abort = 1;

@@ -225,17 +225,18 @@ __device__ void stage_to_f16(const SweepParams& p, uint16_t* xs, int* xexp, floa
     }
 }
 
-// One slab (4 lanes x 16 B of rows r0 and r0 + 8, K elements [e0, e0 + V) for lane c)
-// into the MMA accumulators; accumulator set (mma index & 1) alternates to split the
-// dependence chain.
+// One slab: per lane 16 B of codes of table rows r0 (at cw) and r0 + 8 (at cw + 1 KB,
+// the next 8-row swizzle atom), K elements [e0, e0 + V) for lane c, against the staged
+// inputs at x0 (input row g) and x1 (input row g + 8). For NVFP4, sw points at the
+// lane's two block scales of row r0 and sw + spitch8 at those of row r0 + 8. The
+// accumulator set (mma index & 1) alternates to split the dependence chain.
 template <int FMT, int NT>
-__device__ __forceinline__ void slab_mma(float (&acc)[2][NT][4], const uint8_t* st, int sl,
-                                         int r0, int c, const uint16_t* x0, const uint16_t* x1,
-                                         bool l0, bool l1, int segs) {
-    const uint32_t b = (uint32_t)(sl * 64 + c * 16);  // logical byte in the row chunk
-    const uint32_t la = (b >> 7) * 2048u + (uint32_t)r0 * 128u + (b & 127u);
-    const uint4 ra = lds128(st + swz(la));
-    const uint4 rb = lds128(st + swz(la + 8u * 128u));
+__device__ __forceinline__ void slab_mma(float (&acc)[2][NT][4], const uint8_t* cw,
+                                         const uint8_t* sw, uint32_t spitch8,
+                                         const uint16_t* x0, const uint16_t* x1, bool l0,
+                                         bool l1) {
+    const uint4 ra = lds128(cw);
+    const uint4 rb = lds128(cw + 1024);
     const uint4 z = make_uint4(0, 0, 0, 0);
     if (FMT == 0) {
         const uint4 xa = l0 ? lds128(x0) : z;
@@ -271,13 +272,9 @@ __device__ __forceinline__ void slab_mma(float (&acc)[2][NT][4], const uint8_t* 
     } else {
         const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w};
         const uint32_t wb[4] = {rb.x, rb.y, rb.z, rb.w};
-        // block scales of rows r0 / r0+8: blocks 2c (words 0,1) and 2c+1 (words 2,3);
-        // the stage's scales are [16 rows][16 * segs bytes], unswizzled
-        const uint8_t* sp = st + code_stage_bytes(segs);
-        const uint32_t spitch = 16u * (uint32_t)segs;
-        const uint32_t sbyte = (uint32_t)(sl * 8 + 2 * c);
-        const uint16_t s0v = *reinterpret_cast<const uint16_t*>(sp + (uint32_t)r0 * spitch + sbyte);
-        const uint16_t s1v = *reinterpret_cast<const uint16_t*>(sp + (uint32_t)(r0 + 8) * spitch + sbyte);
+        // block scales of rows r0 / r0+8: blocks 2c (words 0,1) and 2c+1 (words 2,3)
+        const uint16_t s0v = *reinterpret_cast<const uint16_t*>(sw);
+        const uint16_t s1v = *reinterpret_cast<const uint16_t*>(sw + spitch8);
         const uint32_t sa = e4m3x2_to_f16x2(s0v);
         const uint32_t sb = e4m3x2_to_f16x2(s1v);
         const uint32_t sa_lo = __byte_perm(sa, 0, 0x1010), sa_hi = __byte_perm(sa, 0, 0x3232);
@@ -397,20 +394,33 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
 
     // ------------------------------------------------------------ reducer warp
     if (warp == REDUCER) {
-        // lane holds items (row = lane & 15, col = 2q + (lane >> 4)) for q < RED_COLS/2
+        // lane holds items (row = lane & 15, col = 2q + (lane >> 4)) for q < RED_COLS/2 and
+        // keeps, per item, the running (max, lowest row) over the CTA's tiles; the 16 lanes
+        // of a column are folded once, after the last tile
         constexpr int Q = RED_COLS / 2;
         float best_v[Q];
         int32_t best_i[Q];
+        float fa[Q], fb[Q];  // 2^-xexp as two factors: (a fa) fb is exact for a normal result
 #pragma unroll
         for (int q = 0; q < Q; ++q) {
             best_v[q] = -INFINITY;
             best_i[q] = INT_MAX;
+            fa[q] = fb[q] = 1.f;
         }
         const int rrow = lane & 15;
+        const float gsc = FMT == 2 ? __ldg(p.global_scale) : 1.f;
+        bool have_f = FMT == 0;
+        // row scales of the next tile are loaded one tile ahead
+        float rs_next = 0.f;
+        if (FMT == 1 && t_begin < t_end && t_begin * kTileRows + rrow < p.n)
+            rs_next = __ldg(p.row_scale + t_begin * kTileRows + rrow);
         int buf = 0;
         uint32_t fph = 0u;  // bit b: phase parity of red_full[b]
         for (int64_t tile = t_begin; tile < t_end; ++tile) {
             const int64_t row = tile * kTileRows + rrow;
+            const float rs = rs_next;
+            if (FMT == 1 && tile + 1 < t_end && row + kTileRows < p.n)
+                rs_next = __ldg(p.row_scale + row + kTileRows);
             if (!tile_needed(p, tile, lane)) {
                 // every row is masked out for every input: logits -inf, nothing to fold
                 if (MODE == 0 && p.out_logits && row < p.n)
@@ -420,6 +430,16 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
             }
             mbar_wait_bounded(&red_full[buf], (fph >> buf) & 1u, abort_flag);
             fph ^= 1u << buf;
+            if (!have_f) {  // xexp is visible once the first partials have arrived
+#pragma unroll
+                for (int q = 0; q < Q; ++q) {
+                    const int col = 2 * q + (lane >> 4);
+                    const int e = col < M ? -xexp[col] : 0;
+                    fa[q] = ldexpf(1.f, e / 2);
+                    fb[q] = ldexpf(1.f, e - e / 2);
+                }
+                have_f = true;
+            }
             const float* rb = red + (size_t)buf * CW * RED_WARP_FLOATS;
 #pragma unroll
             for (int q = 0; q < Q; ++q) {
@@ -437,29 +457,19 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
                 }
                 const bool valid = row < p.n && col < M;
                 float l = a;
-                if (FMT != 0 && valid) l = ldexpf(a, -xexp[col]);
-                if (FMT == 1 && valid) l *= __ldg(p.row_scale + row);
-                if (FMT == 2 && valid) l *= __ldg(p.global_scale);
+                if (FMT != 0) l = (l * fa[q]) * fb[q];
+                if (FMT == 1) l *= rs;
+                if (FMT == 2) l *= gsc;
                 if (MODE == 1) {
                     if (valid) p.out_y[(int64_t)col * p.n + row] = f32_to_bf16(l);
                 } else {
                     const bool ok = valid && mask_allows(p, col, row);
                     if (valid && p.out_logits)
                         p.out_logits[(int64_t)col * p.n + row] = ok ? f32_to_bf16(l) : (uint16_t)0xFF80u;
-                    float v = ok ? l : -INFINITY;
-                    int32_t i = ok ? (int32_t)row : INT_MAX;
-#pragma unroll
-                    for (int o = 8; o; o >>= 1) {
-                        const float ov = __shfl_xor_sync(0xffffffffu, v, o);
-                        const int32_t oi = __shfl_xor_sync(0xffffffffu, i, o);
-                        if (ov > v || (ov == v && oi < i)) {
-                            v = ov;
-                            i = oi;
-                        }
-                    }
-                    if (v > best_v[q] || (v == best_v[q] && i < best_i[q])) {
-                        best_v[q] = v;
-                        best_i[q] = i;
+                    // rows arrive in increasing order, so the lowest row wins a tie
+                    if (ok && (l > best_v[q] || (l == best_v[q] && best_i[q] == INT_MAX))) {
+                        best_v[q] = l;
+                        best_i[q] = (int32_t)row;
                     }
                 }
             }
@@ -470,6 +480,19 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
         if (*abort_flag) raise_flag(p.dev_err, DEVFLAG_TIMEOUT);
         if (MODE == 1) return;
 
+        // fold the 16 row slots of each column (lanes sharing lane >> 4)
+#pragma unroll
+        for (int q = 0; q < Q; ++q) {
+#pragma unroll
+            for (int o = 8; o; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, best_v[q], o);
+                const int32_t oi = __shfl_xor_sync(0xffffffffu, best_i[q], o);
+                if (ov > best_v[q] || (ov == best_v[q] && oi < best_i[q])) {
+                    best_v[q] = ov;
+                    best_i[q] = oi;
+                }
+            }
+        }
         Partial* parts = reinterpret_cast<Partial*>(p.partials);
 #pragma unroll
         for (int q = 0; q < Q; ++q) {
@@ -544,6 +567,19 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
     const bool xg1 = NT > 1 && (8 + g) < M;
     const int r0 = tile_row(g);  // table rows r0 and r0 + 8 of the tile feed MMA rows g, g+8
 
+    // Per-lane offsets inside a stage. Slab l of a stage is 64 bytes of each row: segment
+    // l / 2 (a 2 KB block of 16 rows x 128 B), half l % 2. With the 128-byte swizzle the
+    // lane's 16-byte chunk of row r0 sits at r0 * 128 + ((64 (l % 2) + 16 c) ^ 16 (r0 % 8));
+    // row r0 + 8 is 1 KB further on. Block scales: [16 rows][16 segs bytes], unswizzled.
+    const uint32_t xr = (uint32_t)(r0 & 7) << 4;
+    const uint32_t coff0 = (uint32_t)r0 * 128u + (((uint32_t)c * 16u) ^ xr);
+    const uint32_t coff1 = (uint32_t)r0 * 128u + ((64u + (uint32_t)c * 16u) ^ xr);
+    const uint32_t spitch = 16u * (uint32_t)segs;
+    const uint32_t soff = (uint32_t)code_stage_bytes(segs) + (uint32_t)r0 * spitch + 2u * (uint32_t)c;
+    const uint16_t* xrow0 = xs + g * p.kpad + c * V;
+    const uint16_t* xrow1 = xs + (8 + g) * p.kpad + c * V;
+    const int total_slabs = (int)(K / SLAB);  // K is a whole number of slabs
+
     // Accumulation chains follow the absolute slab index a (64-byte column block of
     // the row): chain a % 16 takes slabs in increasing a. With 16 compute warps warp w
     // owns chain w; with 8, warp w owns chains w and w + 8. The same chains, summed
@@ -570,19 +606,17 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
             mbar_wait_bounded(&full[slot], phase, abort_flag);
             const uint8_t* st = ring + (size_t)slot * stage_bytes;
             const int a0 = ch * slabs_per_stage;  // absolute slab index of the stage's first slab
-            // this warp's slabs in the stage: a = a0 + l with a % CW == warp
-            for (int l = (warp - a0 % CW + CW) % CW; l < slabs_per_stage; l += CW) {
-                const int a = a0 + l;
-                const int64_t s0 = (int64_t)a * SLAB;
-                if (s0 >= K) break;  // warp-uniform: past the end of K
-                const int64_t e0 = s0 + c * V;
-                const bool kin = e0 < K;  // beyond K the stage holds zeros
-                const uint16_t* x0 = xs + (int64_t)g * p.kpad + e0;
-                const uint16_t* x1 = xs + (int64_t)(8 + g) * p.kpad + e0;
-                if (CH == 2 && ((a >> 3) & 1))
-                    slab_mma<FMT, NT>(acc[CH - 1], st, l, r0, c, x0, x1, xg0 && kin, xg1 && kin, segs);
+            const int nv = min(slabs_per_stage, total_slabs - a0);  // slabs inside the row
+            // this warp's slabs in the stage: l = a - a0 with a % CW == warp
+            int l = (warp - a0) & (CW - 1);
+            const uint8_t* cw = st + (l >> 1) * 2048 + ((l & 1) ? coff1 : coff0);
+            const uint8_t* sw = st + soff + l * 8;
+            int xo = (a0 + l) * SLAB;
+            for (; l < nv; l += CW, cw += CW * 1024, sw += CW * 8, xo += CW * SLAB) {
+                if (CH == 2 && (((a0 + l) >> 3) & 1))
+                    slab_mma<FMT, NT>(acc[CH - 1], cw, sw, 8u * spitch, xrow0 + xo, xrow1 + xo, xg0, xg1);
                 else
-                    slab_mma<FMT, NT>(acc[0], st, l, r0, c, x0, x1, xg0 && kin, xg1 && kin, segs);
+                    slab_mma<FMT, NT>(acc[0], cw, sw, 8u * spitch, xrow0 + xo, xrow1 + xo, xg0, xg1);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[slot]);
