@@ -303,7 +303,48 @@ __device__ __forceinline__ void slab_mma(float (&acc)[2][NT][4], const uint8_t* 
     }
 }
 
-template <int FMT, int NT, int MODE>
+// NVFP4 with one or two inputs: the block scale moves out of the fragments. An MMA's
+// k = 16 covers four elements of each lane group c, and lane group c's elements in
+// MMAs 0-3 of the slab all belong to block 2c of the slab, in MMAs 4-7 to block 2c + 1.
+// B is block-diagonal over the lane groups: column 4m + j holds input m on the k of
+// lane group j and zero elsewhere, so D0 (MMAs 0-3) and D1 (MMAs 4-7) hold, per row,
+// the unscaled E2M1 x input dot products of each block separately (products exact,
+// fp32 sums). The lane holding D columns 2c + e (e = 0, 1; lane group j = 2(c % 2) + e)
+// then adds s(block 2j) D0 + s(block 2j + 1) D1 for rows r0 and r0 + 8 in fp32: eight
+// FFMAs per slab instead of 32 f16 scale multiplies. sw4 points at the row-r0 scale
+// bytes of blocks 4(c % 2) .. 4(c % 2) + 3 of the slab, sw4 + spitch8 at row r0 + 8's.
+__device__ __forceinline__ void slab_mma_blocks(float (&acc)[4], const uint8_t* cw,
+                                                const uint8_t* sw4, uint32_t spitch8,
+                                                const uint16_t* xp, bool lx) {
+    const uint4 ra = lds128(cw);
+    const uint4 rb = lds128(cw + 1024);
+    const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w};
+    const uint32_t wb[4] = {rb.x, rb.y, rb.z, rb.w};
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t qa[4], qb[4];
+        e2m1x8_to_f16x2x4(wa[i], qa);
+        e2m1x8_to_f16x2x4(wb[i], qb);
+        const uint4 xv = lx ? lds128(xp + 8 * i) : z;
+        float(&d)[4] = i < 2 ? d0 : d1;
+        mma_f16_16816(d, qa[0], qb[0], qa[1], qb[1], xv.x, xv.y);
+        mma_f16_16816(d, qa[2], qb[2], qa[3], qb[3], xv.z, xv.w);
+    }
+    const uint32_t sa = *reinterpret_cast<const uint32_t*>(sw4);
+    const uint32_t sb = *reinterpret_cast<const uint32_t*>(sw4 + spitch8);
+    const float2 a01 = f16x2_to_f32x2(e4m3x2_to_f16x2((uint16_t)(sa & 0xFFFFu)));
+    const float2 a23 = f16x2_to_f32x2(e4m3x2_to_f16x2((uint16_t)(sa >> 16)));
+    const float2 b01 = f16x2_to_f32x2(e4m3x2_to_f16x2((uint16_t)(sb & 0xFFFFu)));
+    const float2 b23 = f16x2_to_f32x2(e4m3x2_to_f16x2((uint16_t)(sb >> 16)));
+    acc[0] = fmaf(a01.y, d1[0], fmaf(a01.x, d0[0], acc[0]));
+    acc[1] = fmaf(a23.y, d1[1], fmaf(a23.x, d0[1], acc[1]));
+    acc[2] = fmaf(b01.y, d1[2], fmaf(b01.x, d0[2], acc[2]));
+    acc[3] = fmaf(b23.y, d1[3], fmaf(b23.x, d0[3], acc[3]));
+}
+
+template <int FMT, int NT, int MODE, int BD>
 __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
     sweep_kernel(const __grid_constant__ SweepParams p, const __grid_constant__ CUtensorMap map_codes,
                  const __grid_constant__ CUtensorMap map_scales) {
@@ -579,6 +620,12 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
     const uint16_t* xrow0 = xs + g * p.kpad + c * V;
     const uint16_t* xrow1 = xs + (8 + g) * p.kpad + c * V;
     const int total_slabs = (int)(K / SLAB);  // K is a whole number of slabs
+    // per-block scaling (NVFP4, M <= 2): lane (g, c) feeds B column g, which is input
+    // g / 4 on lane group g % 4, so only lanes with g % 4 == c load an input
+    const bool xbd = (g & 3) == c && (g >> 2) < M;
+    const uint16_t* xrowb = xs + (g >> 2) * p.kpad + c * V;
+    const uint32_t soffb = (uint32_t)code_stage_bytes(segs) + (uint32_t)r0 * spitch + 4u * (uint32_t)(c & 1);
+    float accb[4] = {0.f, 0.f, 0.f, 0.f};
 
     // Accumulation chains follow the absolute slab index a (64-byte column block of
     // the row): chain a % 16 takes slabs in increasing a. With 16 compute warps warp w
@@ -612,11 +659,17 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
             const uint8_t* cw = st + (l >> 1) * 2048 + ((l & 1) ? coff1 : coff0);
             const uint8_t* sw = st + soff + l * 8;
             int xo = (a0 + l) * SLAB;
-            for (; l < nv; l += CW, cw += CW * 1024, sw += CW * 8, xo += CW * SLAB) {
-                if (CH == 2 && (((a0 + l) >> 3) & 1))
-                    slab_mma<FMT, NT>(acc[CH - 1], cw, sw, 8u * spitch, xrow0 + xo, xrow1 + xo, xg0, xg1);
-                else
-                    slab_mma<FMT, NT>(acc[0], cw, sw, 8u * spitch, xrow0 + xo, xrow1 + xo, xg0, xg1);
+            if (BD) {
+                const uint8_t* swb = st + soffb + l * 8;
+                for (; l < nv; l += CW, cw += CW * 1024, swb += CW * 8, xo += CW * SLAB)
+                    slab_mma_blocks(accb, cw, swb, 8u * spitch, xrowb + xo, xbd);
+            } else {
+                for (; l < nv; l += CW, cw += CW * 1024, sw += CW * 8, xo += CW * SLAB) {
+                    if (CH == 2 && (((a0 + l) >> 3) & 1))
+                        slab_mma<FMT, NT>(acc[CH - 1], cw, sw, 8u * spitch, xrow0 + xo, xrow1 + xo, xg0, xg1);
+                    else
+                        slab_mma<FMT, NT>(acc[0], cw, sw, 8u * spitch, xrow0 + xo, xrow1 + xo, xg0, xg1);
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[slot]);
@@ -632,8 +685,20 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
         mbar_wait_bounded(&red_empty[buf], ((eph >> buf) & 1u) ^ 1u, abort_flag);
         eph ^= 1u << buf;
         float* rp = red + (size_t)buf * CW * RED_WARP_FLOATS + warp * RED_WARP_FLOATS;
+        if (BD) {
+            // input m's logit part: lane groups 0, 1 (lane c = 2m) plus 2, 3 (lane 2m + 1)
+            const float v0 = accb[0] + accb[1], v1 = accb[2] + accb[3];
+            const float u0 = __shfl_xor_sync(0xffffffffu, v0, 1);
+            const float u1 = __shfl_xor_sync(0xffffffffu, v1, 1);
+            if ((c & 1) == 0) {
+                rp[r0 * RED_COLS + (c >> 1)] = v0 + u0;
+                rp[(r0 + 8) * RED_COLS + (c >> 1)] = v1 + u1;
+            }
 #pragma unroll
-        for (int t = 0; t < NT; ++t) {
+            for (int i = 0; i < 4; ++i) accb[i] = 0.f;
+        }
+#pragma unroll
+        for (int t = 0; t < (BD ? 0 : NT); ++t) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 float v = acc[0][0][t][i] + acc[0][1][t][i];
@@ -745,9 +810,9 @@ cudaError_t make_scale_map(CUtensorMap* m, const void* base, int64_t rows, int64
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int FMT, int NT, int MODE>
+template <int FMT, int NT, int MODE, int BD>
 cudaError_t launch_one(const SweepParams& p, cudaStream_t s, SweepLaunch* info) {
-    auto kern = sweep_kernel<FMT, NT, MODE>;
+    auto kern = sweep_kernel<FMT, NT, MODE, BD>;
     const Geometry geo = geometry(p.M, p.k, FMT);
     if (geo.stages < 2) return cudaErrorInvalidValue;
     CUtensorMap map_codes, map_scales;
@@ -798,8 +863,9 @@ int sweep_max_grid() { return kMaxGrid; }
 cudaError_t sweep_launch(const SweepParams& p, int fmt, int mode, cudaStream_t s,
                          SweepLaunch* info) {
     const bool two = p.M > 8;
+    if (fmt == 2 && mode == 0 && p.M <= 2) return launch_one<2, 1, 0, 1>(p, s, info);
 #define MTP_SWEEP_CASE(F, NTV, MD) \
-    if (fmt == F && (NTV == 2) == two && mode == MD) return launch_one<F, NTV, MD>(p, s, info);
+    if (fmt == F && (NTV == 2) == two && mode == MD) return launch_one<F, NTV, MD, 0>(p, s, info);
     MTP_SWEEP_CASE(0, 1, 0) MTP_SWEEP_CASE(0, 2, 0)
     MTP_SWEEP_CASE(1, 1, 0) MTP_SWEEP_CASE(1, 2, 0)
     MTP_SWEEP_CASE(2, 1, 0) MTP_SWEEP_CASE(2, 2, 0)
