@@ -108,6 +108,25 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
         : "memory");
 }
 
+// Pulls this CTA's 1/gridDim share of [base, base + bytes) into L2 (bulk prefetches of
+// whole 16-byte units inside the range; the ragged ends are left to demand loads).
+__device__ __forceinline__ void l2_prefetch_share(const void* base, int64_t bytes) {
+    uint64_t g;
+    asm("cvta.to.global.u64 %0, %1;" : "=l"(g) : "l"(base));
+    const uint64_t lo = (g + 15u) & ~(uint64_t)15u;
+    const uint64_t hi = (g + (uint64_t)bytes) & ~(uint64_t)15u;
+    if (bytes <= 0 || hi <= lo) return;
+    const uint64_t per = ((hi - lo) / gridDim.x + 16u) & ~(uint64_t)15u;
+    uint64_t a = lo + per * blockIdx.x;
+    const uint64_t e = a + per < hi ? a + per : hi;
+    while (a < e) {
+        const uint64_t piece = e - a < 65536u ? e - a : 65536u;
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a), "r"((uint32_t)piece)
+                     : "memory");
+        a += piece;
+    }
+}
+
 __device__ __forceinline__ bool mask_allows(const SweepParams& p, int m, int64_t row) {
     if (!p.mask) return true;
     int64_t word = row >> 5;
@@ -219,8 +238,10 @@ __device__ void stage_to_f16(const SweepParams& p, uint16_t* xs, int* xexp, floa
         if (a > 0.f) frexpf(a, &ex);
         int e = (a > 0.f) ? 15 - ex : 0;
         if (tid == 0) xexp[m] = e;
-        for (int j = tid; j < K; j += NTH)
-            row[j] = f32_to_f16(ldexpf(bf16_to_f32(row[j]), e));
+        // 2^e as two factors, each a normal float: the product is exact whenever the
+        // result is a normal float, and a result below that is zero in f16 anyway
+        const float f1 = ldexpf(1.f, e / 2), f2 = ldexpf(1.f, e - e / 2);
+        for (int j = tid; j < K; j += NTH) row[j] = f32_to_f16((bf16_to_f32(row[j]) * f1) * f2);
         named_sync(1, NTH);
     }
 }
@@ -360,9 +381,13 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
     uint64_t* empty = full + kMaxStages;
     uint64_t* red_full = empty + kMaxStages;  // [2]
     uint64_t* red_empty = red_full + 2;       // [2]
-    int* misc = reinterpret_cast<int*>(red_empty + 2);  // [0] abort [2..17] xexp
+    // misc: [0] abort, [2..17] xexp, [18..29] tile of each ring slot, [30..31] tile of
+    // each reducer buffer (-1: no more tiles)
+    int* misc = reinterpret_cast<int*>(red_empty + 2);
     volatile int* abort_flag = misc;
     int* xexp = misc + 2;
+    volatile int* slot_tile = misc + 18;
+    volatile int* red_tile = misc + 30;
     float* red = reinterpret_cast<float*>(misc + 32);  // [2][CW][16][RED_COLS]
     float* scratch = red + 2 * CW * RED_WARP_FLOATS;   // [32]
     uint16_t* xs = reinterpret_cast<uint16_t*>(scratch + 32);
@@ -379,9 +404,14 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
     const int NC = p.stages_per_tile;          // ceil(row segments / segs)
     const int M = p.M;
 
+    // Tiles are handed out at run time (mode 0): CTA b starts with tile b, then takes
+    // gridDim.x + (a counter in the workspace, post-incremented), so SMs that stream
+    // faster take more tiles. Mode 1 (no workspace) splits the tiles evenly up front.
     const int64_t T = p.num_tiles;
-    const int64_t t_begin = (T * blockIdx.x) / gridDim.x;
-    const int64_t t_end = (T * (blockIdx.x + 1)) / gridDim.x;
+    const bool dyn = MODE == 0;
+    const int64_t t_begin = dyn ? blockIdx.x : (T * blockIdx.x) / gridDim.x;
+    const int64_t t_end = dyn ? T : (T * (blockIdx.x + 1)) / gridDim.x;
+    static_assert(kMaxStages <= 12, "slot_tile holds 12 entries");
 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
@@ -404,32 +434,58 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
         int64_t issued = 0;
         const uint32_t tx = code_stage_bytes(segs) + (FMT == 2 ? scale_stage_bytes(segs) : 0);
         bool stop = false;
-        for (int64_t tile = t_begin; tile < t_end && !stop; ++tile) {
-            if (!tile_needed(p, tile, lane)) continue;
-            for (int ch = 0; ch < NC; ++ch) {
-                if (!mbar_wait_bounded(&empty[slot], phase ^ 1u, abort_flag)) {
-                    stop = true;
-                    break;
+        int64_t tile = t_begin;
+        // the next tile is claimed one tile ahead, so the atomic's latency overlaps the
+        // waits for free ring slots
+        int64_t next = 0;
+        if (dyn && lane == 0 && tile < t_end) next = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
+        while (tile < t_end && !stop) {
+            if (tile_needed(p, tile, lane)) {
+                for (int ch = 0; ch < NC; ++ch) {
+                    if (!mbar_wait_bounded(&empty[slot], phase ^ 1u, abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    if (lane == 0) {
+                        uint8_t* dst = ring + (size_t)slot * stage_bytes;
+                        slot_tile[slot] = (int)tile;
+                        mbar_arrive_expect_tx(&full[slot], tx);
+                        tma_load_3d(dst, &map_codes, 0, (int)(tile * kTileRows), ch * segs, &full[slot]);
+                        if (FMT == 2)
+                            tma_load_2d(dst + code_stage_bytes(segs), &map_scales, ch * 8 * segs,
+                                        (int)(tile * kTileRows), &full[slot]);
+                    }
+                    __syncwarp();
+                    ++issued;
+                    if (++slot == S) {
+                        slot = 0;
+                        phase ^= 1u;
+                    }
                 }
-                if (lane == 0) {
-                    uint8_t* dst = ring + (size_t)slot * stage_bytes;
-                    mbar_arrive_expect_tx(&full[slot], tx);
-                    tma_load_3d(dst, &map_codes, 0, (int)(tile * kTileRows), ch * segs, &full[slot]);
-                    if (FMT == 2)
-                        tma_load_2d(dst + code_stage_bytes(segs), &map_scales, ch * 8 * segs,
-                                    (int)(tile * kTileRows), &full[slot]);
-                }
-                __syncwarp();
-                ++issued;
-                if (++slot == S) {
-                    slot = 0;
-                    phase ^= 1u;
-                }
+            } else if (MODE == 0 && p.out_logits) {
+                // every row is masked out for every input: logits -inf, nothing to load
+                const int64_t row = tile * kTileRows + (lane & 15);
+                if (row < p.n)
+                    for (int col = lane >> 4; col < M; col += 2)
+                        p.out_logits[(int64_t)col * p.n + row] = 0xFF80u;
+            }
+            if (dyn) {
+                tile = __shfl_sync(0xffffffffu, next, 0);
+                if (lane == 0 && tile < t_end) next = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
+            } else {
+                ++tile;
             }
         }
-        // leave no copy in flight: wait for the last stages issued (bounded)
+        // Leave no copy in flight: wait for the last stages issued (bounded). This comes
+        // before the end marker, which advances the phase of a slot these waits name.
         for (int64_t j = issued > S ? issued - S : 0; j < issued; ++j)
             if (!mbar_wait_bounded(&full[j % S], (uint32_t)((j / S) & 1), nullptr)) break;
+        // end of the CTA's tiles: a stage tagged -1 (an arrival with no copy)
+        if (!stop && mbar_wait_bounded(&empty[slot], phase ^ 1u, abort_flag) && lane == 0) {
+            slot_tile[slot] = -1;
+            mbar_arrive(&full[slot]);
+        }
+        __syncwarp();
         return;
     }
 
@@ -451,26 +507,22 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
         const int rrow = lane & 15;
         const float gsc = FMT == 2 ? __ldg(p.global_scale) : 1.f;
         bool have_f = FMT == 0;
-        // row scales of the next tile are loaded one tile ahead
-        float rs_next = 0.f;
-        if (FMT == 1 && t_begin < t_end && t_begin * kTileRows + rrow < p.n)
-            rs_next = __ldg(p.row_scale + t_begin * kTileRows + rrow);
+        // The row scales and the mask words are read per tile in an order known only at
+        // run time: each CTA first pulls its share of them into L2.
+        if (lane == 0) {
+            if (FMT == 1) l2_prefetch_share(p.row_scale, p.n * 4);
+            if (MODE == 0 && p.mask) l2_prefetch_share(p.mask, ((p.M - 1) * p.mask_stride + p.mask_words) * 4);
+        }
         int buf = 0;
         uint32_t fph = 0u;  // bit b: phase parity of red_full[b]
-        for (int64_t tile = t_begin; tile < t_end; ++tile) {
-            const int64_t row = tile * kTileRows + rrow;
-            const float rs = rs_next;
-            if (FMT == 1 && tile + 1 < t_end && row + kTileRows < p.n)
-                rs_next = __ldg(p.row_scale + row + kTileRows);
-            if (!tile_needed(p, tile, lane)) {
-                // every row is masked out for every input: logits -inf, nothing to fold
-                if (MODE == 0 && p.out_logits && row < p.n)
-                    for (int col = lane >> 4; col < M; col += 2)
-                        p.out_logits[(int64_t)col * p.n + row] = 0xFF80u;
-                continue;
-            }
-            mbar_wait_bounded(&red_full[buf], (fph >> buf) & 1u, abort_flag);
+        while (true) {
+            if (!mbar_wait_bounded(&red_full[buf], (fph >> buf) & 1u, abort_flag)) break;
             fph ^= 1u << buf;
+            const int tile_id = red_tile[buf];
+            if (tile_id < 0) break;
+            const int64_t tile = tile_id;
+            const int64_t row = tile * kTileRows + rrow;
+            const float rs = (FMT == 1 && row < p.n) ? __ldg(p.row_scale + row) : 0.f;
             if (!have_f) {  // xexp is visible once the first partials have arrived
 #pragma unroll
                 for (int q = 0; q < Q; ++q) {
@@ -595,7 +647,10 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
             }
         }
         __syncwarp();
-        if (lane == 0) *p.ticket = 0u;  // leave the workspace ready for the next call
+        if (lane == 0) {  // leave the workspace ready for the next call
+            p.ticket[0] = 0u;
+            p.ticket[1] = 0u;
+        }
         return;
     }
 
@@ -647,10 +702,13 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
     int slot = 0;
     uint32_t phase = 0;
 
-    for (int64_t tile = t_begin; tile < t_end; ++tile) {
-        if (!tile_needed(p, tile, lane)) continue;  // warp-uniform, same rule as the producer
+    while (true) {
+        // the stages of one tile arrive in order; a stage tagged -1 ends the CTA's work
+        if (!mbar_wait_bounded(&full[slot], phase, abort_flag)) break;
+        const int tile = slot_tile[slot];
+        if (tile < 0) break;
         for (int ch = 0; ch < NC; ++ch) {
-            mbar_wait_bounded(&full[slot], phase, abort_flag);
+            if (ch > 0 && !mbar_wait_bounded(&full[slot], phase, abort_flag)) break;
             const uint8_t* st = ring + (size_t)slot * stage_bytes;
             const int a0 = ch * slabs_per_stage;  // absolute slab index of the stage's first slab
             const int nv = min(slabs_per_stage, total_slabs - a0);  // slabs inside the row
@@ -709,9 +767,16 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
                 for (int j = 0; j < CH; ++j) acc[j][0][t][i] = acc[j][1][t][i] = 0.f;
             }
         }
+        if (warp == 0 && lane == 0) red_tile[buf] = tile;
         __syncwarp();
         if (lane == 0) mbar_arrive(&red_full[buf]);
         buf ^= 1;
+    }
+    // tell the reducer there are no more tiles
+    if (mbar_wait_bounded(&red_empty[buf], ((eph >> buf) & 1u) ^ 1u, abort_flag)) {
+        if (warp == 0 && lane == 0) red_tile[buf] = -1;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&red_full[buf]);
     }
 }
 
