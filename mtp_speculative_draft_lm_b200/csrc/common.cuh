@@ -146,6 +146,19 @@ __device__ __forceinline__ uint4 lds128(const void* p) {
     return *reinterpret_cast<const uint4*>(p);
 }
 
+// Release/acquire fence at GPU scope (orders this thread's memory accesses around a
+// relaxed atomic used as a flag).
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
+// Programmatic dependent launch: let the next kernel in the stream start its prologue
+// (it still waits for this grid before reading anything this grid may write), and wait
+// for the previous grid to complete with its writes visible. Both are no-ops when the
+// launch carries no programmatic-serialization attribute.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Device error word bits (a copy of the public MTP_DEVFLAG_* values).
 enum : int32_t { DEVFLAG_BAD_TOKEN = 1, DEVFLAG_EMPTY_MASK = 2, DEVFLAG_BAD_SLOT = 4,
                  DEVFLAG_TIMEOUT = 8 };

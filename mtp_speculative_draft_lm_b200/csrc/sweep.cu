@@ -246,6 +246,70 @@ __device__ void stage_to_f16(const SweepParams& p, uint16_t* xs, int* xexp, floa
     }
 }
 
+// Quantized tables with one or two inputs, mode 0: x read once from global memory into
+// registers (up to 4 x 8 elements per thread per input), one block-wide max per input,
+// then written to shared memory directly as f16 scaled by 2^e_m (the same scaling as
+// stage_bf16 + stage_to_f16). Returns false (nothing done) when K is too long for it.
+template <int CW>
+__device__ bool stage_x_f16_direct(const SweepParams& p, uint16_t* xs, int* xexp, float* part) {
+    constexpr int NTH = CW * 32, MAXV = 4;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int K = (int)p.k, vecs = K / 8, M = p.M;
+    if (M > 2 || vecs > MAXV * NTH) return false;
+    uint4 r[2][MAXV];
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+        float a = 0.f;
+#pragma unroll
+        for (int j = 0; j < MAXV; ++j) {
+            const int i = tid + j * NTH;
+            r[m][j] = make_uint4(0, 0, 0, 0);
+            if (m < M && i < vecs) {
+                r[m][j] = *reinterpret_cast<const uint4*>(p.x + (int64_t)m * K + (int64_t)i * 8);
+                const uint32_t w[4] = {r[m][j].x, r[m][j].y, r[m][j].z, r[m][j].w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    a = fmaxf(a, fabsf(bf16_to_f32((uint16_t)(w[q] & 0xFFFFu))));
+                    a = fmaxf(a, fabsf(bf16_to_f32((uint16_t)(w[q] >> 16))));
+                }
+            }
+        }
+        for (int o = 16; o; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+        if (lane == 0) part[m * CW + warp] = a;
+    }
+    named_sync(1, NTH);
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+        if (m >= M) break;
+        float a = 0.f;
+#pragma unroll
+        for (int w = 0; w < CW; ++w) a = fmaxf(a, part[m * CW + w]);
+        int ex = 0;
+        if (a > 0.f) frexpf(a, &ex);
+        const int e = (a > 0.f) ? 15 - ex : 0;
+        if (tid == 0) xexp[m] = e;
+        const float f1 = ldexpf(1.f, e / 2), f2 = ldexpf(1.f, e - e / 2);
+        uint16_t* row = xs + (int64_t)m * p.kpad;
+#pragma unroll
+        for (int j = 0; j < MAXV; ++j) {
+            const int i = tid + j * NTH;
+            if (i < vecs) {
+                const uint32_t w[4] = {r[m][j].x, r[m][j].y, r[m][j].z, r[m][j].w};
+                uint32_t o[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t lo = f32_to_f16((bf16_to_f32((uint16_t)(w[q] & 0xFFFFu)) * f1) * f2);
+                    const uint32_t hi = f32_to_f16((bf16_to_f32((uint16_t)(w[q] >> 16)) * f1) * f2);
+                    o[q] = lo | (hi << 16);
+                }
+                *reinterpret_cast<uint4*>(row + (int64_t)i * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+        }
+    }
+    named_sync(1, NTH);
+    return true;
+}
+
 // One slab: per lane 16 B of codes of table rows r0 (at cw) and r0 + 8 (at cw + 1 KB,
 // the next 8-row swizzle atom), K elements [e0, e0 + V) for lane c, against the staged
 // inputs at x0 (input row g) and x1 (input row g + 8). For NVFP4, sw points at the
@@ -426,6 +490,7 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
         mbar_fence_init();
     }
     __syncthreads();
+    pdl_launch_dependents();
 
     // ------------------------------------------------------------ producer warp
     if (warp == PRODUCER) {
@@ -437,8 +502,11 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
         int64_t tile = t_begin;
         // the next tile is claimed one tile ahead, so the atomic's latency overlaps the
         // waits for free ring slots
+        // The first tile's stages read only the table, so they go out before waiting for
+        // the previous grid (unless a mask, which that grid may write, decides them).
         int64_t next = 0;
-        if (dyn && lane == 0 && tile < t_end) next = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
+        bool waited = p.mask != nullptr;
+        if (waited) pdl_wait();
         while (tile < t_end && !stop) {
             if (tile_needed(p, tile, lane)) {
                 for (int ch = 0; ch < NC; ++ch) {
@@ -469,7 +537,12 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
                     for (int col = lane >> 4; col < M; col += 2)
                         p.out_logits[(int64_t)col * p.n + row] = 0xFF80u;
             }
+            if (!waited) {
+                pdl_wait();
+                waited = true;
+            }
             if (dyn) {
+                if (tile == t_begin && lane == 0) next = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
                 tile = __shfl_sync(0xffffffffu, next, 0);
                 if (lane == 0 && tile < t_end) next = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
             } else {
@@ -505,6 +578,7 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
             fa[q] = fb[q] = 1.f;
         }
         const int rrow = lane & 15;
+        pdl_wait();
         const float gsc = FMT == 2 ? __ldg(p.global_scale) : 1.f;
         bool have_f = FMT == 0;
         // The row scales and the mask words are read per tile in an order known only at
@@ -586,21 +660,24 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
                 }
             }
         }
+        // lane 0 publishes the CTA's partials (columns 2q from itself, 2q + 1 from lane
+        // 16), then takes a ticket: release before it, acquire after it
         Partial* parts = reinterpret_cast<Partial*>(p.partials);
 #pragma unroll
         for (int q = 0; q < Q; ++q) {
-            const int col = 2 * q + (lane >> 4);
-            if (rrow == 0 && col < M) parts[(int64_t)blockIdx.x * 16 + col] = Partial{best_v[q], best_i[q]};
+            const float ov = __shfl_sync(0xffffffffu, best_v[q], 16);
+            const int32_t oi = __shfl_sync(0xffffffffu, best_i[q], 16);
+            if (lane == 0 && 2 * q < M) parts[(int64_t)blockIdx.x * 16 + 2 * q] = Partial{best_v[q], best_i[q]};
+            if (lane == 0 && 2 * q + 1 < M) parts[(int64_t)blockIdx.x * 16 + 2 * q + 1] = Partial{ov, oi};
         }
-        __syncwarp();
         int last = 0;
         if (lane == 0) {
-            __threadfence();
+            fence_acq_rel_gpu();
             last = atomicAdd(p.ticket, 1u) == gridDim.x - 1;
         }
         last = __shfl_sync(0xffffffffu, last, 0);
         if (!last) return;
-        __threadfence();
+        fence_acq_rel_gpu();
         // the last CTA folds every CTA's partial: lane l reads CTAs l, l + 32, ...
         // (independent loads in flight together), then a shuffle reduction; ties go
         // to the lowest row index, so the result does not depend on the order
@@ -656,8 +733,11 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
 
     // ------------------------------------------------------------ compute warps
     const int g = lane >> 2, c = lane & 3;
-    stage_bf16<MODE, CW>(p, xs, scratch);
-    if (FMT != 0) stage_to_f16<CW>(p, xs, xexp, scratch);
+    pdl_wait();
+    if (!(MODE == 0 && FMT != 0 && stage_x_f16_direct<CW>(p, xs, xexp, red))) {
+        stage_bf16<MODE, CW>(p, xs, scratch);
+        if (FMT != 0) stage_to_f16<CW>(p, xs, xexp, scratch);
+    }
 
     const bool xg0 = g < M;
     const bool xg1 = NT > 1 && (8 + g) < M;
@@ -907,7 +987,19 @@ cudaError_t launch_one(const SweepParams& p, cudaStream_t s, SweepLaunch* info) 
     q.stage_bytes = geo.stage_bytes;
     q.segs = geo.segs;
     q.stages_per_tile = geo.stages_per_tile;
-    kern<<<(int)grid, Roles<NT>::THREADS, geo.smem, s>>>(q, map_codes, map_scales);
+    // programmatic stream serialization: this launch may begin while the previous
+    // kernel in the stream finishes; the kernel waits for it before touching its data
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(Roles<NT>::THREADS);
+    cfg.dynamicSmemBytes = geo.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if ((e = cudaLaunchKernelEx(&cfg, kern, q, map_codes, map_scales)) != cudaSuccess) return e;
     if (info) {
         info->grid = (int)grid;
         info->smem_bytes = (int)geo.smem;
