@@ -150,6 +150,14 @@ __device__ __forceinline__ uint4 lds128(const void* p) {
 // relaxed atomic used as a flag).
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
+// Atomic add with release (earlier writes visible first) and acquire (later reads see
+// what the releases before it published) semantics at GPU scope; returns the old value.
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
 // Programmatic dependent launch: let the next kernel in the stream start its prologue
 // (it still waits for this grid before reading anything this grid may write), and wait
 // for the previous grid to complete with its writes visible. Both are no-ops when the

@@ -398,24 +398,27 @@ __device__ __forceinline__ void slab_mma(float (&acc)[2][NT][4], const uint8_t* 
 // then adds s(block 2j) D0 + s(block 2j + 1) D1 for rows r0 and r0 + 8 in fp32: eight
 // FFMAs per slab instead of 32 f16 scale multiplies. sw4 points at the row-r0 scale
 // bytes of blocks 4(c % 2) .. 4(c % 2) + 3 of the slab, sw4 + spitch8 at row r0 + 8's.
-__device__ __forceinline__ void slab_mma_blocks(float (&acc)[4], const uint8_t* cw,
+// xv: the lane's B registers; lanes that feed no input (lx false) keep them zero.
+__device__ __forceinline__ void slab_mma_blocks(float (&acc)[4], uint4 (&xv)[4], const uint8_t* cw,
                                                 const uint8_t* sw4, uint32_t spitch8,
                                                 const uint16_t* xp, bool lx) {
     const uint4 ra = lds128(cw);
     const uint4 rb = lds128(cw + 1024);
     const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w};
     const uint32_t wb[4] = {rb.x, rb.y, rb.z, rb.w};
-    const uint4 z = make_uint4(0, 0, 0, 0);
+    if (lx) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) xv[i] = lds128(xp + 8 * i);
+    }
     float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         uint32_t qa[4], qb[4];
         e2m1x8_to_f16x2x4(wa[i], qa);
         e2m1x8_to_f16x2x4(wb[i], qb);
-        const uint4 xv = lx ? lds128(xp + 8 * i) : z;
         float(&d)[4] = i < 2 ? d0 : d1;
-        mma_f16_16816(d, qa[0], qb[0], qa[1], qb[1], xv.x, xv.y);
-        mma_f16_16816(d, qa[2], qb[2], qa[3], qb[3], xv.z, xv.w);
+        mma_f16_16816(d, qa[0], qb[0], qa[1], qb[1], xv[i].x, xv[i].y);
+        mma_f16_16816(d, qa[2], qb[2], qa[3], qb[3], xv[i].z, xv[i].w);
     }
     const uint32_t sa = *reinterpret_cast<const uint32_t*>(sw4);
     const uint32_t sb = *reinterpret_cast<const uint32_t*>(sw4 + spitch8);
@@ -671,10 +674,7 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
             if (lane == 0 && 2 * q + 1 < M) parts[(int64_t)blockIdx.x * 16 + 2 * q + 1] = Partial{ov, oi};
         }
         int last = 0;
-        if (lane == 0) {
-            fence_acq_rel_gpu();
-            last = atomicAdd(p.ticket, 1u) == gridDim.x - 1;
-        }
+        if (lane == 0) last = atom_add_acq_rel_gpu(p.ticket, 1u) == gridDim.x - 1;
         last = __shfl_sync(0xffffffffu, last, 0);
         if (!last) return;
         fence_acq_rel_gpu();
@@ -761,6 +761,9 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
     const uint16_t* xrowb = xs + (g >> 2) * p.kpad + c * V;
     const uint32_t soffb = (uint32_t)code_stage_bytes(segs) + (uint32_t)r0 * spitch + 4u * (uint32_t)(c & 1);
     float accb[4] = {0.f, 0.f, 0.f, 0.f};
+    uint4 xvb[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) xvb[i] = make_uint4(0, 0, 0, 0);
 
     // Accumulation chains follow the absolute slab index a (64-byte column block of
     // the row): chain a % 16 takes slabs in increasing a. With 16 compute warps warp w
@@ -800,7 +803,7 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
             if (BD) {
                 const uint8_t* swb = st + soffb + l * 8;
                 for (; l < nv; l += CW, cw += CW * 1024, swb += CW * 8, xo += CW * SLAB)
-                    slab_mma_blocks(accb, cw, swb, 8u * spitch, xrowb + xo, xbd);
+                    slab_mma_blocks(accb, xvb, cw, swb, 8u * spitch, xrowb + xo, xbd);
             } else {
                 for (; l < nv; l += CW, cw += CW * 1024, sw += CW * 8, xo += CW * SLAB) {
                     if (CH == 2 && (((a0 + l) >> 3) & 1))
