@@ -33,9 +33,9 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum) and
 # the sha256 of sweep.cu when it was captured; reported as null once the source changed.
 # bf16_M1: the 40,000-row capture (profiles/sweep_kernel_bf16_40k_rows.md) read
-# 327,776,000 B and wrote 3,560,192 B; reads scale with the rows swept, so a full
-# 154,880-row launch reads 327,776,000 x 154,880 / 40,000 B (writes kept unscaled).
-NCU_TRAFFIC = {"bf16_M1": (1272708864, "ddf3fbe92253daf5")}
+# 327,760,128 B and wrote 4,286,720 B; reads scale with the rows swept, so a full
+# 154,880-row launch reads 327,760,128 x 154,880 / 40,000 B (writes kept unscaled).
+NCU_TRAFFIC = {"bf16_M1": (1273373935, "4afd4de0b93f304e")}
 
 
 def sweep_source_hash() -> str:

@@ -8,30 +8,38 @@
 // with deq(W) the BF16 value, an E4M3 code (row scale s_n) or an E2M1 code times its
 // E4M3 block scale (global scale s_n = g).
 //
-// Design (B200, HBM-bound): one persistent CTA per SM owns a contiguous range of
-// 16-row tiles. A producer warp streams the table through a shared-memory ring with
-// one TMA tensor copy per stage -- 16 rows x 1 KB of codes, written with the 128-byte
-// swizzle (plus a 16 x 128-byte copy of the NVFP4 block scales) -- completing on an
-// mbarrier. Large single copies matter: the TMA unit's per-copy cost caps a ring fed
-// by 1 KB row copies at about half of HBM bandwidth, while 16 KB tensor boxes stream
-// at the copy peak. Out-of-range rows and K tails arrive as zeros (tensor-map bounds).
-// Sixteen compute warps (eight when M > 8) split each stage's K range into 16 slabs of
-// 4 lanes x 16 B, decode the codes exactly into f16/bf16 fragments and run
-// tensor-core MMAs with 16 table rows as the A operand and up to 16 inputs as the B
-// operand (swap-AB). MMA row g reads table row s(g) of the tile, a fixed permutation
-// that, with the swizzle, makes every shared-memory read conflict-free. E4M3 codes and
-// E2M1 codes times their E4M3 block scale are exact in f16; x is staged once per CTA
+// Design (B200, HBM-bound): one persistent CTA per SM. Tiles of 16 table rows are
+// handed out at run time: CTA b starts with tile b, then takes the next tile from an
+// atomic counter in the workspace, so SMs that stream faster take more tiles (per-SM
+// HBM throughput varies by ~20%; a fixed split leaves a long tail). A producer warp
+// claims tiles one ahead and streams each through a shared-memory ring with ONE TMA
+// tensor copy per stage -- 16 rows x up to 32 128-byte segments (64 KB), written with
+// the 128-byte swizzle, plus one copy of the NVFP4 block scales -- completing on an
+// mbarrier; each stage carries its tile index, and a stage tagged -1 ends the CTA's
+// work. Large copies matter: the TMA unit's per-copy cost caps a ring fed by 1 KB row
+// copies at about half of HBM bandwidth. Out-of-range rows and K tails arrive as
+// zeros (tensor-map bounds). Sixteen compute warps (eight when M > 8) split each
+// stage's K range into slabs of 4 lanes x 16 B per row, decode the codes exactly into
+// f16/bf16 fragments and run tensor-core MMAs with 16 table rows as the A operand and
+// up to 16 inputs as the B operand (swap-AB). MMA row g reads table row s(g) of the
+// tile, a fixed permutation that, with the swizzle, makes every shared-memory read
+// conflict-free. E4M3 codes and E2M1 codes times their E4M3 block scale are exact in
+// f16; NVFP4 with one or two inputs instead keeps the codes unscaled and applies the
+// block scales to per-block fp32 sums (see slab_mma_blocks). x is staged once per CTA
 // (bf16 for BF16 tables; f16 scaled by a per-row power of two for quantized tables,
-// undone in fp32), so the only roundings are the fp32 accumulation. At the end of a
-// tile each compute warp hands its partial to a reducer warp through a double-buffered
-// shared slot (mbarrier hand-off, no CTA-wide barrier on the streaming path). The
-// reducer sums the partials in a fixed warp order (deterministic and independent of
-// M), scales, masks and folds them into a running (max, lowest index) per input row.
-// Tiles whose 16 rows are masked out for every input are neither loaded nor computed.
-// Each CTA writes its partial; the last CTA to finish (atomic ticket, no waiting)
-// reduces them in CTA order and re-zeroes the ticket. Every mbarrier wait is bounded:
-// a wait that runs out sets an abort flag and MTP_DEVFLAG_TIMEOUT, and the kernel runs
-// to its end.
+// undone in fp32), so the only roundings are fp32 ones. At the end of a tile each
+// compute warp hands its partial to a reducer warp through a double-buffered shared
+// slot (mbarrier hand-off, no CTA-wide barrier on the streaming path). The reducer
+// sums the partials in a fixed warp order (deterministic and independent of M),
+// scales, masks and keeps per lane a running (max, lowest row); the 16 row slots are
+// folded once per CTA. Tiles whose 16 rows are masked out for every input are neither
+// loaded nor computed. Each CTA publishes its partial and takes a ticket; the last CTA
+// (no waiting) folds all partials with 32 lanes and re-zeroes the ticket and the tile
+// counter. The launch allows programmatic dependent launch: the next kernel in the
+// stream may set up and start streaming its own table while this grid finishes, and
+// this kernel waits for the previous grid before reading x, masks or the workspace.
+// Every mbarrier wait is bounded: a wait that runs out sets an abort flag and
+// MTP_DEVFLAG_TIMEOUT, and the kernel runs to its end.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
