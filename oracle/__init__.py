@@ -76,6 +76,7 @@ def lib():
             "orc_lm_head_argmax": (_i32, [_i32, _p, _p, _p, C.c_float, _i64, _i64, _p,
                                           _i32, _p, _i64, _i64, _p, _p, _p]),
             "orc_argmax_masked": (_i32, [_p, _i64, _p, _i64, _p, _p]),
+            "orc_top1_logprob": (C.c_double, [_p, _i64, _p, _i64]),
             "orc_rope_neox": (None, [_p, _i32, C.c_double, C.c_double, _p]),
             "orc_slot": (_i64, [_p, _i64, _i32, _i64, _i64]),
             "orc_kv_encode": (None, [_p, _i64, C.c_float, _p]),
@@ -233,6 +234,13 @@ def argmax_masked(logits, mask=None, mask_words=0):
     flags = lib().orc_argmax_masked(_ptr(logits), logits.size, _ptr(mk), int(mask_words),
                                     _ptr(idx), _ptr(val))
     return int(idx[0]), float(val[0]), int(flags)
+
+
+def top1_logprob(logits, mask=None, mask_words=0) -> float:
+    """Log-softmax at the argmax over the allowed tokens of one logit row."""
+    logits = _c(logits, np.float64)
+    mk = None if mask is None else _c(mask, np.int32)
+    return float(lib().orc_top1_logprob(_ptr(logits), logits.size, _ptr(mk), int(mask_words)))
 
 
 # ---- prefill (prefill.c) -------------------------------------------------------

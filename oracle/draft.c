@@ -24,9 +24,21 @@
  * is taken on the unrounded logit, so that a top-2 gap larger than one bf16 ulp of
  * the logit decides the winner.
  *
+ * Top-1 log-probability ([mtp_head.rs] MtpHead fields: argmax_bf16_batch_lp emits
+ * each row's top-1 log-probability; the chain confidence is the smallest top-1
+ * softmax probability across drafts): the log-softmax of the logits over the allowed
+ * tokens, taken at the argmax,
+ *   lp = l[idx] - log(sum over allowed n of exp(l[n])),
+ * evaluated as -log(sum over allowed n of exp(l[n] - l[idx])) since l[idx] is the
+ * allowed maximum. Reading: no temperature, the same unrounded logits and mask as
+ * the argmax; no allowed token -> -inf.
+ *
  * Pins (tests/test_oracle.py): one-hot inputs select exact table entries, numpy's
  * float64 matmul on the dequantized table, planted maxima, masked decoys,
- * duplicate rows (lowest index), the all-masked row, closed forms of RMSNorm.
+ * duplicate rows (lowest index), the all-masked row, closed forms of RMSNorm; for
+ * the log-probability: equal logits give -log(allowed count), a single allowed token
+ * gives 0, two tied maxima far above the rest give -log 2, and adding a constant to
+ * every logit changes nothing.
  */
 #include <math.h>
 #include <stdint.h>
@@ -118,6 +130,17 @@ int32_t orc_argmax_masked(const double* logits, int64_t n, const int32_t* mask,
     *out_idx = best;
     *out_val = best_val;
     return 0;
+}
+
+double orc_top1_logprob(const double* logits, int64_t n, const int32_t* mask,
+                        int64_t mask_words) {
+    int32_t idx = 0;
+    double top = 0.0;
+    if (orc_argmax_masked(logits, n, mask, mask_words, &idx, &top) != 0) return -INFINITY;
+    double sum = 0.0;
+    for (int64_t t = 0; t < n; ++t)
+        if (allowed(mask, mask_words, t)) sum += exp(logits[t] - top);
+    return -log(sum);
 }
 
 int32_t orc_lm_head_argmax(int32_t fmt, const void* data, const float* row_scale,

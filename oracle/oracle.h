@@ -68,6 +68,8 @@ int32_t orc_lm_head_argmax(int32_t fmt, const void* data, const float* row_scale
                            int32_t* out_idx, double* out_val);
 int32_t orc_argmax_masked(const double* logits, int64_t n, const int32_t* mask,
                           int64_t mask_words, int32_t* out_idx, double* out_val);
+double  orc_top1_logprob(const double* logits, int64_t n, const int32_t* mask,
+                         int64_t mask_words);
 
 /* prefill.c */
 void    orc_rope_neox(const double* k, int32_t hd, double pos, double base, double* out);

@@ -501,3 +501,33 @@ def test_head_table_planted_gap_full_size(orc):
     assert idx[0] == d["top"][0]
     srt = np.sort(logits[0])
     assert srt[-1] - srt[-2] >= 0.5
+
+
+def test_top1_logprob_pins(orc):
+    """Log-softmax at the argmax: closed forms that any mistake in the sum, the mask
+    handling or the max subtraction would break."""
+    n = 1000
+    rng = np.random.default_rng(3)
+    for c in (0.0, 3.5, -7.25):  # equal logits: a uniform softmax
+        assert orc.top1_logprob(np.full(n, c)) == pytest.approx(-np.log(n), abs=1e-12)
+    allowed = rng.choice(n, 37, replace=False)
+    mask = np.zeros((n + 31) // 32, np.int32)
+    for t in allowed:
+        mask[t // 32] |= np.int32(np.uint32(1 << (t % 32)).view(np.int32))
+    logits = np.where(np.isin(np.arange(n), allowed), 2.0, 50.0)  # disallowed ones larger
+    assert orc.top1_logprob(logits, mask, mask.size) == pytest.approx(-np.log(37), abs=1e-12)
+    one = np.zeros_like(mask)
+    one[allowed[0] // 32] = np.int32(np.uint32(1 << (allowed[0] % 32)).view(np.int32))
+    assert orc.top1_logprob(rng.normal(size=n), one, one.size) == 0.0
+    tied = rng.normal(size=n)
+    tied[[10, 500]] = 1000.0  # the rest add exp(-1000 + O(1)) = 0 in double
+    assert orc.top1_logprob(tied) == pytest.approx(-np.log(2.0), abs=1e-15)
+    l = rng.normal(size=n) * 3.0
+    assert orc.top1_logprob(l + 123.0) == pytest.approx(orc.top1_logprob(l), abs=1e-12)
+    assert orc.top1_logprob(l) < 0.0
+    assert orc.top1_logprob(l, np.zeros_like(mask), mask.size) == -np.inf
+    # through the sweep: a zero input makes every logit 0
+    k = 256
+    w = synth.as_u16(synth.normal_bf16(synth._gen(31), (300, k), 0.02))
+    lg, idx, _, _ = orc.lm_head_argmax(0, w, k, np.zeros((1, k), np.uint16))
+    assert idx[0] == 0 and orc.top1_logprob(lg[0]) == pytest.approx(-np.log(300), abs=1e-12)
