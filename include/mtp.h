@@ -188,6 +188,26 @@ mtp_status mtp_lm_head_argmax(const mtp_weight* head, int64_t n_eff, const uint1
                               size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------
+ * mtp_lm_head_argmax_lp -- mtp_lm_head_argmax that also writes each input's top-1
+ * log-probability from the same sweep (no extra table bytes).
+ * Source: [mtp_head.rs] MtpHead fields: argmax_bf16_batch_lp, the batched argmax that
+ * also emits each row's top-1 log-probability, and the chain confidence (the smallest
+ * top-1 softmax probability across drafts).
+ *   out_logprob[m] = l[m, idx] - log(sum over allowed r < n_eff of exp(l[m, r]))
+ * over the same fp32 logits and mask as the argmax (no temperature); -inf when no
+ * token is allowed. The sum of exponentials is accumulated in fp32 in an order that
+ * follows the run-time split of the table over SMs, so its last bits can differ from
+ * one call to the next; the argmax, out_val and out_logits do not.
+ *   out_logprob   (device) f32 [M], written; must not be NULL (MTP_ERR_INVALID_ARG)
+ * Every other argument, the workspace and the requirements are mtp_lm_head_argmax's.
+ * ------------------------------------------------------------------------------ */
+mtp_status mtp_lm_head_argmax_lp(const mtp_weight* head, int64_t n_eff, const uint16_t* x,
+                                 int32_t M, const int32_t* mask, int64_t mask_words,
+                                 int64_t mask_stride_words, int32_t* out_idx, float* out_val,
+                                 float* out_logprob, uint16_t* out_logits, int32_t* dev_err,
+                                 void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------
  * mtp_prefill_kv -- the drafter-context prefill: the drafter's K/V cache rows for R
  * prompt rows, written as E4M3 codes into a paged cache.
  * Source: [mtp_head.rs] drafter-prefill docs (the drafter's K/V for prompt row i are a
@@ -248,7 +268,7 @@ mtp_status mtp_debug_kv_write(const uint16_t* k_rot, const uint16_t* v, int64_t 
  * code that must not risk the device synchronisation cudaMalloc/cudaFree can cause).
  * Inputs and outputs are the caller's, exactly as for mtp_lm_head_argmax; the scratch
  * is a static device array inside the library, mtp_noalloc_scratch_bytes() bytes
- * (131,328) held on every GPU that loads the library until the process exits.
+ * (262,400) held on every GPU that loads the library until the process exits.
  *  - The first call made with a device current looks up that array's device address
  *    and zeroes its counter (synchronously); make it before any stream capture.
  *  - All calls on a device share the array: calls that overlap on the GPU race and

@@ -34,7 +34,7 @@ MTP_FMT_NVFP4 = 2
 EXPORTS = (
     "mtp_abi_version", "mtp_status_str", "mtp_devflags_status",
     "mtp_quantize_fp8", "mtp_quantize_nvfp4_ws_bytes", "mtp_quantize_nvfp4",
-    "mtp_combine", "mtp_lm_head_ws_bytes", "mtp_lm_head_argmax",
+    "mtp_combine", "mtp_lm_head_ws_bytes", "mtp_lm_head_argmax", "mtp_lm_head_argmax_lp",
     "mtp_debug_encode_e4m3", "mtp_debug_encode_e2m1", "mtp_nvfp4_scale_pitch",
     "mtp_noalloc_scratch_bytes", "mtp_lm_head_argmax_noalloc",
     "mtp_prefill_ws_bytes", "mtp_prefill_kv", "mtp_debug_gemm_bf16", "mtp_debug_kv_write",
@@ -72,6 +72,8 @@ _SIGS = {
     "mtp_lm_head_ws_bytes": (_SZ, [_W, _I64, _I32]),
     "mtp_lm_head_argmax": (C.c_int, [_W, _I64, _P, _I32, _P, _I64, _I64, _P, _P, _P, _P,
                                      _P, _SZ, _P]),
+    "mtp_lm_head_argmax_lp": (C.c_int, [_W, _I64, _P, _I32, _P, _I64, _I64, _P, _P, _P, _P,
+                                        _P, _P, _SZ, _P]),
     "mtp_prefill_ws_bytes": (_SZ, [_I64, _I32, _I32, _I32]),
     "mtp_prefill_kv": (C.c_int, [_P, _I64, _P, _P, _I64, _I32, _P, _P, C.c_float, _P, _P, _P,
                                  _I32, _I32, C.c_float, _P, _I64, _P, _I64, _I32, _P, _P, _I64,
@@ -183,6 +185,16 @@ def mtp_lm_head_argmax(head, n_eff, x, M, mask, mask_words, mask_stride_words, o
                                      _ptr(out_idx), _ptr(out_val), _ptr(out_logits),
                                      _ptr(dev_err), _ptr(ws), ws_bytes, _stream(stream)),
            "mtp_lm_head_argmax")
+
+
+def mtp_lm_head_argmax_lp(head, n_eff, x, M, mask, mask_words, mask_stride_words, out_idx,
+                          out_val, out_logprob, out_logits, dev_err, ws, ws_bytes, stream=None):
+    _check(load().mtp_lm_head_argmax_lp(C.byref(head) if head is not None else None, n_eff,
+                                        _ptr(x), M, _ptr(mask), mask_words, mask_stride_words,
+                                        _ptr(out_idx), _ptr(out_val), _ptr(out_logprob),
+                                        _ptr(out_logits), _ptr(dev_err), _ptr(ws), ws_bytes,
+                                        _stream(stream)),
+           "mtp_lm_head_argmax_lp")
 
 
 def mtp_prefill_ws_bytes(chunk_rows, h, nkv, hd) -> int:

@@ -83,21 +83,29 @@ class LmHead:
         return int(t.nbytes() * frac) + M * t.k * 2 + mask_words * 4 * (1 if M else 0) + M * 8
 
     def __call__(self, x: torch.Tensor, out_idx: torch.Tensor, out_val=None, out_logits=None,
-                 mask=None, mask_words=0, mask_stride_words=0, stream=None):
+                 mask=None, mask_words=0, mask_stride_words=0, stream=None, out_logprob=None):
         M = x.shape[0]
-        L.mtp_lm_head_argmax(self.table.desc, self.n_eff, x, M, mask, mask_words,
-                             mask_stride_words, out_idx, out_val, out_logits, self.dev_err,
-                             self.ws, self.ws.numel(), stream)
+        if out_logprob is None:
+            L.mtp_lm_head_argmax(self.table.desc, self.n_eff, x, M, mask, mask_words,
+                                 mask_stride_words, out_idx, out_val, out_logits, self.dev_err,
+                                 self.ws, self.ws.numel(), stream)
+        else:
+            L.mtp_lm_head_argmax_lp(self.table.desc, self.n_eff, x, M, mask, mask_words,
+                                    mask_stride_words, out_idx, out_val, out_logprob,
+                                    out_logits, self.dev_err, self.ws, self.ws.numel(), stream)
 
     def argmax(self, x: torch.Tensor, mask=None, mask_words=0, mask_stride_words=0,
-               logits=False, stream=None):
+               logits=False, stream=None, logprob=False):
+        """Returns (idx, val, logits or None), plus the top-1 log-probabilities when
+        logprob is true."""
         M = x.shape[0]
         dev = x.device
         idx = torch.empty((M,), dtype=torch.int32, device=dev)
         val = torch.empty((M,), dtype=torch.float32, device=dev)
         lg = torch.empty((M, self.n_eff), dtype=torch.bfloat16, device=dev) if logits else None
-        self(x, idx, val, lg, mask, mask_words, mask_stride_words, stream)
-        return idx, val, lg
+        lp = torch.empty((M,), dtype=torch.float32, device=dev) if logprob else None
+        self(x, idx, val, lg, mask, mask_words, mask_stride_words, stream, out_logprob=lp)
+        return (idx, val, lg, lp) if logprob else (idx, val, lg)
 
 
 def combine(embed, token_ids, hidden, w_norm_embed, w_norm_hidden, eps, fc: Table,

@@ -54,7 +54,7 @@ int64_t row_bytes(const mtp_weight* w) {
 }
 
 constexpr size_t kTicketBytes = 256;
-constexpr size_t kPartialBytes = 8;  // {float value, int32 index}
+constexpr size_t kPartialBytes = 16;  // {float value, int32 index, float sum of exp, pad}
 constexpr int kMaxM = 16;
 
 }  // namespace
@@ -158,11 +158,13 @@ size_t mtp_lm_head_ws_bytes(const mtp_weight* head, int64_t n_eff, int32_t M) {
     return kTicketBytes + kPartialBytes * 16 * (size_t)mtp::sweep_max_grid();
 }
 
-mtp_status mtp_lm_head_argmax(const mtp_weight* head, int64_t n_eff, const uint16_t* x,
-                              int32_t M, const int32_t* mask, int64_t mask_words,
-                              int64_t mask_stride_words, int32_t* out_idx, float* out_val,
-                              uint16_t* out_logits, int32_t* dev_err, void* ws,
-                              size_t ws_bytes, void* stream) {
+namespace {
+
+mtp_status lm_head_impl(const mtp_weight* head, int64_t n_eff, const uint16_t* x, int32_t M,
+                        const int32_t* mask, int64_t mask_words, int64_t mask_stride_words,
+                        int32_t* out_idx, float* out_val, float* out_logprob,
+                        uint16_t* out_logits, int32_t* dev_err, void* ws, size_t ws_bytes,
+                        void* stream) {
     mtp_status st = check_weight(head);
     if (st != MTP_OK) return st;
     if (!x || !out_idx || n_eff < 1 || n_eff > head->n) return MTP_ERR_INVALID_ARG;
@@ -170,6 +172,7 @@ mtp_status mtp_lm_head_argmax(const mtp_weight* head, int64_t n_eff, const uint1
     if (M < 1 || M > kMaxM) return MTP_ERR_UNSUPPORTED;
     if (mask && (mask_words < 1 || mask_stride_words < 0)) return MTP_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(out_idx, 4) || !aligned(out_val, 4) ||
+        !aligned(out_logprob, 4) ||
         !aligned(out_logits, 2) || !aligned(dev_err, 4) || !aligned(mask, 4))
         return MTP_ERR_INVALID_ARG;
     if (!ws || !aligned(ws, 16) || ws_bytes < mtp_lm_head_ws_bytes(head, n_eff, M))
@@ -192,12 +195,34 @@ mtp_status mtp_lm_head_argmax(const mtp_weight* head, int64_t n_eff, const uint1
     p.out_idx = out_idx;
     p.out_val = out_val;
     p.out_logits = out_logits;
+    p.out_logprob = out_logprob;
     p.dev_err = dev_err;
     p.ticket = static_cast<uint32_t*>(ws);
     p.partials = static_cast<uint8_t*>(ws) + kTicketBytes;
     p.num_tiles = (n_eff + 15) / 16;
     p.scale_pitch = mtp::nvfp4_scale_pitch(head->k);
     return from_cuda(mtp::sweep_launch(p, head->fmt, 0, as_stream(stream), nullptr));
+}
+
+}  // namespace
+
+mtp_status mtp_lm_head_argmax(const mtp_weight* head, int64_t n_eff, const uint16_t* x,
+                              int32_t M, const int32_t* mask, int64_t mask_words,
+                              int64_t mask_stride_words, int32_t* out_idx, float* out_val,
+                              uint16_t* out_logits, int32_t* dev_err, void* ws,
+                              size_t ws_bytes, void* stream) {
+    return lm_head_impl(head, n_eff, x, M, mask, mask_words, mask_stride_words, out_idx, out_val,
+                        nullptr, out_logits, dev_err, ws, ws_bytes, stream);
+}
+
+mtp_status mtp_lm_head_argmax_lp(const mtp_weight* head, int64_t n_eff, const uint16_t* x,
+                                 int32_t M, const int32_t* mask, int64_t mask_words,
+                                 int64_t mask_stride_words, int32_t* out_idx, float* out_val,
+                                 float* out_logprob, uint16_t* out_logits, int32_t* dev_err,
+                                 void* ws, size_t ws_bytes, void* stream) {
+    if (!out_logprob) return MTP_ERR_INVALID_ARG;
+    return lm_head_impl(head, n_eff, x, M, mask, mask_words, mask_stride_words, out_idx, out_val,
+                        out_logprob, out_logits, dev_err, ws, ws_bytes, stream);
 }
 
 size_t mtp_prefill_ws_bytes(int64_t chunk_rows, int32_t h, int32_t nkv, int32_t hd) {

@@ -38,6 +38,7 @@ struct SweepParams {
     int32_t* out_idx;
     float* out_val;
     uint16_t* out_logits;        // bf16 [M, n] or null
+    float* out_logprob;          // f32 [M] top-1 log-probability, or null
     uint16_t* out_y;             // mode 1: bf16 [M, n]
     int32_t* dev_err;
     // workspace (mode 0)

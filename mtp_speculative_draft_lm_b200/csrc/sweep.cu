@@ -68,10 +68,22 @@ template <int NT> struct Roles {
     static constexpr int RED_COLS = 8 * NT;
 };
 
+// A CTA's result for one input: the allowed maximum, its lowest row, and the sum of
+// exp(l - v) over the allowed rows it saw (for the top-1 log-probability).
 struct Partial {
     float v;
     int32_t i;
+    float s;
+    float pad;
 };
+
+// Merges (v2, s2) into (v, s): sums of exp(l - max) over two row sets.
+__device__ __forceinline__ void lse_merge(float& v, float& s, float v2, float s2) {
+    const float m = fmaxf(v, v2);
+    if (m == -INFINITY) return;
+    s = s * expf(v - m) + s2 * expf(v2 - m);
+    v = m;
+}
 
 // V: K elements per 16-byte piece of codes. A slab is 64 bytes of one row (4 lanes x
 // 16 B, 4V elements); a stage holds `segs` 128-byte segments (2 * segs slabs) of each
@@ -582,11 +594,14 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
         float best_v[Q];
         int32_t best_i[Q];
         float fa[Q], fb[Q];  // 2^-xexp as two factors: (a fa) fb is exact for a normal result
+        float se[Q];         // sum of exp(l - best_v) over the allowed rows seen
+        const bool lp = MODE == 0 && p.out_logprob != nullptr;
 #pragma unroll
         for (int q = 0; q < Q; ++q) {
             best_v[q] = -INFINITY;
             best_i[q] = INT_MAX;
             fa[q] = fb[q] = 1.f;
+            se[q] = 0.f;
         }
         const int rrow = lane & 15;
         pdl_wait();
@@ -644,6 +659,10 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
                     const bool ok = valid && mask_allows(p, col, row);
                     if (valid && p.out_logits)
                         p.out_logits[(int64_t)col * p.n + row] = ok ? f32_to_bf16(l) : (uint16_t)0xFF80u;
+                    if (lp && ok && l > -INFINITY) {
+                        float v = best_v[q];
+                        lse_merge(v, se[q], l, 1.f);
+                    }
                     // rows arrive in increasing order, so the lowest row wins a tie
                     if (ok && (l > best_v[q] || (l == best_v[q] && best_i[q] == INT_MAX))) {
                         best_v[q] = l;
@@ -665,6 +684,11 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
             for (int o = 8; o; o >>= 1) {
                 const float ov = __shfl_xor_sync(0xffffffffu, best_v[q], o);
                 const int32_t oi = __shfl_xor_sync(0xffffffffu, best_i[q], o);
+                const float os = __shfl_xor_sync(0xffffffffu, se[q], o);
+                if (lp) {
+                    float v = best_v[q];
+                    lse_merge(v, se[q], ov, os);
+                }
                 if (ov > best_v[q] || (ov == best_v[q] && oi < best_i[q])) {
                     best_v[q] = ov;
                     best_i[q] = oi;
@@ -678,8 +702,11 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
         for (int q = 0; q < Q; ++q) {
             const float ov = __shfl_sync(0xffffffffu, best_v[q], 16);
             const int32_t oi = __shfl_sync(0xffffffffu, best_i[q], 16);
-            if (lane == 0 && 2 * q < M) parts[(int64_t)blockIdx.x * 16 + 2 * q] = Partial{best_v[q], best_i[q]};
-            if (lane == 0 && 2 * q + 1 < M) parts[(int64_t)blockIdx.x * 16 + 2 * q + 1] = Partial{ov, oi};
+            const float os = __shfl_sync(0xffffffffu, se[q], 16);
+            if (lane == 0 && 2 * q < M)
+                parts[(int64_t)blockIdx.x * 16 + 2 * q] = Partial{best_v[q], best_i[q], se[q], 0.f};
+            if (lane == 0 && 2 * q + 1 < M)
+                parts[(int64_t)blockIdx.x * 16 + 2 * q + 1] = Partial{ov, oi, os, 0.f};
         }
         int last = 0;
         if (lane == 0) last = atom_add_acq_rel_gpu(p.ticket, 1u) == gridDim.x - 1;
@@ -690,45 +717,63 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
         // (independent loads in flight together), then a shuffle reduction; ties go
         // to the lowest row index, so the result does not depend on the order
         const int G = (int)gridDim.x;
+        constexpr int FOLD = 8;  // partials per lane in flight at a time
         for (int m = 0; m < M; ++m) {
-            float bv = -INFINITY;
+            float bv = -INFINITY, bs = 0.f;
             int32_t bi = INT_MAX;
-            float qv[kMaxGrid / 32];
-            int32_t qi[kMaxGrid / 32];
+            for (int base = 0; base < G; base += 32 * FOLD) {
+                float qv[FOLD], qs[FOLD];
+                int32_t qi[FOLD];
 #pragma unroll
-            for (int j = 0; j < kMaxGrid / 32; ++j) {
-                const int b = lane + 32 * j;
-                qv[j] = -INFINITY;
-                qi[j] = INT_MAX;
-                if (b < G) {
-                    const Partial* src = parts + (int64_t)b * 16 + m;
-                    qv[j] = __ldcg(&src->v);
-                    qi[j] = __ldcg(&src->i);
+                for (int j = 0; j < FOLD; ++j) {
+                    const int b = base + lane + 32 * j;
+                    qv[j] = -INFINITY;
+                    qi[j] = INT_MAX;
+                    qs[j] = 0.f;
+                    if (b < G) {
+                        const float4 e = __ldcg(reinterpret_cast<const float4*>(parts + (int64_t)b * 16 + m));
+                        qv[j] = e.x;
+                        qi[j] = __float_as_int(e.y);
+                        qs[j] = e.z;
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < FOLD; ++j) {
+                    if (lp) {
+                        float v = bv;
+                        lse_merge(v, bs, qv[j], qs[j]);
+                    }
+                    if (qv[j] > bv || (qv[j] == bv && qi[j] < bi)) {
+                        bv = qv[j];
+                        bi = qi[j];
+                    }
                 }
             }
-#pragma unroll
-            for (int j = 0; j < kMaxGrid / 32; ++j)
-                if (qv[j] > bv || (qv[j] == bv && qi[j] < bi)) {
-                    bv = qv[j];
-                    bi = qi[j];
-                }
 #pragma unroll
             for (int o = 16; o; o >>= 1) {
                 const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
                 const int32_t oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                const float os = __shfl_xor_sync(0xffffffffu, bs, o);
+                if (lp) {
+                    float v = bv;
+                    lse_merge(v, bs, ov, os);
+                }
                 if (ov > bv || (ov == bv && oi < bi)) {
                     bv = ov;
                     bi = oi;
                 }
             }
             if (lane == 0) {
-                if (bi == INT_MAX) {
+                const bool empty = bi == INT_MAX;
+                if (empty) {
                     bi = 0;
                     bv = -INFINITY;
                     raise_flag(p.dev_err, DEVFLAG_EMPTY_MASK);
                 }
                 p.out_idx[m] = bi;
                 if (p.out_val) p.out_val[m] = bv;
+                // the maximum's own term is exp(0) = 1, so bs >= 1 and the result is <= 0
+                if (lp) p.out_logprob[m] = empty ? -INFINITY : -logf(bs);
             }
         }
         __syncwarp();

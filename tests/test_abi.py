@@ -115,6 +115,22 @@ def test_lm_head_rejects(lib):
     assert lm(w) == L.MTP_ERR_INVALID_ARG
 
 
+def test_lm_head_lp_rejects(lib):
+    head = weight()
+    wsb = L.mtp_lm_head_ws_bytes(head, 100, 1)
+
+    def lp(out_lp, x=B2, n_eff=100):
+        return st("mtp_lm_head_argmax_lp", C.byref(head), n_eff, x, 1, None, 0, 0, OUT, None,
+                  out_lp, None, None, 0x40000, wsb, None)
+
+    assert lp(None) == L.MTP_ERR_INVALID_ARG        # the log-probability output is required
+    assert lp(OUT + 2) == L.MTP_ERR_INVALID_ARG     # f32 alignment
+    assert lp(OUT, x=B2 + 4) == L.MTP_ERR_INVALID_ARG  # the same checks as mtp_lm_head_argmax
+    assert lp(OUT, n_eff=101) == L.MTP_ERR_INVALID_ARG
+    # partials are 16 bytes (max, index, sum of exponentials) for up to 1,024 CTAs x 16 rows
+    assert wsb == 256 + 16 * 16 * 1024 and L.mtp_noalloc_scratch_bytes() == wsb
+
+
 def test_combine_rejects(lib):
     fc = weight(n=32, k=64)
     args = [A, 50, B2, B2, 1, 32, OUT, OUT, 1e-6, C.byref(fc), OUT, None, None]

@@ -232,3 +232,66 @@ def test_full_tables(orc, cfg, fmt):
             got = run_sweep(table, x[:M], head=head, mask=d["mask"][:M].reshape(-1),
                             mask_words=words, stride=words, logits=False)
             assert np.array_equal(got[0], d["second"][:M])
+
+
+def oracle_logprobs(orc, ref_l, mask=None, mask_words=0, stride=0):
+    out = []
+    for m in range(ref_l.shape[0]):
+        mrow = None
+        if mask is not None:
+            mrow = mask[m * stride: m * stride + mask_words] if stride else mask[:mask_words]
+        out.append(orc.top1_logprob(ref_l[m], mrow, mask_words))
+    return np.array(out)
+
+
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+@pytest.mark.parametrize("M", [1, 2, 3, 9, 16])
+def test_top1_logprob(orc, fmt, M):
+    """mtp_lm_head_argmax_lp: the argmax outputs equal mtp_lm_head_argmax's bit for bit,
+    and the top-1 log-probability matches the oracle's (fp64 log-softmax at the argmax)
+    within 2e-2 + 1e-2|ref|, with and without a mask; an all-masked row gives -inf."""
+    n, k = 3000, {0: 512, 1: 1024, 2: 1280}[fmt]
+    w = synth.as_u16(synth.normal_bf16(synth._gen(40 + fmt), (n, k), 0.05))
+    x = synth.as_u16(synth.normal_bf16(synth._gen(50 + M), (M, k), 1.0))
+    q = oracle_quant(orc, w, fmt)
+    table = device_table(q, fmt, n, k)
+    head = api.LmHead(table)
+    xd = to_dev_u16(x)
+    i0, v0, l0 = head.argmax(xd, logits=True)
+    i1, v1, l1, lp = head.argmax(xd, logits=True, logprob=True)
+    torch.cuda.synchronize()
+    assert torch.equal(i0, i1) and torch.equal(v0.view(torch.int32), v1.view(torch.int32))
+    assert torch.equal(l0.view(torch.int16), l1.view(torch.int16))
+    ref_l, ref_i, _, _ = oracle_sweep(orc, q, fmt, k, x)
+    assert np.array_equal(i1.cpu().numpy(), ref_i)
+    assert_close(lp.cpu().numpy(), oracle_logprobs(orc, ref_l), "top-1 log-probability")
+    assert np.all(lp.cpu().numpy() <= 0.0)
+    # per-row masks keeping ~5%; row 0 keeps nothing
+    words = (n + 31) // 32
+    rng = np.random.default_rng(60 + M)
+    keep = rng.random((M, words * 32)) < 0.05
+    keep[0] = False
+    bits = keep.reshape(M, words, 32).astype(np.uint64) << np.arange(32, dtype=np.uint64)
+    mask = bits.sum(axis=-1).astype(np.uint32).view(np.int32)
+    md = to_dev(mask.reshape(-1))
+    _, _, _, lpm = head.argmax(xd, mask=md, mask_words=words, mask_stride_words=words,
+                               logprob=True)
+    torch.cuda.synchronize()
+    got = lpm.cpu().numpy()
+    ref = oracle_logprobs(orc, ref_l, mask.reshape(-1), words, words)
+    assert got[0] == -np.inf and ref[0] == -np.inf
+    assert_close(got[1:], ref[1:], "masked top-1 log-probability")
+
+
+@pytest.mark.parametrize("cfg,fmt", FULL, ids=["bf16", "fp8", "nvfp4"])
+def test_top1_logprob_full_tables(orc, cfg, fmt):
+    d = synth.head_table(cfg["seed"], cfg["N"], cfg["K"], 1)
+    w, x = synth.as_u16(d["W"]), synth.as_u16(d["x"])
+    q = oracle_quant(orc, w, fmt)
+    table = device_table(q, fmt, cfg["N"], cfg["K"])
+    head = api.LmHead(table)
+    idx, _, _, lp = head.argmax(to_dev_u16(x), logprob=True)
+    torch.cuda.synchronize()
+    ref_l, ref_i, _, _ = oracle_sweep(orc, q, fmt, cfg["K"], x)
+    assert idx.item() == ref_i[0]
+    assert_close(lp.cpu().numpy(), oracle_logprobs(orc, ref_l), "full-table log-probability")
