@@ -304,8 +304,45 @@ def bench_tiny_draft(dev, steps, warmup):
         step()
     e.record()
     torch.cuda.synchronize()
-    return {"us_per_draft": s.elapsed_time(e) / steps * 1e3, "launches_per_draft": 2,
-            "note": "hidden 256, vocab 4096, M=1, warm (L2-resident)"}
+    eager_us = s.elapsed_time(e) / steps * 1e3
+
+    # a chain of drafts on the device: each combiner gathers the embedding of the previous
+    # draft's argmax from the device index buffer; captured once as a CUDA graph
+    chain = 16
+    ys = [torch.empty((1, d["h"]), dtype=torch.bfloat16, device=dev) for _ in range(chain)]
+    ids = [torch.empty((1,), dtype=torch.int32, device=dev) for _ in range(chain)]
+
+    def run_chain():
+        tok, hid = dd["tokens"], dd["hidden"]
+        for j in range(chain):
+            api.combine(dd["embed"], tok, hid, dd["w_norm_embed"], dd["w_norm_hidden"], d["eps"],
+                        fc, out=ys[j])
+            head(ys[j], ids[j])
+            tok, hid = ids[j], ys[j]
+
+    cs = torch.cuda.Stream(device=dev)
+    cs.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cs):
+        run_chain()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cs):
+            run_chain()
+    torch.cuda.synchronize()
+    reps = max(10, steps // chain)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    s.record()
+    for _ in range(reps):
+        g.replay()
+    e.record()
+    torch.cuda.synchronize()
+    graph_us = s.elapsed_time(e) / (reps * chain) * 1e3
+    del g
+    return {"us_per_draft": eager_us, "launches_per_draft": 2,
+            "chain_graph_us_per_draft": graph_us, "chain_length": chain,
+            "note": "hidden 256, vocab 4096, M=1, warm (L2-resident); chain: 16 drafts fed "
+                    "device-side (argmax index -> next embedding gather) replayed from a CUDA graph"}
 
 
 def bench_prefill(dev, reps, tflops_peak, peak_src, rows=0):
@@ -489,6 +526,25 @@ def main():
             rows[f"{fmt}_M{M}"] = rec
             if fmt == "bf16" and M == 1:
                 main_line = (rec, nbytes, ms_max, kern_max, e2e_max, h2d, d2h, clk, cfg)
+        # the same sweep with the top-1 log-probability (mtp_lm_head_argmax_lp), M = 1
+        x = d["x"][:1].to(dev)
+        idx = torch.empty((1,), dtype=torch.int32, device=dev)
+        lp = torch.empty((1,), dtype=torch.float32, device=dev)
+        for _ in range(args.warmup):
+            head(x, idx, None, stream=stream, out_logprob=lp)
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            s.record(stream)
+            for _ in range(args.steps):
+                head(x, idx, None, stream=stream, out_logprob=lp)
+            e.record(stream)
+        torch.cuda.synchronize()
+        us = s.elapsed_time(e) / args.steps * 1e3
+        rows[f"{fmt}_M1_logprob"] = {"us_per_draft": us,
+                                     "kernel_GB/s": head.bytes_per_call(1) / (us * 1e-6) / 1e9,
+                                     "argmax_ok": int(idx.item()) == int(d["top"][0]),
+                                     "logprob": float(lp.item())}
         if "mask" in d and args.full:
             words = d["mask"].shape[1]
             m = torch.from_numpy(d["mask"][:1].reshape(-1)).to(dev)

@@ -96,3 +96,59 @@ def test_tiny_draft_end_to_end(orc, M):
     for m in range(M):
         assert_argmax(int(idx[m].item()), ref_l[m])
         assert_close(bf16_bits_to_f64(u16_of(lg)[m]), ref_l[m], "logits")
+
+
+def run_chain(dd, d, fc, head, steps, y_buf, idx_bufs, hid0):
+    """Device-side draft chain: step j gathers the embedding of step j-1's argmax
+    straight from the device index buffer (no host round trip); the combiner output
+    stands in for the next hidden state (the drafter layer is not part of this path)."""
+    tok = dd["tokens"]
+    hid = hid0
+    for j in range(steps):
+        api.combine(dd["embed"], tok, hid, dd["w_norm_embed"], dd["w_norm_hidden"], d["eps"], fc,
+                    out=y_buf[j])
+        head(y_buf[j], idx_bufs[j])
+        tok, hid = idx_bufs[j], y_buf[j]
+
+
+@pytest.mark.parametrize("M", [1, 3])
+def test_device_side_draft_chain(orc, M):
+    """Four chained drafts on the device, eager and replayed from a CUDA graph (which
+    admits no host synchronisation), against the oracle step by step."""
+    steps = 4
+    d = draft(M)
+    dd = {k: (to_dev_u16(v) if isinstance(v, np.ndarray) and v.dtype == np.uint16 else v)
+          for k, v in d.items()}
+    dd["tokens"] = to_dev(np.asarray(d["tokens"], np.int32))
+    fc = api.bf16_table(dd["fc"])
+    head = api.LmHead(api.bf16_table(dd["lm_head"]))
+    hid0 = dd["hidden"].clone()
+    y_buf = [torch.empty((M, d["h"]), dtype=torch.bfloat16, device="cuda") for _ in range(steps)]
+    idx_bufs = [torch.empty((M,), dtype=torch.int32, device="cuda") for _ in range(steps)]
+    run_chain(dd, d, fc, head, steps, y_buf, idx_bufs, hid0)
+    torch.cuda.synchronize()
+    eager = [(u16_of(y).copy(), i.cpu().numpy().copy()) for y, i in zip(y_buf, idx_bufs)]
+    # the oracle chain, continuing from the GPU's (valid) picks
+    tok, hid = np.asarray(d["tokens"], np.int32), d["hidden"]
+    for j in range(steps):
+        ref_y, _, _ = orc.combine(d["embed"], tok, hid, d["w_norm_embed"], d["w_norm_hidden"],
+                                  d["eps"], d["fc"])
+        assert_close(bf16_bits_to_f64(eager[j][0]), bf16_bits_to_f64(ref_y), f"y step {j}")
+        ref_l, _, _, _ = orc.lm_head_argmax(0, d["lm_head"], d["h"], eager[j][0])
+        for m in range(M):
+            assert_argmax(int(eager[j][1][m]), ref_l[m])
+        tok, hid = eager[j][1], eager[j][0]
+    # the same chain captured once and replayed: identical results
+    for b in idx_bufs:
+        b.zero_()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            run_chain(dd, d, fc, head, steps, y_buf, idx_bufs, hid0)
+    g.replay()
+    torch.cuda.synchronize()
+    for j in range(steps):
+        assert np.array_equal(u16_of(y_buf[j]), eager[j][0])
+        assert np.array_equal(idx_bufs[j].cpu().numpy(), eager[j][1])
