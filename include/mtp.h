@@ -208,6 +208,41 @@ mtp_status mtp_lm_head_argmax_lp(const mtp_weight* head, int64_t n_eff, const ui
                                  void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------
+ * Vocab-sharded sweep: each of G GPUs sweeps a contiguous range of the table's rows,
+ * writes a 16-byte partial per input, the partials are gathered (G x M x 16 bytes, one
+ * collective, the caller's: NCCL all-gather over NVLink), and every rank merges them.
+ * Source: [init.rs] the draft head split by vocab across tensor-parallel ranks, each
+ * rank sweeping its own rows, followed by one small (max, argmax) exchange.
+ *
+ * mtp_lm_head_shard_partial -- mtp_lm_head_argmax over one shard.
+ *   shard         the shard's rows as a weight [n, k]; n_eff <= n are swept
+ *   row_offset    global index of the shard's first row; row_offset + n_eff < 2^31
+ *   mask          the GLOBAL mask (token t = row_offset + local row; same layout as
+ *                 mtp_lm_head_argmax's)
+ *   out_partial   (device) 16-byte aligned [M] x {f32 max logit, i32 global row of the
+ *                 maximum (lowest on ties; INT32_MAX when no row of the shard is
+ *                 allowed), f32 sum over allowed rows of exp(l - max), 4 bytes unused}
+ *   out_logits    (device) bf16 [M, n_eff] of the shard, or NULL
+ * An empty shard is not an error (no MTP_DEVFLAG_EMPTY_MASK here). Workspace and the
+ * other requirements are mtp_lm_head_argmax's.
+ *
+ * mtp_argmax_merge_partials -- folds n_parts partials per input, laid out
+ * [n_parts][M] (rank-major, as an all-gather leaves them), into out_idx (i32 [M]),
+ * out_val (f32 [M] or NULL) and out_logprob (f32 [M] or NULL, the log-softmax at the
+ * argmax over all shards). Nothing allowed in any shard -> index 0, -inf, -inf and
+ * MTP_DEVFLAG_EMPTY_MASK in dev_err (i32 [1] or NULL). The fold order is fixed, so every
+ * rank that merges the same partials gets the same bits. 1 <= n_parts <= 65536.
+ * ------------------------------------------------------------------------------ */
+mtp_status mtp_lm_head_shard_partial(const mtp_weight* shard, int64_t n_eff, int64_t row_offset,
+                                     const uint16_t* x, int32_t M, const int32_t* mask,
+                                     int64_t mask_words, int64_t mask_stride_words,
+                                     void* out_partial, uint16_t* out_logits, int32_t* dev_err,
+                                     void* ws, size_t ws_bytes, void* stream);
+mtp_status mtp_argmax_merge_partials(const void* partials, int32_t n_parts, int32_t M,
+                                     int32_t* out_idx, float* out_val, float* out_logprob,
+                                     int32_t* dev_err, void* stream);
+
+/* ---------------------------------------------------------------------------------
  * mtp_prefill_kv -- the drafter-context prefill: the drafter's K/V cache rows for R
  * prompt rows, written as E4M3 codes into a paged cache.
  * Source: [mtp_head.rs] drafter-prefill docs (the drafter's K/V for prompt row i are a

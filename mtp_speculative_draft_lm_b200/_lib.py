@@ -35,6 +35,7 @@ EXPORTS = (
     "mtp_abi_version", "mtp_status_str", "mtp_devflags_status",
     "mtp_quantize_fp8", "mtp_quantize_nvfp4_ws_bytes", "mtp_quantize_nvfp4",
     "mtp_combine", "mtp_lm_head_ws_bytes", "mtp_lm_head_argmax", "mtp_lm_head_argmax_lp",
+    "mtp_lm_head_shard_partial", "mtp_argmax_merge_partials",
     "mtp_debug_encode_e4m3", "mtp_debug_encode_e2m1", "mtp_nvfp4_scale_pitch",
     "mtp_noalloc_scratch_bytes", "mtp_lm_head_argmax_noalloc",
     "mtp_prefill_ws_bytes", "mtp_prefill_kv", "mtp_debug_gemm_bf16", "mtp_debug_kv_write",
@@ -74,6 +75,9 @@ _SIGS = {
                                      _P, _SZ, _P]),
     "mtp_lm_head_argmax_lp": (C.c_int, [_W, _I64, _P, _I32, _P, _I64, _I64, _P, _P, _P, _P,
                                         _P, _P, _SZ, _P]),
+    "mtp_lm_head_shard_partial": (C.c_int, [_W, _I64, _I64, _P, _I32, _P, _I64, _I64, _P, _P,
+                                            _P, _P, _SZ, _P]),
+    "mtp_argmax_merge_partials": (C.c_int, [_P, _I32, _I32, _P, _P, _P, _P, _P]),
     "mtp_prefill_ws_bytes": (_SZ, [_I64, _I32, _I32, _I32]),
     "mtp_prefill_kv": (C.c_int, [_P, _I64, _P, _P, _I64, _I32, _P, _P, C.c_float, _P, _P, _P,
                                  _I32, _I32, C.c_float, _P, _I64, _P, _I64, _I32, _P, _P, _I64,
@@ -195,6 +199,25 @@ def mtp_lm_head_argmax_lp(head, n_eff, x, M, mask, mask_words, mask_stride_words
                                         _ptr(out_logits), _ptr(dev_err), _ptr(ws), ws_bytes,
                                         _stream(stream)),
            "mtp_lm_head_argmax_lp")
+
+
+def mtp_lm_head_shard_partial(shard, n_eff, row_offset, x, M, mask, mask_words,
+                              mask_stride_words, out_partial, out_logits, dev_err, ws, ws_bytes,
+                              stream=None):
+    _check(load().mtp_lm_head_shard_partial(C.byref(shard) if shard is not None else None,
+                                            n_eff, row_offset, _ptr(x), M, _ptr(mask),
+                                            mask_words, mask_stride_words, _ptr(out_partial),
+                                            _ptr(out_logits), _ptr(dev_err), _ptr(ws), ws_bytes,
+                                            _stream(stream)),
+           "mtp_lm_head_shard_partial")
+
+
+def mtp_argmax_merge_partials(partials, n_parts, M, out_idx, out_val, out_logprob, dev_err,
+                              stream=None):
+    _check(load().mtp_argmax_merge_partials(_ptr(partials), n_parts, M, _ptr(out_idx),
+                                            _ptr(out_val), _ptr(out_logprob), _ptr(dev_err),
+                                            _stream(stream)),
+           "mtp_argmax_merge_partials")
 
 
 def mtp_prefill_ws_bytes(chunk_rows, h, nkv, hd) -> int:

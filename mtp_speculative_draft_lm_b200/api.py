@@ -108,6 +108,78 @@ class LmHead:
         return (idx, val, lg, lp) if logprob else (idx, val, lg)
 
 
+def table_rows(table: Table, r0: int, r1: int) -> Table:
+    """Rows [r0, r1) of a table as a table of its own (views: rows are contiguous, so a
+    vocab shard is a base-pointer offset and a smaller n)."""
+    rs = table.row_scale[r0:r1] if table.row_scale is not None else None
+    bs = table.block_scale[r0:r1] if table.block_scale is not None else None
+    return Table(table.fmt, r1 - r0, table.k, table.data[r0:r1], row_scale=rs, block_scale=bs,
+                 global_scale=table.global_scale)
+
+
+def shard_range(n: int, world: int, rank: int, align: int = 16) -> tuple[int, int]:
+    """(row_offset, rows) of rank's vocab shard: equal contiguous ranges in units of
+    `align` rows (the sweep's 16-row tiles), the last one shorter; empty when there are
+    more ranks than units."""
+    units = -(-n // align)
+    per = -(-units // world) * align
+    off = min(n, rank * per)
+    return off, min(n, off + per) - off
+
+
+#: a shard partial: {f32 max logit, i32 global row (INT32_MAX: none allowed), f32 sum of
+#: exp(l - max), unused}, stored as 4 float32 words per input row
+EMPTY_PARTIAL = (float("-inf"), 2147483647, 0.0)
+
+
+def exchange_partials(local: torch.Tensor, group=None) -> torch.Tensor:
+    """All-gathers every rank's [M, 4] partials into [world, M, 4] (rank-major), the one
+    collective of the vocab-sharded sweep (NCCL over NVLink on GPUs)."""
+    import torch.distributed as dist
+
+    world = dist.get_world_size(group)
+    parts = [torch.empty_like(local) for _ in range(world)]
+    dist.all_gather(parts, local.contiguous(), group=group)
+    return torch.stack(parts)
+
+
+class ShardedLmHead:
+    """The lm_head sweep + argmax split by vocab over the ranks of a process group: each
+    rank sweeps its own rows (mtp_lm_head_shard_partial), the 16-byte partials are
+    all-gathered, and every rank merges them (mtp_argmax_merge_partials)."""
+
+    def __init__(self, shard: Table | None, row_offset: int, group=None, max_m: int = 16):
+        self.shard = shard
+        self.row_offset = int(row_offset)
+        self.group = group
+        self.head = LmHead(shard, max_m=max_m) if shard is not None and shard.n > 0 else None
+
+    def argmax(self, x: torch.Tensor, mask=None, mask_words=0, mask_stride_words=0,
+               logprob=False, stream=None):
+        import torch.distributed as dist
+
+        M = x.shape[0]
+        dev = x.device
+        local = torch.empty((M, 4), dtype=torch.float32, device=dev)
+        if self.head is None:  # no rows here: an empty partial
+            local.zero_()
+            local[:, 0] = EMPTY_PARTIAL[0]
+            local.view(torch.int32)[:, 1] = EMPTY_PARTIAL[1]
+        else:
+            L.mtp_lm_head_shard_partial(self.shard.desc, self.shard.n, self.row_offset, x, M, mask,
+                                        mask_words, mask_stride_words, local, None,
+                                        self.head.dev_err, self.head.ws, self.head.ws.numel(),
+                                        stream)
+        parts = exchange_partials(local, self.group)
+        idx = torch.empty((M,), dtype=torch.int32, device=dev)
+        val = torch.empty((M,), dtype=torch.float32, device=dev)
+        lp = torch.empty((M,), dtype=torch.float32, device=dev) if logprob else None
+        err = torch.zeros((1,), dtype=torch.int32, device=dev)
+        L.mtp_argmax_merge_partials(parts, dist.get_world_size(self.group), M, idx, val, lp, err,
+                                    stream)
+        return (idx, val, lp, err) if logprob else (idx, val, err)
+
+
 def combine(embed, token_ids, hidden, w_norm_embed, w_norm_hidden, eps, fc: Table,
             out=None, dev_err=None, stream=None):
     M, h = hidden.shape

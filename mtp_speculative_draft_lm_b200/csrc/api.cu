@@ -164,10 +164,12 @@ mtp_status lm_head_impl(const mtp_weight* head, int64_t n_eff, const uint16_t* x
                         const int32_t* mask, int64_t mask_words, int64_t mask_stride_words,
                         int32_t* out_idx, float* out_val, float* out_logprob,
                         uint16_t* out_logits, int32_t* dev_err, void* ws, size_t ws_bytes,
-                        void* stream) {
+                        void* stream, void* out_partial = nullptr, int64_t row_offset = 0) {
     mtp_status st = check_weight(head);
     if (st != MTP_OK) return st;
-    if (!x || !out_idx || n_eff < 1 || n_eff > head->n) return MTP_ERR_INVALID_ARG;
+    if (!x || (!out_idx && !out_partial) || n_eff < 1 || n_eff > head->n) return MTP_ERR_INVALID_ARG;
+    if (row_offset < 0 || row_offset + n_eff > (int64_t)INT32_MAX) return MTP_ERR_INVALID_ARG;
+    if (!aligned(out_partial, 16)) return MTP_ERR_INVALID_ARG;
     if (n_eff > (int64_t)INT32_MAX || row_bytes(head) % 128) return MTP_ERR_UNSUPPORTED;
     if (M < 1 || M > kMaxM) return MTP_ERR_UNSUPPORTED;
     if (mask && (mask_words < 1 || mask_stride_words < 0)) return MTP_ERR_INVALID_ARG;
@@ -196,6 +198,8 @@ mtp_status lm_head_impl(const mtp_weight* head, int64_t n_eff, const uint16_t* x
     p.out_val = out_val;
     p.out_logits = out_logits;
     p.out_logprob = out_logprob;
+    p.out_partial = out_partial;
+    p.row_offset = row_offset;
     p.dev_err = dev_err;
     p.ticket = static_cast<uint32_t*>(ws);
     p.partials = static_cast<uint8_t*>(ws) + kTicketBytes;
@@ -213,6 +217,29 @@ mtp_status mtp_lm_head_argmax(const mtp_weight* head, int64_t n_eff, const uint1
                               size_t ws_bytes, void* stream) {
     return lm_head_impl(head, n_eff, x, M, mask, mask_words, mask_stride_words, out_idx, out_val,
                         nullptr, out_logits, dev_err, ws, ws_bytes, stream);
+}
+
+mtp_status mtp_lm_head_shard_partial(const mtp_weight* shard, int64_t n_eff, int64_t row_offset,
+                                     const uint16_t* x, int32_t M, const int32_t* mask,
+                                     int64_t mask_words, int64_t mask_stride_words,
+                                     void* out_partial, uint16_t* out_logits, int32_t* dev_err,
+                                     void* ws, size_t ws_bytes, void* stream) {
+    if (!out_partial) return MTP_ERR_INVALID_ARG;
+    return lm_head_impl(shard, n_eff, x, M, mask, mask_words, mask_stride_words, nullptr, nullptr,
+                        nullptr, out_logits, dev_err, ws, ws_bytes, stream, out_partial,
+                        row_offset);
+}
+
+mtp_status mtp_argmax_merge_partials(const void* partials, int32_t n_parts, int32_t M,
+                                     int32_t* out_idx, float* out_val, float* out_logprob,
+                                     int32_t* dev_err, void* stream) {
+    if (!partials || !out_idx || n_parts < 1 || n_parts > 65536) return MTP_ERR_INVALID_ARG;
+    if (M < 1 || M > kMaxM) return MTP_ERR_UNSUPPORTED;
+    if (!aligned(partials, 16) || !aligned(out_idx, 4) || !aligned(out_val, 4) ||
+        !aligned(out_logprob, 4) || !aligned(dev_err, 4))
+        return MTP_ERR_INVALID_ARG;
+    return from_cuda(mtp::merge_partials_launch(partials, n_parts, M, out_idx, out_val, out_logprob,
+                                                dev_err, as_stream(stream)));
 }
 
 mtp_status mtp_lm_head_argmax_lp(const mtp_weight* head, int64_t n_eff, const uint16_t* x,

@@ -39,6 +39,8 @@ struct SweepParams {
     float* out_val;
     uint16_t* out_logits;        // bf16 [M, n] or null
     float* out_logprob;          // f32 [M] top-1 log-probability, or null
+    void* out_partial;           // vocab shard: 16-byte (max, row, sum exp) per input, or null
+    int64_t row_offset;          // vocab shard: global index of the table's first row
     uint16_t* out_y;             // mode 1: bf16 [M, n]
     int32_t* dev_err;
     // workspace (mode 0)
@@ -56,6 +58,12 @@ struct SweepLaunch {
     int grid;
     int smem_bytes;
 };
+
+// Folds n_parts 16-byte shard partials per input (rank-major [n_parts][M]) into the
+// argmax, its value and the top-1 log-probability; one warp per input.
+cudaError_t merge_partials_launch(const void* parts, int n_parts, int M, int32_t* out_idx,
+                                  float* out_val, float* out_logprob, int32_t* dev_err,
+                                  cudaStream_t s);
 
 // Picks the kernel instance and grid; returns cudaErrorInvalidValue if the staged
 // input does not fit in shared memory.

@@ -147,12 +147,14 @@ __device__ __forceinline__ void l2_prefetch_share(const void* base, int64_t byte
     }
 }
 
+// Mask bit of table row `row` (token row + row_offset: a vocab shard reads the global mask).
 __device__ __forceinline__ bool mask_allows(const SweepParams& p, int m, int64_t row) {
     if (!p.mask) return true;
-    int64_t word = row >> 5;
+    const int64_t t = row + p.row_offset;
+    int64_t word = t >> 5;
     if (word >= p.mask_words) return false;
     uint32_t bits = (uint32_t)__ldg(p.mask + (int64_t)m * p.mask_stride + word);
-    return (bits >> (row & 31)) & 1u;
+    return (bits >> (t & 31)) & 1u;
 }
 
 __device__ __forceinline__ bool row_needed(const SweepParams& p, int64_t row) {
@@ -595,7 +597,7 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
         int32_t best_i[Q];
         float fa[Q], fb[Q];  // 2^-xexp as two factors: (a fa) fb is exact for a normal result
         float se[Q];         // sum of exp(l - best_v) over the allowed rows seen
-        const bool lp = MODE == 0 && p.out_logprob != nullptr;
+        const bool lp = MODE == 0 && (p.out_logprob != nullptr || p.out_partial != nullptr);
 #pragma unroll
         for (int q = 0; q < Q; ++q) {
             best_v[q] = -INFINITY;
@@ -763,7 +765,11 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
                     bi = oi;
                 }
             }
-            if (lane == 0) {
+            if (lane == 0 && p.out_partial) {
+                // a vocab shard: the global row of its maximum (INT_MAX: nothing allowed here)
+                const int32_t gi = bi == INT_MAX ? INT_MAX : (int32_t)(bi + p.row_offset);
+                reinterpret_cast<Partial*>(p.out_partial)[m] = Partial{bv, gi, bs, 0.f};
+            } else if (lane == 0) {
                 const bool empty = bi == INT_MAX;
                 if (empty) {
                     bi = 0;
@@ -1072,6 +1078,57 @@ size_t sweep_smem_bytes(int M, int64_t k, int fmt, int* kpad_out) {
 }
 
 int sweep_max_grid() { return kMaxGrid; }
+
+namespace {
+
+// One warp per input: lane l folds parts l, l + 32, ... in order, then a fixed shuffle
+// tree; ties go to the lowest row, so the argmax does not depend on the order.
+__global__ void __launch_bounds__(32) merge_partials_kernel(const Partial* parts, int n_parts, int M,
+                                                            int32_t* out_idx, float* out_val,
+                                                            float* out_logprob, int32_t* dev_err) {
+    const int m = blockIdx.x, lane = threadIdx.x;
+    float bv = -INFINITY, bs = 0.f;
+    int32_t bi = INT_MAX;
+    for (int r = lane; r < n_parts; r += 32) {
+        const float4 e = __ldg(reinterpret_cast<const float4*>(parts + (int64_t)r * M + m));
+        const int32_t ei = __float_as_int(e.y);
+        if (ei == INT_MAX) continue;  // nothing allowed in that shard
+        float v = bv;
+        lse_merge(v, bs, e.x, e.z);
+        if (e.x > bv || (e.x == bv && ei < bi)) {
+            bv = e.x;
+            bi = ei;
+        }
+    }
+    for (int o = 16; o; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int32_t oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        const float os = __shfl_xor_sync(0xffffffffu, bs, o);
+        float v = bv;
+        lse_merge(v, bs, ov, os);
+        if (ov > bv || (ov == bv && oi < bi)) {
+            bv = ov;
+            bi = oi;
+        }
+    }
+    if (lane == 0) {
+        const bool empty = bi == INT_MAX;
+        if (empty) raise_flag(dev_err, DEVFLAG_EMPTY_MASK);
+        out_idx[m] = empty ? 0 : bi;
+        if (out_val) out_val[m] = empty ? -INFINITY : bv;
+        if (out_logprob) out_logprob[m] = empty ? -INFINITY : -logf(bs);
+    }
+}
+
+}  // namespace
+
+cudaError_t merge_partials_launch(const void* parts, int n_parts, int M, int32_t* out_idx,
+                                  float* out_val, float* out_logprob, int32_t* dev_err,
+                                  cudaStream_t s) {
+    merge_partials_kernel<<<M, 32, 0, s>>>(static_cast<const Partial*>(parts), n_parts, M, out_idx,
+                                            out_val, out_logprob, dev_err);
+    return cudaGetLastError();
+}
 
 cudaError_t sweep_launch(const SweepParams& p, int fmt, int mode, cudaStream_t s,
                          SweepLaunch* info) {

@@ -131,6 +131,31 @@ def test_lm_head_lp_rejects(lib):
     assert wsb == 256 + 16 * 16 * 1024 and L.mtp_noalloc_scratch_bytes() == wsb
 
 
+def test_shard_and_merge_rejects(lib):
+    head = weight()
+    wsb = L.mtp_lm_head_ws_bytes(head, 100, 1)
+
+    def shard(part, off=0, n_eff=100):
+        return st("mtp_lm_head_shard_partial", C.byref(head), n_eff, off, B2, 1, None, 0, 0,
+                  part, None, None, 0x40000, wsb, None)
+
+    assert shard(None) == L.MTP_ERR_INVALID_ARG          # the partial output is required
+    assert shard(OUT + 8) == L.MTP_ERR_INVALID_ARG       # 16-byte aligned partials
+    assert shard(OUT, off=-16) == L.MTP_ERR_INVALID_ARG
+    assert shard(OUT, off=2**31 - 50) == L.MTP_ERR_INVALID_ARG  # global rows must fit i32
+    assert shard(OUT, n_eff=101) == L.MTP_ERR_INVALID_ARG
+
+    def merge(parts, n, M, idx=OUT):
+        return st("mtp_argmax_merge_partials", parts, n, M, idx, None, None, None, None)
+
+    assert merge(None, 2, 1) == L.MTP_ERR_INVALID_ARG
+    assert merge(A, 0, 1) == L.MTP_ERR_INVALID_ARG
+    assert merge(A, 2, 1, idx=None) == L.MTP_ERR_INVALID_ARG
+    assert merge(A + 8, 2, 1) == L.MTP_ERR_INVALID_ARG
+    assert merge(A, 2, 0) == L.MTP_ERR_UNSUPPORTED
+    assert merge(A, 2, 17) == L.MTP_ERR_UNSUPPORTED
+
+
 def test_combine_rejects(lib):
     fc = weight(n=32, k=64)
     args = [A, 50, B2, B2, 1, 32, OUT, OUT, 1e-6, C.byref(fc), OUT, None, None]
