@@ -132,15 +132,18 @@ def shard_range(n: int, world: int, rank: int, align: int = 16) -> tuple[int, in
 EMPTY_PARTIAL = (float("-inf"), 2147483647, 0.0)
 
 
-def exchange_partials(local: torch.Tensor, group=None) -> torch.Tensor:
+def exchange_partials(local: torch.Tensor, group=None, out: torch.Tensor | None = None) -> torch.Tensor:
     """All-gathers every rank's [M, 4] partials into [world, M, 4] (rank-major), the one
     collective of the vocab-sharded sweep (NCCL over NVLink on GPUs)."""
     import torch.distributed as dist
 
     world = dist.get_world_size(group)
-    parts = [torch.empty_like(local) for _ in range(world)]
-    dist.all_gather(parts, local.contiguous(), group=group)
-    return torch.stack(parts)
+    if out is None:
+        out = torch.empty((world,) + tuple(local.shape), dtype=local.dtype, device=local.device)
+    # gathered along dim 0 ([world * M, 4]); viewed back as [world, M, 4]
+    flat = out.view((world * local.shape[0],) + tuple(local.shape[1:]))
+    dist.all_gather_into_tensor(flat, local.contiguous(), group=group)
+    return out
 
 
 class ShardedLmHead:
@@ -153,14 +156,30 @@ class ShardedLmHead:
         self.row_offset = int(row_offset)
         self.group = group
         self.head = LmHead(shard, max_m=max_m) if shard is not None and shard.n > 0 else None
+        self._bufs = {}
+
+    def _buffers(self, M: int, dev):
+        import torch.distributed as dist
+
+        if M not in self._bufs:
+            world = dist.get_world_size(self.group)
+            self._bufs[M] = dict(
+                local=torch.empty((M, 4), dtype=torch.float32, device=dev),
+                parts=torch.empty((world, M, 4), dtype=torch.float32, device=dev),
+                idx=torch.empty((M,), dtype=torch.int32, device=dev),
+                val=torch.empty((M,), dtype=torch.float32, device=dev),
+                lp=torch.empty((M,), dtype=torch.float32, device=dev),
+                err=torch.zeros((1,), dtype=torch.int32, device=dev), world=world)
+        return self._bufs[M]
 
     def argmax(self, x: torch.Tensor, mask=None, mask_words=0, mask_stride_words=0,
                logprob=False, stream=None):
-        import torch.distributed as dist
-
+        """Returns (idx, val, err) or (idx, val, logprob, err): the merged result, the
+        same on every rank; err is the merge's device error word. The returned tensors
+        are reused by the next call with the same M."""
         M = x.shape[0]
-        dev = x.device
-        local = torch.empty((M, 4), dtype=torch.float32, device=dev)
+        b = self._buffers(M, x.device)
+        local = b["local"]
         if self.head is None:  # no rows here: an empty partial
             local.zero_()
             local[:, 0] = EMPTY_PARTIAL[0]
@@ -170,14 +189,12 @@ class ShardedLmHead:
                                         mask_words, mask_stride_words, local, None,
                                         self.head.dev_err, self.head.ws, self.head.ws.numel(),
                                         stream)
-        parts = exchange_partials(local, self.group)
-        idx = torch.empty((M,), dtype=torch.int32, device=dev)
-        val = torch.empty((M,), dtype=torch.float32, device=dev)
-        lp = torch.empty((M,), dtype=torch.float32, device=dev) if logprob else None
-        err = torch.zeros((1,), dtype=torch.int32, device=dev)
-        L.mtp_argmax_merge_partials(parts, dist.get_world_size(self.group), M, idx, val, lp, err,
+        exchange_partials(local, self.group, out=b["parts"])
+        b["err"].zero_()
+        lp = b["lp"] if logprob else None
+        L.mtp_argmax_merge_partials(b["parts"], b["world"], M, b["idx"], b["val"], lp, b["err"],
                                     stream)
-        return (idx, val, lp, err) if logprob else (idx, val, err)
+        return (b["idx"], b["val"], lp, b["err"]) if logprob else (b["idx"], b["val"], b["err"])
 
 
 def combine(embed, token_ids, hidden, w_norm_embed, w_norm_hidden, eps, fc: Table,
