@@ -165,10 +165,27 @@ __device__ __forceinline__ bool row_needed(const SweepParams& p, int64_t row) {
     return false;
 }
 
-// True when some row of the tile is allowed for some input (whole warp calls it).
-__device__ __forceinline__ bool tile_needed(const SweepParams& p, int64_t tile, int lane) {
-    const bool need = lane < kTileRows && row_needed(p, tile * kTileRows + lane);
-    return __ballot_sync(0xffffffffu, need) != 0u;
+// A tile's 16 rows are 16 consecutive mask bits of each input: lane m < M loads input m's
+// one or two words (issued early; tile_mask_need consumes them later).
+__device__ __forceinline__ void tile_mask_load(const SweepParams& p, int64_t tile, int lane,
+                                               uint32_t& w0, uint32_t& w1) {
+    w0 = w1 = 0u;
+    if (lane >= p.M) return;
+    const int64_t t0 = tile * kTileRows + p.row_offset;
+    const int64_t wi = t0 >> 5;
+    const int32_t* row = p.mask + (int64_t)lane * p.mask_stride;
+    if (wi < p.mask_words) w0 = (uint32_t)__ldg(row + wi);
+    if ((t0 & 31) > 16 && wi + 1 < p.mask_words) w1 = (uint32_t)__ldg(row + wi + 1);
+}
+
+// True when some row of the tile (below n) is allowed for some input (whole warp).
+__device__ __forceinline__ bool tile_mask_need(const SweepParams& p, int64_t tile, int lane,
+                                               uint32_t w0, uint32_t w1) {
+    const int64_t t0 = tile * kTileRows + p.row_offset;
+    uint32_t bits = (uint32_t)((((uint64_t)w1 << 32) | w0) >> (t0 & 31)) & 0xFFFFu;
+    const int64_t rows = p.n - tile * kTileRows;
+    if (rows < kTileRows) bits &= (1u << (rows > 0 ? rows : 0)) - 1u;
+    return __any_sync(0xffffffffu, lane < p.M && bits != 0u);
 }
 
 // Reductions over the CW compute warps (named barrier 1).
@@ -524,54 +541,71 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
         int64_t issued = 0;
         const uint32_t tx = code_stage_bytes(segs) + (FMT == 2 ? scale_stage_bytes(segs) : 0);
         bool stop = false;
-        int64_t tile = t_begin;
+        // the NC stages of one tile, each tagged with the tile
+        auto issue_tile = [&](int64_t tile) {
+            for (int ch = 0; ch < NC; ++ch) {
+                if (!mbar_wait_bounded(&empty[slot], phase ^ 1u, abort_flag)) {
+                    stop = true;
+                    return;
+                }
+                if (lane == 0) {
+                    uint8_t* dst = ring + (size_t)slot * stage_bytes;
+                    slot_tile[slot] = (int)tile;
+                    mbar_arrive_expect_tx(&full[slot], tx);
+                    tma_load_3d(dst, &map_codes, 0, (int)(tile * kTileRows), ch * segs, &full[slot]);
+                    if (FMT == 2)
+                        tma_load_2d(dst + code_stage_bytes(segs), &map_scales, ch * 8 * segs,
+                                    (int)(tile * kTileRows), &full[slot]);
+                }
+                __syncwarp();
+                ++issued;
+                if (++slot == S) {
+                    slot = 0;
+                    phase ^= 1u;
+                }
+            }
+        };
         // the next tile is claimed one tile ahead, so the atomic's latency overlaps the
         // waits for free ring slots
-        // The first tile's stages read only the table, so they go out before waiting for
-        // the previous grid (unless a mask, which that grid may write, decides them).
-        int64_t next = 0;
-        bool waited = p.mask != nullptr;
-        if (waited) pdl_wait();
-        while (tile < t_end && !stop) {
-            if (tile_needed(p, tile, lane)) {
-                for (int ch = 0; ch < NC; ++ch) {
-                    if (!mbar_wait_bounded(&empty[slot], phase ^ 1u, abort_flag)) {
-                        stop = true;
-                        break;
-                    }
-                    if (lane == 0) {
-                        uint8_t* dst = ring + (size_t)slot * stage_bytes;
-                        slot_tile[slot] = (int)tile;
-                        mbar_arrive_expect_tx(&full[slot], tx);
-                        tma_load_3d(dst, &map_codes, 0, (int)(tile * kTileRows), ch * segs, &full[slot]);
-                        if (FMT == 2)
-                            tma_load_2d(dst + code_stage_bytes(segs), &map_scales, ch * 8 * segs,
-                                        (int)(tile * kTileRows), &full[slot]);
-                    }
-                    __syncwarp();
-                    ++issued;
-                    if (++slot == S) {
-                        slot = 0;
-                        phase ^= 1u;
-                    }
+        int64_t tile = t_begin;
+        int64_t pending = 0;
+        if (!p.mask) {
+            // The first tile's stages read only the table, so they go out before waiting
+            // for the previous grid.
+            issue_tile(tile);
+            pdl_wait();
+            if (dyn && lane == 0) pending = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
+            while (!stop) {
+                tile = dyn ? __shfl_sync(0xffffffffu, pending, 0) : tile + 1;
+                if (tile >= t_end) break;
+                if (dyn && lane == 0) pending = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
+                issue_tile(tile);
+            }
+        } else {
+            // With a mask (which the previous grid may write) everything waits for it. The
+            // mask words of the following tile are loaded while this tile's stages go out.
+            pdl_wait();
+            if (dyn && lane == 0) pending = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
+            uint32_t w0, w1;
+            tile_mask_load(p, tile, lane, w0, w1);
+            bool need = tile_mask_need(p, tile, lane, w0, w1);
+            while (tile < t_end && !stop) {
+                const int64_t tnext = dyn ? __shfl_sync(0xffffffffu, pending, 0) : tile + 1;
+                if (dyn && lane == 0 && tnext < t_end)
+                    pending = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
+                uint32_t n0 = 0u, n1 = 0u;
+                if (tnext < t_end) tile_mask_load(p, tnext, lane, n0, n1);
+                if (need) {
+                    issue_tile(tile);
+                } else if (MODE == 0 && p.out_logits) {
+                    // every row is masked out for every input: logits -inf, nothing to load
+                    const int64_t row = tile * kTileRows + (lane & 15);
+                    if (row < p.n)
+                        for (int col = lane >> 4; col < M; col += 2)
+                            p.out_logits[(int64_t)col * p.n + row] = 0xFF80u;
                 }
-            } else if (MODE == 0 && p.out_logits) {
-                // every row is masked out for every input: logits -inf, nothing to load
-                const int64_t row = tile * kTileRows + (lane & 15);
-                if (row < p.n)
-                    for (int col = lane >> 4; col < M; col += 2)
-                        p.out_logits[(int64_t)col * p.n + row] = 0xFF80u;
-            }
-            if (!waited) {
-                pdl_wait();
-                waited = true;
-            }
-            if (dyn) {
-                if (tile == t_begin && lane == 0) next = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
-                tile = __shfl_sync(0xffffffffu, next, 0);
-                if (lane == 0 && tile < t_end) next = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
-            } else {
-                ++tile;
+                tile = tnext;
+                need = tile < t_end && tile_mask_need(p, tile, lane, n0, n1);
             }
         }
         // Leave no copy in flight: wait for the last stages issued (bounded). This comes
