@@ -263,8 +263,13 @@ mtp_status mtp_argmax_merge_partials(const void* partials, int32_t n_parts, int3
  *   hidden (device) bf16 [R, h]; w_norm_* (device) bf16 [h]; fc (device) bf16 [h, 2h];
  *   wk, wv (device) bf16 [nkv * hd, h]; block_table (device) i32 [n_table];
  *   k_cache, v_cache (device) u8 [num_blocks, block_size, nkv, hd], written in place;
- *   ws (device) >= mtp_prefill_ws_bytes(min(chunk_rows, R), h, nkv, hd) bytes, 1 KB
- *   aligned (per chunk: the concat rows, fc output and a RoPE table).
+ *   ws (device) mtp_prefill_ws_bytes(min(chunk_rows, R), h, nkv, hd) bytes, 1 KB
+ *   aligned: two lanes of one chunk's concat rows, fc output and RoPE table. Half of
+ *   that (one lane) is the minimum (MTP_ERR_WORKSPACE below it) and runs the chunks one
+ *   after another on `stream`; with both lanes, consecutive chunks run side by side on
+ *   two library-owned streams (created per device on first use, kept until the process
+ *   exits), forked from and joined back into `stream` with events, so the call still
+ *   orders like one operation on `stream` and can be captured in a CUDA graph.
  * Rows run in chunks of chunk_rows (the GEMMs' M). Requires h % 256 == 0,
  * hd in {64, 128, 256}, nkv * hd % 256 == 0, k_scale, v_scale > 0.
  * ------------------------------------------------------------------------------ */

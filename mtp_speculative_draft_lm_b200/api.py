@@ -207,6 +207,14 @@ def combine(embed, token_ids, hidden, w_norm_embed, w_norm_hidden, eps, fc: Tabl
     return out
 
 
+def aligned_empty(nbytes: int, align: int, device) -> torch.Tensor:
+    """A uint8 device buffer of nbytes whose address is a multiple of align (torch only
+    promises 512 bytes)."""
+    raw = torch.empty((nbytes + align,), dtype=torch.uint8, device=device)
+    off = (-raw.data_ptr()) % align
+    return raw[off: off + nbytes]
+
+
 def prefill_kv(inputs: dict, k_cache: torch.Tensor, v_cache: torch.Tensor, chunk_rows: int = 2048,
                ws: torch.Tensor | None = None, dev_err: torch.Tensor | None = None, stream=None):
     """Drafter-context prefill over device tensors named as in synth.prefill_inputs."""
@@ -216,7 +224,7 @@ def prefill_kv(inputs: dict, k_cache: torch.Tensor, v_cache: torch.Tensor, chunk
     chunk = min(int(chunk_rows), R)
     nbytes = L.mtp_prefill_ws_bytes(chunk, h, nkv, hd)
     if ws is None:
-        ws = torch.empty((nbytes,), dtype=torch.uint8, device=k_cache.device)
+        ws = aligned_empty(nbytes, 1024, k_cache.device)
     L.mtp_prefill_kv(d["embed"], d["embed"].shape[0], d["tokens"], d["hidden"], R, h,
                      d["w_norm_embed"], d["w_norm_hidden"], d["eps"], d["fc"], d["wk"], d["wv"],
                      nkv, hd, d["rope_base"], d["rope_pos"], int(d["cache_start"]),

@@ -285,7 +285,7 @@ mtp_status mtp_prefill_kv(const uint16_t* embed, int64_t vocab, const int32_t* t
         !aligned(rope_pos, 4) || !aligned(block_table, 4) || !aligned(dev_err, 4))
         return MTP_ERR_INVALID_ARG;
     const int64_t chunk = chunk_rows < R ? chunk_rows : R;
-    if (!ws || !aligned(ws, 1024) || ws_bytes < mtp::prefill_ws_bytes(chunk, h, nkv, hd))
+    if (!ws || !aligned(ws, 1024) || ws_bytes < mtp::prefill_lane_bytes(chunk, h, nkv, hd))
         return MTP_ERR_WORKSPACE;
     mtp::PrefillArgs a{};
     a.embed = embed;
@@ -315,6 +315,7 @@ mtp_status mtp_prefill_kv(const uint16_t* embed, int64_t vocab, const int32_t* t
     a.v_scale = v_scale;
     a.chunk_rows = chunk;
     a.ws = ws;
+    a.ws_bytes = ws_bytes;
     a.dev_err = dev_err;
     return from_cuda(mtp::prefill_launch(a, as_stream(stream)));
 }

@@ -108,8 +108,12 @@ struct PrefillArgs {
     float k_scale, v_scale;
     int64_t chunk_rows;
     void* ws;
+    size_t ws_bytes;
     int32_t* dev_err;
 };
+// One chunk's buffers (concat rows, fc output, RoPE table); the workspace holds two such
+// lanes so that consecutive chunks can run side by side.
+size_t prefill_lane_bytes(int64_t chunk_rows, int32_t h, int32_t nkv, int32_t hd);
 size_t prefill_ws_bytes(int64_t chunk_rows, int32_t h, int32_t nkv, int32_t hd);
 cudaError_t prefill_launch(const PrefillArgs& a, cudaStream_t s);
 cudaError_t gemm_bf16_launch(const uint16_t* A, const uint16_t* B, uint16_t* C, int M, int N,

@@ -445,64 +445,137 @@ cudaError_t launch_gemm(const GemmParams& p0, const CUtensorMap& ma, const CUten
 
 }  // namespace
 
-size_t prefill_ws_bytes(int64_t chunk_rows, int32_t h, int32_t nkv, int32_t hd) {
+size_t prefill_lane_bytes(int64_t chunk_rows, int32_t h, int32_t nkv, int32_t hd) {
     (void)nkv;
     auto up = [](size_t b) { return (b + 1023) & ~(size_t)1023; };
     return up((size_t)chunk_rows * 2 * h * 2) + up((size_t)chunk_rows * h * 2) +
            up((size_t)chunk_rows * (hd / 2) * sizeof(float2));
 }
 
-cudaError_t prefill_launch(const PrefillArgs& a, cudaStream_t s) {
+size_t prefill_ws_bytes(int64_t chunk_rows, int32_t h, int32_t nkv, int32_t hd) {
+    return 2 * prefill_lane_bytes(chunk_rows, h, nkv, hd);
+}
+
+namespace {
+
+// Two streams per device on which alternate chunks run: a chunk's fc GEMM (320 tiles of
+// 128 x 256 at 2,048 rows x hidden 5,120) ends in a partial wave on 148 SMs, and the k/v
+// GEMM and the prologue leave SMs idle too; chunks are independent, so the next chunk's
+// kernels fill those SMs. Created on first use and kept for the life of the process.
+struct ChunkLanes {
+    cudaStream_t s[2] = {nullptr, nullptr};
+    cudaEvent_t fork = nullptr, join[2] = {nullptr, nullptr};
+};
+constexpr int kMaxLaneDevices = 64;
+ChunkLanes g_lanes[kMaxLaneDevices];
+std::mutex g_lane_mutex;  // held while a call forks and joins (events are shared)
+
+cudaError_t lanes_for_current_device(ChunkLanes** out) {
+    int dev = 0;
+    cudaError_t e;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxLaneDevices) return cudaErrorInvalidDevice;
+    ChunkLanes& L = g_lanes[dev];
+    if (!L.fork) {
+        for (int i = 0; i < 2; ++i) {
+            if ((e = cudaStreamCreateWithFlags(&L.s[i], cudaStreamNonBlocking)) != cudaSuccess) return e;
+            if ((e = cudaEventCreateWithFlags(&L.join[i], cudaEventDisableTiming)) != cudaSuccess)
+                return e;
+        }
+        if ((e = cudaEventCreateWithFlags(&L.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
+    }
+    *out = &L;
+    return cudaSuccess;
+}
+
+// One chunk: prologue (gather, norms, concat, RoPE table), fc GEMM, k/v GEMM with the
+// RoPE + E4M3 + paged-write epilogue, using one lane of the workspace.
+cudaError_t prefill_chunk(const PrefillArgs& a, int64_t r0, int rows, uint8_t* lane,
+                          const CUtensorMap& m_fc, const CUtensorMap& m_wk, const CUtensorMap& m_wv,
+                          cudaStream_t s) {
     auto up = [](size_t b) { return (b + 1023) & ~(size_t)1023; };
-    uint8_t* ws = static_cast<uint8_t*>(a.ws);
-    uint16_t* cbuf = reinterpret_cast<uint16_t*>(ws);
-    uint16_t* ybuf = reinterpret_cast<uint16_t*>(ws + up((size_t)a.chunk_rows * 2 * a.h * 2));
+    uint16_t* cbuf = reinterpret_cast<uint16_t*>(lane);
+    uint16_t* ybuf = reinterpret_cast<uint16_t*>(lane + up((size_t)a.chunk_rows * 2 * a.h * 2));
     float2* csbuf = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(ybuf) +
                                               up((size_t)a.chunk_rows * a.h * 2));
+    const int kvd = a.nkv * a.hd;
+    cudaError_t e;
+    prefill_prologue_kernel<<<rows, kPrologueThreads, 0, s>>>(
+        a.embed, a.vocab, a.tokens, a.hidden, a.h, a.w_norm_embed, a.w_norm_hidden, a.eps,
+        a.rope_pos, a.rope_base, a.hd, r0, cbuf, csbuf, a.dev_err);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    CUtensorMap m_c, m_y;
+    if ((e = make_operand_map(&m_c, cbuf, rows, 2 * (int64_t)a.h, BM)) != cudaSuccess) return e;
+    if ((e = make_operand_map(&m_y, ybuf, rows, a.h, BM)) != cudaSuccess) return e;
+    GemmParams g1{};
+    g1.M = rows;
+    g1.N = a.h;
+    g1.K = 2 * a.h;
+    g1.C = ybuf;
+    g1.ldc = a.h;
+    g1.dev_err = a.dev_err;
+    if ((e = launch_gemm<0>(g1, m_c, m_fc, m_fc, s)) != cudaSuccess) return e;
+    GemmParams g2{};
+    g2.M = rows;
+    g2.N = 2 * kvd;
+    g2.K = a.h;
+    g2.nkv = a.nkv;
+    g2.hd = a.hd;
+    g2.rope_cs = csbuf;
+    g2.row0 = r0;
+    g2.cache_start = a.cache_start;
+    g2.block_table = a.block_table;
+    g2.n_table = a.n_table;
+    g2.block_size = a.block_size;
+    g2.num_blocks = a.num_blocks;
+    g2.k_cache = a.k_cache;
+    g2.v_cache = a.v_cache;
+    g2.k_scale = a.k_scale;
+    g2.v_scale = a.v_scale;
+    g2.dev_err = a.dev_err;
+    return launch_gemm<1>(g2, m_y, m_wk, m_wv, s);
+}
+
+}  // namespace
+
+cudaError_t prefill_launch(const PrefillArgs& a, cudaStream_t s) {
     const int kvd = a.nkv * a.hd;
     CUtensorMap m_fc, m_wk, m_wv;
     cudaError_t e;
     if ((e = make_operand_map(&m_fc, a.fc, a.h, 2 * (int64_t)a.h, BN)) != cudaSuccess) return e;
     if ((e = make_operand_map(&m_wk, a.wk, kvd, a.h, BN)) != cudaSuccess) return e;
     if ((e = make_operand_map(&m_wv, a.wv, kvd, a.h, BN)) != cudaSuccess) return e;
-    for (int64_t r0 = 0; r0 < a.R; r0 += a.chunk_rows) {
-        const int rows = (int)((a.R - r0) < a.chunk_rows ? (a.R - r0) : a.chunk_rows);
-        prefill_prologue_kernel<<<rows, kPrologueThreads, 0, s>>>(
-            a.embed, a.vocab, a.tokens, a.hidden, a.h, a.w_norm_embed, a.w_norm_hidden, a.eps,
-            a.rope_pos, a.rope_base, a.hd, r0, cbuf, csbuf, a.dev_err);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        CUtensorMap m_c, m_y;
-        if ((e = make_operand_map(&m_c, cbuf, rows, 2 * (int64_t)a.h, BM)) != cudaSuccess) return e;
-        if ((e = make_operand_map(&m_y, ybuf, rows, a.h, BM)) != cudaSuccess) return e;
-        GemmParams g1{};
-        g1.M = rows;
-        g1.N = a.h;
-        g1.K = 2 * a.h;
-        g1.C = ybuf;
-        g1.ldc = a.h;
-        g1.dev_err = a.dev_err;
-        if ((e = launch_gemm<0>(g1, m_c, m_fc, m_fc, s)) != cudaSuccess) return e;
-        GemmParams g2{};
-        g2.M = rows;
-        g2.N = 2 * kvd;
-        g2.K = a.h;
-        g2.nkv = a.nkv;
-        g2.hd = a.hd;
-        g2.rope_cs = csbuf;
-        g2.row0 = r0;
-        g2.cache_start = a.cache_start;
-        g2.block_table = a.block_table;
-        g2.n_table = a.n_table;
-        g2.block_size = a.block_size;
-        g2.num_blocks = a.num_blocks;
-        g2.k_cache = a.k_cache;
-        g2.v_cache = a.v_cache;
-        g2.k_scale = a.k_scale;
-        g2.v_scale = a.v_scale;
-        g2.dev_err = a.dev_err;
-        if ((e = launch_gemm<1>(g2, m_y, m_wk, m_wv, s)) != cudaSuccess) return e;
+    const size_t lane_bytes = prefill_lane_bytes(a.chunk_rows, a.h, a.nkv, a.hd);
+    uint8_t* ws = static_cast<uint8_t*>(a.ws);
+    const bool two = a.R > a.chunk_rows && a.ws_bytes >= 2 * lane_bytes;
+    if (!two) {  // one lane: the chunks in order on the caller's stream
+        for (int64_t r0 = 0; r0 < a.R; r0 += a.chunk_rows) {
+            const int rows = (int)((a.R - r0) < a.chunk_rows ? (a.R - r0) : a.chunk_rows);
+            if ((e = prefill_chunk(a, r0, rows, ws, m_fc, m_wk, m_wv, s)) != cudaSuccess) return e;
+        }
+        return cudaSuccess;
     }
-    return cudaSuccess;
+    // two lanes: chunk i runs on lane stream i % 2 with workspace lane i % 2, forked from
+    // and joined back into the caller's stream (the same pattern works under capture)
+    std::lock_guard<std::mutex> lock(g_lane_mutex);
+    ChunkLanes* L = nullptr;
+    if ((e = lanes_for_current_device(&L)) != cudaSuccess) return e;
+    if ((e = cudaEventRecord(L->fork, s)) != cudaSuccess) return e;
+    for (int i = 0; i < 2; ++i)
+        if ((e = cudaStreamWaitEvent(L->s[i], L->fork, 0)) != cudaSuccess) return e;
+    cudaError_t err = cudaSuccess;
+    int64_t i = 0;
+    for (int64_t r0 = 0; r0 < a.R && err == cudaSuccess; r0 += a.chunk_rows, ++i) {
+        const int rows = (int)((a.R - r0) < a.chunk_rows ? (a.R - r0) : a.chunk_rows);
+        err = prefill_chunk(a, r0, rows, ws + (size_t)(i & 1) * lane_bytes, m_fc, m_wk, m_wv,
+                            L->s[i & 1]);
+    }
+    // join even after a failed launch, so the caller's stream stays ordered after both lanes
+    for (int j = 0; j < 2; ++j) {
+        if ((e = cudaEventRecord(L->join[j], L->s[j])) != cudaSuccess) return e;
+        if ((e = cudaStreamWaitEvent(s, L->join[j], 0)) != cudaSuccess) return e;
+    }
+    return err;
 }
 
 cudaError_t gemm_bf16_launch(const uint16_t* A, const uint16_t* B, uint16_t* C, int M, int N,

@@ -219,6 +219,10 @@ def test_prefill_rejects(lib):
     assert st("mtp_prefill_kv", *prefill_args(ws=None)) == L.MTP_ERR_WORKSPACE
     assert st("mtp_prefill_kv", *prefill_args(ws=0x100000 + 512)) == L.MTP_ERR_WORKSPACE
     assert st("mtp_prefill_kv", *prefill_args(wsb=1024)) == L.MTP_ERR_WORKSPACE
+    # the recommended workspace is two chunk lanes; one lane is the minimum
+    full = L.mtp_prefill_ws_bytes(8, 256, 2, 128)
+    assert full % 2 == 0
+    assert st("mtp_prefill_kv", *prefill_args(wsb=full // 2 - 1024)) == L.MTP_ERR_WORKSPACE
 
 
 def test_gemm_and_kv_stage_reject(lib):

@@ -187,3 +187,34 @@ def test_prefill_full_prompt_sampled_rows(orc):
         [0, 1, 2047, 2048, 32767],
         rng.choice(d["R"], 59, replace=False)]))
     check_rows(orc, d, kc, vc, rows)
+
+
+def test_prefill_lanes_and_graph_capture_agree(orc):
+    """Two workspace lanes (consecutive chunks side by side on two streams), one lane (in
+    order on the caller's stream) and a CUDA-graph capture of the two-lane call write the
+    same cache bytes; the rows match the oracle."""
+    d = synth.prefill_inputs(seed=81, R=700, vocab=500, h=256, nkv=2, hd=128)
+    dev = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    nb, chunk = int(d["num_blocks"]), 128
+    full = L.mtp_prefill_ws_bytes(chunk, 256, 2, 128)
+    outs = []
+    for nbytes in (full, full // 2):
+        kc, vc = new_caches(nb, 16, 2, 128)
+        ws = api.aligned_empty(nbytes, 1024, "cuda")
+        api.prefill_kv(dev, kc, vc, chunk_rows=chunk, ws=ws)
+        torch.cuda.synchronize()
+        outs.append((kc.cpu().numpy(), vc.cpu().numpy()))
+    assert np.array_equal(outs[0][0], outs[1][0]) and np.array_equal(outs[0][1], outs[1][1])
+    kc, vc = new_caches(nb, 16, 2, 128)
+    ws = api.aligned_empty(full, 1024, "cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            api.prefill_kv(dev, kc, vc, chunk_rows=chunk, ws=ws)
+    g.replay()
+    torch.cuda.synchronize()
+    assert np.array_equal(kc.cpu().numpy(), outs[0][0])
+    assert np.array_equal(vc.cpu().numpy(), outs[0][1])
+    check_rows(orc, d, outs[0][0], outs[0][1], np.arange(0, 700, 7))
