@@ -33,9 +33,9 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum) and
 # the sha256 of sweep.cu when it was captured; reported as null once the source changed.
 # bf16_M1: the 40,000-row capture (profiles/sweep_kernel_bf16_40k_rows.md) read
-# 327,760,128 B and wrote 4,286,720 B; reads scale with the rows swept, so a full
-# 154,880-row launch reads 327,760,128 x 154,880 / 40,000 B (writes kept unscaled).
-NCU_TRAFFIC = {"bf16_M1": (1273373935, "4afd4de0b93f304e")}
+# 327,778,304 B and wrote 4,580,096 B; reads scale with the rows swept, so a full
+# 154,880-row launch reads 327,778,304 x 154,880 / 40,000 B (writes kept unscaled).
+NCU_TRAFFIC = {"bf16_M1": (1273737689, "d68f89b3623e2e41")}
 
 
 def sweep_source_hash() -> str:
@@ -254,16 +254,16 @@ def time_e2e(head, x_host, steps, warmup, world, stream):
     M, K = x_host.shape
     dev = torch.device("cuda", torch.cuda.current_device())
     x_dev = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
-    idx = torch.empty((M,), dtype=torch.int32, device=dev)
-    val = torch.empty((M,), dtype=torch.float32, device=dev)
-    idx_h = torch.empty((M,), dtype=torch.int32).pin_memory()
-    val_h = torch.empty((M,), dtype=torch.float32).pin_memory()
+    # the index and the value land in one device buffer, read back with one copy
+    out = torch.empty((2 * M,), dtype=torch.int32, device=dev)
+    idx, val = out[:M], out[M:].view(torch.float32)
+    out_h = torch.empty((2 * M,), dtype=torch.int32).pin_memory()
+    idx_h = out_h[:M]
 
     def step():
         x_dev.copy_(x_host, non_blocking=True)
         head(x_dev, idx, val, stream=stream)
-        idx_h.copy_(idx, non_blocking=True)
-        val_h.copy_(val, non_blocking=True)
+        out_h.copy_(out, non_blocking=True)
 
     with torch.cuda.stream(stream):
         for _ in range(warmup):
