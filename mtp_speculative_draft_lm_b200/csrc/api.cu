@@ -126,7 +126,7 @@ mtp_status mtp_combine(const uint16_t* embed, int64_t vocab, const int32_t* toke
         !aligned(w_norm_embed, 4) || !aligned(w_norm_hidden, 4) || !aligned(token_ids, 4) ||
         !aligned(dev_err, 4))
         return MTP_ERR_INVALID_ARG;
-    if (mtp::sweep_smem_bytes(M, fc->k, fc->fmt, nullptr) > 227 * 1024) return MTP_ERR_UNSUPPORTED;
+    if (mtp::sweep_smem_bytes(M, fc->k, fc->fmt, nullptr, 1) > 227 * 1024) return MTP_ERR_UNSUPPORTED;
     mtp::SweepParams p{};
     p.w = static_cast<const uint8_t*>(fc->data);
     p.row_scale = fc->row_scale;
@@ -152,10 +152,10 @@ mtp_status mtp_combine(const uint16_t* embed, int64_t vocab, const int32_t* toke
 }
 
 size_t mtp_lm_head_ws_bytes(const mtp_weight* head, int64_t n_eff, int32_t M) {
-    (void)head;
     (void)n_eff;
-    (void)M;
-    return kTicketBytes + kPartialBytes * 16 * (size_t)mtp::sweep_max_grid();
+    const size_t base = kTicketBytes + kPartialBytes * 16 * (size_t)mtp::sweep_max_grid();
+    if (!head || M < 1 || M > kMaxM) return base;
+    return base + mtp::sweep_x16_bytes(M, head->k, head->fmt);
 }
 
 namespace {
@@ -179,7 +179,7 @@ mtp_status lm_head_impl(const mtp_weight* head, int64_t n_eff, const uint16_t* x
         return MTP_ERR_INVALID_ARG;
     if (!ws || !aligned(ws, 16) || ws_bytes < mtp_lm_head_ws_bytes(head, n_eff, M))
         return MTP_ERR_WORKSPACE;
-    if (mtp::sweep_smem_bytes(M, head->k, head->fmt, nullptr) > 227 * 1024)
+    if (mtp::sweep_smem_bytes(M, head->k, head->fmt, nullptr, 0) > 227 * 1024)
         return MTP_ERR_UNSUPPORTED;
     mtp::SweepParams p{};
     p.w = static_cast<const uint8_t*>(head->data);
@@ -203,6 +203,12 @@ mtp_status lm_head_impl(const mtp_weight* head, int64_t n_eff, const uint16_t* x
     p.dev_err = dev_err;
     p.ticket = static_cast<uint32_t*>(ws);
     p.partials = static_cast<uint8_t*>(ws) + kTicketBytes;
+    if (mtp::sweep_x16_bytes(M, head->k, head->fmt)) {  // the wide sweep's f16 copy of x
+        uint8_t* xb = static_cast<uint8_t*>(ws) + kTicketBytes + kPartialBytes * 16 *
+                                                                   (size_t)mtp::sweep_max_grid();
+        p.x16 = reinterpret_cast<uint16_t*>(xb);
+        p.xexp = reinterpret_cast<int32_t*>(xb + (((size_t)M * head->k * 2 + 1023) & ~(size_t)1023));
+    }
     p.num_tiles = (n_eff + 15) / 16;
     p.scale_pitch = mtp::nvfp4_scale_pitch(head->k);
     return from_cuda(mtp::sweep_launch(p, head->fmt, 0, as_stream(stream), nullptr));

@@ -41,6 +41,8 @@ struct SweepParams {
     float* out_logprob;          // f32 [M] top-1 log-probability, or null
     void* out_partial;           // vocab shard: 16-byte (max, row, sum exp) per input, or null
     int64_t row_offset;          // vocab shard: global index of the table's first row
+    uint16_t* x16;               // M > 8, quantized tables: f16 copy of x scaled per row [M, k]
+    int32_t* xexp;               // its per-row power of two [M]
     uint16_t* out_y;             // mode 1: bf16 [M, n]
     int32_t* dev_err;
     // workspace (mode 0)
@@ -69,7 +71,9 @@ cudaError_t merge_partials_launch(const void* parts, int n_parts, int M, int32_t
 // input does not fit in shared memory.
 cudaError_t sweep_launch(const SweepParams& p, int fmt, int mode, cudaStream_t s,
                          SweepLaunch* info);
-size_t sweep_smem_bytes(int M, int64_t k, int fmt, int* kpad_out);
+size_t sweep_smem_bytes(int M, int64_t k, int fmt, int* kpad_out, int mode);
+// Workspace bytes the wide sweep (mode 0, M > 8) needs for its f16 copy of x: 0 for BF16.
+size_t sweep_x16_bytes(int M, int64_t k, int fmt);
 int sweep_max_grid();
 
 // Quantizers.

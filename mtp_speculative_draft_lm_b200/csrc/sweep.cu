@@ -471,6 +471,91 @@ __device__ __forceinline__ void slab_mma_blocks(float (&acc)[4], uint4 (&xv)[4],
     acc[3] = fmaf(b23.y, d1[3], fmaf(b23.x, d0[3], acc[3]));
 }
 
+// After a CTA has published its partials: take a ticket (release before, acquire after);
+// the last CTA folds every CTA's partials in a fixed pattern and writes the outputs (or,
+// for a vocab shard, the shard's partial), then re-zeroes the ticket and the tile counter.
+__device__ void ticket_and_fold(const SweepParams& p, int lane, bool lp) {
+    const int M = p.M;
+    const Partial* parts = reinterpret_cast<const Partial*>(p.partials);
+    int last = 0;
+    if (lane == 0) last = atom_add_acq_rel_gpu(p.ticket, 1u) == gridDim.x - 1;
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (!last) return;
+    fence_acq_rel_gpu();
+    // the last CTA folds every CTA's partial: lane l reads CTAs l, l + 32, ...
+    // (independent loads in flight together), then a shuffle reduction; ties go
+    // to the lowest row index, so the result does not depend on the order
+    const int G = (int)gridDim.x;
+    constexpr int FOLD = 8;  // partials per lane in flight at a time
+    for (int m = 0; m < M; ++m) {
+        float bv = -INFINITY, bs = 0.f;
+        int32_t bi = INT_MAX;
+        for (int base = 0; base < G; base += 32 * FOLD) {
+            float qv[FOLD], qs[FOLD];
+            int32_t qi[FOLD];
+#pragma unroll
+            for (int j = 0; j < FOLD; ++j) {
+                const int b = base + lane + 32 * j;
+                qv[j] = -INFINITY;
+                qi[j] = INT_MAX;
+                qs[j] = 0.f;
+                if (b < G) {
+                    const float4 e = __ldcg(reinterpret_cast<const float4*>(parts + (int64_t)b * 16 + m));
+                    qv[j] = e.x;
+                    qi[j] = __float_as_int(e.y);
+                    qs[j] = e.z;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < FOLD; ++j) {
+                if (lp) {
+                    float v = bv;
+                    lse_merge(v, bs, qv[j], qs[j]);
+                }
+                if (qv[j] > bv || (qv[j] == bv && qi[j] < bi)) {
+                    bv = qv[j];
+                    bi = qi[j];
+                }
+            }
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int32_t oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            const float os = __shfl_xor_sync(0xffffffffu, bs, o);
+            if (lp) {
+                float v = bv;
+                lse_merge(v, bs, ov, os);
+            }
+            if (ov > bv || (ov == bv && oi < bi)) {
+                bv = ov;
+                bi = oi;
+            }
+        }
+        if (lane == 0 && p.out_partial) {
+            // a vocab shard: the global row of its maximum (INT_MAX: nothing allowed here)
+            const int32_t gi = bi == INT_MAX ? INT_MAX : (int32_t)(bi + p.row_offset);
+            reinterpret_cast<Partial*>(p.out_partial)[m] = Partial{bv, gi, bs, 0.f};
+        } else if (lane == 0) {
+            const bool empty = bi == INT_MAX;
+            if (empty) {
+                bi = 0;
+                bv = -INFINITY;
+                raise_flag(p.dev_err, DEVFLAG_EMPTY_MASK);
+            }
+            p.out_idx[m] = bi;
+            if (p.out_val) p.out_val[m] = bv;
+            // the maximum's own term is exp(0) = 1, so bs >= 1 and the result is <= 0
+            if (lp) p.out_logprob[m] = empty ? -INFINITY : -logf(bs);
+        }
+    }
+    __syncwarp();
+    if (lane == 0) {  // leave the workspace ready for the next call
+        p.ticket[0] = 0u;
+        p.ticket[1] = 0u;
+    }
+}
+
 template <int FMT, int NT, int MODE, int BD>
 __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
     sweep_kernel(const __grid_constant__ SweepParams p, const __grid_constant__ CUtensorMap map_codes,
@@ -744,83 +829,7 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
             if (lane == 0 && 2 * q + 1 < M)
                 parts[(int64_t)blockIdx.x * 16 + 2 * q + 1] = Partial{ov, oi, os, 0.f};
         }
-        int last = 0;
-        if (lane == 0) last = atom_add_acq_rel_gpu(p.ticket, 1u) == gridDim.x - 1;
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (!last) return;
-        fence_acq_rel_gpu();
-        // the last CTA folds every CTA's partial: lane l reads CTAs l, l + 32, ...
-        // (independent loads in flight together), then a shuffle reduction; ties go
-        // to the lowest row index, so the result does not depend on the order
-        const int G = (int)gridDim.x;
-        constexpr int FOLD = 8;  // partials per lane in flight at a time
-        for (int m = 0; m < M; ++m) {
-            float bv = -INFINITY, bs = 0.f;
-            int32_t bi = INT_MAX;
-            for (int base = 0; base < G; base += 32 * FOLD) {
-                float qv[FOLD], qs[FOLD];
-                int32_t qi[FOLD];
-#pragma unroll
-                for (int j = 0; j < FOLD; ++j) {
-                    const int b = base + lane + 32 * j;
-                    qv[j] = -INFINITY;
-                    qi[j] = INT_MAX;
-                    qs[j] = 0.f;
-                    if (b < G) {
-                        const float4 e = __ldcg(reinterpret_cast<const float4*>(parts + (int64_t)b * 16 + m));
-                        qv[j] = e.x;
-                        qi[j] = __float_as_int(e.y);
-                        qs[j] = e.z;
-                    }
-                }
-#pragma unroll
-                for (int j = 0; j < FOLD; ++j) {
-                    if (lp) {
-                        float v = bv;
-                        lse_merge(v, bs, qv[j], qs[j]);
-                    }
-                    if (qv[j] > bv || (qv[j] == bv && qi[j] < bi)) {
-                        bv = qv[j];
-                        bi = qi[j];
-                    }
-                }
-            }
-#pragma unroll
-            for (int o = 16; o; o >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                const int32_t oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                const float os = __shfl_xor_sync(0xffffffffu, bs, o);
-                if (lp) {
-                    float v = bv;
-                    lse_merge(v, bs, ov, os);
-                }
-                if (ov > bv || (ov == bv && oi < bi)) {
-                    bv = ov;
-                    bi = oi;
-                }
-            }
-            if (lane == 0 && p.out_partial) {
-                // a vocab shard: the global row of its maximum (INT_MAX: nothing allowed here)
-                const int32_t gi = bi == INT_MAX ? INT_MAX : (int32_t)(bi + p.row_offset);
-                reinterpret_cast<Partial*>(p.out_partial)[m] = Partial{bv, gi, bs, 0.f};
-            } else if (lane == 0) {
-                const bool empty = bi == INT_MAX;
-                if (empty) {
-                    bi = 0;
-                    bv = -INFINITY;
-                    raise_flag(p.dev_err, DEVFLAG_EMPTY_MASK);
-                }
-                p.out_idx[m] = bi;
-                if (p.out_val) p.out_val[m] = bv;
-                // the maximum's own term is exp(0) = 1, so bs >= 1 and the result is <= 0
-                if (lp) p.out_logprob[m] = empty ? -INFINITY : -logf(bs);
-            }
-        }
-        __syncwarp();
-        if (lane == 0) {  // leave the workspace ready for the next call
-            p.ticket[0] = 0u;
-            p.ticket[1] = 0u;
-        }
+        ticket_and_fold(p, lane, lp);
         return;
     }
 
@@ -956,6 +965,374 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
     }
 }
 
+// ------------------------------------------------------------------ many inputs (M > 8)
+// With more than eight inputs the staged x no longer fits beside a useful ring (16 inputs
+// x K 5,120 in f16 is 160 KB), so tiles are 64 rows tall and every stage carries, next to
+// the table's K chunk for those rows, the inputs' x chunk for the same K range, loaded by
+// TMA from global memory (L2): x is read once per 64 table rows instead of being held
+// whole. Four row groups of 16 rows; the 16 compute warps are 4 per row group, each
+// taking every fourth slab of its group's rows. Quantized tables read a f16 copy of x,
+// scaled per row by a power of two, written by wide_x16_kernel just before.
+constexpr int kWRows = 64;
+constexpr int kWCW = 16;                  // compute warps
+constexpr int kWThreads = (kWCW + 2) * 32;
+constexpr int kWCols = 16;                // inputs (columns) per sweep
+constexpr int kWRedFloats = 16 * kWCols;  // one warp's tile partial: 16 rows x 16 inputs
+
+__host__ __device__ inline int wide_seg_elems(int fmt) { return fmt == 0 ? 64 : fmt == 1 ? 128 : 256; }
+__host__ __device__ inline int wide_code_bytes(int segs) { return kWRows * 128 * segs; }
+__host__ __device__ inline int wide_scale_bytes(int fmt, int segs) { return fmt == 2 ? kWRows * 16 * segs : 0; }
+__host__ __device__ inline int wide_xsegs(int fmt, int segs) { return segs * wide_seg_elems(fmt) / 64; }
+__host__ __device__ inline int wide_x_bytes(int fmt, int segs) { return wide_xsegs(fmt, segs) * kWCols * 128; }
+
+// x [M, k] bf16 -> f16 scaled by 2^e_m (the largest |x| of row m lands in [2^14, 2^15)),
+// as stage_to_f16 does in shared memory for the narrow sweep. One CTA per input row.
+__global__ void __launch_bounds__(256) wide_x16_kernel(const uint16_t* __restrict__ x, int k,
+                                                        uint16_t* __restrict__ x16,
+                                                        int32_t* __restrict__ xexp) {
+    __shared__ float red[8];
+    const int m = blockIdx.x, tid = threadIdx.x;
+    const uint16_t* row = x + (int64_t)m * k;
+    float a = 0.f;
+    for (int j = tid; j < k; j += 256) a = fmaxf(a, fabsf(bf16_to_f32(row[j])));
+    for (int o = 16; o; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if ((tid & 31) == 0) red[tid >> 5] = a;
+    __syncthreads();
+    a = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) a = fmaxf(a, red[w]);
+    int ex = 0;
+    if (a > 0.f) frexpf(a, &ex);
+    const int e = (a > 0.f) ? 15 - ex : 0;
+    if (tid == 0) xexp[m] = e;
+    const float f1 = ldexpf(1.f, e / 2), f2 = ldexpf(1.f, e - e / 2);
+    for (int j = tid; j < k; j += 256)
+        x16[(int64_t)m * k + j] = f32_to_f16((bf16_to_f32(row[j]) * f1) * f2);
+}
+
+// One slab of one row group for 16 inputs (two MMA column blocks). The codes are read as in
+// slab_mma; the lane's x elements [e, e + V) of inputs g and g + 8 come from the stage's
+// x chunk, [x segment of 64 elements][16 inputs][128 B] with the 128-byte swizzle.
+template <int FMT>
+__device__ __forceinline__ void slab_mma_wide(float (&acc)[2][2][4], const uint8_t* cw,
+                                              const uint8_t* sw, uint32_t spitch8,
+                                              const uint8_t* xst, int e, int g) {
+    const uint4 ra = lds128(cw);
+    const uint4 rb = lds128(cw + 1024);
+    const uint8_t* x0 = xst + (e >> 6) * (kWCols * 128) + g * 128;  // input g
+    const uint8_t* x1 = x0 + 8 * 128;                                // input g + 8
+    const int cb = (e & 63) >> 3;                                    // first 16-byte chunk
+#define XQ(row, q) lds128((row) + ((((cb) + (q)) ^ g) << 4))
+    if (FMT == 0) {
+        const uint4 xa = XQ(x0, 0), xb = XQ(x1, 0);
+        mma_bf16_16816(acc[0][0], ra.x, rb.x, ra.y, rb.y, xa.x, xa.y);
+        mma_bf16_16816(acc[1][0], ra.z, rb.z, ra.w, rb.w, xa.z, xa.w);
+        mma_bf16_16816(acc[0][1], ra.x, rb.x, ra.y, rb.y, xb.x, xb.y);
+        mma_bf16_16816(acc[1][1], ra.z, rb.z, ra.w, rb.w, xb.z, xb.w);
+    } else if (FMT == 1) {
+        const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w};
+        const uint32_t wb[4] = {rb.x, rb.y, rb.z, rb.w};
+        const uint4 xa0 = XQ(x0, 0), xa1 = XQ(x0, 1), xb0 = XQ(x1, 0), xb1 = XQ(x1, 1);
+        const uint32_t xa[8] = {xa0.x, xa0.y, xa0.z, xa0.w, xa1.x, xa1.y, xa1.z, xa1.w};
+        const uint32_t xb[8] = {xb0.x, xb0.y, xb0.z, xb0.w, xb1.x, xb1.y, xb1.z, xb1.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t a0 = e4m3x2_to_f16x2((uint16_t)(wa[i] & 0xFFFFu));
+            const uint32_t a2 = e4m3x2_to_f16x2((uint16_t)(wa[i] >> 16));
+            const uint32_t a1 = e4m3x2_to_f16x2((uint16_t)(wb[i] & 0xFFFFu));
+            const uint32_t a3 = e4m3x2_to_f16x2((uint16_t)(wb[i] >> 16));
+            mma_f16_16816(acc[i & 1][0], a0, a1, a2, a3, xa[2 * i], xa[2 * i + 1]);
+            mma_f16_16816(acc[i & 1][1], a0, a1, a2, a3, xb[2 * i], xb[2 * i + 1]);
+        }
+    } else {
+        const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w};
+        const uint32_t wb[4] = {rb.x, rb.y, rb.z, rb.w};
+        const uint16_t s0v = *reinterpret_cast<const uint16_t*>(sw);
+        const uint16_t s1v = *reinterpret_cast<const uint16_t*>(sw + spitch8);
+        const uint32_t sa = e4m3x2_to_f16x2(s0v);
+        const uint32_t sb = e4m3x2_to_f16x2(s1v);
+        const uint32_t sa_lo = __byte_perm(sa, 0, 0x1010), sa_hi = __byte_perm(sa, 0, 0x3232);
+        const uint32_t sb_lo = __byte_perm(sb, 0, 0x1010), sb_hi = __byte_perm(sb, 0, 0x3232);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            uint32_t qa[4], qb[4];
+            e2m1x8_to_f16x2x4(wa[i], qa);
+            e2m1x8_to_f16x2x4(wb[i], qb);
+            const uint32_t s_a = i < 2 ? sa_lo : sa_hi;
+            const uint32_t s_b = i < 2 ? sb_lo : sb_hi;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                qa[q] = hmul2(qa[q], s_a);
+                qb[q] = hmul2(qb[q], s_b);
+            }
+            const uint4 xv = XQ(x0, i), xw = XQ(x1, i);
+            mma_f16_16816(acc[0][0], qa[0], qb[0], qa[1], qb[1], xv.x, xv.y);
+            mma_f16_16816(acc[1][0], qa[2], qb[2], qa[3], qb[3], xv.z, xv.w);
+            mma_f16_16816(acc[0][1], qa[0], qb[0], qa[1], qb[1], xw.x, xw.y);
+            mma_f16_16816(acc[1][1], qa[2], qb[2], qa[3], qb[3], xw.z, xw.w);
+        }
+    }
+#undef XQ
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kWThreads, 1)
+    sweep_wide_kernel(const __grid_constant__ SweepParams p, const __grid_constant__ CUtensorMap map_codes,
+                      const __grid_constant__ CUtensorMap map_scales,
+                      const __grid_constant__ CUtensorMap map_x) {
+    constexpr int V = Fmt<FMT>::V;
+    constexpr int SLAB = 4 * V;
+    constexpr int CW = kWCW;
+    constexpr int REDUCER = CW, PRODUCER = CW + 1;
+
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + kMaxStages;
+    uint64_t* red_full = empty + kMaxStages;  // [2]
+    uint64_t* red_empty = red_full + 2;       // [2]
+    // misc: [0] abort, [18..29] tile of each ring slot, [30..31] tile of each reducer buffer
+    int* misc = reinterpret_cast<int*>(red_empty + 2);
+    volatile int* abort_flag = misc;
+    volatile int* slot_tile = misc + 18;
+    volatile int* red_tile = misc + 30;
+    float* red = reinterpret_cast<float*>(misc + 32);  // [2][CW][16 rows][16 inputs]
+    const uint32_t head_end = smem_u32(red + 2 * CW * kWRedFloats);
+    uint8_t* ring = smem + (((head_end + 1023u) & ~1023u) - smem_u32(smem));
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t K = p.k;
+    const int S = p.stages;
+    const int stage_bytes = p.stage_bytes;
+    const int segs = p.segs;
+    const int NC = p.stages_per_tile;
+    const int M = p.M;
+    const int code_b = wide_code_bytes(segs);
+    const int scale_b = wide_scale_bytes(FMT, segs);
+    const int xsegs = wide_xsegs(FMT, segs);
+    const int64_t T = p.num_tiles;  // 64-row tiles
+
+    if (tid == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], CW);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&red_full[b], CW);
+            mbar_init(&red_empty[b], 1);
+        }
+        misc[0] = 0;
+        mbar_fence_init();
+    }
+    __syncthreads();
+    pdl_launch_dependents();
+
+    // ------------------------------------------------------------ producer warp
+    if (warp == PRODUCER) {
+        int slot = 0;
+        uint32_t phase = 0;
+        int64_t issued = 0;
+        const uint32_t tx = (uint32_t)(code_b + scale_b + wide_x_bytes(FMT, segs));
+        bool stop = false;
+        // every stage reads x, which the previous kernel (the f16 copy) may write
+        pdl_wait();
+        int64_t tile = blockIdx.x;
+        int64_t pending = 0;
+        if (lane == 0) pending = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
+        while (tile < T && !stop) {
+            for (int ch = 0; ch < NC; ++ch) {
+                if (!mbar_wait_bounded(&empty[slot], phase ^ 1u, abort_flag)) {
+                    stop = true;
+                    break;
+                }
+                if (lane == 0) {
+                    uint8_t* dst = ring + (size_t)slot * stage_bytes;
+                    slot_tile[slot] = (int)tile;
+                    mbar_arrive_expect_tx(&full[slot], tx);
+                    tma_load_3d(dst, &map_codes, 0, (int)(tile * kWRows), ch * segs, &full[slot]);
+                    if (FMT == 2)
+                        tma_load_2d(dst + code_b, &map_scales, ch * 8 * segs, (int)(tile * kWRows),
+                                    &full[slot]);
+                    tma_load_3d(dst + code_b + scale_b, &map_x, 0, 0, ch * xsegs, &full[slot]);
+                }
+                __syncwarp();
+                ++issued;
+                if (++slot == S) {
+                    slot = 0;
+                    phase ^= 1u;
+                }
+            }
+            tile = __shfl_sync(0xffffffffu, pending, 0);
+            if (lane == 0 && tile < T) pending = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
+        }
+        for (int64_t j = issued > S ? issued - S : 0; j < issued; ++j)
+            if (!mbar_wait_bounded(&full[j % S], (uint32_t)((j / S) & 1), nullptr)) break;
+        if (!stop && mbar_wait_bounded(&empty[slot], phase ^ 1u, abort_flag) && lane == 0) {
+            slot_tile[slot] = -1;
+            mbar_arrive(&full[slot]);
+        }
+        __syncwarp();
+        return;
+    }
+
+    // ------------------------------------------------------------ reducer warp
+    if (warp == REDUCER) {
+        // lane holds input m = lane & 15 and the rows of parity h = lane >> 4 of each tile,
+        // with a running (max, lowest row) and sum of exp over them
+        const int m = lane & 15, h = lane >> 4;
+        const bool lp = p.out_logprob != nullptr || p.out_partial != nullptr;
+        pdl_wait();
+        const float gsc = FMT == 2 ? __ldg(p.global_scale) : 1.f;
+        float fa = 1.f, fb = 1.f;  // 2^-xexp[m] as two factors
+        if (FMT != 0 && m < M) {
+            const int e = -__ldg(p.xexp + m);
+            fa = ldexpf(1.f, e / 2);
+            fb = ldexpf(1.f, e - e / 2);
+        }
+        if (lane == 0) {
+            if (FMT == 1) l2_prefetch_share(p.row_scale, p.n * 4);
+            if (p.mask) l2_prefetch_share(p.mask, ((p.M - 1) * p.mask_stride + p.mask_words) * 4);
+        }
+        float best_v = -INFINITY, se = 0.f;
+        int32_t best_i = INT_MAX;
+        int buf = 0;
+        uint32_t fph = 0u;
+        while (true) {
+            if (!mbar_wait_bounded(&red_full[buf], (fph >> buf) & 1u, abort_flag)) break;
+            fph ^= 1u << buf;
+            const int tile_id = red_tile[buf];
+            if (tile_id < 0) break;
+            const int64_t row0 = (int64_t)tile_id * kWRows;
+            float rs_a = 0.f, rs_b = 0.f;  // row scales of rows row0 + lane, row0 + 32 + lane
+            if (FMT == 1) {
+                if (row0 + lane < p.n) rs_a = __ldg(p.row_scale + row0 + lane);
+                if (row0 + 32 + lane < p.n) rs_b = __ldg(p.row_scale + row0 + 32 + lane);
+            }
+            const float* rb = red + (size_t)buf * CW * kWRedFloats;
+#pragma unroll 4
+            for (int j = 0; j < 32; ++j) {
+                const int r = 2 * j + h;  // row within the tile
+                const int rg = r >> 4, rr = r & 15;
+                // the four warps of the row group, in order
+                float a = rb[(rg + 0) * kWRedFloats + rr * kWCols + m];
+                a += rb[(rg + 4) * kWRedFloats + rr * kWCols + m];
+                a += rb[(rg + 8) * kWRedFloats + rr * kWCols + m];
+                a += rb[(rg + 12) * kWRedFloats + rr * kWCols + m];
+                float rs = 1.f;
+                if (FMT == 1) rs = __shfl_sync(0xffffffffu, j < 16 ? rs_a : rs_b, r & 31);
+                const int64_t row = row0 + r;
+                const bool valid = row < p.n && m < M;
+                float l = a;
+                if (FMT != 0) l = (l * fa) * fb;
+                if (FMT == 1) l *= rs;
+                if (FMT == 2) l *= gsc;
+                const bool ok = valid && mask_allows(p, m, row);
+                if (valid && p.out_logits)
+                    p.out_logits[(int64_t)m * p.n + row] = ok ? f32_to_bf16(l) : (uint16_t)0xFF80u;
+                if (lp && ok && l > -INFINITY) {
+                    float v = best_v;
+                    lse_merge(v, se, l, 1.f);
+                }
+                if (ok && (l > best_v || (l == best_v && best_i == INT_MAX))) {
+                    best_v = l;
+                    best_i = (int32_t)row;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&red_empty[buf]);
+            buf ^= 1;
+        }
+        if (*abort_flag) raise_flag(p.dev_err, DEVFLAG_TIMEOUT);
+        // fold the two row parities of each input, then lanes m < M publish
+        {
+            const float ov = __shfl_xor_sync(0xffffffffu, best_v, 16);
+            const int32_t oi = __shfl_xor_sync(0xffffffffu, best_i, 16);
+            const float os = __shfl_xor_sync(0xffffffffu, se, 16);
+            if (lp) {
+                float v = best_v;
+                lse_merge(v, se, ov, os);
+            }
+            if (ov > best_v || (ov == best_v && oi < best_i)) {
+                best_v = ov;
+                best_i = oi;
+            }
+        }
+        Partial* parts = reinterpret_cast<Partial*>(p.partials);
+        if (h == 0 && m < M) parts[(int64_t)blockIdx.x * 16 + m] = Partial{best_v, best_i, se, 0.f};
+        __syncwarp();
+        fence_acq_rel_gpu();  // every publishing lane's store before lane 0's ticket
+        __syncwarp();
+        ticket_and_fold(p, lane, lp);
+        return;
+    }
+
+    // ------------------------------------------------------------ compute warps
+    const int g = lane >> 2, c = lane & 3;
+    const int rg = warp & 3, sub = warp >> 2;
+    const int r0 = tile_row(g);
+    const int rowb = rg * 16 + r0;  // table row of MMA row g within the tile
+    const uint32_t xr = (uint32_t)(r0 & 7) << 4;
+    const uint32_t coff0 = (uint32_t)rowb * 128u + (((uint32_t)c * 16u) ^ xr);
+    const uint32_t coff1 = (uint32_t)rowb * 128u + ((64u + (uint32_t)c * 16u) ^ xr);
+    const uint32_t spitch = 16u * (uint32_t)segs;
+    const uint32_t soff = (uint32_t)code_b + (uint32_t)rowb * spitch + 2u * (uint32_t)c;
+    const int total_slabs = (int)(K / SLAB);
+    const int slabs_per_stage = 2 * segs;
+
+    float acc[2][2][4];
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[a][t][i] = 0.f;
+
+    int buf = 0;
+    uint32_t eph = 0u;
+    int slot = 0;
+    uint32_t phase = 0;
+    while (true) {
+        if (!mbar_wait_bounded(&full[slot], phase, abort_flag)) break;
+        const int tile = slot_tile[slot];
+        if (tile < 0) break;
+        for (int ch = 0; ch < NC; ++ch) {
+            if (ch > 0 && !mbar_wait_bounded(&full[slot], phase, abort_flag)) break;
+            const uint8_t* st = ring + (size_t)slot * stage_bytes;
+            const uint8_t* xst = st + code_b + scale_b;
+            const int a0 = ch * slabs_per_stage;
+            const int nv = min(slabs_per_stage, total_slabs - a0);
+            for (int l = sub; l < nv; l += 4)
+                slab_mma_wide<FMT>(acc, st + (l >> 1) * (kWRows * 128) + ((l & 1) ? coff1 : coff0),
+                                   st + soff + l * 8, 8u * spitch, xst, l * SLAB + c * V, g);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[slot]);
+            if (++slot == S) {
+                slot = 0;
+                phase ^= 1u;
+            }
+        }
+        mbar_wait_bounded(&red_empty[buf], ((eph >> buf) & 1u) ^ 1u, abort_flag);
+        eph ^= 1u << buf;
+        float* rp = red + (size_t)buf * CW * kWRedFloats + warp * kWRedFloats;
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int row = (i < 2 ? r0 : r0 + 8);
+                rp[row * kWCols + t * 8 + 2 * c + (i & 1)] = acc[0][t][i] + acc[1][t][i];
+                acc[0][t][i] = acc[1][t][i] = 0.f;
+            }
+        if (warp == 0 && lane == 0) red_tile[buf] = tile;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&red_full[buf]);
+        buf ^= 1;
+    }
+    if (mbar_wait_bounded(&red_empty[buf], ((eph >> buf) & 1u) ^ 1u, abort_flag)) {
+        if (warp == 0 && lane == 0) red_tile[buf] = -1;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&red_full[buf]);
+    }
+}
+
 struct Geometry {
     int kpad;
     int segs;             // 128-byte segments per row per stage
@@ -1022,12 +1399,12 @@ EncodeTiledFn encode_tiled() {
 // 128 B x 16 rows x 8 segments is a stage, with rows inside the 128-byte swizzle atom.
 // Rows >= rows and segments past the row read as zeros.
 cudaError_t make_code_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes,
-                          int segs) {
+                          int segs, int box_rows = kTileRows) {
     EncodeTiledFn fn = encode_tiled();
     if (!fn) return cudaErrorNotSupported;
     cuuint64_t dims[3] = {128, (cuuint64_t)rows, (cuuint64_t)(row_bytes / 128)};
     cuuint64_t strides[2] = {(cuuint64_t)row_bytes, 128};
-    cuuint32_t box[3] = {128, kTileRows, (cuuint32_t)segs};
+    cuuint32_t box[3] = {128, (cuuint32_t)box_rows, (cuuint32_t)segs};
     cuuint32_t es[3] = {1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
                     box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -1038,17 +1415,125 @@ cudaError_t make_code_map(CUtensorMap* m, const void* base, int64_t rows, int64_
 // NVFP4 block scales: [rows, pitch] bytes viewed as 16-bit elements, boxes of
 // 16 * segs bytes x 16 rows (up to 512 bytes per row: two scale bytes per element).
 cudaError_t make_scale_map(CUtensorMap* m, const void* base, int64_t rows, int64_t pitch,
-                           int segs) {
+                           int segs, int box_rows = kTileRows) {
     EncodeTiledFn fn = encode_tiled();
     if (!fn) return cudaErrorNotSupported;
     cuuint64_t dims[2] = {(cuuint64_t)(pitch / 2), (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)pitch};
-    cuuint32_t box[2] = {(cuuint32_t)(8 * segs), kTileRows};
+    cuuint32_t box[2] = {(cuuint32_t)(8 * segs), (cuuint32_t)box_rows};
     cuuint32_t es[2] = {1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides,
                     box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// x [M, k] of 16-bit elements as 64-element segments: boxes of kWCols rows (inputs past
+// M read as zeros) x xsegs segments, 128-byte swizzle.
+cudaError_t make_x_map(CUtensorMap* m, const void* base, int M, int64_t k, int xsegs) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return cudaErrorNotSupported;
+    cuuint64_t dims[3] = {64, (cuuint64_t)M, (cuuint64_t)(k / 64)};
+    cuuint64_t strides[2] = {(cuuint64_t)k * 2, 128};
+    cuuint32_t box[3] = {64, (cuuint32_t)kWCols, (cuuint32_t)xsegs};
+    cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(base), dims, strides,
+                    box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+struct WideGeometry {
+    int segs;             // 128-byte table segments per row per stage
+    int stages_per_tile;
+    int stage_bytes;
+    int stages;
+    size_t smem;
+};
+
+WideGeometry wide_geometry(int64_t k, int fmt) {
+    WideGeometry g{};
+    size_t head = (size_t)(2 * kMaxStages + 4) * 8 + 32 * sizeof(int) +
+                  (size_t)2 * kWCW * kWRedFloats * sizeof(float);
+    head = ((head + 1023) & ~(size_t)1023) + 1024;
+    const int64_t row_bytes = fmt == 0 ? k * 2 : fmt == 1 ? k : k / 2;
+    const int row_segs = (int)(row_bytes / 128);
+    const long avail = (long)kSmemLimit - (long)head;
+    for (int want = 3; want >= 2 && g.stages < 2; --want) {
+        for (int max_segs = 32; max_segs >= 1; --max_segs) {
+            const int nc = (row_segs + max_segs - 1) / max_segs;
+            const int segs = (row_segs + nc - 1) / nc;
+            const int sb = wide_code_bytes(segs) + wide_scale_bytes(fmt, segs) + wide_x_bytes(fmt, segs);
+            int stages = avail > 0 ? (int)(avail / sb) : 0;
+            if (stages > kMaxStages) stages = kMaxStages;
+            if (stages >= want) {
+                g.segs = segs;
+                g.stages_per_tile = nc;
+                g.stage_bytes = sb;
+                g.stages = stages;
+                break;
+            }
+        }
+    }
+    g.smem = head + (size_t)g.stages * g.stage_bytes;
+    return g;
+}
+
+template <int FMT>
+cudaError_t launch_wide(const SweepParams& p, cudaStream_t s, SweepLaunch* info) {
+    auto kern = sweep_wide_kernel<FMT>;
+    const WideGeometry geo = wide_geometry(p.k, FMT);
+    if (geo.stages < 2) return cudaErrorInvalidValue;
+    const int xsegs = wide_xsegs(FMT, geo.segs);
+    CUtensorMap map_codes, map_scales, map_x;
+    cudaError_t e = make_code_map(&map_codes, p.w, p.n, p.row_bytes, geo.segs, kWRows);
+    if (e != cudaSuccess) return e;
+    if (FMT == 2) {
+        if ((e = make_scale_map(&map_scales, p.block_scale, p.n, p.scale_pitch, geo.segs, kWRows)) !=
+            cudaSuccess)
+            return e;
+    } else {
+        map_scales = map_codes;  // unused
+    }
+    const void* xsrc = FMT == 0 ? static_cast<const void*>(p.x) : static_cast<const void*>(p.x16);
+    if ((e = make_x_map(&map_x, xsrc, p.M, p.k, xsegs)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)geo.smem)) != cudaSuccess)
+        return e;
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return e;
+    SweepParams q = p;
+    q.num_tiles = (p.n + kWRows - 1) / kWRows;
+    q.stages = geo.stages;
+    q.stage_bytes = geo.stage_bytes;
+    q.segs = geo.segs;
+    q.stages_per_tile = geo.stages_per_tile;
+    int64_t grid = sms;
+    if (grid > q.num_tiles) grid = q.num_tiles;
+    if (grid > kMaxGrid) grid = kMaxGrid;
+    if (grid < 1) grid = 1;
+    if (FMT != 0) {  // the f16 copy of x the stages read
+        wide_x16_kernel<<<p.M, 256, 0, s>>>(p.x, (int)p.k, p.x16, p.xexp);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kWThreads);
+    cfg.dynamicSmemBytes = geo.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if ((e = cudaLaunchKernelEx(&cfg, kern, q, map_codes, map_scales, map_x)) != cudaSuccess) return e;
+    if (info) {
+        info->grid = (int)grid;
+        info->smem_bytes = (int)geo.smem;
+    }
+    return cudaGetLastError();
 }
 
 template <int FMT, int NT, int MODE, int BD>
@@ -1105,13 +1590,23 @@ cudaError_t launch_one(const SweepParams& p, cudaStream_t s, SweepLaunch* info) 
 
 }  // namespace
 
-size_t sweep_smem_bytes(int M, int64_t k, int fmt, int* kpad_out) {
+size_t sweep_smem_bytes(int M, int64_t k, int fmt, int* kpad_out, int mode) {
+    if (mode == 0 && M > 8) {  // the wide sweep stages x per K chunk
+        const WideGeometry w = wide_geometry(k, fmt);
+        if (kpad_out) *kpad_out = (int)k;
+        return w.stages >= 2 ? w.smem : (size_t)kSmemLimit + 1;
+    }
     const Geometry g = geometry(M, k, fmt);
     if (kpad_out) *kpad_out = g.kpad;
     return g.stages >= 2 ? g.smem : (size_t)kSmemLimit + 1;
 }
 
 int sweep_max_grid() { return kMaxGrid; }
+
+size_t sweep_x16_bytes(int M, int64_t k, int fmt) {
+    if (M <= 8 || fmt == 0) return 0;
+    return (((size_t)M * (size_t)k * 2 + 1023) & ~(size_t)1023) + 1024;  // x16, then xexp
+}
 
 namespace {
 
@@ -1168,6 +1663,11 @@ cudaError_t sweep_launch(const SweepParams& p, int fmt, int mode, cudaStream_t s
                          SweepLaunch* info) {
     const bool two = p.M > 8;
     if (fmt == 2 && mode == 0 && p.M <= 2) return launch_one<2, 1, 0, 1>(p, s, info);
+    if (mode == 0 && two) {
+        if (fmt == 0) return launch_wide<0>(p, s, info);
+        if (fmt == 1) return launch_wide<1>(p, s, info);
+        if (fmt == 2) return launch_wide<2>(p, s, info);
+    }
 #define MTP_SWEEP_CASE(F, NTV, MD) \
     if (fmt == F && (NTV == 2) == two && mode == MD) return launch_one<F, NTV, MD, 0>(p, s, info);
     MTP_SWEEP_CASE(0, 1, 0) MTP_SWEEP_CASE(0, 2, 0)

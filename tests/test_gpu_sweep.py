@@ -3,8 +3,8 @@
 Small tables span several 16-row tiles, several CTAs and a ragged tail; the full
 tables are the benchmark's (154,880 x 4,096 BF16 and FP8, 131,072 x 5,120 NVFP4) in
 the launch configuration bench.py times. Logits within 2e-2 + 1e-2|ref|; argmax exact
-where the top-2 gap exceeds 1e-2; one-hot inputs and batch invariance bit-exact (NVFP4:
-within M <= 2 and within M > 2)."""
+where the top-2 gap exceeds 1e-2; one-hot inputs and batch invariance bit-exact within
+each range of M that one sweep serves (1-8, 9-16; NVFP4 1-2, 3-8, 9-16)."""
 import numpy as np
 import pytest
 import torch
@@ -123,10 +123,11 @@ def test_batch_invariance(orc, fmt):
     x = synth.as_u16(synth.normal_bf16(synth._gen(10), (16, k), 1.0))
     table = device_table(oracle_quant(orc, w, fmt), fmt, n, k)
     head = api.LmHead(table)
-    # NVFP4 with one or two inputs applies the block scales to per-block fp32 sums (the
-    # same exact products, rounded differently), so it is bit-identical within M <= 2
-    # and within M > 2, and within the tolerance across the two
-    groups = [(1, 2), (3, 4, 8, 9, 16)] if fmt == 2 else [(1, 2, 3, 4, 8, 9, 16)]
+    # Three sweeps share the work: NVFP4 with one or two inputs applies the block scales
+    # to per-block fp32 sums, more than eight inputs use 64-row tiles with x streamed per
+    # K chunk; each sums the same exact products in its own fixed order, so results are
+    # bit-identical within each range of M and within the tolerance across them
+    groups = ([(1, 2), (3, 4, 8), (9, 16)] if fmt == 2 else [(1, 2, 3, 4, 8), (9, 12, 16)])
     bases = []
     for grp in groups:
         base = run_sweep(table, x[:grp[0]], head=head)
@@ -135,8 +136,8 @@ def test_batch_invariance(orc, fmt):
             got = run_sweep(table, x[:M], head=head)
             assert np.array_equal(got[2][0], base[2][0]), M
             assert got[1][0].view(np.uint32) == base[1][0].view(np.uint32)
-    if len(bases) == 2:
-        assert_close(bf16_bits_to_f64(bases[1][2][0]), bf16_bits_to_f64(bases[0][2][0]), "M<=2 vs M>2")
+    for b in bases[1:]:
+        assert_close(bf16_bits_to_f64(b[2][0]), bf16_bits_to_f64(bases[0][2][0]), "across ranges of M")
     # row m keeps its result whatever the other rows are
     x2 = x.copy()
     x2[1:] = x[::-1][:15]
