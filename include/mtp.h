@@ -174,11 +174,14 @@ mtp_status mtp_combine(const uint16_t* embed, int64_t vocab, const int32_t* toke
  *   dev_err       (device) i32 [1] or NULL
  *   ws            (device) >= mtp_lm_head_ws_bytes(head, n_eff, M) bytes, 16-byte
  *                 aligned, ALL ZERO before the first call; each call leaves its
- *                 counter zero again.
- * Requires 1 <= M <= 16, 1 <= n_eff <= n; table rows a multiple of 128 bytes (k % 64
- * for BF16, % 128 for FP8, % 256 for NVFP4; the sweep streams 128-byte segments) and
- * the staged inputs (M * k * 2 bytes) small enough to leave shared memory for the
- * stream (MTP_ERR_UNSUPPORTED otherwise).
+ *                 counter zero again. (For M > 8 on FP8/NVFP4 tables it also holds an
+ *                 f16 copy of x, M * k * 2 bytes, rewritten by each call.)
+ * Requires 1 <= M <= 32, 1 <= n_eff <= n; table rows a multiple of 128 bytes (k % 64
+ * for BF16, % 128 for FP8, % 256 for NVFP4; the sweep streams 128-byte segments); for
+ * M <= 8 the staged inputs (M * k * 2 bytes) must leave shared memory for the stream
+ * (MTP_ERR_UNSUPPORTED otherwise; M > 8 streams x per K chunk instead). Results are
+ * bit-identical for every M within 1-8, 9-16 and 17-32 (NVFP4: 1-2, 3-8, 9-16, 17-32),
+ * whose sweeps sum the same products in different fixed orders.
  * ------------------------------------------------------------------------------ */
 size_t mtp_lm_head_ws_bytes(const mtp_weight* head, int64_t n_eff, int32_t M);
 mtp_status mtp_lm_head_argmax(const mtp_weight* head, int64_t n_eff, const uint16_t* x,

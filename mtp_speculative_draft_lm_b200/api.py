@@ -67,7 +67,7 @@ def quantize_nvfp4(w: torch.Tensor, ws: torch.Tensor | None = None, stream=None)
 class LmHead:
     """The fused sweep + argmax over a table, with its zeroed workspace."""
 
-    def __init__(self, table: Table, n_eff: int | None = None, max_m: int = 16):
+    def __init__(self, table: Table, n_eff: int | None = None, max_m: int = 32):
         self.table = table
         self.n_eff = table.n if n_eff is None else int(n_eff)
         dev = table.data.device
@@ -151,7 +151,7 @@ class ShardedLmHead:
     rank sweeps its own rows (mtp_lm_head_shard_partial), the 16-byte partials are
     all-gathered, and every rank merges them (mtp_argmax_merge_partials)."""
 
-    def __init__(self, shard: Table | None, row_offset: int, group=None, max_m: int = 16):
+    def __init__(self, shard: Table | None, row_offset: int, group=None, max_m: int = 32):
         self.shard = shard
         self.row_offset = int(row_offset)
         self.group = group

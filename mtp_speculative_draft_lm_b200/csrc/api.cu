@@ -55,7 +55,9 @@ int64_t row_bytes(const mtp_weight* w) {
 
 constexpr size_t kTicketBytes = 256;
 constexpr size_t kPartialBytes = 16;  // {float value, int32 index, float sum of exp, pad}
-constexpr int kMaxM = 16;
+constexpr int kMaxM = 32;       // inputs per sweep
+constexpr int kMaxMCombine = 16;
+constexpr int kPartSlots = 32;   // partials per CTA
 
 }  // namespace
 
@@ -117,7 +119,7 @@ mtp_status mtp_combine(const uint16_t* embed, int64_t vocab, const int32_t* toke
     if (!embed || !token_ids || !hidden || !w_norm_embed || !w_norm_hidden || !out)
         return MTP_ERR_INVALID_ARG;
     if (vocab < 1 || h < 16 || h % 16 || !(eps >= 0.f)) return MTP_ERR_INVALID_ARG;
-    if (M < 1 || M > kMaxM) return MTP_ERR_UNSUPPORTED;
+    if (M < 1 || M > kMaxMCombine) return MTP_ERR_UNSUPPORTED;
     mtp_status st = check_weight(fc);
     if (st != MTP_OK) return st;
     if (fc->n != h || fc->k != 2 * (int64_t)h) return MTP_ERR_INVALID_ARG;
@@ -153,7 +155,7 @@ mtp_status mtp_combine(const uint16_t* embed, int64_t vocab, const int32_t* toke
 
 size_t mtp_lm_head_ws_bytes(const mtp_weight* head, int64_t n_eff, int32_t M) {
     (void)n_eff;
-    const size_t base = kTicketBytes + kPartialBytes * 16 * (size_t)mtp::sweep_max_grid();
+    const size_t base = kTicketBytes + kPartialBytes * kPartSlots * (size_t)mtp::sweep_max_grid();
     if (!head || M < 1 || M > kMaxM) return base;
     return base + mtp::sweep_x16_bytes(M, head->k, head->fmt);
 }
@@ -204,7 +206,7 @@ mtp_status lm_head_impl(const mtp_weight* head, int64_t n_eff, const uint16_t* x
     p.ticket = static_cast<uint32_t*>(ws);
     p.partials = static_cast<uint8_t*>(ws) + kTicketBytes;
     if (mtp::sweep_x16_bytes(M, head->k, head->fmt)) {  // the wide sweep's f16 copy of x
-        uint8_t* xb = static_cast<uint8_t*>(ws) + kTicketBytes + kPartialBytes * 16 *
+        uint8_t* xb = static_cast<uint8_t*>(ws) + kTicketBytes + kPartialBytes * kPartSlots *
                                                                    (size_t)mtp::sweep_max_grid();
         p.x16 = reinterpret_cast<uint16_t*>(xb);
         p.xexp = reinterpret_cast<int32_t*>(xb + (((size_t)M * head->k * 2 + 1023) & ~(size_t)1023));

@@ -29,7 +29,7 @@
 namespace {
 
 constexpr size_t kTicketBytes = 256;
-constexpr size_t kScratchBytes = kTicketBytes + 16 * 16 * 1024;  // counter + 1024 CTAs x 16 rows
+constexpr size_t kScratchBytes = kTicketBytes + 16 * 32 * 1024;  // header + 1024 CTAs x 32 partials
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) uint8_t g_sweep_scratch[kScratchBytes];

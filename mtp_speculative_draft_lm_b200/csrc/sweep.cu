@@ -54,6 +54,7 @@ namespace mtp {
 namespace {
 
 constexpr int kTileRows = 16;
+constexpr int kPartSlots = 32;  // partials per CTA (one per input, up to 32 inputs)
 constexpr int kMaxGrid = 1024;
 constexpr int kMaxStages = 12;
 constexpr int kMaxSegs = 32;  // 128-byte segments of a row per stage (box of 16 rows x 4 KB)
@@ -500,7 +501,7 @@ __device__ void ticket_and_fold(const SweepParams& p, int lane, bool lp) {
                 qi[j] = INT_MAX;
                 qs[j] = 0.f;
                 if (b < G) {
-                    const float4 e = __ldcg(reinterpret_cast<const float4*>(parts + (int64_t)b * 16 + m));
+                    const float4 e = __ldcg(reinterpret_cast<const float4*>(parts + (int64_t)b * kPartSlots + m));
                     qv[j] = e.x;
                     qi[j] = __float_as_int(e.y);
                     qs[j] = e.z;
@@ -825,9 +826,9 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
             const int32_t oi = __shfl_sync(0xffffffffu, best_i[q], 16);
             const float os = __shfl_sync(0xffffffffu, se[q], 16);
             if (lane == 0 && 2 * q < M)
-                parts[(int64_t)blockIdx.x * 16 + 2 * q] = Partial{best_v[q], best_i[q], se[q], 0.f};
+                parts[(int64_t)blockIdx.x * kPartSlots + 2 * q] = Partial{best_v[q], best_i[q], se[q], 0.f};
             if (lane == 0 && 2 * q + 1 < M)
-                parts[(int64_t)blockIdx.x * 16 + 2 * q + 1] = Partial{ov, oi, os, 0.f};
+                parts[(int64_t)blockIdx.x * kPartSlots + 2 * q + 1] = Partial{ov, oi, os, 0.f};
         }
         ticket_and_fold(p, lane, lp);
         return;
@@ -976,14 +977,15 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
 constexpr int kWRows = 64;
 constexpr int kWCW = 16;                  // compute warps
 constexpr int kWThreads = (kWCW + 2) * 32;
-constexpr int kWCols = 16;                // inputs (columns) per sweep
-constexpr int kWRedFloats = 16 * kWCols;  // one warp's tile partial: 16 rows x 16 inputs
+// inputs per sweep: 8 NT columns (NT = 2: up to 16 inputs, NT = 4: up to 32)
 
 __host__ __device__ inline int wide_seg_elems(int fmt) { return fmt == 0 ? 64 : fmt == 1 ? 128 : 256; }
 __host__ __device__ inline int wide_code_bytes(int segs) { return kWRows * 128 * segs; }
 __host__ __device__ inline int wide_scale_bytes(int fmt, int segs) { return fmt == 2 ? kWRows * 16 * segs : 0; }
 __host__ __device__ inline int wide_xsegs(int fmt, int segs) { return segs * wide_seg_elems(fmt) / 64; }
-__host__ __device__ inline int wide_x_bytes(int fmt, int segs) { return wide_xsegs(fmt, segs) * kWCols * 128; }
+__host__ __device__ inline int wide_x_bytes(int fmt, int segs, int cols) {
+    return wide_xsegs(fmt, segs) * cols * 128;
+}
 
 // x [M, k] bf16 -> f16 scaled by 2^e_m (the largest |x| of row m lands in [2^14, 2^15)),
 // as stage_to_f16 does in shared memory for the narrow sweep. One CTA per input row.
@@ -1013,36 +1015,40 @@ __global__ void __launch_bounds__(256) wide_x16_kernel(const uint16_t* __restric
 // One slab of one row group for 16 inputs (two MMA column blocks). The codes are read as in
 // slab_mma; the lane's x elements [e, e + V) of inputs g and g + 8 come from the stage's
 // x chunk, [x segment of 64 elements][16 inputs][128 B] with the 128-byte swizzle.
-template <int FMT>
-__device__ __forceinline__ void slab_mma_wide(float (&acc)[2][2][4], const uint8_t* cw,
+template <int FMT, int NT>
+__device__ __forceinline__ void slab_mma_wide(float (&acc)[2][NT][4], const uint8_t* cw,
                                               const uint8_t* sw, uint32_t spitch8,
                                               const uint8_t* xst, int e, int g) {
     const uint4 ra = lds128(cw);
     const uint4 rb = lds128(cw + 1024);
-    const uint8_t* x0 = xst + (e >> 6) * (kWCols * 128) + g * 128;  // input g
-    const uint8_t* x1 = x0 + 8 * 128;                                // input g + 8
-    const int cb = (e & 63) >> 3;                                    // first 16-byte chunk
-#define XQ(row, q) lds128((row) + ((((cb) + (q)) ^ g) << 4))
+    const uint8_t* x0 = xst + (e >> 6) * (8 * NT * 128) + g * 128;  // input g; t*8 + g below
+    const int cb = (e & 63) >> 3;                                     // first 16-byte chunk
+#define XQ(t, q) lds128(x0 + (t) * 1024 + ((((cb) + (q)) ^ g) << 4))
     if (FMT == 0) {
-        const uint4 xa = XQ(x0, 0), xb = XQ(x1, 0);
-        mma_bf16_16816(acc[0][0], ra.x, rb.x, ra.y, rb.y, xa.x, xa.y);
-        mma_bf16_16816(acc[1][0], ra.z, rb.z, ra.w, rb.w, xa.z, xa.w);
-        mma_bf16_16816(acc[0][1], ra.x, rb.x, ra.y, rb.y, xb.x, xb.y);
-        mma_bf16_16816(acc[1][1], ra.z, rb.z, ra.w, rb.w, xb.z, xb.w);
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+            const uint4 xa = XQ(t, 0);
+            mma_bf16_16816(acc[0][t], ra.x, rb.x, ra.y, rb.y, xa.x, xa.y);
+            mma_bf16_16816(acc[1][t], ra.z, rb.z, ra.w, rb.w, xa.z, xa.w);
+        }
     } else if (FMT == 1) {
         const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w};
         const uint32_t wb[4] = {rb.x, rb.y, rb.z, rb.w};
-        const uint4 xa0 = XQ(x0, 0), xa1 = XQ(x0, 1), xb0 = XQ(x1, 0), xb1 = XQ(x1, 1);
-        const uint32_t xa[8] = {xa0.x, xa0.y, xa0.z, xa0.w, xa1.x, xa1.y, xa1.z, xa1.w};
-        const uint32_t xb[8] = {xb0.x, xb0.y, xb0.z, xb0.w, xb1.x, xb1.y, xb1.z, xb1.w};
+        uint32_t a[4][4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const uint32_t a0 = e4m3x2_to_f16x2((uint16_t)(wa[i] & 0xFFFFu));
-            const uint32_t a2 = e4m3x2_to_f16x2((uint16_t)(wa[i] >> 16));
-            const uint32_t a1 = e4m3x2_to_f16x2((uint16_t)(wb[i] & 0xFFFFu));
-            const uint32_t a3 = e4m3x2_to_f16x2((uint16_t)(wb[i] >> 16));
-            mma_f16_16816(acc[i & 1][0], a0, a1, a2, a3, xa[2 * i], xa[2 * i + 1]);
-            mma_f16_16816(acc[i & 1][1], a0, a1, a2, a3, xb[2 * i], xb[2 * i + 1]);
+            a[i][0] = e4m3x2_to_f16x2((uint16_t)(wa[i] & 0xFFFFu));
+            a[i][2] = e4m3x2_to_f16x2((uint16_t)(wa[i] >> 16));
+            a[i][1] = e4m3x2_to_f16x2((uint16_t)(wb[i] & 0xFFFFu));
+            a[i][3] = e4m3x2_to_f16x2((uint16_t)(wb[i] >> 16));
+        }
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+            const uint4 x_0 = XQ(t, 0), x_1 = XQ(t, 1);
+            const uint32_t xa[8] = {x_0.x, x_0.y, x_0.z, x_0.w, x_1.x, x_1.y, x_1.z, x_1.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                mma_f16_16816(acc[i & 1][t], a[i][0], a[i][1], a[i][2], a[i][3], xa[2 * i], xa[2 * i + 1]);
         }
     } else {
         const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w};
@@ -1065,17 +1071,18 @@ __device__ __forceinline__ void slab_mma_wide(float (&acc)[2][2][4], const uint8
                 qa[q] = hmul2(qa[q], s_a);
                 qb[q] = hmul2(qb[q], s_b);
             }
-            const uint4 xv = XQ(x0, i), xw = XQ(x1, i);
-            mma_f16_16816(acc[0][0], qa[0], qb[0], qa[1], qb[1], xv.x, xv.y);
-            mma_f16_16816(acc[1][0], qa[2], qb[2], qa[3], qb[3], xv.z, xv.w);
-            mma_f16_16816(acc[0][1], qa[0], qb[0], qa[1], qb[1], xw.x, xw.y);
-            mma_f16_16816(acc[1][1], qa[2], qb[2], qa[3], qb[3], xw.z, xw.w);
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                const uint4 xv = XQ(t, i);
+                mma_f16_16816(acc[0][t], qa[0], qb[0], qa[1], qb[1], xv.x, xv.y);
+                mma_f16_16816(acc[1][t], qa[2], qb[2], qa[3], qb[3], xv.z, xv.w);
+            }
         }
     }
 #undef XQ
 }
 
-template <int FMT>
+template <int FMT, int NT>
 __global__ void __launch_bounds__(kWThreads, 1)
     sweep_wide_kernel(const __grid_constant__ SweepParams p, const __grid_constant__ CUtensorMap map_codes,
                       const __grid_constant__ CUtensorMap map_scales,
@@ -1084,6 +1091,9 @@ __global__ void __launch_bounds__(kWThreads, 1)
     constexpr int SLAB = 4 * V;
     constexpr int CW = kWCW;
     constexpr int REDUCER = CW, PRODUCER = CW + 1;
+    constexpr int COLS = 8 * NT;          // inputs per tile pass
+    constexpr int kWRedFloats = 16 * COLS;  // one warp's tile partial: 16 rows x COLS inputs
+    constexpr int LPI = 32 / COLS;        // reducer lanes per input (2 or 1)
 
     extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
@@ -1095,7 +1105,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
     volatile int* abort_flag = misc;
     volatile int* slot_tile = misc + 18;
     volatile int* red_tile = misc + 30;
-    float* red = reinterpret_cast<float*>(misc + 32);  // [2][CW][16 rows][16 inputs]
+    float* red = reinterpret_cast<float*>(misc + 32);  // [2][CW][16 rows][COLS inputs]
     const uint32_t head_end = smem_u32(red + 2 * CW * kWRedFloats);
     uint8_t* ring = smem + (((head_end + 1023u) & ~1023u) - smem_u32(smem));
 
@@ -1131,7 +1141,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
         int slot = 0;
         uint32_t phase = 0;
         int64_t issued = 0;
-        const uint32_t tx = (uint32_t)(code_b + scale_b + wide_x_bytes(FMT, segs));
+        const uint32_t tx = (uint32_t)(code_b + scale_b + wide_x_bytes(FMT, segs, COLS));
         bool stop = false;
         // every stage reads x, which the previous kernel (the f16 copy) may write
         pdl_wait();
@@ -1176,9 +1186,9 @@ __global__ void __launch_bounds__(kWThreads, 1)
 
     // ------------------------------------------------------------ reducer warp
     if (warp == REDUCER) {
-        // lane holds input m = lane & 15 and the rows of parity h = lane >> 4 of each tile,
-        // with a running (max, lowest row) and sum of exp over them
-        const int m = lane & 15, h = lane >> 4;
+        // lane holds input m = lane % COLS and the rows r = h (mod LPI), h = lane / COLS,
+        // of each tile, with a running (max, lowest row) and sum of exp over them
+        const int m = lane % COLS, h = lane / COLS;
         const bool lp = p.out_logprob != nullptr || p.out_partial != nullptr;
         pdl_wait();
         const float gsc = FMT == 2 ? __ldg(p.global_scale) : 1.f;
@@ -1209,16 +1219,16 @@ __global__ void __launch_bounds__(kWThreads, 1)
             }
             const float* rb = red + (size_t)buf * CW * kWRedFloats;
 #pragma unroll 4
-            for (int j = 0; j < 32; ++j) {
-                const int r = 2 * j + h;  // row within the tile
+            for (int j = 0; j < kWRows / LPI; ++j) {
+                const int r = LPI * j + h;  // row within the tile
                 const int rg = r >> 4, rr = r & 15;
                 // the four warps of the row group, in order
-                float a = rb[(rg + 0) * kWRedFloats + rr * kWCols + m];
-                a += rb[(rg + 4) * kWRedFloats + rr * kWCols + m];
-                a += rb[(rg + 8) * kWRedFloats + rr * kWCols + m];
-                a += rb[(rg + 12) * kWRedFloats + rr * kWCols + m];
+                float a = rb[(rg + 0) * kWRedFloats + rr * COLS + m];
+                a += rb[(rg + 4) * kWRedFloats + rr * COLS + m];
+                a += rb[(rg + 8) * kWRedFloats + rr * COLS + m];
+                a += rb[(rg + 12) * kWRedFloats + rr * COLS + m];
                 float rs = 1.f;
-                if (FMT == 1) rs = __shfl_sync(0xffffffffu, j < 16 ? rs_a : rs_b, r & 31);
+                if (FMT == 1) rs = __shfl_sync(0xffffffffu, LPI * j < 32 ? rs_a : rs_b, r & 31);
                 const int64_t row = row0 + r;
                 const bool valid = row < p.n && m < M;
                 float l = a;
@@ -1242,8 +1252,8 @@ __global__ void __launch_bounds__(kWThreads, 1)
             buf ^= 1;
         }
         if (*abort_flag) raise_flag(p.dev_err, DEVFLAG_TIMEOUT);
-        // fold the two row parities of each input, then lanes m < M publish
-        {
+        // fold the row parities of each input (two lanes at 16 inputs), then lanes m < M publish
+        if (LPI == 2) {
             const float ov = __shfl_xor_sync(0xffffffffu, best_v, 16);
             const int32_t oi = __shfl_xor_sync(0xffffffffu, best_i, 16);
             const float os = __shfl_xor_sync(0xffffffffu, se, 16);
@@ -1257,7 +1267,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
             }
         }
         Partial* parts = reinterpret_cast<Partial*>(p.partials);
-        if (h == 0 && m < M) parts[(int64_t)blockIdx.x * 16 + m] = Partial{best_v, best_i, se, 0.f};
+        if (h == 0 && m < M) parts[(int64_t)blockIdx.x * kPartSlots + m] = Partial{best_v, best_i, se, 0.f};
         __syncwarp();
         fence_acq_rel_gpu();  // every publishing lane's store before lane 0's ticket
         __syncwarp();
@@ -1278,11 +1288,11 @@ __global__ void __launch_bounds__(kWThreads, 1)
     const int total_slabs = (int)(K / SLAB);
     const int slabs_per_stage = 2 * segs;
 
-    float acc[2][2][4];
+    float acc[2][NT][4];
 #pragma unroll
     for (int a = 0; a < 2; ++a)
 #pragma unroll
-        for (int t = 0; t < 2; ++t)
+        for (int t = 0; t < NT; ++t)
 #pragma unroll
             for (int i = 0; i < 4; ++i) acc[a][t][i] = 0.f;
 
@@ -1301,7 +1311,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
             const int a0 = ch * slabs_per_stage;
             const int nv = min(slabs_per_stage, total_slabs - a0);
             for (int l = sub; l < nv; l += 4)
-                slab_mma_wide<FMT>(acc, st + (l >> 1) * (kWRows * 128) + ((l & 1) ? coff1 : coff0),
+                slab_mma_wide<FMT, NT>(acc, st + (l >> 1) * (kWRows * 128) + ((l & 1) ? coff1 : coff0),
                                    st + soff + l * 8, 8u * spitch, xst, l * SLAB + c * V, g);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[slot]);
@@ -1314,11 +1324,11 @@ __global__ void __launch_bounds__(kWThreads, 1)
         eph ^= 1u << buf;
         float* rp = red + (size_t)buf * CW * kWRedFloats + warp * kWRedFloats;
 #pragma unroll
-        for (int t = 0; t < 2; ++t)
+        for (int t = 0; t < NT; ++t)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int row = (i < 2 ? r0 : r0 + 8);
-                rp[row * kWCols + t * 8 + 2 * c + (i & 1)] = acc[0][t][i] + acc[1][t][i];
+                rp[row * COLS + t * 8 + 2 * c + (i & 1)] = acc[0][t][i] + acc[1][t][i];
                 acc[0][t][i] = acc[1][t][i] = 0.f;
             }
         if (warp == 0 && lane == 0) red_tile[buf] = tile;
@@ -1428,14 +1438,14 @@ cudaError_t make_scale_map(CUtensorMap* m, const void* base, int64_t rows, int64
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// x [M, k] of 16-bit elements as 64-element segments: boxes of kWCols rows (inputs past
+// x [M, k] of 16-bit elements as 64-element segments: boxes of `cols` rows (inputs past
 // M read as zeros) x xsegs segments, 128-byte swizzle.
-cudaError_t make_x_map(CUtensorMap* m, const void* base, int M, int64_t k, int xsegs) {
+cudaError_t make_x_map(CUtensorMap* m, const void* base, int M, int64_t k, int xsegs, int cols) {
     EncodeTiledFn fn = encode_tiled();
     if (!fn) return cudaErrorNotSupported;
     cuuint64_t dims[3] = {64, (cuuint64_t)M, (cuuint64_t)(k / 64)};
     cuuint64_t strides[2] = {(cuuint64_t)k * 2, 128};
-    cuuint32_t box[3] = {64, (cuuint32_t)kWCols, (cuuint32_t)xsegs};
+    cuuint32_t box[3] = {64, (cuuint32_t)cols, (cuuint32_t)xsegs};
     cuuint32_t es[3] = {1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(base), dims, strides,
                     box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -1451,10 +1461,10 @@ struct WideGeometry {
     size_t smem;
 };
 
-WideGeometry wide_geometry(int64_t k, int fmt) {
+WideGeometry wide_geometry(int64_t k, int fmt, int cols) {
     WideGeometry g{};
     size_t head = (size_t)(2 * kMaxStages + 4) * 8 + 32 * sizeof(int) +
-                  (size_t)2 * kWCW * kWRedFloats * sizeof(float);
+                  (size_t)2 * kWCW * 16 * cols * sizeof(float);
     head = ((head + 1023) & ~(size_t)1023) + 1024;
     const int64_t row_bytes = fmt == 0 ? k * 2 : fmt == 1 ? k : k / 2;
     const int row_segs = (int)(row_bytes / 128);
@@ -1463,7 +1473,7 @@ WideGeometry wide_geometry(int64_t k, int fmt) {
         for (int max_segs = 32; max_segs >= 1; --max_segs) {
             const int nc = (row_segs + max_segs - 1) / max_segs;
             const int segs = (row_segs + nc - 1) / nc;
-            const int sb = wide_code_bytes(segs) + wide_scale_bytes(fmt, segs) + wide_x_bytes(fmt, segs);
+            const int sb = wide_code_bytes(segs) + wide_scale_bytes(fmt, segs) + wide_x_bytes(fmt, segs, cols);
             int stages = avail > 0 ? (int)(avail / sb) : 0;
             if (stages > kMaxStages) stages = kMaxStages;
             if (stages >= want) {
@@ -1479,10 +1489,10 @@ WideGeometry wide_geometry(int64_t k, int fmt) {
     return g;
 }
 
-template <int FMT>
+template <int FMT, int NT>
 cudaError_t launch_wide(const SweepParams& p, cudaStream_t s, SweepLaunch* info) {
-    auto kern = sweep_wide_kernel<FMT>;
-    const WideGeometry geo = wide_geometry(p.k, FMT);
+    auto kern = sweep_wide_kernel<FMT, NT>;
+    const WideGeometry geo = wide_geometry(p.k, FMT, 8 * NT);
     if (geo.stages < 2) return cudaErrorInvalidValue;
     const int xsegs = wide_xsegs(FMT, geo.segs);
     CUtensorMap map_codes, map_scales, map_x;
@@ -1496,7 +1506,7 @@ cudaError_t launch_wide(const SweepParams& p, cudaStream_t s, SweepLaunch* info)
         map_scales = map_codes;  // unused
     }
     const void* xsrc = FMT == 0 ? static_cast<const void*>(p.x) : static_cast<const void*>(p.x16);
-    if ((e = make_x_map(&map_x, xsrc, p.M, p.k, xsegs)) != cudaSuccess) return e;
+    if ((e = make_x_map(&map_x, xsrc, p.M, p.k, xsegs, 8 * NT)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)geo.smem)) != cudaSuccess)
         return e;
@@ -1592,7 +1602,7 @@ cudaError_t launch_one(const SweepParams& p, cudaStream_t s, SweepLaunch* info) 
 
 size_t sweep_smem_bytes(int M, int64_t k, int fmt, int* kpad_out, int mode) {
     if (mode == 0 && M > 8) {  // the wide sweep stages x per K chunk
-        const WideGeometry w = wide_geometry(k, fmt);
+        const WideGeometry w = wide_geometry(k, fmt, M > 16 ? 32 : 16);
         if (kpad_out) *kpad_out = (int)k;
         return w.stages >= 2 ? w.smem : (size_t)kSmemLimit + 1;
     }
@@ -1664,9 +1674,10 @@ cudaError_t sweep_launch(const SweepParams& p, int fmt, int mode, cudaStream_t s
     const bool two = p.M > 8;
     if (fmt == 2 && mode == 0 && p.M <= 2) return launch_one<2, 1, 0, 1>(p, s, info);
     if (mode == 0 && two) {
-        if (fmt == 0) return launch_wide<0>(p, s, info);
-        if (fmt == 1) return launch_wide<1>(p, s, info);
-        if (fmt == 2) return launch_wide<2>(p, s, info);
+        const bool four = p.M > 16;
+        if (fmt == 0) return four ? launch_wide<0, 4>(p, s, info) : launch_wide<0, 2>(p, s, info);
+        if (fmt == 1) return four ? launch_wide<1, 4>(p, s, info) : launch_wide<1, 2>(p, s, info);
+        if (fmt == 2) return four ? launch_wide<2, 4>(p, s, info) : launch_wide<2, 2>(p, s, info);
     }
 #define MTP_SWEEP_CASE(F, NTV, MD) \
     if (fmt == F && (NTV == 2) == two && mode == MD) return launch_one<F, NTV, MD, 0>(p, s, info);

@@ -99,7 +99,7 @@ def test_lm_head_rejects(lib):
     assert lm(weight(), n_eff=101) == L.MTP_ERR_INVALID_ARG       # n_eff > n
     assert lm(weight(), n_eff=0) == L.MTP_ERR_INVALID_ARG
     assert lm(weight(), M=0) == L.MTP_ERR_UNSUPPORTED
-    assert lm(weight(), M=17) == L.MTP_ERR_UNSUPPORTED
+    assert lm(weight(), M=33) == L.MTP_ERR_UNSUPPORTED
     assert lm(weight(), x=B2 + 4) == L.MTP_ERR_INVALID_ARG
     assert lm(weight(), mask=OUT, mw=0) == L.MTP_ERR_INVALID_ARG
     assert lm(weight(), ws=None) == L.MTP_ERR_WORKSPACE
@@ -109,7 +109,9 @@ def test_lm_head_rejects(lib):
     assert lm(weight(fmt=1, k=80, rs=OUT)) == L.MTP_ERR_UNSUPPORTED
     assert lm(weight(fmt=2, k=224, bs=OUT, gs=OUT)) == L.MTP_ERR_UNSUPPORTED
     # staged inputs larger than shared memory
-    assert lm(weight(n=100, k=16384), M=16) == L.MTP_ERR_UNSUPPORTED
+    assert lm(weight(n=100, k=16384), M=8) == L.MTP_ERR_UNSUPPORTED
+    # more than eight inputs stream x per K chunk, so the same width is fine there
+    assert lm(weight(n=100, k=16384), M=16, ws=None) == L.MTP_ERR_WORKSPACE
     w = weight()
     w.reserved = 1
     assert lm(w) == L.MTP_ERR_INVALID_ARG
@@ -127,8 +129,12 @@ def test_lm_head_lp_rejects(lib):
     assert lp(OUT + 2) == L.MTP_ERR_INVALID_ARG     # f32 alignment
     assert lp(OUT, x=B2 + 4) == L.MTP_ERR_INVALID_ARG  # the same checks as mtp_lm_head_argmax
     assert lp(OUT, n_eff=101) == L.MTP_ERR_INVALID_ARG
-    # partials are 16 bytes (max, index, sum of exponentials) for up to 1,024 CTAs x 16 rows
-    assert wsb == 256 + 16 * 16 * 1024 and L.mtp_noalloc_scratch_bytes() == wsb
+    # partials are 16 bytes (max, index, sum of exponentials) for up to 1,024 CTAs x 32 inputs
+    assert wsb == 256 + 16 * 32 * 1024 and L.mtp_noalloc_scratch_bytes() == wsb
+    # more than eight inputs on a quantized table add an f16 copy of x (+ 1 KB of exponents)
+    fp8 = weight(fmt=1, k=128, rs=OUT)
+    assert L.mtp_lm_head_ws_bytes(fp8, 100, 9) == wsb + ((9 * 128 * 2 + 1023) // 1024) * 1024 + 1024
+    assert L.mtp_lm_head_ws_bytes(weight(k=128), 100, 32) == wsb
 
 
 def test_shard_and_merge_rejects(lib):
@@ -153,7 +159,7 @@ def test_shard_and_merge_rejects(lib):
     assert merge(A, 2, 1, idx=None) == L.MTP_ERR_INVALID_ARG
     assert merge(A + 8, 2, 1) == L.MTP_ERR_INVALID_ARG
     assert merge(A, 2, 0) == L.MTP_ERR_UNSUPPORTED
-    assert merge(A, 2, 17) == L.MTP_ERR_UNSUPPORTED
+    assert merge(A, 2, 33) == L.MTP_ERR_UNSUPPORTED
 
 
 def test_combine_rejects(lib):

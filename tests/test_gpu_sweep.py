@@ -4,7 +4,7 @@ Small tables span several 16-row tiles, several CTAs and a ragged tail; the full
 tables are the benchmark's (154,880 x 4,096 BF16 and FP8, 131,072 x 5,120 NVFP4) in
 the launch configuration bench.py times. Logits within 2e-2 + 1e-2|ref|; argmax exact
 where the top-2 gap exceeds 1e-2; one-hot inputs and batch invariance bit-exact within
-each range of M that one sweep serves (1-8, 9-16; NVFP4 1-2, 3-8, 9-16)."""
+each range of M that one sweep serves (1-8, 9-16, 17-32; NVFP4 1-2, 3-8, 9-16, 17-32)."""
 import numpy as np
 import pytest
 import torch
@@ -88,7 +88,7 @@ SHAPES = {0: [(1000, 256), (1000, 4096), (4133, 576)],
 
 
 @pytest.mark.parametrize("fmt", [0, 1, 2])
-@pytest.mark.parametrize("M", [1, 3, 8, 9, 16])
+@pytest.mark.parametrize("M", [1, 3, 8, 9, 16, 17, 32])
 def test_sweep_small_tables(orc, fmt, M):
     for n, k in SHAPES[fmt]:
         w = synth.as_u16(synth.normal_bf16(synth._gen(n + k + fmt), (n, k), 0.02))
@@ -120,14 +120,15 @@ def test_one_hot_inputs_are_bit_exact(orc, fmt):
 def test_batch_invariance(orc, fmt):
     n, k = 2000, 1024
     w = synth.as_u16(synth.normal_bf16(synth._gen(9), (n, k), 0.02))
-    x = synth.as_u16(synth.normal_bf16(synth._gen(10), (16, k), 1.0))
+    x = synth.as_u16(synth.normal_bf16(synth._gen(10), (32, k), 1.0))
     table = device_table(oracle_quant(orc, w, fmt), fmt, n, k)
     head = api.LmHead(table)
     # Three sweeps share the work: NVFP4 with one or two inputs applies the block scales
     # to per-block fp32 sums, more than eight inputs use 64-row tiles with x streamed per
     # K chunk; each sums the same exact products in its own fixed order, so results are
     # bit-identical within each range of M and within the tolerance across them
-    groups = ([(1, 2), (3, 4, 8), (9, 16)] if fmt == 2 else [(1, 2, 3, 4, 8), (9, 12, 16)])
+    groups = ([(1, 2), (3, 4, 8), (9, 12, 16), (17, 24, 32)] if fmt == 2
+              else [(1, 2, 3, 4, 8), (9, 12, 16), (17, 24, 32)])
     bases = []
     for grp in groups:
         base = run_sweep(table, x[:grp[0]], head=head)
@@ -140,8 +141,8 @@ def test_batch_invariance(orc, fmt):
         assert_close(bf16_bits_to_f64(b[2][0]), bf16_bits_to_f64(bases[0][2][0]), "across ranges of M")
     # row m keeps its result whatever the other rows are
     x2 = x.copy()
-    x2[1:] = x[::-1][:15]
-    for M in (2, 16):
+    x2[1:] = x[::-1][:31]
+    for M in (2, 16, 32):
         a = run_sweep(table, x[:M], head=head)
         b = run_sweep(table, x2[:M], head=head)
         assert np.array_equal(a[2][0], b[2][0]), M
@@ -246,7 +247,7 @@ def oracle_logprobs(orc, ref_l, mask=None, mask_words=0, stride=0):
 
 
 @pytest.mark.parametrize("fmt", [0, 1, 2])
-@pytest.mark.parametrize("M", [1, 2, 3, 9, 16])
+@pytest.mark.parametrize("M", [1, 2, 3, 9, 16, 32])
 def test_top1_logprob(orc, fmt, M):
     """mtp_lm_head_argmax_lp: the argmax outputs equal mtp_lm_head_argmax's bit for bit,
     and the top-1 log-probability matches the oracle's (fp64 log-softmax at the argmax)
