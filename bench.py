@@ -590,6 +590,26 @@ def main():
             rows[f"{fmt}_M{M}"] = rec
             if fmt == "bf16" and M == 1:
                 main_line = (rec, nbytes, ms_max, kern_max, e2e_max, h2d, d2h, clk, cfg)
+        if args.full:  # wide batches: 16 and 32 inputs (seeded N(0, 1) rows; timing only)
+            for Mw in (16, 32):
+                gen = torch.Generator().manual_seed(Mw)
+                xw = torch.randn((Mw, cfg["K"]), generator=gen).to(torch.bfloat16).to(dev)
+                iw = torch.empty((Mw,), dtype=torch.int32, device=dev)
+                for _ in range(args.warmup):
+                    head(xw, iw, None, stream=stream)
+                torch.cuda.synchronize()
+                s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                with torch.cuda.stream(stream):
+                    s.record(stream)
+                    for _ in range(max(1, args.steps // 4)):
+                        head(xw, iw, None, stream=stream)
+                    e.record(stream)
+                torch.cuda.synchronize()
+                us = s.elapsed_time(e) / max(1, args.steps // 4) * 1e3
+                rows.setdefault(f"{fmt}_M{Mw}", {"us_per_draft": us,
+                                                 "kernel_GB/s": head.bytes_per_call(Mw) / (us * 1e-6) / 1e9,
+                                                 "frac_of_peak": head.bytes_per_call(Mw) / (us * 1e-6) / 1e9 / peak,
+                                                 "note": "timing only (random inputs)"})
         # the same sweep with the top-1 log-probability (mtp_lm_head_argmax_lp), M = 1
         x = d["x"][:1].to(dev)
         idx = torch.empty((1,), dtype=torch.int32, device=dev)
