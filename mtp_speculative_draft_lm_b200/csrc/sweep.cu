@@ -977,6 +977,7 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
 constexpr int kWRows = 64;
 constexpr int kWCW = 16;                  // compute warps
 constexpr int kWThreads = (kWCW + 2) * 32;
+constexpr int kWRedBuffers = 2;           // reducer hand-off buffers (double-buffered)
 // inputs per sweep: 8 NT columns (NT = 2: up to 16 inputs, NT = 4: up to 32)
 
 __host__ __device__ inline int wide_seg_elems(int fmt) { return fmt == 0 ? 64 : fmt == 1 ? 128 : 256; }
@@ -1094,6 +1095,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
     constexpr int COLS = 8 * NT;          // inputs per tile pass
     constexpr int kWRedFloats = 16 * COLS;  // one warp's tile partial: 16 rows x COLS inputs
     constexpr int LPI = 32 / COLS;        // reducer lanes per input (2 or 1)
+    constexpr int NB = kWRedBuffers;  // tile hand-off buffers (one measured slower)
 
     extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
@@ -1105,8 +1107,8 @@ __global__ void __launch_bounds__(kWThreads, 1)
     volatile int* abort_flag = misc;
     volatile int* slot_tile = misc + 18;
     volatile int* red_tile = misc + 30;
-    float* red = reinterpret_cast<float*>(misc + 32);  // [2][CW][16 rows][COLS inputs]
-    const uint32_t head_end = smem_u32(red + 2 * CW * kWRedFloats);
+    float* red = reinterpret_cast<float*>(misc + 32);  // [NB][CW][16 rows][COLS inputs]
+    const uint32_t head_end = smem_u32(red + NB * CW * kWRedFloats);
     uint8_t* ring = smem + (((head_end + 1023u) & ~1023u) - smem_u32(smem));
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1249,7 +1251,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&red_empty[buf]);
-            buf ^= 1;
+            buf = (buf + 1) % NB;
         }
         if (*abort_flag) raise_flag(p.dev_err, DEVFLAG_TIMEOUT);
         // fold the row parities of each input (two lanes at 16 inputs), then lanes m < M publish
@@ -1334,7 +1336,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
         if (warp == 0 && lane == 0) red_tile[buf] = tile;
         __syncwarp();
         if (lane == 0) mbar_arrive(&red_full[buf]);
-        buf ^= 1;
+        buf = (buf + 1) % NB;
     }
     if (mbar_wait_bounded(&red_empty[buf], ((eph >> buf) & 1u) ^ 1u, abort_flag)) {
         if (warp == 0 && lane == 0) red_tile[buf] = -1;
@@ -1464,7 +1466,7 @@ struct WideGeometry {
 WideGeometry wide_geometry(int64_t k, int fmt, int cols) {
     WideGeometry g{};
     size_t head = (size_t)(2 * kMaxStages + 4) * 8 + 32 * sizeof(int) +
-                  (size_t)2 * kWCW * 16 * cols * sizeof(float);
+                  (size_t)kWRedBuffers * kWCW * 16 * cols * sizeof(float);
     head = ((head + 1023) & ~(size_t)1023) + 1024;
     const int64_t row_bytes = fmt == 0 ? k * 2 : fmt == 1 ? k : k / 2;
     const int row_segs = (int)(row_bytes / 128);
@@ -1681,9 +1683,8 @@ cudaError_t sweep_launch(const SweepParams& p, int fmt, int mode, cudaStream_t s
     }
 #define MTP_SWEEP_CASE(F, NTV, MD) \
     if (fmt == F && (NTV == 2) == two && mode == MD) return launch_one<F, NTV, MD, 0>(p, s, info);
-    MTP_SWEEP_CASE(0, 1, 0) MTP_SWEEP_CASE(0, 2, 0)
-    MTP_SWEEP_CASE(1, 1, 0) MTP_SWEEP_CASE(1, 2, 0)
-    MTP_SWEEP_CASE(2, 1, 0) MTP_SWEEP_CASE(2, 2, 0)
+    // (mode 0 with more than eight inputs went to the wide sweep above)
+    MTP_SWEEP_CASE(0, 1, 0) MTP_SWEEP_CASE(1, 1, 0) MTP_SWEEP_CASE(2, 1, 0)
     MTP_SWEEP_CASE(0, 1, 1) MTP_SWEEP_CASE(0, 2, 1)
     MTP_SWEEP_CASE(1, 1, 1) MTP_SWEEP_CASE(1, 2, 1)
     MTP_SWEEP_CASE(2, 1, 1) MTP_SWEEP_CASE(2, 2, 1)

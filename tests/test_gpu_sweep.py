@@ -181,6 +181,32 @@ def test_masks_decoys_and_edge_cases(orc):
     assert np.array_equal(got[0][[0, 1, 3]], d["second"][[0, 1, 3]])
 
 
+@pytest.mark.parametrize("M", [12, 32])
+def test_masks_and_n_eff_many_inputs(orc, M):
+    """The 64-row-tile sweep (more than eight inputs): per-row masks with a decoy, a shared
+    mask, an all-zero mask row, masked logits -inf, and an n_eff that ends mid-tile."""
+    n, k = 4133, 512
+    d = synth.head_table(13 + M, n, k, M, mask_keep=0.1)
+    w, x = synth.as_u16(d["W"]), synth.as_u16(d["x"])
+    words = d["mask"].shape[1]
+    for fmt in (0, 1, 2):
+        q = oracle_quant(orc, w, fmt)
+        table = device_table(q, fmt, n, k)
+        got = run_sweep(table, x)
+        assert np.array_equal(got[0], d["top"])
+        mask = d["mask"].copy()
+        mask[M // 2] = 0
+        got = run_sweep(table, x, mask=mask.reshape(-1), mask_words=words, stride=words)
+        check(orc, fmt, q, k, x, got, mask=mask.reshape(-1), mask_words=words, stride=words)
+        keep = [m for m in range(M) if m != M // 2]
+        assert np.array_equal(got[0][keep], d["second"][keep])
+        assert got[0][M // 2] == 0 and got[1][M // 2] == -np.inf
+        got = run_sweep(table, x, mask=d["mask"][0], mask_words=words, stride=0)
+        check(orc, fmt, q, k, x, got, mask=d["mask"][0], mask_words=words, stride=0)
+        got = run_sweep(table, x, n_eff=2011)
+        check(orc, fmt, q, k, x, got, n_eff=2011)
+
+
 def test_duplicate_rows_lowest_index_and_n_eff(orc):
     n, k = 3000, 256
     d = synth.head_table(12, n, k, 1)
