@@ -311,7 +311,10 @@ mtp_status mtp_debug_kv_write(const uint16_t* k_rot, const uint16_t* v, int64_t 
  * code that must not risk the device synchronisation cudaMalloc/cudaFree can cause).
  * Inputs and outputs are the caller's, exactly as for mtp_lm_head_argmax; the scratch
  * is a static device array inside the library, mtp_noalloc_scratch_bytes() bytes
- * (262,400) held on every GPU that loads the library until the process exits.
+ * (524,544: a 256-byte header + 16-byte partials of up to 1,024 CTAs x 32 input rows)
+ * held on every GPU that loads the library until the process exits. It has no room
+ * for the f16 copy of x that FP8 and NVFP4 tables need above M = 8, so those calls
+ * return MTP_ERR_WORKSPACE here; BF16 tables run at every M up to 32.
  *  - The first call made with a device current looks up that array's device address
  *    and zeroes its counter (synchronously); make it before any stream capture.
  *  - All calls on a device share the array: calls that overlap on the GPU race and

@@ -135,6 +135,11 @@ def test_lm_head_lp_rejects(lib):
     fp8 = weight(fmt=1, k=128, rs=OUT)
     assert L.mtp_lm_head_ws_bytes(fp8, 100, 9) == wsb + ((9 * 128 * 2 + 1023) // 1024) * 1024 + 1024
     assert L.mtp_lm_head_ws_bytes(weight(k=128), 100, 32) == wsb
+    # the no-alloc array has no room for that copy: rejected before any CUDA call
+    noalloc = lambda head, M: st("mtp_lm_head_argmax_noalloc", C.byref(head), 100, B2, M, None,
+                                 0, 0, OUT, None, None, None, None)
+    assert noalloc(fp8, 9) == L.MTP_ERR_WORKSPACE
+    assert noalloc(weight(fmt=2, k=128, bs=OUT, gs=OUT), 12) == L.MTP_ERR_WORKSPACE
 
 
 def test_shard_and_merge_rejects(lib):
