@@ -205,11 +205,11 @@ mtp_status lm_head_impl(const mtp_weight* head, int64_t n_eff, const uint16_t* x
     p.dev_err = dev_err;
     p.ticket = static_cast<uint32_t*>(ws);
     p.partials = static_cast<uint8_t*>(ws) + kTicketBytes;
-    if (mtp::sweep_x16_bytes(M, head->k, head->fmt)) {  // the wide sweep's f16 copy of x
+    if (mtp::sweep_x16_bytes(M, head->k, head->fmt)) {  // x as the many-input sweeps read it
         uint8_t* xb = static_cast<uint8_t*>(ws) + kTicketBytes + kPartialBytes * kPartSlots *
                                                                    (size_t)mtp::sweep_max_grid();
         p.x16 = reinterpret_cast<uint16_t*>(xb);
-        p.xexp = reinterpret_cast<int32_t*>(xb + (((size_t)M * head->k * 2 + 1023) & ~(size_t)1023));
+        p.xexp = reinterpret_cast<int32_t*>(xb + mtp::sweep_x16_bytes(M, head->k, head->fmt) - 1024);
     }
     p.num_tiles = (n_eff + 15) / 16;
     p.scale_pitch = mtp::nvfp4_scale_pitch(head->k);

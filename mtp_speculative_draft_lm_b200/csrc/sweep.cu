@@ -49,6 +49,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tcgen05.cuh"
 
 namespace mtp {
 namespace {
@@ -1345,6 +1346,348 @@ __global__ void __launch_bounds__(kWThreads, 1)
     }
 }
 
+// ---------------------------------------------------------------- tcgen05 sweep
+// BF16 and FP8 tables with 9-32 inputs run the contraction on the tcgen05 tensor cores:
+// one 128 x N x k MMA per 16 (BF16) or 32 (FP8) elements of K, with 128 table rows as A
+// and the N = 16 or 32 (padded) inputs as B, both read by the tensor core straight from
+// the TMA-written stage (K-major, 128-byte swizzle), the fp32 accumulator in tensor
+// memory. Nothing is decoded: FP8 codes are E4M3 operands as stored. x enters FP8 MMAs as
+// two E4M3 terms, hi = e4m3(x 2^e) and lo = e4m3(x 2^e - hi), with e_m chosen per input
+// so that its largest |x| lands in [128, 256); hi + lo equals x 2^e exactly wherever
+// x 2^e >= 1/4 (a bf16 value has 8 significant bits, hi keeps 4 and the rest fits lo's 4),
+// and within 2^-10 below that, i.e. within 2^-17 of the input's largest |x|.
+// Roles: warp 0 streams stages (128 table rows x segs 128-byte segments, plus the inputs'
+// same K range) through an mbarrier ring; warp 1 allocates tensor memory, issues the
+// MMAs from one thread and releases each stage with tcgen05.commit; warps 2-5 (tensor
+// memory lane quarters warp % 4) read the accumulator, one table row per thread, scale,
+// mask, keep per input a running (max, lowest row, sum of exp) and write the optional
+// logits. Two accumulators alternate so the MMAs of a tile overlap the previous tile's
+// epilogue. Tiles of 128 rows are handed out at run time as in the narrow sweep; the CTA
+// partials are folded by the last CTA (ticket_and_fold).
+constexpr int kTRows = 128;     // table rows per tile: the MMA's M
+constexpr int kTThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int kTEpiWarps = 4;
+
+__host__ __device__ inline int tc_x_rows(int fmt, int N) { return fmt == 1 ? 2 * N : N; }
+__host__ __device__ inline int tc_stage_bytes(int fmt, int N, int segs) {
+    return (kTRows + tc_x_rows(fmt, N)) * 128 * segs;
+}
+
+// x [M, k] bf16 -> the two E4M3 planes the FP8 MMAs read, [hi: N rows | lo: N rows] x k,
+// of x scaled by 2^e_m (the largest |x| of row m lands in [128, 256)); rows m >= M are
+// zero. One CTA per plane row.
+__global__ void __launch_bounds__(256) tc_xq_kernel(const uint16_t* __restrict__ x, int M, int k,
+                                                    int N, uint8_t* __restrict__ xq,
+                                                    int32_t* __restrict__ xexp) {
+    __shared__ float red[8];
+    const int m = blockIdx.x, tid = threadIdx.x;
+    uint8_t* hi = xq + (int64_t)m * k;
+    uint8_t* lo = xq + (int64_t)(N + m) * k;
+    if (m >= M) {
+        for (int j = tid; j < k; j += 256) hi[j] = lo[j] = 0;
+        return;
+    }
+    const uint16_t* row = x + (int64_t)m * k;
+    float a = 0.f;
+    for (int j = tid; j < k; j += 256) a = fmaxf(a, fabsf(bf16_to_f32(row[j])));
+    for (int o = 16; o; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if ((tid & 31) == 0) red[tid >> 5] = a;
+    __syncthreads();
+    a = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) a = fmaxf(a, red[w]);
+    int ex = 0;
+    if (a > 0.f) frexpf(a, &ex);  // a in [2^(ex-1), 2^ex)
+    const int e = (a > 0.f) ? 8 - ex : 0;
+    if (tid == 0) xexp[m] = e;
+    const float f1 = ldexpf(1.f, e / 2), f2 = ldexpf(1.f, e - e / 2);
+    for (int j = 2 * tid; j < k; j += 512) {  // k is even
+        const float v0 = (bf16_to_f32(row[j]) * f1) * f2;
+        const float v1 = (bf16_to_f32(row[j + 1]) * f1) * f2;
+        const uint16_t h = f32x2_to_e4m3x2(v0, v1);
+        const float r0 = v0 - e4m3_to_f32(h & 0xFFu), r1 = v1 - e4m3_to_f32(h >> 8);
+        const uint16_t l = f32x2_to_e4m3x2(r0, r1);
+        *reinterpret_cast<uint16_t*>(hi + j) = h;
+        *reinterpret_cast<uint16_t*>(lo + j) = l;
+    }
+}
+
+template <int FMT, int N>
+__global__ void __launch_bounds__(kTThreads, 1)
+    sweep_tc_kernel(const __grid_constant__ SweepParams p, const __grid_constant__ CUtensorMap map_codes,
+                    const __grid_constant__ CUtensorMap map_x) {
+    static_assert(FMT == 0 || FMT == 1, "BF16 and FP8 tables");
+    static_assert(N == 16 || N == 32, "16 or 32 input columns");
+    constexpr int XR = FMT == 1 ? 2 * N : N;  // x rows per stage segment (hi and lo for FP8)
+    constexpr uint32_t kTmemCols = 2 * N < 32 ? 32 : 2 * N;
+
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + kMaxStages;
+    uint64_t* tfull = empty + kMaxStages;  // [2]: the tile's MMAs done + its tile index posted
+    uint64_t* tempty = tfull + 2;          // [2]: the epilogue has read the accumulator
+    uint64_t* done = tempty + 2;           // every MMA done (before tensor memory is freed)
+    // bytes [0, 232): barriers; [232, 360): misc; [512, 768): sfac; [768, 2816): fold
+    int* misc = reinterpret_cast<int*>(done + 1);
+    volatile int* abort_flag = misc;            // [0]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 1);
+    volatile int* slot_tile = misc + 2;         // [2 .. 2 + kMaxStages)
+    volatile int* acc_tile = misc + 2 + kMaxStages;  // [2]
+    float* sfac = reinterpret_cast<float*>(smem + 512);    // [2][32]: 2^-e_m as two factors
+    float4* fold = reinterpret_cast<float4*>(smem + 768);  // [4 warps][32 inputs]
+    const uint32_t head_end = smem_u32(fold + kTEpiWarps * 32);
+    uint8_t* ring = smem + (((head_end + 1023u) & ~1023u) - smem_u32(smem));
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int S = p.stages;
+    const int stage_bytes = p.stage_bytes;
+    const int segs = p.segs;
+    const int NC = p.stages_per_tile;
+    const int M = p.M;
+    const int64_t T = p.num_tiles;
+    const int a_bytes = kTRows * 128 * segs;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 2);
+            mbar_init(&tempty[b], kTEpiWarps);
+        }
+        mbar_init(done, 1);
+        misc[0] = 0;
+        mbar_fence_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    pdl_launch_dependents();
+
+    if (warp == 0) {
+        // ---------------- producer: the tiles' stages, each tagged with its tile
+        int slot = 0;
+        uint32_t phase = 0;
+        int64_t issued = 0;
+        const uint32_t tx = (uint32_t)stage_bytes;
+        bool stop = false;
+        pdl_wait();  // x (and for FP8 its E4M3 planes) come from the previous grid
+        int64_t tile = blockIdx.x;
+        int64_t pending = 0;
+        if (lane == 0) pending = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
+        while (tile < T && !stop) {
+            for (int ch = 0; ch < NC; ++ch) {
+                if (!mbar_wait_bounded(&empty[slot], phase ^ 1u, abort_flag)) {
+                    stop = true;
+                    break;
+                }
+                if (lane == 0) {
+                    uint8_t* dst = ring + (size_t)slot * stage_bytes;
+                    slot_tile[slot] = (int)tile;
+                    mbar_arrive_expect_tx(&full[slot], tx);
+                    tma_load_3d(dst, &map_codes, 0, (int)(tile * kTRows), ch * segs, &full[slot]);
+                    tma_load_3d(dst + a_bytes, &map_x, 0, 0, ch * segs, &full[slot]);
+                }
+                __syncwarp();
+                ++issued;
+                if (++slot == S) {
+                    slot = 0;
+                    phase ^= 1u;
+                }
+            }
+            tile = __shfl_sync(0xffffffffu, pending, 0);
+            if (lane == 0 && tile < T) pending = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
+        }
+        // no copy left in flight; then the end marker (a stage tagged -1, no copy)
+        for (int64_t j = issued > S ? issued - S : 0; j < issued; ++j)
+            if (!mbar_wait_bounded(&full[j % S], (uint32_t)((j / S) & 1), nullptr)) break;
+        if (!stop && mbar_wait_bounded(&empty[slot], phase ^ 1u, abort_flag) && lane == 0) {
+            slot_tile[slot] = -1;
+            mbar_arrive(&full[slot]);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------- MMA issuer (lane 0)
+        constexpr uint32_t idesc = FMT == 0 ? idesc_bf16(kTRows, N) : idesc_e4m3(kTRows, N);
+        int slot = 0;
+        uint32_t phase = 0;
+        int local = 0;
+        while (true) {
+            if (!mbar_wait_bounded(&full[slot], phase, abort_flag)) break;
+            const int tile = slot_tile[slot];
+            const int buf = local & 1;
+            const uint32_t tph = (uint32_t)((local >> 1) & 1);
+            if (!mbar_wait_bounded(&tempty[buf], tph ^ 1u, abort_flag)) break;
+            if (lane == 0) {  // the tile index for the epilogue (its own arrival, release)
+                acc_tile[buf] = tile;
+                mbar_arrive(&tfull[buf]);
+                if (tile < 0) mbar_arrive(&tfull[buf]);  // no MMAs behind the end marker
+            }
+            __syncwarp();
+            if (tile < 0) break;
+            const uint32_t d_tmem = tmem_base + (uint32_t)(buf * N);
+            bool ok = true;
+            for (int ch = 0; ch < NC; ++ch) {
+                if (ch > 0 && !mbar_wait_bounded(&full[slot], phase, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t a0 = smem_u32(ring + (size_t)slot * stage_bytes);
+                    const uint32_t x0 = a0 + (uint32_t)a_bytes;
+                    for (int sg = 0; sg < segs; ++sg) {
+                        const uint32_t as = a0 + (uint32_t)sg * (kTRows * 128);
+                        const uint32_t xs = x0 + (uint32_t)sg * (XR * 128);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint32_t acc = (ch > 0 || sg > 0 || k > 0) ? 1u : 0u;
+                            if (FMT == 0) {
+                                umma_bf16(d_tmem, sdesc_k128(as + k * 32), sdesc_k128(xs + k * 32), idesc, acc);
+                            } else {
+                                umma_e4m3(d_tmem, sdesc_k128(as + k * 32), sdesc_k128(xs + k * 32), idesc, acc);
+                                umma_e4m3(d_tmem, sdesc_k128(as + k * 32), sdesc_k128(xs + N * 128 + k * 32),
+                                          idesc, 1u);
+                            }
+                        }
+                    }
+                    umma_commit(&empty[slot]);  // frees the stage once these MMAs have read it
+                }
+                __syncwarp();
+                if (++slot == S) {
+                    slot = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (lane == 0) umma_commit(&tfull[buf]);  // the accumulator, once complete
+            __syncwarp();
+            ++local;
+            if (!ok) break;
+        }
+        if (lane == 0) umma_commit(done);
+        __syncwarp();
+        mbar_wait_bounded(done, 0u, nullptr);
+    } else {
+        // ---------------- epilogue: warp w reads tensor memory lanes 32 (w % 4) + [0, 32)
+        const int q = warp & 3;
+        const int ew = warp - 2;  // 0..3
+        const bool lp = p.out_logprob != nullptr || p.out_partial != nullptr;
+        pdl_wait();
+        if (ew == 0) {
+            const int e = (FMT == 1 && lane < M) ? -__ldg(p.xexp + lane) : 0;
+            sfac[lane] = ldexpf(1.f, e / 2);
+            sfac[32 + lane] = ldexpf(1.f, e - e / 2);
+        }
+        named_sync(1, kTEpiWarps * 32);
+        float best_v[N], se[N];
+        int32_t best_i[N];
+#pragma unroll
+        for (int m = 0; m < N; ++m) {
+            best_v[m] = -INFINITY;
+            best_i[m] = INT_MAX;
+            se[m] = 0.f;
+        }
+        int local = 0;
+        while (true) {
+            const int buf = local & 1;
+            const uint32_t tph = (uint32_t)((local >> 1) & 1);
+            if (!mbar_wait_bounded(&tfull[buf], tph, abort_flag)) break;
+            const int tile = acc_tile[buf];
+            if (tile < 0) break;
+            tc_fence_after();
+            uint32_t v[N];
+            const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * N);
+            if constexpr (N == 32)
+                tmem_ld32(ta, v);
+            else
+                tmem_ld16(ta, v);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[buf]);  // the accumulator is free again
+            const int64_t row = (int64_t)tile * kTRows + q * 32 + lane;
+            const bool rvalid = row < p.n;
+            const float rs = (FMT == 1 && rvalid) ? __ldg(p.row_scale + row) : 1.f;
+#pragma unroll
+            for (int m = 0; m < N; ++m) {
+                if (m >= M) break;
+                float l = __uint_as_float(v[m]);
+                if (FMT == 1) l = ((l * sfac[m]) * sfac[32 + m]) * rs;
+                const bool ok = rvalid && mask_allows(p, m, row);
+                if (rvalid && p.out_logits)
+                    p.out_logits[(int64_t)m * p.n + row] = ok ? f32_to_bf16(l) : (uint16_t)0xFF80u;
+                if (lp && ok && l > -INFINITY) {
+                    float bv = best_v[m];
+                    lse_merge(bv, se[m], l, 1.f);
+                }
+                // each thread's rows arrive in increasing order: the lowest wins a tie
+                if (ok && (l > best_v[m] || (l == best_v[m] && best_i[m] == INT_MAX))) {
+                    best_v[m] = l;
+                    best_i[m] = (int32_t)row;
+                }
+            }
+            ++local;
+        }
+        // per input: fold the 32 lanes, then the four warps in order; publish; ticket
+#pragma unroll
+        for (int m = 0; m < N; ++m) {
+            if (m >= M) break;
+#pragma unroll
+            for (int o = 16; o; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, best_v[m], o);
+                const int32_t oi = __shfl_xor_sync(0xffffffffu, best_i[m], o);
+                const float os = __shfl_xor_sync(0xffffffffu, se[m], o);
+                if (lp) {
+                    float bv = best_v[m];
+                    lse_merge(bv, se[m], ov, os);
+                }
+                if (ov > best_v[m] || (ov == best_v[m] && oi < best_i[m])) {
+                    best_v[m] = ov;
+                    best_i[m] = oi;
+                }
+            }
+            if (lane == 0) fold[ew * 32 + m] = make_float4(best_v[m], __int_as_float(best_i[m]), se[m], 0.f);
+        }
+        named_sync(1, kTEpiWarps * 32);
+        if (ew == 0) {
+            if (lane < M) {
+                float bv = -INFINITY, bs = 0.f;
+                int32_t bi = INT_MAX;
+                for (int w = 0; w < kTEpiWarps; ++w) {
+                    const float4 f = fold[w * 32 + lane];
+                    const int32_t fi = __float_as_int(f.y);
+                    if (lp) {
+                        float t = bv;
+                        lse_merge(t, bs, f.x, f.z);
+                    }
+                    if (f.x > bv || (f.x == bv && fi < bi)) {
+                        bv = f.x;
+                        bi = fi;
+                    }
+                }
+                reinterpret_cast<Partial*>(p.partials)[(int64_t)blockIdx.x * kPartSlots + lane] =
+                    Partial{bv, bi, bs, 0.f};
+            }
+            __syncwarp();
+            fence_acq_rel_gpu();  // every publishing lane's store before lane 0's ticket
+            __syncwarp();
+            if (*abort_flag && lane == 0) raise_flag(p.dev_err, DEVFLAG_TIMEOUT);
+            ticket_and_fold(p, lane, lp);
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
 struct Geometry {
     int kpad;
     int segs;             // 128-byte segments per row per stage
@@ -1600,11 +1943,94 @@ cudaError_t launch_one(const SweepParams& p, cudaStream_t s, SweepLaunch* info) 
     return cudaGetLastError();
 }
 
+// Stage geometry of the tcgen05 sweep: the largest number of 128-byte segments per
+// stage (at most 4) that still leaves at least four stages (else three, else two).
+WideGeometry tc_geometry(int64_t k, int fmt, int N) {
+    WideGeometry g{};
+    size_t head = 768 + (size_t)kTEpiWarps * 32 * 16;  // barriers, misc, sfac, fold
+    head = ((head + 1023) & ~(size_t)1023) + 1024;
+    const int64_t row_bytes = fmt == 0 ? k * 2 : k;
+    const int row_segs = (int)(row_bytes / 128);
+    const long avail = (long)kSmemLimit - (long)head;
+    for (int want = 4; want >= 2 && g.stages < 2; --want) {
+        for (int max_segs = 4; max_segs >= 1; --max_segs) {
+            const int nc = (row_segs + max_segs - 1) / max_segs;
+            const int segs = (row_segs + nc - 1) / nc;
+            const int sb = tc_stage_bytes(fmt, N, segs);
+            int stages = avail > 0 ? (int)(avail / sb) : 0;
+            if (stages > kMaxStages) stages = kMaxStages;
+            if (stages >= want) {
+                g.segs = segs;
+                g.stages_per_tile = nc;
+                g.stage_bytes = sb;
+                g.stages = stages;
+                break;
+            }
+        }
+    }
+    g.smem = head + (size_t)g.stages * g.stage_bytes;
+    return g;
+}
+
+template <int FMT, int N>
+cudaError_t launch_tc(const SweepParams& p, cudaStream_t s, SweepLaunch* info) {
+    auto kern = sweep_tc_kernel<FMT, N>;
+    const WideGeometry geo = tc_geometry(p.k, FMT, N);
+    if (geo.stages < 2) return cudaErrorInvalidValue;
+    CUtensorMap map_codes, map_x;
+    cudaError_t e = make_code_map(&map_codes, p.w, p.n, p.row_bytes, geo.segs, kTRows);
+    if (e != cudaSuccess) return e;
+    uint8_t* xq = reinterpret_cast<uint8_t*>(p.x16);
+    if (FMT == 0)
+        e = make_x_map(&map_x, p.x, p.M, p.k, geo.segs, N);
+    else
+        e = make_code_map(&map_x, xq, 2 * N, p.k, geo.segs, 2 * N);
+    if (e != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)geo.smem)) != cudaSuccess)
+        return e;
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return e;
+    SweepParams q = p;
+    q.num_tiles = (p.n + kTRows - 1) / kTRows;
+    q.stages = geo.stages;
+    q.stage_bytes = geo.stage_bytes;
+    q.segs = geo.segs;
+    q.stages_per_tile = geo.stages_per_tile;
+    int64_t grid = sms;
+    if (grid > q.num_tiles) grid = q.num_tiles;
+    if (grid > kMaxGrid) grid = kMaxGrid;
+    if (grid < 1) grid = 1;
+    if (FMT == 1) {  // the two E4M3 planes of x the FP8 MMAs read
+        tc_xq_kernel<<<N, 256, 0, s>>>(p.x, p.M, (int)p.k, N, xq, p.xexp);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kTThreads);
+    cfg.dynamicSmemBytes = geo.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if ((e = cudaLaunchKernelEx(&cfg, kern, q, map_codes, map_x)) != cudaSuccess) return e;
+    if (info) {
+        info->grid = (int)grid;
+        info->smem_bytes = (int)geo.smem;
+    }
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 size_t sweep_smem_bytes(int M, int64_t k, int fmt, int* kpad_out, int mode) {
-    if (mode == 0 && M > 8) {  // the wide sweep stages x per K chunk
-        const WideGeometry w = wide_geometry(k, fmt, M > 16 ? 32 : 16);
+    if (mode == 0 && M > 8) {  // the tcgen05 / wide sweeps stage x per K chunk
+        const WideGeometry w = fmt == 2 ? wide_geometry(k, fmt, M > 16 ? 32 : 16)
+                                        : tc_geometry(k, fmt, M > 16 ? 32 : 16);
         if (kpad_out) *kpad_out = (int)k;
         return w.stages >= 2 ? w.smem : (size_t)kSmemLimit + 1;
     }
@@ -1617,7 +2043,10 @@ int sweep_max_grid() { return kMaxGrid; }
 
 size_t sweep_x16_bytes(int M, int64_t k, int fmt) {
     if (M <= 8 || fmt == 0) return 0;
-    return (((size_t)M * (size_t)k * 2 + 1023) & ~(size_t)1023) + 1024;  // x16, then xexp
+    // FP8: x's two E4M3 planes of 16 or 32 rows; NVFP4: the f16 copy of x. Then 1 KB
+    // for the per-input exponents.
+    const size_t body = fmt == 1 ? (size_t)2 * (M > 16 ? 32 : 16) * (size_t)k : (size_t)M * (size_t)k * 2;
+    return ((body + 1023) & ~(size_t)1023) + 1024;
 }
 
 namespace {
@@ -1677,8 +2106,8 @@ cudaError_t sweep_launch(const SweepParams& p, int fmt, int mode, cudaStream_t s
     if (fmt == 2 && mode == 0 && p.M <= 2) return launch_one<2, 1, 0, 1>(p, s, info);
     if (mode == 0 && two) {
         const bool four = p.M > 16;
-        if (fmt == 0) return four ? launch_wide<0, 4>(p, s, info) : launch_wide<0, 2>(p, s, info);
-        if (fmt == 1) return four ? launch_wide<1, 4>(p, s, info) : launch_wide<1, 2>(p, s, info);
+        if (fmt == 0) return four ? launch_tc<0, 32>(p, s, info) : launch_tc<0, 16>(p, s, info);
+        if (fmt == 1) return four ? launch_tc<1, 32>(p, s, info) : launch_tc<1, 16>(p, s, info);
         if (fmt == 2) return four ? launch_wide<2, 4>(p, s, info) : launch_wide<2, 2>(p, s, info);
     }
 #define MTP_SWEEP_CASE(F, NTV, MD) \

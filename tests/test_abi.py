@@ -131,9 +131,13 @@ def test_lm_head_lp_rejects(lib):
     assert lp(OUT, n_eff=101) == L.MTP_ERR_INVALID_ARG
     # partials are 16 bytes (max, index, sum of exponentials) for up to 1,024 CTAs x 32 inputs
     assert wsb == 256 + 16 * 32 * 1024 and L.mtp_noalloc_scratch_bytes() == wsb
-    # more than eight inputs on a quantized table add an f16 copy of x (+ 1 KB of exponents)
+    # more than eight inputs on a quantized table add x as those sweeps read it (+ 1 KB of
+    # exponents): FP8, two E4M3 planes of 16 or 32 rows; NVFP4, an f16 copy of the M rows
     fp8 = weight(fmt=1, k=128, rs=OUT)
-    assert L.mtp_lm_head_ws_bytes(fp8, 100, 9) == wsb + ((9 * 128 * 2 + 1023) // 1024) * 1024 + 1024
+    assert L.mtp_lm_head_ws_bytes(fp8, 100, 9) == wsb + 2 * 16 * 128 + 1024
+    assert L.mtp_lm_head_ws_bytes(fp8, 100, 17) == wsb + 2 * 32 * 128 + 1024
+    nv = weight(fmt=2, k=256, bs=OUT, gs=OUT)
+    assert L.mtp_lm_head_ws_bytes(nv, 100, 9) == wsb + ((9 * 256 * 2 + 1023) // 1024) * 1024 + 1024
     assert L.mtp_lm_head_ws_bytes(weight(k=128), 100, 32) == wsb
     # the no-alloc array has no room for that copy: rejected before any CUDA call
     noalloc = lambda head, M: st("mtp_lm_head_argmax_noalloc", C.byref(head), 100, B2, M, None,
