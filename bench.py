@@ -521,6 +521,9 @@ def main():
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the tiny-draft and prefill rows")
     ap.add_argument("--only", default="", help="profiling: run only 'prefill' or 'tiny'")
+    ap.add_argument("--ms", default="",
+                    help="profiling: time only these input counts (comma list, e.g. 16,32), "
+                         "seeded N(0, 1) inputs")
     ap.add_argument("--sharded", action="store_true",
                     help="N > 1: split the BF16 table by vocab over the ranks (strong scaling) "
                          "instead of one replica per rank")
@@ -556,7 +559,7 @@ def main():
     for fmt in args.formats.split(","):
         cfg, d, table, qinfo = build_table(fmt, dev, args.rows)
         head = api.LmHead(table)
-        Ms = cfg["Ms"] if args.full else (1,)
+        Ms = () if args.ms else (cfg["Ms"] if args.full else (1,))
         for M in Ms:
             x = d["x"][:M].to(dev)
             clocks = ClockSampler(dev)
@@ -590,26 +593,30 @@ def main():
             rows[f"{fmt}_M{M}"] = rec
             if fmt == "bf16" and M == 1:
                 main_line = (rec, nbytes, ms_max, kern_max, e2e_max, h2d, d2h, clk, cfg)
-        if args.full:  # wide batches: 16 and 32 inputs (seeded N(0, 1) rows; timing only)
-            for Mw in (16, 32):
-                gen = torch.Generator().manual_seed(Mw)
-                xw = torch.randn((Mw, cfg["K"]), generator=gen).to(torch.bfloat16).to(dev)
-                iw = torch.empty((Mw,), dtype=torch.int32, device=dev)
-                for _ in range(args.warmup):
+        wide = [int(v) for v in args.ms.split(",")] if args.ms else ((16, 32) if args.full else ())
+        for Mw in wide:  # wide batches: 16 and 32 inputs (seeded N(0, 1) rows; timing only)
+            gen = torch.Generator().manual_seed(Mw)
+            xw = torch.randn((Mw, cfg["K"]), generator=gen).to(torch.bfloat16).to(dev)
+            iw = torch.empty((Mw,), dtype=torch.int32, device=dev)
+            for _ in range(args.warmup):
+                head(xw, iw, None, stream=stream)
+            torch.cuda.synchronize()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                s.record(stream)
+                for _ in range(max(1, args.steps // 4)):
                     head(xw, iw, None, stream=stream)
-                torch.cuda.synchronize()
-                s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                with torch.cuda.stream(stream):
-                    s.record(stream)
-                    for _ in range(max(1, args.steps // 4)):
-                        head(xw, iw, None, stream=stream)
-                    e.record(stream)
-                torch.cuda.synchronize()
-                us = s.elapsed_time(e) / max(1, args.steps // 4) * 1e3
-                rows.setdefault(f"{fmt}_M{Mw}", {"us_per_draft": us,
-                                                 "kernel_GB/s": head.bytes_per_call(Mw) / (us * 1e-6) / 1e9,
-                                                 "frac_of_peak": head.bytes_per_call(Mw) / (us * 1e-6) / 1e9 / peak,
-                                                 "note": "timing only (random inputs)"})
+                e.record(stream)
+            torch.cuda.synchronize()
+            us = s.elapsed_time(e) / max(1, args.steps // 4) * 1e3
+            rows.setdefault(f"{fmt}_M{Mw}", {"us_per_draft": us,
+                                             "kernel_GB/s": head.bytes_per_call(Mw) / (us * 1e-6) / 1e9,
+                                             "frac_of_peak": head.bytes_per_call(Mw) / (us * 1e-6) / 1e9 / peak,
+                                             "note": "timing only (random inputs)"})
+        if args.ms:  # profiling run: only the requested input counts
+            del head, table, d
+            torch.cuda.empty_cache()
+            continue
         # the same sweep with the top-1 log-probability (mtp_lm_head_argmax_lp), M = 1
         x = d["x"][:1].to(dev)
         idx = torch.empty((1,), dtype=torch.int32, device=dev)
@@ -653,7 +660,7 @@ def main():
         del head, table, d
         torch.cuda.empty_cache()
 
-    if world == 1 and not args.no_extra and not args.rows:
+    if world == 1 and not args.no_extra and not args.rows and not args.ms:
         rows["tiny_draft_M1"] = bench_tiny_draft(dev, max(200, args.steps // 10), args.warmup)
         tpk, tsrc = measured_tflops()
         rows["prefill_32k"] = bench_prefill(dev, 5, tpk, tsrc)
@@ -695,6 +702,8 @@ def main():
             "rows": rows,
         }
         print(json.dumps(line), flush=True)
+    elif rank == 0:  # a profiling run without the M = 1 BF16 row
+        print(json.dumps({"rows": rows}), flush=True)
     if world > 1:
         import torch.distributed as dist
 

@@ -1352,7 +1352,8 @@ __global__ void __launch_bounds__(kWThreads, 1)
 // and the N = 16 or 32 (padded) inputs as B, both read by the tensor core straight from
 // the TMA-written stage (K-major, 128-byte swizzle), the fp32 accumulator in tensor
 // memory. Nothing is decoded: FP8 codes are E4M3 operands as stored. x enters FP8 MMAs as
-// two E4M3 terms, hi = e4m3(x 2^e) and lo = e4m3(x 2^e - hi), with e_m chosen per input
+// two E4M3 terms, hi = e4m3(x 2^e) and lo = e4m3(x 2^e - hi) (one B operand of 2N rows;
+// the two dot products are added in fp32 in the epilogue), with e_m chosen per input
 // so that its largest |x| lands in [128, 256); hi + lo equals x 2^e exactly wherever
 // x 2^e >= 1/4 (a bf16 value has 8 significant bits, hi keeps 4 and the rest fits lo's 4),
 // and within 2^-10 below that, i.e. within 2^-17 of the input's largest |x|.
@@ -1418,8 +1419,12 @@ __global__ void __launch_bounds__(kTThreads, 1)
                     const __grid_constant__ CUtensorMap map_x) {
     static_assert(FMT == 0 || FMT == 1, "BF16 and FP8 tables");
     static_assert(N == 16 || N == 32, "16 or 32 input columns");
-    constexpr int XR = FMT == 1 ? 2 * N : N;  // x rows per stage segment (hi and lo for FP8)
-    constexpr uint32_t kTmemCols = 2 * N < 32 ? 32 : 2 * N;
+    // x rows per stage segment, and accumulator columns per tile: for FP8 the hi and lo
+    // rows of x are one B operand of 2N rows, so D holds x_hi and x_lo dot products side
+    // by side (columns m and N + m), added in the epilogue
+    constexpr int XR = FMT == 1 ? 2 * N : N;
+    constexpr int DC = XR;
+    constexpr uint32_t kTmemCols = 2 * DC < 32 ? 32 : 2 * DC;
 
     extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
@@ -1514,7 +1519,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
         __syncwarp();
     } else if (warp == 1) {
         // ---------------- MMA issuer (lane 0)
-        constexpr uint32_t idesc = FMT == 0 ? idesc_bf16(kTRows, N) : idesc_e4m3(kTRows, N);
+        constexpr uint32_t idesc = FMT == 0 ? idesc_bf16(kTRows, DC) : idesc_e4m3(kTRows, DC);
         int slot = 0;
         uint32_t phase = 0;
         int local = 0;
@@ -1531,7 +1536,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
             }
             __syncwarp();
             if (tile < 0) break;
-            const uint32_t d_tmem = tmem_base + (uint32_t)(buf * N);
+            const uint32_t d_tmem = tmem_base + (uint32_t)(buf * DC);
             bool ok = true;
             for (int ch = 0; ch < NC; ++ch) {
                 if (ch > 0 && !mbar_wait_bounded(&full[slot], phase, abort_flag)) {
@@ -1548,13 +1553,10 @@ __global__ void __launch_bounds__(kTThreads, 1)
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             const uint32_t acc = (ch > 0 || sg > 0 || k > 0) ? 1u : 0u;
-                            if (FMT == 0) {
+                            if (FMT == 0)
                                 umma_bf16(d_tmem, sdesc_k128(as + k * 32), sdesc_k128(xs + k * 32), idesc, acc);
-                            } else {
+                            else
                                 umma_e4m3(d_tmem, sdesc_k128(as + k * 32), sdesc_k128(xs + k * 32), idesc, acc);
-                                umma_e4m3(d_tmem, sdesc_k128(as + k * 32), sdesc_k128(xs + N * 128 + k * 32),
-                                          idesc, 1u);
-                            }
                         }
                     }
                     umma_commit(&empty[slot]);  // frees the stage once these MMAs have read it
@@ -1602,11 +1604,21 @@ __global__ void __launch_bounds__(kTThreads, 1)
             if (tile < 0) break;
             tc_fence_after();
             uint32_t v[N];
-            const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * N);
+            const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * DC);
             if constexpr (N == 32)
                 tmem_ld32(ta, v);
             else
                 tmem_ld16(ta, v);
+            if constexpr (FMT == 1) {  // + the x_lo dot products
+                uint32_t w[N];
+                if constexpr (N == 32)
+                    tmem_ld32(ta + N, w);
+                else
+                    tmem_ld16(ta + N, w);
+                tmem_ld_wait();
+#pragma unroll
+                for (int m = 0; m < N; ++m) v[m] = __float_as_uint(__uint_as_float(v[m]) + __uint_as_float(w[m]));
+            }
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
