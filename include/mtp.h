@@ -174,14 +174,20 @@ mtp_status mtp_combine(const uint16_t* embed, int64_t vocab, const int32_t* toke
  *   dev_err       (device) i32 [1] or NULL
  *   ws            (device) >= mtp_lm_head_ws_bytes(head, n_eff, M) bytes, 16-byte
  *                 aligned, ALL ZERO before the first call; each call leaves its
- *                 counter zero again. (For M > 8 on FP8/NVFP4 tables it also holds an
- *                 f16 copy of x, M * k * 2 bytes, rewritten by each call.)
+ *                 counter zero again. It also holds x as the many-input sweeps read
+ *                 it, rewritten by each call: for FP8 tables with M >= 7 two E4M3
+ *                 planes of 16 or 32 rows (2 * 16 * k or 2 * 32 * k bytes), for NVFP4
+ *                 with M > 8 an f16 copy (M * k * 2 bytes).
  * Requires 1 <= M <= 32, 1 <= n_eff <= n; table rows a multiple of 128 bytes (k % 64
  * for BF16, % 128 for FP8, % 256 for NVFP4; the sweep streams 128-byte segments); for
- * M <= 8 the staged inputs (M * k * 2 bytes) must leave shared memory for the stream
- * (MTP_ERR_UNSUPPORTED otherwise; M > 8 streams x per K chunk instead). Results are
- * bit-identical for every M within 1-8, 9-16 and 17-32 (NVFP4: 1-2, 3-8, 9-16, 17-32),
- * whose sweeps sum the same products in different fixed orders.
+ * M <= 8 (FP8: M <= 6) the staged inputs (M * k * 2 bytes) must leave shared memory for
+ * the stream (MTP_ERR_UNSUPPORTED otherwise; more inputs stream x per K chunk instead).
+ * Results are bit-identical for every M within BF16 1-8, 9-16, 17-32; FP8 1-6, 7-16,
+ * 17-32; NVFP4 1-2, 3-8, 9-16, 17-32, whose sweeps sum the same products in different
+ * fixed orders. BF16 and FP8 tables with more inputs run on the tcgen05 tensor cores;
+ * there x enters FP8 products as two E4M3 terms whose sum is x exactly except for
+ * elements below 2^-9 of the input's largest |x|, which keep an absolute error of at
+ * most 2^-17 of that largest |x|.
  * ------------------------------------------------------------------------------ */
 size_t mtp_lm_head_ws_bytes(const mtp_weight* head, int64_t n_eff, int32_t M);
 mtp_status mtp_lm_head_argmax(const mtp_weight* head, int64_t n_eff, const uint16_t* x,

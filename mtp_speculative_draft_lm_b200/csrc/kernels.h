@@ -41,7 +41,8 @@ struct SweepParams {
     float* out_logprob;          // f32 [M] top-1 log-probability, or null
     void* out_partial;           // vocab shard: 16-byte (max, row, sum exp) per input, or null
     int64_t row_offset;          // vocab shard: global index of the table's first row
-    uint16_t* x16;               // M > 8, quantized tables: f16 copy of x scaled per row [M, k]
+    uint16_t* x16;               // many inputs, quantized tables: x as those sweeps read it
+                                 // (FP8: E4M3 hi / lo planes; NVFP4: f16 [M, k]), scaled per row
     int32_t* xexp;               // its per-row power of two [M]
     uint16_t* out_y;             // mode 1: bf16 [M, n]
     int32_t* dev_err;
@@ -72,7 +73,9 @@ cudaError_t merge_partials_launch(const void* parts, int n_parts, int M, int32_t
 cudaError_t sweep_launch(const SweepParams& p, int fmt, int mode, cudaStream_t s,
                          SweepLaunch* info);
 size_t sweep_smem_bytes(int M, int64_t k, int fmt, int* kpad_out, int mode);
-// Workspace bytes the wide sweep (mode 0, M > 8) needs for its f16 copy of x: 0 for BF16.
+// Workspace bytes the many-input argmax sweeps need for x in their own form (FP8 tables
+// from 7 inputs: two E4M3 planes; NVFP4 from 9: an f16 copy) plus 1 KB of per-input
+// exponents: 0 for BF16 and for fewer inputs.
 size_t sweep_x16_bytes(int M, int64_t k, int fmt);
 int sweep_max_grid();
 

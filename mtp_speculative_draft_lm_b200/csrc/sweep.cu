@@ -18,8 +18,9 @@
 // mbarrier; each stage carries its tile index, and a stage tagged -1 ends the CTA's
 // work. Large copies matter: the TMA unit's per-copy cost caps a ring fed by 1 KB row
 // copies at about half of HBM bandwidth. Out-of-range rows and K tails arrive as
-// zeros (tensor-map bounds). Sixteen compute warps (eight when M > 8) split each
-// stage's K range into slabs of 4 lanes x 16 B per row, decode the codes exactly into
+// zeros (tensor-map bounds). Sixteen compute warps (eight for the combiner past eight
+// inputs) split each stage's K range into slabs of 4 lanes x 16 B per row, decode the
+// codes exactly into
 // f16/bf16 fragments and run tensor-core MMAs with 16 table rows as the A operand and
 // up to 16 inputs as the B operand (swap-AB). MMA row g reads table row s(g) of the
 // tile, a fixed permutation that, with the swizzle, makes every shared-memory read
@@ -40,6 +41,8 @@
 // this kernel waits for the previous grid before reading x, masks or the workspace.
 // Every mbarrier wait is bounded: a wait that runs out sets an abort flag and
 // MTP_DEVFLAG_TIMEOUT, and the kernel runs to its end.
+// More inputs than this design serves well (BF16 from 9, FP8 from 7) go to the tcgen05
+// sweep further down; NVFP4 from 9 inputs to the 64-row-tile wide sweep.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -2037,10 +2040,15 @@ cudaError_t launch_tc(const SweepParams& p, cudaStream_t s, SweepLaunch* info) {
     return cudaGetLastError();
 }
 
+// Argmax sweeps that stream x per K chunk -- the tcgen05 sweep (BF16, FP8), the wide
+// sweep (NVFP4) -- take FP8 tables from 7 inputs on (measured faster than 16-row tiles
+// from there), the others from 9.
+inline bool streams_x(int M, int fmt) { return fmt == 1 ? M >= 7 : M > 8; }
+
 }  // namespace
 
 size_t sweep_smem_bytes(int M, int64_t k, int fmt, int* kpad_out, int mode) {
-    if (mode == 0 && M > 8) {  // the tcgen05 / wide sweeps stage x per K chunk
+    if (mode == 0 && streams_x(M, fmt)) {  // the tcgen05 / wide sweeps stage x per K chunk
         const WideGeometry w = fmt == 2 ? wide_geometry(k, fmt, M > 16 ? 32 : 16)
                                         : tc_geometry(k, fmt, M > 16 ? 32 : 16);
         if (kpad_out) *kpad_out = (int)k;
@@ -2054,7 +2062,7 @@ size_t sweep_smem_bytes(int M, int64_t k, int fmt, int* kpad_out, int mode) {
 int sweep_max_grid() { return kMaxGrid; }
 
 size_t sweep_x16_bytes(int M, int64_t k, int fmt) {
-    if (M <= 8 || fmt == 0) return 0;
+    if (fmt == 0 || !streams_x(M, fmt)) return 0;
     // FP8: x's two E4M3 planes of 16 or 32 rows; NVFP4: the f16 copy of x. Then 1 KB
     // for the per-input exponents.
     const size_t body = fmt == 1 ? (size_t)2 * (M > 16 ? 32 : 16) * (size_t)k : (size_t)M * (size_t)k * 2;
@@ -2116,7 +2124,7 @@ cudaError_t sweep_launch(const SweepParams& p, int fmt, int mode, cudaStream_t s
                          SweepLaunch* info) {
     const bool two = p.M > 8;
     if (fmt == 2 && mode == 0 && p.M <= 2) return launch_one<2, 1, 0, 1>(p, s, info);
-    if (mode == 0 && two) {
+    if (mode == 0 && streams_x(p.M, fmt)) {
         const bool four = p.M > 16;
         if (fmt == 0) return four ? launch_tc<0, 32>(p, s, info) : launch_tc<0, 16>(p, s, info);
         if (fmt == 1) return four ? launch_tc<1, 32>(p, s, info) : launch_tc<1, 16>(p, s, info);
@@ -2124,7 +2132,7 @@ cudaError_t sweep_launch(const SweepParams& p, int fmt, int mode, cudaStream_t s
     }
 #define MTP_SWEEP_CASE(F, NTV, MD) \
     if (fmt == F && (NTV == 2) == two && mode == MD) return launch_one<F, NTV, MD, 0>(p, s, info);
-    // (mode 0 with more than eight inputs went to the wide sweep above)
+    // (mode 0 inputs past streams_x went to the tcgen05 / wide sweeps above)
     MTP_SWEEP_CASE(0, 1, 0) MTP_SWEEP_CASE(1, 1, 0) MTP_SWEEP_CASE(2, 1, 0)
     MTP_SWEEP_CASE(0, 1, 1) MTP_SWEEP_CASE(0, 2, 1)
     MTP_SWEEP_CASE(1, 1, 1) MTP_SWEEP_CASE(1, 2, 1)

@@ -134,6 +134,8 @@ def test_lm_head_lp_rejects(lib):
     # more than eight inputs on a quantized table add x as those sweeps read it (+ 1 KB of
     # exponents): FP8, two E4M3 planes of 16 or 32 rows; NVFP4, an f16 copy of the M rows
     fp8 = weight(fmt=1, k=128, rs=OUT)
+    assert L.mtp_lm_head_ws_bytes(fp8, 100, 6) == wsb  # FP8 streams x from 7 inputs on
+    assert L.mtp_lm_head_ws_bytes(fp8, 100, 7) == wsb + 2 * 16 * 128 + 1024
     assert L.mtp_lm_head_ws_bytes(fp8, 100, 9) == wsb + 2 * 16 * 128 + 1024
     assert L.mtp_lm_head_ws_bytes(fp8, 100, 17) == wsb + 2 * 32 * 128 + 1024
     nv = weight(fmt=2, k=256, bs=OUT, gs=OUT)
@@ -142,7 +144,7 @@ def test_lm_head_lp_rejects(lib):
     # the no-alloc array has no room for that copy: rejected before any CUDA call
     noalloc = lambda head, M: st("mtp_lm_head_argmax_noalloc", C.byref(head), 100, B2, M, None,
                                  0, 0, OUT, None, None, None, None)
-    assert noalloc(fp8, 9) == L.MTP_ERR_WORKSPACE
+    assert noalloc(fp8, 7) == L.MTP_ERR_WORKSPACE
     assert noalloc(weight(fmt=2, k=128, bs=OUT, gs=OUT), 12) == L.MTP_ERR_WORKSPACE
 
 

@@ -4,7 +4,8 @@ Small tables span several 16-row tiles, several CTAs and a ragged tail; the full
 tables are the benchmark's (154,880 x 4,096 BF16 and FP8, 131,072 x 5,120 NVFP4) in
 the launch configuration bench.py times. Logits within 2e-2 + 1e-2|ref|; argmax exact
 where the top-2 gap exceeds 1e-2; one-hot inputs and batch invariance bit-exact within
-each range of M that one sweep serves (1-8, 9-16, 17-32; NVFP4 1-2, 3-8, 9-16, 17-32)."""
+each range of M that one sweep serves (BF16 1-8, 9-16, 17-32; FP8 1-6, 7-16, 17-32; NVFP4
+1-2, 3-8, 9-16, 17-32)."""
 import numpy as np
 import pytest
 import torch
@@ -88,7 +89,7 @@ SHAPES = {0: [(1000, 256), (1000, 4096), (4133, 576)],
 
 
 @pytest.mark.parametrize("fmt", [0, 1, 2])
-@pytest.mark.parametrize("M", [1, 3, 8, 9, 16, 17, 32])
+@pytest.mark.parametrize("M", [1, 3, 6, 7, 8, 9, 16, 17, 32])
 def test_sweep_small_tables(orc, fmt, M):
     for n, k in SHAPES[fmt]:
         w = synth.as_u16(synth.normal_bf16(synth._gen(n + k + fmt), (n, k), 0.02))
@@ -123,12 +124,14 @@ def test_batch_invariance(orc, fmt):
     x = synth.as_u16(synth.normal_bf16(synth._gen(10), (32, k), 1.0))
     table = device_table(oracle_quant(orc, w, fmt), fmt, n, k)
     head = api.LmHead(table)
-    # Three sweeps share the work: NVFP4 with one or two inputs applies the block scales
-    # to per-block fp32 sums, more than eight inputs use 64-row tiles with x streamed per
-    # K chunk; each sums the same exact products in its own fixed order, so results are
-    # bit-identical within each range of M and within the tolerance across them
-    groups = ([(1, 2), (3, 4, 8), (9, 12, 16), (17, 24, 32)] if fmt == 2
-              else [(1, 2, 3, 4, 8), (9, 12, 16), (17, 24, 32)])
+    # Several sweeps share the work: NVFP4 with one or two inputs applies the block scales
+    # to per-block fp32 sums; more inputs (BF16 from 9, FP8 from 7) go to the tcgen05 sweep
+    # with 16 or 32 MMA columns, NVFP4 from 9 to 64-row tiles with x streamed per K chunk.
+    # Each sums its products in its own fixed order, so results are bit-identical within
+    # each range of M and within the tolerance across them
+    groups = {0: [(1, 2, 3, 4, 8), (9, 12, 16), (17, 24, 32)],
+              1: [(1, 2, 3, 4, 6), (7, 8, 12, 16), (17, 24, 32)],
+              2: [(1, 2), (3, 4, 8), (9, 12, 16), (17, 24, 32)]}[fmt]
     bases = []
     for grp in groups:
         base = run_sweep(table, x[:grp[0]], head=head)
@@ -181,10 +184,11 @@ def test_masks_decoys_and_edge_cases(orc):
     assert np.array_equal(got[0][[0, 1, 3]], d["second"][[0, 1, 3]])
 
 
-@pytest.mark.parametrize("M", [12, 32])
+@pytest.mark.parametrize("M", [7, 12, 32])
 def test_masks_and_n_eff_many_inputs(orc, M):
-    """The 64-row-tile sweep (more than eight inputs): per-row masks with a decoy, a shared
-    mask, an all-zero mask row, masked logits -inf, and an n_eff that ends mid-tile."""
+    """The sweeps that stream x per K chunk (tcgen05 for BF16 / FP8, 64-row tiles for
+    NVFP4): per-row masks with a decoy, a shared mask, an all-zero mask row, masked logits
+    -inf, and an n_eff that ends mid-tile."""
     n, k = 4133, 512
     d = synth.head_table(13 + M, n, k, M, mask_keep=0.1)
     w, x = synth.as_u16(d["W"]), synth.as_u16(d["x"])
