@@ -319,8 +319,9 @@ mtp_status mtp_debug_kv_write(const uint16_t* k_rot, const uint16_t* v, int64_t 
  * is a static device array inside the library, mtp_noalloc_scratch_bytes() bytes
  * (524,544: a 256-byte header + 16-byte partials of up to 1,024 CTAs x 32 input rows)
  * held on every GPU that loads the library until the process exits. It has no room
- * for the f16 copy of x that FP8 and NVFP4 tables need above M = 8, so those calls
- * return MTP_ERR_WORKSPACE here; BF16 tables run at every M up to 32.
+ * for x in the form the many-input sweeps read it (FP8 tables from M = 7, NVFP4 from
+ * M = 9), so those calls return MTP_ERR_WORKSPACE here; BF16 tables run at every M up
+ * to 32.
  *  - The first call made with a device current looks up that array's device address
  *    and zeroes its counter (synchronously); make it before any stream capture.
  *  - All calls on a device share the array: calls that overlap on the GPU race and
