@@ -197,6 +197,31 @@ mtp_status mtp_lm_head_argmax(const mtp_weight* head, int64_t n_eff, const uint1
                               size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------
+ * mtp_lm_head_argmax_host -- mtp_lm_head_argmax with the input and the result in pinned
+ * host memory: the whole draft step (host -> device input, sweep, device -> host result)
+ * in one call on `stream`, with no separate copy operations in the stream.
+ * The pages' draft step reads the argmax back to the host every draft ([init.rs] /
+ * [v4_mtp.rs] argmax then a 4-byte device-to-host read); this entry point is that step.
+ *   x_host    pinned host bf16 [M, k] (cudaHostAlloc / cudaHostRegister; torch
+ *             pin_memory), 16-byte aligned; read by the device during the call
+ *   out_host  pinned host i32 [2M]: out_host[m] = index, then M f32 values (the winning
+ *             logits) at out_host + M; written by the device; valid after the stream
+ *             has synchronised
+ *   ws        (device) >= mtp_lm_head_host_ws_bytes(head, n_eff, M) bytes: the sweep's
+ *             workspace followed by the device copy of x
+ * A small kernel copies x into the workspace (it reads before and writes after waiting
+ * for the previous kernel in the stream, so the host-link latency overlaps that kernel's
+ * tail); the sweep then writes its results straight into out_host. Returns
+ * MTP_ERR_INVALID_ARG if x_host or out_host is not pinned host memory; otherwise the
+ * requirements and results of mtp_lm_head_argmax (no logits output).
+ * ------------------------------------------------------------------------------ */
+size_t mtp_lm_head_host_ws_bytes(const mtp_weight* head, int64_t n_eff, int32_t M);
+mtp_status mtp_lm_head_argmax_host(const mtp_weight* head, int64_t n_eff, const uint16_t* x_host,
+                                   int32_t M, const int32_t* mask, int64_t mask_words,
+                                   int64_t mask_stride_words, int32_t* out_host, int32_t* dev_err,
+                                   void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------
  * mtp_lm_head_argmax_lp -- mtp_lm_head_argmax that also writes each input's top-1
  * log-probability from the same sweep (no extra table bytes).
  * Source: [mtp_head.rs] MtpHead fields: argmax_bf16_batch_lp, the batched argmax that

@@ -35,6 +35,7 @@ EXPORTS = (
     "mtp_abi_version", "mtp_status_str", "mtp_devflags_status",
     "mtp_quantize_fp8", "mtp_quantize_nvfp4_ws_bytes", "mtp_quantize_nvfp4",
     "mtp_combine", "mtp_lm_head_ws_bytes", "mtp_lm_head_argmax", "mtp_lm_head_argmax_lp",
+    "mtp_lm_head_host_ws_bytes", "mtp_lm_head_argmax_host",
     "mtp_lm_head_shard_partial", "mtp_argmax_merge_partials",
     "mtp_debug_encode_e4m3", "mtp_debug_encode_e2m1", "mtp_nvfp4_scale_pitch",
     "mtp_noalloc_scratch_bytes", "mtp_lm_head_argmax_noalloc",
@@ -75,6 +76,9 @@ _SIGS = {
                                      _P, _SZ, _P]),
     "mtp_lm_head_argmax_lp": (C.c_int, [_W, _I64, _P, _I32, _P, _I64, _I64, _P, _P, _P, _P,
                                         _P, _P, _SZ, _P]),
+    "mtp_lm_head_host_ws_bytes": (_SZ, [_W, _I64, _I32]),
+    "mtp_lm_head_argmax_host": (C.c_int, [_W, _I64, _P, _I32, _P, _I64, _I64, _P, _P, _P, _SZ,
+                                          _P]),
     "mtp_lm_head_shard_partial": (C.c_int, [_W, _I64, _I64, _P, _I32, _P, _I64, _I64, _P, _P,
                                             _P, _P, _SZ, _P]),
     "mtp_argmax_merge_partials": (C.c_int, [_P, _I32, _I32, _P, _P, _P, _P, _P]),
@@ -199,6 +203,19 @@ def mtp_lm_head_argmax_lp(head, n_eff, x, M, mask, mask_words, mask_stride_words
                                         _ptr(out_logits), _ptr(dev_err), _ptr(ws), ws_bytes,
                                         _stream(stream)),
            "mtp_lm_head_argmax_lp")
+
+
+def mtp_lm_head_host_ws_bytes(head, n_eff, M) -> int:
+    return load().mtp_lm_head_host_ws_bytes(C.byref(head), n_eff, M)
+
+
+def mtp_lm_head_argmax_host(head, n_eff, x_host, M, mask, mask_words, mask_stride_words,
+                            out_host, dev_err, ws, ws_bytes, stream=None):
+    _check(load().mtp_lm_head_argmax_host(C.byref(head) if head is not None else None, n_eff,
+                                          _ptr(x_host), M, _ptr(mask), mask_words,
+                                          mask_stride_words, _ptr(out_host), _ptr(dev_err),
+                                          _ptr(ws), ws_bytes, _stream(stream)),
+           "mtp_lm_head_argmax_host")
 
 
 def mtp_lm_head_shard_partial(shard, n_eff, row_offset, x, M, mask, mask_words,

@@ -71,7 +71,8 @@ class LmHead:
         self.table = table
         self.n_eff = table.n if n_eff is None else int(n_eff)
         dev = table.data.device
-        nbytes = L.mtp_lm_head_ws_bytes(table.desc, self.n_eff, max_m)
+        # room for the host-input entry point's copy of x as well
+        nbytes = L.mtp_lm_head_host_ws_bytes(table.desc, self.n_eff, max_m)
         self.ws = torch.zeros((nbytes,), dtype=torch.uint8, device=dev)
         self.dev_err = torch.zeros((1,), dtype=torch.int32, device=dev)
 
@@ -93,6 +94,16 @@ class LmHead:
             L.mtp_lm_head_argmax_lp(self.table.desc, self.n_eff, x, M, mask, mask_words,
                                     mask_stride_words, out_idx, out_val, out_logprob,
                                     out_logits, self.dev_err, self.ws, self.ws.numel(), stream)
+
+    def argmax_host(self, x_host: torch.Tensor, out_host: torch.Tensor, mask=None, mask_words=0,
+                    mask_stride_words=0, stream=None):
+        """One draft step from pinned host memory to pinned host memory: x_host bf16
+        [M, k] pinned; out_host int32 [2M] pinned receives the indices, then the values
+        (float32 bits). Valid once the stream has synchronised."""
+        M = x_host.shape[0]
+        L.mtp_lm_head_argmax_host(self.table.desc, self.n_eff, x_host, M, mask, mask_words,
+                                  mask_stride_words, out_host, self.dev_err, self.ws,
+                                  self.ws.numel(), stream)
 
     def argmax(self, x: torch.Tensor, mask=None, mask_words=0, mask_stride_words=0,
                logits=False, stream=None, logprob=False):

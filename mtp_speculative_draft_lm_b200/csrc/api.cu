@@ -227,6 +227,53 @@ mtp_status mtp_lm_head_argmax(const mtp_weight* head, int64_t n_eff, const uint1
                         nullptr, out_logits, dev_err, ws, ws_bytes, stream);
 }
 
+size_t mtp_lm_head_host_ws_bytes(const mtp_weight* head, int64_t n_eff, int32_t M) {
+    const size_t base = mtp_lm_head_ws_bytes(head, n_eff, M);
+    if (!head || M < 1 || M > kMaxM || head->k < 1) return base;
+    return base + (((size_t)M * (size_t)head->k * 2 + 15) & ~(size_t)15);
+}
+
+namespace {
+
+// The device address of pinned (page-locked) host memory, or null if `p` is not pinned.
+void* pinned_device_ptr(const void* p) {
+    cudaPointerAttributes a{};
+    if (!p || cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();  // clear the error a non-registered pointer leaves behind
+        return nullptr;
+    }
+    if (a.type != cudaMemoryTypeHost || !a.devicePointer) return nullptr;
+    return a.devicePointer;
+}
+
+}  // namespace
+
+mtp_status mtp_lm_head_argmax_host(const mtp_weight* head, int64_t n_eff, const uint16_t* x_host,
+                                   int32_t M, const int32_t* mask, int64_t mask_words,
+                                   int64_t mask_stride_words, int32_t* out_host, int32_t* dev_err,
+                                   void* ws, size_t ws_bytes, void* stream) {
+    mtp_status st = check_weight(head);
+    if (st != MTP_OK) return st;
+    if (!x_host || !out_host) return MTP_ERR_INVALID_ARG;
+    if (M < 1 || M > kMaxM) return MTP_ERR_UNSUPPORTED;
+    if (!aligned(x_host, 16) || !aligned(out_host, 4) || (head->k * 2) % 16)
+        return MTP_ERR_INVALID_ARG;
+    const size_t base = mtp_lm_head_ws_bytes(head, n_eff, M);
+    if (!ws || !aligned(ws, 16) || ws_bytes < mtp_lm_head_host_ws_bytes(head, n_eff, M))
+        return MTP_ERR_WORKSPACE;
+    void* xd = pinned_device_ptr(x_host);
+    void* od = pinned_device_ptr(out_host);
+    if (!xd || !od) return MTP_ERR_INVALID_ARG;  // both must be pinned host memory
+    uint16_t* x_dev = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + base);
+    const size_t xbytes = (size_t)M * (size_t)head->k * 2;
+    cudaError_t e = mtp::fetch_x_launch(xd, x_dev, xbytes, as_stream(stream));
+    if (e != cudaSuccess) return from_cuda(e);
+    int32_t* idx = static_cast<int32_t*>(od);
+    float* val = reinterpret_cast<float*>(idx + M);
+    return lm_head_impl(head, n_eff, x_dev, M, mask, mask_words, mask_stride_words, idx, val,
+                        nullptr, nullptr, dev_err, ws, base, stream);
+}
+
 mtp_status mtp_lm_head_shard_partial(const mtp_weight* shard, int64_t n_eff, int64_t row_offset,
                                      const uint16_t* x, int32_t M, const int32_t* mask,
                                      int64_t mask_words, int64_t mask_stride_words,

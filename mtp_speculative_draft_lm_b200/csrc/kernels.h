@@ -79,6 +79,11 @@ size_t sweep_smem_bytes(int M, int64_t k, int fmt, int* kpad_out, int mode);
 size_t sweep_x16_bytes(int M, int64_t k, int fmt);
 int sweep_max_grid();
 
+// Copies `bytes` (a multiple of 16) from device-reachable host memory into device memory
+// with a programmatic-dependent-launch kernel (loads before, stores after waiting for the
+// previous grid).
+cudaError_t fetch_x_launch(const void* src, void* dst, size_t bytes, cudaStream_t s);
+
 // Quantizers.
 cudaError_t quant_fp8_launch(const uint16_t* w, int64_t n, int64_t k, uint8_t* codes,
                              float* row_scale, cudaStream_t s);

@@ -148,6 +148,26 @@ def test_lm_head_lp_rejects(lib):
     assert noalloc(weight(fmt=2, k=128, bs=OUT, gs=OUT), 12) == L.MTP_ERR_WORKSPACE
 
 
+def test_lm_head_host_rejects(lib):
+    head = weight()
+    wsb = L.mtp_lm_head_host_ws_bytes(head, 100, 2)
+    # the sweep's workspace, then the device copy of x (M k 2 bytes, 16-byte multiple)
+    assert wsb == L.mtp_lm_head_ws_bytes(head, 100, 2) + 2 * 64 * 2
+
+    def host(x=B2, out=OUT, M=2, ws=0x40000, nb=wsb):
+        return st("mtp_lm_head_argmax_host", C.byref(head), 100, x, M, None, 0, 0, out, None,
+                  ws, nb, None)
+
+    assert host(x=None) == L.MTP_ERR_INVALID_ARG
+    assert host(out=None) == L.MTP_ERR_INVALID_ARG
+    assert host(M=33) == L.MTP_ERR_UNSUPPORTED
+    assert host(x=B2 + 4) == L.MTP_ERR_INVALID_ARG
+    assert host(ws=None) == L.MTP_ERR_WORKSPACE
+    assert host(nb=wsb - 16) == L.MTP_ERR_WORKSPACE
+    # addresses that are not pinned host memory (here: no device at all) are refused
+    assert host() == L.MTP_ERR_INVALID_ARG
+
+
 def test_shard_and_merge_rejects(lib):
     head = weight()
     wsb = L.mtp_lm_head_ws_bytes(head, 100, 1)

@@ -327,3 +327,33 @@ def test_top1_logprob_full_tables(orc, cfg, fmt):
     ref_l, ref_i, _, _ = oracle_sweep(orc, q, fmt, cfg["K"], x)
     assert idx.item() == ref_i[0]
     assert_close(lp.cpu().numpy(), oracle_logprobs(orc, ref_l), "full-table log-probability")
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("M", [1, 3, 12])
+def test_host_input_and_result(orc, fmt, M):
+    """mtp_lm_head_argmax_host: x read from pinned host memory and (index, value) written
+    to pinned host memory by the call itself; several calls in a row on one stream, each
+    with new input bytes, match the device-buffer entry point."""
+    n, k = 1500, 512
+    d = synth.head_table(21 + M, n, k, M)
+    q = oracle_quant(orc, synth.as_u16(d["W"]), fmt)
+    table = device_table(q, fmt, n, k)
+    head = api.LmHead(table)
+    out = torch.empty((3, 2 * M), dtype=torch.int32).pin_memory()
+    xs = []
+    for j in range(3):
+        x = d["x"] if j == 0 else synth.normal_bf16(synth._gen(50 + j), (M, k), 1.0)
+        xh = x.contiguous().pin_memory()
+        xs.append(xh)
+        head.argmax_host(xh, out[j])  # three steps queued back to back
+    torch.cuda.synchronize()
+    assert np.array_equal(out[0, :M].numpy(), d["top"])
+    for j in range(3):
+        idx, val, _ = head.argmax(xs[j].cuda())
+        torch.cuda.synchronize()
+        assert np.array_equal(out[j, :M].numpy(), idx.cpu().numpy())
+        assert np.array_equal(out[j, M:].numpy(), val.cpu().view(torch.int32).numpy())
+    # pageable host memory is refused
+    with pytest.raises(L.MtpError):
+        head.argmax_host(d["x"].contiguous(), out[0])
