@@ -531,3 +531,33 @@ def test_top1_logprob_pins(orc):
     w = synth.as_u16(synth.normal_bf16(synth._gen(31), (300, k), 0.02))
     lg, idx, _, _ = orc.lm_head_argmax(0, w, k, np.zeros((1, k), np.uint16))
     assert idx[0] == 0 and orc.top1_logprob(lg[0]) == pytest.approx(-np.log(300), abs=1e-12)
+
+
+def test_fp8_x_two_term_split(orc):
+    """The reading behind the tensor-core FP8 sweep: an input row scaled by 2^e (its
+    largest |x| in [128, 256)) and split into hi = e4m3(x 2^e), lo = e4m3(x 2^e - hi)
+    sums back to x 2^e exactly for every element with |x| >= 2^-9 max|x| (8 significant
+    bits = 4 + 4), and within 2^-10 (scaled units, i.e. 2^-17 max|x|) below that."""
+    rng = np.random.default_rng(11)
+    for scale in (1.0, 3e-3, 7e5, 1e-20):
+        v = np.concatenate([rng.standard_normal(3000), rng.standard_normal(500) * 1e-3,
+                            rng.standard_normal(500) * 1e-6, [0.0, 1.0, -1.0, 2.0 ** -9]])
+        xb = orc.f64_to_bf16(v * scale)
+        x = orc.bf16_to_f64(xb)
+        a = np.abs(x).max()
+        e = 8 - math.frexp(a)[1]
+        xs = x * 2.0 ** e
+        assert 128 <= np.abs(xs).max() < 256
+        hi = orc.e4m3_value(orc.e4m3_encode(xs))
+        lo = orc.e4m3_value(orc.e4m3_encode(xs - hi))
+        err = np.abs(hi + lo - xs)
+        big = np.abs(x) >= 2.0 ** -9 * a
+        assert big.sum() > 2900 and np.all(err[big] == 0.0)
+        assert np.all(err <= 2.0 ** -10)
+        assert np.all(err * 2.0 ** -e <= 2.0 ** -17 * a)
+    # the bound is reached: an element whose scaled value sits halfway between two
+    # subnormal E4M3 steps keeps half a step
+    xs = np.array([200.0, 2.0 ** -10 * 3])
+    hi = orc.e4m3_value(orc.e4m3_encode(xs))
+    lo = orc.e4m3_value(orc.e4m3_encode(xs - hi))
+    assert abs(hi[1] + lo[1] - xs[1]) == 2.0 ** -10
