@@ -162,6 +162,9 @@ def test_lm_head_host_rejects(lib):
     assert host(out=None) == L.MTP_ERR_INVALID_ARG
     assert host(M=33) == L.MTP_ERR_UNSUPPORTED
     assert host(x=B2 + 4) == L.MTP_ERR_INVALID_ARG
+    assert host(out=OUT + 2) == L.MTP_ERR_INVALID_ARG
+    assert st("mtp_lm_head_argmax_host", None, 100, B2, 2, None, 0, 0, OUT, None, 0x40000, wsb,
+              None) == L.MTP_ERR_INVALID_ARG  # no table
     assert host(ws=None) == L.MTP_ERR_WORKSPACE
     assert host(nb=wsb - 16) == L.MTP_ERR_WORKSPACE
     # addresses that are not pinned host memory (here: no device at all) are refused
