@@ -32,7 +32,7 @@ FALLBACK_HBM_GBS = 6650.0
 
 # DRAM traffic per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum) and
 # the sha256 of sweep.cu when it was captured; reported as null once the source changed.
-# bf16_M1: the 40,000-row capture (profiles/sweep_kernel_bf16_40k_rows.md) read
+# bf16_M1: the 40,000-row capture of the BF16 sweep read
 # 327,776,256 B and wrote 3,843,584 B; reads scale with the rows swept, so a full
 # 154,880-row launch reads 327,776,256 x 154,880 / 40,000 B (writes kept unscaled).
 NCU_TRAFFIC = {"bf16_M1": (1272993247, "ebea71e05b1b11fa")}

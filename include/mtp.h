@@ -211,7 +211,9 @@ mtp_status mtp_lm_head_argmax(const mtp_weight* head, int64_t n_eff, const uint1
  *             workspace followed by the device copy of x
  * A small kernel copies x into the workspace (it reads before and writes after waiting
  * for the previous kernel in the stream, so the host-link latency overlaps that kernel's
- * tail); the sweep then writes its results straight into out_host. Returns
+ * tail); the sweep then writes its results straight into out_host. Because x_host is
+ * read before earlier work in the stream has finished, its contents must be final when
+ * the call is made: work queued earlier on the stream must not write x_host. Returns
  * MTP_ERR_INVALID_ARG if x_host or out_host is not pinned host memory; otherwise the
  * requirements and results of mtp_lm_head_argmax (no logits output).
  * ------------------------------------------------------------------------------ */
@@ -347,12 +349,17 @@ mtp_status mtp_debug_kv_write(const uint16_t* k_rot, const uint16_t* v, int64_t 
  * for x in the form the many-input sweeps read it (FP8 tables from M = 7, NVFP4 from
  * M = 9), so those calls return MTP_ERR_WORKSPACE here; BF16 tables run at every M up
  * to 32.
- *  - The first call made with a device current looks up that array's device address
- *    and zeroes its counter (synchronously); make it before any stream capture.
- *  - All calls on a device share the array: calls that overlap on the GPU race and
- *    must be serialised by the caller. Each call leaves the counter zero again.
- *  - Returns MTP_ERR_WORKSPACE if a call would need more scratch than the array holds;
- *    it never allocates.
+ *  - The first call made with a device current looks up that array's device address.
+ *    Under the CUDA runtime's lazy module loading (the default since CUDA 12.2) that
+ *    look-up is also when the array is committed on the device, so make the first call
+ *    on each device before reserving the device's free memory, and before any stream
+ *    capture; later calls change no device memory outside their inputs and outputs.
+ *  - The array is zero when its module loads, and each call leaves its counter zero
+ *    again. All calls on a device share the array: calls that overlap on the GPU race
+ *    and must be serialised by the caller.
+ *  - Arguments are checked as mtp_lm_head_argmax checks them, before anything else;
+ *    then MTP_ERR_WORKSPACE if the call would need more scratch than the array holds.
+ *    It never allocates.
  * ------------------------------------------------------------------------------ */
 size_t mtp_noalloc_scratch_bytes(void);
 mtp_status mtp_lm_head_argmax_noalloc(const mtp_weight* head, int64_t n_eff, const uint16_t* x,

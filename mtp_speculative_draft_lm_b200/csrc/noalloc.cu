@@ -13,11 +13,14 @@
 // holds it (kScratchBytes) until the process exits, and every call on that GPU shares
 // it. In host code `g_sweep_scratch` names a host-side stand-in, not device memory, so
 // the kernel is given the address that cudaGetSymbolAddress returns for the current
-// device. That set-up runs on the first call made with each device current (it also
-// zeroes the counter once, with a synchronous cudaMemset); make that first call
-// before any stream capture. Afterwards each call leaves the counter at zero again.
-// Calls that overlap on the GPU (two streams, or two host threads) share the array
-// and race: serialise them. Nothing here allocates: no cudaMalloc, no cudaFree.
+// device. That look-up runs on the first call made with each device current. With the
+// CUDA runtime's lazy module loading (the default since CUDA 12.2) it is also the moment
+// the array is committed on that device, so make the first call before reserving the
+// device's free memory, and before any stream capture. A __device__ array without an
+// initialiser is zero when its module loads, so the counter starts at zero; each call
+// leaves it at zero again. Calls that overlap on the GPU (two streams, or two host
+// threads) share the array and race: serialise them. Nothing here allocates: no
+// cudaMalloc, no cudaFree, no memset.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -45,7 +48,6 @@ mtp_status scratch_for_current_device(void** out) {
     if (!g_scratch_ptr[dev]) {
         void* ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_sweep_scratch) != cudaSuccess || !ptr) return MTP_ERR_CUDA;
-        if (cudaMemset(ptr, 0, kTicketBytes) != cudaSuccess) return MTP_ERR_CUDA;
         g_scratch_ptr[dev] = ptr;
     }
     *out = g_scratch_ptr[dev];
@@ -62,13 +64,15 @@ extern "C" mtp_status mtp_lm_head_argmax_noalloc(const mtp_weight* head, int64_t
                                                  int64_t mask_stride_words, int32_t* out_idx,
                                                  float* out_val, uint16_t* out_logits,
                                                  int32_t* dev_err, void* stream) {
-    if (head && mtp_lm_head_ws_bytes(head, n_eff, M) > kScratchBytes) return MTP_ERR_WORKSPACE;
-    void* scratch = nullptr;
-    // argument checks first, so that a rejected call never triggers the set-up
+    // Argument checks first (a null workspace is the one thing left to reject), so that a
+    // rejected call never reads an unchecked table descriptor nor triggers the set-up;
+    // then the scratch size this call needs.
     mtp_status st = mtp_lm_head_argmax(head, n_eff, x, M, mask, mask_words, mask_stride_words,
                                        out_idx, out_val, out_logits, dev_err, nullptr,
                                        kScratchBytes, nullptr);
     if (st != MTP_ERR_WORKSPACE) return st == MTP_OK ? MTP_ERR_CUDA : st;
+    if (mtp_lm_head_ws_bytes(head, n_eff, M) > kScratchBytes) return MTP_ERR_WORKSPACE;
+    void* scratch = nullptr;
     if ((st = scratch_for_current_device(&scratch)) != MTP_OK) return st;
     return mtp_lm_head_argmax(head, n_eff, x, M, mask, mask_words, mask_stride_words, out_idx,
                               out_val, out_logits, dev_err, scratch, kScratchBytes, stream);

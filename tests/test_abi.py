@@ -145,7 +145,14 @@ def test_lm_head_lp_rejects(lib):
     noalloc = lambda head, M: st("mtp_lm_head_argmax_noalloc", C.byref(head), 100, B2, M, None,
                                  0, 0, OUT, None, None, None, None)
     assert noalloc(fp8, 7) == L.MTP_ERR_WORKSPACE
-    assert noalloc(weight(fmt=2, k=128, bs=OUT, gs=OUT), 12) == L.MTP_ERR_WORKSPACE
+    assert noalloc(weight(fmt=2, k=256, bs=OUT, gs=OUT), 12) == L.MTP_ERR_WORKSPACE
+    # the table descriptor is checked before its size is looked at: a bad format, a bad k
+    # or a missing scale is an argument error, not a workspace one
+    assert noalloc(weight(fmt=7, k=128), 12) == L.MTP_ERR_INVALID_ARG
+    assert noalloc(weight(fmt=1, k=100, rs=OUT), 7) == L.MTP_ERR_INVALID_ARG
+    assert noalloc(weight(fmt=2, k=256, bs=OUT), 12) == L.MTP_ERR_INVALID_ARG
+    # rows that are not a whole number of 128-byte segments are unsupported, at any M
+    assert noalloc(weight(fmt=2, k=128, bs=OUT, gs=OUT), 12) == L.MTP_ERR_UNSUPPORTED
 
 
 def test_lm_head_host_rejects(lib):
