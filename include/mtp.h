@@ -177,17 +177,18 @@ mtp_status mtp_combine(const uint16_t* embed, int64_t vocab, const int32_t* toke
  *                 counter zero again. It also holds x as the many-input sweeps read
  *                 it, rewritten by each call: for FP8 tables with M >= 7 two E4M3
  *                 planes of 16 or 32 rows (2 * 16 * k or 2 * 32 * k bytes), for NVFP4
- *                 with M > 8 an f16 copy (M * k * 2 bytes).
+ *                 with M >= 3 an f16 copy (M * k * 2 bytes).
  * Requires 1 <= M <= 32, 1 <= n_eff <= n; table rows a multiple of 128 bytes (k % 64
  * for BF16, % 128 for FP8, % 256 for NVFP4; the sweep streams 128-byte segments); for
  * M <= 8 (FP8: M <= 6) the staged inputs (M * k * 2 bytes) must leave shared memory for
  * the stream (MTP_ERR_UNSUPPORTED otherwise; more inputs stream x per K chunk instead).
  * Results are bit-identical for every M within BF16 1-8, 9-16, 17-32; FP8 1-6, 7-16,
  * 17-32; NVFP4 1-2, 3-8, 9-16, 17-32, whose sweeps sum the same products in different
- * fixed orders. BF16 and FP8 tables with more inputs run on the tcgen05 tensor cores;
- * there x enters FP8 products as two E4M3 terms whose sum is x exactly except for
- * elements below 2^-9 of the input's largest |x|, which keep an absolute error of at
- * most 2^-17 of that largest |x|.
+ * fixed orders. BF16 tables from 9 inputs, FP8 from 7 and NVFP4 from 3 run on the
+ * tcgen05 tensor cores; there x enters FP8 products as two E4M3 terms whose sum is x
+ * exactly except for elements below 2^-9 of the input's largest |x|, which keep an
+ * absolute error of at most 2^-17 of that largest |x|. With a grammar mask and up to 8
+ * inputs only the table rows that some input's mask allows are read.
  * ------------------------------------------------------------------------------ */
 size_t mtp_lm_head_ws_bytes(const mtp_weight* head, int64_t n_eff, int32_t M);
 mtp_status mtp_lm_head_argmax(const mtp_weight* head, int64_t n_eff, const uint16_t* x,
@@ -300,13 +301,17 @@ mtp_status mtp_argmax_merge_partials(const void* partials, int32_t n_parts, int3
  *   wk, wv (device) bf16 [nkv * hd, h]; block_table (device) i32 [n_table];
  *   k_cache, v_cache (device) u8 [num_blocks, block_size, nkv, hd], written in place;
  *   ws (device) mtp_prefill_ws_bytes(min(chunk_rows, R), h, nkv, hd) bytes, 1 KB
- *   aligned: two lanes of one chunk's concat rows, fc output and RoPE table. Half of
- *   that (one lane) is the minimum (MTP_ERR_WORKSPACE below it) and runs the chunks one
- *   after another on `stream`; with both lanes, consecutive chunks run side by side on
- *   two library-owned streams (created per device on first use, kept until the process
- *   exits), forked from and joined back into `stream` with events, so the call still
- *   orders like one operation on `stream` and can be captured in a CUDA graph.
- * Rows run in chunks of chunk_rows (the GEMMs' M). Requires h % 256 == 0,
+ *   aligned, no initial contents required: a small counter header (zeroed by the call
+ *   itself with a memset on `stream`), then two lanes of a chunk's concat rows and fc
+ *   output and three RoPE tables. Half of that size (one lane, two RoPE tables) is the
+ *   minimum (MTP_ERR_WORKSPACE below it); with one lane consecutive chunks take turns on
+ *   the same buffers, with two they overlap. The whole call is one kernel on `stream`
+ *   (after the memset): every SM takes the chunks' prologue, fc and k/v tiles in one fixed
+ *   order from a counter in the header, waiting (bounded) on per-chunk completion counters
+ *   there, so the next chunk's tiles fill the SMs the current one leaves idle. The library
+ *   creates no streams or events; the call can be captured in a CUDA graph. Calls that
+ *   share a workspace must not overlap.
+ * Rows run in chunks of chunk_rows (the GEMMs' M). Requires h % 256 == 0, h <= 12288,
  * hd in {64, 128, 256}, nkv * hd % 256 == 0, k_scale, v_scale > 0.
  * ------------------------------------------------------------------------------ */
 size_t mtp_prefill_ws_bytes(int64_t chunk_rows, int32_t h, int32_t nkv, int32_t hd);
@@ -347,7 +352,7 @@ mtp_status mtp_debug_kv_write(const uint16_t* k_rot, const uint16_t* v, int64_t 
  * (524,544: a 256-byte header + 16-byte partials of up to 1,024 CTAs x 32 input rows)
  * held on every GPU that loads the library until the process exits. It has no room
  * for x in the form the many-input sweeps read it (FP8 tables from M = 7, NVFP4 from
- * M = 9), so those calls return MTP_ERR_WORKSPACE here; BF16 tables run at every M up
+ * M = 3), so those calls return MTP_ERR_WORKSPACE here; BF16 tables run at every M up
  * to 32.
  *  - The first call made with a device current looks up that array's device address.
  *    Under the CUDA runtime's lazy module loading (the default since CUDA 12.2) that
@@ -366,6 +371,18 @@ mtp_status mtp_lm_head_argmax_noalloc(const mtp_weight* head, int64_t n_eff, con
                                       int32_t M, const int32_t* mask, int64_t mask_words,
                                       int64_t mask_stride_words, int32_t* out_idx, float* out_val,
                                       uint16_t* out_logits, int32_t* dev_err, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * mtp_debug_wait_timeout -- self-check of the bounded waits every pipelined kernel here
+ * uses (the pages have no counterpart: it tests this library's failure handling). One
+ * small kernel waits, through the same helpers, on something that never happens --
+ * which 0: an mbarrier phase no thread completes; which 1: the device u32 *counter
+ * reaching 1 (the caller keeps it 0) -- gives up after limit_cycles SM clock cycles
+ * (1 .. 4e9; the pipelines use about one second), ORs MTP_DEVFLAG_TIMEOUT into *dev_err
+ * (device i32, required) and ends; the context stays usable.
+ * ------------------------------------------------------------------------------ */
+mtp_status mtp_debug_wait_timeout(int32_t which, int64_t limit_cycles, const uint32_t* counter,
+                                  int32_t* dev_err, void* stream);
 
 /* Maps a device error word read back by the caller to a status: MTP_OK, or
  * MTP_WARN_EMPTY_MASK when only the empty-mask bit is set, else MTP_ERR_INVALID_ARG. */

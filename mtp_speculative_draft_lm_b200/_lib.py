@@ -38,6 +38,7 @@ EXPORTS = (
     "mtp_lm_head_host_ws_bytes", "mtp_lm_head_argmax_host",
     "mtp_lm_head_shard_partial", "mtp_argmax_merge_partials",
     "mtp_debug_encode_e4m3", "mtp_debug_encode_e2m1", "mtp_nvfp4_scale_pitch",
+    "mtp_debug_wait_timeout",
     "mtp_noalloc_scratch_bytes", "mtp_lm_head_argmax_noalloc",
     "mtp_prefill_ws_bytes", "mtp_prefill_kv", "mtp_debug_gemm_bf16", "mtp_debug_kv_write",
 )
@@ -92,6 +93,7 @@ _SIGS = {
     "mtp_noalloc_scratch_bytes": (_SZ, []),
     "mtp_lm_head_argmax_noalloc": (C.c_int, [_W, _I64, _P, _I32, _P, _I64, _I64, _P, _P, _P,
                                              _P, _P]),
+    "mtp_debug_wait_timeout": (C.c_int, [_I32, _I64, _P, _P, _P]),
     "mtp_debug_encode_e4m3": (C.c_int, [_P, _I64, _P, _P]),
     "mtp_debug_encode_e2m1": (C.c_int, [_P, _I64, _P, _P]),
 }
@@ -278,6 +280,12 @@ def mtp_lm_head_argmax_noalloc(head, n_eff, x, M, mask, mask_words, mask_stride_
                                              mask_stride_words, _ptr(out_idx), _ptr(out_val),
                                              _ptr(out_logits), _ptr(dev_err), _stream(stream)),
            "mtp_lm_head_argmax_noalloc")
+
+
+def mtp_debug_wait_timeout(which, limit_cycles, counter, dev_err, stream=None):
+    _check(load().mtp_debug_wait_timeout(int(which), int(limit_cycles), _ptr(counter),
+                                         _ptr(dev_err), _stream(stream)),
+           "mtp_debug_wait_timeout")
 
 
 def mtp_debug_encode_e4m3(inp, n, out, stream=None):

@@ -76,12 +76,13 @@ class LmHead:
         self.ws = torch.zeros((nbytes,), dtype=torch.uint8, device=dev)
         self.dev_err = torch.zeros((1,), dtype=torch.int32, device=dev)
 
-    def bytes_per_call(self, M: int, mask_words: int = 0) -> int:
-        """Algorithmic bytes of one unmasked sweep: the swept table rows, the inputs,
-        the mask words and the outputs."""
+    def bytes_per_call(self, M: int, mask_words: int = 0, rows: int | None = None) -> int:
+        """Algorithmic bytes of one sweep: the table rows it must read (all n_eff rows, or
+        `rows` of them under a grammar mask), the inputs, the mask words and the
+        outputs."""
         t = self.table
-        frac = self.n_eff / t.n
-        return int(t.nbytes() * frac) + M * t.k * 2 + mask_words * 4 * (1 if M else 0) + M * 8
+        frac = (self.n_eff if rows is None else rows) / t.n
+        return int(t.nbytes() * frac) + M * t.k * 2 + mask_words * 4 + M * 8
 
     def __call__(self, x: torch.Tensor, out_idx: torch.Tensor, out_val=None, out_logits=None,
                  mask=None, mask_words=0, mask_stride_words=0, stream=None, out_logprob=None):

@@ -181,7 +181,7 @@ mtp_status lm_head_impl(const mtp_weight* head, int64_t n_eff, const uint16_t* x
         return MTP_ERR_INVALID_ARG;
     if (!ws || !aligned(ws, 16) || ws_bytes < mtp_lm_head_ws_bytes(head, n_eff, M))
         return MTP_ERR_WORKSPACE;
-    if (mtp::sweep_smem_bytes(M, head->k, head->fmt, nullptr, 0) > 227 * 1024)
+    if (mtp::sweep_smem_bytes(M, head->k, head->fmt, nullptr, 0, mask != nullptr) > 227 * 1024)
         return MTP_ERR_UNSUPPORTED;
     mtp::SweepParams p{};
     p.w = static_cast<const uint8_t*>(head->data);
@@ -331,8 +331,8 @@ mtp_status mtp_prefill_kv(const uint16_t* embed, int64_t vocab, const int32_t* t
         !finite_pos(v_scale) || !(rope_base > 0.f) || cache_start < 0)
         return MTP_ERR_INVALID_ARG;
     const int tn = mtp::gemm_tile_n();
-    if (h % tn || (hd != 64 && hd != 128 && hd != 256) || ((int64_t)nkv * hd) % tn ||
-        chunk_rows > (int64_t)1 << 30)
+    if (h % tn || h > mtp::prefill_max_hidden() || (hd != 64 && hd != 128 && hd != 256) ||
+        ((int64_t)nkv * hd) % tn || chunk_rows > (int64_t)1 << 30)
         return MTP_ERR_UNSUPPORTED;
     if (!aligned(embed, 16) || !aligned(hidden, 16) || !aligned(fc, 16) || !aligned(wk, 16) ||
         !aligned(wv, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
@@ -398,6 +398,15 @@ mtp_status mtp_debug_kv_write(const uint16_t* k_rot, const uint16_t* v, int64_t 
     return from_cuda(mtp::kv_write_launch(k_rot, v, R, nkv, hd, cache_start, block_table, n_table,
                                           block_size, num_blocks, k_cache, v_cache, k_scale,
                                           v_scale, dev_err, as_stream(stream)));
+}
+
+mtp_status mtp_debug_wait_timeout(int32_t which, int64_t limit_cycles, const uint32_t* counter,
+                                  int32_t* dev_err, void* stream) {
+    if ((which != 0 && which != 1) || limit_cycles < 1 || limit_cycles > 4000000000LL || !dev_err ||
+        !aligned(dev_err, 4) || (which == 1 && (!counter || !aligned(counter, 4))))
+        return MTP_ERR_INVALID_ARG;
+    return from_cuda(mtp::wait_timeout_launch(which, (long long)limit_cycles, counter, dev_err,
+                                              as_stream(stream)));
 }
 
 mtp_status mtp_debug_encode_e4m3(const float* in, int64_t n, uint8_t* out, void* stream) {

@@ -238,14 +238,40 @@ constexpr long long kWaitLimitCycles = 2000000000LL;
 // thread still reaches the end of the kernel. With abort == nullptr only the time limit
 // applies (used to drain copies in flight at exit).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort) {
+                                                  volatile int* abort,
+                                                  long long limit = kWaitLimitCycles) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait_sleep(bar, parity, 2000u)) return true;
         if (abort && *abort) return false;
-        if (clock64() - t0 > kWaitLimitCycles) {
+        if (clock64() - t0 > limit) {
             if (abort) *abort = 1;
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* a) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+    return v;
+}
+
+// Waits until the global counter *a reaches `target` (GPU-scope acquire loads), sleeping
+// between checks; gives up like mbar_wait_bounded (at once when *abort is set, or after
+// `limit` cycles, setting *abort).
+__device__ __forceinline__ bool counter_wait_bounded(const uint32_t* a, uint32_t target,
+                                                     volatile int* abort,
+                                                     long long limit = kWaitLimitCycles) {
+    if (ld_acquire_gpu(a) >= target) return true;
+    const long long t0 = clock64();
+    while (true) {
+        __nanosleep(500);
+        if (ld_acquire_gpu(a) >= target) return true;
+        if (*abort) return false;
+        if (clock64() - t0 > limit) {
+            *abort = 1;
             return false;
         }
     }

@@ -72,7 +72,8 @@ cudaError_t merge_partials_launch(const void* parts, int n_parts, int M, int32_t
 // input does not fit in shared memory.
 cudaError_t sweep_launch(const SweepParams& p, int fmt, int mode, cudaStream_t s,
                          SweepLaunch* info);
-size_t sweep_smem_bytes(int M, int64_t k, int fmt, int* kpad_out, int mode);
+// Shared memory the sweep for these inputs needs (masked: the gathered sweep, M <= 8).
+size_t sweep_smem_bytes(int M, int64_t k, int fmt, int* kpad_out, int mode, bool masked = false);
 // Workspace bytes the many-input argmax sweeps need for x in their own form (FP8 tables
 // from 7 inputs: two E4M3 planes; NVFP4 from 9: an f16 copy) plus 1 KB of per-input
 // exponents: 0 for BF16 and for fewer inputs.
@@ -123,10 +124,12 @@ struct PrefillArgs {
     size_t ws_bytes;
     int32_t* dev_err;
 };
-// One chunk's buffers (concat rows, fc output, RoPE table); the workspace holds two such
-// lanes so that consecutive chunks can run side by side.
+// Workspace of the prefill: a counter header, then one or two lanes of a chunk's concat
+// rows and fc output rows, and one more RoPE table than lanes. prefill_lane_bytes is the
+// one-lane minimum, prefill_ws_bytes the two-lane size (consecutive chunks overlap).
 size_t prefill_lane_bytes(int64_t chunk_rows, int32_t h, int32_t nkv, int32_t hd);
 size_t prefill_ws_bytes(int64_t chunk_rows, int32_t h, int32_t nkv, int32_t hd);
+int prefill_max_hidden();
 cudaError_t prefill_launch(const PrefillArgs& a, cudaStream_t s);
 cudaError_t gemm_bf16_launch(const uint16_t* A, const uint16_t* B, uint16_t* C, int M, int N,
                              int K, int32_t* dev_err, cudaStream_t s);
@@ -136,6 +139,12 @@ cudaError_t kv_write_launch(const uint16_t* k_rot, const uint16_t* v, int64_t R,
                             float k_scale, float v_scale, int32_t* dev_err, cudaStream_t s);
 int gemm_tile_n();
 int gemm_tile_k();
+
+// Self-check of the bounded waits (selfcheck.cu): which 0 waits on an mbarrier phase that
+// nothing completes, 1 on a global counter (device u32, kept at 0 by the caller) that
+// nothing increments; either gives up after limit_cycles and sets DEVFLAG_TIMEOUT.
+cudaError_t wait_timeout_launch(int which, long long limit_cycles, const uint32_t* counter,
+                                int32_t* dev_err, cudaStream_t s);
 
 // Encoders exposed for exhaustive checks.
 cudaError_t debug_encode_launch(const float* in, int64_t n, uint8_t* out, int which,

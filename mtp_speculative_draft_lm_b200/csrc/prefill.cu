@@ -5,22 +5,38 @@
 // (embed(token_{i+1}), target_hidden_i), so no attention runs; block size 16 and the
 // FP8 cache in metrale_model_layers/layers/mtp_head/new.rs; the slot rule of
 // metrale_model_arch/deepseek_v4_mtp.rs forward_one step 4). Per prompt row r:
-//   c  = [bf16(rms(embed[tok_r]) w_e) || bf16(rms(hidden_r) w_h)]          (prologue)
-//   y  = bf16(fc . c)                                           (GEMM 1, tcgen05)
-//   k  = bf16(Wk . y), v = bf16(Wv . y)                         (GEMM 2, tcgen05)
+//   c  = [bf16(rms(embed[tok_r]) w_e) || bf16(rms(hidden_r) w_h)]           (prologue)
+//   y  = bf16(fc . c)                                                   (fc GEMM)
+//   k  = bf16(Wk . y), v = bf16(Wv . y)                                 (k/v GEMM)
 //   k' = bf16(RoPE_neox(k, pos_r)) per head, codes = e4m3(k' / k_scale), e4m3(v / v_scale)
 //   cache row p = cache_start + r, slot = block_table[p / bs] * bs + p % bs,
-//   element (slot, head, d) of a [num_blocks, bs, nkv, hd] cache.        (GEMM 2 epilogue)
+//   element (slot, head, d) of a [num_blocks, bs, nkv, hd] cache.       (k/v epilogue)
 //
-// Design (B200): rows are processed in chunks (the reference's PREFILL_CHUNK). The two
-// projections are the only dense contractions, so they run on the 5th-generation tensor
-// cores: one persistent kernel per GEMM, 128 x 256 output tiles, a 4-stage TMA ring
-// (128-byte swizzle, K-major A and B), tcgen05.mma issued by one thread into a
-// double-buffered 512-column TMEM accumulator, and four epilogue warps that read it back
-// with tcgen05.ld while the next tile accumulates. GEMM 2's epilogue applies RoPE from a
-// per-row cos/sin table (computed in double by the prologue), encodes E4M3 and scatters
-// each row's 32-byte pieces straight into the paged cache: K/V never round-trip through
-// HBM in bf16. All waits are bounded (abort flag + MTP_DEVFLAG_TIMEOUT).
+// Design (B200): rows are processed in chunks (the reference's PREFILL_CHUNK), whose
+// buffers (concat rows, fc output, RoPE table) live in the caller's workspace. The whole
+// call is ONE persistent kernel on the caller's stream: every CTA takes work items
+// ("tiles") from one counter, in a fixed global order, so that the tiles of the next
+// chunk fill the SMs the current chunk leaves idle (a 2,048-row chunk's fc GEMM is 320
+// output tiles, 2.16 waves on 148 SMs). Three kinds of tile:
+//   P (chunk c, row block m): the prologue of 128 rows -- the producer warp bulk-copies
+//     each row's embedding row and hidden row into the shared-memory ring, the four
+//     epilogue warps take the two RMSNorms, write the bf16 concat rows and the rows'
+//     RoPE table (cos, sin in double).
+//   F (c, m, n): a 128 x 256 tile of the fc GEMM, y = c . fc^T, bf16 out.
+//   V (c, m, n): a 128 x 256 tile of the k/v GEMM whose epilogue rotates k (RoPE),
+//     encodes E4M3 and writes each row's 32-byte pieces at its paged slot.
+// Order: for b = 0..chunks: P(b), F(b), then V(b - 1) (with a single lane V(b - 1)
+// first). A tile only ever waits for tiles earlier in that order (completion counters per chunk slot and row block, in the
+// workspace header, release/acquire at GPU scope): F(c, m, .) for P(c, m); V(c, m, .)
+// for all of F(c, m, .); and a tile that overwrites a buffer another chunk used (two
+// lanes of concat and fc-output rows, three of RoPE rows) for that chunk's readers.
+// Tiles are claimed only by running CTAs, so the oldest unfinished tile can always
+// finish. GEMM tiles run on the 5th-generation tensor cores: a 4-stage TMA ring
+// (128-byte swizzle, K-major A and B), tcgen05.mma from one thread into a double-
+// buffered 512-column TMEM accumulator, four epilogue warps reading it back with
+// tcgen05.ld while the next tile accumulates. A small FIFO in shared memory tells the
+// MMA and epilogue warps which tile comes next. Every wait is bounded (abort flag +
+// MTP_DEVFLAG_TIMEOUT): nothing hangs.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -40,20 +56,33 @@ constexpr int kAStageBytes = BM * BK * 2;  // 16 KB
 constexpr int kBStageBytes = BN * BK * 2;  // 32 KB
 constexpr int kGStageBytes = kAStageBytes + kBStageBytes;
 constexpr int kGemmThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int kEpiThreads = 128;
 constexpr int kTmemCols = 2 * BN;  // two fp32 accumulators of 128 lanes x 256 columns
-constexpr int kGemmSmem = kGStages * kGStageBytes + 1024 /* barriers */ + 1024 /* align */;
-constexpr int kPrologueThreads = 256;
+constexpr int kFifo = 8;           // tiles announced ahead to the MMA and epilogue warps
+constexpr int kCtrSlots = 4;       // completion counters: chunk c uses slot c % 4
+constexpr int kMaxRowsPerPStage = 8;
+constexpr int kMaxLanes = 2;       // concat / fc-output lanes (RoPE rows: lanes + 1)
+// shared memory after the ring: barriers, the tile FIFO, per-stage row tokens, the
+// epilogue's reduction scratch and inverse frequencies
+constexpr int kHeadBytes = 4096;
+constexpr int kGemmSmem = kGStages * kGStageBytes + kHeadBytes + 1024 /* align */;
 
-struct GemmParams {
-    int M, N, K;        // rows of A (valid), columns of the output, reduction length
-    int m_tiles, n_tiles;
-    // epilogue 0: bf16 output
-    uint16_t* C;
-    int64_t ldc;
-    // epilogue 1: k/v -> RoPE (k) -> E4M3 -> paged cache
+enum : int { TILE_P = 0, TILE_F = 1, TILE_V = 2 };
+
+struct PrefillParams {
+    // inputs
+    const uint16_t* embed;
+    int64_t vocab;
+    const int32_t* tokens;
+    const uint16_t* hidden;
+    int64_t R;
+    int h;
+    const uint16_t* w_ne;
+    const uint16_t* w_nh;
+    float eps;
     int nkv, hd;
-    const float2* rope_cs;  // [M][hd/2] (cos, sin)
-    int64_t row0;           // prompt row of this chunk's first row
+    double rope_base;
+    const int32_t* rope_pos;
     int64_t cache_start;
     const int32_t* block_table;
     int64_t n_table;
@@ -63,10 +92,128 @@ struct GemmParams {
     uint8_t* v_cache;
     float k_scale, v_scale;
     int32_t* dev_err;
+    // schedule
+    int plain;           // 1: a plain GEMM C = A . B^T (stage check), F tiles only
+    int64_t chunk;       // rows per chunk
+    int n_chunks;
+    int mt_full;         // 128-row blocks of a full chunk
+    int mt_last;         // of the last chunk
+    int nf;              // fc GEMM column tiles (h / 256)
+    int nv;              // k/v GEMM column tiles (2 nkv hd / 256)
+    int64_t b0, s_mid, n_mid, b_last;  // tiles in block 0, a middle block, the last but one
+    int64_t total;       // tiles in all
+    int lanes;           // 1 or 2
+    int rows_per_pstage;
+    uint32_t* ctr;       // [0] tile counter; then done counters [3][kCtrSlots][mt_full]
+    uint16_t* concat[kMaxLanes];
+    uint16_t* y[kMaxLanes];
+    float2* rope[kMaxLanes + 1];
+    // plain GEMM
+    uint16_t* C;
+    int M, N, K;
 };
 
-// Cache slot of prompt row (row0 + r), or -1 when its block is missing / out of range.
-__device__ __forceinline__ int64_t cache_slot(const GemmParams& p, int64_t prompt_row) {
+struct Tile {
+    int kind, c, m, n;
+};
+
+__device__ __forceinline__ int mt_of(const PrefillParams& p, int c) {
+    return c == p.n_chunks - 1 ? p.mt_last : p.mt_full;
+}
+
+// Tile t of the global order: block b holds P(b), F(b) (b < chunks) and V(b - 1) (b >= 1).
+__device__ Tile decode(const PrefillParams& p, int64_t t) {
+    Tile r{};
+    if (p.plain) {  // F tiles of one GEMM, M-fastest
+        const int mt = (p.M + BM - 1) / BM;
+        r.kind = TILE_F;
+        r.c = 0;
+        r.m = (int)(t % mt);
+        r.n = (int)(t / mt);
+        return r;
+    }
+    int b;
+    int64_t off;
+    if (t < p.b0) {
+        b = 0;
+        off = t;
+    } else {
+        t -= p.b0;
+        if (t < p.n_mid * p.s_mid) {
+            b = 1 + (int)(t / p.s_mid);
+            off = t % p.s_mid;
+        } else {
+            t -= p.n_mid * p.s_mid;
+            if (p.n_chunks >= 2 && t < p.b_last) {
+                b = p.n_chunks - 1;
+                off = t;
+            } else {
+                if (p.n_chunks >= 2) t -= p.b_last;
+                b = p.n_chunks;
+                off = t;
+            }
+        }
+    }
+    // with two lanes a block is P(b), F(b), V(b - 1); with one lane V(b - 1) comes first,
+    // since F(b) then reuses the fc-output rows V(b - 1) reads
+    const int mtb = b < p.n_chunks ? mt_of(p, b) : 0;
+    if (p.lanes == 1 && b >= 1) {
+        const int mtv = mt_of(p, b - 1);
+        const int64_t nvb = (int64_t)mtv * p.nv;
+        if (off < nvb) {
+            r.kind = TILE_V;
+            r.c = b - 1;
+            r.m = (int)(off % mtv);
+            r.n = (int)(off / mtv);
+            return r;
+        }
+        off -= nvb;
+    }
+    if (off < mtb) {
+        r.kind = TILE_P;
+        r.c = b;
+        r.m = (int)off;
+    } else if (off < (int64_t)mtb * (1 + p.nf)) {
+        const int64_t i = off - mtb;
+        r.kind = TILE_F;
+        r.c = b;
+        r.m = (int)(i % mtb);
+        r.n = (int)(i / mtb);
+    } else {
+        const int64_t i = off - (int64_t)mtb * (1 + p.nf);
+        const int mtv = mt_of(p, b - 1);
+        r.kind = TILE_V;
+        r.c = b - 1;
+        r.m = (int)(i % mtv);
+        r.n = (int)(i / mtv);
+    }
+    return r;
+}
+
+// Completion counters: kind k (P, F, V) of the chunks in slot c % 4, row block m. They
+// only grow within a call: after chunk c's tiles of row block m are all done, the P
+// counter reads c / 4 + 1, F (c / 4 + 1) nf, V (c / 4 + 1) nv.
+__device__ __forceinline__ uint32_t* counter(const PrefillParams& p, int kind, int c, int m) {
+    return p.ctr + 64 + ((size_t)kind * kCtrSlots + (size_t)(c % kCtrSlots)) * p.mt_full + m;
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ bool wait_counter(const uint32_t* a, uint32_t target, volatile int* abort) {
+    return counter_wait_bounded(a, target, abort);
+}
+
+// One thread of the writers adds 1 once every writer's stores are visible (the caller
+// has synchronised the writers): a GPU-scope release.
+__device__ __forceinline__ void counter_release_add(uint32_t* a, uint32_t v) {
+    fence_acq_rel_gpu();
+    atomicAdd(a, v);
+}
+
+// Cache slot of prompt row `prompt_row`, or -1 when its block is missing / out of range.
+__device__ __forceinline__ int64_t cache_slot(const PrefillParams& p, int64_t prompt_row) {
     const int64_t pos = p.cache_start + prompt_row;
     if (pos < 0) return -1;
     const int64_t b = pos / p.block_size;
@@ -104,85 +251,60 @@ __device__ __forceinline__ void rope32(float (&lo)[32], float (&hi)[32], const f
     }
 }
 
-// ------------------------------------------------------------------------------ prologue
-// One CTA per chunk row: the combiner's concat row c[r] = [ne || nh] and the RoPE table.
-__global__ void __launch_bounds__(kPrologueThreads) prefill_prologue_kernel(
-    const uint16_t* __restrict__ embed, int64_t vocab, const int32_t* __restrict__ tokens,
-    const uint16_t* __restrict__ hidden, int h, const uint16_t* __restrict__ w_ne,
-    const uint16_t* __restrict__ w_nh, float eps, const int32_t* __restrict__ rope_pos,
-    double rope_base, int hd, int64_t row0, uint16_t* __restrict__ c_out,
-    float2* __restrict__ cs_out, int32_t* dev_err) {
-    __shared__ float red[2][kPrologueThreads / 32];
-    const int r = blockIdx.x, tid = threadIdx.x;
-    const int64_t pr = row0 + r;
-    const int64_t tok = tokens[pr];
-    const bool bad = tok < 0 || tok >= vocab;
-    if (bad && tid == 0) raise_flag(dev_err, DEVFLAG_BAD_TOKEN);
-    const uint16_t* e = bad ? nullptr : embed + tok * h;
-    const uint16_t* x = hidden + pr * h;
-    float se = 0.f, sx = 0.f;
-    for (int j = tid; j < h; j += kPrologueThreads) {
-        const float ev = e ? bf16_to_f32(e[j]) : 0.f;
-        const float xv = bf16_to_f32(x[j]);
-        se += ev * ev;
-        sx += xv * xv;
-    }
-    for (int o = 16; o; o >>= 1) {
-        se += __shfl_xor_sync(0xffffffffu, se, o);
-        sx += __shfl_xor_sync(0xffffffffu, sx, o);
-    }
-    if ((tid & 31) == 0) {
-        red[0][tid >> 5] = se;
-        red[1][tid >> 5] = sx;
-    }
-    __syncthreads();
-    se = 0.f;
-    sx = 0.f;
+// 8 bf16 (one 16-byte piece) times a row factor and 8 norm weights, rounded to bf16.
+__device__ __forceinline__ uint4 norm8(uint4 v, float inv, uint4 w) {
+    const uint32_t a[4] = {v.x, v.y, v.z, v.w}, b[4] = {w.x, w.y, w.z, w.w};
+    uint32_t o[4];
 #pragma unroll
-    for (int w = 0; w < kPrologueThreads / 32; ++w) {
-        se += red[0][w];
-        sx += red[1][w];
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t lo = f32_to_bf16(bf16_lo(a[i]) * inv * bf16_lo(b[i]));
+        const uint32_t hi = f32_to_bf16(bf16_hi(a[i]) * inv * bf16_hi(b[i]));
+        o[i] = lo | (hi << 16);
     }
-    const float inv_e = 1.0f / sqrtf(se / (float)h + eps);
-    const float inv_x = 1.0f / sqrtf(sx / (float)h + eps);
-    uint16_t* row = c_out + (int64_t)r * 2 * h;
-    for (int j = tid; j < h; j += kPrologueThreads) {
-        const float ev = e ? bf16_to_f32(e[j]) : 0.f;
-        row[j] = f32_to_bf16(ev * inv_e * bf16_to_f32(w_ne[j]));
-        row[h + j] = f32_to_bf16(bf16_to_f32(x[j]) * inv_x * bf16_to_f32(w_nh[j]));
-    }
-    const int half = hd / 2;
-    for (int j = tid; j < half; j += kPrologueThreads) {
-        const double inv_freq = pow(rope_base, -2.0 * (double)j / (double)hd);
-        const double th = (double)rope_pos[pr] * inv_freq;
-        double s, c;
-        sincos(th, &s, &c);
-        cs_out[(int64_t)r * half + j] = make_float2((float)c, (float)s);
-    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// ------------------------------------------------------------------------------ GEMM
-// out[M, N] = A[M, K] . B[N, K]^T with A, B bf16 K-major. EPI 0 stores bf16; EPI 1 is
-// the k/v epilogue (B rows [0, nkv*hd) from map_b0 = Wk, the rest from map_b1 = Wv).
-template <int EPI>
+__device__ __forceinline__ float sumsq8(uint4 v) {
+    const uint32_t a[4] = {v.x, v.y, v.z, v.w};
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float lo = bf16_lo(a[i]), hi = bf16_hi(a[i]);
+        s += lo * lo;
+        s += hi * hi;
+    }
+    return s;
+}
+
+struct Maps {
+    CUtensorMap a_concat[kMaxLanes];  // plain GEMM: a_concat[0] is A
+    CUtensorMap a_y[kMaxLanes];
+    CUtensorMap b_fc;                 // plain GEMM: B
+    CUtensorMap b_wk, b_wv;
+};
+
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap map_a,
-                const __grid_constant__ CUtensorMap map_b0,
-                const __grid_constant__ CUtensorMap map_b1) {
+    prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ Maps maps) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* stages = smem;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kGStages * kGStageBytes);
+    uint8_t* head = smem + kGStages * kGStageBytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(head);
     uint64_t* empty = full + kGStages;
-    uint64_t* tfull = empty + kGStages;   // [2]
-    uint64_t* tempty = tfull + 2;         // [2]
-    uint64_t* done = tempty + 2;          // MMA drain at exit
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    uint64_t* tfull = empty + kGStages;    // [2]
+    uint64_t* tempty = tfull + 2;          // [2]
+    uint64_t* done = tempty + 2;           // MMA drain at exit
+    uint64_t* qfull = done + 1;            // [kFifo] a tile index is in the FIFO slot
+    uint64_t* qempty = qfull + kFifo;      // [kFifo] both readers took it
+    int* fifo = reinterpret_cast<int*>(qempty + kFifo);          // [kFifo]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fifo + kFifo);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* stage_tok = reinterpret_cast<int*>(head + 512);         // [kGStages][8]
+    float* red = reinterpret_cast<float*>(head + 1024);          // [2][4 warps][2]
+    double* inv_freq = reinterpret_cast<double*>(head + 2048);   // [hd / 2 <= 128]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int total = p.m_tiles * p.n_tiles;
-    const int kb_count = p.K / BK;
+    const int kvd = p.nkv * p.hd;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kGStages; ++s) {
@@ -192,6 +314,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
             mbar_init(&tempty[b], 4);
+        }
+        for (int q = 0; q < kFifo; ++q) {
+            mbar_init(&qfull[q], 1);
+            mbar_init(&qempty[q], 2);  // the MMA warp and the epilogue warps
         }
         mbar_init(done, 1);
         *abort_flag = 0;
@@ -206,52 +332,176 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
+    // stages of a tile in the ring: a GEMM tile's K blocks, or a P tile's row groups
+    auto tile_stages = [&](const Tile& tl) -> int {
+        if (tl.kind == TILE_P) {
+            const int64_t rows_c = min(p.chunk, p.R - (int64_t)tl.c * p.chunk);
+            const int rows = (int)min((int64_t)BM, rows_c - (int64_t)tl.m * BM);
+            return (rows + p.rows_per_pstage - 1) / p.rows_per_pstage;
+        }
+        if (p.plain) return p.K / BK;
+        return (tl.kind == TILE_F ? 2 * p.h : p.h) / BK;
+    };
+
     if (warp == 0) {
-        // ---------------- TMA producer
+        // ---------------- producer: claims tiles, announces them, streams their stages
         int s = 0;
         uint32_t ph = 0;
-        bool stop = false;
+        int q = 0;
+        uint32_t qph = 0;
         int64_t issued = 0;
-        for (int t = blockIdx.x; t < total && !stop; t += gridDim.x) {
-            const int m = t % p.m_tiles, n = t / p.m_tiles;
-            const int brow = n * BN;
-            const bool second = EPI == 1 && brow >= p.nkv * p.hd;
-            for (int kb = 0; kb < kb_count; ++kb) {
-                if (!mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag)) {
-                    stop = true;
-                    break;
+        bool stop = false;
+        // the plain GEMM (no dependencies) takes tiles b, b + grid, ...; the prefill claims
+        // every tile from the counter, so a claimed tile always belongs to a running CTA
+        int64_t t = blockIdx.x;
+        if (!p.plain && lane == 0) t = atomicAdd(p.ctr, 1u);
+        t = __shfl_sync(0xffffffffu, t, 0);
+        while (!stop) {
+            const bool end = t >= p.total;
+            // announce the tile (or the end) to the MMA and epilogue warps
+            if (!mbar_wait_bounded(&qempty[q], qph ^ 1u, abort_flag)) break;
+            if (lane == 0) {
+                fifo[q] = end ? -1 : (int)t;
+                mbar_arrive(&qfull[q]);
+            }
+            __syncwarp();
+            if (++q == kFifo) {
+                q = 0;
+                qph ^= 1u;
+            }
+            if (end) break;
+            int64_t tn = t + gridDim.x;  // the next claim, issued early
+            if (!p.plain && lane == 0) tn = atomicAdd(p.ctr, 1u);
+            const Tile tl = decode(p, t);
+            const int nst = tile_stages(tl);
+            if (tl.kind == TILE_P) {
+                const int64_t row0 = (int64_t)tl.c * p.chunk + (int64_t)tl.m * BM;  // prompt row
+                const int64_t rows_c = min(p.chunk, p.R - (int64_t)tl.c * p.chunk);
+                const int rows = (int)min((int64_t)BM, rows_c - (int64_t)tl.m * BM);
+                const uint32_t rb = 2u * (uint32_t)p.h;  // bytes of one bf16 row
+                for (int st = 0; st < nst && !stop; ++st) {
+                    if (!mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    const int r0 = st * p.rows_per_pstage;
+                    const int nr = min(p.rows_per_pstage, rows - r0);
+                    int64_t tok = -1;
+                    if (lane < nr) {
+                        tok = p.tokens[row0 + r0 + lane];
+                        if (tok < 0 || tok >= p.vocab) {
+                            raise_flag(p.dev_err, DEVFLAG_BAD_TOKEN);
+                            tok = -1;
+                        }
+                        stage_tok[s * kMaxRowsPerPStage + lane] = (int)tok;
+                    }
+                    const uint32_t mine = lane < nr ? (tok >= 0 ? 2u * rb : rb) : 0u;
+                    uint32_t bytes = mine;
+#pragma unroll
+                    for (int o = 16; o; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_expect_tx(&full[s], bytes);
+                    __syncwarp();
+                    if (lane < nr) {
+                        uint8_t* dst = stages + (size_t)s * kGStageBytes + (size_t)lane * 2u * rb;
+                        if (tok >= 0) bulk_copy_g2s(dst, p.embed + tok * p.h, rb, &full[s]);
+                        bulk_copy_g2s(dst + rb, p.hidden + (row0 + r0 + lane) * p.h, rb, &full[s]);
+                    }
+                    __syncwarp();
+                    ++issued;
+                    if (++s == kGStages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
-                if (lane == 0) {
-                    uint8_t* st = stages + s * kGStageBytes;
-                    mbar_arrive_expect_tx(&full[s], kGStageBytes);
-                    tma_load_2d_g(st, &map_a, kb * BK, m * BM, &full[s]);
-                    tma_load_2d_g(st + kAStageBytes, second ? &map_b1 : &map_b0, kb * BK,
-                                  second ? brow - p.nkv * p.hd : brow, &full[s]);
+            } else {
+                // operands: F reads the chunk's concat rows, V its fc output rows; each only
+                // once the tiles that write them are done
+                const CUtensorMap* ma;
+                const CUtensorMap* mb;
+                int brow = tl.n * BN;
+                if (p.plain) {
+                    ma = &maps.a_concat[0];
+                    mb = &maps.b_fc;
+                } else if (tl.kind == TILE_F) {
+                    ma = &maps.a_concat[tl.c % p.lanes];
+                    mb = &maps.b_fc;
+                    if (lane == 0 && !wait_counter(counter(p, TILE_P, tl.c, tl.m),
+                                                   (uint32_t)(tl.c / kCtrSlots + 1), abort_flag))
+                        stop = true;
+                } else {
+                    ma = &maps.a_y[tl.c % p.lanes];
+                    mb = brow < kvd ? &maps.b_wk : &maps.b_wv;
+                    if (brow >= kvd) brow -= kvd;
+                    if (lane == 0 && !wait_counter(counter(p, TILE_F, tl.c, tl.m),
+                                                   (uint32_t)((tl.c / kCtrSlots + 1) * p.nf), abort_flag))
+                        stop = true;
                 }
-                __syncwarp();
-                ++issued;
-                if (++s == kGStages) {
-                    s = 0;
-                    ph ^= 1u;
+                stop = __shfl_sync(0xffffffffu, (int)stop, 0) != 0;
+                if (!p.plain && lane == 0) fence_proxy_async_global();  // then async reads
+                for (int kb = 0; kb < nst && !stop; ++kb) {
+                    if (!mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    if (lane == 0) {
+                        uint8_t* st = stages + (size_t)s * kGStageBytes;
+                        mbar_arrive_expect_tx(&full[s], kGStageBytes);
+                        tma_load_2d_g(st, ma, kb * BK, tl.m * BM, &full[s]);
+                        tma_load_2d_g(st + kAStageBytes, mb, kb * BK, brow, &full[s]);
+                    }
+                    __syncwarp();
+                    ++issued;
+                    if (++s == kGStages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
             }
+            t = __shfl_sync(0xffffffffu, tn, 0);
         }
+        // no copy left in flight
         for (int64_t j = issued > kGStages ? issued - kGStages : 0; j < issued; ++j)
             if (!mbar_wait_bounded(&full[j % kGStages], (uint32_t)((j / kGStages) & 1), nullptr)) break;
+        // if the loop stopped early, still tell the readers that no tile follows
+        if (stop && mbar_wait_bounded(&qempty[q], qph ^ 1u, nullptr) && lane == 0) {
+            fifo[q] = -1;
+            mbar_arrive(&qfull[q]);
+        }
+        __syncwarp();
     } else if (warp == 1) {
-        // ---------------- MMA issuer (one thread)
+        // ---------------- MMA issuer (one thread); P tiles' stages are the epilogue's
         constexpr uint32_t idesc = idesc_bf16(BM, BN);
         int s = 0;
         uint32_t ph = 0;
+        int q = 0;
+        uint32_t qph = 0;
         int local = 0;
         bool stop = false;
-        for (int t = blockIdx.x; t < total && !stop; t += gridDim.x, ++local) {
+        while (!stop) {
+            if (!mbar_wait_bounded(&qfull[q], qph, abort_flag)) break;
+            const int t = fifo[q];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&qempty[q]);
+            if (++q == kFifo) {
+                q = 0;
+                qph ^= 1u;
+            }
+            if (t < 0) break;
+            const Tile tl = decode(p, t);
+            const int nst = tile_stages(tl);
+            if (tl.kind == TILE_P) {  // skip the P tile's stages
+                s += nst;
+                ph ^= (uint32_t)((s / kGStages) & 1);
+                s %= kGStages;
+                continue;
+            }
             const int buf = local & 1;
             const uint32_t tph = (uint32_t)((local >> 1) & 1);
             if (!mbar_wait_bounded(&tempty[buf], tph ^ 1u, abort_flag)) break;
             tc_fence_after();
             const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
-            for (int kb = 0; kb < kb_count; ++kb) {
+            for (int kb = 0; kb < nst; ++kb) {
                 if (!mbar_wait_bounded(&full[s], ph, abort_flag)) {
                     stop = true;
                     break;
@@ -274,6 +524,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             if (lane == 0) umma_commit(&tfull[buf]);  // accumulator ready for the epilogue
             __syncwarp();
+            ++local;
         }
         // every MMA this thread issued has completed before TMEM is released
         if (lane == 0) umma_commit(done);
@@ -281,22 +532,143 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         mbar_wait_bounded(done, 0u, nullptr);
     } else {
         // ---------------- epilogue warps 2..5: TMEM lane quarter = warp % 4
-        const int q = warp & 3;
-        const int r_in_tile = q * 32 + lane;
+        const int qd = warp & 3;
+        const int et = threadIdx.x - 64;  // 0..127
+        const int ew = et >> 5;
+        const int half = p.hd / 2;
+        int s = 0;
+        uint32_t ph = 0;
+        int q = 0;
+        uint32_t qph = 0;
         int local = 0;
-        for (int t = blockIdx.x; t < total; t += gridDim.x, ++local) {
-            const int m = t % p.m_tiles, n = t / p.m_tiles;
+        int rbuf = 0;  // reduction scratch buffer (alternates per row)
+        if (!p.plain)
+            for (int j = et; j < half; j += kEpiThreads)
+                inv_freq[j] = pow(p.rope_base, -2.0 * (double)j / (double)p.hd);
+        named_sync(1, kEpiThreads);
+        while (true) {
+            if (!mbar_wait_bounded(&qfull[q], qph, abort_flag)) break;
+            const int t = fifo[q];
+            named_sync(1, kEpiThreads);  // every epilogue thread has read the slot
+            if (et == 0) mbar_arrive(&qempty[q]);
+            if (++q == kFifo) {
+                q = 0;
+                qph ^= 1u;
+            }
+            if (t < 0) break;
+            const Tile tl = decode(p, t);
+            const int nst = tile_stages(tl);
+            const int64_t crow0 = (int64_t)tl.c * p.chunk;  // prompt row of the chunk's row 0
+            const int64_t rows_c = p.plain ? p.M : min(p.chunk, p.R - crow0);
+            if (tl.kind == TILE_P) {
+                // ---- prologue of rows m*128 .. : the lanes' buffers are free once the
+                // chunks that used them before are done with them
+                const int lane_c = tl.c % p.lanes, slot_r = tl.c % (p.lanes + 1);
+                bool ok = true;
+                if (et == 0) {
+                    const int ca = tl.c - p.lanes, cr = tl.c - p.lanes - 1;
+                    if (ca >= 0)
+                        ok = wait_counter(counter(p, TILE_F, ca, tl.m),
+                                          (uint32_t)((ca / kCtrSlots + 1) * p.nf), abort_flag);
+                    if (ok && cr >= 0)
+                        ok = wait_counter(counter(p, TILE_V, cr, tl.m),
+                                          (uint32_t)((cr / kCtrSlots + 1) * p.nv), abort_flag);
+                }
+                named_sync(1, kEpiThreads);
+                const int rows = (int)min((int64_t)BM, rows_c - (int64_t)tl.m * BM);
+                const int h = p.h, pieces = h / 8;  // 16-byte pieces of a row
+                const uint32_t rb = 2u * (uint32_t)h;
+                for (int st = 0; st < nst; ++st) {
+                    const bool got = mbar_wait_bounded(&full[s], ph, abort_flag);
+                    const int r0 = st * p.rows_per_pstage;
+                    const int nr = min(p.rows_per_pstage, rows - r0);
+                    for (int i = 0; i < nr && got; ++i) {
+                        const int tok = stage_tok[s * kMaxRowsPerPStage + i];
+                        const uint8_t* erow = stages + (size_t)s * kGStageBytes + (size_t)i * 2u * rb;
+                        const uint8_t* xrow = erow + rb;
+                        float se = 0.f, sx = 0.f;
+                        for (int j = et; j < pieces; j += kEpiThreads) {
+                            if (tok >= 0) se += sumsq8(lds128(erow + 16 * j));
+                            sx += sumsq8(lds128(xrow + 16 * j));
+                        }
+#pragma unroll
+                        for (int o = 16; o; o >>= 1) {
+                            se += __shfl_xor_sync(0xffffffffu, se, o);
+                            sx += __shfl_xor_sync(0xffffffffu, sx, o);
+                        }
+                        float* rr = red + rbuf * 8;
+                        if (lane == 0) {
+                            rr[ew * 2] = se;
+                            rr[ew * 2 + 1] = sx;
+                        }
+                        named_sync(1, kEpiThreads);
+                        se = (rr[0] + rr[2]) + (rr[4] + rr[6]);
+                        sx = (rr[1] + rr[3]) + (rr[5] + rr[7]);
+                        rbuf ^= 1;
+                        const float inv_e = 1.0f / sqrtf(se / (float)h + p.eps);
+                        const float inv_x = 1.0f / sqrtf(sx / (float)h + p.eps);
+                        uint16_t* crow = p.concat[lane_c] + ((int64_t)tl.m * BM + r0 + i) * 2 * h;
+                        for (int j = et; j < pieces; j += kEpiThreads) {
+                            const uint4 e = tok >= 0 ? lds128(erow + 16 * j) : make_uint4(0, 0, 0, 0);
+                            const uint4 we = __ldg(reinterpret_cast<const uint4*>(p.w_ne) + j);
+                            const uint4 wh = __ldg(reinterpret_cast<const uint4*>(p.w_nh) + j);
+                            reinterpret_cast<uint4*>(crow)[j] = norm8(e, inv_e, we);
+                            reinterpret_cast<uint4*>(crow + h)[j] = norm8(lds128(xrow + 16 * j), inv_x, wh);
+                        }
+                    }
+                    named_sync(1, kEpiThreads);  // everyone is done with the stage
+                    if (et == 0) mbar_arrive(&empty[s]);
+                    if (++s == kGStages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                // RoPE table of the rows (cos, sin of pos * base^(-2j / hd), in double)
+                float2* cs = p.rope[slot_r] + (int64_t)tl.m * BM * half;
+                for (int k = et; k < rows * half; k += kEpiThreads) {
+                    const int r = k / half, j = k - r * half;
+                    const double th = (double)p.rope_pos[crow0 + (int64_t)tl.m * BM + r] * inv_freq[j];
+                    double sn, cn;
+                    sincos(th, &sn, &cn);
+                    cs[k] = make_float2((float)cn, (float)sn);
+                }
+                fence_proxy_async_global();  // the concat rows are read by TMA
+                named_sync(1, kEpiThreads);
+                if (et == 0 && !*abort_flag) counter_release_add(counter(p, TILE_P, tl.c, tl.m), 1u);
+                continue;
+            }
+            // ---- GEMM tile: its stages are the MMA warp's
+            s += nst;
+            ph ^= (uint32_t)((s / kGStages) & 1);
+            s %= kGStages;
             const int buf = local & 1;
             const uint32_t tph = (uint32_t)((local >> 1) & 1);
-            const bool ok = mbar_wait_bounded(&tfull[buf], tph, abort_flag);
+            ++local;
+            bool ok = mbar_wait_bounded(&tfull[buf], tph, abort_flag);
+            // F writes the chunk lane's fc output rows: free once the chunk that used the
+            // lane before has run its k/v tiles of these rows; V reads the RoPE rows
+            if (et == 0 && ok && !p.plain) {
+                if (tl.kind == TILE_F && tl.c >= p.lanes) {
+                    const int ca = tl.c - p.lanes;
+                    ok = wait_counter(counter(p, TILE_V, ca, tl.m),
+                                      (uint32_t)((ca / kCtrSlots + 1) * p.nv), abort_flag);
+                } else if (tl.kind == TILE_V) {
+                    ok = wait_counter(counter(p, TILE_P, tl.c, tl.m),
+                                      (uint32_t)(tl.c / kCtrSlots + 1), abort_flag);
+                }
+            }
+            named_sync(1, kEpiThreads);
+            ok = ok && !*abort_flag;
             tc_fence_after();
-            const int row = m * BM + r_in_tile;  // row of A / of this chunk
-            const bool row_ok = ok && row < p.M;
-            const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN);
-            if (EPI == 0) {
-                for (int c = 0; c < BN / 32; ++c) {
+            const int row = tl.m * BM + qd * 32 + lane;  // row of the chunk (of A)
+            const bool row_ok = ok && row < rows_c;
+            const uint32_t tb = tmem_base + ((uint32_t)(qd * 32) << 16) + (uint32_t)(buf * BN);
+            if (tl.kind == TILE_F) {
+                uint16_t* C = p.plain ? p.C : p.y[tl.c % p.lanes];
+                const int64_t ldc = p.plain ? p.N : p.h;
+                for (int cc = 0; cc < BN / 32; ++cc) {
                     uint32_t v[32];
-                    tmem_ld32(tb + c * 32, v);
+                    tmem_ld32(tb + cc * 32, v);
                     tmem_ld_wait();
                     if (row_ok) {
                         uint32_t pk[16];
@@ -304,27 +676,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         for (int i = 0; i < 16; ++i)
                             pk[i] = (uint32_t)f32_to_bf16(__uint_as_float(v[2 * i])) |
                                     ((uint32_t)f32_to_bf16(__uint_as_float(v[2 * i + 1])) << 16);
-                        uint4* dst = reinterpret_cast<uint4*>(p.C + (int64_t)row * p.ldc + n * BN + c * 32);
+                        uint4* dst = reinterpret_cast<uint4*>(C + (int64_t)row * ldc + tl.n * BN + cc * 32);
 #pragma unroll
                         for (int i = 0; i < 4; ++i)
                             dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
                     }
                 }
+                if (!p.plain) fence_proxy_async_global();  // read by the k/v tiles' TMA
             } else {
-                const int kvd = p.nkv * p.hd;
-                const int col0 = n * BN;
+                const int col0 = tl.n * BN;
                 const bool is_v = col0 >= kvd;
-                const int half = p.hd / 2;
                 int64_t slot = -1;
                 if (row_ok) {
-                    slot = cache_slot(p, p.row0 + row);
+                    slot = cache_slot(p, crow0 + row);
                     if (slot < 0) raise_flag(p.dev_err, DEVFLAG_BAD_SLOT);
                 }
                 uint8_t* cache = is_v ? p.v_cache : p.k_cache;
                 const float scale = is_v ? p.v_scale : p.k_scale;
+                const float2* cs = p.rope[tl.c % (p.lanes + 1)] + (int64_t)row * half;
                 for (int h0 = 0; h0 < BN; h0 += p.hd) {
-                    const int head = ((is_v ? col0 - kvd : col0) + h0) / p.hd;
-                    uint8_t* hdst = cache + (slot * p.nkv + head) * (int64_t)p.hd;
+                    const int head_i = ((is_v ? col0 - kvd : col0) + h0) / p.hd;
+                    uint8_t* hdst = cache + (slot * p.nkv + head_i) * (int64_t)p.hd;
                     for (int j0 = 0; j0 < half; j0 += 32) {
                         uint32_t a[32], b[32];
                         tmem_ld32(tb + h0 + j0, a);
@@ -336,7 +708,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             lo[i] = round_bf16(__uint_as_float(a[i]));
                             hi[i] = round_bf16(__uint_as_float(b[i]));
                         }
-                        if (!is_v && row_ok) rope32(lo, hi, p.rope_cs + (int64_t)row * half + j0);
+                        if (!is_v && row_ok) rope32(lo, hi, cs + j0);
                         if (row_ok && slot >= 0) {
                             store_codes32(hdst + j0, lo, scale);
                             store_codes32(hdst + half + j0, hi, scale);
@@ -345,8 +717,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
             }
             tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[buf]);
+            named_sync(1, kEpiThreads);  // the accumulator is read, every store issued
+            if (et == 0) {
+                mbar_arrive(&tempty[buf]);
+                if (!p.plain && !*abort_flag)
+                    counter_release_add(counter(p, tl.kind, tl.c, tl.m), 1u);
+            }
         }
     }
     __syncthreads();
@@ -358,9 +734,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // Stage check: bf16 k' (already rotated) and v rows -> E4M3 codes in the paged cache,
-// through the same encode and slot code the GEMM epilogue uses. One warp per row.
+// through the same encode and slot code the k/v epilogue uses. One warp per row.
 __global__ void kv_write_kernel(const uint16_t* __restrict__ k_rot, const uint16_t* __restrict__ v,
-                                int64_t R, const GemmParams p) {
+                                int64_t R, const PrefillParams p) {
     const int64_t r = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (r >= R) return;
@@ -419,186 +795,165 @@ cudaError_t make_operand_map(CUtensorMap* m, const void* base, int64_t rows, int
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-int sm_count_now() {
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    return sms;
-}
-
-template <int EPI>
-cudaError_t launch_gemm(const GemmParams& p0, const CUtensorMap& ma, const CUtensorMap& mb0,
-                        const CUtensorMap& mb1, cudaStream_t s) {
-    GemmParams p = p0;
-    p.m_tiles = (p.M + BM - 1) / BM;
-    p.n_tiles = p.N / BN;
-    const int total = p.m_tiles * p.n_tiles;
-    if (total < 1) return cudaSuccess;
-    auto kern = gemm_kernel<EPI>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+cudaError_t launch(const PrefillParams& p, const Maps& maps, cudaStream_t s) {
+    if (p.total < 1) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kGemmSmem);
     if (e != cudaSuccess) return e;
-    int grid = sm_count_now();
-    if (grid > total) grid = total;
-    kern<<<grid, kGemmThreads, kGemmSmem, s>>>(p, ma, mb0, mb1);
+    int dev = 0, sms = 148;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return e;
+    int64_t grid = sms;
+    if (grid > p.total) grid = p.total;
+    prefill_kernel<<<(unsigned)grid, kGemmThreads, kGemmSmem, s>>>(p, maps);
     return cudaGetLastError();
 }
 
+// Workspace layout: a counter header, then `lanes` x (concat rows, fc output rows), then
+// lanes + 1 RoPE tables.
+constexpr size_t kCtrHeader = 256;  // tile counter (and room), before the done counters
+size_t up1k(size_t b) { return (b + 1023) & ~(size_t)1023; }
+size_t header_bytes(int64_t chunk_rows) {
+    const size_t mt = (size_t)((chunk_rows + BM - 1) / BM);
+    return up1k(kCtrHeader + 3 * kCtrSlots * mt * sizeof(uint32_t));
+}
+size_t concat_bytes(int64_t c, int32_t h) { return up1k((size_t)c * 2 * h * 2); }
+size_t y_bytes(int64_t c, int32_t h) { return up1k((size_t)c * h * 2); }
+size_t rope_bytes(int64_t c, int32_t hd) { return up1k((size_t)c * (hd / 2) * sizeof(float2)); }
+
 }  // namespace
+
+size_t prefill_ws_bytes_lanes(int64_t chunk_rows, int32_t h, int32_t hd, int lanes) {
+    return header_bytes(chunk_rows) +
+           (size_t)lanes * (concat_bytes(chunk_rows, h) + y_bytes(chunk_rows, h)) +
+           (size_t)(lanes + 1) * rope_bytes(chunk_rows, hd);
+}
 
 size_t prefill_lane_bytes(int64_t chunk_rows, int32_t h, int32_t nkv, int32_t hd) {
     (void)nkv;
-    auto up = [](size_t b) { return (b + 1023) & ~(size_t)1023; };
-    return up((size_t)chunk_rows * 2 * h * 2) + up((size_t)chunk_rows * h * 2) +
-           up((size_t)chunk_rows * (hd / 2) * sizeof(float2));
+    return prefill_ws_bytes_lanes(chunk_rows, h, hd, 1);  // the minimum: one lane
 }
 
 size_t prefill_ws_bytes(int64_t chunk_rows, int32_t h, int32_t nkv, int32_t hd) {
-    return 2 * prefill_lane_bytes(chunk_rows, h, nkv, hd);
+    (void)nkv;
+    // twice the one-lane minimum (which covers the two-lane layout), so that half of the
+    // full size is always a valid one-lane workspace
+    return 2 * prefill_ws_bytes_lanes(chunk_rows, h, hd, 1);
 }
 
-namespace {
-
-// Two streams per device on which alternate chunks run: a chunk's fc GEMM (320 tiles of
-// 128 x 256 at 2,048 rows x hidden 5,120) ends in a partial wave on 148 SMs, and the k/v
-// GEMM and the prologue leave SMs idle too; chunks are independent, so the next chunk's
-// kernels fill those SMs. Created on first use and kept for the life of the process.
-struct ChunkLanes {
-    cudaStream_t s[2] = {nullptr, nullptr};
-    cudaEvent_t fork = nullptr, join[2] = {nullptr, nullptr};
-};
-constexpr int kMaxLaneDevices = 64;
-ChunkLanes g_lanes[kMaxLaneDevices];
-std::mutex g_lane_mutex;  // held while a call forks and joins (events are shared)
-
-cudaError_t lanes_for_current_device(ChunkLanes** out) {
-    int dev = 0;
-    cudaError_t e;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxLaneDevices) return cudaErrorInvalidDevice;
-    ChunkLanes& L = g_lanes[dev];
-    if (!L.fork) {
-        for (int i = 0; i < 2; ++i) {
-            if ((e = cudaStreamCreateWithFlags(&L.s[i], cudaStreamNonBlocking)) != cudaSuccess) return e;
-            if ((e = cudaEventCreateWithFlags(&L.join[i], cudaEventDisableTiming)) != cudaSuccess)
-                return e;
-        }
-        if ((e = cudaEventCreateWithFlags(&L.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
-    }
-    *out = &L;
-    return cudaSuccess;
-}
-
-// One chunk: prologue (gather, norms, concat, RoPE table), fc GEMM, k/v GEMM with the
-// RoPE + E4M3 + paged-write epilogue, using one lane of the workspace.
-cudaError_t prefill_chunk(const PrefillArgs& a, int64_t r0, int rows, uint8_t* lane,
-                          const CUtensorMap& m_fc, const CUtensorMap& m_wk, const CUtensorMap& m_wv,
-                          cudaStream_t s) {
-    auto up = [](size_t b) { return (b + 1023) & ~(size_t)1023; };
-    uint16_t* cbuf = reinterpret_cast<uint16_t*>(lane);
-    uint16_t* ybuf = reinterpret_cast<uint16_t*>(lane + up((size_t)a.chunk_rows * 2 * a.h * 2));
-    float2* csbuf = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(ybuf) +
-                                              up((size_t)a.chunk_rows * a.h * 2));
-    const int kvd = a.nkv * a.hd;
-    cudaError_t e;
-    prefill_prologue_kernel<<<rows, kPrologueThreads, 0, s>>>(
-        a.embed, a.vocab, a.tokens, a.hidden, a.h, a.w_norm_embed, a.w_norm_hidden, a.eps,
-        a.rope_pos, a.rope_base, a.hd, r0, cbuf, csbuf, a.dev_err);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    CUtensorMap m_c, m_y;
-    if ((e = make_operand_map(&m_c, cbuf, rows, 2 * (int64_t)a.h, BM)) != cudaSuccess) return e;
-    if ((e = make_operand_map(&m_y, ybuf, rows, a.h, BM)) != cudaSuccess) return e;
-    GemmParams g1{};
-    g1.M = rows;
-    g1.N = a.h;
-    g1.K = 2 * a.h;
-    g1.C = ybuf;
-    g1.ldc = a.h;
-    g1.dev_err = a.dev_err;
-    if ((e = launch_gemm<0>(g1, m_c, m_fc, m_fc, s)) != cudaSuccess) return e;
-    GemmParams g2{};
-    g2.M = rows;
-    g2.N = 2 * kvd;
-    g2.K = a.h;
-    g2.nkv = a.nkv;
-    g2.hd = a.hd;
-    g2.rope_cs = csbuf;
-    g2.row0 = r0;
-    g2.cache_start = a.cache_start;
-    g2.block_table = a.block_table;
-    g2.n_table = a.n_table;
-    g2.block_size = a.block_size;
-    g2.num_blocks = a.num_blocks;
-    g2.k_cache = a.k_cache;
-    g2.v_cache = a.v_cache;
-    g2.k_scale = a.k_scale;
-    g2.v_scale = a.v_scale;
-    g2.dev_err = a.dev_err;
-    return launch_gemm<1>(g2, m_y, m_wk, m_wv, s);
-}
-
-}  // namespace
+int prefill_max_hidden() { return kGStageBytes / 4; }  // one P row (two bf16 rows) per stage
 
 cudaError_t prefill_launch(const PrefillArgs& a, cudaStream_t s) {
     const int kvd = a.nkv * a.hd;
-    CUtensorMap m_fc, m_wk, m_wv;
+    PrefillParams p{};
+    p.embed = a.embed;
+    p.vocab = a.vocab;
+    p.tokens = a.tokens;
+    p.hidden = a.hidden;
+    p.R = a.R;
+    p.h = a.h;
+    p.w_ne = a.w_norm_embed;
+    p.w_nh = a.w_norm_hidden;
+    p.eps = a.eps;
+    p.nkv = a.nkv;
+    p.hd = a.hd;
+    p.rope_base = a.rope_base;
+    p.rope_pos = a.rope_pos;
+    p.cache_start = a.cache_start;
+    p.block_table = a.block_table;
+    p.n_table = a.n_table;
+    p.block_size = a.block_size;
+    p.num_blocks = a.num_blocks;
+    p.k_cache = a.k_cache;
+    p.v_cache = a.v_cache;
+    p.k_scale = a.k_scale;
+    p.v_scale = a.v_scale;
+    p.dev_err = a.dev_err;
+    p.chunk = a.chunk_rows;
+    p.n_chunks = (int)((a.R + a.chunk_rows - 1) / a.chunk_rows);
+    p.mt_full = (int)((a.chunk_rows + BM - 1) / BM);
+    const int64_t last_rows = a.R - (int64_t)(p.n_chunks - 1) * a.chunk_rows;
+    p.mt_last = (int)((last_rows + BM - 1) / BM);
+    p.nf = a.h / BN;
+    p.nv = 2 * kvd / BN;
+    const int64_t full_p_f = (int64_t)p.mt_full * (1 + p.nf);
+    if (p.n_chunks == 1) {
+        p.b0 = (int64_t)p.mt_last * (1 + p.nf);
+        p.n_mid = 0;
+        p.s_mid = 1;
+        p.b_last = 0;
+        p.total = p.b0 + (int64_t)p.mt_last * p.nv;
+    } else {
+        p.b0 = full_p_f;
+        p.s_mid = full_p_f + (int64_t)p.mt_full * p.nv;
+        p.n_mid = p.n_chunks - 2;
+        p.b_last = (int64_t)p.mt_last * (1 + p.nf) + (int64_t)p.mt_full * p.nv;
+        p.total = p.b0 + p.n_mid * p.s_mid + p.b_last + (int64_t)p.mt_last * p.nv;
+    }
+    p.lanes = (a.R > a.chunk_rows && a.ws_bytes >= prefill_ws_bytes_lanes(a.chunk_rows, a.h, a.hd, 2))
+                  ? 2 : 1;
+    int rps = kGStageBytes / (4 * a.h);
+    p.rows_per_pstage = rps > kMaxRowsPerPStage ? kMaxRowsPerPStage : rps;
+    if (p.rows_per_pstage < 1 || a.hd / 2 > 128) return cudaErrorInvalidValue;
+    // workspace carving
+    uint8_t* w = static_cast<uint8_t*>(a.ws);
+    p.ctr = reinterpret_cast<uint32_t*>(w);
+    size_t off = header_bytes(a.chunk_rows);
+    for (int l = 0; l < p.lanes; ++l) {
+        p.concat[l] = reinterpret_cast<uint16_t*>(w + off);
+        off += concat_bytes(a.chunk_rows, a.h);
+        p.y[l] = reinterpret_cast<uint16_t*>(w + off);
+        off += y_bytes(a.chunk_rows, a.h);
+    }
+    for (int l = 0; l < p.lanes + 1; ++l) {
+        p.rope[l] = reinterpret_cast<float2*>(w + off);
+        off += rope_bytes(a.chunk_rows, a.hd);
+    }
+    Maps maps{};
     cudaError_t e;
-    if ((e = make_operand_map(&m_fc, a.fc, a.h, 2 * (int64_t)a.h, BN)) != cudaSuccess) return e;
-    if ((e = make_operand_map(&m_wk, a.wk, kvd, a.h, BN)) != cudaSuccess) return e;
-    if ((e = make_operand_map(&m_wv, a.wv, kvd, a.h, BN)) != cudaSuccess) return e;
-    const size_t lane_bytes = prefill_lane_bytes(a.chunk_rows, a.h, a.nkv, a.hd);
-    uint8_t* ws = static_cast<uint8_t*>(a.ws);
-    const bool two = a.R > a.chunk_rows && a.ws_bytes >= 2 * lane_bytes;
-    if (!two) {  // one lane: the chunks in order on the caller's stream
-        for (int64_t r0 = 0; r0 < a.R; r0 += a.chunk_rows) {
-            const int rows = (int)((a.R - r0) < a.chunk_rows ? (a.R - r0) : a.chunk_rows);
-            if ((e = prefill_chunk(a, r0, rows, ws, m_fc, m_wk, m_wv, s)) != cudaSuccess) return e;
-        }
-        return cudaSuccess;
+    for (int l = 0; l < p.lanes; ++l) {
+        if ((e = make_operand_map(&maps.a_concat[l], p.concat[l], a.chunk_rows, 2 * (int64_t)a.h, BM)) !=
+            cudaSuccess)
+            return e;
+        if ((e = make_operand_map(&maps.a_y[l], p.y[l], a.chunk_rows, a.h, BM)) != cudaSuccess) return e;
     }
-    // two lanes: chunk i runs on lane stream i % 2 with workspace lane i % 2, forked from
-    // and joined back into the caller's stream (the same pattern works under capture)
-    std::lock_guard<std::mutex> lock(g_lane_mutex);
-    ChunkLanes* L = nullptr;
-    if ((e = lanes_for_current_device(&L)) != cudaSuccess) return e;
-    if ((e = cudaEventRecord(L->fork, s)) != cudaSuccess) return e;
-    for (int i = 0; i < 2; ++i)
-        if ((e = cudaStreamWaitEvent(L->s[i], L->fork, 0)) != cudaSuccess) return e;
-    cudaError_t err = cudaSuccess;
-    int64_t i = 0;
-    for (int64_t r0 = 0; r0 < a.R && err == cudaSuccess; r0 += a.chunk_rows, ++i) {
-        const int rows = (int)((a.R - r0) < a.chunk_rows ? (a.R - r0) : a.chunk_rows);
-        err = prefill_chunk(a, r0, rows, ws + (size_t)(i & 1) * lane_bytes, m_fc, m_wk, m_wv,
-                            L->s[i & 1]);
-    }
-    // join even after a failed launch, so the caller's stream stays ordered after both lanes
-    for (int j = 0; j < 2; ++j) {
-        if ((e = cudaEventRecord(L->join[j], L->s[j])) != cudaSuccess) return e;
-        if ((e = cudaStreamWaitEvent(s, L->join[j], 0)) != cudaSuccess) return e;
-    }
-    return err;
+    if ((e = make_operand_map(&maps.b_fc, a.fc, a.h, 2 * (int64_t)a.h, BN)) != cudaSuccess) return e;
+    if ((e = make_operand_map(&maps.b_wk, a.wk, kvd, a.h, BN)) != cudaSuccess) return e;
+    if ((e = make_operand_map(&maps.b_wv, a.wv, kvd, a.h, BN)) != cudaSuccess) return e;
+    // the counters start at zero on every call (a memset node in the caller's stream)
+    if ((e = cudaMemsetAsync(p.ctr, 0, header_bytes(a.chunk_rows), s)) != cudaSuccess) return e;
+    return launch(p, maps, s);
 }
 
 cudaError_t gemm_bf16_launch(const uint16_t* A, const uint16_t* B, uint16_t* C, int M, int N,
                              int K, int32_t* dev_err, cudaStream_t s) {
-    CUtensorMap ma, mb;
+    PrefillParams p{};
+    p.plain = 1;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.C = C;
+    p.R = M;
+    p.chunk = M;
+    p.n_chunks = 1;
+    p.lanes = 1;
+    p.nf = N / BN;
+    p.total = (int64_t)((M + BM - 1) / BM) * (N / BN);
+    p.dev_err = dev_err;
+    p.rows_per_pstage = 1;
+    Maps maps{};
     cudaError_t e;
-    if ((e = make_operand_map(&ma, A, M, K, BM)) != cudaSuccess) return e;
-    if ((e = make_operand_map(&mb, B, N, K, BN)) != cudaSuccess) return e;
-    GemmParams g{};
-    g.M = M;
-    g.N = N;
-    g.K = K;
-    g.C = C;
-    g.ldc = N;
-    g.dev_err = dev_err;
-    return launch_gemm<0>(g, ma, mb, mb, s);
+    if ((e = make_operand_map(&maps.a_concat[0], A, M, K, BM)) != cudaSuccess) return e;
+    if ((e = make_operand_map(&maps.b_fc, B, N, K, BN)) != cudaSuccess) return e;
+    return launch(p, maps, s);
 }
 
 cudaError_t kv_write_launch(const uint16_t* k_rot, const uint16_t* v, int64_t R, int nkv, int hd,
                             int64_t cache_start, const int32_t* block_table, int64_t n_table,
                             int block_size, int64_t num_blocks, uint8_t* k_cache, uint8_t* v_cache,
                             float k_scale, float v_scale, int32_t* dev_err, cudaStream_t s) {
-    GemmParams p{};
+    PrefillParams p{};
     p.nkv = nkv;
     p.hd = hd;
     p.cache_start = cache_start;

@@ -63,6 +63,11 @@ constexpr int kMaxGrid = 1024;
 constexpr int kMaxStages = 12;
 constexpr int kMaxSegs = 32;  // 128-byte segments of a row per stage (box of 16 rows x 4 KB)
 constexpr int kSmemLimit = 227 * 1024;
+// Gathered (masked) sweep: rows claimed per hand-out (8 mask words per input), the
+// producer's queue of allowed rows, and the shared-memory ints it adds.
+constexpr int kGatherRows = 256;
+constexpr int kGatherQueue = 64;  // a power of two above 15 + 32
+constexpr int kGatherInts = kGatherQueue + kMaxStages * 16 + 2 * 16;
 
 // Warp roles: CW compute warps, then one reducer warp, then one producer warp.
 // M <= 8 uses 16 compute warps; M > 8 uses 8, which leaves shared memory for the
@@ -100,8 +105,10 @@ template <> struct Fmt<2> { static constexpr int V = 32; };
 
 __host__ __device__ inline int code_stage_bytes(int segs) { return kTileRows * 128 * segs; }
 __host__ __device__ inline int scale_stage_bytes(int segs) { return kTileRows * 16 * segs; }
-__host__ __device__ inline int stage_bytes_for(int fmt, int segs) {
-    int b = code_stage_bytes(segs) + (fmt == 2 ? scale_stage_bytes(segs) : 0);
+__host__ __device__ inline int stage_bytes_for(int fmt, int segs, bool gather = false) {
+    // a gathered stage skews its 16 rows by 16 bytes each
+    int b = code_stage_bytes(segs) + (gather ? kTileRows * 16 : 0) +
+            (fmt == 2 ? scale_stage_bytes(segs) : 0);
     return (b + 1023) & ~1023;
 }
 
@@ -162,35 +169,39 @@ __device__ __forceinline__ bool mask_allows(const SweepParams& p, int m, int64_t
     return (bits >> (t & 31)) & 1u;
 }
 
-__device__ __forceinline__ bool row_needed(const SweepParams& p, int64_t row) {
-    if (row >= p.n) return false;
-    if (!p.mask) return true;
-    for (int m = 0; m < p.M; ++m)
-        if (mask_allows(p, m, row)) return true;
-    return false;
-}
-
-// A tile's 16 rows are 16 consecutive mask bits of each input: lane m < M loads input m's
-// one or two words (issued early; tile_mask_need consumes them later).
-__device__ __forceinline__ void tile_mask_load(const SweepParams& p, int64_t tile, int lane,
-                                               uint32_t& w0, uint32_t& w1) {
-    w0 = w1 = 0u;
-    if (lane >= p.M) return;
-    const int64_t t0 = tile * kTileRows + p.row_offset;
+// Gathered sweep: the mask words of a claimed range of kGatherRows rows. Lane l loads
+// word (l % 8) of the range for inputs l / 8 and l / 8 + 4 (two words each, since a vocab
+// shard's rows start at any token), issued early; gather_union consumes them.
+__device__ __forceinline__ void gather_mask_load(const SweepParams& p, int64_t claim, int lane,
+                                                 uint32_t (&w)[4]) {
+    const int64_t t0 = claim * kGatherRows + (lane & 7) * 32 + p.row_offset;
     const int64_t wi = t0 >> 5;
-    const int32_t* row = p.mask + (int64_t)lane * p.mask_stride;
-    if (wi < p.mask_words) w0 = (uint32_t)__ldg(row + wi);
-    if ((t0 & 31) > 16 && wi + 1 < p.mask_words) w1 = (uint32_t)__ldg(row + wi + 1);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const int m = (lane >> 3) + 4 * j;
+        w[2 * j] = w[2 * j + 1] = 0u;
+        if (m >= p.M) continue;
+        const int32_t* row = p.mask + (int64_t)m * p.mask_stride;
+        if (wi < p.mask_words) w[2 * j] = (uint32_t)__ldg(row + wi);
+        if ((t0 & 31) != 0 && wi + 1 < p.mask_words) w[2 * j + 1] = (uint32_t)__ldg(row + wi + 1);
+    }
 }
 
-// True when some row of the tile (below n) is allowed for some input (whole warp).
-__device__ __forceinline__ bool tile_mask_need(const SweepParams& p, int64_t tile, int lane,
-                                               uint32_t w0, uint32_t w1) {
-    const int64_t t0 = tile * kTileRows + p.row_offset;
-    uint32_t bits = (uint32_t)((((uint64_t)w1 << 32) | w0) >> (t0 & 31)) & 0xFFFFu;
-    const int64_t rows = p.n - tile * kTileRows;
-    if (rows < kTileRows) bits &= (1u << (rows > 0 ? rows : 0)) - 1u;
-    return __any_sync(0xffffffffu, lane < p.M && bits != 0u);
+// The OR over the inputs of the allowed bits of rows claim * kGatherRows + 32 j + [0, 32),
+// rows at or past n cleared; lane j (j < 8) returns word j (whole warp).
+__device__ __forceinline__ uint32_t gather_union(const SweepParams& p, int64_t claim, int lane,
+                                                 const uint32_t (&w)[4]) {
+    const int64_t row0 = claim * kGatherRows + (lane & 7) * 32;
+    const int sh = (int)((row0 + p.row_offset) & 31);
+    uint32_t v = 0u;
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+        v |= (uint32_t)((((uint64_t)w[2 * j + 1] << 32) | w[2 * j]) >> sh);
+    v |= __shfl_xor_sync(0xffffffffu, v, 8);
+    v |= __shfl_xor_sync(0xffffffffu, v, 16);
+    const int64_t rows = p.n - row0;
+    if (rows < 32) v &= rows > 0 ? (1u << rows) - 1u : 0u;
+    return v;
 }
 
 // Reductions over the CW compute warps (named barrier 1).
@@ -354,18 +365,19 @@ __device__ bool stage_x_f16_direct(const SweepParams& p, uint16_t* xs, int* xexp
     return true;
 }
 
-// One slab: per lane 16 B of codes of table rows r0 (at cw) and r0 + 8 (at cw + 1 KB,
-// the next 8-row swizzle atom), K elements [e0, e0 + V) for lane c, against the staged
+// One slab: per lane 16 B of codes of table rows r0 (at cw) and r0 + 8 (at cw + r8: 1 KB,
+// the next 8-row swizzle atom, in a tensor-box stage; eight row pitches in a gathered
+// stage), K elements [e0, e0 + V) for lane c, against the staged
 // inputs at x0 (input row g) and x1 (input row g + 8). For NVFP4, sw points at the
 // lane's two block scales of row r0 and sw + spitch8 at those of row r0 + 8. The
 // accumulator set (mma index & 1) alternates to split the dependence chain.
 template <int FMT, int NT>
-__device__ __forceinline__ void slab_mma(float (&acc)[2][NT][4], const uint8_t* cw,
+__device__ __forceinline__ void slab_mma(float (&acc)[2][NT][4], const uint8_t* cw, uint32_t r8,
                                          const uint8_t* sw, uint32_t spitch8,
                                          const uint16_t* x0, const uint16_t* x1, bool l0,
                                          bool l1) {
     const uint4 ra = lds128(cw);
-    const uint4 rb = lds128(cw + 1024);
+    const uint4 rb = lds128(cw + r8);
     const uint4 z = make_uint4(0, 0, 0, 0);
     if (FMT == 0) {
         const uint4 xa = l0 ? lds128(x0) : z;
@@ -444,10 +456,10 @@ __device__ __forceinline__ void slab_mma(float (&acc)[2][NT][4], const uint8_t* 
 // bytes of blocks 4(c % 2) .. 4(c % 2) + 3 of the slab, sw4 + spitch8 at row r0 + 8's.
 // xv: the lane's B registers; lanes that feed no input (lx false) keep them zero.
 __device__ __forceinline__ void slab_mma_blocks(float (&acc)[4], uint4 (&xv)[4], const uint8_t* cw,
-                                                const uint8_t* sw4, uint32_t spitch8,
+                                                uint32_t r8, const uint8_t* sw4, uint32_t spitch8,
                                                 const uint16_t* xp, bool lx) {
     const uint4 ra = lds128(cw);
-    const uint4 rb = lds128(cw + 1024);
+    const uint4 rb = lds128(cw + r8);
     const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w};
     const uint32_t wb[4] = {rb.x, rb.y, rb.z, rb.w};
     if (lx) {
@@ -561,7 +573,7 @@ __device__ void ticket_and_fold(const SweepParams& p, int lane, bool lp) {
     }
 }
 
-template <int FMT, int NT, int MODE, int BD>
+template <int FMT, int NT, int MODE, int BD, int G>
 __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
     sweep_kernel(const __grid_constant__ SweepParams p, const __grid_constant__ CUtensorMap map_codes,
                  const __grid_constant__ CUtensorMap map_scales) {
@@ -571,6 +583,7 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
     constexpr int RED_COLS = Roles<NT>::RED_COLS;
     constexpr int RED_WARP_FLOATS = kTileRows * RED_COLS;
     constexpr int REDUCER = CW, PRODUCER = CW + 1;
+    static_assert(G == 0 || MODE == 0, "the gathered sweep is an argmax sweep");
 
     extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
@@ -586,7 +599,13 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
     volatile int* red_tile = misc + 30;
     float* red = reinterpret_cast<float*>(misc + 32);  // [2][CW][16][RED_COLS]
     float* scratch = red + 2 * CW * RED_WARP_FLOATS;   // [32]
-    uint16_t* xs = reinterpret_cast<uint16_t*>(scratch + 32);
+    // gathered sweep: the producer's queue of allowed rows [256], the 16 table rows of
+    // each ring slot's tile [kMaxStages][16] (-1: an unused row slot), and those of each
+    // reducer buffer [2][16]
+    int* gq = reinterpret_cast<int*>(scratch + 32);
+    volatile int* slot_rows = gq + kGatherQueue;
+    volatile int* red_rows = slot_rows + kMaxStages * kTileRows;
+    uint16_t* xs = reinterpret_cast<uint16_t*>(scratch + 32 + (G ? kGatherInts : 0));
     // the ring starts on a 1 KB boundary of the shared window (the 128-byte swizzle atom)
     const uint32_t head_end = smem_u32(xs) + (uint32_t)p.M * (uint32_t)p.kpad * 2u;
     uint8_t* ring = smem + (((head_end + 1023u) & ~1023u) - smem_u32(smem));
@@ -599,10 +618,16 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
     const int slabs_per_stage = 2 * segs;
     const int NC = p.stages_per_tile;          // ceil(row segments / segs)
     const int M = p.M;
+    // a gathered stage holds row j's segments at j * gpitch (a 16-byte skew between rows
+    // keeps the compute warps' reads conflict-free without a swizzle); its block scales
+    // follow the 16 rows
+    const uint32_t gpitch = (uint32_t)segs * 128u + 16u;
+    const uint32_t code_area = G ? (uint32_t)kTileRows * gpitch : (uint32_t)code_stage_bytes(segs);
 
     // Tiles are handed out at run time (mode 0): CTA b starts with tile b, then takes
     // gridDim.x + (a counter in the workspace, post-incremented), so SMs that stream
     // faster take more tiles. Mode 1 (no workspace) splits the tiles evenly up front.
+    // The gathered sweep hands out ranges of kGatherRows table rows the same way.
     const int64_t T = p.num_tiles;
     const bool dyn = MODE == 0;
     const int64_t t_begin = dyn ? blockIdx.x : (T * blockIdx.x) / gridDim.x;
@@ -631,38 +656,37 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
         int64_t issued = 0;
         const uint32_t tx = code_stage_bytes(segs) + (FMT == 2 ? scale_stage_bytes(segs) : 0);
         bool stop = false;
-        // the NC stages of one tile, each tagged with the tile
-        auto issue_tile = [&](int64_t tile) {
-            for (int ch = 0; ch < NC; ++ch) {
-                if (!mbar_wait_bounded(&empty[slot], phase ^ 1u, abort_flag)) {
-                    stop = true;
-                    return;
+        if (!G) {
+            // the NC stages of one tile, each tagged with the tile
+            auto issue_tile = [&](int64_t tile) {
+                for (int ch = 0; ch < NC; ++ch) {
+                    if (!mbar_wait_bounded(&empty[slot], phase ^ 1u, abort_flag)) {
+                        stop = true;
+                        return;
+                    }
+                    if (lane == 0) {
+                        uint8_t* dst = ring + (size_t)slot * stage_bytes;
+                        slot_tile[slot] = (int)tile;
+                        mbar_arrive_expect_tx(&full[slot], tx);
+                        tma_load_3d(dst, &map_codes, 0, (int)(tile * kTileRows), ch * segs, &full[slot]);
+                        if (FMT == 2)
+                            tma_load_2d(dst + code_stage_bytes(segs), &map_scales, ch * 8 * segs,
+                                        (int)(tile * kTileRows), &full[slot]);
+                    }
+                    __syncwarp();
+                    ++issued;
+                    if (++slot == S) {
+                        slot = 0;
+                        phase ^= 1u;
+                    }
                 }
-                if (lane == 0) {
-                    uint8_t* dst = ring + (size_t)slot * stage_bytes;
-                    slot_tile[slot] = (int)tile;
-                    mbar_arrive_expect_tx(&full[slot], tx);
-                    tma_load_3d(dst, &map_codes, 0, (int)(tile * kTileRows), ch * segs, &full[slot]);
-                    if (FMT == 2)
-                        tma_load_2d(dst + code_stage_bytes(segs), &map_scales, ch * 8 * segs,
-                                    (int)(tile * kTileRows), &full[slot]);
-                }
-                __syncwarp();
-                ++issued;
-                if (++slot == S) {
-                    slot = 0;
-                    phase ^= 1u;
-                }
-            }
-        };
-        // the next tile is claimed one tile ahead, so the atomic's latency overlaps the
-        // waits for free ring slots
-        int64_t tile = t_begin;
-        int64_t pending = 0;
-        if (!p.mask) {
+            };
             // The first tile's stages read only the table, so they go out before waiting
-            // for the previous grid.
-            issue_tile(tile);
+            // for the previous grid. The next tile is claimed one tile ahead, so the
+            // atomic's latency overlaps the waits for free ring slots.
+            int64_t tile = t_begin;
+            int64_t pending = 0;
+            if (tile < t_end) issue_tile(tile);
             pdl_wait();
             if (dyn && lane == 0) pending = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
             while (!stop) {
@@ -672,31 +696,87 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
                 issue_tile(tile);
             }
         } else {
-            // With a mask (which the previous grid may write) everything waits for it. The
-            // mask words of the following tile are loaded while this tile's stages go out.
-            pdl_wait();
-            if (dyn && lane == 0) pending = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
-            uint32_t w0, w1;
-            tile_mask_load(p, tile, lane, w0, w1);
-            bool need = tile_mask_need(p, tile, lane, w0, w1);
-            while (tile < t_end && !stop) {
-                const int64_t tnext = dyn ? __shfl_sync(0xffffffffu, pending, 0) : tile + 1;
-                if (dyn && lane == 0 && tnext < t_end)
-                    pending = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
-                uint32_t n0 = 0u, n1 = 0u;
-                if (tnext < t_end) tile_mask_load(p, tnext, lane, n0, n1);
-                if (need) {
-                    issue_tile(tile);
-                } else if (MODE == 0 && p.out_logits) {
-                    // every row is masked out for every input: logits -inf, nothing to load
-                    const int64_t row = tile * kTileRows + (lane & 15);
-                    if (row < p.n)
-                        for (int col = lane >> 4; col < M; col += 2)
-                            p.out_logits[(int64_t)col * p.n + row] = 0xFF80u;
+            // Gathered sweep (a grammar mask): only rows that some input's mask allows are
+            // read. Each claimed range of kGatherRows rows is scanned (the OR of the
+            // inputs' mask words), its allowed rows join a queue in increasing order, and
+            // every 16 queued rows become one tile whose rows are fetched by one bulk copy
+            // each (their codes, plus for NVFP4 their block scales). The mask may be
+            // written by the previous grid, so everything waits for it.
+            const int row_segs = (int)(p.row_bytes / 128);
+            int qhead = 0, qtail = 0;  // queue positions (warp-uniform; entries mod 256)
+            int64_t vtile = 0;         // tiles issued (the tag a stage carries)
+            auto issue_gtile = [&](int cnt) {
+                const int myrow = lane < cnt ? gq[(qhead + lane) & (kGatherQueue - 1)] : -1;
+                for (int ch = 0; ch < NC && !stop; ++ch) {
+                    if (!mbar_wait_bounded(&empty[slot], phase ^ 1u, abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    const int seg0 = ch * segs;
+                    const int nseg = min(segs, row_segs - seg0);
+                    const uint32_t cbytes = (uint32_t)nseg * 128u;
+                    const uint32_t sbytes = FMT == 2 ? (uint32_t)nseg * 16u : 0u;
+                    uint8_t* dst = ring + (size_t)slot * stage_bytes;
+                    if (lane < kTileRows) slot_rows[slot * kTileRows + lane] = myrow;
+                    __syncwarp();
+                    if (lane == 0) {
+                        slot_tile[slot] = (int)vtile;
+                        mbar_arrive_expect_tx(&full[slot], (uint32_t)cnt * (cbytes + sbytes));
+                    }
+                    __syncwarp();
+                    if (lane < cnt) {
+                        bulk_copy_g2s(dst + lane * gpitch,
+                                      p.w + (int64_t)myrow * p.row_bytes + (int64_t)seg0 * 128,
+                                      cbytes, &full[slot]);
+                        if (FMT == 2)
+                            bulk_copy_g2s(dst + code_area + lane * 16u * (uint32_t)segs,
+                                          p.block_scale + (int64_t)myrow * p.scale_pitch +
+                                              (int64_t)seg0 * 16,
+                                          sbytes, &full[slot]);
+                    }
+                    __syncwarp();
+                    ++issued;
+                    if (++slot == S) {
+                        slot = 0;
+                        phase ^= 1u;
+                    }
                 }
-                tile = tnext;
-                need = tile < t_end && tile_mask_need(p, tile, lane, n0, n1);
+                qhead += cnt;
+                ++vtile;
+            };
+            pdl_wait();
+            int64_t claim = t_begin;
+            int64_t pending = 0;
+            if (lane == 0) pending = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
+            uint32_t wc[4];
+            gather_mask_load(p, claim, lane, wc);
+            while (claim < t_end && !stop) {
+                // claim the next range and start loading its mask words before this one
+                // is scanned
+                const int64_t cnext = __shfl_sync(0xffffffffu, pending, 0);
+                if (lane == 0 && cnext < t_end) pending = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
+                uint32_t wn[4] = {0u, 0u, 0u, 0u};
+                if (cnext < t_end) gather_mask_load(p, cnext, lane, wn);
+                const uint32_t u = gather_union(p, claim, lane, wc);  // lanes 0..7: words
+#pragma unroll 1
+                for (int w = 0; w < kGatherRows / 32; ++w) {
+                    const uint32_t uw = __shfl_sync(0xffffffffu, u, w);
+                    const int64_t row = claim * kGatherRows + w * 32 + lane;
+                    const bool bit = (uw >> lane) & 1u;
+                    const uint32_t bal = __ballot_sync(0xffffffffu, bit);
+                    if (bit) gq[(qtail + __popc(bal & ((1u << lane) - 1u))) & (kGatherQueue - 1)] = (int)row;
+                    qtail += __popc(bal);
+                    if (!bit && p.out_logits && row < p.n)  // masked out for every input
+                        for (int m = 0; m < M; ++m) p.out_logits[(int64_t)m * p.n + row] = 0xFF80u;
+                    // drain whole tiles after every word: at most 15 + 32 rows stay queued
+                    __syncwarp();
+                    while (qtail - qhead >= kTileRows && !stop) issue_gtile(kTileRows);
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) wc[j] = wn[j];
+                claim = cnext;
             }
+            if (!stop && qtail > qhead) issue_gtile(qtail - qhead);  // the CTA's last rows
         }
         // Leave no copy in flight: wait for the last stages issued (bounded). This comes
         // before the end marker, which advances the phase of a slot these waits name.
@@ -747,8 +827,10 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
             const int tile_id = red_tile[buf];
             if (tile_id < 0) break;
             const int64_t tile = tile_id;
-            const int64_t row = tile * kTileRows + rrow;
-            const float rs = (FMT == 1 && row < p.n) ? __ldg(p.row_scale + row) : 0.f;
+            // a gathered tile names its rows (-1: an unused row slot)
+            const int64_t row = G ? (int64_t)red_rows[buf * kTileRows + rrow] : tile * kTileRows + rrow;
+            const bool rvalid = row >= 0 && row < p.n;
+            const float rs = (FMT == 1 && rvalid) ? __ldg(p.row_scale + row) : 0.f;
             if (!have_f) {  // xexp is visible once the first partials have arrived
 #pragma unroll
                 for (int q = 0; q < Q; ++q) {
@@ -774,7 +856,7 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
 #pragma unroll
                     for (int w = 0; w < CW; ++w) a += rb[w * RED_WARP_FLOATS + rrow * RED_COLS + col];
                 }
-                const bool valid = row < p.n && col < M;
+                const bool valid = rvalid && col < M;
                 float l = a;
                 if (FMT != 0) l = (l * fa[q]) * fb[q];
                 if (FMT == 1) l *= rs;
@@ -853,12 +935,19 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
     // Per-lane offsets inside a stage. Slab l of a stage is 64 bytes of each row: segment
     // l / 2 (a 2 KB block of 16 rows x 128 B), half l % 2. With the 128-byte swizzle the
     // lane's 16-byte chunk of row r0 sits at r0 * 128 + ((64 (l % 2) + 16 c) ^ 16 (r0 % 8));
-    // row r0 + 8 is 1 KB further on. Block scales: [16 rows][16 segs bytes], unswizzled.
+    // row r0 + 8 is 1 KB further on. A gathered stage keeps each row whole instead (row j
+    // at j * gpitch, segment l / 2 at 128 (l / 2) within it); the 16-byte skew of gpitch
+    // spreads the 8 rows x 4 chunks of a read over all banks. Block scales: [16 rows]
+    // [16 segs bytes], unswizzled, after the codes.
     const uint32_t xr = (uint32_t)(r0 & 7) << 4;
-    const uint32_t coff0 = (uint32_t)r0 * 128u + (((uint32_t)c * 16u) ^ xr);
-    const uint32_t coff1 = (uint32_t)r0 * 128u + ((64u + (uint32_t)c * 16u) ^ xr);
+    const uint32_t coff0 = G ? (uint32_t)r0 * gpitch + (uint32_t)c * 16u
+                             : (uint32_t)r0 * 128u + (((uint32_t)c * 16u) ^ xr);
+    const uint32_t coff1 = G ? (uint32_t)r0 * gpitch + 64u + (uint32_t)c * 16u
+                             : (uint32_t)r0 * 128u + ((64u + (uint32_t)c * 16u) ^ xr);
+    const uint32_t seg_stride = G ? 128u : 2048u;  // bytes between a row's segments
+    const uint32_t r8 = G ? 8u * gpitch : 1024u;   // row r0 + 8 relative to row r0
     const uint32_t spitch = 16u * (uint32_t)segs;
-    const uint32_t soff = (uint32_t)code_stage_bytes(segs) + (uint32_t)r0 * spitch + 2u * (uint32_t)c;
+    const uint32_t soff = code_area + (uint32_t)r0 * spitch + 2u * (uint32_t)c;
     const uint16_t* xrow0 = xs + g * p.kpad + c * V;
     const uint16_t* xrow1 = xs + (8 + g) * p.kpad + c * V;
     const int total_slabs = (int)(K / SLAB);  // K is a whole number of slabs
@@ -866,7 +955,7 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
     // g / 4 on lane group g % 4, so only lanes with g % 4 == c load an input
     const bool xbd = (g & 3) == c && (g >> 2) < M;
     const uint16_t* xrowb = xs + (g >> 2) * p.kpad + c * V;
-    const uint32_t soffb = (uint32_t)code_stage_bytes(segs) + (uint32_t)r0 * spitch + 4u * (uint32_t)(c & 1);
+    const uint32_t soffb = code_area + (uint32_t)r0 * spitch + 4u * (uint32_t)(c & 1);
     float accb[4] = {0.f, 0.f, 0.f, 0.f};
     uint4 xvb[4];
 #pragma unroll
@@ -897,6 +986,9 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
         if (!mbar_wait_bounded(&full[slot], phase, abort_flag)) break;
         const int tile = slot_tile[slot];
         if (tile < 0) break;
+        // gathered sweep: the table row behind row slot `lane` of this tile (warp 0 hands
+        // the tile's rows to the reducer)
+        const int vrow = (G && warp == 0 && lane < kTileRows) ? slot_rows[slot * kTileRows + lane] : -1;
         for (int ch = 0; ch < NC; ++ch) {
             if (ch > 0 && !mbar_wait_bounded(&full[slot], phase, abort_flag)) break;
             const uint8_t* st = ring + (size_t)slot * stage_bytes;
@@ -904,19 +996,20 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
             const int nv = min(slabs_per_stage, total_slabs - a0);  // slabs inside the row
             // this warp's slabs in the stage: l = a - a0 with a % CW == warp
             int l = (warp - a0) & (CW - 1);
-            const uint8_t* cw = st + (l >> 1) * 2048 + ((l & 1) ? coff1 : coff0);
+            const uint8_t* cw = st + (l >> 1) * seg_stride + ((l & 1) ? coff1 : coff0);
+            const uint32_t cstep = (CW / 2) * seg_stride;  // l += CW moves CW / 2 segments
             const uint8_t* sw = st + soff + l * 8;
             int xo = (a0 + l) * SLAB;
             if (BD) {
                 const uint8_t* swb = st + soffb + l * 8;
-                for (; l < nv; l += CW, cw += CW * 1024, swb += CW * 8, xo += CW * SLAB)
-                    slab_mma_blocks(accb, xvb, cw, swb, 8u * spitch, xrowb + xo, xbd);
+                for (; l < nv; l += CW, cw += cstep, swb += CW * 8, xo += CW * SLAB)
+                    slab_mma_blocks(accb, xvb, cw, r8, swb, 8u * spitch, xrowb + xo, xbd);
             } else {
-                for (; l < nv; l += CW, cw += CW * 1024, sw += CW * 8, xo += CW * SLAB) {
+                for (; l < nv; l += CW, cw += cstep, sw += CW * 8, xo += CW * SLAB) {
                     if (CH == 2 && (((a0 + l) >> 3) & 1))
-                        slab_mma<FMT, NT>(acc[CH - 1], cw, sw, 8u * spitch, xrow0 + xo, xrow1 + xo, xg0, xg1);
+                        slab_mma<FMT, NT>(acc[CH - 1], cw, r8, sw, 8u * spitch, xrow0 + xo, xrow1 + xo, xg0, xg1);
                     else
-                        slab_mma<FMT, NT>(acc[0], cw, sw, 8u * spitch, xrow0 + xo, xrow1 + xo, xg0, xg1);
+                        slab_mma<FMT, NT>(acc[0], cw, r8, sw, 8u * spitch, xrow0 + xo, xrow1 + xo, xg0, xg1);
                 }
             }
             __syncwarp();
@@ -958,6 +1051,7 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
             }
         }
         if (warp == 0 && lane == 0) red_tile[buf] = tile;
+        if (G && warp == 0 && lane < kTileRows) red_rows[buf * kTileRows + lane] = vrow;
         __syncwarp();
         if (lane == 0) mbar_arrive(&red_full[buf]);
         buf ^= 1;
@@ -1703,6 +1797,388 @@ __global__ void __launch_bounds__(kTThreads, 1)
     }
 }
 
+// ---------------------------------------------------------------- NVFP4 tcgen05 sweep
+// NVFP4 tables with 3-32 inputs run the contraction on the tcgen05 tensor cores with A in
+// tensor memory. Four decode warps turn each table row's E2M1 codes times their E4M3 block
+// scale into f16 -- exact: a code has at most 2 significant bits and a scale 4, and every
+// product lies in [2^-10, 2688] -- and store them with tcgen05.st into tensor memory, one
+// table row per lane; one thread issues tcgen05.mma kind::f16 with A from tensor memory and
+// the f16 copy of x (scaled per input by a power of two, as the wide sweep reads it) as B
+// from shared memory, fp32 accumulator in tensor memory. Decoding into tensor memory keeps
+// the 4x larger f16 operand out of shared memory. A tile is H x 128 table rows (H MMA
+// halves sharing every x chunk, so x is read once per 128 H rows); each stage carries the
+// tile's code segments, their block scales and x's same K range (one TMA box each, 128-byte
+// swizzle for codes and x). A segment (256 elements) of one half fills one of three
+// 128-column A slots, so decoding runs a slot ahead of the MMAs. Four epilogue warps drain
+// the double-buffered accumulators as the tcgen05 sweep does (per input a running max,
+// lowest row, sum of exp), and the CTA partials go through the shared last-CTA fold.
+constexpr int kQThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2-5 decode, warps 6-9 epilogue
+constexpr int kQSlots = 3;      // tensor-memory A slots (one half's segment each)
+constexpr int kQAcol = 128;     // first A column; the accumulators use columns [0, 4N)
+constexpr int kQHead = 3072;    // barriers, misc, factors, fold; then the ring
+
+__host__ __device__ inline int tc4_code_bytes(int H, int segs) { return H * 128 * 128 * segs; }
+__host__ __device__ inline int tc4_scale_bytes(int H, int segs) { return H * 128 * 16 * segs; }
+__host__ __device__ inline int tc4_x_bytes(int N, int segs) { return 4 * segs * N * 128; }
+__host__ __device__ inline int tc4_stage_bytes(int N, int H, int segs) {
+    return tc4_code_bytes(H, segs) + tc4_scale_bytes(H, segs) + tc4_x_bytes(N, segs);
+}
+
+template <int N, int H>
+__global__ void __launch_bounds__(kQThreads, 1)
+    sweep_tc4_kernel(const __grid_constant__ SweepParams p, const __grid_constant__ CUtensorMap map_codes,
+                     const __grid_constant__ CUtensorMap map_scales,
+                     const __grid_constant__ CUtensorMap map_x) {
+    static_assert(N == 16 || N == 32, "16 or 32 input columns");
+    static_assert(H == 1 || H == 2, "one or two 128-row halves");
+    constexpr uint32_t kTmemCols = 512;
+    constexpr int TR = 128 * H;  // table rows per tile
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + kMaxStages;   // 4 decode warps + the MMA commit
+    uint64_t* afull = empty + kMaxStages;  // [kQSlots] 4 decode warps
+    uint64_t* aempty = afull + kQSlots;    // [kQSlots] the MMA commit
+    uint64_t* tfull = aempty + kQSlots;    // [2] the tile index posted + the MMA commit
+    uint64_t* tempty = tfull + 2;          // [2] 4 epilogue warps
+    uint64_t* done = tempty + 2;
+    int* misc = reinterpret_cast<int*>(done + 1);
+    volatile int* abort_flag = misc;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 1);
+    volatile int* slot_tile = misc + 2;             // [kMaxStages]
+    volatile int* acc_tile = misc + 2 + kMaxStages;  // [2]
+    float* sfac = reinterpret_cast<float*>(smem + 512);    // [2][32]: 2^-e_m as two factors
+    float4* fold = reinterpret_cast<float4*>(smem + 768);  // [4 warps][32 inputs]
+    uint8_t* ring = smem + kQHead;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int S = p.stages;
+    const int stage_bytes = p.stage_bytes;
+    const int segs = p.segs;
+    const int NC = p.stages_per_tile;
+    const int M = p.M;
+    const int64_t T = p.num_tiles;
+    const int row_segs = (int)(p.row_bytes / 128);
+    const int code_b = tc4_code_bytes(H, segs), scale_b = tc4_scale_bytes(H, segs);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 5);
+        }
+        for (int k = 0; k < kQSlots; ++k) {
+            mbar_init(&afull[k], 4);
+            mbar_init(&aempty[k], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 2);
+            mbar_init(&tempty[b], 4);
+        }
+        mbar_init(done, 1);
+        misc[0] = 0;
+        mbar_fence_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    pdl_launch_dependents();
+
+    if (warp == 0) {
+        // ---------------- producer: the tiles' stages, each tagged with its tile
+        int slot = 0;
+        uint32_t phase = 0;
+        int64_t issued = 0;
+        bool stop = false;
+        pdl_wait();  // x's f16 copy comes from the previous grid
+        int64_t tile = blockIdx.x;
+        int64_t pending = 0;
+        if (lane == 0) pending = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
+        while (tile < T && !stop) {
+            for (int ch = 0; ch < NC; ++ch) {
+                if (!mbar_wait_bounded(&empty[slot], phase ^ 1u, abort_flag)) {
+                    stop = true;
+                    break;
+                }
+                if (lane == 0) {
+                    uint8_t* dst = ring + (size_t)slot * stage_bytes;
+                    slot_tile[slot] = (int)tile;
+                    mbar_arrive_expect_tx(&full[slot], (uint32_t)stage_bytes);
+                    tma_load_3d(dst, &map_codes, 0, (int)(tile * TR), ch * segs, &full[slot]);
+                    tma_load_2d(dst + code_b, &map_scales, ch * 8 * segs, (int)(tile * TR), &full[slot]);
+                    tma_load_3d(dst + code_b + scale_b, &map_x, 0, 0, ch * 4 * segs, &full[slot]);
+                }
+                __syncwarp();
+                ++issued;
+                if (++slot == S) {
+                    slot = 0;
+                    phase ^= 1u;
+                }
+            }
+            tile = __shfl_sync(0xffffffffu, pending, 0);
+            if (lane == 0 && tile < T) pending = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
+        }
+        for (int64_t j = issued > S ? issued - S : 0; j < issued; ++j)
+            if (!mbar_wait_bounded(&full[j % S], (uint32_t)((j / S) & 1), nullptr)) break;
+        if (!stop && mbar_wait_bounded(&empty[slot], phase ^ 1u, abort_flag) && lane == 0) {
+            slot_tile[slot] = -1;
+            mbar_arrive(&full[slot]);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------- MMA issuer (lane 0)
+        constexpr uint32_t idesc = idesc_f16(128, N);
+        int slot = 0, aslot = 0, local = 0;
+        uint32_t phase = 0, aphase = 0;
+        while (true) {
+            if (!mbar_wait_bounded(&full[slot], phase, abort_flag)) break;
+            const int tile = slot_tile[slot];
+            const int buf = local & 1;
+            const uint32_t tph = (uint32_t)((local >> 1) & 1);
+            if (!mbar_wait_bounded(&tempty[buf], tph ^ 1u, abort_flag)) break;
+            if (lane == 0) {  // the tile index for the epilogue (its own arrival, release)
+                acc_tile[buf] = tile;
+                mbar_arrive(&tfull[buf]);
+                if (tile < 0) mbar_arrive(&tfull[buf]);  // no MMAs behind the end marker
+            }
+            __syncwarp();
+            if (tile < 0) break;
+            const uint32_t d0 = tmem_base + (uint32_t)(buf * H * N);
+            bool ok = true;
+            for (int ch = 0; ch < NC && ok; ++ch) {
+                if (ch > 0 && !mbar_wait_bounded(&full[slot], phase, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t x0 = smem_u32(ring + (size_t)slot * stage_bytes) + (uint32_t)(code_b + scale_b);
+                const int nseg = min(segs, row_segs - ch * segs);
+                for (int sg = 0; sg < nseg && ok; ++sg) {
+                    for (int h = 0; h < H; ++h) {
+                        if (!mbar_wait_bounded(&afull[aslot], aphase, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        if (lane == 0) {
+                            const uint32_t a0 = tmem_base + (uint32_t)(kQAcol + aslot * 128);
+#pragma unroll
+                            for (int kk = 0; kk < 16; ++kk) {
+                                const uint32_t xa = x0 + (uint32_t)((4 * sg + (kk >> 2)) * (N * 128) + (kk & 3) * 32);
+                                umma_f16_ta(d0 + (uint32_t)(h * N), a0 + (uint32_t)(kk * 8), sdesc_k128(xa), idesc,
+                                            (ch > 0 || sg > 0 || kk > 0) ? 1u : 0u);
+                            }
+                            umma_commit(&aempty[aslot]);  // the slot is free once these have read it
+                        }
+                        __syncwarp();
+                        if (++aslot == kQSlots) {
+                            aslot = 0;
+                            aphase ^= 1u;
+                        }
+                    }
+                }
+                if (lane == 0) umma_commit(&empty[slot]);  // x of the stage is read
+                __syncwarp();
+                if (++slot == S) {
+                    slot = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (lane == 0) umma_commit(&tfull[buf]);  // the accumulators, once complete
+            __syncwarp();
+            ++local;
+            if (!ok) break;
+        }
+        if (lane == 0) umma_commit(done);
+        __syncwarp();
+        mbar_wait_bounded(done, 0u, nullptr);
+    } else if (warp < 6) {
+        // ---------------- decode warps: tensor-memory lane quarter q = warp % 4, one table
+        // row per thread and half (row h * 128 + 32 q + lane of the tile)
+        const int q = warp & 3;
+        int slot = 0, aslot = 0;
+        uint32_t phase = 0, aphase = 0;
+        while (true) {
+            if (!mbar_wait_bounded(&full[slot], phase, abort_flag)) break;
+            if (slot_tile[slot] < 0) break;
+            bool ok = true;
+            for (int ch = 0; ch < NC && ok; ++ch) {
+                if (ch > 0 && !mbar_wait_bounded(&full[slot], phase, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t* st = ring + (size_t)slot * stage_bytes;
+                const int nseg = min(segs, row_segs - ch * segs);
+                for (int sg = 0; sg < nseg && ok; ++sg) {
+                    for (int h = 0; h < H; ++h) {
+                        const int r = h * 128 + q * 32 + lane;  // row of the tile
+                        if (!mbar_wait_bounded(&aempty[aslot], aphase ^ 1u, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        // the row's 128 code bytes (8 chunks, 128-byte swizzle) and 16 scales
+                        const uint8_t* crow = st + (size_t)sg * (TR * 128) + (size_t)r * 128;
+                        const uint4 sc = lds128(st + code_b + (size_t)r * 16 * segs + sg * 16);
+                        const uint32_t scw[4] = {sc.x, sc.y, sc.z, sc.w};
+                        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) +
+                                               (uint32_t)(kQAcol + aslot * 128);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {  // 64 elements (two chunks, four blocks)
+                            const uint4 c0 = lds128(crow + (((2 * j) ^ (r & 7)) << 4));
+                            const uint4 c1 = lds128(crow + (((2 * j + 1) ^ (r & 7)) << 4));
+                            const uint32_t wd[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                            // the four blocks' E4M3 scales as f16, each in both halves
+                            const uint32_t s01 = e4m3x2_to_f16x2((uint16_t)(scw[j] & 0xFFFFu));
+                            const uint32_t s23 = e4m3x2_to_f16x2((uint16_t)(scw[j] >> 16));
+                            const uint32_t bs[4] = {__byte_perm(s01, 0, 0x1010), __byte_perm(s01, 0, 0x3232),
+                                                    __byte_perm(s23, 0, 0x1010), __byte_perm(s23, 0, 0x3232)};
+                            uint32_t out[32];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                uint32_t o[4];
+                                e2m1x8_to_f16x2x4(wd[i], o);
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) out[4 * i + e] = hmul2(o[e], bs[i >> 1]);
+                            }
+                            tmem_st32(taddr + (uint32_t)(j * 32), out);
+                        }
+                        tmem_st_wait();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&afull[aslot]);
+                        if (++aslot == kQSlots) {
+                            aslot = 0;
+                            aphase ^= 1u;
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[slot]);  // codes and scales of the stage read
+                if (++slot == S) {
+                    slot = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) break;
+        }
+    } else {
+        // ---------------- epilogue: warp w reads tensor memory lanes 32 (w % 4) + [0, 32)
+        // (one table row per lane); per tile and input the warp folds its 32 rows with
+        // shuffles and lane m keeps input m's running (max, lowest row, sum of exp)
+        const int q = warp & 3;
+        const int ew = warp - 6;  // 0..3
+        const bool lp = p.out_logprob != nullptr || p.out_partial != nullptr;
+        pdl_wait();
+        if (ew == 0) {
+            const int e = lane < M ? -__ldg(p.xexp + lane) : 0;
+            sfac[lane] = ldexpf(1.f, e / 2);
+            sfac[32 + lane] = ldexpf(1.f, e - e / 2);
+        }
+        const float gsc = __ldg(p.global_scale);
+        named_sync(1, 4 * 32);
+        float my_v = -INFINITY, my_s = 0.f;  // input `lane`'s state
+        int32_t my_i = INT_MAX;
+        int local = 0;
+        while (true) {
+            const int buf = local & 1;
+            const uint32_t tph = (uint32_t)((local >> 1) & 1);
+            if (!mbar_wait_bounded(&tfull[buf], tph, abort_flag)) break;
+            const int tile = acc_tile[buf];
+            if (tile < 0) break;
+            tc_fence_after();
+            // one half at a time (registers); the accumulators are released after the last
+#pragma unroll 1
+            for (int h = 0; h < H; ++h) {
+                uint32_t v[N];
+                const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)((buf * H + h) * N);
+                if constexpr (N == 32)
+                    tmem_ld32(ta, v);
+                else
+                    tmem_ld16(ta, v);
+                tmem_ld_wait();
+                if (h == H - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tempty[buf]);  // the accumulators are free again
+                }
+                const int64_t row = (int64_t)tile * TR + h * 128 + q * 32 + lane;
+                const bool rvalid = row < p.n;
+#pragma unroll
+                for (int m = 0; m < N; ++m) {
+                    if (m >= M) break;  // warp-uniform
+                    const float l = (((__uint_as_float(v[m]) * sfac[m]) * sfac[32 + m])) * gsc;
+                    const bool ok = rvalid && mask_allows(p, m, row);
+                    if (rvalid && p.out_logits)
+                        p.out_logits[(int64_t)m * p.n + row] = ok ? f32_to_bf16(l) : (uint16_t)0xFF80u;
+                    // the 32 rows' (max, lowest row, sum of exp), lanes in a fixed tree
+                    float bv = ok ? l : -INFINITY, bs = (ok && l > -INFINITY) ? 1.f : 0.f;
+                    int32_t bi = ok ? (int32_t)row : INT_MAX;
+#pragma unroll
+                    for (int o = 16; o; o >>= 1) {
+                        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                        const int32_t oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                        const float os = __shfl_xor_sync(0xffffffffu, bs, o);
+                        if (lp) {
+                            float t = bv;
+                            lse_merge(t, bs, ov, os);
+                        }
+                        if (ov > bv || (ov == bv && oi < bi)) {
+                            bv = ov;
+                            bi = oi;
+                        }
+                    }
+                    if (lane == m) {  // rows arrive in increasing order: the earlier wins a tie
+                        if (lp) {
+                            float t = my_v;
+                            lse_merge(t, my_s, bv, bs);
+                        }
+                        if (bv > my_v || (bv == my_v && bi < my_i)) {
+                            my_v = bv;
+                            my_i = bi;
+                        }
+                    }
+                }
+            }
+            ++local;
+        }
+        if (lane < M) fold[ew * 32 + lane] = make_float4(my_v, __int_as_float(my_i), my_s, 0.f);
+        named_sync(1, 4 * 32);
+        if (ew == 0) {
+            if (lane < M) {
+                float bv = -INFINITY, bs = 0.f;
+                int32_t bi = INT_MAX;
+                for (int w = 0; w < 4; ++w) {
+                    const float4 f = fold[w * 32 + lane];
+                    const int32_t fi = __float_as_int(f.y);
+                    if (lp) {
+                        float t = bv;
+                        lse_merge(t, bs, f.x, f.z);
+                    }
+                    if (f.x > bv || (f.x == bv && fi < bi)) {
+                        bv = f.x;
+                        bi = fi;
+                    }
+                }
+                reinterpret_cast<Partial*>(p.partials)[(int64_t)blockIdx.x * kPartSlots + lane] =
+                    Partial{bv, bi, bs, 0.f};
+            }
+            __syncwarp();
+            fence_acq_rel_gpu();  // every publishing lane's store before lane 0's ticket
+            __syncwarp();
+            if (*abort_flag && lane == 0) raise_flag(p.dev_err, DEVFLAG_TIMEOUT);
+            ticket_and_fold(p, lane, lp);
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
 struct Geometry {
     int kpad;
     int segs;             // 128-byte segments per row per stage
@@ -1712,14 +2188,14 @@ struct Geometry {
     size_t smem;
 };
 
-Geometry geometry(int M, int64_t k, int fmt) {
+Geometry geometry(int M, int64_t k, int fmt, bool gather = false) {
     Geometry g{};
     g.kpad = (int)(k + 8);  // 16-byte skew between staged rows
     const int NT = M > 8 ? 2 : 1;
     const int CW = NT == 1 ? Roles<1>::CW : Roles<2>::CW;
     size_t head = (size_t)(2 * kMaxStages + 4) * 8 + 32 * sizeof(int) +
                   (size_t)2 * CW * kTileRows * 8 * NT * sizeof(float) + 32 * sizeof(float) +
-                  (size_t)M * g.kpad * 2;
+                  (gather ? (size_t)kGatherInts * sizeof(int) : 0) + (size_t)M * g.kpad * 2;
     head = ((head + 1023) & ~(size_t)1023) + 1024;  // 1 KB-aligned ring, plus slack
     const int64_t row_bytes = fmt == 0 ? k * 2 : fmt == 1 ? k : k / 2;
     const int row_segs = (int)(row_bytes / 128);
@@ -1730,7 +2206,7 @@ Geometry geometry(int M, int64_t k, int fmt) {
         for (int max_segs = kMaxSegs; max_segs >= 1; max_segs /= 2) {
             const int nc = (row_segs + max_segs - 1) / max_segs;
             const int segs = (row_segs + nc - 1) / nc;
-            const int sb = stage_bytes_for(fmt, segs);
+            const int sb = stage_bytes_for(fmt, segs, gather);
             int stages = avail > 0 ? (int)(avail / sb) : 0;
             if (stages > kMaxStages) stages = kMaxStages;
             if (stages >= want) {
@@ -1906,20 +2382,22 @@ cudaError_t launch_wide(const SweepParams& p, cudaStream_t s, SweepLaunch* info)
     return cudaGetLastError();
 }
 
-template <int FMT, int NT, int MODE, int BD>
+template <int FMT, int NT, int MODE, int BD, int G>
 cudaError_t launch_one(const SweepParams& p, cudaStream_t s, SweepLaunch* info) {
-    auto kern = sweep_kernel<FMT, NT, MODE, BD>;
-    const Geometry geo = geometry(p.M, p.k, FMT);
+    auto kern = sweep_kernel<FMT, NT, MODE, BD, G>;
+    const Geometry geo = geometry(p.M, p.k, FMT, G != 0);
     if (geo.stages < 2) return cudaErrorInvalidValue;
-    CUtensorMap map_codes, map_scales;
-    cudaError_t e = make_code_map(&map_codes, p.w, p.n, p.row_bytes, geo.segs);
-    if (e != cudaSuccess) return e;
-    if (FMT == 2) {
-        if ((e = make_scale_map(&map_scales, p.block_scale, p.n, p.scale_pitch, geo.segs)) !=
-            cudaSuccess)
-            return e;
-    } else {
-        map_scales = map_codes;  // unused
+    CUtensorMap map_codes{}, map_scales{};  // the gathered sweep copies rows without them
+    cudaError_t e = cudaSuccess;
+    if (!G) {
+        if ((e = make_code_map(&map_codes, p.w, p.n, p.row_bytes, geo.segs)) != cudaSuccess) return e;
+        if (FMT == 2) {
+            if ((e = make_scale_map(&map_scales, p.block_scale, p.n, p.scale_pitch, geo.segs)) !=
+                cudaSuccess)
+                return e;
+        } else {
+            map_scales = map_codes;  // unused
+        }
     }
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)geo.smem)) != cudaSuccess)
@@ -1928,11 +2406,12 @@ cudaError_t launch_one(const SweepParams& p, cudaStream_t s, SweepLaunch* info) 
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
         return e;
+    SweepParams q = p;
+    if (G) q.num_tiles = (p.n + kGatherRows - 1) / kGatherRows;  // claims of kGatherRows rows
     int64_t grid = sms;
-    if (grid > p.num_tiles) grid = p.num_tiles;
+    if (grid > q.num_tiles) grid = q.num_tiles;
     if (grid > kMaxGrid) grid = kMaxGrid;
     if (grid < 1) grid = 1;
-    SweepParams q = p;
     q.kpad = geo.kpad;
     q.stages = geo.stages;
     q.stage_bytes = geo.stage_bytes;
@@ -2040,16 +2519,99 @@ cudaError_t launch_tc(const SweepParams& p, cudaStream_t s, SweepLaunch* info) {
     return cudaGetLastError();
 }
 
-// Argmax sweeps that stream x per K chunk -- the tcgen05 sweep (BF16, FP8), the wide
-// sweep (NVFP4) -- take FP8 tables from 7 inputs on (measured faster than 16-row tiles
-// from there), the others from 9.
-inline bool streams_x(int M, int fmt) { return fmt == 1 ? M >= 7 : M > 8; }
+// Stage geometry of the NVFP4 tcgen05 sweep: two 128-byte segments per row per stage when
+// that leaves at least three stages, else one segment (at least two stages).
+WideGeometry tc4_geometry(int64_t k, int N, int H) {
+    WideGeometry g{};
+    const int row_segs = (int)(k / 2 / 128);
+    const long avail = (long)kSmemLimit - (long)kQHead;
+    for (int want = 3; want >= 2 && g.stages < 2; --want) {
+        for (int segs = 2; segs >= 1; --segs) {
+            if (segs > row_segs) continue;
+            const int sb = tc4_stage_bytes(N, H, segs);
+            int stages = avail > 0 ? (int)(avail / sb) : 0;
+            if (stages > kMaxStages) stages = kMaxStages;
+            if (stages >= want) {
+                g.segs = segs;
+                g.stages_per_tile = (row_segs + segs - 1) / segs;
+                g.stage_bytes = sb;
+                g.stages = stages;
+                break;
+            }
+        }
+    }
+    g.smem = (size_t)kQHead + (size_t)g.stages * g.stage_bytes;
+    return g;
+}
+
+template <int N, int H>
+cudaError_t launch_tc4(const SweepParams& p, cudaStream_t s, SweepLaunch* info) {
+    auto kern = sweep_tc4_kernel<N, H>;
+    const WideGeometry geo = tc4_geometry(p.k, N, H);
+    if (geo.stages < 2) return cudaErrorInvalidValue;
+    CUtensorMap map_codes, map_scales, map_x;
+    cudaError_t e = make_code_map(&map_codes, p.w, p.n, p.row_bytes, geo.segs, 128 * H);
+    if (e != cudaSuccess) return e;
+    if ((e = make_scale_map(&map_scales, p.block_scale, p.n, p.scale_pitch, geo.segs, 128 * H)) !=
+        cudaSuccess)
+        return e;
+    if ((e = make_x_map(&map_x, p.x16, p.M, p.k, 4 * geo.segs, N)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)geo.smem)) != cudaSuccess)
+        return e;
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return e;
+    SweepParams q = p;
+    q.num_tiles = (p.n + 128 * H - 1) / (128 * H);
+    q.stages = geo.stages;
+    q.stage_bytes = geo.stage_bytes;
+    q.segs = geo.segs;
+    q.stages_per_tile = geo.stages_per_tile;
+    int64_t grid = sms;
+    if (grid > q.num_tiles) grid = q.num_tiles;
+    if (grid > kMaxGrid) grid = kMaxGrid;
+    if (grid < 1) grid = 1;
+    wide_x16_kernel<<<p.M, 256, 0, s>>>(p.x, (int)p.k, p.x16, p.xexp);  // x as f16, per-input 2^e
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kQThreads);
+    cfg.dynamicSmemBytes = geo.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if ((e = cudaLaunchKernelEx(&cfg, kern, q, map_codes, map_scales, map_x)) != cudaSuccess) return e;
+    if (info) {
+        info->grid = (int)grid;
+        info->smem_bytes = (int)geo.smem;
+    }
+    return cudaGetLastError();
+}
+
+// Argmax sweeps that stream x per K chunk -- the tcgen05 sweeps -- take FP8 tables from 7
+// inputs on (measured faster than 16-row tiles from there), NVFP4 from 3 (its tensor-memory
+// A path), BF16 from 9.
+inline bool streams_x(int M, int fmt) { return fmt == 1 ? M >= 7 : fmt == 2 ? M >= 3 : M > 8; }
 
 }  // namespace
 
-size_t sweep_smem_bytes(int M, int64_t k, int fmt, int* kpad_out, int mode) {
+// A grammar mask with up to eight inputs: the gathered sweep, which reads only the rows
+// some input's mask allows.
+inline bool gathers(int M, bool masked) { return masked && M <= 8; }
+
+size_t sweep_smem_bytes(int M, int64_t k, int fmt, int* kpad_out, int mode, bool masked) {
+    if (mode == 0 && gathers(M, masked)) {
+        const Geometry g = geometry(M, k, fmt, true);
+        if (kpad_out) *kpad_out = g.kpad;
+        return g.stages >= 2 ? g.smem : (size_t)kSmemLimit + 1;
+    }
     if (mode == 0 && streams_x(M, fmt)) {  // the tcgen05 / wide sweeps stage x per K chunk
-        const WideGeometry w = fmt == 2 ? wide_geometry(k, fmt, M > 16 ? 32 : 16)
+        const WideGeometry w = fmt == 2 ? tc4_geometry(k, M > 16 ? 32 : 16, M > 8 ? 2 : 1)
                                         : tc_geometry(k, fmt, M > 16 ? 32 : 16);
         if (kpad_out) *kpad_out = (int)k;
         return w.stages >= 2 ? w.smem : (size_t)kSmemLimit + 1;
@@ -2123,15 +2685,23 @@ cudaError_t merge_partials_launch(const void* parts, int n_parts, int M, int32_t
 cudaError_t sweep_launch(const SweepParams& p, int fmt, int mode, cudaStream_t s,
                          SweepLaunch* info) {
     const bool two = p.M > 8;
-    if (fmt == 2 && mode == 0 && p.M <= 2) return launch_one<2, 1, 0, 1>(p, s, info);
+    if (mode == 0 && gathers(p.M, p.mask != nullptr)) {
+        if (fmt == 0) return launch_one<0, 1, 0, 0, 1>(p, s, info);
+        if (fmt == 1) return launch_one<1, 1, 0, 0, 1>(p, s, info);
+        if (fmt == 2)
+            return p.M <= 2 ? launch_one<2, 1, 0, 1, 1>(p, s, info) : launch_one<2, 1, 0, 0, 1>(p, s, info);
+    }
+    if (fmt == 2 && mode == 0 && p.M <= 2) return launch_one<2, 1, 0, 1, 0>(p, s, info);
     if (mode == 0 && streams_x(p.M, fmt)) {
         const bool four = p.M > 16;
         if (fmt == 0) return four ? launch_tc<0, 32>(p, s, info) : launch_tc<0, 16>(p, s, info);
         if (fmt == 1) return four ? launch_tc<1, 32>(p, s, info) : launch_tc<1, 16>(p, s, info);
-        if (fmt == 2) return four ? launch_wide<2, 4>(p, s, info) : launch_wide<2, 2>(p, s, info);
+        if (fmt == 2)
+            return four ? launch_tc4<32, 2>(p, s, info)
+                        : (p.M > 8 ? launch_tc4<16, 2>(p, s, info) : launch_tc4<16, 1>(p, s, info));
     }
 #define MTP_SWEEP_CASE(F, NTV, MD) \
-    if (fmt == F && (NTV == 2) == two && mode == MD) return launch_one<F, NTV, MD, 0>(p, s, info);
+    if (fmt == F && (NTV == 2) == two && mode == MD) return launch_one<F, NTV, MD, 0, 0>(p, s, info);
     // (mode 0 inputs past streams_x went to the tcgen05 / wide sweeps above)
     MTP_SWEEP_CASE(0, 1, 0) MTP_SWEEP_CASE(1, 1, 0) MTP_SWEEP_CASE(2, 1, 0)
     MTP_SWEEP_CASE(0, 1, 1) MTP_SWEEP_CASE(0, 2, 1)

@@ -71,6 +71,14 @@ def pack_mask(allowed: np.ndarray) -> np.ndarray:
     return w.astype(np.uint32).view(np.int32)
 
 
+def keep_mask(seed: int, M: int, N: int, keep: float) -> tuple[np.ndarray, np.ndarray]:
+    """Per-row grammar masks keeping a seeded fraction `keep` of N tokens: ([M, N] bool
+    allowed, [M, ceil(N/32)] int32 packed words)."""
+    g = _gen(seed)
+    allowed = (torch.rand((M, N), generator=g) < keep).numpy()
+    return allowed, pack_mask(allowed)
+
+
 def tiny_draft(seed: int = TINY["seed"], vocab: int = TINY["vocab"], h: int = TINY["h"],
                M: int = 1) -> dict:
     g = _gen(seed)

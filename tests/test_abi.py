@@ -131,7 +131,7 @@ def test_lm_head_lp_rejects(lib):
     assert lp(OUT, n_eff=101) == L.MTP_ERR_INVALID_ARG
     # partials are 16 bytes (max, index, sum of exponentials) for up to 1,024 CTAs x 32 inputs
     assert wsb == 256 + 16 * 32 * 1024 and L.mtp_noalloc_scratch_bytes() == wsb
-    # more than eight inputs on a quantized table add x as those sweeps read it (+ 1 KB of
+    # quantized tables with many inputs add x as those sweeps read it (+ 1 KB of
     # exponents): FP8, two E4M3 planes of 16 or 32 rows; NVFP4, an f16 copy of the M rows
     fp8 = weight(fmt=1, k=128, rs=OUT)
     assert L.mtp_lm_head_ws_bytes(fp8, 100, 6) == wsb  # FP8 streams x from 7 inputs on
@@ -139,6 +139,8 @@ def test_lm_head_lp_rejects(lib):
     assert L.mtp_lm_head_ws_bytes(fp8, 100, 9) == wsb + 2 * 16 * 128 + 1024
     assert L.mtp_lm_head_ws_bytes(fp8, 100, 17) == wsb + 2 * 32 * 128 + 1024
     nv = weight(fmt=2, k=256, bs=OUT, gs=OUT)
+    assert L.mtp_lm_head_ws_bytes(nv, 100, 2) == wsb  # NVFP4 reads its f16 x copy from 3 inputs
+    assert L.mtp_lm_head_ws_bytes(nv, 100, 3) == wsb + ((3 * 256 * 2 + 1023) // 1024) * 1024 + 1024
     assert L.mtp_lm_head_ws_bytes(nv, 100, 9) == wsb + ((9 * 256 * 2 + 1023) // 1024) * 1024 + 1024
     assert L.mtp_lm_head_ws_bytes(weight(k=128), 100, 32) == wsb
     # the no-alloc array has no room for that copy: rejected before any CUDA call
@@ -146,6 +148,7 @@ def test_lm_head_lp_rejects(lib):
                                  0, 0, OUT, None, None, None, None)
     assert noalloc(fp8, 7) == L.MTP_ERR_WORKSPACE
     assert noalloc(weight(fmt=2, k=256, bs=OUT, gs=OUT), 12) == L.MTP_ERR_WORKSPACE
+    assert noalloc(weight(fmt=2, k=256, bs=OUT, gs=OUT), 3) == L.MTP_ERR_WORKSPACE
     # the table descriptor is checked before its size is looked at: a bad format, a bad k
     # or a missing scale is an argument error, not a workspace one
     assert noalloc(weight(fmt=7, k=128), 12) == L.MTP_ERR_INVALID_ARG
@@ -261,6 +264,8 @@ def test_prefill_rejects(lib):
     assert st("mtp_prefill_kv", *prefill_args(ks=0.0)) == L.MTP_ERR_INVALID_ARG
     assert st("mtp_prefill_kv", *prefill_args(h=320)) == L.MTP_ERR_UNSUPPORTED   # h % 256
     assert st("mtp_prefill_kv", *prefill_args(hd=96)) == L.MTP_ERR_UNSUPPORTED
+    # a prologue row (embedding + hidden row) must fit one 48 KB ring stage
+    assert st("mtp_prefill_kv", *prefill_args(h=12544)) == L.MTP_ERR_UNSUPPORTED
     assert st("mtp_prefill_kv", *prefill_args(nkv=1)) == L.MTP_ERR_UNSUPPORTED  # nkv*hd % 256
     assert st("mtp_prefill_kv", *prefill_args(hidden=A + 8)) == L.MTP_ERR_INVALID_ARG
     assert st("mtp_prefill_kv", *prefill_args(ws=None)) == L.MTP_ERR_WORKSPACE
@@ -278,3 +283,13 @@ def test_gemm_and_kv_stage_reject(lib):
     assert st("mtp_debug_gemm_bf16", None, B2, OUT, 128, 256, 64, None) == L.MTP_ERR_INVALID_ARG
     assert st("mtp_debug_kv_write", A, B2, 10, 2, 100, 0, B2, 4, 16, 4, OUT, OUT, 1.0, 1.0,
               None, None) == L.MTP_ERR_INVALID_ARG  # hd % 32
+
+
+def test_wait_timeout_rejects(lib):
+    w = lambda which, lim, ctr=OUT, err=OUT: st("mtp_debug_wait_timeout", which, lim, ctr, err, None)
+    assert w(2, 1000) == L.MTP_ERR_INVALID_ARG          # which is 0 or 1
+    assert w(0, 0) == L.MTP_ERR_INVALID_ARG             # limit in [1, 4e9] cycles
+    assert w(0, 5_000_000_000) == L.MTP_ERR_INVALID_ARG
+    assert w(0, 1000, err=None) == L.MTP_ERR_INVALID_ARG  # the error word is required
+    assert w(1, 1000, ctr=None) == L.MTP_ERR_INVALID_ARG  # the counter wait needs its counter
+    assert w(1, 1000, ctr=OUT + 2) == L.MTP_ERR_INVALID_ARG

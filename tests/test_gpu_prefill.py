@@ -143,6 +143,7 @@ def check_rows(orc, d, kc, vc, rows, min_exact=0.98):
             exact += int((got == want).sum())
             total += got.size
     assert exact / total >= min_exact, exact / total
+    return exact / total
 
 
 def test_prefill_small_multi_chunk(orc):
@@ -186,13 +187,15 @@ def test_prefill_full_prompt_sampled_rows(orc):
     rows = np.unique(np.concatenate([
         [0, 1, 2047, 2048, 32767],
         rng.choice(d["R"], 59, replace=False)]))
-    check_rows(orc, d, kc, vc, rows)
+    frac = check_rows(orc, d, kc, vc, rows)
+    print(f"prefill 32,768 rows: {frac:.4%} of sampled codes identical to the oracle's")
 
 
 def test_prefill_lanes_and_graph_capture_agree(orc):
-    """Two workspace lanes (consecutive chunks side by side on two streams), one lane (in
-    order on the caller's stream) and a CUDA-graph capture of the two-lane call write the
-    same cache bytes; the rows match the oracle."""
+    """The whole call is one kernel on the caller's stream. Two workspace lanes
+    (consecutive chunks overlapping), one lane (chunks ordered through the same buffers),
+    the two-lane call on a side stream and a CUDA-graph capture of it write the same cache
+    bytes; the rows match the oracle."""
     d = synth.prefill_inputs(seed=81, R=700, vocab=500, h=256, nkv=2, hd=128)
     dev = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
     nb, chunk = int(d["num_blocks"]), 128
@@ -205,10 +208,15 @@ def test_prefill_lanes_and_graph_capture_agree(orc):
         torch.cuda.synchronize()
         outs.append((kc.cpu().numpy(), vc.cpu().numpy()))
     assert np.array_equal(outs[0][0], outs[1][0]) and np.array_equal(outs[0][1], outs[1][1])
-    kc, vc = new_caches(nb, 16, 2, 128)
-    ws = api.aligned_empty(full, 1024, "cuda")
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
+    kc, vc = new_caches(nb, 16, 2, 128)
+    ws = api.aligned_empty(full, 1024, "cuda")
+    with torch.cuda.stream(s):
+        api.prefill_kv(dev, kc, vc, chunk_rows=chunk, ws=ws)
+    s.synchronize()
+    assert np.array_equal(kc.cpu().numpy(), outs[0][0])
+    kc, vc = new_caches(nb, 16, 2, 128)
     g = torch.cuda.CUDAGraph()
     with torch.cuda.stream(s):
         with torch.cuda.graph(g, stream=s):
@@ -218,3 +226,13 @@ def test_prefill_lanes_and_graph_capture_agree(orc):
     assert np.array_equal(kc.cpu().numpy(), outs[0][0])
     assert np.array_equal(vc.cpu().numpy(), outs[0][1])
     check_rows(orc, d, outs[0][0], outs[0][1], np.arange(0, 700, 7))
+
+
+def test_prefill_ragged_chunks_and_one_row(orc):
+    """A last chunk of a single row, a chunk that is not a multiple of 128 rows, and a
+    one-row prompt."""
+    for R, chunk in ((257, 128), (200, 72), (1, 2048)):
+        d = synth.prefill_inputs(seed=90 + R, R=R, vocab=400, h=256, nkv=2, hd=128)
+        kc, vc, err = run_prefill(d, chunk=chunk)
+        assert err == 0
+        check_rows(orc, d, kc, vc, np.arange(R))

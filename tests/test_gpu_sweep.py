@@ -266,6 +266,41 @@ def test_full_tables(orc, cfg, fmt):
             assert np.array_equal(got[0], d["second"][:M])
 
 
+@pytest.mark.parametrize("cfg,fmt", FULL, ids=["bf16", "fp8", "nvfp4"])
+def test_masked_full_tables(orc, cfg, fmt):
+    """Grammar masks keeping 1% and 50% of the tokens on the full tables (the masked sweep
+    reads only the rows some input allows): the masked argmax and value against the oracle,
+    every disallowed logit -inf, and every allowed logit identical to the unmasked sweep's."""
+    Ms = (1, 4, 8) if fmt != 2 else (1, 2, 4)
+    Mmax = max(Ms)
+    N, K = cfg["N"], cfg["K"]
+    d = synth.head_table(cfg["seed"], N, K, Mmax)
+    w, x = synth.as_u16(d["W"]), synth.as_u16(d["x"])
+    q = oracle_quant(orc, w, fmt)
+    table = device_table(q, fmt, N, K)
+    head = api.LmHead(table)
+    ref_l, _, _, _ = oracle_sweep(orc, q, fmt, K, x)
+    _, _, dense_lg, _ = run_sweep(table, x, head=head)
+    for keep in (0.01, 0.5):
+        allowed, words = synth.keep_mask(int(keep * 1000) + fmt, Mmax, N, keep)
+        W = words.shape[1]
+        for M in Ms:
+            idx, val, lg, flags = run_sweep(table, x[:M], head=head, mask=words[:M].reshape(-1),
+                                            mask_words=W, stride=W)
+            assert flags == 0
+            for m in range(M):
+                a = allowed[m]
+                assert_argmax(int(idx[m]), ref_l[m], a)
+                assert_close([val[m]], [ref_l[m][a].max()], "masked out_val")
+                assert np.all(lg[m][~a] == 0xFF80)
+                assert np.array_equal(lg[m][a], dense_lg[m][a]), (keep, M, m)
+        # one mask shared by every input (stride 0)
+        idx, val, lg, _ = run_sweep(table, x[:4], head=head, mask=words[0], mask_words=W, stride=0)
+        for m in range(4):
+            assert_argmax(int(idx[m]), ref_l[m], allowed[0])
+            assert np.array_equal(lg[m][allowed[0]], dense_lg[m][allowed[0]])
+
+
 def oracle_logprobs(orc, ref_l, mask=None, mask_words=0, stride=0):
     out = []
     for m in range(ref_l.shape[0]):
