@@ -302,8 +302,11 @@ def time_e2e(head, x_host, steps, warmup, world, stream):
 
 
 def bench_tiny_draft(dev, steps, warmup):
-    """The tiny draft step (hidden 256, vocab 4096): combiner + lm_head sweep + argmax,
-    M = 1; everything is L2-resident, so this is latency (reported warm)."""
+    """The tiny draft step (hidden 256, vocab 4096), M = 1: everything is L2-resident, so
+    this is latency (reported warm). The fused step (mtp_draft_step, one cluster launch)
+    is the headline; the two-launch path (mtp_combine + mtp_lm_head_argmax) beside it.
+    Each is timed eager (one call after another) and as a 16-draft device-side chain
+    (the argmax index and y of one step feed the next) replayed from a CUDA graph."""
     import torch
 
     from mtp_speculative_draft_lm_b200 import api, synth
@@ -312,62 +315,69 @@ def bench_tiny_draft(dev, steps, warmup):
     dd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
     fc = api.bf16_table(dd["fc"])
     head = api.LmHead(api.bf16_table(dd["lm_head"]))
-    y = torch.empty((1, d["h"]), dtype=torch.bfloat16, device=dev)
-    idx = torch.empty((1,), dtype=torch.int32, device=dev)
-
-    def step():
-        api.combine(dd["embed"], dd["tokens"], dd["hidden"], dd["w_norm_embed"],
-                    dd["w_norm_hidden"], d["eps"], fc, out=y)
-        head(y, idx)
-
-    for _ in range(warmup):
-        step()
-    torch.cuda.synchronize()
-    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record()
-    for _ in range(steps):
-        step()
-    e.record()
-    torch.cuda.synchronize()
-    eager_us = s.elapsed_time(e) / steps * 1e3
-
-    # a chain of drafts on the device: each combiner gathers the embedding of the previous
-    # draft's argmax from the device index buffer; captured once as a CUDA graph
     chain = 16
     ys = [torch.empty((1, d["h"]), dtype=torch.bfloat16, device=dev) for _ in range(chain)]
     ids = [torch.empty((1,), dtype=torch.int32, device=dev) for _ in range(chain)]
+    vals = [torch.empty((1,), dtype=torch.float32, device=dev) for _ in range(chain)]
 
-    def run_chain():
-        tok, hid = dd["tokens"], dd["hidden"]
-        for j in range(chain):
-            api.combine(dd["embed"], tok, hid, dd["w_norm_embed"], dd["w_norm_hidden"], d["eps"],
-                        fc, out=ys[j])
-            head(ys[j], ids[j])
-            tok, hid = ids[j], ys[j]
+    def fused(tok, hid, j):
+        api.draft_step(dd["embed"], tok, hid, dd["w_norm_embed"], dd["w_norm_hidden"], d["eps"],
+                       dd["fc"], dd["lm_head"],
+                       out_y=ys[j], out_idx=ids[j], out_val=vals[j])
 
-    cs = torch.cuda.Stream(device=dev)
-    cs.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(cs):
-        run_chain()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=cs):
+    def two_launch(tok, hid, j):
+        api.combine(dd["embed"], tok, hid, dd["w_norm_embed"], dd["w_norm_hidden"], d["eps"], fc,
+                    out=ys[j])
+        head(ys[j], ids[j])
+
+    def timed(step_fn):
+        for _ in range(warmup):
+            step_fn(dd["tokens"], dd["hidden"], 0)
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(steps):
+            step_fn(dd["tokens"], dd["hidden"], 0)
+        e.record()
+        torch.cuda.synchronize()
+        eager_us = s.elapsed_time(e) / steps * 1e3
+
+        def run_chain():
+            tok, hid = dd["tokens"], dd["hidden"]
+            for j in range(chain):
+                step_fn(tok, hid, j)
+                tok, hid = ids[j], ys[j]
+
+        cs = torch.cuda.Stream(device=dev)
+        cs.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(cs):
             run_chain()
-    torch.cuda.synchronize()
-    reps = max(10, steps // chain)
-    for _ in range(3):
-        g.replay()
-    torch.cuda.synchronize()
-    s.record()
-    for _ in range(reps):
-        g.replay()
-    e.record()
-    torch.cuda.synchronize()
-    graph_us = s.elapsed_time(e) / (reps * chain) * 1e3
-    del g
-    return {"us_per_draft": eager_us, "launches_per_draft": 2,
-            "chain_graph_us_per_draft": graph_us, "chain_length": chain,
-            "note": "hidden 256, vocab 4096, M=1, warm (L2-resident); chain: 16 drafts fed "
-                    "device-side (argmax index -> next embedding gather) replayed from a CUDA graph"}
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cs):
+                run_chain()
+        torch.cuda.synchronize()
+        reps = max(10, steps // chain)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        s.record()
+        for _ in range(reps):
+            g.replay()
+        e.record()
+        torch.cuda.synchronize()
+        graph_us = s.elapsed_time(e) / (reps * chain) * 1e3
+        del g
+        return eager_us, graph_us
+
+    f_eager, f_graph = timed(fused)
+    t_eager, t_graph = timed(two_launch)
+    return {"us_per_draft": f_eager, "chain_graph_us_per_draft": f_graph, "launches_per_draft": 1,
+            "two_launch_us_per_draft": t_eager, "two_launch_chain_graph_us_per_draft": t_graph,
+            "chain_length": chain,
+            "note": "hidden 256, vocab 4096, M=1, warm (L2-resident); fused: mtp_draft_step, one "
+                    "cluster launch; two-launch: mtp_combine + mtp_lm_head_argmax; chain: 16 "
+                    "drafts fed device-side (argmax index and y -> next step) replayed from a "
+                    "CUDA graph"}
 
 
 def bench_prefill(dev, reps, tflops_peak, peak_src, rows=0):

@@ -245,6 +245,38 @@ mtp_status mtp_lm_head_argmax_lp(const mtp_weight* head, int64_t n_eff, const ui
                                  void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------
+ * mtp_draft_step -- one whole draft step for a small BF16 draft head in ONE launch:
+ * mtp_combine (BF16 fc) followed by mtp_lm_head_argmax (BF16 head, no logits), fused.
+ * Source: [v4_mtp.rs] forward_one steps 1-2 and 6-7 (embedding row, two RMSNorms with plain
+ * weights, e_proj / h_proj combiner, lm_head GEMV over the first n_eff rows, argmax,
+ * grammar-masked when a bitmask is given) and [mtp_head.rs] module docs (concat -> fc).
+ *   c[m] = [bf16(rms(embed[token_ids[m]]) w_norm_embed) || bf16(rms(hidden[m]) w_norm_hidden)]
+ *   y[m] = bf16(fc . c[m]);  l[m, r] = sum_j head[r, j] y[m, j] (fp32), r < n_eff
+ *   out_idx[m] = lowest allowed r with the largest l[m, r] (mask as mtp_lm_head_argmax;
+ *   nothing allowed -> 0, -inf and MTP_DEVFLAG_EMPTY_MASK)
+ *   embed (device) bf16 [vocab, h]; token_ids (device) i32 [M] (a bad id reads as a zero row
+ *   and sets MTP_DEVFLAG_BAD_TOKEN); hidden (device) bf16 [M, h]; w_norm_* (device) bf16 [h];
+ *   fc (device) bf16 [h, 2h]; head (device) bf16 [>= n_eff, h], rows packed at h;
+ *   out_y (device) bf16 [M, h] or NULL: y, for instance the next step's hidden rows;
+ *   out_idx (device) i32 [M]; out_val (device) f32 [M] or NULL; dev_err i32 [1] or NULL.
+ * One thread-block cluster does the whole step (no workspace), so it suits heads that sit
+ * in L2 (a few MB, as the tiny draft head's 2 MB); a large head belongs to
+ * mtp_lm_head_argmax, which spreads over every SM. The launch allows programmatic
+ * dependent launch: a chain of steps, each reading the previous one's out_idx and out_y
+ * as its token_ids and hidden, overlaps each launch with the previous step's end.
+ * Requires 1 <= M <= 4, 8 <= h <= 1024, h % 8 == 0; embed, hidden, fc, head 16-byte
+ * aligned. fc products are summed in fp32 in a fixed order, so y can differ from
+ * mtp_combine's in the last bit.
+ * ------------------------------------------------------------------------------ */
+mtp_status mtp_draft_step(const uint16_t* embed, int64_t vocab, const int32_t* token_ids,
+                          const uint16_t* hidden, int32_t M, int32_t h,
+                          const uint16_t* w_norm_embed, const uint16_t* w_norm_hidden, float eps,
+                          const uint16_t* fc, const uint16_t* head, int64_t n_eff,
+                          const int32_t* mask, int64_t mask_words, int64_t mask_stride_words,
+                          uint16_t* out_y, int32_t* out_idx, float* out_val, int32_t* dev_err,
+                          void* stream);
+
+/* ---------------------------------------------------------------------------------
  * Vocab-sharded sweep: each of G GPUs sweeps a contiguous range of the table's rows,
  * writes a 16-byte partial per input, the partials are gathered (G x M x 16 bytes, one
  * collective, the caller's: NCCL all-gather over NVLink), and every rank merges them.

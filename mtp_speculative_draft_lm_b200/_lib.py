@@ -38,7 +38,7 @@ EXPORTS = (
     "mtp_lm_head_host_ws_bytes", "mtp_lm_head_argmax_host",
     "mtp_lm_head_shard_partial", "mtp_argmax_merge_partials",
     "mtp_debug_encode_e4m3", "mtp_debug_encode_e2m1", "mtp_nvfp4_scale_pitch",
-    "mtp_debug_wait_timeout",
+    "mtp_debug_wait_timeout", "mtp_draft_step",
     "mtp_noalloc_scratch_bytes", "mtp_lm_head_argmax_noalloc",
     "mtp_prefill_ws_bytes", "mtp_prefill_kv", "mtp_debug_gemm_bf16", "mtp_debug_kv_write",
 )
@@ -94,6 +94,8 @@ _SIGS = {
     "mtp_lm_head_argmax_noalloc": (C.c_int, [_W, _I64, _P, _I32, _P, _I64, _I64, _P, _P, _P,
                                              _P, _P]),
     "mtp_debug_wait_timeout": (C.c_int, [_I32, _I64, _P, _P, _P]),
+    "mtp_draft_step": (C.c_int, [_P, _I64, _P, _P, _I32, _I32, _P, _P, C.c_float, _P, _P, _I64,
+                                 _P, _I64, _I64, _P, _P, _P, _P, _P]),
     "mtp_debug_encode_e4m3": (C.c_int, [_P, _I64, _P, _P]),
     "mtp_debug_encode_e2m1": (C.c_int, [_P, _I64, _P, _P]),
 }
@@ -280,6 +282,16 @@ def mtp_lm_head_argmax_noalloc(head, n_eff, x, M, mask, mask_words, mask_stride_
                                              mask_stride_words, _ptr(out_idx), _ptr(out_val),
                                              _ptr(out_logits), _ptr(dev_err), _stream(stream)),
            "mtp_lm_head_argmax_noalloc")
+
+
+def mtp_draft_step(embed, vocab, token_ids, hidden, M, h, w_norm_embed, w_norm_hidden, eps, fc,
+                   head, n_eff, mask, mask_words, mask_stride_words, out_y, out_idx, out_val,
+                   dev_err=None, stream=None):
+    _check(load().mtp_draft_step(_ptr(embed), vocab, _ptr(token_ids), _ptr(hidden), M, h,
+                                 _ptr(w_norm_embed), _ptr(w_norm_hidden), float(eps), _ptr(fc),
+                                 _ptr(head), n_eff, _ptr(mask), mask_words, mask_stride_words,
+                                 _ptr(out_y), _ptr(out_idx), _ptr(out_val), _ptr(dev_err),
+                                 _stream(stream)), "mtp_draft_step")
 
 
 def mtp_debug_wait_timeout(which, limit_cycles, counter, dev_err, stream=None):

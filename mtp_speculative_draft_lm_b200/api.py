@@ -219,6 +219,23 @@ def combine(embed, token_ids, hidden, w_norm_embed, w_norm_hidden, eps, fc: Tabl
     return out
 
 
+def draft_step(embed, token_ids, hidden, w_norm_embed, w_norm_hidden, eps, fc, head,
+               n_eff=None, mask=None, mask_words=0, mask_stride_words=0, out_y=None,
+               out_idx=None, out_val=None, dev_err=None, stream=None):
+    """One whole draft step (combiner + lm_head sweep + argmax) for a small BF16 head in
+    one launch: returns (idx, val, y)."""
+    M, h = hidden.shape
+    dev = hidden.device
+    n = head.shape[0] if n_eff is None else int(n_eff)
+    out_y = torch.empty((M, h), dtype=torch.bfloat16, device=dev) if out_y is None else out_y
+    out_idx = torch.empty((M,), dtype=torch.int32, device=dev) if out_idx is None else out_idx
+    out_val = torch.empty((M,), dtype=torch.float32, device=dev) if out_val is None else out_val
+    L.mtp_draft_step(embed, embed.shape[0], token_ids, hidden, M, h, w_norm_embed, w_norm_hidden,
+                     eps, fc, head, n, mask, mask_words, mask_stride_words, out_y, out_idx,
+                     out_val, dev_err, stream)
+    return out_idx, out_val, out_y
+
+
 def aligned_empty(nbytes: int, align: int, device) -> torch.Tensor:
     """A uint8 device buffer of nbytes whose address is a multiple of align (torch only
     promises 512 bytes)."""

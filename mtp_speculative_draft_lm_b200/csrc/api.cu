@@ -307,6 +307,31 @@ mtp_status mtp_lm_head_argmax_lp(const mtp_weight* head, int64_t n_eff, const ui
                         out_logprob, out_logits, dev_err, ws, ws_bytes, stream);
 }
 
+mtp_status mtp_draft_step(const uint16_t* embed, int64_t vocab, const int32_t* token_ids,
+                          const uint16_t* hidden, int32_t M, int32_t h,
+                          const uint16_t* w_norm_embed, const uint16_t* w_norm_hidden, float eps,
+                          const uint16_t* fc, const uint16_t* head, int64_t n_eff,
+                          const int32_t* mask, int64_t mask_words, int64_t mask_stride_words,
+                          uint16_t* out_y, int32_t* out_idx, float* out_val, int32_t* dev_err,
+                          void* stream) {
+    if (!embed || !token_ids || !hidden || !w_norm_embed || !w_norm_hidden || !fc || !head ||
+        !out_idx)
+        return MTP_ERR_INVALID_ARG;
+    if (vocab < 1 || n_eff < 1 || n_eff > (int64_t)INT32_MAX || h < 8 || h % 8 || !(eps >= 0.f))
+        return MTP_ERR_INVALID_ARG;
+    if (mask && (mask_words < 1 || mask_stride_words < 0)) return MTP_ERR_INVALID_ARG;
+    if (M < 1 || M > mtp::draft_step_max_m() || h > mtp::draft_step_max_h()) return MTP_ERR_UNSUPPORTED;
+    if (!aligned(embed, 16) || !aligned(hidden, 16) || !aligned(fc, 16) || !aligned(head, 16) ||
+        !aligned(w_norm_embed, 2) || !aligned(w_norm_hidden, 2) || !aligned(token_ids, 4) ||
+        !aligned(out_y, 2) || !aligned(out_idx, 4) || !aligned(out_val, 4) || !aligned(mask, 4) ||
+        !aligned(dev_err, 4))
+        return MTP_ERR_INVALID_ARG;
+    return from_cuda(mtp::draft_step_launch(embed, vocab, token_ids, hidden, M, h, w_norm_embed,
+                                            w_norm_hidden, eps, fc, head, n_eff, mask, mask_words,
+                                            mask_stride_words, out_y, out_idx, out_val, dev_err,
+                                            as_stream(stream)));
+}
+
 size_t mtp_prefill_ws_bytes(int64_t chunk_rows, int32_t h, int32_t nkv, int32_t hd) {
     if (chunk_rows < 1 || h < 1 || nkv < 1 || hd < 2) return 0;
     return mtp::prefill_ws_bytes(chunk_rows, h, nkv, hd);

@@ -140,6 +140,16 @@ cudaError_t kv_write_launch(const uint16_t* k_rot, const uint16_t* v, int64_t R,
 int gemm_tile_n();
 int gemm_tile_k();
 
+// One whole draft step for a small BF16 head in one cluster launch (draft.cu).
+int draft_step_max_m();
+int draft_step_max_h();
+cudaError_t draft_step_launch(const uint16_t* embed, int64_t vocab, const int32_t* tokens,
+                              const uint16_t* hidden, int M, int h, const uint16_t* w_ne,
+                              const uint16_t* w_nh, float eps, const uint16_t* fc,
+                              const uint16_t* head, int64_t n, const int32_t* mask,
+                              int64_t mask_words, int64_t mask_stride, uint16_t* out_y,
+                              int32_t* out_idx, float* out_val, int32_t* dev_err, cudaStream_t s);
+
 // Self-check of the bounded waits (selfcheck.cu): which 0 waits on an mbarrier phase that
 // nothing completes, 1 on a global counter (device u32, kept at 0 by the caller) that
 // nothing increments; either gives up after limit_cycles and sets DEVFLAG_TIMEOUT.

@@ -21,7 +21,7 @@ import sys
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_SRCS = ["formats.c", "quant.c", "draft.c", "prefill.c"]
+_SRCS = ["formats.c", "quant.c", "draft.c", "prefill.c", "attn.c"]
 LIB_PATH = os.path.join(_HERE, "liborc.so")
 
 FLAG_BAD_TOKEN = 1
@@ -84,6 +84,9 @@ def lib():
                                         _p, _p, _i32, _i32, C.c_double, _p, _i64, _p,
                                         _i64, _i32, _i64, C.c_float, C.c_float, _p,
                                         _i64, _p, _p, _p, _p, _p, _p]),
+            "orc_paged_decode_attn": (_i32, [_p, _i32, _i32, _i32, _p, _p, _p, _i64, _i32,
+                                             _i64, _i64, C.c_double, C.c_double, C.c_double,
+                                             _p]),
             "orc_num_threads": (_i32, []),
         }
         for name, (res, args) in sig.items():
@@ -293,6 +296,26 @@ def prefill_rows(embed, tokens, hidden, w_norm_embed, w_norm_hidden, eps, fc, wk
         int(block_size), int(num_blocks), float(k_scale), float(v_scale), _ptr(rows), n,
         _ptr(y), _ptr(k_rot), _ptr(v), _ptr(kc), _ptr(vc), _ptr(sl))
     return dict(y=y, k_rot=k_rot, v=v, k_codes=kc, v_codes=vc, slot=sl, flags=int(flags))
+
+
+# ---- decode attention (attn.c) ----------------------------------------------------
+
+def paged_decode_attn(q, nkv, k_cache, v_cache, block_table, block_size, num_blocks, seq_len,
+                      k_scale=1.0, v_scale=1.0, scale=None):
+    """Single-token attention of q [nq, hd] (bf16 bits) over cache rows 0 .. seq_len - 1
+    of an E4M3 cache [num_blocks, bs, nkv, hd]; scale defaults to 1/sqrt(hd). Returns
+    (out [nq, hd] float64, flags)."""
+    q = _c(q, np.uint16)
+    nq, hd = q.shape
+    scale = 1.0 / np.sqrt(hd) if scale is None else float(scale)
+    kc = _c(k_cache, np.uint8)
+    vc = _c(v_cache, np.uint8)
+    bt = _c(block_table, np.int32)
+    out = np.empty((nq, hd), dtype=np.float64)
+    flags = lib().orc_paged_decode_attn(_ptr(q), nq, int(nkv), hd, _ptr(kc), _ptr(vc), _ptr(bt),
+                                        bt.size, int(block_size), int(num_blocks), int(seq_len),
+                                        float(k_scale), float(v_scale), scale, _ptr(out))
+    return out, int(flags)
 
 
 if __name__ == "__main__":  # pragma: no cover

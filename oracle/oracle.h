@@ -88,6 +88,13 @@ int32_t orc_prefill_rows(const uint16_t* embed, int64_t vocab, const int32_t* to
                          uint8_t* out_k_codes, uint8_t* out_v_codes, int64_t* out_slot);
 void orc_kv_encode(const uint16_t* vals, int64_t n, float scale, uint8_t* codes);
 
+/* attn.c: single-token paged decode attention over an E4M3 cache [num_blocks, bs, nkv, hd] */
+int32_t orc_paged_decode_attn(const uint16_t* q, int32_t nq, int32_t nkv, int32_t hd,
+                              const uint8_t* k_cache, const uint8_t* v_cache,
+                              const int32_t* block_table, int64_t n_table, int32_t block_size,
+                              int64_t num_blocks, int64_t seq_len, double k_scale, double v_scale,
+                              double scale, double* out);
+
 /* threads the OpenMP loops use */
 int32_t orc_num_threads(void);
 

@@ -293,3 +293,17 @@ def test_wait_timeout_rejects(lib):
     assert w(0, 1000, err=None) == L.MTP_ERR_INVALID_ARG  # the error word is required
     assert w(1, 1000, ctr=None) == L.MTP_ERR_INVALID_ARG  # the counter wait needs its counter
     assert w(1, 1000, ctr=OUT + 2) == L.MTP_ERR_INVALID_ARG
+
+
+def test_draft_step_rejects(lib):
+    def ds(M=1, h=256, embed=A, head=B2, mask=None, mw=0, ms=0, idx=OUT, n=100):
+        return st("mtp_draft_step", embed, 100, OUT, A, M, h, A, A, 1e-6, A, head, n, mask, mw, ms,
+                  None, idx, None, None, None)
+    assert ds(embed=None) == L.MTP_ERR_INVALID_ARG
+    assert ds(idx=None) == L.MTP_ERR_INVALID_ARG
+    assert ds(h=260) == L.MTP_ERR_INVALID_ARG       # h % 8
+    assert ds(n=0) == L.MTP_ERR_INVALID_ARG
+    assert ds(mask=OUT, mw=0) == L.MTP_ERR_INVALID_ARG
+    assert ds(M=5) == L.MTP_ERR_UNSUPPORTED         # up to 4 inputs
+    assert ds(h=2048) == L.MTP_ERR_UNSUPPORTED      # up to hidden 1024
+    assert ds(head=B2 + 8) == L.MTP_ERR_INVALID_ARG  # 16-byte aligned head

@@ -152,3 +152,112 @@ def test_device_side_draft_chain(orc, M):
     for j in range(steps):
         assert np.array_equal(u16_of(y_buf[j]), eager[j][0])
         assert np.array_equal(idx_bufs[j].cpu().numpy(), eager[j][1])
+
+
+def gpu_draft_step(d, dd=None, mask=None, mask_words=0, stride=0, tokens=None):
+    dd = dd or {k: (to_dev_u16(v) if isinstance(v, np.ndarray) and v.dtype == np.uint16 else v)
+                for k, v in d.items()}
+    err = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    tok = to_dev(np.asarray(d["tokens"] if tokens is None else tokens, np.int32))
+    m = to_dev(mask) if mask is not None else None
+    idx, val, y = api.draft_step(dd["embed"], tok, dd["hidden"], dd["w_norm_embed"],
+                                 dd["w_norm_hidden"], d["eps"], dd["fc"], dd["lm_head"], mask=m,
+                                 mask_words=mask_words, mask_stride_words=stride, dev_err=err)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy(), val.cpu().numpy(), u16_of(y), int(err.item())
+
+
+@pytest.mark.parametrize("M", [1, 2, 4])
+def test_draft_step_one_launch(orc, M):
+    """The fused draft step (one cluster launch): y and the argmax against the oracle."""
+    d = draft(M)
+    idx, val, y, err = gpu_draft_step(d)
+    assert err == 0
+    ref_y, _, _ = orc.combine(d["embed"], d["tokens"].numpy(), d["hidden"], d["w_norm_embed"],
+                              d["w_norm_hidden"], d["eps"], d["fc"])
+    assert_close(bf16_bits_to_f64(y), bf16_bits_to_f64(ref_y), "y")
+    # the argmax over the GPU's own y (a bf16 ulp of y may move close logits)
+    ref_l, _, _, _ = orc.lm_head_argmax(0, d["lm_head"], d["h"], y)
+    for m in range(M):
+        assert_argmax(int(idx[m]), ref_l[m])
+        assert_close([val[m]], [ref_l[m].max()], "out_val")
+
+
+@pytest.mark.parametrize("h,vocab", [(64, 1000), (512, 3333), (1024, 5000)])
+def test_draft_step_other_widths(orc, h, vocab):
+    d = draft(2, seed=31 + h, h=h, vocab=vocab)
+    idx, val, y, err = gpu_draft_step(d)
+    assert err == 0
+    ref_y, _, _ = orc.combine(d["embed"], d["tokens"].numpy(), d["hidden"], d["w_norm_embed"],
+                              d["w_norm_hidden"], d["eps"], d["fc"])
+    assert_close(bf16_bits_to_f64(y), bf16_bits_to_f64(ref_y), "y")
+    ref_l, _, _, _ = orc.lm_head_argmax(0, d["lm_head"], d["h"], y)
+    for m in range(2):
+        assert_argmax(int(idx[m]), ref_l[m])
+
+
+def test_draft_step_mask_and_flags(orc):
+    """Per-input masks (one allowing nothing: index 0, -inf, the empty-mask flag) and a bad
+    token id (a zero embedding row and the bad-token flag)."""
+    d = draft(3)
+    allowed, words = synth.keep_mask(17, 3, d["vocab"], 0.1)
+    allowed[1] = False
+    words[1] = 0
+    W = words.shape[1]
+    toks = np.asarray(d["tokens"], np.int32).copy()
+    toks[2] = d["vocab"] + 5
+    idx, val, y, err = gpu_draft_step(d, mask=words.reshape(-1), mask_words=W, stride=W, tokens=toks)
+    assert err == (L.MTP_DEVFLAG_EMPTY_MASK | L.MTP_DEVFLAG_BAD_TOKEN)
+    ref_y, _, _ = orc.combine(d["embed"], toks, d["hidden"], d["w_norm_embed"], d["w_norm_hidden"],
+                              d["eps"], d["fc"])
+    assert_close(bf16_bits_to_f64(y), bf16_bits_to_f64(ref_y), "y")
+    ref_l, _, _, _ = orc.lm_head_argmax(0, d["lm_head"], d["h"], y)
+    assert idx[1] == 0 and val[1] == -np.inf
+    for m in (0, 2):
+        assert_argmax(int(idx[m]), ref_l[m], allowed[m])
+
+
+def test_draft_step_chain_eager_and_graph(orc):
+    """Eight chained fused steps (token and hidden from the previous step's outputs on the
+    device), eager and replayed from a CUDA graph: identical, and each step matches the
+    oracle from the previous step's GPU outputs."""
+    steps, M = 8, 1
+    d = draft(M)
+    dd = {k: (to_dev_u16(v) if isinstance(v, np.ndarray) and v.dtype == np.uint16 else v)
+          for k, v in d.items()}
+    tok0 = to_dev(np.asarray(d["tokens"], np.int32))
+    ys = [torch.empty((M, d["h"]), dtype=torch.bfloat16, device="cuda") for _ in range(steps)]
+    ids = [torch.empty((M,), dtype=torch.int32, device="cuda") for _ in range(steps)]
+    vals = [torch.empty((M,), dtype=torch.float32, device="cuda") for _ in range(steps)]
+
+    def chain():
+        tok, hid = tok0, dd["hidden"]
+        for j in range(steps):
+            api.draft_step(dd["embed"], tok, hid, dd["w_norm_embed"], dd["w_norm_hidden"], d["eps"],
+                           dd["fc"], dd["lm_head"], out_y=ys[j], out_idx=ids[j], out_val=vals[j])
+            tok, hid = ids[j], ys[j]
+
+    chain()
+    torch.cuda.synchronize()
+    eager = [(u16_of(y).copy(), i.cpu().numpy().copy()) for y, i in zip(ys, ids)]
+    tok, hid = np.asarray(d["tokens"], np.int32), d["hidden"]
+    for j in range(steps):
+        ref_y, _, _ = orc.combine(d["embed"], tok, hid, d["w_norm_embed"], d["w_norm_hidden"],
+                                  d["eps"], d["fc"])
+        assert_close(bf16_bits_to_f64(eager[j][0]), bf16_bits_to_f64(ref_y), f"y step {j}")
+        ref_l, _, _, _ = orc.lm_head_argmax(0, d["lm_head"], d["h"], eager[j][0])
+        assert_argmax(int(eager[j][1][0]), ref_l[0])
+        tok, hid = eager[j][1], eager[j][0]
+    for b in ids:
+        b.zero_()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            chain()
+    g.replay()
+    torch.cuda.synchronize()
+    for j in range(steps):
+        assert np.array_equal(u16_of(ys[j]), eager[j][0])
+        assert np.array_equal(ids[j].cpu().numpy(), eager[j][1])

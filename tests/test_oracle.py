@@ -561,3 +561,89 @@ def test_fp8_x_two_term_split(orc):
     hi = orc.e4m3_value(orc.e4m3_encode(xs))
     lo = orc.e4m3_value(orc.e4m3_encode(xs - hi))
     assert abs(hi[1] + lo[1] - xs[1]) == 2.0 ** -10
+
+
+# ---------------------------------------------------------------- decode attention pins
+def _attn_case(orc, seed, nq=8, nkv=2, hd=64, seq=40, bs=16, extra_blocks=3):
+    rng = np.random.default_rng(seed)
+    nb = seq // bs + 1 + extra_blocks
+    bt = rng.permutation(nb).astype(np.int32)
+    kc = orc_codes(orc, rng, (nb, bs, nkv, hd))
+    vc = orc_codes(orc, rng, (nb, bs, nkv, hd))
+    q = orc.f64_to_bf16(rng.normal(0, 1, (nq, hd)))
+    return q, kc, vc, bt, nb
+
+
+def orc_codes(orc, rng, shape):
+    # E4M3 codes of N(0, 1) values (finite codes only: the NaN pattern never occurs)
+    return orc.e4m3_encode(rng.normal(0, 1, shape)).reshape(shape)
+
+
+def _dq(orc, codes):
+    return orc.e4m3_value(codes.reshape(-1)).reshape(codes.shape)
+
+
+def test_attn_single_row_returns_its_values(orc):
+    q, kc, vc, bt, nb = _attn_case(orc, 1, seq=1)
+    out, flags = orc.paged_decode_attn(q, 2, kc, vc, bt, 16, nb, 1, k_scale=0.5, v_scale=0.25)
+    assert flags == 0
+    slot = orc.slot(bt, 16, nb, 0)
+    vrow = _dq(orc, vc.reshape(-1, 2, 64)[slot])  # [nkv, hd]
+    for i in range(8):
+        assert np.array_equal(out[i], 0.25 * vrow[i // 4])  # exact: one weight of 1
+
+
+def test_attn_zero_scale_and_equal_keys_average_the_values(orc):
+    q, kc, vc, bt, nb = _attn_case(orc, 2, seq=40)
+    slots = [orc.slot(bt, 16, nb, p) for p in range(40)]
+    vrows = _dq(orc, vc.reshape(-1, 2, 64)[slots])  # [seq, nkv, hd]
+    mean = vrows.mean(axis=0)
+    out, _ = orc.paged_decode_attn(q, 2, kc, vc, bt, 16, nb, 40, scale=0.0)
+    for i in range(8):
+        assert np.allclose(out[i], mean[i // 4], rtol=0, atol=1e-12)
+    kc2 = kc.copy().reshape(-1, 2, 64)
+    kc2[slots] = kc2[slots[0]]  # every row the same key
+    out2, _ = orc.paged_decode_attn(q, 2, kc2.reshape(kc.shape), vc, bt, 16, nb, 40)
+    for i in range(8):
+        assert np.allclose(out2[i], mean[i // 4], rtol=0, atol=1e-12)
+
+
+def test_attn_planted_key_dominates_without_overflow(orc):
+    q, kc, vc, bt, nb = _attn_case(orc, 3, nq=2, nkv=1, seq=33)
+    qv = np.zeros((2, 64))
+    qv[:, 0] = 1.0
+    q = orc.f64_to_bf16(qv)
+    kflat = kc.reshape(-1, 1, 64).copy()
+    slots = [orc.slot(bt, 16, nb, p) for p in range(33)]
+    kflat[slots] = orc.e4m3_encode(np.zeros(64))
+    kflat[slots[17], 0, 0] = orc.e4m3_encode(np.array([448.0]))[0]
+    out, _ = orc.paged_decode_attn(q, 1, kflat.reshape(kc.shape), vc, bt, 16, nb, 33, scale=2.0)
+    # the planted row scores 896 against 0 for the rest: its weight is 1 - 32 e^-896
+    assert np.all(np.isfinite(out))
+    want = _dq(orc, vc.reshape(-1, 1, 64)[slots[17], 0])
+    assert np.array_equal(out[0], want) and np.array_equal(out[1], want)
+
+
+def test_attn_block_permutation_and_head_groups(orc):
+    q, kc, vc, bt, nb = _attn_case(orc, 4, seq=45)
+    out, _ = orc.paged_decode_attn(q, 2, kc, vc, bt, 16, nb, 45)
+    # move every physical block to a new place and rewrite the block table to match
+    perm = np.random.default_rng(9).permutation(nb)
+    kc2, vc2 = np.empty_like(kc), np.empty_like(vc)
+    kc2[perm] = kc
+    vc2[perm] = vc
+    out2, _ = orc.paged_decode_attn(q, 2, kc2, vc2, perm[bt].astype(np.int32), 16, nb, 45)
+    assert np.array_equal(out, out2)
+    # query heads 0-3 read kv head 0 and 4-7 kv head 1: head 5 equals a one-group run of
+    # kv head 1 alone
+    out1, _ = orc.paged_decode_attn(q[5:6], 1, np.ascontiguousarray(kc[:, :, 1:2]),
+                                    np.ascontiguousarray(vc[:, :, 1:2]), bt, 16, nb, 45)
+    assert np.array_equal(out[5], out1[0])
+
+
+def test_attn_missing_block_flags_and_skips(orc):
+    q, kc, vc, bt, nb = _attn_case(orc, 5, seq=40)
+    out, flags = orc.paged_decode_attn(q, 2, kc, vc, bt[:2], 16, nb, 40)  # rows 32.. have no block
+    assert flags & orc.FLAG_BAD_SLOT
+    ref, _ = orc.paged_decode_attn(q, 2, kc, vc, bt, 16, nb, 32)
+    assert np.array_equal(out, ref)
