@@ -410,6 +410,37 @@ def bench_prefill(dev, reps, tflops_peak, peak_src, rows=0):
             "rows": R, "hidden": h, "chunk": synth.PREFILL["chunk"]}
 
 
+def bench_attn(dev, steps, warmup, seq=32768, nq=64, nkv=8, hd=128):
+    """Single-token decode attention over a paged E4M3 cache of seq rows (the prefill
+    workload's 8 KV heads x 128; 64 query heads, a reading: the pages give no head count):
+    every cached K and V byte is read once, so HBM GB/s is the figure."""
+    import torch
+
+    from mtp_speculative_draft_lm_b200 import api, synth
+
+    g = synth._gen(1006)
+    nb = seq // 16 + 1
+    kc = torch.randint(0, 0x7E, (nb, 16, nkv, hd), generator=g, dtype=torch.uint8).to(dev)
+    vc = torch.randint(0, 0x7E, (nb, 16, nkv, hd), generator=g, dtype=torch.uint8).to(dev)
+    bt = torch.randperm(nb, generator=g).to(torch.int32).to(dev)
+    q = synth.normal_bf16(g, (nq, hd), 1.0).to(dev)
+    out, ws = api.paged_decode_attn(q, nkv, kc, vc, bt, seq)
+    for _ in range(warmup):
+        api.paged_decode_attn(q, nkv, kc, vc, bt, seq, out=out, ws=ws)
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        api.paged_decode_attn(q, nkv, kc, vc, bt, seq, out=out, ws=ws)
+    e.record()
+    torch.cuda.synchronize()
+    us = s.elapsed_time(e) / steps * 1e3
+    nbytes = 2 * seq * nkv * hd + 2 * 2 * nq * hd + bt.numel() * 4
+    return {"us_per_draft_position": us, "GB/s": nbytes / (us * 1e-6) / 1e9,
+            "bytes_per_step": nbytes, "seq_len": seq, "nq": nq, "nkv": nkv, "hd": hd,
+            "note": "K and V rows of every cached position read once; launches: 2"}
+
+
 def _median_runs(fn, budget_s, max_runs=3):
     """Median wall time of up to max_runs calls of fn, stopping once budget_s is spent."""
     times = []
@@ -640,6 +671,8 @@ def main():
         tpk, tsrc = measured_tflops()
         if args.only == "prefill":
             out = bench_prefill(dev, 2, tpk, tsrc, args.prefill_rows)
+        elif args.only == "attn":
+            out = bench_attn(dev, args.steps, args.warmup)
         else:
             out = bench_tiny_draft(dev, args.steps, args.warmup)
         print(json.dumps({"only": args.only, **out}), flush=True)
@@ -751,6 +784,7 @@ def main():
         rows["tiny_draft_M1"] = bench_tiny_draft(dev, max(200, args.steps // 10), args.warmup)
         tpk, tsrc = measured_tflops()
         rows["prefill_32k"] = bench_prefill(dev, 5, tpk, tsrc)
+        rows["decode_attn_32k"] = bench_attn(dev, max(100, args.steps // 10), args.warmup)
         torch.cuda.empty_cache()
         if cpu_rows:
             rows["tiny_draft_M1"]["cpu_baseline"] = cpu_baseline_tiny()

@@ -358,6 +358,35 @@ mtp_status mtp_prefill_kv(const uint16_t* embed, int64_t vocab, const int32_t* t
                           void* ws, size_t ws_bytes, int32_t* dev_err, void* stream);
 
 /* ---------------------------------------------------------------------------------
+ * mtp_paged_decode_attn -- single-token decode attention of the drafter over its paged
+ * E4M3 KV cache (the cache mtp_prefill_kv writes).
+ * Source: [new.rs] MtpHead::new (one attention layer with its own paged KV cache, block
+ * size 16, FP8 cache fed unit K/V scales by default, a single-token decode-attention
+ * kernel for that FP8 cache); [mtp_head.rs] module docs (attention follows fc);
+ * [v4_mtp.rs] forward_one step 4 (cache row p at block_table[p / bs] * bs + p % bs).
+ * The pages print no formula; this is the standard one, per query head i with kv head
+ * g = i / (nq / nkv), over the sequence's cache rows p = 0 .. seq_len - 1:
+ *   s_p = scale * sum_d q[i, d] k_scale e4m3(k_cache[(slot(p) * nkv + g) * hd + d])
+ *   out[i, d] = bf16(sum_p softmax(s)_p v_scale e4m3(v_cache[(slot(p) * nkv + g) * hd + d]))
+ * (fp32 sums, fp32 softmax). A row whose block is missing (p / block_size >= n_table) or
+ * out of range is skipped and sets MTP_DEVFLAG_BAD_SLOT; no readable row -> zeros.
+ *   q (device) bf16 [nq, hd]; k_cache, v_cache (device) u8 [num_blocks, block_size, nkv,
+ *   hd], 16-byte aligned; block_table (device) i32 [n_table]; out (device) bf16 [nq, hd];
+ *   dev_err i32 [1] or NULL; ws (device) >= mtp_paged_decode_attn_ws_bytes(nq, hd,
+ *   seq_len) bytes, 16-byte aligned (per-piece partial sums; no initial contents).
+ * Requires hd in {64, 128, 256}, nq % nkv == 0, nq / nkv <= 16, scale >= 0 (the usual
+ * choice is 1 / sqrt(hd)), k_scale, v_scale > 0. Two kernels on `stream`: one CTA per kv
+ * head and 256 cache rows (the K and V rows read once), then a merge per query head.
+ * ------------------------------------------------------------------------------ */
+size_t mtp_paged_decode_attn_ws_bytes(int32_t nq, int32_t hd, int64_t seq_len);
+mtp_status mtp_paged_decode_attn(const uint16_t* q, int32_t nq, int32_t nkv, int32_t hd,
+                                 const uint8_t* k_cache, const uint8_t* v_cache,
+                                 const int32_t* block_table, int64_t n_table, int32_t block_size,
+                                 int64_t num_blocks, int64_t seq_len, float k_scale, float v_scale,
+                                 float scale, uint16_t* out, int32_t* dev_err, void* ws,
+                                 size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------
  * Stage checks of the prefill, each through the code the prefill itself runs:
  * mtp_debug_gemm_bf16: C = bf16(A . B^T), A bf16 [M, K], B bf16 [N, K], C bf16 [M, N]
  *   (the tcgen05 GEMM); requires N % 256 == 0, K % 64 == 0, 16-byte aligned pointers.

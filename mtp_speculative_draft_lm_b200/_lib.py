@@ -38,7 +38,8 @@ EXPORTS = (
     "mtp_lm_head_host_ws_bytes", "mtp_lm_head_argmax_host",
     "mtp_lm_head_shard_partial", "mtp_argmax_merge_partials",
     "mtp_debug_encode_e4m3", "mtp_debug_encode_e2m1", "mtp_nvfp4_scale_pitch",
-    "mtp_debug_wait_timeout", "mtp_draft_step",
+    "mtp_debug_wait_timeout", "mtp_draft_step", "mtp_paged_decode_attn_ws_bytes",
+    "mtp_paged_decode_attn",
     "mtp_noalloc_scratch_bytes", "mtp_lm_head_argmax_noalloc",
     "mtp_prefill_ws_bytes", "mtp_prefill_kv", "mtp_debug_gemm_bf16", "mtp_debug_kv_write",
 )
@@ -94,6 +95,10 @@ _SIGS = {
     "mtp_lm_head_argmax_noalloc": (C.c_int, [_W, _I64, _P, _I32, _P, _I64, _I64, _P, _P, _P,
                                              _P, _P]),
     "mtp_debug_wait_timeout": (C.c_int, [_I32, _I64, _P, _P, _P]),
+    "mtp_paged_decode_attn_ws_bytes": (_SZ, [_I32, _I32, _I64]),
+    "mtp_paged_decode_attn": (C.c_int, [_P, _I32, _I32, _I32, _P, _P, _P, _I64, _I32, _I64,
+                                        _I64, C.c_float, C.c_float, C.c_float, _P, _P, _P, _SZ,
+                                        _P]),
     "mtp_draft_step": (C.c_int, [_P, _I64, _P, _P, _I32, _I32, _P, _P, C.c_float, _P, _P, _I64,
                                  _P, _I64, _I64, _P, _P, _P, _P, _P]),
     "mtp_debug_encode_e4m3": (C.c_int, [_P, _I64, _P, _P]),
@@ -292,6 +297,20 @@ def mtp_draft_step(embed, vocab, token_ids, hidden, M, h, w_norm_embed, w_norm_h
                                  _ptr(head), n_eff, _ptr(mask), mask_words, mask_stride_words,
                                  _ptr(out_y), _ptr(out_idx), _ptr(out_val), _ptr(dev_err),
                                  _stream(stream)), "mtp_draft_step")
+
+
+def mtp_paged_decode_attn_ws_bytes(nq, hd, seq_len) -> int:
+    return load().mtp_paged_decode_attn_ws_bytes(nq, hd, seq_len)
+
+
+def mtp_paged_decode_attn(q, nq, nkv, hd, k_cache, v_cache, block_table, n_table, block_size,
+                          num_blocks, seq_len, k_scale, v_scale, scale, out, dev_err, ws, ws_bytes,
+                          stream=None):
+    _check(load().mtp_paged_decode_attn(_ptr(q), nq, nkv, hd, _ptr(k_cache), _ptr(v_cache),
+                                        _ptr(block_table), n_table, block_size, num_blocks,
+                                        seq_len, float(k_scale), float(v_scale), float(scale),
+                                        _ptr(out), _ptr(dev_err), _ptr(ws), ws_bytes,
+                                        _stream(stream)), "mtp_paged_decode_attn")
 
 
 def mtp_debug_wait_timeout(which, limit_cycles, counter, dev_err, stream=None):

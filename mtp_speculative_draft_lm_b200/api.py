@@ -236,6 +236,24 @@ def draft_step(embed, token_ids, hidden, w_norm_embed, w_norm_hidden, eps, fc, h
     return out_idx, out_val, out_y
 
 
+def paged_decode_attn(q, nkv, k_cache, v_cache, block_table, seq_len, k_scale=1.0, v_scale=1.0,
+                      scale=None, out=None, ws=None, dev_err=None, stream=None):
+    """Single-token decode attention of q [nq, hd] (bf16) over cache rows 0 .. seq_len - 1 of
+    a paged E4M3 cache [num_blocks, block_size, nkv, hd]; returns (out, ws)."""
+    nq, hd = q.shape
+    num_blocks, block_size = k_cache.shape[0], k_cache.shape[1]
+    scale = 1.0 / float(hd) ** 0.5 if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((nq, hd), dtype=torch.bfloat16, device=q.device)
+    nbytes = L.mtp_paged_decode_attn_ws_bytes(nq, hd, seq_len)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.empty((nbytes,), dtype=torch.uint8, device=q.device)
+    L.mtp_paged_decode_attn(q, nq, nkv, hd, k_cache, v_cache, block_table, block_table.numel(),
+                            block_size, num_blocks, seq_len, k_scale, v_scale, scale, out, dev_err,
+                            ws, ws.numel(), stream)
+    return out, ws
+
+
 def aligned_empty(nbytes: int, align: int, device) -> torch.Tensor:
     """A uint8 device buffer of nbytes whose address is a multiple of align (torch only
     promises 512 bytes)."""

@@ -10,6 +10,8 @@ namespace {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+bool finite_pos(float v) { return v > 0.f && v < 3.0e38f; }
+
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
 mtp_status from_cuda(cudaError_t e) {
@@ -332,12 +334,39 @@ mtp_status mtp_draft_step(const uint16_t* embed, int64_t vocab, const int32_t* t
                                             as_stream(stream)));
 }
 
+size_t mtp_paged_decode_attn_ws_bytes(int32_t nq, int32_t hd, int64_t seq_len) {
+    if (nq < 1 || hd < 1 || seq_len < 1) return 0;
+    return mtp::attn_ws_bytes(nq, hd, seq_len);
+}
+
+mtp_status mtp_paged_decode_attn(const uint16_t* q, int32_t nq, int32_t nkv, int32_t hd,
+                                 const uint8_t* k_cache, const uint8_t* v_cache,
+                                 const int32_t* block_table, int64_t n_table, int32_t block_size,
+                                 int64_t num_blocks, int64_t seq_len, float k_scale, float v_scale,
+                                 float scale, uint16_t* out, int32_t* dev_err, void* ws,
+                                 size_t ws_bytes, void* stream) {
+    if (!q || !k_cache || !v_cache || !block_table || !out) return MTP_ERR_INVALID_ARG;
+    if (nq < 1 || nkv < 1 || nq % nkv || n_table < 1 || block_size < 1 || num_blocks < 1 ||
+        seq_len < 1 || !finite_pos(k_scale) || !finite_pos(v_scale) || !(scale >= 0.f) ||
+        !(scale < 3.0e38f))
+        return MTP_ERR_INVALID_ARG;
+    if ((hd != 64 && hd != 128 && hd != 256) || nq / nkv > mtp::attn_max_group() ||
+        seq_len > ((int64_t)1 << 31) * 128)
+        return MTP_ERR_UNSUPPORTED;
+    if (!aligned(q, 2) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(block_table, 4) || !aligned(out, 2) || !aligned(dev_err, 4))
+        return MTP_ERR_INVALID_ARG;
+    if (!ws || !aligned(ws, 16) || ws_bytes < mtp::attn_ws_bytes(nq, hd, seq_len))
+        return MTP_ERR_WORKSPACE;
+    return from_cuda(mtp::attn_launch(q, nq, nkv, hd, k_cache, v_cache, block_table, n_table,
+                                      block_size, num_blocks, seq_len, k_scale, v_scale, scale,
+                                      out, dev_err, ws, as_stream(stream)));
+}
+
 size_t mtp_prefill_ws_bytes(int64_t chunk_rows, int32_t h, int32_t nkv, int32_t hd) {
     if (chunk_rows < 1 || h < 1 || nkv < 1 || hd < 2) return 0;
     return mtp::prefill_ws_bytes(chunk_rows, h, nkv, hd);
 }
-
-static bool finite_pos(float v) { return v > 0.f && v < 3.0e38f; }
 
 mtp_status mtp_prefill_kv(const uint16_t* embed, int64_t vocab, const int32_t* token_ids,
                           const uint16_t* hidden, int64_t R, int32_t h,

@@ -150,6 +150,15 @@ cudaError_t draft_step_launch(const uint16_t* embed, int64_t vocab, const int32_
                               int64_t mask_words, int64_t mask_stride, uint16_t* out_y,
                               int32_t* out_idx, float* out_val, int32_t* dev_err, cudaStream_t s);
 
+// Single-token paged decode attention over the E4M3 KV cache (attn.cu).
+int attn_max_group();
+size_t attn_ws_bytes(int nq, int hd, int64_t seq_len);
+cudaError_t attn_launch(const uint16_t* q, int nq, int nkv, int hd, const uint8_t* k_cache,
+                        const uint8_t* v_cache, const int32_t* block_table, int64_t n_table,
+                        int block_size, int64_t num_blocks, int64_t seq_len, float k_scale,
+                        float v_scale, float scale, uint16_t* out, int32_t* dev_err, void* ws,
+                        cudaStream_t s);
+
 // Self-check of the bounded waits (selfcheck.cu): which 0 waits on an mbarrier phase that
 // nothing completes, 1 on a global counter (device u32, kept at 0 by the caller) that
 // nothing increments; either gives up after limit_cycles and sets DEVFLAG_TIMEOUT.

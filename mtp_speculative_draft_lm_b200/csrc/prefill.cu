@@ -313,7 +313,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 4);
+            mbar_init(&tempty[b], 1);  // one epilogue thread, after the epilogue warps sync
         }
         for (int q = 0; q < kFifo; ++q) {
             mbar_init(&qfull[q], 1);

@@ -307,3 +307,22 @@ def test_draft_step_rejects(lib):
     assert ds(M=5) == L.MTP_ERR_UNSUPPORTED         # up to 4 inputs
     assert ds(h=2048) == L.MTP_ERR_UNSUPPORTED      # up to hidden 1024
     assert ds(head=B2 + 8) == L.MTP_ERR_INVALID_ARG  # 16-byte aligned head
+
+
+def test_paged_decode_attn_rejects(lib):
+    ws = L.mtp_paged_decode_attn_ws_bytes(8, 128, 300)
+    assert ws == 2 * 8 * 130 * 4  # two 256-row pieces x heads x (hd + max + sum) floats
+
+    def at(q=A, nq=8, nkv=2, hd=128, seq=300, ks=1.0, sc=0.1, w=0x40000, wb=ws, kc=B2):
+        return st("mtp_paged_decode_attn", q, nq, nkv, hd, kc, B2, OUT, 20, 16, 30, seq, ks, 1.0,
+                  sc, OUT, None, w, wb, None)
+    assert at(q=None) == L.MTP_ERR_INVALID_ARG
+    assert at(nq=9) == L.MTP_ERR_INVALID_ARG        # nq % nkv
+    assert at(seq=0) == L.MTP_ERR_INVALID_ARG
+    assert at(ks=0.0) == L.MTP_ERR_INVALID_ARG
+    assert at(sc=-1.0) == L.MTP_ERR_INVALID_ARG
+    assert at(hd=96) == L.MTP_ERR_UNSUPPORTED
+    assert at(nq=34, nkv=2) == L.MTP_ERR_UNSUPPORTED  # at most 16 query heads per kv head
+    assert at(kc=B2 + 8) == L.MTP_ERR_INVALID_ARG
+    assert at(w=None) == L.MTP_ERR_WORKSPACE
+    assert at(wb=ws - 4) == L.MTP_ERR_WORKSPACE

@@ -37,7 +37,8 @@ def gemm(A, B):
     return u16_of(C)
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (300, 512, 640), (1000, 1024, 4096)])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (300, 512, 640), (1000, 1024, 4096),
+                                   (2048, 4096, 256)])  # the last: several tiles per SM
 def test_gemm_matches_numpy(orc, M, N, K):
     A = synth.as_u16(synth.normal_bf16(synth._gen(M + N), (M, K), 1.0))
     B = synth.as_u16(synth.normal_bf16(synth._gen(K + 3), (N, K), 0.02))
@@ -226,6 +227,28 @@ def test_prefill_lanes_and_graph_capture_agree(orc):
     assert np.array_equal(kc.cpu().numpy(), outs[0][0])
     assert np.array_equal(vc.cpu().numpy(), outs[0][1])
     check_rows(orc, d, outs[0][0], outs[0][1], np.arange(0, 700, 7))
+
+
+def test_prefill_many_tiles_per_sm(orc):
+    """More tiles than SMs (hidden 1,024, 8 KV heads x 128, chunks of 256 rows: 208 tiles),
+    so every SM runs several prologue, fc and k/v tiles back to back; both lane counts."""
+    d = synth.prefill_inputs(seed=83, R=2048, vocab=900, h=1024, nkv=8, hd=128)
+    dev = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    nb = int(d["num_blocks"])
+    full = L.mtp_prefill_ws_bytes(256, 1024, 8, 128)
+    outs = []
+    for nbytes in (full, full // 2):
+        kc, vc = new_caches(nb, 16, 8, 128)
+        err = torch.zeros((1,), dtype=torch.int32, device="cuda")
+        ws = api.aligned_empty(nbytes, 1024, "cuda")
+        api.prefill_kv(dev, kc, vc, chunk_rows=256, ws=ws, dev_err=err)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        outs.append((kc.cpu().numpy(), vc.cpu().numpy()))
+    assert np.array_equal(outs[0][0], outs[1][0]) and np.array_equal(outs[0][1], outs[1][1])
+    rows = np.unique(np.concatenate([[0, 255, 256, 2047],
+                                     np.random.default_rng(6).choice(2048, 40, replace=False)]))
+    check_rows(orc, d, outs[0][0], outs[0][1], rows)
 
 
 def test_prefill_ragged_chunks_and_one_row(orc):

@@ -266,11 +266,17 @@ def test_full_tables(orc, cfg, fmt):
             assert np.array_equal(got[0], d["second"][:M])
 
 
+# Inputs for which the masked sweep (which reads only allowed rows) and the unmasked one
+# run the same kernel, so that their logits must agree bit for bit.
+SAME_KERNEL_M = {0: 8, 1: 6, 2: 2}
+
+
 @pytest.mark.parametrize("cfg,fmt", FULL, ids=["bf16", "fp8", "nvfp4"])
 def test_masked_full_tables(orc, cfg, fmt):
     """Grammar masks keeping 1% and 50% of the tokens on the full tables (the masked sweep
     reads only the rows some input allows): the masked argmax and value against the oracle,
-    every disallowed logit -inf, and every allowed logit identical to the unmasked sweep's."""
+    every disallowed logit -inf, every allowed logit within tolerance of the oracle on a
+    sample, and identical to the unmasked sweep's where both run the same kernel."""
     Ms = (1, 4, 8) if fmt != 2 else (1, 2, 4)
     Mmax = max(Ms)
     N, K = cfg["N"], cfg["K"]
@@ -280,7 +286,8 @@ def test_masked_full_tables(orc, cfg, fmt):
     table = device_table(q, fmt, N, K)
     head = api.LmHead(table)
     ref_l, _, _, _ = oracle_sweep(orc, q, fmt, K, x)
-    _, _, dense_lg, _ = run_sweep(table, x, head=head)
+    dense = {M: run_sweep(table, x[:M], head=head)[2] for M in Ms if M <= SAME_KERNEL_M[fmt]}
+    sample = np.random.default_rng(fmt).choice(N, 5000, replace=False)
     for keep in (0.01, 0.5):
         allowed, words = synth.keep_mask(int(keep * 1000) + fmt, Mmax, N, keep)
         W = words.shape[1]
@@ -293,12 +300,17 @@ def test_masked_full_tables(orc, cfg, fmt):
                 assert_argmax(int(idx[m]), ref_l[m], a)
                 assert_close([val[m]], [ref_l[m][a].max()], "masked out_val")
                 assert np.all(lg[m][~a] == 0xFF80)
-                assert np.array_equal(lg[m][a], dense_lg[m][a]), (keep, M, m)
+                rs = sample[a[sample]]
+                assert_close(bf16_bits_to_f64(lg[m][rs]), ref_l[m][rs], "masked logits sample")
+                if M in dense:
+                    assert np.array_equal(lg[m][a], dense[M][m][a]), (keep, M, m)
         # one mask shared by every input (stride 0)
-        idx, val, lg, _ = run_sweep(table, x[:4], head=head, mask=words[0], mask_words=W, stride=0)
-        for m in range(4):
+        idx, val, lg, _ = run_sweep(table, x[:2], head=head, mask=words[0], mask_words=W, stride=0)
+        for m in range(2):
             assert_argmax(int(idx[m]), ref_l[m], allowed[0])
-            assert np.array_equal(lg[m][allowed[0]], dense_lg[m][allowed[0]])
+            if 2 <= SAME_KERNEL_M[fmt]:
+                two = run_sweep(table, x[:2], head=head)[2]
+                assert np.array_equal(lg[m][allowed[0]], two[m][allowed[0]])
 
 
 def oracle_logprobs(orc, ref_l, mask=None, mask_words=0, stride=0):
