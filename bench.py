@@ -644,7 +644,8 @@ def main():
                     help="sweep a smaller table of this many rows (profiling cases)")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the tiny-draft and prefill rows")
-    ap.add_argument("--only", default="", help="profiling: run only 'prefill' or 'tiny'")
+    ap.add_argument("--only", default="",
+                    help="profiling: run only 'prefill', 'tiny', 'attn' or 'masked'")
     ap.add_argument("--ms", default="",
                     help="profiling: time only these input counts (comma list, e.g. 16,32), "
                          "seeded N(0, 1) inputs")
@@ -673,6 +674,19 @@ def main():
             out = bench_prefill(dev, 2, tpk, tsrc, args.prefill_rows)
         elif args.only == "attn":
             out = bench_attn(dev, args.steps, args.warmup)
+        elif args.only == "masked":  # profiling: the masked M = 1 sweep alone
+            out = {}
+            for fmt in args.formats.split(","):
+                cfg, d, table, _ = build_table(fmt, dev, args.rows)
+                head = api.LmHead(table)
+                words = d["mask"].shape[1]
+                m = torch.from_numpy(d["mask"][:1].reshape(-1)).to(dev)
+                tm = time_sweep(head, d["x"][:1].to(dev), args.steps, args.warmup, 1, stream,
+                                mask=m, mask_words=words)
+                out[f"{fmt}_M1_masked"] = {"us_per_draft": tm["mean_ms"] * 1e3,
+                                           "argmax_ok": int(tm["idx"][0]) == int(d["second"][0])}
+                del head, table, d
+                torch.cuda.empty_cache()
         else:
             out = bench_tiny_draft(dev, args.steps, args.warmup)
         print(json.dumps({"only": args.only, **out}), flush=True)

@@ -374,7 +374,8 @@ mtp_status mtp_prefill_kv(const uint16_t* embed, int64_t vocab, const int32_t* t
  *   hd], 16-byte aligned; block_table (device) i32 [n_table]; out (device) bf16 [nq, hd];
  *   dev_err i32 [1] or NULL; ws (device) >= mtp_paged_decode_attn_ws_bytes(nq, hd,
  *   seq_len) bytes, 16-byte aligned (per-piece partial sums; no initial contents).
- * Requires hd in {64, 128, 256}, nq % nkv == 0, nq / nkv <= 16, scale >= 0 (the usual
+ * Requires hd in {64, 128, 256}, nq % nkv == 0, nq / nkv <= 16, seq_len <= 2,097,152
+ * (MTP_ERR_UNSUPPORTED otherwise), scale >= 0 (the usual
  * choice is 1 / sqrt(hd)), k_scale, v_scale > 0. Two kernels on `stream`: one CTA per kv
  * head and 256 cache rows (the K and V rows read once), then a merge per query head.
  * ------------------------------------------------------------------------------ */

@@ -351,7 +351,7 @@ mtp_status mtp_paged_decode_attn(const uint16_t* q, int32_t nq, int32_t nkv, int
         !(scale < 3.0e38f))
         return MTP_ERR_INVALID_ARG;
     if ((hd != 64 && hd != 128 && hd != 256) || nq / nkv > mtp::attn_max_group() ||
-        seq_len > ((int64_t)1 << 31) * 128)
+        seq_len > (int64_t)8192 * 256)
         return MTP_ERR_UNSUPPORTED;
     if (!aligned(q, 2) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
         !aligned(block_table, 4) || !aligned(out, 2) || !aligned(dev_err, 4))

@@ -30,6 +30,7 @@ constexpr int kAPos = 256;      // positions per CTA
 constexpr int kAThreads = 128;
 constexpr int kAMaxGroup = 16;  // query heads per kv head
 constexpr int kAMaxHd = 256;
+constexpr int kAMaxPieces = 8192;  // cache rows up to 2M (the merge keeps a factor per piece)
 
 struct AttnParams {
     const uint16_t* q;  // [nq, hd] bf16
@@ -192,23 +193,56 @@ __global__ void __launch_bounds__(kAThreads) attn_piece_kernel(const __grid_cons
     }
 }
 
-// One CTA per query head: merges the pieces in order, out = sum_s e^(m_s - M) acc_s /
-// sum_s e^(m_s - M) l_s (zero when no row was readable), as bf16.
+// One CTA per query head: out = sum_s e^(m_s - M) acc_s / sum_s e^(m_s - M) l_s (zero
+// when no row was readable), as bf16. The pieces' (max, sum) pairs are loaded in parallel
+// and their factors folded in a fixed order; each thread then sums its dimension over the
+// pieces with many loads in flight.
 __global__ void __launch_bounds__(kAMaxHd) attn_merge_kernel(const __grid_constant__ AttnParams p) {
+    __shared__ float fac[kAMaxPieces];
+    __shared__ float red[kAMaxHd / 32];
+    __shared__ float tot[2];
     const int i = blockIdx.x, d = threadIdx.x, hd = p.hd;
+    const int lane = d & 31, warp = d >> 5;
     pdl_wait();
-    float M = -INFINITY;
-    for (int s = 0; s < p.pieces; ++s) M = fmaxf(M, p.part[((int64_t)s * p.nq + i) * (hd + 2)]);
-    float L = 0.f, a = 0.f;
-    if (M > -INFINITY) {
-        for (int s = 0; s < p.pieces; ++s) {
-            const float* src = p.part + ((int64_t)s * p.nq + i) * (hd + 2);
-            if (src[0] == -INFINITY) continue;
-            const float f = expf(src[0] - M);
-            L = fmaf(f, src[1], L);
-            if (d < hd) a = fmaf(f, src[2 + d], a);
-        }
+    const int64_t rs = (int64_t)p.nq * (hd + 2);  // floats between a head's pieces
+    const float* base = p.part + (int64_t)i * (hd + 2);
+    float mloc = -INFINITY;
+    for (int s = d; s < p.pieces; s += kAMaxHd) mloc = fmaxf(mloc, base[s * rs]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, o));
+    if (lane == 0) red[warp] = mloc;
+    __syncthreads();
+    if (d == 0) {
+        float M = -INFINITY;
+        for (int w = 0; w < kAMaxHd / 32; ++w) M = fmaxf(M, red[w]);
+        tot[0] = M;
     }
+    __syncthreads();
+    const float M = tot[0];
+    for (int s = d; s < p.pieces; s += kAMaxHd) {
+        const float m = base[s * rs];
+        fac[s] = (M == -INFINITY || m == -INFINITY) ? 0.f : expf(m - M);
+    }
+    __syncthreads();
+    if (d == 0) {  // the denominator in piece order
+        float L = 0.f;
+        for (int s = 0; s < p.pieces; ++s) L = fmaf(fac[s], base[s * rs + 1], L);
+        tot[1] = L;
+    }
+    float a = 0.f;
+    if (d < hd) {
+        int s = 0;
+        for (; s + 8 <= p.pieces; s += 8) {  // eight independent loads in flight
+            float v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = base[(s + j) * rs + 2 + d];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) a = fmaf(fac[s + j], v[j], a);
+        }
+        for (; s < p.pieces; ++s) a = fmaf(fac[s], base[s * rs + 2 + d], a);
+    }
+    __syncthreads();
+    const float L = tot[1];
     if (d < hd) p.out[(int64_t)i * hd + d] = f32_to_bf16(L > 0.f ? a / L * p.v_scale : 0.f);
 }
 

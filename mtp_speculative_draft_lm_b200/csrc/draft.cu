@@ -16,8 +16,9 @@
 // warp keeping 16 rows' 16-byte loads in flight; per input the CTAs' (max, lowest row)
 // partials go to CTA 0's shared memory and CTA 0 writes the result. Two cluster barriers,
 // no global workspace. Launched with programmatic stream serialization, so in a chain of
-// drafts the next step's launch overlaps this one's end (it waits for it before reading
-// the token and hidden rows this step writes).
+// drafts the next step's launch overlaps this one's end: it prefetches its weight rows into
+// L1 first and waits for the previous step only before reading the token and hidden rows
+// that step writes.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -123,6 +124,22 @@ __global__ void __launch_bounds__(kDThreads, 1) draft_step_kernel(const __grid_c
     const uint32_t rank = cluster_rank(), CL = cluster_size();
     const int M = p.M, h = p.h, h2 = 2 * h;
     pdl_launch_dependents();
+    // The weights never change: pull this CTA's fc rows and head rows into L1 before
+    // waiting for the previous step, so that their latency overlaps its end.
+    {
+        const int rows_per = (h + (int)CL - 1) / (int)CL;
+        const int f0 = (int)rank * rows_per, f1 = min(h, f0 + rows_per);
+        const int64_t per = (p.n + CL - 1) / CL;
+        const int64_t q0 = (int64_t)rank * per, q1 = min(p.n, q0 + per);
+        const int64_t fl = (int64_t)(f1 - f0) * h2 * 2 / 128;  // 128-byte lines
+        const int64_t hl = (q1 - q0) * h * 2 / 128;
+        const uint8_t* fb = reinterpret_cast<const uint8_t*>(p.fc + (int64_t)f0 * h2);
+        const uint8_t* hb = reinterpret_cast<const uint8_t*>(p.head + q0 * h);
+        for (int64_t i = tid; i < fl + hl; i += kDThreads) {
+            const uint8_t* a = i < fl ? fb + 128 * i : hb + 128 * (i - fl);
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(a));
+        }
+    }
     pdl_wait();  // tokens and hidden rows may come from the previous step
 
     // 1. concat rows (every CTA): two RMSNorms with plain weights, bf16 rounding
@@ -173,7 +190,7 @@ __global__ void __launch_bounds__(kDThreads, 1) draft_step_kernel(const __grid_c
 #pragma unroll
         for (int m = 0; m < MM; ++m) acc[m] = 0.f;
         for (int c = lane; c < h2 / 8; c += 32) {
-            const uint4 a = ldg_stream(frow + 8 * c);
+            const uint4 a = __ldg(reinterpret_cast<const uint4*>(frow + 8 * c));
 #pragma unroll
             for (int m = 0; m < MM; ++m)
                 if (m < M) acc[m] += dot8(a, &cs[m][8 * c]);
@@ -230,8 +247,9 @@ __global__ void __launch_bounds__(kDThreads, 1) draft_step_kernel(const __grid_c
             uint4 a[RPW];
 #pragma unroll
             for (int j = 0; j < RPW; ++j)
-                a[j] = (c < pieces && g + j < n1) ? ldg_stream(p.head + (g + j) * h + 8 * c)
-                                                  : make_uint4(0, 0, 0, 0);
+                a[j] = (c < pieces && g + j < n1)
+                           ? __ldg(reinterpret_cast<const uint4*>(p.head + (g + j) * h + 8 * c))
+                           : make_uint4(0, 0, 0, 0);
             if (c < pieces) {
 #pragma unroll
                 for (int j = 0; j < RPW; ++j)
