@@ -1799,7 +1799,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
 
 // ---------------------------------------------------------------- NVFP4 tcgen05 sweep
 // NVFP4 tables with 3-32 inputs run the contraction on the tcgen05 tensor cores with A in
-// tensor memory. Four decode warps turn each table row's E2M1 codes times their E4M3 block
+// tensor memory. Eight decode warps (two per lane quarter, each half of every segment)
+// turn each table row's E2M1 codes times their E4M3 block
 // scale into f16 -- exact: a code has at most 2 significant bits and a scale 4, and every
 // product lies in [2^-10, 2688] -- and store them with tcgen05.st into tensor memory, one
 // table row per lane; one thread issues tcgen05.mma kind::f16 with A from tensor memory and
@@ -1812,7 +1813,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
 // 128-column A slots, so decoding runs a slot ahead of the MMAs. Four epilogue warps drain
 // the double-buffered accumulators as the tcgen05 sweep does (per input a running max,
 // lowest row, sum of exp), and the CTA partials go through the shared last-CTA fold.
-constexpr int kQThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2-5 decode, warps 6-9 epilogue
+constexpr int kQDecWarps = 8;    // two per tensor-memory lane quarter, each half of a segment
+constexpr int kQThreads = (2 + kQDecWarps + 4) * 32;  // TMA, MMA, decode, four epilogue warps
 constexpr int kQSlots = 3;      // tensor-memory A slots (one half's segment each)
 constexpr int kQAcol = 128;     // first A column; the accumulators use columns [0, 4N)
 constexpr int kQHead = 3072;    // barriers, misc, factors, fold; then the ring
@@ -1835,8 +1837,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
     constexpr int TR = 128 * H;  // table rows per tile
     extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
-    uint64_t* empty = full + kMaxStages;   // 4 decode warps + the MMA commit
-    uint64_t* afull = empty + kMaxStages;  // [kQSlots] 4 decode warps
+    uint64_t* empty = full + kMaxStages;   // the decode warps + the MMA commit
+    uint64_t* afull = empty + kMaxStages;  // [kQSlots] the decode warps
     uint64_t* aempty = afull + kQSlots;    // [kQSlots] the MMA commit
     uint64_t* tfull = aempty + kQSlots;    // [2] the tile index posted + the MMA commit
     uint64_t* tempty = tfull + 2;          // [2] 4 epilogue warps
@@ -1863,10 +1865,10 @@ __global__ void __launch_bounds__(kQThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 5);
+            mbar_init(&empty[s], kQDecWarps + 1);
         }
         for (int k = 0; k < kQSlots; ++k) {
-            mbar_init(&afull[k], 4);
+            mbar_init(&afull[k], kQDecWarps);
             mbar_init(&aempty[k], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -1994,10 +1996,12 @@ __global__ void __launch_bounds__(kQThreads, 1)
         if (lane == 0) umma_commit(done);
         __syncwarp();
         mbar_wait_bounded(done, 0u, nullptr);
-    } else if (warp < 6) {
+    } else if (warp < 2 + kQDecWarps) {
         // ---------------- decode warps: tensor-memory lane quarter q = warp % 4, one table
-        // row per thread and half (row h * 128 + 32 q + lane of the tile)
+        // row per thread and half (row h * 128 + 32 q + lane of the tile); warp pair
+        // (q, part) splits each segment's four 64-element pieces two and two
         const int q = warp & 3;
+        const int part = (warp - 2) >> 2;  // 0 or 1
         int slot = 0, aslot = 0;
         uint32_t phase = 0, aphase = 0;
         while (true) {
@@ -2021,18 +2025,21 @@ __global__ void __launch_bounds__(kQThreads, 1)
                         tc_fence_after();
                         // the row's 128 code bytes (8 chunks, 128-byte swizzle) and 16 scales
                         const uint8_t* crow = st + (size_t)sg * (TR * 128) + (size_t)r * 128;
-                        const uint4 sc = lds128(st + code_b + (size_t)r * 16 * segs + sg * 16);
-                        const uint32_t scw[4] = {sc.x, sc.y, sc.z, sc.w};
+                        // this warp's eight block scales (blocks 8 part .. 8 part + 7)
+                        const uint2 sc = *reinterpret_cast<const uint2*>(
+                            st + code_b + (size_t)r * 16 * segs + sg * 16 + 8 * part);
+                        const uint32_t scw[2] = {sc.x, sc.y};
                         const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) +
                                                (uint32_t)(kQAcol + aslot * 128);
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {  // 64 elements (two chunks, four blocks)
+                        for (int jj = 0; jj < 2; ++jj) {  // 64 elements (two chunks, four blocks)
+                            const int j = 2 * part + jj;
                             const uint4 c0 = lds128(crow + (((2 * j) ^ (r & 7)) << 4));
                             const uint4 c1 = lds128(crow + (((2 * j + 1) ^ (r & 7)) << 4));
                             const uint32_t wd[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
                             // the four blocks' E4M3 scales as f16, each in both halves
-                            const uint32_t s01 = e4m3x2_to_f16x2((uint16_t)(scw[j] & 0xFFFFu));
-                            const uint32_t s23 = e4m3x2_to_f16x2((uint16_t)(scw[j] >> 16));
+                            const uint32_t s01 = e4m3x2_to_f16x2((uint16_t)(scw[jj] & 0xFFFFu));
+                            const uint32_t s23 = e4m3x2_to_f16x2((uint16_t)(scw[jj] >> 16));
                             const uint32_t bs[4] = {__byte_perm(s01, 0, 0x1010), __byte_perm(s01, 0, 0x3232),
                                                     __byte_perm(s23, 0, 0x1010), __byte_perm(s23, 0, 0x3232)};
                             uint32_t out[32];
@@ -2069,7 +2076,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
         // (one table row per lane); per tile and input the warp folds its 32 rows with
         // shuffles and lane m keeps input m's running (max, lowest row, sum of exp)
         const int q = warp & 3;
-        const int ew = warp - 6;  // 0..3
+        const int ew = warp - (2 + kQDecWarps);  // 0..3
         const bool lp = p.out_logprob != nullptr || p.out_partial != nullptr;
         pdl_wait();
         if (ew == 0) {

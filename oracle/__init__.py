@@ -84,6 +84,13 @@ def lib():
                                         _p, _p, _i32, _i32, C.c_double, _p, _i64, _p,
                                         _i64, _i32, _i64, C.c_float, C.c_float, _p,
                                         _i64, _p, _p, _p, _p, _p, _p]),
+            "orc_rmsnorm_row_mode": (None, [_p, _p, _i64, C.c_double, _i32, _p]),
+            "orc_combine_mode": (_i32, [_p, _i64, _p, _p, _i32, _i32, _p, _p, C.c_double, _i32,
+                                        _p, _p, _p]),
+            "orc_prefill_rows_ext": (_i32, [_p, _i64, _p, _p, _i32, _p, _p, C.c_double, _p,
+                                            _p, _p, _i32, _i32, C.c_double, _p, _i64, _p,
+                                            _i64, _i32, _i64, C.c_float, C.c_float, _i32, _p,
+                                            _p, _i64, _p, _p, _p, _p, _p, _p]),
             "orc_paged_decode_attn": (_i32, [_p, _i32, _i32, _i32, _p, _p, _p, _i64, _i32,
                                              _i64, _i64, C.c_double, C.c_double, C.c_double,
                                              _p]),
@@ -184,25 +191,26 @@ def dequant(fmt, data, k, row_scale=None, block_scale=None, global_scale=0.0, ro
 
 # ---- draft step (draft.c) ------------------------------------------------------
 
-def rmsnorm(x, w, eps):
+def rmsnorm(x, w, eps, norm_mode=0):
+    """orc_rmsnorm_row_mode: weights w (norm_mode 0) or 1 + w (norm_mode 1)."""
     x = _c(x, np.uint16)
     w = _c(w, np.uint16)
     y = np.empty_like(x)
-    lib().orc_rmsnorm_row(_ptr(x), _ptr(w), x.size, float(eps), _ptr(y))
+    lib().orc_rmsnorm_row_mode(_ptr(x), _ptr(w), x.size, float(eps), int(norm_mode), _ptr(y))
     return y
 
 
-def combine(embed, tokens, hidden, w_norm_embed, w_norm_hidden, eps, fc):
+def combine(embed, tokens, hidden, w_norm_embed, w_norm_hidden, eps, fc, norm_mode=0):
     embed = _c(embed, np.uint16)
     tokens = _c(tokens, np.int32)
     hidden = _c(hidden, np.uint16)
     M, h = hidden.shape
     concat = np.empty((M, 2 * h), dtype=np.uint16)
     y = np.empty((M, h), dtype=np.uint16)
-    flags = lib().orc_combine(_ptr(embed), embed.shape[0], _ptr(tokens), _ptr(hidden), M, h,
-                              _ptr(_c(w_norm_embed, np.uint16)),
-                              _ptr(_c(w_norm_hidden, np.uint16)), float(eps),
-                              _ptr(_c(fc, np.uint16)), _ptr(concat), _ptr(y))
+    flags = lib().orc_combine_mode(_ptr(embed), embed.shape[0], _ptr(tokens), _ptr(hidden), M, h,
+                                   _ptr(_c(w_norm_embed, np.uint16)),
+                                   _ptr(_c(w_norm_hidden, np.uint16)), float(eps), int(norm_mode),
+                                   _ptr(_c(fc, np.uint16)), _ptr(concat), _ptr(y))
     return y, concat, int(flags)
 
 
@@ -269,7 +277,7 @@ def kv_encode(vals_bf16, scale):
 
 def prefill_rows(embed, tokens, hidden, w_norm_embed, w_norm_hidden, eps, fc, wk, wv,
                  nkv, hd, rope_base, rope_pos, cache_start, block_table, block_size,
-                 num_blocks, k_scale, v_scale, rows):
+                 num_blocks, k_scale, v_scale, rows, norm_mode=0, k_norm=None):
     """Oracle K/V cache entries for the listed prompt rows.
 
     Returns dict with y [n,h], k_rot [n,nkv*hd], v [n,nkv*hd] (bf16 bits), k_codes,
@@ -288,13 +296,14 @@ def prefill_rows(embed, tokens, hidden, w_norm_embed, w_norm_hidden, eps, fc, wk
     vc = np.empty((n, kvd), dtype=np.uint8)
     sl = np.empty((n,), dtype=np.int64)
     bt = _c(block_table, np.int32)
-    flags = lib().orc_prefill_rows(
+    kn = None if k_norm is None else _c(k_norm, np.uint16)
+    flags = lib().orc_prefill_rows_ext(
         _ptr(embed), embed.shape[0], _ptr(_c(tokens, np.int32)), _ptr(hidden), h,
         _ptr(_c(w_norm_embed, np.uint16)), _ptr(_c(w_norm_hidden, np.uint16)), float(eps),
         _ptr(_c(fc, np.uint16)), _ptr(_c(wk, np.uint16)), _ptr(_c(wv, np.uint16)), nkv, hd,
         float(rope_base), _ptr(_c(rope_pos, np.int32)), int(cache_start), _ptr(bt), bt.size,
-        int(block_size), int(num_blocks), float(k_scale), float(v_scale), _ptr(rows), n,
-        _ptr(y), _ptr(k_rot), _ptr(v), _ptr(kc), _ptr(vc), _ptr(sl))
+        int(block_size), int(num_blocks), float(k_scale), float(v_scale), int(norm_mode),
+        _ptr(kn), _ptr(rows), n, _ptr(y), _ptr(k_rot), _ptr(v), _ptr(kc), _ptr(vc), _ptr(sl))
     return dict(y=y, k_rot=k_rot, v=v, k_codes=kc, v_codes=vc, slot=sl, flags=int(flags))
 
 

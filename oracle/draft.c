@@ -58,16 +58,26 @@ int32_t orc_num_threads(void) {
 #endif
 }
 
-void orc_rmsnorm_row(const uint16_t* x, const uint16_t* w, int64_t h, double eps,
-                     uint16_t* y) {
+/* RMSNorm of one row, y_i = bf16(x_i / sqrt(mean(x^2) + eps) * w'_i), with w' = w (mode 0,
+ * the plain weights of the V4 page) or w' = 1 + w (mode 1: the V4 page notes that the
+ * shared rms_norm kernel applies 1 + w). */
+void orc_rmsnorm_row_mode(const uint16_t* x, const uint16_t* w, int64_t h, double eps,
+                          int32_t mode, uint16_t* y) {
     double ss = 0.0;
     for (int64_t i = 0; i < h; ++i) {
         double v = orc_bf16_to_f64(x[i]);
         ss += v * v;
     }
     double inv = 1.0 / sqrt(ss / (double)h + eps);
-    for (int64_t i = 0; i < h; ++i)
-        y[i] = orc_f64_to_bf16(orc_bf16_to_f64(x[i]) * inv * orc_bf16_to_f64(w[i]));
+    for (int64_t i = 0; i < h; ++i) {
+        double wi = orc_bf16_to_f64(w[i]) + (mode == 1 ? 1.0 : 0.0);
+        y[i] = orc_f64_to_bf16(orc_bf16_to_f64(x[i]) * inv * wi);
+    }
+}
+
+void orc_rmsnorm_row(const uint16_t* x, const uint16_t* w, int64_t h, double eps,
+                     uint16_t* y) {
+    orc_rmsnorm_row_mode(x, w, h, eps, 0, y);
 }
 
 int32_t orc_combine(const uint16_t* embed, int64_t vocab, const int32_t* tokens,
@@ -75,6 +85,15 @@ int32_t orc_combine(const uint16_t* embed, int64_t vocab, const int32_t* tokens,
                     const uint16_t* w_norm_embed, const uint16_t* w_norm_hidden,
                     double eps, const uint16_t* fc, uint16_t* out_concat,
                     uint16_t* out_y) {
+    return orc_combine_mode(embed, vocab, tokens, hidden, M, h, w_norm_embed, w_norm_hidden,
+                            eps, 0, fc, out_concat, out_y);
+}
+
+int32_t orc_combine_mode(const uint16_t* embed, int64_t vocab, const int32_t* tokens,
+                         const uint16_t* hidden, int32_t M, int32_t h,
+                         const uint16_t* w_norm_embed, const uint16_t* w_norm_hidden,
+                         double eps, int32_t mode, const uint16_t* fc, uint16_t* out_concat,
+                         uint16_t* out_y) {
     int32_t flags = 0;
     uint16_t* c = (uint16_t*)malloc(sizeof(uint16_t) * 2 * (size_t)h);
     uint16_t* zero = (uint16_t*)calloc((size_t)h, sizeof(uint16_t));
@@ -85,8 +104,8 @@ int32_t orc_combine(const uint16_t* embed, int64_t vocab, const int32_t* tokens,
             e = embed + tok * (int64_t)h;
         else
             flags |= ORC_FLAG_BAD_TOKEN;
-        orc_rmsnorm_row(e, w_norm_embed, h, eps, c);
-        orc_rmsnorm_row(hidden + (int64_t)m * h, w_norm_hidden, h, eps, c + h);
+        orc_rmsnorm_row_mode(e, w_norm_embed, h, eps, mode, c);
+        orc_rmsnorm_row_mode(hidden + (int64_t)m * h, w_norm_hidden, h, eps, mode, c + h);
         if (out_concat)
             for (int64_t j = 0; j < 2 * h; ++j) out_concat[(int64_t)m * 2 * h + j] = c[j];
 #pragma omp parallel for schedule(static)

@@ -55,6 +55,25 @@ void orc_dequant_row(int32_t fmt, const void* data, const float* row_scale,
 /* draft.c */
 void orc_rmsnorm_row(const uint16_t* x, const uint16_t* w, int64_t h, double eps,
                      uint16_t* y);
+void orc_rmsnorm_row_mode(const uint16_t* x, const uint16_t* w, int64_t h, double eps,
+                          int32_t mode, uint16_t* y);
+int32_t orc_combine_mode(const uint16_t* embed, int64_t vocab, const int32_t* tokens,
+                         const uint16_t* hidden, int32_t M, int32_t h,
+                         const uint16_t* w_norm_embed, const uint16_t* w_norm_hidden,
+                         double eps, int32_t mode, const uint16_t* fc, uint16_t* out_concat,
+                         uint16_t* out_y);
+int32_t orc_prefill_rows_ext(const uint16_t* embed, int64_t vocab, const int32_t* tokens,
+                             const uint16_t* hidden, int32_t h,
+                             const uint16_t* w_norm_embed, const uint16_t* w_norm_hidden,
+                             double eps, const uint16_t* fc, const uint16_t* wk,
+                             const uint16_t* wv, int32_t nkv, int32_t hd, double rope_base,
+                             const int32_t* rope_pos, int64_t cache_start,
+                             const int32_t* block_table, int64_t n_table,
+                             int32_t block_size, int64_t num_blocks, float k_scale,
+                             float v_scale, int32_t mode, const uint16_t* k_norm,
+                             const int64_t* rows, int64_t nrows,
+                             uint16_t* out_y, uint16_t* out_k_rot, uint16_t* out_v,
+                             uint8_t* out_k_codes, uint8_t* out_v_codes, int64_t* out_slot);
 int32_t orc_combine(const uint16_t* embed, int64_t vocab, const int32_t* tokens,
                     const uint16_t* hidden, int32_t M, int32_t h,
                     const uint16_t* w_norm_embed, const uint16_t* w_norm_hidden,

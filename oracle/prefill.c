@@ -19,9 +19,12 @@
  * A row whose block-table entry is missing or out of range is not written and
  * raises ORC_FLAG_BAD_SLOT.
  *
- * Readings (the pages are silent): no norm sits between fc and the k/v projections
- * and no per-head k norm is applied (the benchmark's step list has neither, though
- * the reference scratch has a `normed2` buffer); RoPE style, rotary dim and theta come from the
+ * Readings (the pages are silent): by default no norm sits between fc and the k/v
+ * projections and no per-head k norm is applied (the benchmark's step list has neither,
+ * though the reference scratch has a `normed2` buffer and the head a `k_norm` weight);
+ * with `k_norm` given (orc_prefill_rows_ext), each bf16 k head is RMS-normalized over hd
+ * with those weights (same eps and weight mode as the combiner's norms) and rounded to
+ * bf16 before RoPE, the usual order of a per-head k norm; RoPE style, rotary dim and theta come from the
  * benchmark configuration (NeoX, full head, base given); the RoPE position of each
  * row is an explicit input because a forward_one at RoPE position p writes pair key
  * p - 1 ([mtp_head.rs] MtpProposerState docs), i.e. position and cache row differ.
@@ -76,7 +79,7 @@ static void matvec_bf16(const uint16_t* W, int64_t n, int64_t k, const uint16_t*
     }
 }
 
-int32_t orc_prefill_rows(const uint16_t* embed, int64_t vocab, const int32_t* tokens,
+int32_t orc_prefill_rows_ext(const uint16_t* embed, int64_t vocab, const int32_t* tokens,
                          const uint16_t* hidden, int32_t h,
                          const uint16_t* w_norm_embed, const uint16_t* w_norm_hidden,
                          double eps, const uint16_t* fc, const uint16_t* wk,
@@ -84,7 +87,8 @@ int32_t orc_prefill_rows(const uint16_t* embed, int64_t vocab, const int32_t* to
                          const int32_t* rope_pos, int64_t cache_start,
                          const int32_t* block_table, int64_t n_table,
                          int32_t block_size, int64_t num_blocks, float k_scale,
-                         float v_scale, const int64_t* rows, int64_t nrows,
+                         float v_scale, int32_t mode, const uint16_t* k_norm,
+                         const int64_t* rows, int64_t nrows,
                          uint16_t* out_y, uint16_t* out_k_rot, uint16_t* out_v,
                          uint8_t* out_k_codes, uint8_t* out_v_codes, int64_t* out_slot) {
     int32_t flags = 0;
@@ -98,11 +102,13 @@ int32_t orc_prefill_rows(const uint16_t* embed, int64_t vocab, const int32_t* to
         double* kd = (double*)malloc(sizeof(double) * (size_t)hd);
         double* kr = (double*)malloc(sizeof(double) * (size_t)hd);
         int32_t tok = tokens[r];
-        flags |= orc_combine(embed, vocab, &tok, hidden + r * (int64_t)h, 1, h,
-                             w_norm_embed, w_norm_hidden, eps, fc, NULL, y);
+        flags |= orc_combine_mode(embed, vocab, &tok, hidden + r * (int64_t)h, 1, h,
+                                  w_norm_embed, w_norm_hidden, eps, mode, fc, NULL, y);
         matvec_bf16(wk, kvd, h, y, kb);
         matvec_bf16(wv, kvd, h, y, vb);
         for (int32_t hh = 0; hh < nkv; ++hh) {
+            if (k_norm)  /* per-head RMSNorm of k over hd, before RoPE */
+                orc_rmsnorm_row_mode(kb + hh * hd, k_norm, hd, eps, mode, kb + hh * hd);
             for (int32_t d = 0; d < hd; ++d) kd[d] = orc_bf16_to_f64(kb[hh * hd + d]);
             orc_rope_neox(kd, hd, (double)rope_pos[r], rope_base, kr);
             for (int32_t d = 0; d < hd; ++d) kb[hh * hd + d] = orc_f64_to_bf16(kr[d]);
@@ -125,4 +131,21 @@ int32_t orc_prefill_rows(const uint16_t* embed, int64_t vocab, const int32_t* to
         free(kr);
     }
     return flags;
+}
+
+int32_t orc_prefill_rows(const uint16_t* embed, int64_t vocab, const int32_t* tokens,
+                         const uint16_t* hidden, int32_t h,
+                         const uint16_t* w_norm_embed, const uint16_t* w_norm_hidden,
+                         double eps, const uint16_t* fc, const uint16_t* wk,
+                         const uint16_t* wv, int32_t nkv, int32_t hd, double rope_base,
+                         const int32_t* rope_pos, int64_t cache_start,
+                         const int32_t* block_table, int64_t n_table,
+                         int32_t block_size, int64_t num_blocks, float k_scale,
+                         float v_scale, const int64_t* rows, int64_t nrows,
+                         uint16_t* out_y, uint16_t* out_k_rot, uint16_t* out_v,
+                         uint8_t* out_k_codes, uint8_t* out_v_codes, int64_t* out_slot) {
+    return orc_prefill_rows_ext(embed, vocab, tokens, hidden, h, w_norm_embed, w_norm_hidden, eps,
+                                fc, wk, wv, nkv, hd, rope_base, rope_pos, cache_start, block_table,
+                                n_table, block_size, num_blocks, k_scale, v_scale, 0, NULL, rows,
+                                nrows, out_y, out_k_rot, out_v, out_k_codes, out_v_codes, out_slot);
 }

@@ -647,3 +647,96 @@ def test_attn_missing_block_flags_and_skips(orc):
     assert flags & orc.FLAG_BAD_SLOT
     ref, _ = orc.paged_decode_attn(q, 2, kc, vc, bt, 16, nb, 32)
     assert np.array_equal(out, ref)
+
+
+
+# ---------------------------------------------------------------- norm mode and k norm pins
+def test_one_plus_w_mode_is_plain_mode_on_shifted_weights(orc):
+    """norm_mode 1 multiplies by 1 + w: with w = 0 it is plain mode with unit weights, and
+    with weights whose 1 + w is a bf16 value it is plain mode with those values."""
+    rng = np.random.default_rng(31)
+    x = orc.f64_to_bf16(rng.normal(0, 1, 64))
+    zero = np.zeros(64, np.uint16)
+    one = orc.f64_to_bf16(np.ones(64))
+    assert np.array_equal(orc.rmsnorm(x, zero, 1e-6, norm_mode=1), orc.rmsnorm(x, one, 1e-6))
+    w = rng.choice([0.0, 0.5, -0.25, 0.125, 1.0, -0.5], 64)
+    assert np.array_equal(orc.rmsnorm(x, orc.f64_to_bf16(w), 1e-6, norm_mode=1),
+                          orc.rmsnorm(x, orc.f64_to_bf16(1.0 + w), 1e-6))
+    d = synth.tiny_draft(seed=5, vocab=50, h=32, M=2)
+    u = synth.as_u16
+    y1, c1, _ = orc.combine(u(d["embed"]), d["tokens"].numpy(), u(d["hidden"]), zero[:32],
+                            zero[:32], 1e-6, u(d["fc"]), norm_mode=1)
+    y0, c0, _ = orc.combine(u(d["embed"]), d["tokens"].numpy(), u(d["hidden"]), one[:32],
+                            one[:32], 1e-6, u(d["fc"]))
+    assert np.array_equal(c1, c0) and np.array_equal(y1, y0)
+
+
+def _kn_case(orc, seed, k_norm, pos0=0, norm_mode=0, same_rows=False, norm_w=None):
+    d = synth.prefill_inputs(seed=seed, R=6, vocab=40, h=256, nkv=2, hd=64)
+    if norm_w is not None:  # both combiner norm weights set to this constant
+        d["w_norm_embed"] = torch.full((256,), norm_w, dtype=torch.bfloat16)
+        d["w_norm_hidden"] = torch.full((256,), norm_w, dtype=torch.bfloat16)
+    if same_rows:  # every row of a head's Wk the same: each k head is a constant vector
+        wk = d["wk"].clone()
+        for hh in range(2):
+            wk[hh * 64:(hh + 1) * 64] = wk[hh * 64]
+        d["wk"] = wk
+    d["rope_pos"] = torch.full((6,), pos0, dtype=torch.int32)
+    U = {k: (synth.as_u16(v) if isinstance(v, torch.Tensor) and v.dtype == torch.bfloat16 else
+             (v.numpy() if isinstance(v, torch.Tensor) else v)) for k, v in d.items()}
+    out = orc.prefill_rows(U["embed"], U["tokens"], U["hidden"], U["w_norm_embed"],
+                           U["w_norm_hidden"], U["eps"], U["fc"], U["wk"], U["wv"], 2, 64,
+                           U["rope_base"], U["rope_pos"], 0, U["block_table"], 16,
+                           U["num_blocks"], 1.0, 1.0, np.arange(6), norm_mode=norm_mode,
+                           k_norm=k_norm)
+    return out, U
+
+
+def test_k_norm_constant_head_closed_form(orc):
+    """A head whose Wk rows are all equal gives k = c 1; its k norm at RoPE position 0 (the
+    identity) is bf16(c / sqrt(c^2 + eps) w_j)."""
+    rng = np.random.default_rng(32)
+    w = orc.f64_to_bf16(rng.normal(1.0, 0.1, 64))
+    plain, _ = _kn_case(orc, 41, None, same_rows=True)
+    normed, U = _kn_case(orc, 41, w, same_rows=True)
+    c = bf16_to_f64_(plain["k_rot"].reshape(6, 2, 64)[:, :, 0])  # pos 0: k itself
+    want = orc.f64_to_bf16(c[:, :, None] / np.sqrt(c[:, :, None] ** 2 + U["eps"])
+                           * bf16_to_f64_(w)[None, None, :])
+    assert np.array_equal(normed["k_rot"].reshape(6, 2, 64), want)
+    assert np.array_equal(normed["v"], plain["v"])  # v is untouched
+
+
+def test_k_norm_unit_rms_and_mode(orc):
+    """With unit weights every k head has RMS 1 before RoPE; RoPE keeps pair norms, so the
+    stored head's RMS stays 1 up to bf16 rounding. Mode 1 with w = 0 equals unit weights."""
+    ones = orc.f64_to_bf16(np.ones(64))
+    out, _ = _kn_case(orc, 42, ones, pos0=100)
+    k = bf16_to_f64_(out["k_rot"]).reshape(6, 2, 64)
+    rms = np.sqrt((k ** 2).mean(axis=2))
+    assert np.all(np.abs(rms - 1.0) < 5e-3), rms
+    # mode 1 applies 1 + w to every norm of the call: zero weights there are unit weights
+    out0, _ = _kn_case(orc, 42, ones, pos0=100, norm_w=1.0)
+    out1, _ = _kn_case(orc, 42, np.zeros(64, np.uint16), pos0=100, norm_mode=1, norm_w=0.0)
+    assert np.array_equal(out1["k_rot"], out0["k_rot"]) and np.array_equal(out1["v"], out0["v"])
+
+
+def bf16_to_f64_(b):
+    return (np.asarray(b, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def test_k_norm_comes_before_rope(orc):
+    """A constant head k = c 1 with non-uniform k-norm weights w at RoPE position 37: the
+    normed head bf16(s w), s = c / sqrt(c^2 + eps), rotated by RoPE (pinned above), then
+    rounded -- which fixes the order (rotating first and normalizing after differs)."""
+    rng = np.random.default_rng(33)
+    w = orc.f64_to_bf16(rng.normal(1.0, 0.3, 64))
+    plain, _ = _kn_case(orc, 41, None, same_rows=True)  # position 0: k itself
+    normed, U = _kn_case(orc, 41, w, pos0=37, same_rows=True)
+    c = bf16_to_f64_(plain["k_rot"].reshape(6, 2, 64)[:, :, 0])
+    got = normed["k_rot"].reshape(6, 2, 64)
+    for r in range(6):
+        for hh in range(2):
+            s = c[r, hh] / np.sqrt(c[r, hh] ** 2 + U["eps"])
+            kn = bf16_to_f64_(orc.f64_to_bf16(s * bf16_to_f64_(w)))
+            want = orc.f64_to_bf16(orc.rope_neox(kn, 37.0, U["rope_base"]))
+            assert np.array_equal(got[r, hh], want), (r, hh)
