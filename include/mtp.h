@@ -40,7 +40,9 @@
 extern "C" {
 #endif
 
-#define MTP_ABI_VERSION 1
+/* 2: mtp_combine, mtp_draft_step and mtp_prefill_kv take norm_mode; mtp_prefill_kv takes
+ * k_norm. */
+#define MTP_ABI_VERSION 2
 
 typedef enum {
     MTP_OK = 0,
@@ -50,6 +52,12 @@ typedef enum {
     MTP_ERR_CUDA = 4,        /* a CUDA launch or API call failed */
     MTP_WARN_EMPTY_MASK = 5  /* mtp_devflags_status(): a mask allowed no token */
 } mtp_status;
+
+/* RMSNorm weight modes (every norm of a call): the plain w * x_normed of the V4 head
+ * ([v4_mtp.rs] DeepseekV4MtpHead::new: "the norm weights are plain"), or (1 + w) * x_normed,
+ * what that page says the shared rms_norm kernel applies. */
+#define MTP_NORM_W 0
+#define MTP_NORM_ONE_PLUS_W 1
 
 /* Bits a kernel ORs into the caller's device error word. */
 #define MTP_DEVFLAG_BAD_TOKEN 1  /* token id outside [0, vocab): its row read as zeros */
@@ -134,6 +142,8 @@ mtp_status mtp_quantize_nvfp4(const uint16_t* w, int64_t n, int64_t k, uint8_t* 
  *   e = embed[token_ids[m]];  ne = bf16(e / sqrt(mean(e^2) + eps) * w_norm_embed)
  *   nh = bf16(x / sqrt(mean(x^2) + eps) * w_norm_hidden),  x = hidden[m]
  *   out[m] = bf16(fc . [ne || nh])           (embedding half first)
+ *   (with norm_mode MTP_NORM_ONE_PLUS_W the weights are 1 + w_norm_*; any other value
+ *   than the two MTP_NORM_* is MTP_ERR_INVALID_ARG)
  *   embed         (device) bf16 [vocab, h]
  *   token_ids     (device) i32 [M]; an id outside [0, vocab) reads as a zero row and
  *                 sets MTP_DEVFLAG_BAD_TOKEN
@@ -150,8 +160,8 @@ mtp_status mtp_quantize_nvfp4(const uint16_t* w, int64_t n, int64_t k, uint8_t* 
 mtp_status mtp_combine(const uint16_t* embed, int64_t vocab, const int32_t* token_ids,
                        const uint16_t* hidden, int32_t M, int32_t h,
                        const uint16_t* w_norm_embed, const uint16_t* w_norm_hidden,
-                       float eps, const mtp_weight* fc, uint16_t* out, int32_t* dev_err,
-                       void* stream);
+                       float eps, int32_t norm_mode, const mtp_weight* fc, uint16_t* out,
+                       int32_t* dev_err, void* stream);
 
 /* ---------------------------------------------------------------------------------
  * mtp_lm_head_argmax -- the draft lm_head sweep fused with a (masked) argmax.
@@ -251,6 +261,7 @@ mtp_status mtp_lm_head_argmax_lp(const mtp_weight* head, int64_t n_eff, const ui
  * weights, e_proj / h_proj combiner, lm_head GEMV over the first n_eff rows, argmax,
  * grammar-masked when a bitmask is given) and [mtp_head.rs] module docs (concat -> fc).
  *   c[m] = [bf16(rms(embed[token_ids[m]]) w_norm_embed) || bf16(rms(hidden[m]) w_norm_hidden)]
+ *   (weights 1 + w_norm_* with norm_mode MTP_NORM_ONE_PLUS_W, as mtp_combine)
  *   y[m] = bf16(fc . c[m]);  l[m, r] = sum_j head[r, j] y[m, j] (fp32), r < n_eff
  *   out_idx[m] = lowest allowed r with the largest l[m, r] (mask as mtp_lm_head_argmax;
  *   nothing allowed -> 0, -inf and MTP_DEVFLAG_EMPTY_MASK)
@@ -271,7 +282,7 @@ mtp_status mtp_lm_head_argmax_lp(const mtp_weight* head, int64_t n_eff, const ui
 mtp_status mtp_draft_step(const uint16_t* embed, int64_t vocab, const int32_t* token_ids,
                           const uint16_t* hidden, int32_t M, int32_t h,
                           const uint16_t* w_norm_embed, const uint16_t* w_norm_hidden, float eps,
-                          const uint16_t* fc, const uint16_t* head, int64_t n_eff,
+                          int32_t norm_mode, const uint16_t* fc, const uint16_t* head, int64_t n_eff,
                           const int32_t* mask, int64_t mask_words, int64_t mask_stride_words,
                           uint16_t* out_y, int32_t* out_idx, float* out_val, int32_t* dev_err,
                           void* stream);
@@ -322,7 +333,10 @@ mtp_status mtp_argmax_merge_partials(const void* partials, int32_t n_parts, int3
  * Per row r (all intermediate activations rounded to bf16):
  *   c = [rms(embed[token_ids[r]]) w_norm_embed || rms(hidden[r]) w_norm_hidden]
  *   y = fc . c;  k = wk . y;  v = wv . y;  k' = NeoX RoPE over each head of hd at
- *   position rope_pos[r] (theta_j = pos * rope_base^(-2j/hd));
+ *   position rope_pos[r] (theta_j = pos * rope_base^(-2j/hd)) of k, or, when k_norm is
+ *   given, of bf16(k_head / sqrt(mean(k_head^2) + eps) * k_norm) per head ([new.rs] and
+ *   [mtp_head.rs] list the head's per-head k_norm weight; the norm precedes RoPE here);
+ *   norm_mode MTP_NORM_ONE_PLUS_W makes every norm weight of the call 1 + w;
  *   p = cache_start + r;  slot = block_table[p / block_size] * block_size + p % block_size
  *   k_cache[(slot * nkv + head) * hd + d] = e4m3_satfinite(k'[head, d] / k_scale), same
  *   for v with v_scale. A row whose block is missing (p / block_size >= n_table) or out of
@@ -330,7 +344,8 @@ mtp_status mtp_argmax_merge_partials(const void* partials, int32_t n_parts, int3
  *   embedding row and sets MTP_DEVFLAG_BAD_TOKEN.
  *   embed (device) bf16 [vocab, h]; token_ids, rope_pos (device) i32 [R];
  *   hidden (device) bf16 [R, h]; w_norm_* (device) bf16 [h]; fc (device) bf16 [h, 2h];
- *   wk, wv (device) bf16 [nkv * hd, h]; block_table (device) i32 [n_table];
+ *   wk, wv (device) bf16 [nkv * hd, h]; k_norm (device) bf16 [hd] or NULL;
+ *   block_table (device) i32 [n_table];
  *   k_cache, v_cache (device) u8 [num_blocks, block_size, nkv, hd], written in place;
  *   ws (device) mtp_prefill_ws_bytes(min(chunk_rows, R), h, nkv, hd) bytes, 1 KB
  *   aligned, no initial contents required: a small counter header (zeroed by the call
@@ -350,7 +365,8 @@ size_t mtp_prefill_ws_bytes(int64_t chunk_rows, int32_t h, int32_t nkv, int32_t 
 mtp_status mtp_prefill_kv(const uint16_t* embed, int64_t vocab, const int32_t* token_ids,
                           const uint16_t* hidden, int64_t R, int32_t h,
                           const uint16_t* w_norm_embed, const uint16_t* w_norm_hidden, float eps,
-                          const uint16_t* fc, const uint16_t* wk, const uint16_t* wv, int32_t nkv,
+                          int32_t norm_mode, const uint16_t* fc, const uint16_t* wk,
+                          const uint16_t* wv, const uint16_t* k_norm, int32_t nkv,
                           int32_t hd, float rope_base, const int32_t* rope_pos,
                           int64_t cache_start, const int32_t* block_table, int64_t n_table,
                           int32_t block_size, uint8_t* k_cache, uint8_t* v_cache,

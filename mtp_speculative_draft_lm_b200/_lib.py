@@ -26,6 +26,9 @@ MTP_DEVFLAG_EMPTY_MASK = 2
 MTP_DEVFLAG_BAD_SLOT = 4
 MTP_DEVFLAG_TIMEOUT = 8
 
+MTP_NORM_W = 0
+MTP_NORM_ONE_PLUS_W = 1
+
 MTP_FMT_BF16 = 0
 MTP_FMT_FP8_ROW = 1
 MTP_FMT_NVFP4 = 2
@@ -71,8 +74,8 @@ _SIGS = {
     "mtp_quantize_nvfp4_ws_bytes": (_SZ, [_I64, _I64]),
     "mtp_nvfp4_scale_pitch": (_I64, [_I64]),
     "mtp_quantize_nvfp4": (C.c_int, [_P, _I64, _I64, _P, _P, _P, _P, _SZ, _P]),
-    "mtp_combine": (C.c_int, [_P, _I64, _P, _P, _I32, _I32, _P, _P, C.c_float, _W, _P, _P,
-                              _P]),
+    "mtp_combine": (C.c_int, [_P, _I64, _P, _P, _I32, _I32, _P, _P, C.c_float, _I32, _W, _P,
+                              _P, _P]),
     "mtp_lm_head_ws_bytes": (_SZ, [_W, _I64, _I32]),
     "mtp_lm_head_argmax": (C.c_int, [_W, _I64, _P, _I32, _P, _I64, _I64, _P, _P, _P, _P,
                                      _P, _SZ, _P]),
@@ -85,9 +88,9 @@ _SIGS = {
                                             _P, _P, _SZ, _P]),
     "mtp_argmax_merge_partials": (C.c_int, [_P, _I32, _I32, _P, _P, _P, _P, _P]),
     "mtp_prefill_ws_bytes": (_SZ, [_I64, _I32, _I32, _I32]),
-    "mtp_prefill_kv": (C.c_int, [_P, _I64, _P, _P, _I64, _I32, _P, _P, C.c_float, _P, _P, _P,
-                                 _I32, _I32, C.c_float, _P, _I64, _P, _I64, _I32, _P, _P, _I64,
-                                 C.c_float, C.c_float, _I64, _P, _SZ, _P, _P]),
+    "mtp_prefill_kv": (C.c_int, [_P, _I64, _P, _P, _I64, _I32, _P, _P, C.c_float, _I32, _P, _P,
+                                 _P, _P, _I32, _I32, C.c_float, _P, _I64, _P, _I64, _I32, _P, _P,
+                                 _I64, C.c_float, C.c_float, _I64, _P, _SZ, _P, _P]),
     "mtp_debug_gemm_bf16": (C.c_int, [_P, _P, _P, _I32, _I32, _I32, _P]),
     "mtp_debug_kv_write": (C.c_int, [_P, _P, _I64, _I32, _I32, _I64, _P, _I64, _I32, _I64, _P,
                                      _P, C.c_float, C.c_float, _P, _P]),
@@ -99,8 +102,8 @@ _SIGS = {
     "mtp_paged_decode_attn": (C.c_int, [_P, _I32, _I32, _I32, _P, _P, _P, _I64, _I32, _I64,
                                         _I64, C.c_float, C.c_float, C.c_float, _P, _P, _P, _SZ,
                                         _P]),
-    "mtp_draft_step": (C.c_int, [_P, _I64, _P, _P, _I32, _I32, _P, _P, C.c_float, _P, _P, _I64,
-                                 _P, _I64, _I64, _P, _P, _P, _P, _P]),
+    "mtp_draft_step": (C.c_int, [_P, _I64, _P, _P, _I32, _I32, _P, _P, C.c_float, _I32, _P, _P,
+                                 _I64, _P, _I64, _I64, _P, _P, _P, _P, _P]),
     "mtp_debug_encode_e4m3": (C.c_int, [_P, _I64, _P, _P]),
     "mtp_debug_encode_e2m1": (C.c_int, [_P, _I64, _P, _P]),
 }
@@ -183,10 +186,10 @@ def mtp_quantize_nvfp4(w, n, k, codes, block_scale, global_scale, ws, ws_bytes, 
            "mtp_quantize_nvfp4")
 
 
-def mtp_combine(embed, vocab, token_ids, hidden, M, h, w_norm_embed, w_norm_hidden, eps, fc,
-                out, dev_err=None, stream=None):
+def mtp_combine(embed, vocab, token_ids, hidden, M, h, w_norm_embed, w_norm_hidden, eps,
+                norm_mode, fc, out, dev_err=None, stream=None):
     _check(load().mtp_combine(_ptr(embed), vocab, _ptr(token_ids), _ptr(hidden), M, h,
-                              _ptr(w_norm_embed), _ptr(w_norm_hidden), float(eps),
+                              _ptr(w_norm_embed), _ptr(w_norm_hidden), float(eps), int(norm_mode),
                               C.byref(fc) if fc is not None else None, _ptr(out),
                               _ptr(dev_err), _stream(stream)), "mtp_combine")
 
@@ -250,13 +253,14 @@ def mtp_prefill_ws_bytes(chunk_rows, h, nkv, hd) -> int:
     return load().mtp_prefill_ws_bytes(chunk_rows, h, nkv, hd)
 
 
-def mtp_prefill_kv(embed, vocab, token_ids, hidden, R, h, w_norm_embed, w_norm_hidden, eps, fc,
-                   wk, wv, nkv, hd, rope_base, rope_pos, cache_start, block_table, n_table,
-                   block_size, k_cache, v_cache, num_blocks, k_scale, v_scale, chunk_rows, ws,
-                   ws_bytes, dev_err=None, stream=None):
+def mtp_prefill_kv(embed, vocab, token_ids, hidden, R, h, w_norm_embed, w_norm_hidden, eps,
+                   norm_mode, fc, wk, wv, k_norm, nkv, hd, rope_base, rope_pos, cache_start,
+                   block_table, n_table, block_size, k_cache, v_cache, num_blocks, k_scale,
+                   v_scale, chunk_rows, ws, ws_bytes, dev_err=None, stream=None):
     _check(load().mtp_prefill_kv(_ptr(embed), vocab, _ptr(token_ids), _ptr(hidden), R, h,
-                                 _ptr(w_norm_embed), _ptr(w_norm_hidden), float(eps), _ptr(fc),
-                                 _ptr(wk), _ptr(wv), nkv, hd, float(rope_base), _ptr(rope_pos),
+                                 _ptr(w_norm_embed), _ptr(w_norm_hidden), float(eps),
+                                 int(norm_mode), _ptr(fc), _ptr(wk), _ptr(wv), _ptr(k_norm), nkv,
+                                 hd, float(rope_base), _ptr(rope_pos),
                                  cache_start, _ptr(block_table), n_table, block_size,
                                  _ptr(k_cache), _ptr(v_cache), num_blocks, float(k_scale),
                                  float(v_scale), chunk_rows, _ptr(ws), ws_bytes, _ptr(dev_err),
@@ -289,11 +293,12 @@ def mtp_lm_head_argmax_noalloc(head, n_eff, x, M, mask, mask_words, mask_stride_
            "mtp_lm_head_argmax_noalloc")
 
 
-def mtp_draft_step(embed, vocab, token_ids, hidden, M, h, w_norm_embed, w_norm_hidden, eps, fc,
-                   head, n_eff, mask, mask_words, mask_stride_words, out_y, out_idx, out_val,
-                   dev_err=None, stream=None):
+def mtp_draft_step(embed, vocab, token_ids, hidden, M, h, w_norm_embed, w_norm_hidden, eps,
+                   norm_mode, fc, head, n_eff, mask, mask_words, mask_stride_words, out_y,
+                   out_idx, out_val, dev_err=None, stream=None):
     _check(load().mtp_draft_step(_ptr(embed), vocab, _ptr(token_ids), _ptr(hidden), M, h,
-                                 _ptr(w_norm_embed), _ptr(w_norm_hidden), float(eps), _ptr(fc),
+                                 _ptr(w_norm_embed), _ptr(w_norm_hidden), float(eps),
+                                 int(norm_mode), _ptr(fc),
                                  _ptr(head), n_eff, _ptr(mask), mask_words, mask_stride_words,
                                  _ptr(out_y), _ptr(out_idx), _ptr(out_val), _ptr(dev_err),
                                  _stream(stream)), "mtp_draft_step")

@@ -210,18 +210,18 @@ class ShardedLmHead:
 
 
 def combine(embed, token_ids, hidden, w_norm_embed, w_norm_hidden, eps, fc: Table,
-            out=None, dev_err=None, stream=None):
+            out=None, dev_err=None, stream=None, norm_mode=L.MTP_NORM_W):
     M, h = hidden.shape
     if out is None:
         out = torch.empty((M, h), dtype=torch.bfloat16, device=hidden.device)
     L.mtp_combine(embed, embed.shape[0], token_ids, hidden, M, h, w_norm_embed, w_norm_hidden,
-                  eps, fc.desc, out, dev_err, stream)
+                  eps, norm_mode, fc.desc, out, dev_err, stream)
     return out
 
 
 def draft_step(embed, token_ids, hidden, w_norm_embed, w_norm_hidden, eps, fc, head,
                n_eff=None, mask=None, mask_words=0, mask_stride_words=0, out_y=None,
-               out_idx=None, out_val=None, dev_err=None, stream=None):
+               out_idx=None, out_val=None, dev_err=None, stream=None, norm_mode=L.MTP_NORM_W):
     """One whole draft step (combiner + lm_head sweep + argmax) for a small BF16 head in
     one launch: returns (idx, val, y)."""
     M, h = hidden.shape
@@ -231,8 +231,8 @@ def draft_step(embed, token_ids, hidden, w_norm_embed, w_norm_hidden, eps, fc, h
     out_idx = torch.empty((M,), dtype=torch.int32, device=dev) if out_idx is None else out_idx
     out_val = torch.empty((M,), dtype=torch.float32, device=dev) if out_val is None else out_val
     L.mtp_draft_step(embed, embed.shape[0], token_ids, hidden, M, h, w_norm_embed, w_norm_hidden,
-                     eps, fc, head, n, mask, mask_words, mask_stride_words, out_y, out_idx,
-                     out_val, dev_err, stream)
+                     eps, norm_mode, fc, head, n, mask, mask_words, mask_stride_words, out_y,
+                     out_idx, out_val, dev_err, stream)
     return out_idx, out_val, out_y
 
 
@@ -264,7 +264,8 @@ def aligned_empty(nbytes: int, align: int, device) -> torch.Tensor:
 
 def prefill_kv(inputs: dict, k_cache: torch.Tensor, v_cache: torch.Tensor, chunk_rows: int = 2048,
                ws: torch.Tensor | None = None, dev_err: torch.Tensor | None = None, stream=None):
-    """Drafter-context prefill over device tensors named as in synth.prefill_inputs."""
+    """Drafter-context prefill over device tensors named as in synth.prefill_inputs (plus the
+    optional "norm_mode" and "k_norm" [hd] entries)."""
     d = inputs
     R, h = d["hidden"].shape
     nkv, hd = int(d["nkv"]), int(d["hd"])
@@ -273,8 +274,9 @@ def prefill_kv(inputs: dict, k_cache: torch.Tensor, v_cache: torch.Tensor, chunk
     if ws is None:
         ws = aligned_empty(nbytes, 1024, k_cache.device)
     L.mtp_prefill_kv(d["embed"], d["embed"].shape[0], d["tokens"], d["hidden"], R, h,
-                     d["w_norm_embed"], d["w_norm_hidden"], d["eps"], d["fc"], d["wk"], d["wv"],
-                     nkv, hd, d["rope_base"], d["rope_pos"], int(d["cache_start"]),
+                     d["w_norm_embed"], d["w_norm_hidden"], d["eps"], int(d.get("norm_mode", 0)),
+                     d["fc"], d["wk"], d["wv"], d.get("k_norm"), nkv, hd, d["rope_base"],
+                     d["rope_pos"], int(d["cache_start"]),
                      d["block_table"], d["block_table"].numel(), int(d["block_size"]), k_cache,
                      v_cache, k_cache.shape[0], d["k_scale"], d["v_scale"], chunk, ws, ws.numel(),
                      dev_err, stream)

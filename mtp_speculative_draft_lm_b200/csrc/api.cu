@@ -116,11 +116,13 @@ mtp_status mtp_quantize_nvfp4(const uint16_t* w, int64_t n, int64_t k, uint8_t* 
 mtp_status mtp_combine(const uint16_t* embed, int64_t vocab, const int32_t* token_ids,
                        const uint16_t* hidden, int32_t M, int32_t h,
                        const uint16_t* w_norm_embed, const uint16_t* w_norm_hidden,
-                       float eps, const mtp_weight* fc, uint16_t* out, int32_t* dev_err,
-                       void* stream) {
+                       float eps, int32_t norm_mode, const mtp_weight* fc, uint16_t* out,
+                       int32_t* dev_err, void* stream) {
     if (!embed || !token_ids || !hidden || !w_norm_embed || !w_norm_hidden || !out)
         return MTP_ERR_INVALID_ARG;
-    if (vocab < 1 || h < 16 || h % 16 || !(eps >= 0.f)) return MTP_ERR_INVALID_ARG;
+    if (vocab < 1 || h < 16 || h % 16 || !(eps >= 0.f) ||
+        (norm_mode != MTP_NORM_W && norm_mode != MTP_NORM_ONE_PLUS_W))
+        return MTP_ERR_INVALID_ARG;
     if (M < 1 || M > kMaxMCombine) return MTP_ERR_UNSUPPORTED;
     mtp_status st = check_weight(fc);
     if (st != MTP_OK) return st;
@@ -148,6 +150,7 @@ mtp_status mtp_combine(const uint16_t* embed, int64_t vocab, const int32_t* toke
     p.w_norm_hidden = w_norm_hidden;
     p.eps = eps;
     p.h = h;
+    p.norm_mode = norm_mode;
     p.out_y = out;
     p.dev_err = dev_err;
     p.num_tiles = (fc->n + 15) / 16;
@@ -312,14 +315,15 @@ mtp_status mtp_lm_head_argmax_lp(const mtp_weight* head, int64_t n_eff, const ui
 mtp_status mtp_draft_step(const uint16_t* embed, int64_t vocab, const int32_t* token_ids,
                           const uint16_t* hidden, int32_t M, int32_t h,
                           const uint16_t* w_norm_embed, const uint16_t* w_norm_hidden, float eps,
-                          const uint16_t* fc, const uint16_t* head, int64_t n_eff,
+                          int32_t norm_mode, const uint16_t* fc, const uint16_t* head, int64_t n_eff,
                           const int32_t* mask, int64_t mask_words, int64_t mask_stride_words,
                           uint16_t* out_y, int32_t* out_idx, float* out_val, int32_t* dev_err,
                           void* stream) {
     if (!embed || !token_ids || !hidden || !w_norm_embed || !w_norm_hidden || !fc || !head ||
         !out_idx)
         return MTP_ERR_INVALID_ARG;
-    if (vocab < 1 || n_eff < 1 || n_eff > (int64_t)INT32_MAX || h < 8 || h % 8 || !(eps >= 0.f))
+    if (vocab < 1 || n_eff < 1 || n_eff > (int64_t)INT32_MAX || h < 8 || h % 8 || !(eps >= 0.f) ||
+        (norm_mode != MTP_NORM_W && norm_mode != MTP_NORM_ONE_PLUS_W))
         return MTP_ERR_INVALID_ARG;
     if (mask && (mask_words < 1 || mask_stride_words < 0)) return MTP_ERR_INVALID_ARG;
     if (M < 1 || M > mtp::draft_step_max_m() || h > mtp::draft_step_max_h()) return MTP_ERR_UNSUPPORTED;
@@ -329,7 +333,8 @@ mtp_status mtp_draft_step(const uint16_t* embed, int64_t vocab, const int32_t* t
         !aligned(dev_err, 4))
         return MTP_ERR_INVALID_ARG;
     return from_cuda(mtp::draft_step_launch(embed, vocab, token_ids, hidden, M, h, w_norm_embed,
-                                            w_norm_hidden, eps, fc, head, n_eff, mask, mask_words,
+                                            w_norm_hidden, eps, norm_mode, fc, head, n_eff, mask,
+                                            mask_words,
                                             mask_stride_words, out_y, out_idx, out_val, dev_err,
                                             as_stream(stream)));
 }
@@ -371,7 +376,8 @@ size_t mtp_prefill_ws_bytes(int64_t chunk_rows, int32_t h, int32_t nkv, int32_t 
 mtp_status mtp_prefill_kv(const uint16_t* embed, int64_t vocab, const int32_t* token_ids,
                           const uint16_t* hidden, int64_t R, int32_t h,
                           const uint16_t* w_norm_embed, const uint16_t* w_norm_hidden, float eps,
-                          const uint16_t* fc, const uint16_t* wk, const uint16_t* wv, int32_t nkv,
+                          int32_t norm_mode, const uint16_t* fc, const uint16_t* wk,
+                          const uint16_t* wv, const uint16_t* k_norm, int32_t nkv,
                           int32_t hd, float rope_base, const int32_t* rope_pos,
                           int64_t cache_start, const int32_t* block_table, int64_t n_table,
                           int32_t block_size, uint8_t* k_cache, uint8_t* v_cache,
@@ -382,7 +388,8 @@ mtp_status mtp_prefill_kv(const uint16_t* embed, int64_t vocab, const int32_t* t
         return MTP_ERR_INVALID_ARG;
     if (vocab < 1 || R < 1 || h < 1 || nkv < 1 || hd < 2 || block_size < 1 || n_table < 1 ||
         num_blocks < 1 || chunk_rows < 1 || !(eps >= 0.f) || !finite_pos(k_scale) ||
-        !finite_pos(v_scale) || !(rope_base > 0.f) || cache_start < 0)
+        !finite_pos(v_scale) || !(rope_base > 0.f) || cache_start < 0 ||
+        (norm_mode != MTP_NORM_W && norm_mode != MTP_NORM_ONE_PLUS_W) || !aligned(k_norm, 2))
         return MTP_ERR_INVALID_ARG;
     const int tn = mtp::gemm_tile_n();
     if (h % tn || h > mtp::prefill_max_hidden() || (hd != 64 && hd != 128 && hd != 256) ||
@@ -406,9 +413,11 @@ mtp_status mtp_prefill_kv(const uint16_t* embed, int64_t vocab, const int32_t* t
     a.w_norm_embed = w_norm_embed;
     a.w_norm_hidden = w_norm_hidden;
     a.eps = eps;
+    a.norm_mode = norm_mode;
     a.fc = fc;
     a.wk = wk;
     a.wv = wv;
+    a.k_norm = k_norm;
     a.nkv = nkv;
     a.hd = hd;
     a.rope_base = (double)rope_base;

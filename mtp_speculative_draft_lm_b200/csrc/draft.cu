@@ -47,6 +47,7 @@ struct DraftParams {
     const uint16_t* w_ne;
     const uint16_t* w_nh;
     float eps;
+    int norm_mode;          // 0: weights w, 1: weights 1 + w
     const uint16_t* fc;     // bf16 [h, 2h]
     const uint16_t* head;   // bf16 [n, h]
     int64_t n;              // rows swept
@@ -173,10 +174,11 @@ __global__ void __launch_bounds__(kDThreads, 1) draft_step_kernel(const __grid_c
         }
         const float inv_e = 1.0f / sqrtf(se / (float)h + p.eps);
         const float inv_x = 1.0f / sqrtf(sx / (float)h + p.eps);
+        const float add = p.norm_mode ? 1.f : 0.f;  // weights w or 1 + w
         for (int j = tid; j < h; j += kDThreads) {
             const float ev = e ? bf16_to_f32(e[j]) : 0.f;
-            cs[m][j] = f32_to_bf16(ev * inv_e * bf16_to_f32(p.w_ne[j]));
-            cs[m][h + j] = f32_to_bf16(bf16_to_f32(x[j]) * inv_x * bf16_to_f32(p.w_nh[j]));
+            cs[m][j] = f32_to_bf16(ev * inv_e * (bf16_to_f32(p.w_ne[j]) + add));
+            cs[m][h + j] = f32_to_bf16(bf16_to_f32(x[j]) * inv_x * (bf16_to_f32(p.w_nh[j]) + add));
         }
         __syncthreads();
     }
@@ -321,7 +323,7 @@ int draft_step_max_h() { return kDMaxH; }
 
 cudaError_t draft_step_launch(const uint16_t* embed, int64_t vocab, const int32_t* tokens,
                               const uint16_t* hidden, int M, int h, const uint16_t* w_ne,
-                              const uint16_t* w_nh, float eps, const uint16_t* fc,
+                              const uint16_t* w_nh, float eps, int norm_mode, const uint16_t* fc,
                               const uint16_t* head, int64_t n, const int32_t* mask,
                               int64_t mask_words, int64_t mask_stride, uint16_t* out_y,
                               int32_t* out_idx, float* out_val, int32_t* dev_err, cudaStream_t s) {
@@ -335,6 +337,7 @@ cudaError_t draft_step_launch(const uint16_t* embed, int64_t vocab, const int32_
     p.w_ne = w_ne;
     p.w_nh = w_nh;
     p.eps = eps;
+    p.norm_mode = norm_mode;
     p.fc = fc;
     p.head = head;
     p.n = n;

@@ -30,6 +30,7 @@ struct SweepParams {
     const uint16_t* w_norm_hidden;
     float eps;
     int32_t h;
+    int32_t norm_mode;           // 0: weights w, 1: weights 1 + w
     // grammar mask (mode 0)
     const int32_t* mask;
     int64_t mask_words;
@@ -105,9 +106,11 @@ struct PrefillArgs {
     const uint16_t* w_norm_embed;
     const uint16_t* w_norm_hidden;
     float eps;
+    int32_t norm_mode;
     const uint16_t* fc;
     const uint16_t* wk;
     const uint16_t* wv;
+    const uint16_t* k_norm;  // [hd] or null: per-head RMSNorm of k before RoPE
     int32_t nkv, hd;
     double rope_base;
     const int32_t* rope_pos;
@@ -145,7 +148,7 @@ int draft_step_max_m();
 int draft_step_max_h();
 cudaError_t draft_step_launch(const uint16_t* embed, int64_t vocab, const int32_t* tokens,
                               const uint16_t* hidden, int M, int h, const uint16_t* w_ne,
-                              const uint16_t* w_nh, float eps, const uint16_t* fc,
+                              const uint16_t* w_nh, float eps, int norm_mode, const uint16_t* fc,
                               const uint16_t* head, int64_t n, const int32_t* mask,
                               int64_t mask_words, int64_t mask_stride, uint16_t* out_y,
                               int32_t* out_idx, float* out_val, int32_t* dev_err, cudaStream_t s);

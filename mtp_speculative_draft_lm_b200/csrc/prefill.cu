@@ -80,6 +80,8 @@ struct PrefillParams {
     const uint16_t* w_ne;
     const uint16_t* w_nh;
     float eps;
+    int norm_mode;           // 0: weights w, 1: weights 1 + w
+    const uint16_t* k_norm;  // [hd] or null: per-head RMSNorm of k before RoPE
     int nkv, hd;
     double rope_base;
     const int32_t* rope_pos;
@@ -251,14 +253,15 @@ __device__ __forceinline__ void rope32(float (&lo)[32], float (&hi)[32], const f
     }
 }
 
-// 8 bf16 (one 16-byte piece) times a row factor and 8 norm weights, rounded to bf16.
-__device__ __forceinline__ uint4 norm8(uint4 v, float inv, uint4 w) {
+// 8 bf16 (one 16-byte piece) times a row factor and 8 norm weights (plus `add`: 0 for
+// weights w, 1 for 1 + w), rounded to bf16.
+__device__ __forceinline__ uint4 norm8(uint4 v, float inv, uint4 w, float add) {
     const uint32_t a[4] = {v.x, v.y, v.z, v.w}, b[4] = {w.x, w.y, w.z, w.w};
     uint32_t o[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const uint32_t lo = f32_to_bf16(bf16_lo(a[i]) * inv * bf16_lo(b[i]));
-        const uint32_t hi = f32_to_bf16(bf16_hi(a[i]) * inv * bf16_hi(b[i]));
+        const uint32_t lo = f32_to_bf16(bf16_lo(a[i]) * inv * (bf16_lo(b[i]) + add));
+        const uint32_t hi = f32_to_bf16(bf16_hi(a[i]) * inv * (bf16_hi(b[i]) + add));
         o[i] = lo | (hi << 16);
     }
     return make_uint4(o[0], o[1], o[2], o[3]);
@@ -577,6 +580,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 named_sync(1, kEpiThreads);
                 const int rows = (int)min((int64_t)BM, rows_c - (int64_t)tl.m * BM);
                 const int h = p.h, pieces = h / 8;  // 16-byte pieces of a row
+                const float wadd = p.norm_mode ? 1.f : 0.f;
                 const uint32_t rb = 2u * (uint32_t)h;
                 for (int st = 0; st < nst; ++st) {
                     const bool got = mbar_wait_bounded(&full[s], ph, abort_flag);
@@ -612,8 +616,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             const uint4 e = tok >= 0 ? lds128(erow + 16 * j) : make_uint4(0, 0, 0, 0);
                             const uint4 we = __ldg(reinterpret_cast<const uint4*>(p.w_ne) + j);
                             const uint4 wh = __ldg(reinterpret_cast<const uint4*>(p.w_nh) + j);
-                            reinterpret_cast<uint4*>(crow)[j] = norm8(e, inv_e, we);
-                            reinterpret_cast<uint4*>(crow + h)[j] = norm8(lds128(xrow + 16 * j), inv_x, wh);
+                            reinterpret_cast<uint4*>(crow)[j] = norm8(e, inv_e, we, wadd);
+                            reinterpret_cast<uint4*>(crow + h)[j] = norm8(lds128(xrow + 16 * j), inv_x, wh, wadd);
                         }
                     }
                     named_sync(1, kEpiThreads);  // everyone is done with the stage
@@ -694,9 +698,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 uint8_t* cache = is_v ? p.v_cache : p.k_cache;
                 const float scale = is_v ? p.v_scale : p.k_scale;
                 const float2* cs = p.rope[tl.c % (p.lanes + 1)] + (int64_t)row * half;
+                const bool kn = !is_v && p.k_norm != nullptr;
+                const float kadd = p.norm_mode ? 1.f : 0.f;
                 for (int h0 = 0; h0 < BN; h0 += p.hd) {
                     const int head_i = ((is_v ? col0 - kvd : col0) + h0) / p.hd;
                     uint8_t* hdst = cache + (slot * p.nkv + head_i) * (int64_t)p.hd;
+                    float kinv = 1.f;
+                    if (kn) {  // per-head k norm: the head's sum of squares of bf16(k) first
+                        float ss = 0.f;
+                        for (int j0 = 0; j0 < p.hd; j0 += 32) {
+                            uint32_t a[32];
+                            tmem_ld32(tb + h0 + j0, a);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) {
+                                const float v = round_bf16(__uint_as_float(a[i]));
+                                ss = fmaf(v, v, ss);
+                            }
+                        }
+                        kinv = 1.0f / sqrtf(ss / (float)p.hd + p.eps);
+                    }
                     for (int j0 = 0; j0 < half; j0 += 32) {
                         uint32_t a[32], b[32];
                         tmem_ld32(tb + h0 + j0, a);
@@ -707,6 +728,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         for (int i = 0; i < 32; ++i) {
                             lo[i] = round_bf16(__uint_as_float(a[i]));
                             hi[i] = round_bf16(__uint_as_float(b[i]));
+                        }
+                        if (kn) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) {
+                                lo[i] = round_bf16(lo[i] * kinv * (bf16_to_f32(p.k_norm[j0 + i]) + kadd));
+                                hi[i] = round_bf16(hi[i] * kinv * (bf16_to_f32(p.k_norm[half + j0 + i]) + kadd));
+                            }
                         }
                         if (!is_v && row_ok) rope32(lo, hi, cs + j0);
                         if (row_ok && slot >= 0) {
@@ -856,6 +884,8 @@ cudaError_t prefill_launch(const PrefillArgs& a, cudaStream_t s) {
     p.w_ne = a.w_norm_embed;
     p.w_nh = a.w_norm_hidden;
     p.eps = a.eps;
+    p.norm_mode = a.norm_mode;
+    p.k_norm = a.k_norm;
     p.nkv = a.nkv;
     p.hd = a.hd;
     p.rope_base = a.rope_base;

@@ -264,12 +264,13 @@ __device__ void stage_bf16(const SweepParams& p, uint16_t* xs, float* scratch) {
             sx = compute_sum<CW>(sx, scratch + CW);
             float inv_e = 1.0f / sqrtf(se / (float)h + p.eps);
             float inv_x = 1.0f / sqrtf(sx / (float)h + p.eps);
+            const float add = p.norm_mode ? 1.f : 0.f;  // weights w or 1 + w
             uint16_t* row = xs + (int64_t)m * p.kpad;
             for (int j = tid; j < h; j += NTH) {
                 float ev = e ? bf16_to_f32(e[j]) : 0.f;
-                row[j] = f32_to_bf16(ev * inv_e * bf16_to_f32(p.w_norm_embed[j]));
+                row[j] = f32_to_bf16(ev * inv_e * (bf16_to_f32(p.w_norm_embed[j]) + add));
                 row[h + j] = f32_to_bf16(bf16_to_f32(hx[j]) * inv_x *
-                                         bf16_to_f32(p.w_norm_hidden[j]));
+                                         (bf16_to_f32(p.w_norm_hidden[j]) + add));
             }
         }
     }

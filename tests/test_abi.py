@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert L.mtp_abi_version() == 1
+    assert L.mtp_abi_version() == 2
     for s in range(6):
         assert L.status_str(s)
     assert L.mtp_devflags_status(0) == L.MTP_OK
@@ -208,7 +208,7 @@ def test_shard_and_merge_rejects(lib):
 
 def test_combine_rejects(lib):
     fc = weight(n=32, k=64)
-    args = [A, 50, B2, B2, 1, 32, OUT, OUT, 1e-6, C.byref(fc), OUT, None, None]
+    args = [A, 50, B2, B2, 1, 32, OUT, OUT, 1e-6, 0, C.byref(fc), OUT, None, None]
     bad = list(args)
     bad[0] = None
     assert st("mtp_combine", *bad) == L.MTP_ERR_INVALID_ARG
@@ -218,17 +218,20 @@ def test_combine_rejects(lib):
     bad = list(args)
     bad[5] = 48
     fc48 = weight(n=48, k=96)  # 192-byte fc rows: not a multiple of 128
-    bad[9] = C.byref(fc48)
+    bad[10] = C.byref(fc48)
     assert st("mtp_combine", *bad) == L.MTP_ERR_UNSUPPORTED
     bad = list(args)
     bad[5] = 24  # h % 16
     assert st("mtp_combine", *bad) == L.MTP_ERR_INVALID_ARG
     fc2 = weight(n=32, k=32)  # fc must be [h, 2h]
     bad = list(args)
-    bad[9] = C.byref(fc2)
+    bad[10] = C.byref(fc2)
     assert st("mtp_combine", *bad) == L.MTP_ERR_INVALID_ARG
     bad = list(args)
     bad[8] = -1.0
+    assert st("mtp_combine", *bad) == L.MTP_ERR_INVALID_ARG
+    bad = list(args)
+    bad[9] = 2  # norm_mode is MTP_NORM_W or MTP_NORM_ONE_PLUS_W
     assert st("mtp_combine", *bad) == L.MTP_ERR_INVALID_ARG
 
 
@@ -245,14 +248,14 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
 
 def prefill_args(**kw):
     a = dict(embed=A, vocab=100, tok=B2, hidden=A, R=10, h=256, wne=OUT, wnh=OUT, eps=1e-6,
-             fc=A, wk=A, wv=A, nkv=2, hd=128, base=1e6, pos=B2, start=0, table=B2, n_table=4,
+             mode=0, fc=A, wk=A, wv=A, kn=None, nkv=2, hd=128, base=1e6, pos=B2, start=0, table=B2, n_table=4,
              bs=16, kc=OUT, vc=OUT, nb=4, ks=1.0, vs=1.0, chunk=8, ws=0x100000, wsb=None,
              err=None)
     a.update(kw)
     if a["wsb"] is None:
         a["wsb"] = L.mtp_prefill_ws_bytes(min(a["chunk"], a["R"]), a["h"], a["nkv"], a["hd"])
     return [a[k] for k in ("embed", "vocab", "tok", "hidden", "R", "h", "wne", "wnh", "eps",
-                           "fc", "wk", "wv", "nkv", "hd", "base", "pos", "start", "table",
+                           "mode", "fc", "wk", "wv", "kn", "nkv", "hd", "base", "pos", "start", "table",
                            "n_table", "bs", "kc", "vc", "nb", "ks", "vs", "chunk", "ws", "wsb",
                            "err")] + [None]
 
@@ -262,6 +265,8 @@ def test_prefill_rejects(lib):
     assert st("mtp_prefill_kv", *prefill_args(embed=None)) == L.MTP_ERR_INVALID_ARG
     assert st("mtp_prefill_kv", *prefill_args(R=0)) == L.MTP_ERR_INVALID_ARG
     assert st("mtp_prefill_kv", *prefill_args(ks=0.0)) == L.MTP_ERR_INVALID_ARG
+    assert st("mtp_prefill_kv", *prefill_args(mode=-1)) == L.MTP_ERR_INVALID_ARG
+    assert st("mtp_prefill_kv", *prefill_args(kn=OUT + 1)) == L.MTP_ERR_INVALID_ARG  # 2-byte
     assert st("mtp_prefill_kv", *prefill_args(h=320)) == L.MTP_ERR_UNSUPPORTED   # h % 256
     assert st("mtp_prefill_kv", *prefill_args(hd=96)) == L.MTP_ERR_UNSUPPORTED
     # a prologue row (embedding + hidden row) must fit one 48 KB ring stage
@@ -296,13 +301,14 @@ def test_wait_timeout_rejects(lib):
 
 
 def test_draft_step_rejects(lib):
-    def ds(M=1, h=256, embed=A, head=B2, mask=None, mw=0, ms=0, idx=OUT, n=100):
-        return st("mtp_draft_step", embed, 100, OUT, A, M, h, A, A, 1e-6, A, head, n, mask, mw, ms,
-                  None, idx, None, None, None)
+    def ds(M=1, h=256, embed=A, head=B2, mask=None, mw=0, ms=0, idx=OUT, n=100, mode=0):
+        return st("mtp_draft_step", embed, 100, OUT, A, M, h, A, A, 1e-6, mode, A, head, n, mask,
+                  mw, ms, None, idx, None, None, None)
     assert ds(embed=None) == L.MTP_ERR_INVALID_ARG
     assert ds(idx=None) == L.MTP_ERR_INVALID_ARG
     assert ds(h=260) == L.MTP_ERR_INVALID_ARG       # h % 8
     assert ds(n=0) == L.MTP_ERR_INVALID_ARG
+    assert ds(mode=3) == L.MTP_ERR_INVALID_ARG
     assert ds(mask=OUT, mw=0) == L.MTP_ERR_INVALID_ARG
     assert ds(M=5) == L.MTP_ERR_UNSUPPORTED         # up to 4 inputs
     assert ds(h=2048) == L.MTP_ERR_UNSUPPORTED      # up to hidden 1024

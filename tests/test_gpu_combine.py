@@ -18,13 +18,13 @@ def draft(M, seed=synth.TINY["seed"], h=synth.TINY["h"], vocab=synth.TINY["vocab
                 else v) for k, v in d.items()}
 
 
-def gpu_combine(d, fc_table=None, tokens=None):
+def gpu_combine(d, fc_table=None, tokens=None, norm_mode=0):
     fc = fc_table or api.bf16_table(to_dev_u16(d["fc"]))
     err = torch.zeros((1,), dtype=torch.int32, device="cuda")
     tok = to_dev(np.asarray(d["tokens"] if tokens is None else tokens, np.int32))
     y = api.combine(to_dev_u16(d["embed"]), tok, to_dev_u16(d["hidden"]),
                     to_dev_u16(d["w_norm_embed"]), to_dev_u16(d["w_norm_hidden"]), d["eps"], fc,
-                    dev_err=err)
+                    dev_err=err, norm_mode=norm_mode)
     torch.cuda.synchronize()
     return u16_of(y), int(err.item())
 
@@ -40,6 +40,20 @@ def test_combine_matches_oracle(orc, M):
     # bf16 outputs: all but a handful identical, none more than one bf16 ulp apart
     diff = np.abs(y.astype(np.int32) - ref.astype(np.int32))
     assert diff.max() <= 1 and (diff > 0).mean() < 0.02
+
+
+@pytest.mark.parametrize("M", [1, 7])
+def test_combine_one_plus_w(orc, M):
+    """norm_mode 1: every norm weight is 1 + w; the plain mode's output must differ."""
+    d = draft(M, seed=77)
+    y, err = gpu_combine(d, norm_mode=L.MTP_NORM_ONE_PLUS_W)
+    ref, _, flags = orc.combine(d["embed"], d["tokens"].numpy(), d["hidden"], d["w_norm_embed"],
+                                d["w_norm_hidden"], d["eps"], d["fc"], norm_mode=1)
+    plain, _, _ = orc.combine(d["embed"], d["tokens"].numpy(), d["hidden"], d["w_norm_embed"],
+                              d["w_norm_hidden"], d["eps"], d["fc"], norm_mode=0)
+    assert err == 0 and flags == 0
+    assert_close(bf16_bits_to_f64(y), bf16_bits_to_f64(ref), "y")
+    assert not np.allclose(bf16_bits_to_f64(plain), bf16_bits_to_f64(ref), rtol=0.05)
 
 
 @pytest.mark.parametrize("h", [32, 512, 1024])
@@ -154,7 +168,7 @@ def test_device_side_draft_chain(orc, M):
         assert np.array_equal(idx_bufs[j].cpu().numpy(), eager[j][1])
 
 
-def gpu_draft_step(d, dd=None, mask=None, mask_words=0, stride=0, tokens=None):
+def gpu_draft_step(d, dd=None, mask=None, mask_words=0, stride=0, tokens=None, norm_mode=0):
     dd = dd or {k: (to_dev_u16(v) if isinstance(v, np.ndarray) and v.dtype == np.uint16 else v)
                 for k, v in d.items()}
     err = torch.zeros((1,), dtype=torch.int32, device="cuda")
@@ -162,7 +176,8 @@ def gpu_draft_step(d, dd=None, mask=None, mask_words=0, stride=0, tokens=None):
     m = to_dev(mask) if mask is not None else None
     idx, val, y = api.draft_step(dd["embed"], tok, dd["hidden"], dd["w_norm_embed"],
                                  dd["w_norm_hidden"], d["eps"], dd["fc"], dd["lm_head"], mask=m,
-                                 mask_words=mask_words, mask_stride_words=stride, dev_err=err)
+                                 mask_words=mask_words, mask_stride_words=stride, dev_err=err,
+                                 norm_mode=norm_mode)
     torch.cuda.synchronize()
     return idx.cpu().numpy(), val.cpu().numpy(), u16_of(y), int(err.item())
 
@@ -181,6 +196,19 @@ def test_draft_step_one_launch(orc, M):
     for m in range(M):
         assert_argmax(int(idx[m]), ref_l[m])
         assert_close([val[m]], [ref_l[m].max()], "out_val")
+
+
+@pytest.mark.parametrize("M", [1, 3])
+def test_draft_step_one_plus_w(orc, M):
+    d = draft(M, seed=78)
+    idx, val, y, err = gpu_draft_step(d, norm_mode=L.MTP_NORM_ONE_PLUS_W)
+    assert err == 0
+    ref_y, _, _ = orc.combine(d["embed"], d["tokens"].numpy(), d["hidden"], d["w_norm_embed"],
+                              d["w_norm_hidden"], d["eps"], d["fc"], norm_mode=1)
+    assert_close(bf16_bits_to_f64(y), bf16_bits_to_f64(ref_y), "y")
+    ref_l, _, _, _ = orc.lm_head_argmax(0, d["lm_head"], d["h"], y)
+    for m in range(M):
+        assert_argmax(int(idx[m]), ref_l[m])
 
 
 @pytest.mark.parametrize("h,vocab", [(64, 1000), (512, 3333), (1024, 5000)])

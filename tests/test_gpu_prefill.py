@@ -112,7 +112,8 @@ def oracle_rows(orc, d, rows):
                             U["w_norm_hidden"], U["eps"], U["fc"], U["wk"], U["wv"], d["nkv"],
                             d["hd"], d["rope_base"], U["rope_pos"], d["cache_start"],
                             U["block_table"], d["block_size"], d["num_blocks"], d["k_scale"],
-                            d["v_scale"], rows)
+                            d["v_scale"], rows, norm_mode=int(d.get("norm_mode", 0)),
+                            k_norm=U.get("k_norm"))
 
 
 def e4m3_step(v):
@@ -168,6 +169,23 @@ def test_prefill_other_heads_and_positions(orc):
     kc, vc, err = run_prefill(d, chunk=64)
     assert err == 0
     check_rows(orc, d, kc, vc, np.arange(70))
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_prefill_k_norm_and_one_plus_w(orc, mode):
+    """A per-head k norm before RoPE, with plain and 1 + w norm weights."""
+    d = synth.prefill_inputs(seed=84 + mode, R=150, vocab=300, h=256, nkv=2, hd=128)
+    g = synth._gen(12 + mode)
+    d["k_norm"] = synth.normal_bf16(g, (128,), 0.3, mean=0.0 if mode else 1.0)
+    d["norm_mode"] = mode
+    kc, vc, err = run_prefill(d, chunk=64)
+    assert err == 0
+    check_rows(orc, d, kc, vc, np.arange(150))
+    # the k norm changes the keys: without it the K codes differ
+    d0 = dict(d)
+    del d0["k_norm"]
+    kc0, _, _ = run_prefill(d0, chunk=64)
+    assert (kc0 != kc).mean() > 0.3
 
 
 def test_prefill_bad_slot_and_token_flags(orc):
