@@ -90,7 +90,7 @@ def lib():
             "orc_prefill_rows_ext": (_i32, [_p, _i64, _p, _p, _i32, _p, _p, C.c_double, _p,
                                             _p, _p, _i32, _i32, C.c_double, _p, _i64, _p,
                                             _i64, _i32, _i64, C.c_float, C.c_float, _i32, _p,
-                                            _p, _i64, _p, _p, _p, _p, _p, _p]),
+                                            _p, _p, _i64, _p, _p, _p, _p, _p, _p]),
             "orc_paged_decode_attn": (_i32, [_p, _i32, _i32, _i32, _p, _p, _p, _i64, _i32,
                                              _i64, _i64, C.c_double, C.c_double, C.c_double,
                                              _p]),
@@ -277,8 +277,9 @@ def kv_encode(vals_bf16, scale):
 
 def prefill_rows(embed, tokens, hidden, w_norm_embed, w_norm_hidden, eps, fc, wk, wv,
                  nkv, hd, rope_base, rope_pos, cache_start, block_table, block_size,
-                 num_blocks, k_scale, v_scale, rows, norm_mode=0, k_norm=None):
-    """Oracle K/V cache entries for the listed prompt rows.
+                 num_blocks, k_scale, v_scale, rows, norm_mode=0, k_norm=None, in_norm=None):
+    """Oracle K/V cache entries for the listed prompt rows (k_norm: per-head k norm
+    weights [hd]; in_norm: the input norm weights [h] applied to y before k and v).
 
     Returns dict with y [n,h], k_rot [n,nkv*hd], v [n,nkv*hd] (bf16 bits), k_codes,
     v_codes [n,nkv*hd] (u8), slot [n] (int64, -1 = not written) and flags.
@@ -297,13 +298,14 @@ def prefill_rows(embed, tokens, hidden, w_norm_embed, w_norm_hidden, eps, fc, wk
     sl = np.empty((n,), dtype=np.int64)
     bt = _c(block_table, np.int32)
     kn = None if k_norm is None else _c(k_norm, np.uint16)
+    inn = None if in_norm is None else _c(in_norm, np.uint16)
     flags = lib().orc_prefill_rows_ext(
         _ptr(embed), embed.shape[0], _ptr(_c(tokens, np.int32)), _ptr(hidden), h,
         _ptr(_c(w_norm_embed, np.uint16)), _ptr(_c(w_norm_hidden, np.uint16)), float(eps),
         _ptr(_c(fc, np.uint16)), _ptr(_c(wk, np.uint16)), _ptr(_c(wv, np.uint16)), nkv, hd,
         float(rope_base), _ptr(_c(rope_pos, np.int32)), int(cache_start), _ptr(bt), bt.size,
         int(block_size), int(num_blocks), float(k_scale), float(v_scale), int(norm_mode),
-        _ptr(kn), _ptr(rows), n, _ptr(y), _ptr(k_rot), _ptr(v), _ptr(kc), _ptr(vc), _ptr(sl))
+        _ptr(kn), _ptr(inn), _ptr(rows), n, _ptr(y), _ptr(k_rot), _ptr(v), _ptr(kc), _ptr(vc), _ptr(sl))
     return dict(y=y, k_rot=k_rot, v=v, k_codes=kc, v_codes=vc, slot=sl, flags=int(flags))
 
 

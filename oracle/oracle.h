@@ -71,6 +71,7 @@ int32_t orc_prefill_rows_ext(const uint16_t* embed, int64_t vocab, const int32_t
                              const int32_t* block_table, int64_t n_table,
                              int32_t block_size, int64_t num_blocks, float k_scale,
                              float v_scale, int32_t mode, const uint16_t* k_norm,
+                             const uint16_t* in_norm,
                              const int64_t* rows, int64_t nrows,
                              uint16_t* out_y, uint16_t* out_k_rot, uint16_t* out_v,
                              uint8_t* out_k_codes, uint8_t* out_v_codes, int64_t* out_slot);

@@ -22,7 +22,10 @@
  * Readings (the pages are silent): by default no norm sits between fc and the k/v
  * projections and no per-head k norm is applied (the benchmark's step list has neither,
  * though the reference scratch has a `normed2` buffer and the head a `k_norm` weight);
- * with `k_norm` given (orc_prefill_rows_ext), each bf16 k head is RMS-normalized over hd
+ * with `in_norm` given (orc_prefill_rows_ext), k and v are projected from
+ * bf16(rms(y) in_norm) -- the decoder layer's input norm, the scratch's `normed2`
+ * buffer -- instead of y (same eps and weight mode as the combiner's norms);
+ * with `k_norm` given, each bf16 k head is RMS-normalized over hd
  * with those weights (same eps and weight mode as the combiner's norms) and rounded to
  * bf16 before RoPE, the usual order of a per-head k norm; RoPE style, rotary dim and theta come from the
  * benchmark configuration (NeoX, full head, base given); the RoPE position of each
@@ -88,7 +91,7 @@ int32_t orc_prefill_rows_ext(const uint16_t* embed, int64_t vocab, const int32_t
                          const int32_t* block_table, int64_t n_table,
                          int32_t block_size, int64_t num_blocks, float k_scale,
                          float v_scale, int32_t mode, const uint16_t* k_norm,
-                         const int64_t* rows, int64_t nrows,
+                         const uint16_t* in_norm, const int64_t* rows, int64_t nrows,
                          uint16_t* out_y, uint16_t* out_k_rot, uint16_t* out_v,
                          uint8_t* out_k_codes, uint8_t* out_v_codes, int64_t* out_slot) {
     int32_t flags = 0;
@@ -97,6 +100,7 @@ int32_t orc_prefill_rows_ext(const uint16_t* embed, int64_t vocab, const int32_t
     for (int64_t i = 0; i < nrows; ++i) {
         int64_t r = rows[i];
         uint16_t* y = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)h);
+        uint16_t* n2 = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)h);
         uint16_t* kb = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)kvd);
         uint16_t* vb = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)kvd);
         double* kd = (double*)malloc(sizeof(double) * (size_t)hd);
@@ -104,8 +108,14 @@ int32_t orc_prefill_rows_ext(const uint16_t* embed, int64_t vocab, const int32_t
         int32_t tok = tokens[r];
         flags |= orc_combine_mode(embed, vocab, &tok, hidden + r * (int64_t)h, 1, h,
                                   w_norm_embed, w_norm_hidden, eps, mode, fc, NULL, y);
-        matvec_bf16(wk, kvd, h, y, kb);
-        matvec_bf16(wv, kvd, h, y, vb);
+        /* the decoder layer's input norm (the scratch's normed2), when given, feeds k and v */
+        const uint16_t* a = y;
+        if (in_norm) {
+            orc_rmsnorm_row_mode(y, in_norm, h, eps, mode, n2);
+            a = n2;
+        }
+        matvec_bf16(wk, kvd, h, a, kb);
+        matvec_bf16(wv, kvd, h, a, vb);
         for (int32_t hh = 0; hh < nkv; ++hh) {
             if (k_norm)  /* per-head RMSNorm of k over hd, before RoPE */
                 orc_rmsnorm_row_mode(kb + hh * hd, k_norm, hd, eps, mode, kb + hh * hd);
@@ -125,6 +135,7 @@ int32_t orc_prefill_rows_ext(const uint16_t* embed, int64_t vocab, const int32_t
         if (s < 0) flags |= ORC_FLAG_BAD_SLOT;
         out_slot[i] = s;
         free(y);
+        free(n2);
         free(kb);
         free(vb);
         free(kd);
@@ -146,6 +157,7 @@ int32_t orc_prefill_rows(const uint16_t* embed, int64_t vocab, const int32_t* to
                          uint8_t* out_k_codes, uint8_t* out_v_codes, int64_t* out_slot) {
     return orc_prefill_rows_ext(embed, vocab, tokens, hidden, h, w_norm_embed, w_norm_hidden, eps,
                                 fc, wk, wv, nkv, hd, rope_base, rope_pos, cache_start, block_table,
-                                n_table, block_size, num_blocks, k_scale, v_scale, 0, NULL, rows,
+                                n_table, block_size, num_blocks, k_scale, v_scale, 0, NULL, NULL,
+                                rows,
                                 nrows, out_y, out_k_rot, out_v, out_k_codes, out_v_codes, out_slot);
 }

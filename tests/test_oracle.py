@@ -740,3 +740,57 @@ def test_k_norm_comes_before_rope(orc):
             kn = bf16_to_f64_(orc.f64_to_bf16(s * bf16_to_f64_(w)))
             want = orc.f64_to_bf16(orc.rope_neox(kn, 37.0, U["rope_base"]))
             assert np.array_equal(got[r, hh], want), (r, hh)
+
+
+# ---------------------------------------------------------------- input norm (normed2) pins
+def _in_case(orc, seed, in_norm, norm_mode=0, fc_scale=1.0, eps=None, onehot_v=False):
+    d = synth.prefill_inputs(seed=seed, R=5, vocab=40, h=256, nkv=2, hd=64)
+    if fc_scale != 1.0:
+        d["fc"] = (d["fc"].float() * fc_scale).to(torch.bfloat16)
+    if eps is not None:
+        d["eps"] = eps
+    if onehot_v:  # row i of Wv selects element (7 i + 3) mod h
+        wv = torch.zeros_like(d["wv"])
+        for i in range(wv.shape[0]):
+            wv[i, (7 * i + 3) % 256] = 1.0
+        d["wv"] = wv
+    U = {k: (synth.as_u16(v) if isinstance(v, torch.Tensor) and v.dtype == torch.bfloat16 else
+             (v.numpy() if isinstance(v, torch.Tensor) else v)) for k, v in d.items()}
+    out = orc.prefill_rows(U["embed"], U["tokens"], U["hidden"], U["w_norm_embed"],
+                           U["w_norm_hidden"], U["eps"], U["fc"], U["wk"], U["wv"], 2, 64,
+                           U["rope_base"], U["rope_pos"], 0, U["block_table"], 16,
+                           U["num_blocks"], 1.0, 1.0, np.arange(5), norm_mode=norm_mode,
+                           in_norm=in_norm)
+    return out, U
+
+
+def test_in_norm_feeds_k_and_v_through_the_pinned_rmsnorm(orc):
+    """One-hot Wv rows read single elements of k/v's input: with the input norm that input is
+    the (separately pinned) RMSNorm of the stored fc output y, in both weight modes."""
+    rng = np.random.default_rng(35)
+    w = orc.f64_to_bf16(rng.normal(0.5, 0.4, 256))
+    for mode in (0, 1):
+        out, U = _in_case(orc, 51, w, norm_mode=mode, onehot_v=True)
+        for r in range(5):
+            n2 = orc.rmsnorm(out["y"][r], w, U["eps"], norm_mode=mode)
+            want = n2[(7 * np.arange(128) + 3) % 256]
+            assert np.array_equal(out["v"][r], want), (mode, r)
+    plain, _ = _in_case(orc, 51, None, onehot_v=True)
+    assert np.array_equal(plain["v"][0], plain["y"][0][(7 * np.arange(128) + 3) % 256])
+
+
+def test_in_norm_zero_weights_and_scale_invariance(orc):
+    """Zero input-norm weights (plain mode) zero k and v. With eps = 0, doubling fc doubles
+    y exactly; the normed input, hence k and v, stay bit-identical -- and without the input
+    norm v doubles exactly, so the invariance is the norm's."""
+    zero = np.zeros(256, np.uint16)
+    out, _ = _in_case(orc, 52, zero)
+    assert np.all(bf16_to_f64_(out["k_rot"]) == 0) and np.all(bf16_to_f64_(out["v"]) == 0)
+    w = orc.f64_to_bf16(np.random.default_rng(36).normal(1.0, 0.2, 256))
+    a, _ = _in_case(orc, 53, w, eps=0.0)
+    b, _ = _in_case(orc, 53, w, eps=0.0, fc_scale=2.0)
+    assert np.array_equal(bf16_to_f64_(b["y"]), 2 * bf16_to_f64_(a["y"]))
+    assert np.array_equal(a["k_rot"], b["k_rot"]) and np.array_equal(a["v"], b["v"])
+    pa, _ = _in_case(orc, 53, None, eps=0.0)
+    pb, _ = _in_case(orc, 53, None, eps=0.0, fc_scale=2.0)
+    assert np.array_equal(bf16_to_f64_(pb["v"]), 2 * bf16_to_f64_(pa["v"]))
