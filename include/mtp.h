@@ -41,7 +41,7 @@ extern "C" {
 #endif
 
 /* 2: mtp_combine, mtp_draft_step and mtp_prefill_kv take norm_mode; mtp_prefill_kv takes
- * k_norm. */
+ * k_norm and in_norm. */
 #define MTP_ABI_VERSION 2
 
 typedef enum {
@@ -332,7 +332,9 @@ mtp_status mtp_argmax_merge_partials(const void* partials, int32_t n_parts, int3
  * forward_one step 4 (block = block_table[pos / bs], slot = block * bs + pos % bs).
  * Per row r (all intermediate activations rounded to bf16):
  *   c = [rms(embed[token_ids[r]]) w_norm_embed || rms(hidden[r]) w_norm_hidden]
- *   y = fc . c;  k = wk . y;  v = wv . y;  k' = NeoX RoPE over each head of hd at
+ *   y = fc . c;  a = y, or, when in_norm is given, a = rms(y) in_norm (the decoder
+ *   layer's input norm, the scratch's normed2 buffer);
+ *   k = wk . a;  v = wv . a;  k' = NeoX RoPE over each head of hd at
  *   position rope_pos[r] (theta_j = pos * rope_base^(-2j/hd)) of k, or, when k_norm is
  *   given, of bf16(k_head / sqrt(mean(k_head^2) + eps) * k_norm) per head ([new.rs] and
  *   [mtp_head.rs] list the head's per-head k_norm weight; the norm precedes RoPE here);
@@ -345,6 +347,7 @@ mtp_status mtp_argmax_merge_partials(const void* partials, int32_t n_parts, int3
  *   embed (device) bf16 [vocab, h]; token_ids, rope_pos (device) i32 [R];
  *   hidden (device) bf16 [R, h]; w_norm_* (device) bf16 [h]; fc (device) bf16 [h, 2h];
  *   wk, wv (device) bf16 [nkv * hd, h]; k_norm (device) bf16 [hd] or NULL;
+ *   in_norm (device) bf16 [h] or NULL (16-byte aligned);
  *   block_table (device) i32 [n_table];
  *   k_cache, v_cache (device) u8 [num_blocks, block_size, nkv, hd], written in place;
  *   ws (device) mtp_prefill_ws_bytes(min(chunk_rows, R), h, nkv, hd) bytes, 1 KB
@@ -366,8 +369,8 @@ mtp_status mtp_prefill_kv(const uint16_t* embed, int64_t vocab, const int32_t* t
                           const uint16_t* hidden, int64_t R, int32_t h,
                           const uint16_t* w_norm_embed, const uint16_t* w_norm_hidden, float eps,
                           int32_t norm_mode, const uint16_t* fc, const uint16_t* wk,
-                          const uint16_t* wv, const uint16_t* k_norm, int32_t nkv,
-                          int32_t hd, float rope_base, const int32_t* rope_pos,
+                          const uint16_t* wv, const uint16_t* k_norm, const uint16_t* in_norm,
+                          int32_t nkv, int32_t hd, float rope_base, const int32_t* rope_pos,
                           int64_t cache_start, const int32_t* block_table, int64_t n_table,
                           int32_t block_size, uint8_t* k_cache, uint8_t* v_cache,
                           int64_t num_blocks, float k_scale, float v_scale, int64_t chunk_rows,

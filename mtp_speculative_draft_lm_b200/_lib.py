@@ -89,7 +89,7 @@ _SIGS = {
     "mtp_argmax_merge_partials": (C.c_int, [_P, _I32, _I32, _P, _P, _P, _P, _P]),
     "mtp_prefill_ws_bytes": (_SZ, [_I64, _I32, _I32, _I32]),
     "mtp_prefill_kv": (C.c_int, [_P, _I64, _P, _P, _I64, _I32, _P, _P, C.c_float, _I32, _P, _P,
-                                 _P, _P, _I32, _I32, C.c_float, _P, _I64, _P, _I64, _I32, _P, _P,
+                                 _P, _P, _P, _I32, _I32, C.c_float, _P, _I64, _P, _I64, _I32, _P, _P,
                                  _I64, C.c_float, C.c_float, _I64, _P, _SZ, _P, _P]),
     "mtp_debug_gemm_bf16": (C.c_int, [_P, _P, _P, _I32, _I32, _I32, _P]),
     "mtp_debug_kv_write": (C.c_int, [_P, _P, _I64, _I32, _I32, _I64, _P, _I64, _I32, _I64, _P,
@@ -254,12 +254,14 @@ def mtp_prefill_ws_bytes(chunk_rows, h, nkv, hd) -> int:
 
 
 def mtp_prefill_kv(embed, vocab, token_ids, hidden, R, h, w_norm_embed, w_norm_hidden, eps,
-                   norm_mode, fc, wk, wv, k_norm, nkv, hd, rope_base, rope_pos, cache_start,
+                   norm_mode, fc, wk, wv, k_norm, in_norm, nkv, hd, rope_base, rope_pos,
+                   cache_start,
                    block_table, n_table, block_size, k_cache, v_cache, num_blocks, k_scale,
                    v_scale, chunk_rows, ws, ws_bytes, dev_err=None, stream=None):
     _check(load().mtp_prefill_kv(_ptr(embed), vocab, _ptr(token_ids), _ptr(hidden), R, h,
                                  _ptr(w_norm_embed), _ptr(w_norm_hidden), float(eps),
-                                 int(norm_mode), _ptr(fc), _ptr(wk), _ptr(wv), _ptr(k_norm), nkv,
+                                 int(norm_mode), _ptr(fc), _ptr(wk), _ptr(wv), _ptr(k_norm),
+                                 _ptr(in_norm), nkv,
                                  hd, float(rope_base), _ptr(rope_pos),
                                  cache_start, _ptr(block_table), n_table, block_size,
                                  _ptr(k_cache), _ptr(v_cache), num_blocks, float(k_scale),

@@ -265,7 +265,7 @@ def aligned_empty(nbytes: int, align: int, device) -> torch.Tensor:
 def prefill_kv(inputs: dict, k_cache: torch.Tensor, v_cache: torch.Tensor, chunk_rows: int = 2048,
                ws: torch.Tensor | None = None, dev_err: torch.Tensor | None = None, stream=None):
     """Drafter-context prefill over device tensors named as in synth.prefill_inputs (plus the
-    optional "norm_mode" and "k_norm" [hd] entries)."""
+    optional "norm_mode", "k_norm" [hd] and "in_norm" [h] entries)."""
     d = inputs
     R, h = d["hidden"].shape
     nkv, hd = int(d["nkv"]), int(d["hd"])
@@ -275,7 +275,7 @@ def prefill_kv(inputs: dict, k_cache: torch.Tensor, v_cache: torch.Tensor, chunk
         ws = aligned_empty(nbytes, 1024, k_cache.device)
     L.mtp_prefill_kv(d["embed"], d["embed"].shape[0], d["tokens"], d["hidden"], R, h,
                      d["w_norm_embed"], d["w_norm_hidden"], d["eps"], int(d.get("norm_mode", 0)),
-                     d["fc"], d["wk"], d["wv"], d.get("k_norm"), nkv, hd, d["rope_base"],
+                     d["fc"], d["wk"], d["wv"], d.get("k_norm"), d.get("in_norm"), nkv, hd, d["rope_base"],
                      d["rope_pos"], int(d["cache_start"]),
                      d["block_table"], d["block_table"].numel(), int(d["block_size"]), k_cache,
                      v_cache, k_cache.shape[0], d["k_scale"], d["v_scale"], chunk, ws, ws.numel(),

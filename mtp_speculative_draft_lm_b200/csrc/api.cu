@@ -377,8 +377,8 @@ mtp_status mtp_prefill_kv(const uint16_t* embed, int64_t vocab, const int32_t* t
                           const uint16_t* hidden, int64_t R, int32_t h,
                           const uint16_t* w_norm_embed, const uint16_t* w_norm_hidden, float eps,
                           int32_t norm_mode, const uint16_t* fc, const uint16_t* wk,
-                          const uint16_t* wv, const uint16_t* k_norm, int32_t nkv,
-                          int32_t hd, float rope_base, const int32_t* rope_pos,
+                          const uint16_t* wv, const uint16_t* k_norm, const uint16_t* in_norm,
+                          int32_t nkv, int32_t hd, float rope_base, const int32_t* rope_pos,
                           int64_t cache_start, const int32_t* block_table, int64_t n_table,
                           int32_t block_size, uint8_t* k_cache, uint8_t* v_cache,
                           int64_t num_blocks, float k_scale, float v_scale, int64_t chunk_rows,
@@ -389,7 +389,8 @@ mtp_status mtp_prefill_kv(const uint16_t* embed, int64_t vocab, const int32_t* t
     if (vocab < 1 || R < 1 || h < 1 || nkv < 1 || hd < 2 || block_size < 1 || n_table < 1 ||
         num_blocks < 1 || chunk_rows < 1 || !(eps >= 0.f) || !finite_pos(k_scale) ||
         !finite_pos(v_scale) || !(rope_base > 0.f) || cache_start < 0 ||
-        (norm_mode != MTP_NORM_W && norm_mode != MTP_NORM_ONE_PLUS_W) || !aligned(k_norm, 2))
+        (norm_mode != MTP_NORM_W && norm_mode != MTP_NORM_ONE_PLUS_W) || !aligned(k_norm, 2) ||
+        !aligned(in_norm, 16))
         return MTP_ERR_INVALID_ARG;
     const int tn = mtp::gemm_tile_n();
     if (h % tn || h > mtp::prefill_max_hidden() || (hd != 64 && hd != 128 && hd != 256) ||
@@ -418,6 +419,7 @@ mtp_status mtp_prefill_kv(const uint16_t* embed, int64_t vocab, const int32_t* t
     a.wk = wk;
     a.wv = wv;
     a.k_norm = k_norm;
+    a.in_norm = in_norm;
     a.nkv = nkv;
     a.hd = hd;
     a.rope_base = (double)rope_base;

@@ -111,6 +111,7 @@ struct PrefillArgs {
     const uint16_t* wk;
     const uint16_t* wv;
     const uint16_t* k_norm;  // [hd] or null: per-head RMSNorm of k before RoPE
+    const uint16_t* in_norm;  // [h] or null: RMSNorm of the fc output before k and v
     int32_t nkv, hd;
     double rope_base;
     const int32_t* rope_pos;

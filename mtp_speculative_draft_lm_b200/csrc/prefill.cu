@@ -7,7 +7,9 @@
 // metrale_model_arch/deepseek_v4_mtp.rs forward_one step 4). Per prompt row r:
 //   c  = [bf16(rms(embed[tok_r]) w_e) || bf16(rms(hidden_r) w_h)]           (prologue)
 //   y  = bf16(fc . c)                                                   (fc GEMM)
+//   (optional input norm: y <- bf16(rms(y) w_in), by the row block's last fc tile)
 //   k  = bf16(Wk . y), v = bf16(Wv . y)                                 (k/v GEMM)
+//   (optional per-head k norm before RoPE, in the k/v epilogue)
 //   k' = bf16(RoPE_neox(k, pos_r)) per head, codes = e4m3(k' / k_scale), e4m3(v / v_scale)
 //   cache row p = cache_start + r, slot = block_table[p / bs] * bs + p % bs,
 //   element (slot, head, d) of a [num_blocks, bs, nkv, hd] cache.       (k/v epilogue)
@@ -68,6 +70,7 @@ constexpr int kHeadBytes = 4096;
 constexpr int kGemmSmem = kGStages * kGStageBytes + kHeadBytes + 1024 /* align */;
 
 enum : int { TILE_P = 0, TILE_F = 1, TILE_V = 2 };
+constexpr int kArrivals = 3;  // counter kind: F tiles that finished (input norm only)
 
 struct PrefillParams {
     // inputs
@@ -82,6 +85,7 @@ struct PrefillParams {
     float eps;
     int norm_mode;           // 0: weights w, 1: weights 1 + w
     const uint16_t* k_norm;  // [hd] or null: per-head RMSNorm of k before RoPE
+    const uint16_t* in_norm;  // [h] or null: RMSNorm of y (in place) before the k/v GEMM
     int nkv, hd;
     double rope_base;
     const int32_t* rope_pos;
@@ -106,7 +110,7 @@ struct PrefillParams {
     int64_t total;       // tiles in all
     int lanes;           // 1 or 2
     int rows_per_pstage;
-    uint32_t* ctr;       // [0] tile counter; then done counters [3][kCtrSlots][mt_full]
+    uint32_t* ctr;       // [0] tile counter; then done counters [4][kCtrSlots][mt_full]
     uint16_t* concat[kMaxLanes];
     uint16_t* y[kMaxLanes];
     float2* rope[kMaxLanes + 1];
@@ -192,9 +196,11 @@ __device__ Tile decode(const PrefillParams& p, int64_t t) {
     return r;
 }
 
-// Completion counters: kind k (P, F, V) of the chunks in slot c % 4, row block m. They
-// only grow within a call: after chunk c's tiles of row block m are all done, the P
-// counter reads c / 4 + 1, F (c / 4 + 1) nf, V (c / 4 + 1) nv.
+// Completion counters: kind k (P, F, V, F arrivals) of the chunks in slot c % 4, row
+// block m. They only grow within a call: after chunk c's tiles of row block m are all
+// done, the P counter reads c / 4 + 1, F (c / 4 + 1) nf, V (c / 4 + 1) nv. With the input
+// norm the F tiles count themselves on the arrivals counter instead, and the last of a row
+// block normalizes the block's fc output rows in place, then adds nf to the F counter.
 __device__ __forceinline__ uint32_t* counter(const PrefillParams& p, int kind, int c, int m) {
     return p.ctr + 64 + ((size_t)kind * kCtrSlots + (size_t)(c % kCtrSlots)) * p.mt_full + m;
 }
@@ -302,6 +308,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int* fifo = reinterpret_cast<int*>(qempty + kFifo);          // [kFifo]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fifo + kFifo);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* last_flag = abort_flag + 1;  // this F tile was its row block's last
     int* stage_tok = reinterpret_cast<int*>(head + 512);         // [kGStages][8]
     float* red = reinterpret_cast<float*>(head + 1024);          // [2][4 warps][2]
     double* inv_freq = reinterpret_cast<double*>(head + 2048);   // [hd / 2 <= 128]
@@ -746,10 +753,46 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             tc_fence_before();
             named_sync(1, kEpiThreads);  // the accumulator is read, every store issued
+            const bool norm_y = tl.kind == TILE_F && !p.plain && p.in_norm != nullptr;
             if (et == 0) {
                 mbar_arrive(&tempty[buf]);
-                if (!p.plain && !*abort_flag)
+                if (!p.plain && !*abort_flag && !norm_y)
                     counter_release_add(counter(p, tl.kind, tl.c, tl.m), 1u);
+                if (norm_y) {
+                    int last = 0;
+                    if (!*abort_flag) {
+                        fence_acq_rel_gpu();  // release this tile's y stores
+                        const uint32_t old = atomicAdd(counter(p, kArrivals, tl.c, tl.m), 1u);
+                        last = old + 1u == (uint32_t)((tl.c / kCtrSlots + 1) * p.nf);
+                        fence_acq_rel_gpu();  // acquire the other tiles' stores
+                    }
+                    *last_flag = last;
+                }
+            }
+            if (norm_y) {
+                named_sync(1, kEpiThreads);
+                if (*last_flag) {
+                    // the row block's input norm, in place: a warp per row, L2 loads (the
+                    // rows were written by other SMs)
+                    uint16_t* Y = p.y[tl.c % p.lanes];
+                    const int h = p.h, pieces = h / 8;
+                    const int nrow = (int)min((int64_t)BM, rows_c - (int64_t)tl.m * BM);
+                    const float wadd = p.norm_mode ? 1.f : 0.f;
+                    const uint4* wn = reinterpret_cast<const uint4*>(p.in_norm);
+                    for (int r = ew; r < nrow; r += kEpiThreads / 32) {
+                        uint4* yr = reinterpret_cast<uint4*>(Y + ((int64_t)tl.m * BM + r) * h);
+                        float ss = 0.f;
+                        for (int j = lane; j < pieces; j += 32) ss += sumsq8(__ldcg(yr + j));
+#pragma unroll
+                        for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+                        const float inv = 1.0f / sqrtf(ss / (float)h + p.eps);
+                        for (int j = lane; j < pieces; j += 32)
+                            __stcg(yr + j, norm8(__ldcg(yr + j), inv, __ldg(wn + j), wadd));
+                    }
+                    fence_proxy_async_global();  // read by the k/v tiles' TMA
+                    named_sync(1, kEpiThreads);
+                    if (et == 0) counter_release_add(counter(p, TILE_F, tl.c, tl.m), (uint32_t)p.nf);
+                }
             }
         }
     }
@@ -844,7 +887,7 @@ constexpr size_t kCtrHeader = 256;  // tile counter (and room), before the done 
 size_t up1k(size_t b) { return (b + 1023) & ~(size_t)1023; }
 size_t header_bytes(int64_t chunk_rows) {
     const size_t mt = (size_t)((chunk_rows + BM - 1) / BM);
-    return up1k(kCtrHeader + 3 * kCtrSlots * mt * sizeof(uint32_t));
+    return up1k(kCtrHeader + 4 * kCtrSlots * mt * sizeof(uint32_t));
 }
 size_t concat_bytes(int64_t c, int32_t h) { return up1k((size_t)c * 2 * h * 2); }
 size_t y_bytes(int64_t c, int32_t h) { return up1k((size_t)c * h * 2); }
@@ -886,6 +929,7 @@ cudaError_t prefill_launch(const PrefillArgs& a, cudaStream_t s) {
     p.eps = a.eps;
     p.norm_mode = a.norm_mode;
     p.k_norm = a.k_norm;
+    p.in_norm = a.in_norm;
     p.nkv = a.nkv;
     p.hd = a.hd;
     p.rope_base = a.rope_base;

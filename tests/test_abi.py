@@ -248,14 +248,14 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
 
 def prefill_args(**kw):
     a = dict(embed=A, vocab=100, tok=B2, hidden=A, R=10, h=256, wne=OUT, wnh=OUT, eps=1e-6,
-             mode=0, fc=A, wk=A, wv=A, kn=None, nkv=2, hd=128, base=1e6, pos=B2, start=0, table=B2, n_table=4,
+             mode=0, fc=A, wk=A, wv=A, kn=None, inn=None, nkv=2, hd=128, base=1e6, pos=B2, start=0, table=B2, n_table=4,
              bs=16, kc=OUT, vc=OUT, nb=4, ks=1.0, vs=1.0, chunk=8, ws=0x100000, wsb=None,
              err=None)
     a.update(kw)
     if a["wsb"] is None:
         a["wsb"] = L.mtp_prefill_ws_bytes(min(a["chunk"], a["R"]), a["h"], a["nkv"], a["hd"])
     return [a[k] for k in ("embed", "vocab", "tok", "hidden", "R", "h", "wne", "wnh", "eps",
-                           "mode", "fc", "wk", "wv", "kn", "nkv", "hd", "base", "pos", "start", "table",
+                           "mode", "fc", "wk", "wv", "kn", "inn", "nkv", "hd", "base", "pos", "start", "table",
                            "n_table", "bs", "kc", "vc", "nb", "ks", "vs", "chunk", "ws", "wsb",
                            "err")] + [None]
 
@@ -267,6 +267,7 @@ def test_prefill_rejects(lib):
     assert st("mtp_prefill_kv", *prefill_args(ks=0.0)) == L.MTP_ERR_INVALID_ARG
     assert st("mtp_prefill_kv", *prefill_args(mode=-1)) == L.MTP_ERR_INVALID_ARG
     assert st("mtp_prefill_kv", *prefill_args(kn=OUT + 1)) == L.MTP_ERR_INVALID_ARG  # 2-byte
+    assert st("mtp_prefill_kv", *prefill_args(inn=OUT + 8)) == L.MTP_ERR_INVALID_ARG  # 16-byte
     assert st("mtp_prefill_kv", *prefill_args(h=320)) == L.MTP_ERR_UNSUPPORTED   # h % 256
     assert st("mtp_prefill_kv", *prefill_args(hd=96)) == L.MTP_ERR_UNSUPPORTED
     # a prologue row (embedding + hidden row) must fit one 48 KB ring stage

@@ -113,7 +113,7 @@ def oracle_rows(orc, d, rows):
                             d["hd"], d["rope_base"], U["rope_pos"], d["cache_start"],
                             U["block_table"], d["block_size"], d["num_blocks"], d["k_scale"],
                             d["v_scale"], rows, norm_mode=int(d.get("norm_mode", 0)),
-                            k_norm=U.get("k_norm"))
+                            k_norm=U.get("k_norm"), in_norm=U.get("in_norm"))
 
 
 def e4m3_step(v):
@@ -186,6 +186,26 @@ def test_prefill_k_norm_and_one_plus_w(orc, mode):
     del d0["k_norm"]
     kc0, _, _ = run_prefill(d0, chunk=64)
     assert (kc0 != kc).mean() > 0.3
+
+
+@pytest.mark.parametrize("mode,k_norm", [(0, False), (1, True)])
+def test_prefill_input_norm(orc, mode, k_norm):
+    """The input norm between fc and k/v (done in place by each row block's last fc tile):
+    three chunks (the last ragged), two fc column tiles per row block, with and without
+    the k norm."""
+    d = synth.prefill_inputs(seed=86 + mode, R=300, vocab=300, h=512, nkv=2, hd=128)
+    g = synth._gen(14 + mode)
+    d["in_norm"] = synth.normal_bf16(g, (512,), 0.3, mean=0.0 if mode else 1.0)
+    if k_norm:
+        d["k_norm"] = synth.normal_bf16(g, (128,), 0.3, mean=0.0 if mode else 1.0)
+    d["norm_mode"] = mode
+    kc, vc, err = run_prefill(d, chunk=128)
+    assert err == 0
+    check_rows(orc, d, kc, vc, np.arange(300))
+    d0 = dict(d)
+    del d0["in_norm"]
+    _, vc0, _ = run_prefill(d0, chunk=128)
+    assert (vc0 != vc).mean() > 0.3
 
 
 def test_prefill_bad_slot_and_token_flags(orc):
