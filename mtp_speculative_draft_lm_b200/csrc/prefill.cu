@@ -27,8 +27,8 @@
 //   F (c, m, n): a 128 x 256 tile of the fc GEMM, y = c . fc^T, bf16 out.
 //   V (c, m, n): a 128 x 256 tile of the k/v GEMM whose epilogue rotates k (RoPE),
 //     encodes E4M3 and writes each row's 32-byte pieces at its paged slot.
-// Order: for b = 0..chunks: P(b), F(b), then V(b - 1) (with a single lane V(b - 1)
-// first). A tile only ever waits for tiles earlier in that order (completion counters per chunk slot and row block, in the
+// Order: for b = 0..chunks: P(b + 1), F(b), then V(b - 1) (block 0 starts with P(0); with a
+// single lane the order is V(b - 1), P(b), F(b)). A tile only ever waits for tiles earlier in that order (completion counters per chunk slot and row block, in the
 // workspace header, release/acquire at GPU scope): F(c, m, .) for P(c, m); V(c, m, .)
 // for all of F(c, m, .); and a tile that overwrites a buffer another chunk used (two
 // lanes of concat and fc-output rows, three of RoPE rows) for that chunk's readers.
@@ -64,8 +64,8 @@ constexpr int kFifo = 8;           // tiles announced ahead to the MMA and epilo
 constexpr int kCtrSlots = 4;       // completion counters: chunk c uses slot c % 4
 constexpr int kMaxRowsPerPStage = 8;
 constexpr int kMaxLanes = 2;       // concat / fc-output lanes (RoPE rows: lanes + 1)
-// shared memory after the ring: barriers, the tile FIFO, per-stage row tokens, the
-// epilogue's reduction scratch and inverse frequencies
+// shared memory after the ring: barriers, the tile FIFO, per-stage row tokens and the
+// inverse frequencies
 constexpr int kHeadBytes = 4096;
 constexpr int kGemmSmem = kGStages * kGStageBytes + kHeadBytes + 1024 /* align */;
 
@@ -106,7 +106,6 @@ struct PrefillParams {
     int mt_last;         // of the last chunk
     int nf;              // fc GEMM column tiles (h / 256)
     int nv;              // k/v GEMM column tiles (2 nkv hd / 256)
-    int64_t b0, s_mid, n_mid, b_last;  // tiles in block 0, a middle block, the last but one
     int64_t total;       // tiles in all
     int lanes;           // 1 or 2
     int rows_per_pstage;
@@ -127,7 +126,23 @@ __device__ __forceinline__ int mt_of(const PrefillParams& p, int c) {
     return c == p.n_chunks - 1 ? p.mt_last : p.mt_full;
 }
 
-// Tile t of the global order: block b holds P(b), F(b) (b < chunks) and V(b - 1) (b >= 1).
+// Row blocks of chunks 0 .. k - 1.
+__device__ __forceinline__ int64_t cum_mt(const PrefillParams& p, int k) {
+    k = max(0, min(k, p.n_chunks));
+    return k <= p.n_chunks - 1 ? (int64_t)k * p.mt_full
+                               : (int64_t)(p.n_chunks - 1) * p.mt_full + p.mt_last;
+}
+
+// First tile of block b (b = 0 .. n_chunks + 1). With two lanes block b holds P(b + 1),
+// F(b), V(b - 1) -- the prologue runs a chunk ahead, so a chunk's fc tiles find their
+// concat rows ready -- and block 0 also P(0) first; with one lane V(b - 1), P(b), F(b),
+// since F(b) then reuses the fc-output rows V(b - 1) reads.
+__device__ __forceinline__ int64_t block_start(const PrefillParams& p, int b) {
+    const int64_t pc = p.lanes == 2 ? (b == 0 ? 0 : cum_mt(p, b + 1)) : cum_mt(p, b);
+    return pc + p.nf * cum_mt(p, b) + p.nv * cum_mt(p, b - 1);
+}
+
+// Tile t of the global order.
 __device__ Tile decode(const PrefillParams& p, int64_t t) {
     Tile r{};
     if (p.plain) {  // F tiles of one GEMM, M-fastest
@@ -138,60 +153,41 @@ __device__ Tile decode(const PrefillParams& p, int64_t t) {
         r.n = (int)(t / mt);
         return r;
     }
-    int b;
-    int64_t off;
-    if (t < p.b0) {
-        b = 0;
-        off = t;
-    } else {
-        t -= p.b0;
-        if (t < p.n_mid * p.s_mid) {
-            b = 1 + (int)(t / p.s_mid);
-            off = t % p.s_mid;
+    int lo = 0, hi = p.n_chunks;  // the last block starting at or before t
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (block_start(p, mid) <= t) lo = mid;
+        else hi = mid - 1;
+    }
+    const int b = lo, n = p.n_chunks;
+    int64_t off = t - block_start(p, b);
+    // the block's segments in order; the tile is in the first one that still covers off
+    bool found = false;
+    auto seg = [&](int kind, int c) {
+        if (found) return;
+        const int mt = mt_of(p, c);
+        const int64_t cnt = (int64_t)mt * (kind == TILE_P ? 1 : kind == TILE_F ? p.nf : p.nv);
+        if (off < cnt) {
+            r.kind = kind;
+            r.c = c;
+            r.m = (int)(off % mt);
+            r.n = (int)(off / mt);
+            found = true;
         } else {
-            t -= p.n_mid * p.s_mid;
-            if (p.n_chunks >= 2 && t < p.b_last) {
-                b = p.n_chunks - 1;
-                off = t;
-            } else {
-                if (p.n_chunks >= 2) t -= p.b_last;
-                b = p.n_chunks;
-                off = t;
-            }
+            off -= cnt;
         }
-    }
-    // with two lanes a block is P(b), F(b), V(b - 1); with one lane V(b - 1) comes first,
-    // since F(b) then reuses the fc-output rows V(b - 1) reads
-    const int mtb = b < p.n_chunks ? mt_of(p, b) : 0;
-    if (p.lanes == 1 && b >= 1) {
-        const int mtv = mt_of(p, b - 1);
-        const int64_t nvb = (int64_t)mtv * p.nv;
-        if (off < nvb) {
-            r.kind = TILE_V;
-            r.c = b - 1;
-            r.m = (int)(off % mtv);
-            r.n = (int)(off / mtv);
-            return r;
-        }
-        off -= nvb;
-    }
-    if (off < mtb) {
-        r.kind = TILE_P;
-        r.c = b;
-        r.m = (int)off;
-    } else if (off < (int64_t)mtb * (1 + p.nf)) {
-        const int64_t i = off - mtb;
-        r.kind = TILE_F;
-        r.c = b;
-        r.m = (int)(i % mtb);
-        r.n = (int)(i / mtb);
+    };
+    if (p.lanes == 2) {
+        if (b == 0) seg(TILE_P, 0);
+        if (b + 1 < n) seg(TILE_P, b + 1);
+        if (b < n) seg(TILE_F, b);
+        if (b >= 1) seg(TILE_V, b - 1);
     } else {
-        const int64_t i = off - (int64_t)mtb * (1 + p.nf);
-        const int mtv = mt_of(p, b - 1);
-        r.kind = TILE_V;
-        r.c = b - 1;
-        r.m = (int)(i % mtv);
-        r.n = (int)(i / mtv);
+        if (b >= 1) seg(TILE_V, b - 1);
+        if (b < n) {
+            seg(TILE_P, b);
+            seg(TILE_F, b);
+        }
     }
     return r;
 }
@@ -310,7 +306,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     volatile int* last_flag = abort_flag + 1;  // this F tile was its row block's last
     int* stage_tok = reinterpret_cast<int*>(head + 512);         // [kGStages][8]
-    float* red = reinterpret_cast<float*>(head + 1024);          // [2][4 warps][2]
     double* inv_freq = reinterpret_cast<double*>(head + 2048);   // [hd / 2 <= 128]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -551,7 +546,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int q = 0;
         uint32_t qph = 0;
         int local = 0;
-        int rbuf = 0;  // reduction scratch buffer (alternates per row)
         if (!p.plain)
             for (int j = et; j < half; j += kEpiThreads)
                 inv_freq[j] = pow(p.rope_base, -2.0 * (double)j / (double)p.hd);
@@ -589,16 +583,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int h = p.h, pieces = h / 8;  // 16-byte pieces of a row
                 const float wadd = p.norm_mode ? 1.f : 0.f;
                 const uint32_t rb = 2u * (uint32_t)h;
-                for (int st = 0; st < nst; ++st) {
-                    const bool got = mbar_wait_bounded(&full[s], ph, abort_flag);
+                const uint4* wne = reinterpret_cast<const uint4*>(p.w_ne);
+                const uint4* wnh = reinterpret_cast<const uint4*>(p.w_nh);
+                // warp ew takes the tile's stages ew, ew + 4, ... (with a 4-stage ring always
+                // the same ring slot), each of its rows with warp-wide reductions, so the
+                // four warps run independently
+                static_assert(kGStages == kEpiThreads / 32, "one ring slot per epilogue warp");
+                for (int st = ew; st < nst; st += kGStages) {
+                    const int sl = (s + st) % kGStages;
+                    const uint32_t sph = ph ^ (uint32_t)(((s + st) / kGStages) & 1);
+                    if (!mbar_wait_bounded(&full[sl], sph, abort_flag)) break;
                     const int r0 = st * p.rows_per_pstage;
                     const int nr = min(p.rows_per_pstage, rows - r0);
-                    for (int i = 0; i < nr && got; ++i) {
-                        const int tok = stage_tok[s * kMaxRowsPerPStage + i];
-                        const uint8_t* erow = stages + (size_t)s * kGStageBytes + (size_t)i * 2u * rb;
+                    for (int i = 0; i < nr; ++i) {
+                        const int tok = stage_tok[sl * kMaxRowsPerPStage + i];
+                        const uint8_t* erow = stages + (size_t)sl * kGStageBytes + (size_t)i * 2u * rb;
                         const uint8_t* xrow = erow + rb;
                         float se = 0.f, sx = 0.f;
-                        for (int j = et; j < pieces; j += kEpiThreads) {
+                        for (int j = lane; j < pieces; j += 32) {
                             if (tok >= 0) se += sumsq8(lds128(erow + 16 * j));
                             sx += sumsq8(lds128(xrow + 16 * j));
                         }
@@ -607,33 +609,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             se += __shfl_xor_sync(0xffffffffu, se, o);
                             sx += __shfl_xor_sync(0xffffffffu, sx, o);
                         }
-                        float* rr = red + rbuf * 8;
-                        if (lane == 0) {
-                            rr[ew * 2] = se;
-                            rr[ew * 2 + 1] = sx;
-                        }
-                        named_sync(1, kEpiThreads);
-                        se = (rr[0] + rr[2]) + (rr[4] + rr[6]);
-                        sx = (rr[1] + rr[3]) + (rr[5] + rr[7]);
-                        rbuf ^= 1;
                         const float inv_e = 1.0f / sqrtf(se / (float)h + p.eps);
                         const float inv_x = 1.0f / sqrtf(sx / (float)h + p.eps);
-                        uint16_t* crow = p.concat[lane_c] + ((int64_t)tl.m * BM + r0 + i) * 2 * h;
-                        for (int j = et; j < pieces; j += kEpiThreads) {
+                        uint4* crow = reinterpret_cast<uint4*>(
+                            p.concat[lane_c] + ((int64_t)tl.m * BM + r0 + i) * 2 * h);
+                        for (int j = lane; j < pieces; j += 32) {
                             const uint4 e = tok >= 0 ? lds128(erow + 16 * j) : make_uint4(0, 0, 0, 0);
-                            const uint4 we = __ldg(reinterpret_cast<const uint4*>(p.w_ne) + j);
-                            const uint4 wh = __ldg(reinterpret_cast<const uint4*>(p.w_nh) + j);
-                            reinterpret_cast<uint4*>(crow)[j] = norm8(e, inv_e, we, wadd);
-                            reinterpret_cast<uint4*>(crow + h)[j] = norm8(lds128(xrow + 16 * j), inv_x, wh, wadd);
+                            crow[j] = norm8(e, inv_e, __ldg(wne + j), wadd);
+                            crow[pieces + j] = norm8(lds128(xrow + 16 * j), inv_x, __ldg(wnh + j), wadd);
                         }
                     }
-                    named_sync(1, kEpiThreads);  // everyone is done with the stage
-                    if (et == 0) mbar_arrive(&empty[s]);
-                    if (++s == kGStages) {
-                        s = 0;
-                        ph ^= 1u;
-                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[sl]);  // done with the stage
                 }
+                s += nst;
+                ph ^= (uint32_t)((s / kGStages) & 1);
+                s %= kGStages;
                 // RoPE table of the rows (cos, sin of pos * base^(-2j / hd), in double)
                 float2* cs = p.rope[slot_r] + (int64_t)tl.m * BM * half;
                 for (int k = et; k < rows * half; k += kEpiThreads) {
@@ -951,22 +942,11 @@ cudaError_t prefill_launch(const PrefillArgs& a, cudaStream_t s) {
     p.mt_last = (int)((last_rows + BM - 1) / BM);
     p.nf = a.h / BN;
     p.nv = 2 * kvd / BN;
-    const int64_t full_p_f = (int64_t)p.mt_full * (1 + p.nf);
-    if (p.n_chunks == 1) {
-        p.b0 = (int64_t)p.mt_last * (1 + p.nf);
-        p.n_mid = 0;
-        p.s_mid = 1;
-        p.b_last = 0;
-        p.total = p.b0 + (int64_t)p.mt_last * p.nv;
-    } else {
-        p.b0 = full_p_f;
-        p.s_mid = full_p_f + (int64_t)p.mt_full * p.nv;
-        p.n_mid = p.n_chunks - 2;
-        p.b_last = (int64_t)p.mt_last * (1 + p.nf) + (int64_t)p.mt_full * p.nv;
-        p.total = p.b0 + p.n_mid * p.s_mid + p.b_last + (int64_t)p.mt_last * p.nv;
-    }
     p.lanes = (a.R > a.chunk_rows && a.ws_bytes >= prefill_ws_bytes_lanes(a.chunk_rows, a.h, a.hd, 2))
                   ? 2 : 1;
+    p.total = 0;
+    for (int c = 0; c < p.n_chunks; ++c)
+        p.total += (int64_t)(c == p.n_chunks - 1 ? p.mt_last : p.mt_full) * (1 + p.nf + p.nv);
     int rps = kGStageBytes / (4 * a.h);
     p.rows_per_pstage = rps > kMaxRowsPerPStage ? kMaxRowsPerPStage : rps;
     if (p.rows_per_pstage < 1 || a.hd / 2 > 128) return cudaErrorInvalidValue;
