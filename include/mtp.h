@@ -387,7 +387,9 @@ mtp_status mtp_prefill_kv(const uint16_t* embed, int64_t vocab, const int32_t* t
  * g = i / (nq / nkv), over the sequence's cache rows p = 0 .. seq_len - 1:
  *   s_p = scale * sum_d q[i, d] k_scale e4m3(k_cache[(slot(p) * nkv + g) * hd + d])
  *   out[i, d] = bf16(sum_p softmax(s)_p v_scale e4m3(v_cache[(slot(p) * nkv + g) * hd + d]))
- * (fp32 sums, fp32 softmax). A row whose block is missing (p / block_size >= n_table) or
+ * (fp32 sums and softmax; the tensor cores take q as f16 scaled per head by a power of two
+ * -- exact -- and the weights exp(s_p - max) in (0, 1] rounded to f16, the same rounded
+ * weights in the denominator). A row whose block is missing (p / block_size >= n_table) or
  * out of range is skipped and sets MTP_DEVFLAG_BAD_SLOT; no readable row -> zeros.
  *   q (device) bf16 [nq, hd]; k_cache, v_cache (device) u8 [num_blocks, block_size, nkv,
  *   hd], 16-byte aligned; block_table (device) i32 [n_table]; out (device) bf16 [nq, hd];
@@ -395,8 +397,9 @@ mtp_status mtp_prefill_kv(const uint16_t* embed, int64_t vocab, const int32_t* t
  *   seq_len) bytes, 16-byte aligned (per-piece partial sums; no initial contents).
  * Requires hd in {64, 128, 256}, nq % nkv == 0, nq / nkv <= 16, seq_len <= 2,097,152
  * (MTP_ERR_UNSUPPORTED otherwise), scale >= 0 (the usual
- * choice is 1 / sqrt(hd)), k_scale, v_scale > 0. Two kernels on `stream`: one CTA per kv
- * head and 256 cache rows (the K and V rows read once), then a merge per query head.
+ * choice is 1 / sqrt(hd)), k_scale, v_scale > 0. Two kernels on `stream`: CTAs of one kv
+ * head over a contiguous range of cache rows (about two per SM; every K and V row read
+ * once), then a merge per query head in a fixed order.
  * ------------------------------------------------------------------------------ */
 size_t mtp_paged_decode_attn_ws_bytes(int32_t nq, int32_t hd, int64_t seq_len);
 mtp_status mtp_paged_decode_attn(const uint16_t* q, int32_t nq, int32_t nkv, int32_t hd,

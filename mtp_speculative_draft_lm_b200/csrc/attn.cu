@@ -10,11 +10,16 @@
 //   s_p = scale * sum_d q[i, d] k_scale e4m3(K[slot(p), g, d]),  p < seq_len
 //   out[i, d] = sum_p softmax(s)_p v_scale e4m3(V[slot(p), g, d])
 //
-// Design (B200, HBM-bound: every cached K and V byte is read once): the positions are split
-// into pieces of kAPos; CTA (g, piece) loads its positions' K and V rows for kv head g with
-// 16-byte loads (many in flight per thread), keeps V in shared memory, computes the scores
-// of every query head of the group with fp32 sums, then per head the piece's maximum, its
-// sum of exp(s - max) and the exp-weighted sum of V rows; a second kernel merges the pieces
+// Design (B200, HBM-bound: every cached K and V byte is read once): CTA (g, piece) takes
+// kv head g over a contiguous range of positions (about two CTAs per SM in all), in
+// sub-pieces of 64 positions that a three-stage ring of 16-byte asynchronous copies
+// brings into shared memory (rows of a missing block zero-filled). Both contractions run
+// on the tensor cores (mma.sync m16n8k16, f16 operands, fp32 accumulators): the scores as
+// K[64 positions, hd] . Q^T, with E4M3 K decoded exactly to f16 and each query head in
+// f16 scaled by a power of two (exact), then an online softmax over the sub-pieces (fp32
+// running maximum and sum) and the weighted V sum as V^T . W^T, the weights
+// exp(s - max) in (0, 1] rounded to f16 (the same rounded weights in the sum of exps).
+// Each CTA writes its heads' (max, sum, weighted V sum); a second kernel merges the pieces
 // of each head in a fixed order (deterministic) and writes bf16. Rows whose block is
 // missing or out of range are skipped and set MTP_DEVFLAG_BAD_SLOT.
 #include <cuda_runtime.h>
@@ -26,11 +31,13 @@
 namespace mtp {
 namespace {
 
-constexpr int kAPos = 256;      // positions per CTA
+constexpr int kSP = 64;          // positions per sub-piece (four warps x 16)
 constexpr int kAThreads = 128;
+constexpr int kAStages = 3;
 constexpr int kAMaxGroup = 16;  // query heads per kv head
 constexpr int kAMaxHd = 256;
-constexpr int kAMaxPieces = 8192;  // cache rows up to 2M (the merge keeps a factor per piece)
+constexpr int kAMaxPieces = 1024;  // pieces per kv head (the merge keeps a factor per piece)
+constexpr int kWPitch = kSP + 8;   // f16 weights per head row in shared memory
 
 struct AttnParams {
     const uint16_t* q;  // [nq, hd] bf16
@@ -42,155 +49,279 @@ struct AttnParams {
     int block_size;
     int64_t num_blocks;
     int64_t seq_len;
-    float qk_scale;  // scale * k_scale
+    int64_t per_piece;  // positions per piece (a multiple of kSP)
+    float qk_scale;     // scale * k_scale
     float v_scale;
-    float* part;     // [pieces][nq][hd + 2]: (max, sum of exp, weighted V sum)
+    float* part;        // [pieces][nq][hd + 2]: (max, sum of exp, weighted V sum)
     int pieces;
     uint16_t* out;
     int32_t* dev_err;
 };
 
-// 16-byte asynchronous copy global -> shared (L2 only), and the wait for this thread's.
+// 16-byte asynchronous copy global -> shared (L2 only), group commit and wait.
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// 16 E4M3 codes -> 16 floats (exact).
-__device__ __forceinline__ void e4m3x16(uint4 c, float (&f)[16]) {
-    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float2 a = f16x2_to_f32x2(e4m3x2_to_f16x2((uint16_t)(w[i] & 0xFFFFu)));
-        const float2 b = f16x2_to_f32x2(e4m3x2_to_f16x2((uint16_t)(w[i] >> 16)));
-        f[4 * i] = a.x;
-        f[4 * i + 1] = a.y;
-        f[4 * i + 2] = b.x;
-        f[4 * i + 3] = b.y;
-    }
+__device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %2, %1;" : "=r"(r) : "f"(lo), "f"(hi));
+    return r;
 }
 
 template <int HD>
+__host__ __device__ constexpr int attn_row_pitch() { return HD + 16; }  // bank-conflict-free
+template <int HD>
+__host__ __device__ constexpr int attn_q_pitch() { return HD + 8; }     // f16 elements
+
+template <int HD>
+__host__ __device__ constexpr size_t attn_smem_bytes() {
+    return (size_t)kAStages * 2 * kSP * attn_row_pitch<HD>()  // K and V rings
+           + (size_t)kAMaxGroup * attn_q_pitch<HD>() * 2         // q in f16
+           + (size_t)kAMaxGroup * kWPitch * 2                    // weights in f16
+           + (size_t)kAStages * kSP * 4                          // row valid flags
+           + (size_t)2 * 4 * kAMaxGroup * 4                      // per-warp max and sum
+           + (size_t)kAMaxGroup * 4;                             // per-head score factor
+}
+
+template <int HD, int NT>
 __global__ void __launch_bounds__(kAThreads) attn_piece_kernel(const __grid_constant__ AttnParams p) {
     extern __shared__ __align__(16) uint8_t smem[];
-    constexpr int hd = HD;
-    const int G = p.group;
-    float* qs = reinterpret_cast<float*>(smem);              // [G][hd]
-    float* sc = qs + G * hd;                                  // [G][kAPos] scores, then weights
-    float* stat = sc + G * kAPos;                             // [G][2] max, sum
-    uint8_t* vs = reinterpret_cast<uint8_t*>(stat + 2 * kAMaxGroup);  // [kAPos][hd] V codes
+    constexpr int RP = attn_row_pitch<HD>();
+    constexpr int QP = attn_q_pitch<HD>();
+    constexpr int KC = HD / 16;          // 16-byte pieces of a row, and MMA K chunks
+    constexpr int MT = HD / 64;          // 16-dim tiles of the V sum per warp
+    uint8_t* kring = smem;                                          // [stages][kSP][RP]
+    uint8_t* vring = kring + kAStages * kSP * RP;                   // [stages][kSP][RP]
+    uint16_t* qh = reinterpret_cast<uint16_t*>(vring + kAStages * kSP * RP);  // [16][QP] f16
+    uint16_t* wsm = qh + kAMaxGroup * QP;                           // [16][kWPitch] f16
+    int* valid = reinterpret_cast<int*>(wsm + kAMaxGroup * kWPitch);  // [stages][kSP]
+    float* redm = reinterpret_cast<float*>(valid + kAStages * kSP);   // [4][16]
+    float* redl = redm + 4 * kAMaxGroup;                               // [4][16]
+    float* hfac = redl + 4 * kAMaxGroup;                               // [16]
+
     const int g = blockIdx.x, piece = blockIdx.y, tid = threadIdx.x;
-    const int warp = tid >> 5, lane = tid & 31;
-    const int64_t p0 = (int64_t)piece * kAPos;
-    const int npos = (int)min((int64_t)kAPos, p.seq_len - p0);
+    const int warp = tid >> 5, lane = tid & 31, gid = lane >> 2, tig = lane & 3;
+    const int G = p.group;
+    const int64_t pbeg = (int64_t)piece * p.per_piece;
+    const int64_t pend = min(p.seq_len, pbeg + p.per_piece);
+    const int nsub = (int)((pend - pbeg + kSP - 1) / kSP);
     pdl_launch_dependents();
 
-    for (int i = tid; i < G * hd; i += kAThreads)
-        qs[i] = bf16_to_f32(p.q[(int64_t)(g * G) * hd + i]) * p.qk_scale;
-    __syncthreads();
-
-    // scores: a thread per position; its K row in 16-byte pieces, V row into shared memory
-    constexpr int pieces16 = HD / 16;
-    for (int t = tid; t < kAPos; t += kAThreads) {
-        float s[kAMaxGroup];
-#pragma unroll
-        for (int i = 0; i < kAMaxGroup; ++i) s[i] = -INFINITY;
-        int64_t slot = -1;
-        if (t < npos) {
-            const int64_t pos = p0 + t;
-            const int64_t b = pos / p.block_size;
-            if (b < p.n_table) {
-                const int64_t blk = p.block_table[b];
-                if (blk >= 0 && blk < p.num_blocks) slot = blk * p.block_size + pos % p.block_size;
-            }
-            if (slot < 0) raise_flag(p.dev_err, DEVFLAG_BAD_SLOT);
-        }
-        if (slot >= 0) {
-            const uint8_t* krow = p.k_cache + (slot * p.nkv + g) * (int64_t)hd;
-            const uint8_t* vrow = p.v_cache + (slot * p.nkv + g) * (int64_t)hd;
-#pragma unroll
-            for (int i = 0; i < kAMaxGroup; ++i) s[i] = 0.f;
-            // every 16-byte piece of both rows in flight before any is used: V straight
-            // into shared memory (asynchronous copies), K into registers
-#pragma unroll
-            for (int c = 0; c < pieces16; ++c) cp_async16(vs + (size_t)t * hd + 16 * c, vrow + 16 * c);
-            uint4 kr[pieces16];
-#pragma unroll
-            for (int c = 0; c < pieces16; ++c) kr[c] = ldg_stream(krow + 16 * c);
-#pragma unroll
-            for (int c = 0; c < pieces16; ++c) {
-                float kf[16];
-                e4m3x16(kr[c], kf);
-#pragma unroll
-                for (int i = 0; i < kAMaxGroup; ++i) {
-                    if (i >= G) break;
-                    const float* qr = qs + i * hd + 16 * c;
-                    float a = s[i];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) a = fmaf(qr[j], kf[j], a);
-                    s[i] = a;
+    // copies of sub-piece i into ring stage i % 3 (positions past the piece: invalid)
+    auto issue = [&](int i) {
+        if (i < nsub) {
+            const int st = i % kAStages;
+            uint8_t* kd = kring + st * kSP * RP;
+            uint8_t* vd = vring + st * kSP * RP;
+            for (int c = tid; c < kSP * KC; c += kAThreads) {
+                const int r = c / KC, pc = c - r * KC;
+                const int64_t pos = pbeg + (int64_t)i * kSP + r;
+                int64_t slot = -1;
+                if (pos < pend) {
+                    const int64_t b = pos / p.block_size;
+                    if (b < p.n_table) {
+                        const int64_t blk = p.block_table[b];
+                        if (blk >= 0 && blk < p.num_blocks) slot = blk * p.block_size + pos % p.block_size;
+                    }
+                    if (slot < 0 && pc == 0) raise_flag(p.dev_err, DEVFLAG_BAD_SLOT);
+                }
+                if (pc == 0) valid[st * kSP + r] = slot >= 0;
+                uint8_t* kdst = kd + r * RP + 16 * pc;
+                uint8_t* vdst = vd + r * RP + 16 * pc;
+                if (slot >= 0) {
+                    const int64_t off = (slot * p.nkv + g) * (int64_t)HD + 16 * pc;
+                    cp_async16(kdst, p.k_cache + off);
+                    cp_async16(vdst, p.v_cache + off);
+                } else {  // zeros: the weight of the row is 0, and 0 * NaN would not be
+                    *reinterpret_cast<uint4*>(kdst) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4*>(vdst) = make_uint4(0, 0, 0, 0);
                 }
             }
         }
-#pragma unroll
-        for (int i = 0; i < kAMaxGroup; ++i)
-            if (i < G) sc[i * kAPos + t] = s[i];
-    }
-    cp_async_wait_all();
-    __syncthreads();
+        cp_async_commit();  // one group per sub-piece, empty past the end
+    };
+    issue(0);
+    issue(1);
 
-    // per head: the piece's maximum and sum of exp(s - max); scores become weights
-    for (int i = warp; i < G; i += kAThreads / 32) {
-        float m = -INFINITY;
-        for (int t = lane; t < kAPos; t += 32) m = fmaxf(m, sc[i * kAPos + t]);
+    // the group's query heads in f16, each scaled by 2^e so its largest |q| lies in
+    // [2^14, 2^15) (exact: a bf16 value has 8 significant bits); heads past G are zero
+    for (int h = warp; h < kAMaxGroup; h += kAThreads / 32) {
+        float mx = 0.f;
+        if (h < G)
+            for (int d = lane; d < HD; d += 32)
+                mx = fmaxf(mx, fabsf(bf16_to_f32(p.q[(int64_t)(g * G + h) * HD + d])));
 #pragma unroll
-        for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        float l = 0.f;
-        for (int t = lane; t < kAPos; t += 32) {
-            const float s = sc[i * kAPos + t];
-            const float w = (m == -INFINITY || s == -INFINITY) ? 0.f : expf(s - m);
-            sc[i * kAPos + t] = w;
-            l += w;
+        for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        int e = 0;
+        if (mx > 0.f) e = 14 - ilogbf(mx);
+        for (int d = lane; d < HD; d += 32) {
+            const float v = h < G ? ldexpf(bf16_to_f32(p.q[(int64_t)(g * G + h) * HD + d]), e) : 0.f;
+            qh[h * QP + d] = (uint16_t)(f32x2_to_f16x2(v, 0.f) & 0xFFFFu);
         }
-#pragma unroll
-        for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-        if (lane == 0) {
-            stat[2 * i] = m;
-            stat[2 * i + 1] = l;
-        }
+        if (lane == 0) hfac[h] = ldexpf(p.qk_scale, -e);
     }
-    __syncthreads();
 
-    // weighted V sums: a thread per (head, 8 dims), positions in order
-    const int dch = hd / 8;
-    for (int u = tid; u < G * dch; u += kAThreads) {
-        const int i = u / dch, d0 = 8 * (u - i * dch);
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int t = 0; t < npos; ++t) {
-            const float w = sc[i * kAPos + t];
-            if (w == 0.f) continue;
-            const uint2 c = *reinterpret_cast<const uint2*>(vs + (size_t)t * hd + d0);
-            const uint32_t cw[2] = {c.x, c.y};
+    float m_run[NT][2], l_run[NT][2], acc[MT][NT][4];
 #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-                const float2 a = f16x2_to_f32x2(e4m3x2_to_f16x2((uint16_t)(cw[h2] & 0xFFFFu)));
-                const float2 b = f16x2_to_f32x2(e4m3x2_to_f16x2((uint16_t)(cw[h2] >> 16)));
-                acc[4 * h2] = fmaf(w, a.x, acc[4 * h2]);
-                acc[4 * h2 + 1] = fmaf(w, a.y, acc[4 * h2 + 1]);
-                acc[4 * h2 + 2] = fmaf(w, b.x, acc[4 * h2 + 2]);
-                acc[4 * h2 + 3] = fmaf(w, b.y, acc[4 * h2 + 3]);
+    for (int j = 0; j < NT; ++j) {
+        m_run[j][0] = m_run[j][1] = -INFINITY;
+        l_run[j][0] = l_run[j][1] = 0.f;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[mt][j][k] = 0.f;
+    }
+
+    for (int i = 0; i < nsub; ++i) {
+        cp_async_wait<1>();  // this thread's copies of sub-piece i have landed
+        __syncthreads();     // everyone's; and sub-piece i - 1 is fully consumed
+        issue(i + 2);
+        const int st = i % kAStages;
+        const uint8_t* ks = kring + st * kSP * RP;
+        const uint8_t* vs = vring + st * kSP * RP;
+
+        // scores of positions 16 warp + [0, 16) for every head: K (A) . Q^T (B). The K
+        // dimension of each MMA is permuted -- k index 2t, 2t+1 is dims 4t, 4t+1 and
+        // 2t+8, 2t+9 dims 4t+2, 4t+3 of the 16-dim chunk -- in A and B alike
+        float sc[NT][4];
+#pragma unroll
+        for (int j = 0; j < NT; ++j)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) sc[j][k] = 0.f;
+        const uint8_t* kr0 = ks + (16 * warp + gid) * RP + 4 * tig;
+#pragma unroll
+        for (int c = 0; c < KC; ++c) {
+            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(kr0 + 16 * c);
+            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(kr0 + 8 * RP + 16 * c);
+            const uint32_t a0 = e4m3x2_to_f16x2((uint16_t)(w0 & 0xFFFFu));
+            const uint32_t a2 = e4m3x2_to_f16x2((uint16_t)(w0 >> 16));
+            const uint32_t a1 = e4m3x2_to_f16x2((uint16_t)(w1 & 0xFFFFu));
+            const uint32_t a3 = e4m3x2_to_f16x2((uint16_t)(w1 >> 16));
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                const uint2 b = *reinterpret_cast<const uint2*>(qh + (8 * j + gid) * QP + 16 * c + 4 * tig);
+                mma_f16_16816(sc[j], a0, a1, a2, a3, b.x, b.y);
             }
         }
-        float* dst = p.part + ((int64_t)piece * p.nq + g * G + i) * (hd + 2);
+        // scale per head; rows that are not readable score -inf
+        const bool v0 = valid[st * kSP + 16 * warp + gid] != 0;
+        const bool v1 = valid[st * kSP + 16 * warp + gid + 8] != 0;
+        float mloc[NT][2];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) dst[2 + d0 + j] = acc[j];
-        if (d0 == 0) {
-            dst[0] = stat[2 * i];
-            dst[1] = stat[2 * i + 1];
+        for (int j = 0; j < NT; ++j)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float f = hfac[8 * j + 2 * tig + e];
+                sc[j][e] = v0 ? sc[j][e] * f : -INFINITY;
+                sc[j][2 + e] = v1 ? sc[j][2 + e] * f : -INFINITY;
+                float m = fmaxf(sc[j][e], sc[j][2 + e]);
+#pragma unroll
+                for (int o = 4; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                mloc[j][e] = m;
+            }
+        if (gid == 0)
+#pragma unroll
+            for (int j = 0; j < NT; ++j)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) redm[warp * kAMaxGroup + 8 * j + 2 * tig + e] = mloc[j][e];
+        __syncthreads();
+        // the new running maximum; weights exp(s - max) as f16 into shared memory
+        // ([head][position]); their sum per warp
+        float alpha[NT][2];
+#pragma unroll
+        for (int j = 0; j < NT; ++j)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int h = 8 * j + 2 * tig + e;
+                const float msub = fmaxf(fmaxf(redm[h], redm[kAMaxGroup + h]),
+                                         fmaxf(redm[2 * kAMaxGroup + h], redm[3 * kAMaxGroup + h]));
+                const float mnew = fmaxf(m_run[j][e], msub);
+                alpha[j][e] = (m_run[j][e] == -INFINITY) ? 0.f : expf(m_run[j][e] - mnew);
+                m_run[j][e] = mnew;
+                float lsum = 0.f;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const float s = sc[j][2 * half + e];
+                    const float w = (s == -INFINITY) ? 0.f : expf(s - mnew);
+                    const uint16_t wh = (uint16_t)(f32x2_to_f16x2(w, 0.f) & 0xFFFFu);
+                    wsm[h * kWPitch + 16 * warp + gid + 8 * half] = wh;
+                    lsum += f16x2_to_f32x2((uint32_t)wh).x;
+                }
+#pragma unroll
+                for (int o = 4; o < 32; o <<= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+                if (gid == 0) redl[warp * kAMaxGroup + h] = lsum;
+            }
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < NT; ++j)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int h = 8 * j + 2 * tig + e;
+                const float ls = (redl[h] + redl[kAMaxGroup + h]) + (redl[2 * kAMaxGroup + h] + redl[3 * kAMaxGroup + h]);
+                l_run[j][e] = l_run[j][e] * alpha[j][e] + ls;
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    acc[mt][j][e] *= alpha[j][e];
+                    acc[mt][j][2 + e] *= alpha[j][e];
+                }
+            }
+        // the weighted V sum of dims warp * HD/4 + [0, HD/4): V^T (A) . W^T (B). The M
+        // dimension is permuted -- row g is dim 2g, row g + 8 dim 2g + 1 of the 16-dim
+        // tile -- so a thread's two dims are one 16-bit load per position
+#pragma unroll
+        for (int kk = 0; kk < kSP / 16; ++kk) {
+            const int pr = 16 * kk + 2 * tig;  // positions pr, pr + 1, pr + 8, pr + 9
+            uint32_t b[NT][2];
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                b[j][0] = *reinterpret_cast<const uint32_t*>(wsm + (8 * j + gid) * kWPitch + pr);
+                b[j][1] = *reinterpret_cast<const uint32_t*>(wsm + (8 * j + gid) * kWPitch + pr + 8);
+            }
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                const int d0 = warp * (HD / 4) + 16 * mt + 2 * gid;
+                const uint32_t x0 = *reinterpret_cast<const uint16_t*>(vs + pr * RP + d0);
+                const uint32_t x1 = *reinterpret_cast<const uint16_t*>(vs + (pr + 1) * RP + d0);
+                const uint32_t x8 = *reinterpret_cast<const uint16_t*>(vs + (pr + 8) * RP + d0);
+                const uint32_t x9 = *reinterpret_cast<const uint16_t*>(vs + (pr + 9) * RP + d0);
+                const uint32_t lo = x0 | (x1 << 16), hi = x8 | (x9 << 16);
+                // (dim d0: positions pr, pr + 1), (d0 + 1: pr, pr + 1), then pr + 8, pr + 9
+                const uint32_t a0 = e4m3x2_to_f16x2((uint16_t)__byte_perm(lo, 0, 0x0020));
+                const uint32_t a1 = e4m3x2_to_f16x2((uint16_t)__byte_perm(lo, 0, 0x0031));
+                const uint32_t a2 = e4m3x2_to_f16x2((uint16_t)__byte_perm(hi, 0, 0x0020));
+                const uint32_t a3 = e4m3x2_to_f16x2((uint16_t)__byte_perm(hi, 0, 0x0031));
+#pragma unroll
+                for (int j = 0; j < NT; ++j) mma_f16_16816(acc[mt][j], a0, a1, a2, a3, b[j][0], b[j][1]);
+            }
         }
     }
+
+    // this CTA's partials: (max, sum) per head, then its dims of the weighted V sums
+    const int64_t rs = (int64_t)HD + 2;
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int h = 8 * j + 2 * tig + e;
+            if (h >= G) continue;
+            float* dst = p.part + ((int64_t)piece * p.nq + g * G + h) * rs;
+            if (warp == 0 && gid == 0) {
+                dst[0] = m_run[j][e];
+                dst[1] = l_run[j][e];
+            }
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                const int d0 = warp * (HD / 4) + 16 * mt + 2 * gid;
+                dst[2 + d0] = acc[mt][j][e];
+                dst[2 + d0 + 1] = acc[mt][j][2 + e];
+            }
+        }
 }
 
 // One CTA per query head: out = sum_s e^(m_s - M) acc_s / sum_s e^(m_s - M) l_s (zero
@@ -250,9 +381,26 @@ __global__ void __launch_bounds__(kAMaxHd) attn_merge_kernel(const __grid_consta
 
 int attn_max_group() { return kAMaxGroup; }
 
+// Pieces per kv head: about two CTAs per SM over all kv heads, at least one sub-piece
+// each, at most kAMaxPieces; the positions per piece a multiple of kSP.
+static int64_t attn_pieces_cap(int64_t seq_len) {
+    const int64_t subs = (seq_len + kSP - 1) / kSP;
+    return subs < kAMaxPieces ? subs : kAMaxPieces;
+}
+
 size_t attn_ws_bytes(int nq, int hd, int64_t seq_len) {
-    const int64_t pieces = (seq_len + kAPos - 1) / kAPos;
+    const int64_t pieces = attn_pieces_cap(seq_len);
     return (size_t)(pieces < 1 ? 1 : pieces) * (size_t)nq * (size_t)(hd + 2) * sizeof(float);
+}
+
+template <int HD, int NT>
+cudaError_t launch_pieces(const AttnParams& p, cudaStream_t s) {
+    constexpr size_t smem = attn_smem_bytes<HD>();
+    auto kern = attn_piece_kernel<HD, NT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<dim3((unsigned)p.nkv, (unsigned)p.pieces), kAThreads, smem, s>>>(p);
+    return cudaGetLastError();
 }
 
 cudaError_t attn_launch(const uint16_t* q, int nq, int nkv, int hd, const uint8_t* k_cache,
@@ -276,17 +424,23 @@ cudaError_t attn_launch(const uint16_t* q, int nq, int nkv, int hd, const uint8_
     p.qk_scale = scale * k_scale;
     p.v_scale = v_scale;
     p.part = static_cast<float*>(ws);
-    p.pieces = (int)((seq_len + kAPos - 1) / kAPos);
     p.out = out;
     p.dev_err = dev_err;
-    const size_t smem = (size_t)p.group * hd * 4 + (size_t)p.group * kAPos * 4 +
-                        2 * kAMaxGroup * 4 + (size_t)kAPos * hd;
-    cudaError_t e = cudaSuccess;
-    auto kern = hd == 64 ? attn_piece_kernel<64> : hd == 128 ? attn_piece_kernel<128> : attn_piece_kernel<256>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    int dev = 0, sms = 148;
+    cudaError_t e;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    int64_t pieces = (2 * (int64_t)sms + nkv - 1) / nkv;
+    const int64_t cap = attn_pieces_cap(seq_len);
+    if (pieces > cap) pieces = cap;
+    const int64_t subs = (seq_len + kSP - 1) / kSP;
+    p.per_piece = (int64_t)kSP * ((subs + pieces - 1) / pieces);
+    p.pieces = (int)((seq_len + p.per_piece - 1) / p.per_piece);
+    const bool two = p.group > 8;
+    if (hd == 64) e = two ? launch_pieces<64, 2>(p, s) : launch_pieces<64, 1>(p, s);
+    else if (hd == 128) e = two ? launch_pieces<128, 2>(p, s) : launch_pieces<128, 1>(p, s);
+    else e = two ? launch_pieces<256, 2>(p, s) : launch_pieces<256, 1>(p, s);
     if (e != cudaSuccess) return e;
-    kern<<<dim3((unsigned)nkv, (unsigned)p.pieces), kAThreads, smem, s>>>(p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)nq);
     cfg.blockDim = dim3(kAMaxHd);

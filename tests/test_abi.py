@@ -318,7 +318,9 @@ def test_draft_step_rejects(lib):
 
 def test_paged_decode_attn_rejects(lib):
     ws = L.mtp_paged_decode_attn_ws_bytes(8, 128, 300)
-    assert ws == 2 * 8 * 130 * 4  # two 256-row pieces x heads x (hd + max + sum) floats
+    # up to one piece per 64 cache rows: 5 pieces x heads x (hd + max + sum) floats
+    assert ws == 5 * 8 * 130 * 4
+    assert L.mtp_paged_decode_attn_ws_bytes(8, 128, 2_000_000) == 1024 * 8 * 130 * 4  # at most 1,024
 
     def at(q=A, nq=8, nkv=2, hd=128, seq=300, ks=1.0, sc=0.1, w=0x40000, wb=ws, kc=B2):
         return st("mtp_paged_decode_attn", q, nq, nkv, hd, kc, B2, OUT, 20, 16, 30, seq, ks, 1.0,
