@@ -396,10 +396,10 @@ mtp_status mtp_prefill_kv(const uint16_t* embed, int64_t vocab, const int32_t* t
  *   dev_err i32 [1] or NULL; ws (device) >= mtp_paged_decode_attn_ws_bytes(nq, hd,
  *   seq_len) bytes, 16-byte aligned (per-piece partial sums; no initial contents).
  * Requires hd in {64, 128, 256}, nq % nkv == 0, nq / nkv <= 16, seq_len <= 2,097,152
- * (MTP_ERR_UNSUPPORTED otherwise), scale >= 0 (the usual
- * choice is 1 / sqrt(hd)), k_scale, v_scale > 0. Two kernels on `stream`: CTAs of one kv
- * head over a contiguous range of cache rows (about two per SM; every K and V row read
- * once), then a merge per query head in a fixed order.
+ * (MTP_ERR_UNSUPPORTED otherwise), scale >= 0 (the usual choice is 1 / sqrt(hd)),
+ * k_scale, v_scale > 0. Two kernels on `stream`: CTAs of one kv head over a contiguous
+ * range of cache rows (as many as the SMs hold at once; every K and V row read once),
+ * then a merge per query head in a fixed order.
  * ------------------------------------------------------------------------------ */
 size_t mtp_paged_decode_attn_ws_bytes(int32_t nq, int32_t hd, int64_t seq_len);
 mtp_status mtp_paged_decode_attn(const uint16_t* q, int32_t nq, int32_t nkv, int32_t hd,

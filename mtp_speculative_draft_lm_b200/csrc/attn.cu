@@ -11,7 +11,7 @@
 //   out[i, d] = sum_p softmax(s)_p v_scale e4m3(V[slot(p), g, d])
 //
 // Design (B200, HBM-bound: every cached K and V byte is read once): CTA (g, piece) takes
-// kv head g over a contiguous range of positions (about two CTAs per SM in all), in
+// kv head g over a contiguous range of positions (as many CTAs as the SMs hold at once), in
 // sub-pieces of 64 positions that a three-stage ring of 16-byte asynchronous copies
 // brings into shared memory (rows of a missing block zero-filled). Both contractions run
 // on the tensor cores (mma.sync m16n8k16, f16 operands, fp32 accumulators): the scores as
@@ -47,6 +47,7 @@ struct AttnParams {
     const int32_t* block_table;
     int64_t n_table;
     int block_size;
+    int bs_shift;       // log2(block_size) when a power of two, else -1
     int64_t num_blocks;
     int64_t seq_len;
     int64_t per_piece;  // positions per piece (a multiple of kSP)
@@ -114,20 +115,24 @@ __global__ void __launch_bounds__(kAThreads) attn_piece_kernel(const __grid_cons
     pdl_launch_dependents();
 
     // copies of sub-piece i into ring stage i % 3 (positions past the piece: invalid)
+    // 32-bit position arithmetic (seq_len <= 2^21); a power-of-two block size shifts
+    const int pend32 = (int)pend;
     auto issue = [&](int i) {
         if (i < nsub) {
             const int st = i % kAStages;
             uint8_t* kd = kring + st * kSP * RP;
             uint8_t* vd = vring + st * kSP * RP;
-            for (int c = tid; c < kSP * KC; c += kAThreads) {
-                const int r = c / KC, pc = c - r * KC;
-                const int64_t pos = pbeg + (int64_t)i * kSP + r;
+            const int pc = tid % KC;
+            const int pos0 = (int)pbeg + i * kSP;
+            for (int r = tid / KC; r < kSP; r += kAThreads / KC) {
+                const int pos = pos0 + r;
                 int64_t slot = -1;
-                if (pos < pend) {
-                    const int64_t b = pos / p.block_size;
+                if (pos < pend32) {
+                    const int b = p.bs_shift >= 0 ? pos >> p.bs_shift : pos / p.block_size;
                     if (b < p.n_table) {
-                        const int64_t blk = p.block_table[b];
-                        if (blk >= 0 && blk < p.num_blocks) slot = blk * p.block_size + pos % p.block_size;
+                        const int32_t blk = __ldg(p.block_table + b);
+                        if (blk >= 0 && blk < p.num_blocks)
+                            slot = (int64_t)blk * p.block_size + (pos - b * p.block_size);
                     }
                     if (slot < 0 && pc == 0) raise_flag(p.dev_err, DEVFLAG_BAD_SLOT);
                 }
@@ -381,8 +386,8 @@ __global__ void __launch_bounds__(kAMaxHd) attn_merge_kernel(const __grid_consta
 
 int attn_max_group() { return kAMaxGroup; }
 
-// Pieces per kv head: about two CTAs per SM over all kv heads, at least one sub-piece
-// each, at most kAMaxPieces; the positions per piece a multiple of kSP.
+// Pieces per kv head: as many CTAs over all kv heads as the SMs hold at once, at least one
+// sub-piece each, at most kAMaxPieces; the positions per piece a multiple of kSP.
 static int64_t attn_pieces_cap(int64_t seq_len) {
     const int64_t subs = (seq_len + kSP - 1) / kSP;
     return subs < kAMaxPieces ? subs : kAMaxPieces;
@@ -419,6 +424,7 @@ cudaError_t attn_launch(const uint16_t* q, int nq, int nkv, int hd, const uint8_
     p.block_table = block_table;
     p.n_table = n_table;
     p.block_size = block_size;
+    p.bs_shift = (block_size & (block_size - 1)) == 0 ? __builtin_ctz((unsigned)block_size) : -1;
     p.num_blocks = num_blocks;
     p.seq_len = seq_len;
     p.qk_scale = scale * k_scale;
@@ -430,7 +436,12 @@ cudaError_t attn_launch(const uint16_t* q, int nq, int nkv, int hd, const uint8_
     cudaError_t e;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    int64_t pieces = (2 * (int64_t)sms + nkv - 1) / nkv;
+    // as many CTAs as fit on the SMs at once (shared memory bound, at most four per SM)
+    const size_t smem = hd == 64 ? attn_smem_bytes<64>() : hd == 128 ? attn_smem_bytes<128>()
+                                                                      : attn_smem_bytes<256>();
+    int per_sm = (int)((size_t)227 * 1024 / smem);
+    per_sm = per_sm < 1 ? 1 : per_sm > 4 ? 4 : per_sm;
+    int64_t pieces = ((int64_t)per_sm * sms + nkv - 1) / nkv;
     const int64_t cap = attn_pieces_cap(seq_len);
     if (pieces > cap) pieces = cap;
     const int64_t subs = (seq_len + kSP - 1) / kSP;

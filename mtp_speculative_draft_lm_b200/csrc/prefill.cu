@@ -23,7 +23,7 @@
 //   P (chunk c, row block m): the prologue of 128 rows -- the producer warp bulk-copies
 //     each row's embedding row and hidden row into the shared-memory ring, the four
 //     epilogue warps take the two RMSNorms, write the bf16 concat rows and the rows'
-//     RoPE table (cos, sin in double).
+//     RoPE table (the angle reduced in double, cos and sin in fp32).
 //   F (c, m, n): a 128 x 256 tile of the fc GEMM, y = c . fc^T, bf16 out.
 //   V (c, m, n): a 128 x 256 tile of the k/v GEMM whose epilogue rotates k (RoPE),
 //     encodes E4M3 and writes each row's 32-byte pieces at its paged slot.
@@ -68,6 +68,9 @@ constexpr int kMaxLanes = 2;       // concat / fc-output lanes (RoPE rows: lanes
 // inverse frequencies
 constexpr int kHeadBytes = 4096;
 constexpr int kGemmSmem = kGStages * kGStageBytes + kHeadBytes + 1024 /* align */;
+// After those, when they fit: the norm weights (w_ne, w_nh, then the input norm's), read
+// by the epilogue warps for every row from shared memory instead of through L1.
+constexpr int kSmemMax = 227 * 1024;
 
 enum : int { TILE_P = 0, TILE_F = 1, TILE_V = 2 };
 constexpr int kArrivals = 3;  // counter kind: F tiles that finished (input norm only)
@@ -109,6 +112,7 @@ struct PrefillParams {
     int64_t total;       // tiles in all
     int lanes;           // 1 or 2
     int rows_per_pstage;
+    int w_in_smem;       // 1: the norm weights are staged in shared memory
     uint32_t* ctr;       // [0] tile counter; then done counters [4][kCtrSlots][mt_full]
     uint16_t* concat[kMaxLanes];
     uint16_t* y[kMaxLanes];
@@ -306,7 +310,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     volatile int* last_flag = abort_flag + 1;  // this F tile was its row block's last
     int* stage_tok = reinterpret_cast<int*>(head + 512);         // [kGStages][8]
-    double* inv_freq = reinterpret_cast<double*>(head + 2048);   // [hd / 2 <= 128]
+    double* inv_freq = reinterpret_cast<double*>(head + 2048);   // [hd / 2 <= 128], in turns
+    uint16_t* kn_s = reinterpret_cast<uint16_t*>(head + 3072);   // [hd <= 256] k norm weights
+    uint4* w_s = reinterpret_cast<uint4*>(head + kHeadBytes);    // [2 or 3][h / 8] norm weights
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int kvd = p.nkv * p.hd;
@@ -546,9 +552,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int q = 0;
         uint32_t qph = 0;
         int local = 0;
-        if (!p.plain)
+        if (!p.plain) {  // the rotation per position of each pair, in turns
             for (int j = et; j < half; j += kEpiThreads)
-                inv_freq[j] = pow(p.rope_base, -2.0 * (double)j / (double)p.hd);
+                inv_freq[j] = pow(p.rope_base, -2.0 * (double)j / (double)p.hd) /
+                              (2.0 * 3.14159265358979323846);
+            if (p.k_norm)
+                for (int j = et; j < p.hd; j += kEpiThreads) kn_s[j] = p.k_norm[j];
+            if (p.w_in_smem) {
+                const int pc = p.h / 8;
+                for (int j = et; j < pc; j += kEpiThreads) {
+                    w_s[j] = __ldg(reinterpret_cast<const uint4*>(p.w_ne) + j);
+                    w_s[pc + j] = __ldg(reinterpret_cast<const uint4*>(p.w_nh) + j);
+                    if (p.in_norm) w_s[2 * pc + j] = __ldg(reinterpret_cast<const uint4*>(p.in_norm) + j);
+                }
+            }
+        }
         named_sync(1, kEpiThreads);
         while (true) {
             if (!mbar_wait_bounded(&qfull[q], qph, abort_flag)) break;
@@ -583,8 +601,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int h = p.h, pieces = h / 8;  // 16-byte pieces of a row
                 const float wadd = p.norm_mode ? 1.f : 0.f;
                 const uint32_t rb = 2u * (uint32_t)h;
-                const uint4* wne = reinterpret_cast<const uint4*>(p.w_ne);
-                const uint4* wnh = reinterpret_cast<const uint4*>(p.w_nh);
+                // generic loads: shared memory when staged, else global
+                const uint4* wne = p.w_in_smem ? w_s : reinterpret_cast<const uint4*>(p.w_ne);
+                const uint4* wnh = p.w_in_smem ? w_s + pieces : reinterpret_cast<const uint4*>(p.w_nh);
                 // warp ew takes the tile's stages ew, ew + 4, ... (with a 4-stage ring always
                 // the same ring slot), each of its rows with warp-wide reductions, so the
                 // four warps run independently
@@ -600,6 +619,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         const uint8_t* erow = stages + (size_t)sl * kGStageBytes + (size_t)i * 2u * rb;
                         const uint8_t* xrow = erow + rb;
                         float se = 0.f, sx = 0.f;
+#pragma unroll 4
                         for (int j = lane; j < pieces; j += 32) {
                             if (tok >= 0) se += sumsq8(lds128(erow + 16 * j));
                             sx += sumsq8(lds128(xrow + 16 * j));
@@ -613,10 +633,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         const float inv_x = 1.0f / sqrtf(sx / (float)h + p.eps);
                         uint4* crow = reinterpret_cast<uint4*>(
                             p.concat[lane_c] + ((int64_t)tl.m * BM + r0 + i) * 2 * h);
+#pragma unroll 4
                         for (int j = lane; j < pieces; j += 32) {
                             const uint4 e = tok >= 0 ? lds128(erow + 16 * j) : make_uint4(0, 0, 0, 0);
-                            crow[j] = norm8(e, inv_e, __ldg(wne + j), wadd);
-                            crow[pieces + j] = norm8(lds128(xrow + 16 * j), inv_x, __ldg(wnh + j), wadd);
+                            crow[j] = norm8(e, inv_e, wne[j], wadd);
+                            crow[pieces + j] = norm8(lds128(xrow + 16 * j), inv_x, wnh[j], wadd);
                         }
                     }
                     __syncwarp();
@@ -625,14 +646,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 s += nst;
                 ph ^= (uint32_t)((s / kGStages) & 1);
                 s %= kGStages;
-                // RoPE table of the rows (cos, sin of pos * base^(-2j / hd), in double)
+                // RoPE table of the rows: the angle pos * base^(-2j / hd) in turns, reduced to
+                // [-1/2, 1/2] in double (exact to ~1e-12 turns), then cos and sin of the
+                // remainder in fp32 (sincospif: no further range reduction)
                 float2* cs = p.rope[slot_r] + (int64_t)tl.m * BM * half;
                 for (int k = et; k < rows * half; k += kEpiThreads) {
                     const int r = k / half, j = k - r * half;
-                    const double th = (double)p.rope_pos[crow0 + (int64_t)tl.m * BM + r] * inv_freq[j];
-                    double sn, cn;
-                    sincos(th, &sn, &cn);
-                    cs[k] = make_float2((float)cn, (float)sn);
+                    const double turns = (double)p.rope_pos[crow0 + (int64_t)tl.m * BM + r] * inv_freq[j];
+                    const float f = (float)(turns - rint(turns));
+                    float sn, cn;
+                    sincospif(f, &sn, &cn);
+                    cs[k] = make_float2(cn, sn);
                 }
                 fence_proxy_async_global();  // the concat rows are read by TMA
                 named_sync(1, kEpiThreads);
@@ -730,8 +754,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         if (kn) {
 #pragma unroll
                             for (int i = 0; i < 32; ++i) {
-                                lo[i] = round_bf16(lo[i] * kinv * (bf16_to_f32(p.k_norm[j0 + i]) + kadd));
-                                hi[i] = round_bf16(hi[i] * kinv * (bf16_to_f32(p.k_norm[half + j0 + i]) + kadd));
+                                lo[i] = round_bf16(lo[i] * kinv * (bf16_to_f32(kn_s[j0 + i]) + kadd));
+                                hi[i] = round_bf16(hi[i] * kinv * (bf16_to_f32(kn_s[half + j0 + i]) + kadd));
                             }
                         }
                         if (!is_v && row_ok) rope32(lo, hi, cs + j0);
@@ -769,16 +793,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const int h = p.h, pieces = h / 8;
                     const int nrow = (int)min((int64_t)BM, rows_c - (int64_t)tl.m * BM);
                     const float wadd = p.norm_mode ? 1.f : 0.f;
-                    const uint4* wn = reinterpret_cast<const uint4*>(p.in_norm);
+                    const uint4* wn = p.w_in_smem ? w_s + 2 * pieces : reinterpret_cast<const uint4*>(p.in_norm);
                     for (int r = ew; r < nrow; r += kEpiThreads / 32) {
                         uint4* yr = reinterpret_cast<uint4*>(Y + ((int64_t)tl.m * BM + r) * h);
                         float ss = 0.f;
+#pragma unroll 4
                         for (int j = lane; j < pieces; j += 32) ss += sumsq8(__ldcg(yr + j));
 #pragma unroll
                         for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
                         const float inv = 1.0f / sqrtf(ss / (float)h + p.eps);
+#pragma unroll 4
                         for (int j = lane; j < pieces; j += 32)
-                            __stcg(yr + j, norm8(__ldcg(yr + j), inv, __ldg(wn + j), wadd));
+                            __stcg(yr + j, norm8(__ldcg(yr + j), inv, wn[j], wadd));
                     }
                     fence_proxy_async_global();  // read by the k/v tiles' TMA
                     named_sync(1, kEpiThreads);
@@ -857,10 +883,17 @@ cudaError_t make_operand_map(CUtensorMap* m, const void* base, int64_t rows, int
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-cudaError_t launch(const PrefillParams& p, const Maps& maps, cudaStream_t s) {
+int weight_smem_bytes(const PrefillParams& p) {
+    return p.plain ? 0 : (p.in_norm ? 3 : 2) * 2 * p.h;
+}
+
+cudaError_t launch(PrefillParams p, const Maps& maps, cudaStream_t s) {
     if (p.total < 1) return cudaSuccess;
+    const int wb = weight_smem_bytes(p);
+    p.w_in_smem = wb > 0 && kGemmSmem + wb <= kSmemMax;
+    const int smem = kGemmSmem + (p.w_in_smem ? wb : 0);
     cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kGemmSmem);
+                                         smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
@@ -868,7 +901,7 @@ cudaError_t launch(const PrefillParams& p, const Maps& maps, cudaStream_t s) {
         return e;
     int64_t grid = sms;
     if (grid > p.total) grid = p.total;
-    prefill_kernel<<<(unsigned)grid, kGemmThreads, kGemmSmem, s>>>(p, maps);
+    prefill_kernel<<<(unsigned)grid, kGemmThreads, smem, s>>>(p, maps);
     return cudaGetLastError();
 }
 
