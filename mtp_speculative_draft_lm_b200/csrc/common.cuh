@@ -27,6 +27,13 @@ __device__ __forceinline__ uint16_t f32_to_bf16(float f) {
     return r;
 }
 
+// Two fp32 -> bf16x2 (`lo` in bits 0..15), round to nearest even: one packed convert.
+__device__ __forceinline__ uint32_t f32x2_to_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
 // fp32 -> f16, round to nearest even.
 __device__ __forceinline__ uint16_t f32_to_f16(float f) {
     uint16_t r;

@@ -73,6 +73,9 @@ constexpr int kGemmSmem = kGStages * kGStageBytes + kHeadBytes + 1024 /* align *
 constexpr int kSmemMax = 227 * 1024;
 
 enum : int { TILE_P = 0, TILE_F = 1, TILE_V = 2 };
+// A 128-row block's prologue is split into kPParts P tiles of kPRows rows, so that several
+// SMs share it (its row loop is latency-bound on the four epilogue warps).
+constexpr int kPParts = 4, kPRows = BM / kPParts;
 constexpr int kArrivals = 3;  // counter kind: F tiles that finished (input norm only)
 
 struct PrefillParams {
@@ -143,7 +146,7 @@ __device__ __forceinline__ int64_t cum_mt(const PrefillParams& p, int k) {
 // since F(b) then reuses the fc-output rows V(b - 1) reads.
 __device__ __forceinline__ int64_t block_start(const PrefillParams& p, int b) {
     const int64_t pc = p.lanes == 2 ? (b == 0 ? 0 : cum_mt(p, b + 1)) : cum_mt(p, b);
-    return pc + p.nf * cum_mt(p, b) + p.nv * cum_mt(p, b - 1);
+    return kPParts * pc + p.nf * cum_mt(p, b) + p.nv * cum_mt(p, b - 1);
 }
 
 // Tile t of the global order.
@@ -170,12 +173,17 @@ __device__ Tile decode(const PrefillParams& p, int64_t t) {
     auto seg = [&](int kind, int c) {
         if (found) return;
         const int mt = mt_of(p, c);
-        const int64_t cnt = (int64_t)mt * (kind == TILE_P ? 1 : kind == TILE_F ? p.nf : p.nv);
+        const int64_t cnt = (int64_t)mt * (kind == TILE_P ? kPParts : kind == TILE_F ? p.nf : p.nv);
         if (off < cnt) {
             r.kind = kind;
             r.c = c;
-            r.m = (int)(off % mt);
-            r.n = (int)(off / mt);
+            if (kind == TILE_P) {  // (row block, part), parts of a block adjacent
+                r.m = (int)(off / kPParts);
+                r.n = (int)(off % kPParts);
+            } else {  // GEMM tiles M-fastest
+                r.m = (int)(off % mt);
+                r.n = (int)(off / mt);
+            }
             found = true;
         } else {
             off -= cnt;
@@ -196,9 +204,16 @@ __device__ Tile decode(const PrefillParams& p, int64_t t) {
     return r;
 }
 
+// Prompt rows of P tile (c, m, part n): up to kPRows, none past the chunk's last row.
+__device__ __forceinline__ int p_tile_rows(const PrefillParams& p, const Tile& tl) {
+    const int64_t rows_c = min(p.chunk, p.R - (int64_t)tl.c * p.chunk);
+    const int64_t r = rows_c - (int64_t)tl.m * BM - (int64_t)tl.n * kPRows;
+    return (int)max((int64_t)0, min((int64_t)kPRows, r));
+}
+
 // Completion counters: kind k (P, F, V, F arrivals) of the chunks in slot c % 4, row
 // block m. They only grow within a call: after chunk c's tiles of row block m are all
-// done, the P counter reads c / 4 + 1, F (c / 4 + 1) nf, V (c / 4 + 1) nv. With the input
+// done, the P counter reads (c / 4 + 1) kPParts, F (c / 4 + 1) nf, V (c / 4 + 1) nv. With the input
 // norm the F tiles count themselves on the arrivals counter instead, and the last of a row
 // block normalizes the block's fc output rows in place, then adds nf to the F counter.
 __device__ __forceinline__ uint32_t* counter(const PrefillParams& p, int kind, int c, int m) {
@@ -246,7 +261,12 @@ __device__ __forceinline__ void store_codes32(uint8_t* dst, const float (&v)[32]
     d[1] = make_uint4(w[4], w[5], w[6], w[7]);
 }
 
-__device__ __forceinline__ float round_bf16(float f) { return bf16_to_f32(f32_to_bf16(f)); }
+// Both values rounded to bf16 (round to nearest even) by one packed convert.
+__device__ __forceinline__ void round_bf16x2(float& a, float& b) {
+    const uint32_t r = f32x2_to_bf16x2(a, b);
+    a = bf16_lo(r);
+    b = bf16_hi(r);
+}
 
 // NeoX rotation of one head's pair block: lo = k[j], hi = k[j + hd/2] for 32 j's.
 __device__ __forceinline__ void rope32(float (&lo)[32], float (&hi)[32], const float2* cs) {
@@ -254,35 +274,64 @@ __device__ __forceinline__ void rope32(float (&lo)[32], float (&hi)[32], const f
     for (int j = 0; j < 32; ++j) {
         const float2 t = cs[j];
         const float a = lo[j], b = hi[j];
-        lo[j] = round_bf16(fmaf(a, t.x, -b * t.y));
-        hi[j] = round_bf16(fmaf(b, t.x, a * t.y));
+        lo[j] = fmaf(a, t.x, -b * t.y);
+        hi[j] = fmaf(b, t.x, a * t.y);
+        round_bf16x2(lo[j], hi[j]);
     }
+}
+
+// Packed fp32 pairs (element 0 in the low word) and their round-to-nearest arithmetic:
+// one instruction for two IEEE operations.
+__device__ __forceinline__ uint64_t f32x2_of_bf16x2(uint32_t w) {
+    return ((uint64_t)(w & 0xFFFF0000u) << 32) | (uint64_t)(w << 16);
+}
+__device__ __forceinline__ uint64_t f32x2_splat(float f) {
+    const uint64_t b = __float_as_uint(f);
+    return (b << 32) | b;
+}
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint32_t bf16x2_of_f32x2(uint64_t v) {
+    return f32x2_to_bf16x2(__uint_as_float((uint32_t)v), __uint_as_float((uint32_t)(v >> 32)));
 }
 
 // 8 bf16 (one 16-byte piece) times a row factor and 8 norm weights (plus `add`: 0 for
-// weights w, 1 for 1 + w), rounded to bf16.
-__device__ __forceinline__ uint4 norm8(uint4 v, float inv, uint4 w, float add) {
+// weights w, 1 for 1 + w), rounded to bf16: bf16((x inv) (w + add)) per element.
+__device__ __forceinline__ uint4 norm8(uint4 v, uint64_t inv2, uint4 w, uint64_t add2) {
     const uint32_t a[4] = {v.x, v.y, v.z, v.w}, b[4] = {w.x, w.y, w.z, w.w};
     uint32_t o[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t lo = f32_to_bf16(bf16_lo(a[i]) * inv * (bf16_lo(b[i]) + add));
-        const uint32_t hi = f32_to_bf16(bf16_hi(a[i]) * inv * (bf16_hi(b[i]) + add));
-        o[i] = lo | (hi << 16);
-    }
+    for (int i = 0; i < 4; ++i)
+        o[i] = bf16x2_of_f32x2(mul_f32x2(mul_f32x2(f32x2_of_bf16x2(a[i]), inv2),
+                                         add_f32x2(f32x2_of_bf16x2(b[i]), add2)));
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-__device__ __forceinline__ float sumsq8(uint4 v) {
+// Sum of squares of 8 bf16, accumulated as even and odd elements in a packed pair.
+__device__ __forceinline__ uint64_t sumsq8(uint4 v, uint64_t acc) {
     const uint32_t a[4] = {v.x, v.y, v.z, v.w};
-    float s = 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const float lo = bf16_lo(a[i]), hi = bf16_hi(a[i]);
-        s += lo * lo;
-        s += hi * hi;
+        const uint64_t x = f32x2_of_bf16x2(a[i]);
+        acc = fma_f32x2(x, x, acc);
     }
-    return s;
+    return acc;
+}
+__device__ __forceinline__ float hsum_f32x2(uint64_t v) {
+    return __uint_as_float((uint32_t)v) + __uint_as_float((uint32_t)(v >> 32));
 }
 
 struct Maps {
@@ -346,8 +395,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // stages of a tile in the ring: a GEMM tile's K blocks, or a P tile's row groups
     auto tile_stages = [&](const Tile& tl) -> int {
         if (tl.kind == TILE_P) {
-            const int64_t rows_c = min(p.chunk, p.R - (int64_t)tl.c * p.chunk);
-            const int rows = (int)min((int64_t)BM, rows_c - (int64_t)tl.m * BM);
+            const int rows = p_tile_rows(p, tl);
             return (rows + p.rows_per_pstage - 1) / p.rows_per_pstage;
         }
         if (p.plain) return p.K / BK;
@@ -386,9 +434,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const Tile tl = decode(p, t);
             const int nst = tile_stages(tl);
             if (tl.kind == TILE_P) {
-                const int64_t row0 = (int64_t)tl.c * p.chunk + (int64_t)tl.m * BM;  // prompt row
-                const int64_t rows_c = min(p.chunk, p.R - (int64_t)tl.c * p.chunk);
-                const int rows = (int)min((int64_t)BM, rows_c - (int64_t)tl.m * BM);
+                const int64_t row0 = (int64_t)tl.c * p.chunk + (int64_t)tl.m * BM +
+                                     (int64_t)tl.n * kPRows;  // prompt row
+                const int rows = p_tile_rows(p, tl);
                 const uint32_t rb = 2u * (uint32_t)p.h;  // bytes of one bf16 row
                 for (int st = 0; st < nst && !stop; ++st) {
                     if (!mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag)) {
@@ -438,7 +486,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     ma = &maps.a_concat[tl.c % p.lanes];
                     mb = &maps.b_fc;
                     if (lane == 0 && !wait_counter(counter(p, TILE_P, tl.c, tl.m),
-                                                   (uint32_t)(tl.c / kCtrSlots + 1), abort_flag))
+                                                   (uint32_t)((tl.c / kCtrSlots + 1) * kPParts), abort_flag))
                         stop = true;
                 } else {
                     ma = &maps.a_y[tl.c % p.lanes];
@@ -583,8 +631,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int64_t crow0 = (int64_t)tl.c * p.chunk;  // prompt row of the chunk's row 0
             const int64_t rows_c = p.plain ? p.M : min(p.chunk, p.R - crow0);
             if (tl.kind == TILE_P) {
-                // ---- prologue of rows m*128 .. : the lanes' buffers are free once the
-                // chunks that used them before are done with them
+                // ---- prologue of rows m*128 + n*32 .. : the lanes' buffers are free once
+                // the chunks that used them before are done with them
                 const int lane_c = tl.c % p.lanes, slot_r = tl.c % (p.lanes + 1);
                 bool ok = true;
                 if (et == 0) {
@@ -597,9 +645,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                           (uint32_t)((cr / kCtrSlots + 1) * p.nv), abort_flag);
                 }
                 named_sync(1, kEpiThreads);
-                const int rows = (int)min((int64_t)BM, rows_c - (int64_t)tl.m * BM);
+                const int rows = p_tile_rows(p, tl);
+                const int prow0 = tl.m * BM + tl.n * kPRows;  // the tile's first row of the chunk
                 const int h = p.h, pieces = h / 8;  // 16-byte pieces of a row
-                const float wadd = p.norm_mode ? 1.f : 0.f;
+                const uint64_t wadd = f32x2_splat(p.norm_mode ? 1.f : 0.f);
                 const uint32_t rb = 2u * (uint32_t)h;
                 // generic loads: shared memory when staged, else global
                 const uint4* wne = p.w_in_smem ? w_s : reinterpret_cast<const uint4*>(p.w_ne);
@@ -618,21 +667,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         const int tok = stage_tok[sl * kMaxRowsPerPStage + i];
                         const uint8_t* erow = stages + (size_t)sl * kGStageBytes + (size_t)i * 2u * rb;
                         const uint8_t* xrow = erow + rb;
-                        float se = 0.f, sx = 0.f;
+                        uint64_t se2 = 0, sx2 = 0;
 #pragma unroll 4
                         for (int j = lane; j < pieces; j += 32) {
-                            if (tok >= 0) se += sumsq8(lds128(erow + 16 * j));
-                            sx += sumsq8(lds128(xrow + 16 * j));
+                            if (tok >= 0) se2 = sumsq8(lds128(erow + 16 * j), se2);
+                            sx2 = sumsq8(lds128(xrow + 16 * j), sx2);
                         }
+                        float se = hsum_f32x2(se2), sx = hsum_f32x2(sx2);
 #pragma unroll
                         for (int o = 16; o; o >>= 1) {
                             se += __shfl_xor_sync(0xffffffffu, se, o);
                             sx += __shfl_xor_sync(0xffffffffu, sx, o);
                         }
-                        const float inv_e = 1.0f / sqrtf(se / (float)h + p.eps);
-                        const float inv_x = 1.0f / sqrtf(sx / (float)h + p.eps);
+                        const uint64_t inv_e = f32x2_splat(1.0f / sqrtf(se / (float)h + p.eps));
+                        const uint64_t inv_x = f32x2_splat(1.0f / sqrtf(sx / (float)h + p.eps));
                         uint4* crow = reinterpret_cast<uint4*>(
-                            p.concat[lane_c] + ((int64_t)tl.m * BM + r0 + i) * 2 * h);
+                            p.concat[lane_c] + ((int64_t)prow0 + r0 + i) * 2 * h);
 #pragma unroll 4
                         for (int j = lane; j < pieces; j += 32) {
                             const uint4 e = tok >= 0 ? lds128(erow + 16 * j) : make_uint4(0, 0, 0, 0);
@@ -649,13 +699,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 // RoPE table of the rows: the angle pos * base^(-2j / hd) in turns, reduced to
                 // [-1/2, 1/2] in double (exact to ~1e-12 turns), then cos and sin of the
                 // remainder in fp32 (sincospif: no further range reduction)
-                float2* cs = p.rope[slot_r] + (int64_t)tl.m * BM * half;
+                float2* cs = p.rope[slot_r] + (int64_t)prow0 * half;
                 for (int k = et; k < rows * half; k += kEpiThreads) {
                     const int r = k / half, j = k - r * half;
-                    const double turns = (double)p.rope_pos[crow0 + (int64_t)tl.m * BM + r] * inv_freq[j];
+                    const double turns = (double)p.rope_pos[crow0 + prow0 + r] * inv_freq[j];
                     const float f = (float)(turns - rint(turns));
                     float sn, cn;
-                    sincospif(f, &sn, &cn);
+                    sincospif(2.0f * f, &sn, &cn);  // sin and cos of pi x: x in half turns
                     cs[k] = make_float2(cn, sn);
                 }
                 fence_proxy_async_global();  // the concat rows are read by TMA
@@ -680,7 +730,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                       (uint32_t)((ca / kCtrSlots + 1) * p.nv), abort_flag);
                 } else if (tl.kind == TILE_V) {
                     ok = wait_counter(counter(p, TILE_P, tl.c, tl.m),
-                                      (uint32_t)(tl.c / kCtrSlots + 1), abort_flag);
+                                      (uint32_t)((tl.c / kCtrSlots + 1) * kPParts), abort_flag);
                 }
             }
             named_sync(1, kEpiThreads);
@@ -700,8 +750,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         uint32_t pk[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i)
-                            pk[i] = (uint32_t)f32_to_bf16(__uint_as_float(v[2 * i])) |
-                                    ((uint32_t)f32_to_bf16(__uint_as_float(v[2 * i + 1])) << 16);
+                            pk[i] = f32x2_to_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
                         uint4* dst = reinterpret_cast<uint4*>(C + (int64_t)row * ldc + tl.n * BN + cc * 32);
 #pragma unroll
                         for (int i = 0; i < 4; ++i)
@@ -733,9 +782,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             tmem_ld32(tb + h0 + j0, a);
                             tmem_ld_wait();
 #pragma unroll
-                            for (int i = 0; i < 32; ++i) {
-                                const float v = round_bf16(__uint_as_float(a[i]));
-                                ss = fmaf(v, v, ss);
+                            for (int i = 0; i < 32; i += 2) {
+                                float v0 = __uint_as_float(a[i]), v1 = __uint_as_float(a[i + 1]);
+                                round_bf16x2(v0, v1);
+                                ss = fmaf(v0, v0, ss);
+                                ss = fmaf(v1, v1, ss);
                             }
                         }
                         kinv = 1.0f / sqrtf(ss / (float)p.hd + p.eps);
@@ -748,14 +799,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         float lo[32], hi[32];
 #pragma unroll
                         for (int i = 0; i < 32; ++i) {
-                            lo[i] = round_bf16(__uint_as_float(a[i]));
-                            hi[i] = round_bf16(__uint_as_float(b[i]));
+                            lo[i] = __uint_as_float(a[i]);
+                            hi[i] = __uint_as_float(b[i]);
+                            round_bf16x2(lo[i], hi[i]);
                         }
                         if (kn) {
 #pragma unroll
                             for (int i = 0; i < 32; ++i) {
-                                lo[i] = round_bf16(lo[i] * kinv * (bf16_to_f32(kn_s[j0 + i]) + kadd));
-                                hi[i] = round_bf16(hi[i] * kinv * (bf16_to_f32(kn_s[half + j0 + i]) + kadd));
+                                lo[i] = lo[i] * kinv * (bf16_to_f32(kn_s[j0 + i]) + kadd);
+                                hi[i] = hi[i] * kinv * (bf16_to_f32(kn_s[half + j0 + i]) + kadd);
+                                round_bf16x2(lo[i], hi[i]);
                             }
                         }
                         if (!is_v && row_ok) rope32(lo, hi, cs + j0);
@@ -792,16 +845,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     uint16_t* Y = p.y[tl.c % p.lanes];
                     const int h = p.h, pieces = h / 8;
                     const int nrow = (int)min((int64_t)BM, rows_c - (int64_t)tl.m * BM);
-                    const float wadd = p.norm_mode ? 1.f : 0.f;
+                    const uint64_t wadd = f32x2_splat(p.norm_mode ? 1.f : 0.f);
                     const uint4* wn = p.w_in_smem ? w_s + 2 * pieces : reinterpret_cast<const uint4*>(p.in_norm);
                     for (int r = ew; r < nrow; r += kEpiThreads / 32) {
                         uint4* yr = reinterpret_cast<uint4*>(Y + ((int64_t)tl.m * BM + r) * h);
-                        float ss = 0.f;
+                        uint64_t ss2 = 0;
 #pragma unroll 4
-                        for (int j = lane; j < pieces; j += 32) ss += sumsq8(__ldcg(yr + j));
+                        for (int j = lane; j < pieces; j += 32) ss2 = sumsq8(__ldcg(yr + j), ss2);
+                        float ss = hsum_f32x2(ss2);
 #pragma unroll
                         for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-                        const float inv = 1.0f / sqrtf(ss / (float)h + p.eps);
+                        const uint64_t inv = f32x2_splat(1.0f / sqrtf(ss / (float)h + p.eps));
 #pragma unroll 4
                         for (int j = lane; j < pieces; j += 32)
                             __stcg(yr + j, norm8(__ldcg(yr + j), inv, wn[j], wadd));
@@ -979,7 +1033,7 @@ cudaError_t prefill_launch(const PrefillArgs& a, cudaStream_t s) {
                   ? 2 : 1;
     p.total = 0;
     for (int c = 0; c < p.n_chunks; ++c)
-        p.total += (int64_t)(c == p.n_chunks - 1 ? p.mt_last : p.mt_full) * (1 + p.nf + p.nv);
+        p.total += (int64_t)(c == p.n_chunks - 1 ? p.mt_last : p.mt_full) * (kPParts + p.nf + p.nv);
     int rps = kGStageBytes / (4 * a.h);
     p.rows_per_pstage = rps > kMaxRowsPerPStage ? kMaxRowsPerPStage : rps;
     if (p.rows_per_pstage < 1 || a.hd / 2 > 128) return cudaErrorInvalidValue;
