@@ -187,15 +187,16 @@ mtp_status mtp_combine(const uint16_t* embed, int64_t vocab, const int32_t* toke
  *                 counter zero again. It also holds x as the many-input sweeps read
  *                 it, rewritten by each call: for FP8 tables with M >= 7 two E4M3
  *                 planes of 16 or 32 rows (2 * 16 * k or 2 * 32 * k bytes), for NVFP4
- *                 with M >= 3 an f16 copy (M * k * 2 bytes).
+ *                 with M >= 9 an f16 copy (M * k * 2 bytes).
  * Requires 1 <= M <= 32, 1 <= n_eff <= n; table rows a multiple of 128 bytes (k % 64
  * for BF16, % 128 for FP8, % 256 for NVFP4; the sweep streams 128-byte segments); for
  * M <= 8 (FP8: M <= 6) the staged inputs (M * k * 2 bytes) must leave shared memory for
  * the stream (MTP_ERR_UNSUPPORTED otherwise; more inputs stream x per K chunk instead).
  * Results are bit-identical for every M within BF16 1-8, 9-16, 17-32; FP8 1-6, 7-16,
  * 17-32; NVFP4 1-2, 3-8, 9-16, 17-32, whose sweeps sum the same products in different
- * fixed orders. BF16 tables from 9 inputs, FP8 from 7 and NVFP4 from 3 run on the
- * tcgen05 tensor cores; there x enters FP8 products as two E4M3 terms whose sum is x
+ * fixed orders. BF16 tables from 9 inputs, FP8 from 7 and NVFP4 from 17 run on the
+ * tcgen05 tensor cores (NVFP4 9-16 on legacy MMAs with x streamed per K chunk, decoding
+ * to f16 in registers); there x enters FP8 products as two E4M3 terms whose sum is x
  * exactly except for elements below 2^-9 of the input's largest |x|, which keep an
  * absolute error of at most 2^-17 of that largest |x|. With a grammar mask and up to 8
  * inputs only the table rows that some input's mask allows are read.
@@ -436,7 +437,7 @@ mtp_status mtp_debug_kv_write(const uint16_t* k_rot, const uint16_t* v, int64_t 
  * (524,544: a 256-byte header + 16-byte partials of up to 1,024 CTAs x 32 input rows)
  * held on every GPU that loads the library until the process exits. It has no room
  * for x in the form the many-input sweeps read it (FP8 tables from M = 7, NVFP4 from
- * M = 3), so those calls return MTP_ERR_WORKSPACE here; BF16 tables run at every M up
+ * M = 9), so those calls return MTP_ERR_WORKSPACE here; BF16 tables run at every M up
  * to 32.
  *  - The first call made with a device current looks up that array's device address.
  *    Under the CUDA runtime's lazy module loading (the default since CUDA 12.2) that

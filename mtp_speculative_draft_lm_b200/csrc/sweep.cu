@@ -1799,7 +1799,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
 }
 
 // ---------------------------------------------------------------- NVFP4 tcgen05 sweep
-// NVFP4 tables with 3-32 inputs run the contraction on the tcgen05 tensor cores with A in
+// NVFP4 tables with 17-32 inputs run the contraction on the tcgen05 tensor cores with A in
 // tensor memory. Eight decode warps (two per lane quarter, each half of every segment)
 // turn each table row's E2M1 codes times their E4M3 block
 // scale into f16 -- exact: a code has at most 2 significant bits and a scale 4, and every
@@ -2601,10 +2601,15 @@ cudaError_t launch_tc4(const SweepParams& p, cudaStream_t s, SweepLaunch* info) 
     return cudaGetLastError();
 }
 
-// Argmax sweeps that stream x per K chunk -- the tcgen05 sweeps -- take FP8 tables from 7
-// inputs on (measured faster than 16-row tiles from there), NVFP4 from 3 (its tensor-memory
-// A path), BF16 from 9.
-inline bool streams_x(int M, int fmt) { return fmt == 1 ? M >= 7 : fmt == 2 ? M >= 3 : M > 8; }
+// Argmax sweeps that stream x per K chunk -- the tcgen05 sweeps, and for NVFP4 the wide
+// mma.sync sweep -- take FP8 tables from 7 inputs on (measured faster than 16-row tiles
+// from there), BF16 and NVFP4 from 9. NVFP4 runs 9-16 inputs on the wide sweep and 17-32
+// on the tcgen05 sweep with A in tensor memory: measured on a B200, M = 4 / 16 / 32 took
+// 86 / 134 / 258 us on the narrow / wide / wide sweeps and 152 / 186 / 221 us on the
+// tensor-memory sweep, whose decode -> tensor memory -> MMA round trip per 128-column
+// slot (three slots) bounds it.
+inline bool streams_x(int M, int fmt) { return fmt == 1 ? M >= 7 : M > 8; }
+inline bool nvfp4_tc4(int M) { return M > 16; }
 
 }  // namespace
 
@@ -2619,7 +2624,7 @@ size_t sweep_smem_bytes(int M, int64_t k, int fmt, int* kpad_out, int mode, bool
         return g.stages >= 2 ? g.smem : (size_t)kSmemLimit + 1;
     }
     if (mode == 0 && streams_x(M, fmt)) {  // the tcgen05 / wide sweeps stage x per K chunk
-        const WideGeometry w = fmt == 2 ? tc4_geometry(k, M > 16 ? 32 : 16, M > 8 ? 2 : 1)
+        const WideGeometry w = fmt == 2 ? (nvfp4_tc4(M) ? tc4_geometry(k, 32, 2) : wide_geometry(k, 2, 16))
                                         : tc_geometry(k, fmt, M > 16 ? 32 : 16);
         if (kpad_out) *kpad_out = (int)k;
         return w.stages >= 2 ? w.smem : (size_t)kSmemLimit + 1;
@@ -2704,9 +2709,7 @@ cudaError_t sweep_launch(const SweepParams& p, int fmt, int mode, cudaStream_t s
         const bool four = p.M > 16;
         if (fmt == 0) return four ? launch_tc<0, 32>(p, s, info) : launch_tc<0, 16>(p, s, info);
         if (fmt == 1) return four ? launch_tc<1, 32>(p, s, info) : launch_tc<1, 16>(p, s, info);
-        if (fmt == 2)
-            return four ? launch_tc4<32, 2>(p, s, info)
-                        : (p.M > 8 ? launch_tc4<16, 2>(p, s, info) : launch_tc4<16, 1>(p, s, info));
+        if (fmt == 2) return nvfp4_tc4(p.M) ? launch_tc4<32, 2>(p, s, info) : launch_wide<2, 2>(p, s, info);
     }
 #define MTP_SWEEP_CASE(F, NTV, MD) \
     if (fmt == F && (NTV == 2) == two && mode == MD) return launch_one<F, NTV, MD, 0, 0>(p, s, info);

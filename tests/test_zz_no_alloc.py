@@ -23,8 +23,9 @@ def bits(t):
 
 @pytest.mark.parametrize("fmt", [0, 1, 2])
 def test_noalloc_matches_workspace_entry_point(fmt):
-    # two inputs: NVFP4 from three reads an f16 copy of x the static array has no room for
-    n, k, M = 5000, 1024, 2
+    # four inputs: FP8 from seven and NVFP4 from nine read x in a form (E4M3 planes, an f16
+    # copy) the static array has no room for
+    n, k, M = 5000, 1024, 4
     d = synth.head_table(21 + fmt, n, k, M)
     w = d["W"].cuda()
     table = api.bf16_table(w) if fmt == 0 else (api.quantize_fp8(w) if fmt == 1 else
