@@ -147,7 +147,7 @@ def test_lm_head_lp_rejects(lib):
                                  0, 0, OUT, None, None, None, None)
     assert noalloc(fp8, 7) == L.MTP_ERR_WORKSPACE
     assert noalloc(weight(fmt=2, k=256, bs=OUT, gs=OUT), 12) == L.MTP_ERR_WORKSPACE
-    assert noalloc(weight(fmt=2, k=256, bs=OUT, gs=OUT), 3) == L.MTP_ERR_WORKSPACE
+    assert noalloc(weight(fmt=2, k=256, bs=OUT, gs=OUT), 9) == L.MTP_ERR_WORKSPACE
     # the table descriptor is checked before its size is looked at: a bad format, a bad k
     # or a missing scale is an argument error, not a workspace one
     assert noalloc(weight(fmt=7, k=128), 12) == L.MTP_ERR_INVALID_ARG
