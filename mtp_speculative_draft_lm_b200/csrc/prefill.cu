@@ -17,23 +17,26 @@
 // Design (B200): rows are processed in chunks (the reference's PREFILL_CHUNK), whose
 // buffers (concat rows, fc output, RoPE table) live in the caller's workspace. The whole
 // call is ONE persistent kernel on the caller's stream: every CTA takes work items
-// ("tiles") from one counter, in a fixed global order, so that the tiles of the next
-// chunk fill the SMs the current chunk leaves idle (a 2,048-row chunk's fc GEMM is 320
-// output tiles, 2.16 waves on 148 SMs). Three kinds of tile:
-//   P (chunk c, row block m): the prologue of 128 rows -- the producer warp bulk-copies
-//     each row's embedding row and hidden row into the shared-memory ring, the four
-//     epilogue warps take the two RMSNorms, write the bf16 concat rows and the rows'
-//     RoPE table (the angle reduced in double, cos and sin in fp32).
+// ("tiles") from two counters, each in a fixed global order, so that the tiles of the
+// next chunk fill the SMs the current chunk leaves idle (a 2,048-row chunk's fc GEMM is
+// 320 output tiles, 2.16 waves on 148 SMs). Three kinds of tile:
+//   P (chunk c, row block m, part n): the prologue of 8 rows, taken from its own counter
+//     by each CTA's two prologue warps whenever they are free: they read each row's
+//     embedding row and hidden row into registers, take the two RMSNorms, write the
+//     bf16 concat rows and the rows' RoPE table (the angle reduced in double, cos and
+//     sin in fp32), alongside the GEMM tiles, whose shared-memory ring they never use.
 //   F (c, m, n): a 128 x 256 tile of the fc GEMM, y = c . fc^T, bf16 out.
 //   V (c, m, n): a 128 x 256 tile of the k/v GEMM whose epilogue rotates k (RoPE),
 //     encodes E4M3 and writes each row's 32-byte pieces at its paged slot.
-// Order: for b = 0..chunks: P(b + 1), F(b), then V(b - 1) (block 0 starts with P(0); with a
-// single lane the order is V(b - 1), P(b), F(b)). A tile only ever waits for tiles earlier in that order (completion counters per chunk slot and row block, in the
-// workspace header, release/acquire at GPU scope): F(c, m, .) for P(c, m); V(c, m, .)
-// for all of F(c, m, .); and a tile that overwrites a buffer another chunk used (two
-// lanes of concat and fc-output rows, three of RoPE rows) for that chunk's readers.
-// Tiles are claimed only by running CTAs, so the oldest unfinished tile can always
-// finish. GEMM tiles run on the 5th-generation tensor cores: a 4-stage TMA ring
+// GEMM order: for b = 0..chunks: F(b), then V(b - 1) (with a single lane V(b - 1) first).
+// Completion counters per chunk slot and row block (in the workspace header,
+// release/acquire at GPU scope) order the tiles: F(c, m, .) waits for P(c, m, .);
+// V(c, m, .) for all of F(c, m, .); and a tile that overwrites a buffer another chunk
+// used (two lanes of concat and fc-output rows, three of RoPE rows) for that chunk's
+// readers. A GEMM tile only waits for GEMM tiles earlier in its order and for P tiles; a
+// P tile only for GEMM tiles of chunks two and three back, whose own P tiles were taken
+// earlier from the P counter. Tiles are claimed only by running CTAs, so every wait
+// ends. GEMM tiles run on the 5th-generation tensor cores: a 4-stage TMA ring
 // (128-byte swizzle, K-major A and B), tcgen05.mma from one thread into a double-
 // buffered 512-column TMEM accumulator, four epilogue warps reading it back with
 // tcgen05.ld while the next tile accumulates. A small FIFO in shared memory tells the
@@ -57,12 +60,13 @@ constexpr int kGStages = 4;
 constexpr int kAStageBytes = BM * BK * 2;  // 16 KB
 constexpr int kBStageBytes = BN * BK * 2;  // 32 KB
 constexpr int kGStageBytes = kAStageBytes + kBStageBytes;
-constexpr int kGemmThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+// warp 0 TMA, warp 1 MMA, warps 2-5 epilogue, warps 6-7 prologue
+constexpr int kGemmThreads = 256;
 constexpr int kEpiThreads = 128;
+constexpr int kProThreads = 64;
 constexpr int kTmemCols = 2 * BN;  // two fp32 accumulators of 128 lanes x 256 columns
 constexpr int kFifo = 8;           // tiles announced ahead to the MMA and epilogue warps
 constexpr int kCtrSlots = 4;       // completion counters: chunk c uses slot c % 4
-constexpr int kMaxRowsPerPStage = 8;
 constexpr int kMaxLanes = 2;       // concat / fc-output lanes (RoPE rows: lanes + 1)
 // shared memory after the ring: barriers, the tile FIFO, per-stage row tokens and the
 // inverse frequencies
@@ -73,9 +77,9 @@ constexpr int kGemmSmem = kGStages * kGStageBytes + kHeadBytes + 1024 /* align *
 constexpr int kSmemMax = 227 * 1024;
 
 enum : int { TILE_P = 0, TILE_F = 1, TILE_V = 2 };
-// A 128-row block's prologue is split into kPParts P tiles of kPRows rows, so that several
-// SMs share it (its row loop is latency-bound on the four epilogue warps).
-constexpr int kPParts = 4, kPRows = BM / kPParts;
+// A 128-row block's prologue is split into kPParts P tiles of kPRows rows, so that every
+// SM's prologue warps share a chunk's prologue.
+constexpr int kPParts = 16, kPRows = BM / kPParts;
 constexpr int kArrivals = 3;  // counter kind: F tiles that finished (input norm only)
 
 struct PrefillParams {
@@ -112,11 +116,12 @@ struct PrefillParams {
     int mt_last;         // of the last chunk
     int nf;              // fc GEMM column tiles (h / 256)
     int nv;              // k/v GEMM column tiles (2 nkv hd / 256)
-    int64_t total;       // tiles in all
+    int64_t total;       // GEMM tiles (the tile counter's range)
+    int64_t p_total;     // prologue tiles (the prologue counter's range)
     int lanes;           // 1 or 2
-    int rows_per_pstage;
     int w_in_smem;       // 1: the norm weights are staged in shared memory
-    uint32_t* ctr;       // [0] tile counter; then done counters [4][kCtrSlots][mt_full]
+    uint32_t* ctr;       // [0] GEMM tile counter, [1] prologue tile counter; then done
+                         // counters [4][kCtrSlots][mt_full] from word 64
     uint16_t* concat[kMaxLanes];
     uint16_t* y[kMaxLanes];
     float2* rope[kMaxLanes + 1];
@@ -140,16 +145,14 @@ __device__ __forceinline__ int64_t cum_mt(const PrefillParams& p, int k) {
                                : (int64_t)(p.n_chunks - 1) * p.mt_full + p.mt_last;
 }
 
-// First tile of block b (b = 0 .. n_chunks + 1). With two lanes block b holds P(b + 1),
-// F(b), V(b - 1) -- the prologue runs a chunk ahead, so a chunk's fc tiles find their
-// concat rows ready -- and block 0 also P(0) first; with one lane V(b - 1), P(b), F(b),
-// since F(b) then reuses the fc-output rows V(b - 1) reads.
+// First GEMM tile of block b (b = 0 .. n_chunks + 1). With two lanes block b holds F(b),
+// then V(b - 1); with one lane V(b - 1), then F(b), since F(b) then reuses the fc-output
+// rows V(b - 1) reads.
 __device__ __forceinline__ int64_t block_start(const PrefillParams& p, int b) {
-    const int64_t pc = p.lanes == 2 ? (b == 0 ? 0 : cum_mt(p, b + 1)) : cum_mt(p, b);
-    return kPParts * pc + p.nf * cum_mt(p, b) + p.nv * cum_mt(p, b - 1);
+    return p.nf * cum_mt(p, b) + p.nv * cum_mt(p, b - 1);
 }
 
-// Tile t of the global order.
+// GEMM tile t of the global order.
 __device__ Tile decode(const PrefillParams& p, int64_t t) {
     Tile r{};
     if (p.plain) {  // F tiles of one GEMM, M-fastest
@@ -173,34 +176,41 @@ __device__ Tile decode(const PrefillParams& p, int64_t t) {
     auto seg = [&](int kind, int c) {
         if (found) return;
         const int mt = mt_of(p, c);
-        const int64_t cnt = (int64_t)mt * (kind == TILE_P ? kPParts : kind == TILE_F ? p.nf : p.nv);
-        if (off < cnt) {
+        const int64_t cnt = (int64_t)mt * (kind == TILE_F ? p.nf : p.nv);
+        if (off < cnt) {  // M-fastest
             r.kind = kind;
             r.c = c;
-            if (kind == TILE_P) {  // (row block, part), parts of a block adjacent
-                r.m = (int)(off / kPParts);
-                r.n = (int)(off % kPParts);
-            } else {  // GEMM tiles M-fastest
-                r.m = (int)(off % mt);
-                r.n = (int)(off / mt);
-            }
+            r.m = (int)(off % mt);
+            r.n = (int)(off / mt);
             found = true;
         } else {
             off -= cnt;
         }
     };
     if (p.lanes == 2) {
-        if (b == 0) seg(TILE_P, 0);
-        if (b + 1 < n) seg(TILE_P, b + 1);
         if (b < n) seg(TILE_F, b);
         if (b >= 1) seg(TILE_V, b - 1);
     } else {
         if (b >= 1) seg(TILE_V, b - 1);
-        if (b < n) {
-            seg(TILE_P, b);
-            seg(TILE_F, b);
-        }
+        if (b < n) seg(TILE_F, b);
     }
+    return r;
+}
+
+// Prologue tile i: chunk by chunk, row block by row block, part by part.
+__device__ Tile decode_p(const PrefillParams& p, int64_t i) {
+    int lo = 0, hi = p.n_chunks - 1;  // the last chunk whose first P tile is at or before i
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (kPParts * cum_mt(p, mid) <= i) lo = mid;
+        else hi = mid - 1;
+    }
+    const int64_t off = i - kPParts * cum_mt(p, lo);
+    Tile r{};
+    r.kind = TILE_P;
+    r.c = lo;
+    r.m = (int)(off / kPParts);
+    r.n = (int)(off % kPParts);
     return r;
 }
 
@@ -334,6 +344,44 @@ __device__ __forceinline__ float hsum_f32x2(uint64_t v) {
     return __uint_as_float((uint32_t)v) + __uint_as_float((uint32_t)(v >> 32));
 }
 
+// One warp: dst[j] = bf16((src[j] inv) (w[j] + add)) over a bf16 row of `pieces` 16-byte
+// pieces, inv = 1 / sqrt(mean(src^2) + eps); src null reads as a zero row. Up to 32 x
+// kNormRegs pieces are held in registers (one read), longer rows are read twice.
+constexpr int kNormRegs = 20;
+__device__ __forceinline__ void norm_row(const uint4* src, const uint4* w, uint4* dst, int pieces,
+                                         int lane, float eps, uint64_t wadd) {
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    uint64_t s2 = 0;
+    if (pieces <= 32 * kNormRegs) {
+        uint4 v[kNormRegs];
+#pragma unroll
+        for (int i = 0; i < kNormRegs; ++i) {
+            const int j = lane + 32 * i;
+            v[i] = (src && j < pieces) ? ldg_stream(src + j) : z;
+        }
+#pragma unroll
+        for (int i = 0; i < kNormRegs; ++i) s2 = sumsq8(v[i], s2);
+        float ss = hsum_f32x2(s2);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const uint64_t inv = f32x2_splat(1.0f / sqrtf(ss / (float)(8 * pieces) + eps));
+#pragma unroll
+        for (int i = 0; i < kNormRegs; ++i) {
+            const int j = lane + 32 * i;
+            if (j < pieces) dst[j] = norm8(v[i], inv, w[j], wadd);
+        }
+        return;
+    }
+#pragma unroll 4
+    for (int j = lane; j < pieces; j += 32) s2 = sumsq8(src ? __ldg(src + j) : z, s2);
+    float ss = hsum_f32x2(s2);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const uint64_t inv = f32x2_splat(1.0f / sqrtf(ss / (float)(8 * pieces) + eps));
+#pragma unroll 4
+    for (int j = lane; j < pieces; j += 32) dst[j] = norm8(src ? __ldg(src + j) : z, inv, w[j], wadd);
+}
+
 struct Maps {
     CUtensorMap a_concat[kMaxLanes];  // plain GEMM: a_concat[0] is A
     CUtensorMap a_y[kMaxLanes];
@@ -358,7 +406,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fifo + kFifo);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     volatile int* last_flag = abort_flag + 1;  // this F tile was its row block's last
-    int* stage_tok = reinterpret_cast<int*>(head + 512);         // [kGStages][8]
     double* inv_freq = reinterpret_cast<double*>(head + 2048);   // [hd / 2 <= 128], in turns
     uint16_t* kn_s = reinterpret_cast<uint16_t*>(head + 3072);   // [hd <= 256] k norm weights
     uint4* w_s = reinterpret_cast<uint4*>(head + kHeadBytes);    // [2 or 3][h / 8] norm weights
@@ -387,6 +434,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
+    const int half = p.hd / 2;
+    if (!p.plain) {  // the rotation per position of each pair, in turns; norm weights
+        for (int j = threadIdx.x; j < half; j += kGemmThreads)
+            inv_freq[j] = pow(p.rope_base, -2.0 * (double)j / (double)p.hd) /
+                          (2.0 * 3.14159265358979323846);
+        if (p.k_norm)
+            for (int j = threadIdx.x; j < p.hd; j += kGemmThreads) kn_s[j] = p.k_norm[j];
+        if (p.w_in_smem) {
+            const int pc = p.h / 8;
+            for (int j = threadIdx.x; j < pc; j += kGemmThreads) {
+                w_s[j] = __ldg(reinterpret_cast<const uint4*>(p.w_ne) + j);
+                w_s[pc + j] = __ldg(reinterpret_cast<const uint4*>(p.w_nh) + j);
+                if (p.in_norm) w_s[2 * pc + j] = __ldg(reinterpret_cast<const uint4*>(p.in_norm) + j);
+            }
+        }
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -394,10 +457,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     // stages of a tile in the ring: a GEMM tile's K blocks, or a P tile's row groups
     auto tile_stages = [&](const Tile& tl) -> int {
-        if (tl.kind == TILE_P) {
-            const int rows = p_tile_rows(p, tl);
-            return (rows + p.rows_per_pstage - 1) / p.rows_per_pstage;
-        }
+        if (tl.kind == TILE_P) return 0;  // read by the epilogue warps, not through the ring
         if (p.plain) return p.K / BK;
         return (tl.kind == TILE_F ? 2 * p.h : p.h) / BK;
     };
@@ -429,51 +489,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 qph ^= 1u;
             }
             if (end) break;
+            const Tile tl = decode(p, t);
             int64_t tn = t + gridDim.x;  // the next claim, issued early
             if (!p.plain && lane == 0) tn = atomicAdd(p.ctr, 1u);
-            const Tile tl = decode(p, t);
             const int nst = tile_stages(tl);
-            if (tl.kind == TILE_P) {
-                const int64_t row0 = (int64_t)tl.c * p.chunk + (int64_t)tl.m * BM +
-                                     (int64_t)tl.n * kPRows;  // prompt row
-                const int rows = p_tile_rows(p, tl);
-                const uint32_t rb = 2u * (uint32_t)p.h;  // bytes of one bf16 row
-                for (int st = 0; st < nst && !stop; ++st) {
-                    if (!mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag)) {
-                        stop = true;
-                        break;
-                    }
-                    const int r0 = st * p.rows_per_pstage;
-                    const int nr = min(p.rows_per_pstage, rows - r0);
-                    int64_t tok = -1;
-                    if (lane < nr) {
-                        tok = p.tokens[row0 + r0 + lane];
-                        if (tok < 0 || tok >= p.vocab) {
-                            raise_flag(p.dev_err, DEVFLAG_BAD_TOKEN);
-                            tok = -1;
-                        }
-                        stage_tok[s * kMaxRowsPerPStage + lane] = (int)tok;
-                    }
-                    const uint32_t mine = lane < nr ? (tok >= 0 ? 2u * rb : rb) : 0u;
-                    uint32_t bytes = mine;
-#pragma unroll
-                    for (int o = 16; o; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_expect_tx(&full[s], bytes);
-                    __syncwarp();
-                    if (lane < nr) {
-                        uint8_t* dst = stages + (size_t)s * kGStageBytes + (size_t)lane * 2u * rb;
-                        if (tok >= 0) bulk_copy_g2s(dst, p.embed + tok * p.h, rb, &full[s]);
-                        bulk_copy_g2s(dst + rb, p.hidden + (row0 + r0 + lane) * p.h, rb, &full[s]);
-                    }
-                    __syncwarp();
-                    ++issued;
-                    if (++s == kGStages) {
-                        s = 0;
-                        ph ^= 1u;
-                    }
-                }
-            } else {
+            {
                 // operands: F reads the chunk's concat rows, V its fc output rows; each only
                 // once the tiles that write them are done
                 const CUtensorMap* ma;
@@ -529,7 +549,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------- MMA issuer (one thread); P tiles' stages are the epilogue's
+        // ---------------- MMA issuer (one thread)
         constexpr uint32_t idesc = idesc_bf16(BM, BN);
         int s = 0;
         uint32_t ph = 0;
@@ -549,12 +569,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (t < 0) break;
             const Tile tl = decode(p, t);
             const int nst = tile_stages(tl);
-            if (tl.kind == TILE_P) {  // skip the P tile's stages
-                s += nst;
-                ph ^= (uint32_t)((s / kGStages) & 1);
-                s %= kGStages;
-                continue;
-            }
             const int buf = local & 1;
             const uint32_t tph = (uint32_t)((local >> 1) & 1);
             if (!mbar_wait_bounded(&tempty[buf], tph ^ 1u, abort_flag)) break;
@@ -589,33 +603,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (lane == 0) umma_commit(done);
         __syncwarp();
         mbar_wait_bounded(done, 0u, nullptr);
-    } else {
+    } else if (warp < 6) {
         // ---------------- epilogue warps 2..5: TMEM lane quarter = warp % 4
         const int qd = warp & 3;
         const int et = threadIdx.x - 64;  // 0..127
         const int ew = et >> 5;
-        const int half = p.hd / 2;
         int s = 0;
         uint32_t ph = 0;
         int q = 0;
         uint32_t qph = 0;
         int local = 0;
-        if (!p.plain) {  // the rotation per position of each pair, in turns
-            for (int j = et; j < half; j += kEpiThreads)
-                inv_freq[j] = pow(p.rope_base, -2.0 * (double)j / (double)p.hd) /
-                              (2.0 * 3.14159265358979323846);
-            if (p.k_norm)
-                for (int j = et; j < p.hd; j += kEpiThreads) kn_s[j] = p.k_norm[j];
-            if (p.w_in_smem) {
-                const int pc = p.h / 8;
-                for (int j = et; j < pc; j += kEpiThreads) {
-                    w_s[j] = __ldg(reinterpret_cast<const uint4*>(p.w_ne) + j);
-                    w_s[pc + j] = __ldg(reinterpret_cast<const uint4*>(p.w_nh) + j);
-                    if (p.in_norm) w_s[2 * pc + j] = __ldg(reinterpret_cast<const uint4*>(p.in_norm) + j);
-                }
-            }
-        }
-        named_sync(1, kEpiThreads);
         while (true) {
             if (!mbar_wait_bounded(&qfull[q], qph, abort_flag)) break;
             const int t = fifo[q];
@@ -630,89 +627,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int nst = tile_stages(tl);
             const int64_t crow0 = (int64_t)tl.c * p.chunk;  // prompt row of the chunk's row 0
             const int64_t rows_c = p.plain ? p.M : min(p.chunk, p.R - crow0);
-            if (tl.kind == TILE_P) {
-                // ---- prologue of rows m*128 + n*32 .. : the lanes' buffers are free once
-                // the chunks that used them before are done with them
-                const int lane_c = tl.c % p.lanes, slot_r = tl.c % (p.lanes + 1);
-                bool ok = true;
-                if (et == 0) {
-                    const int ca = tl.c - p.lanes, cr = tl.c - p.lanes - 1;
-                    if (ca >= 0)
-                        ok = wait_counter(counter(p, TILE_F, ca, tl.m),
-                                          (uint32_t)((ca / kCtrSlots + 1) * p.nf), abort_flag);
-                    if (ok && cr >= 0)
-                        ok = wait_counter(counter(p, TILE_V, cr, tl.m),
-                                          (uint32_t)((cr / kCtrSlots + 1) * p.nv), abort_flag);
-                }
-                named_sync(1, kEpiThreads);
-                const int rows = p_tile_rows(p, tl);
-                const int prow0 = tl.m * BM + tl.n * kPRows;  // the tile's first row of the chunk
-                const int h = p.h, pieces = h / 8;  // 16-byte pieces of a row
-                const uint64_t wadd = f32x2_splat(p.norm_mode ? 1.f : 0.f);
-                const uint32_t rb = 2u * (uint32_t)h;
-                // generic loads: shared memory when staged, else global
-                const uint4* wne = p.w_in_smem ? w_s : reinterpret_cast<const uint4*>(p.w_ne);
-                const uint4* wnh = p.w_in_smem ? w_s + pieces : reinterpret_cast<const uint4*>(p.w_nh);
-                // warp ew takes the tile's stages ew, ew + 4, ... (with a 4-stage ring always
-                // the same ring slot), each of its rows with warp-wide reductions, so the
-                // four warps run independently
-                static_assert(kGStages == kEpiThreads / 32, "one ring slot per epilogue warp");
-                for (int st = ew; st < nst; st += kGStages) {
-                    const int sl = (s + st) % kGStages;
-                    const uint32_t sph = ph ^ (uint32_t)(((s + st) / kGStages) & 1);
-                    if (!mbar_wait_bounded(&full[sl], sph, abort_flag)) break;
-                    const int r0 = st * p.rows_per_pstage;
-                    const int nr = min(p.rows_per_pstage, rows - r0);
-                    for (int i = 0; i < nr; ++i) {
-                        const int tok = stage_tok[sl * kMaxRowsPerPStage + i];
-                        const uint8_t* erow = stages + (size_t)sl * kGStageBytes + (size_t)i * 2u * rb;
-                        const uint8_t* xrow = erow + rb;
-                        uint64_t se2 = 0, sx2 = 0;
-#pragma unroll 4
-                        for (int j = lane; j < pieces; j += 32) {
-                            if (tok >= 0) se2 = sumsq8(lds128(erow + 16 * j), se2);
-                            sx2 = sumsq8(lds128(xrow + 16 * j), sx2);
-                        }
-                        float se = hsum_f32x2(se2), sx = hsum_f32x2(sx2);
-#pragma unroll
-                        for (int o = 16; o; o >>= 1) {
-                            se += __shfl_xor_sync(0xffffffffu, se, o);
-                            sx += __shfl_xor_sync(0xffffffffu, sx, o);
-                        }
-                        const uint64_t inv_e = f32x2_splat(1.0f / sqrtf(se / (float)h + p.eps));
-                        const uint64_t inv_x = f32x2_splat(1.0f / sqrtf(sx / (float)h + p.eps));
-                        uint4* crow = reinterpret_cast<uint4*>(
-                            p.concat[lane_c] + ((int64_t)prow0 + r0 + i) * 2 * h);
-#pragma unroll 4
-                        for (int j = lane; j < pieces; j += 32) {
-                            const uint4 e = tok >= 0 ? lds128(erow + 16 * j) : make_uint4(0, 0, 0, 0);
-                            crow[j] = norm8(e, inv_e, wne[j], wadd);
-                            crow[pieces + j] = norm8(lds128(xrow + 16 * j), inv_x, wnh[j], wadd);
-                        }
-                    }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&empty[sl]);  // done with the stage
-                }
-                s += nst;
-                ph ^= (uint32_t)((s / kGStages) & 1);
-                s %= kGStages;
-                // RoPE table of the rows: the angle pos * base^(-2j / hd) in turns, reduced to
-                // [-1/2, 1/2] in double (exact to ~1e-12 turns), then cos and sin of the
-                // remainder in fp32 (sincospif: no further range reduction)
-                float2* cs = p.rope[slot_r] + (int64_t)prow0 * half;
-                for (int k = et; k < rows * half; k += kEpiThreads) {
-                    const int r = k / half, j = k - r * half;
-                    const double turns = (double)p.rope_pos[crow0 + prow0 + r] * inv_freq[j];
-                    const float f = (float)(turns - rint(turns));
-                    float sn, cn;
-                    sincospif(2.0f * f, &sn, &cn);  // sin and cos of pi x: x in half turns
-                    cs[k] = make_float2(cn, sn);
-                }
-                fence_proxy_async_global();  // the concat rows are read by TMA
-                named_sync(1, kEpiThreads);
-                if (et == 0 && !*abort_flag) counter_release_add(counter(p, TILE_P, tl.c, tl.m), 1u);
-                continue;
-            }
             // ---- GEMM tile: its stages are the MMA warp's
             s += nst;
             ph ^= (uint32_t)((s / kGStages) & 1);
@@ -866,6 +780,78 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
             }
         }
+    } else {
+        // ---------------- prologue warps 6..7: claim prologue tiles from their own counter
+        // (every SM's pair takes the next one when it is free) and run them
+        const int pt = threadIdx.x - 192;  // 0..63
+        const int pw = pt >> 5;
+        volatile int* pclaim = last_flag + 1;
+        while (!p.plain) {
+            if (pt == 0) *pclaim = (int)atomicAdd(p.ctr + 1, 1u);
+            named_sync(2, kProThreads);
+            const int64_t t = *pclaim;
+            named_sync(2, kProThreads);  // everyone has read it before the next claim
+            if (t >= p.p_total || *abort_flag) break;
+            const Tile tl = decode_p(p, t);
+            const int64_t crow0 = (int64_t)tl.c * p.chunk;  // prompt row of the chunk's row 0
+            {
+                // ---- rows m*128 + n*kPRows .. : the lanes' buffers are free once the chunks
+                // that used them before are done with them
+                const int lane_c = tl.c % p.lanes, slot_r = tl.c % (p.lanes + 1);
+                bool ok = true;
+                if (pt == 0) {
+                    const int ca = tl.c - p.lanes, cr = tl.c - p.lanes - 1;
+                    if (ca >= 0)
+                        ok = wait_counter(counter(p, TILE_F, ca, tl.m),
+                                          (uint32_t)((ca / kCtrSlots + 1) * p.nf), abort_flag);
+                    if (ok && cr >= 0)
+                        ok = wait_counter(counter(p, TILE_V, cr, tl.m),
+                                          (uint32_t)((cr / kCtrSlots + 1) * p.nv), abort_flag);
+                }
+                named_sync(2, kProThreads);
+                const int rows = p_tile_rows(p, tl);
+                const int prow0 = tl.m * BM + tl.n * kPRows;  // the tile's first row of the chunk
+                const int h = p.h, pieces = h / 8;  // 16-byte pieces of a row
+                const uint64_t wadd = f32x2_splat(p.norm_mode ? 1.f : 0.f);
+                // generic loads: shared memory when staged, else global
+                const uint4* wne = p.w_in_smem ? w_s : reinterpret_cast<const uint4*>(p.w_ne);
+                const uint4* wnh = p.w_in_smem ? w_s + pieces : reinterpret_cast<const uint4*>(p.w_nh);
+                // warp pw takes rows pw, pw + 2, ...: each half of the concat row (embedding
+                // row, hidden row) is loaded straight from global memory into registers (up
+                // to 5,120 wide in one pass, else in two), reduced with warp shuffles and
+                // written normalized
+                for (int r = pw; r < rows; r += kProThreads / 32) {
+                    const int64_t prow = crow0 + prow0 + r;  // prompt row
+                    int64_t tok = p.tokens[prow];
+                    if (tok < 0 || tok >= p.vocab) {
+                        if (lane == 0) raise_flag(p.dev_err, DEVFLAG_BAD_TOKEN);
+                        tok = -1;
+                    }
+                    uint4* crow = reinterpret_cast<uint4*>(p.concat[lane_c] + ((int64_t)prow0 + r) * 2 * h);
+#pragma unroll 1
+                    for (int side = 0; side < 2; ++side) {  // embedding half, then hidden half
+                        const uint4* src = reinterpret_cast<const uint4*>(
+                            side == 0 ? (tok >= 0 ? p.embed + tok * h : nullptr) : p.hidden + prow * h);
+                        norm_row(src, side == 0 ? wne : wnh, crow + side * pieces, pieces, lane, p.eps, wadd);
+                    }
+                }
+                // RoPE table of the rows: the angle pos * base^(-2j / hd) in turns, reduced to
+                // [-1/2, 1/2] in double (exact to ~1e-12 turns), then cos and sin of the
+                // remainder in fp32 (sincospif: no further range reduction)
+                float2* cs = p.rope[slot_r] + (int64_t)prow0 * half;
+                for (int k = pt; k < rows * half; k += kProThreads) {
+                    const int r = k / half, j = k - r * half;
+                    const double turns = (double)p.rope_pos[crow0 + prow0 + r] * inv_freq[j];
+                    const float f = (float)(turns - rint(turns));
+                    float sn, cn;
+                    sincospif(2.0f * f, &sn, &cn);  // sin and cos of pi x: x in half turns
+                    cs[k] = make_float2(cn, sn);
+                }
+                fence_proxy_async_global();  // the concat rows are read by TMA
+                named_sync(2, kProThreads);
+                if (pt == 0 && !*abort_flag) counter_release_add(counter(p, TILE_P, tl.c, tl.m), 1u);
+            }
+        }
     }
     __syncthreads();
     if (*abort_flag && threadIdx.x == 0) raise_flag(p.dev_err, DEVFLAG_TIMEOUT);
@@ -991,7 +977,8 @@ size_t prefill_ws_bytes(int64_t chunk_rows, int32_t h, int32_t nkv, int32_t hd) 
     return 2 * prefill_ws_bytes_lanes(chunk_rows, h, hd, 1);
 }
 
-int prefill_max_hidden() { return kGStageBytes / 4; }  // one P row (two bf16 rows) per stage
+// The widest hidden size the prefill takes (the fc GEMM's K is twice it).
+int prefill_max_hidden() { return 12288; }
 
 cudaError_t prefill_launch(const PrefillArgs& a, cudaStream_t s) {
     const int kvd = a.nkv * a.hd;
@@ -1032,11 +1019,13 @@ cudaError_t prefill_launch(const PrefillArgs& a, cudaStream_t s) {
     p.lanes = (a.R > a.chunk_rows && a.ws_bytes >= prefill_ws_bytes_lanes(a.chunk_rows, a.h, a.hd, 2))
                   ? 2 : 1;
     p.total = 0;
-    for (int c = 0; c < p.n_chunks; ++c)
-        p.total += (int64_t)(c == p.n_chunks - 1 ? p.mt_last : p.mt_full) * (kPParts + p.nf + p.nv);
-    int rps = kGStageBytes / (4 * a.h);
-    p.rows_per_pstage = rps > kMaxRowsPerPStage ? kMaxRowsPerPStage : rps;
-    if (p.rows_per_pstage < 1 || a.hd / 2 > 128) return cudaErrorInvalidValue;
+    p.p_total = 0;
+    for (int c = 0; c < p.n_chunks; ++c) {
+        const int mt = c == p.n_chunks - 1 ? p.mt_last : p.mt_full;
+        p.total += (int64_t)mt * (p.nf + p.nv);
+        p.p_total += (int64_t)mt * kPParts;
+    }
+    if (a.hd / 2 > 128) return cudaErrorInvalidValue;
     // workspace carving
     uint8_t* w = static_cast<uint8_t*>(a.ws);
     p.ctr = reinterpret_cast<uint32_t*>(w);
@@ -1082,7 +1071,6 @@ cudaError_t gemm_bf16_launch(const uint16_t* A, const uint16_t* B, uint16_t* C, 
     p.nf = N / BN;
     p.total = (int64_t)((M + BM - 1) / BM) * (N / BN);
     p.dev_err = dev_err;
-    p.rows_per_pstage = 1;
     Maps maps{};
     cudaError_t e;
     if ((e = make_operand_map(&maps.a_concat[0], A, M, K, BM)) != cudaSuccess) return e;

@@ -269,7 +269,7 @@ def test_prefill_rejects(lib):
     assert st("mtp_prefill_kv", *prefill_args(inn=OUT + 8)) == L.MTP_ERR_INVALID_ARG  # 16-byte
     assert st("mtp_prefill_kv", *prefill_args(h=320)) == L.MTP_ERR_UNSUPPORTED   # h % 256
     assert st("mtp_prefill_kv", *prefill_args(hd=96)) == L.MTP_ERR_UNSUPPORTED
-    # a prologue row (embedding + hidden row) must fit one 48 KB ring stage
+    # hidden sizes up to 12,288
     assert st("mtp_prefill_kv", *prefill_args(h=12544)) == L.MTP_ERR_UNSUPPORTED
     assert st("mtp_prefill_kv", *prefill_args(nkv=1)) == L.MTP_ERR_UNSUPPORTED  # nkv*hd % 256
     assert st("mtp_prefill_kv", *prefill_args(hidden=A + 8)) == L.MTP_ERR_INVALID_ARG
