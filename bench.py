@@ -391,23 +391,32 @@ def bench_prefill(dev, reps, tflops_peak, peak_src, rows=0):
     kc = torch.zeros((d["num_blocks"], d["block_size"], d["nkv"], d["hd"]), dtype=torch.uint8,
                      device=dev)
     vc = torch.zeros_like(kc)
+    import numpy as np
+
     ws = api.prefill_kv(dd, kc, vc, chunk_rows=synth.PREFILL["chunk"])
-    for _ in range(2):
+    for _ in range(3):
         api.prefill_kv(dd, kc, vc, chunk_rows=synth.PREFILL["chunk"], ws=ws)
     torch.cuda.synchronize()
-    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record()
-    for _ in range(reps):
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    clocks = ClockSampler(dev)
+    clocks.start()
+    for s, e in ev:  # one call per event pair (each call is ~3 ms: the pair's gap is noise)
+        s.record()
         api.prefill_kv(dd, kc, vc, chunk_rows=synth.PREFILL["chunk"], ws=ws)
-    e.record()
+        e.record()
     torch.cuda.synchronize()
-    ms = s.elapsed_time(e) / reps
+    clk = clocks.stop()
+    per = np.array([s.elapsed_time(e) for s, e in ev])
+    ms = float(np.median(per))
     R, h, kvd = d["R"], d["h"], d["nkv"] * d["hd"]
     flops = 2.0 * R * (2 * h) * h + 2.0 * R * h * (2 * kvd)
     tf = flops / (ms * 1e-3) / 1e12
-    return {"ms": ms, "TFLOP/s": tf, "frac_of_peak": tf / tflops_peak,
-            "peak_source": peak_src, "flops": flops,
-            "rows": R, "hidden": h, "chunk": synth.PREFILL["chunk"]}
+    sus, _ = measured_tflops("bf16_tflops_sustained")
+    return {"ms": ms, "statistic": f"median of {reps} calls", "ms_min_max": [float(per.min()), float(per.max())],
+            "TFLOP/s": tf, "frac_of_peak": tf / tflops_peak,
+            "peak_source": peak_src, "frac_of_sustained_peak": tf / sus, "flops": flops,
+            "rows": R, "hidden": h, "chunk": synth.PREFILL["chunk"], "clocks": clk}
 
 
 def bench_attn(dev, steps, warmup, seq=32768, nq=64, nkv=8, hd=128):
@@ -671,7 +680,7 @@ def main():
     if args.only:
         tpk, tsrc = measured_tflops()
         if args.only == "prefill":
-            out = bench_prefill(dev, 2, tpk, tsrc, args.prefill_rows)
+            out = bench_prefill(dev, 10, tpk, tsrc, args.prefill_rows)
         elif args.only == "attn":
             out = bench_attn(dev, args.steps, args.warmup)
         elif args.only == "masked":  # profiling: the masked M = 1 sweep alone
@@ -797,7 +806,7 @@ def main():
     if world == 1 and not args.no_extra and not args.rows and not args.ms:
         rows["tiny_draft_M1"] = bench_tiny_draft(dev, max(200, args.steps // 10), args.warmup)
         tpk, tsrc = measured_tflops()
-        rows["prefill_32k"] = bench_prefill(dev, 5, tpk, tsrc)
+        rows["prefill_32k"] = bench_prefill(dev, 10, tpk, tsrc)
         rows["decode_attn_32k"] = bench_attn(dev, max(100, args.steps // 10), args.warmup)
         torch.cuda.empty_cache()
         if cpu_rows:

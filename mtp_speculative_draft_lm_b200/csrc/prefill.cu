@@ -344,9 +344,19 @@ __device__ __forceinline__ float hsum_f32x2(uint64_t v) {
     return __uint_as_float((uint32_t)v) + __uint_as_float((uint32_t)(v >> 32));
 }
 
+// 32 bytes of a row that is read once: not kept in L1 and first out of L2, so that it does
+// not push out the GEMM operands. `p` 32-byte aligned.
+__device__ __forceinline__ void ld256_once(const void* p, uint4& a, uint4& b) {
+    asm volatile(
+        "ld.global.nc.L1::no_allocate.L2::evict_first.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+        : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+        : "l"(p));
+}
+
 // One warp: dst[j] = bf16((src[j] inv) (w[j] + add)) over a bf16 row of `pieces` 16-byte
-// pieces, inv = 1 / sqrt(mean(src^2) + eps); src null reads as a zero row. Up to 32 x
-// kNormRegs pieces are held in registers (one read), longer rows are read twice.
+// pieces (an even number; src 32-byte aligned), inv = 1 / sqrt(mean(src^2) + eps); src
+// null reads as a zero row. Up to 32 x kNormRegs pieces are held in registers (one read,
+// 32 bytes per lane and load), longer rows are read twice.
 constexpr int kNormRegs = 20;
 __device__ __forceinline__ void norm_row(const uint4* src, const uint4* w, uint4* dst, int pieces,
                                          int lane, float eps, uint64_t wadd) {
@@ -355,9 +365,10 @@ __device__ __forceinline__ void norm_row(const uint4* src, const uint4* w, uint4
     if (pieces <= 32 * kNormRegs) {
         uint4 v[kNormRegs];
 #pragma unroll
-        for (int i = 0; i < kNormRegs; ++i) {
-            const int j = lane + 32 * i;
-            v[i] = (src && j < pieces) ? ldg_stream(src + j) : z;
+        for (int i = 0; i < kNormRegs / 2; ++i) {
+            const int j = 2 * (lane + 32 * i);  // this lane's pair of pieces
+            v[2 * i] = v[2 * i + 1] = z;
+            if (src && j < pieces) ld256_once(src + j, v[2 * i], v[2 * i + 1]);
         }
 #pragma unroll
         for (int i = 0; i < kNormRegs; ++i) s2 = sumsq8(v[i], s2);
@@ -366,9 +377,12 @@ __device__ __forceinline__ void norm_row(const uint4* src, const uint4* w, uint4
         for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
         const uint64_t inv = f32x2_splat(1.0f / sqrtf(ss / (float)(8 * pieces) + eps));
 #pragma unroll
-        for (int i = 0; i < kNormRegs; ++i) {
-            const int j = lane + 32 * i;
-            if (j < pieces) dst[j] = norm8(v[i], inv, w[j], wadd);
+        for (int i = 0; i < kNormRegs / 2; ++i) {
+            const int j = 2 * (lane + 32 * i);
+            if (j < pieces) {
+                dst[j] = norm8(v[2 * i], inv, w[j], wadd);
+                dst[j + 1] = norm8(v[2 * i + 1], inv, w[j + 1], wadd);
+            }
         }
         return;
     }
