@@ -16,8 +16,9 @@
 // warp keeping 16 rows' 16-byte loads in flight; per input the CTAs' (max, lowest row)
 // partials go to CTA 0's shared memory and CTA 0 writes the result. Two cluster barriers,
 // no global workspace. Launched with programmatic stream serialization, so in a chain of
-// drafts the next step's launch overlaps this one's end: it prefetches its weight rows into
-// L1 first and waits for the previous step only before reading the token and hidden rows
+// drafts the next step's launch overlaps this one's end: it first copies its fc and head
+// rows into shared memory (bulk copies, when they fit in about 192 KB; else it pulls them
+// into L1) and waits for the previous step only before reading the token and hidden rows
 // that step writes.
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -57,6 +58,7 @@ struct DraftParams {
     int32_t* out_idx;
     float* out_val;
     int32_t* dev_err;
+    int staged;             // 1: the CTA's fc and head rows are copied into shared memory
 };
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -120,20 +122,47 @@ __global__ void __launch_bounds__(kDThreads, 1) draft_step_kernel(const __grid_c
     __shared__ float wv[kDWarps][kDMaxM];
     __shared__ int32_t wi[kDWarps][kDMaxM];
     __shared__ __align__(8) float2 cpart[kDMaxCluster][kDMaxM];  // CTA 0: (value, row bits)
+    __shared__ __align__(8) uint64_t wbar;                        // the staged weights landed
+    extern __shared__ __align__(128) uint8_t dsm[];               // staged fc rows, head rows
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     constexpr int RPW = MM == 1 ? kDRowsPerWarp : kDRowsPerWarp / 2;
     const uint32_t rank = cluster_rank(), CL = cluster_size();
     const int M = p.M, h = p.h, h2 = 2 * h;
     pdl_launch_dependents();
-    // The weights never change: pull this CTA's fc rows and head rows into L1 before
-    // waiting for the previous step, so that their latency overlaps its end.
-    {
-        const int rows_per = (h + (int)CL - 1) / (int)CL;
-        const int f0 = (int)rank * rows_per, f1 = min(h, f0 + rows_per);
-        const int64_t per = (p.n + CL - 1) / CL;
-        const int64_t q0 = (int64_t)rank * per, q1 = min(p.n, q0 + per);
-        const int64_t fl = (int64_t)(f1 - f0) * h2 * 2 / 128;  // 128-byte lines
-        const int64_t hl = (q1 - q0) * h * 2 / 128;
+    // The weights never change: this CTA's fc rows and head rows are fetched before waiting
+    // for the previous step, so that their latency overlaps its end -- copied into shared
+    // memory by bulk copies when they fit (staged), else pulled into L1.
+    const int rows_per = (h + (int)CL - 1) / (int)CL;
+    const int f0 = (int)rank * rows_per, f1 = min(h, f0 + rows_per);
+    const int64_t per = (p.n + CL - 1) / CL;
+    const int64_t q0 = (int64_t)rank * per, q1 = min(p.n, q0 + per);
+    const uint32_t fbytes = (uint32_t)max(0, f1 - f0) * (uint32_t)h2 * 2u;
+    const uint32_t hbytes = (uint32_t)max((int64_t)0, q1 - q0) * (uint32_t)h * 2u;
+    const uint32_t hoff = (fbytes + 127u) & ~127u;  // head rows after the fc rows
+    const uint16_t* fc_s = reinterpret_cast<const uint16_t*>(dsm);
+    const uint16_t* head_s = reinterpret_cast<const uint16_t*>(dsm + hoff);
+    if (p.staged) {
+        if (tid == 0) {
+            mbar_init(&wbar, 1);
+            mbar_fence_init();
+        }
+        __syncthreads();
+        if (warp == 0) {
+            constexpr uint32_t kPiece = 16384;
+            const uint32_t nf = (fbytes + kPiece - 1) / kPiece, nh = (hbytes + kPiece - 1) / kPiece;
+            if (lane == 0) mbar_arrive_expect_tx(&wbar, fbytes + hbytes);
+            __syncwarp();
+            const uint8_t* fb = reinterpret_cast<const uint8_t*>(p.fc + (int64_t)f0 * h2);
+            const uint8_t* hb = reinterpret_cast<const uint8_t*>(p.head + q0 * h);
+            for (uint32_t i = lane; i < nf + nh; i += 32) {
+                const bool isf = i < nf;
+                const uint32_t o = (isf ? i : i - nf) * kPiece;
+                const uint32_t n = min(kPiece, (isf ? fbytes : hbytes) - o);
+                bulk_copy_g2s(dsm + (isf ? 0u : hoff) + o, (isf ? fb : hb) + o, n, &wbar);
+            }
+        }
+    } else {
+        const int64_t fl = fbytes / 128, hl = hbytes / 128;  // 128-byte lines
         const uint8_t* fb = reinterpret_cast<const uint8_t*>(p.fc + (int64_t)f0 * h2);
         const uint8_t* hb = reinterpret_cast<const uint8_t*>(p.head + q0 * h);
         for (int64_t i = tid; i < fl + hl; i += kDThreads) {
@@ -184,15 +213,16 @@ __global__ void __launch_bounds__(kDThreads, 1) draft_step_kernel(const __grid_c
     }
 
     // 2. this CTA's slice of y = bf16(fc . c): a warp per fc row, 16-byte pieces per lane
-    const int rows_per = (h + (int)CL - 1) / (int)CL;
-    const int r0 = (int)rank * rows_per, r1 = min(h, r0 + rows_per);
+    if (p.staged && !mbar_wait_bounded(&wbar, 0u, nullptr) && tid == 0)
+        raise_flag(p.dev_err, DEVFLAG_TIMEOUT);  // (the copies' bytes never arrived)
+    const int r0 = f0, r1 = f1;
     for (int r = r0 + warp; r < r1; r += kDWarps) {
-        const uint16_t* frow = p.fc + (int64_t)r * h2;
+        const uint16_t* frow = p.staged ? fc_s + (int64_t)(r - r0) * h2 : p.fc + (int64_t)r * h2;
         float acc[MM];
 #pragma unroll
         for (int m = 0; m < MM; ++m) acc[m] = 0.f;
         for (int c = lane; c < h2 / 8; c += 32) {
-            const uint4 a = __ldg(reinterpret_cast<const uint4*>(frow + 8 * c));
+            const uint4 a = p.staged ? lds128(frow + 8 * c) : __ldg(reinterpret_cast<const uint4*>(frow + 8 * c));
 #pragma unroll
             for (int m = 0; m < MM; ++m)
                 if (m < M) acc[m] += dot8(a, &cs[m][8 * c]);
@@ -235,8 +265,7 @@ __global__ void __launch_bounds__(kDThreads, 1) draft_step_kernel(const __grid_c
         bv[m] = -INFINITY;
         bi[m] = INT_MAX;
     }
-    const int64_t per = (p.n + CL - 1) / CL;
-    const int64_t n0 = (int64_t)rank * per, n1 = min(p.n, n0 + per);
+    const int64_t n0 = q0, n1 = q1;
     const int pieces = h / 8;
     for (int64_t g = n0 + (int64_t)warp * RPW; g < n1; g += (int64_t)kDWarps * RPW) {
         float acc[RPW][MM];
@@ -250,7 +279,8 @@ __global__ void __launch_bounds__(kDThreads, 1) draft_step_kernel(const __grid_c
 #pragma unroll
             for (int j = 0; j < RPW; ++j)
                 a[j] = (c < pieces && g + j < n1)
-                           ? __ldg(reinterpret_cast<const uint4*>(p.head + (g + j) * h + 8 * c))
+                           ? (p.staged ? lds128(head_s + (g + j - n0) * h + 8 * c)
+                                       : __ldg(reinterpret_cast<const uint4*>(p.head + (g + j) * h + 8 * c)))
                            : make_uint4(0, 0, 0, 0);
             if (c < pieces) {
 #pragma unroll
@@ -348,13 +378,24 @@ cudaError_t draft_step_launch(const uint16_t* embed, int64_t vocab, const int32_
     p.out_idx = out_idx;
     p.out_val = out_val;
     p.dev_err = dev_err;
-    // 16 CTAs per cluster where the device allows it, else the portable 8
+    // 16 CTAs per cluster where the device allows it, else the portable 8; each CTA's fc
+    // and head rows staged in shared memory when they fit beside the static arrays
     auto kern = M == 1 ? draft_step_kernel<1> : draft_step_kernel<kDMaxM>;
+    auto staged_bytes = [&](int clusters) -> size_t {
+        const size_t rows_per = (size_t)((h + clusters - 1) / clusters);
+        const size_t per = (size_t)((n + clusters - 1) / clusters);
+        return ((rows_per * 2 * (size_t)h * 2 + 127) & ~(size_t)127) + per * (size_t)h * 2;
+    };
+    constexpr size_t kStageLimit = 192 * 1024;  // beside ~26 KB of static shared memory
     static int cl_cached[2][64] = {{0}};  // per instance and device: the cluster size used
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     const int inst = M == 1 ? 0 : 1;
+    // the cluster size is the same for every head: it is chosen with the staging limit
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStageLimit) !=
+        cudaSuccess)
+        cudaGetLastError();
     int cl = dev >= 0 && dev < 64 ? cl_cached[inst][dev] : 0;
     if (cl == 0) {
         cl = 8;
@@ -363,6 +404,7 @@ cudaError_t draft_step_launch(const uint16_t* embed, int64_t vocab, const int32_
             cudaLaunchConfig_t q{};
             q.gridDim = dim3(kDMaxCluster);
             q.blockDim = dim3(kDThreads);
+            q.dynamicSmemBytes = kStageLimit;
             cudaLaunchAttribute qa[1];
             qa[0].id = cudaLaunchAttributeClusterDimension;
             qa[0].val.clusterDim.x = kDMaxCluster;
@@ -378,10 +420,12 @@ cudaError_t draft_step_launch(const uint16_t* embed, int64_t vocab, const int32_
         cudaGetLastError();  // a refused attribute or query leaves nothing behind
         if (dev >= 0 && dev < 64) cl_cached[inst][dev] = cl;
     }
+    const size_t sb = staged_bytes(cl);
+    p.staged = sb <= kStageLimit;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)cl);
     cfg.blockDim = dim3(kDThreads);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = p.staged ? sb : 0;
     cfg.stream = s;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
