@@ -32,10 +32,9 @@ FALLBACK_HBM_GBS = 6650.0
 
 # DRAM traffic per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum) and
 # the sha256 of sweep.cu when it was captured; reported as null once the source changed.
-# bf16_M1: the 40,000-row capture of the BF16 sweep read
-# 327,776,256 B and wrote 3,843,584 B; reads scale with the rows swept, so a full
-# 154,880-row launch reads 327,776,256 x 154,880 / 40,000 B (writes kept unscaled).
-NCU_TRAFFIC = {"bf16_M1": (1272993247, "ebea71e05b1b11fa")}
+# bf16_M1: a full-size capture (one-pass metrics) of the headline sweep, the mean of two
+# launches: 1,268,870,144 + 128,256 and 1,268,873,728 + 133,632 B.
+NCU_TRAFFIC = {"bf16_M1": (1269002880, "e2d56e5da49d5793")}
 
 
 def sweep_source_hash() -> str:

@@ -117,35 +117,36 @@ __global__ void __launch_bounds__(kAThreads) attn_piece_kernel(const __grid_cons
     // copies of sub-piece i into ring stage i % 3 (positions past the piece: invalid)
     // 32-bit position arithmetic (seq_len <= 2^21); a power-of-two block size shifts
     const int pend32 = (int)pend;
+    // copies of sub-piece i: thread t takes half of row t / 2 (its slot looked up once)
+    static_assert(kAThreads == 2 * kSP, "two threads per row of a sub-piece");
     auto issue = [&](int i) {
         if (i < nsub) {
             const int st = i % kAStages;
-            uint8_t* kd = kring + st * kSP * RP;
-            uint8_t* vd = vring + st * kSP * RP;
-            const int pc = tid % KC;
-            const int pos0 = (int)pbeg + i * kSP;
-            for (int r = tid / KC; r < kSP; r += kAThreads / KC) {
-                const int pos = pos0 + r;
-                int64_t slot = -1;
-                if (pos < pend32) {
-                    const int b = p.bs_shift >= 0 ? pos >> p.bs_shift : pos / p.block_size;
-                    if (b < p.n_table) {
-                        const int32_t blk = __ldg(p.block_table + b);
-                        if (blk >= 0 && blk < p.num_blocks)
-                            slot = (int64_t)blk * p.block_size + (pos - b * p.block_size);
-                    }
-                    if (slot < 0 && pc == 0) raise_flag(p.dev_err, DEVFLAG_BAD_SLOT);
+            const int r = tid >> 1, hf = tid & 1;
+            const int pos = (int)pbeg + i * kSP + r;
+            int64_t slot = -1;
+            if (pos < pend32) {
+                const int b = p.bs_shift >= 0 ? pos >> p.bs_shift : pos / p.block_size;
+                if (b < p.n_table) {
+                    const int32_t blk = __ldg(p.block_table + b);
+                    if (blk >= 0 && blk < p.num_blocks)
+                        slot = (int64_t)blk * p.block_size + (pos - b * p.block_size);
                 }
-                if (pc == 0) valid[st * kSP + r] = slot >= 0;
-                uint8_t* kdst = kd + r * RP + 16 * pc;
-                uint8_t* vdst = vd + r * RP + 16 * pc;
+                if (slot < 0 && hf == 0) raise_flag(p.dev_err, DEVFLAG_BAD_SLOT);
+            }
+            if (hf == 0) valid[st * kSP + r] = slot >= 0;
+            uint8_t* kdst = kring + (st * kSP + r) * RP;
+            uint8_t* vdst = vring + (st * kSP + r) * RP;
+            const int64_t off = (slot * p.nkv + g) * (int64_t)HD;
+#pragma unroll
+            for (int c = 0; c < KC / 2; ++c) {
+                const int pc = hf * (KC / 2) + c;
                 if (slot >= 0) {
-                    const int64_t off = (slot * p.nkv + g) * (int64_t)HD + 16 * pc;
-                    cp_async16(kdst, p.k_cache + off);
-                    cp_async16(vdst, p.v_cache + off);
+                    cp_async16(kdst + 16 * pc, p.k_cache + off + 16 * pc);
+                    cp_async16(vdst + 16 * pc, p.v_cache + off + 16 * pc);
                 } else {  // zeros: the weight of the row is 0, and 0 * NaN would not be
-                    *reinterpret_cast<uint4*>(kdst) = make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4*>(vdst) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4*>(kdst + 16 * pc) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4*>(vdst + 16 * pc) = make_uint4(0, 0, 0, 0);
                 }
             }
         }
@@ -277,8 +278,9 @@ __global__ void __launch_bounds__(kAThreads) attn_piece_kernel(const __grid_cons
                 }
             }
         // the weighted V sum of dims warp * HD/4 + [0, HD/4): V^T (A) . W^T (B). The M
-        // dimension is permuted -- row g is dim 2g, row g + 8 dim 2g + 1 of the 16-dim
-        // tile -- so a thread's two dims are one 16-bit load per position
+        // dimension is permuted (vdim below gives the dim of each tile row), so that a
+        // thread's dims are one 16-bit load (one 16-dim tile) or one 32-bit load (a pair
+        // of tiles) per position
 #pragma unroll
         for (int kk = 0; kk < kSP / 16; ++kk) {
             const int pr = 16 * kk + 2 * tig;  // positions pr, pr + 1, pr + 8, pr + 9
@@ -288,26 +290,52 @@ __global__ void __launch_bounds__(kAThreads) attn_piece_kernel(const __grid_cons
                 b[j][0] = *reinterpret_cast<const uint32_t*>(wsm + (8 * j + gid) * kWPitch + pr);
                 b[j][1] = *reinterpret_cast<const uint32_t*>(wsm + (8 * j + gid) * kWPitch + pr + 8);
             }
+            if constexpr (MT % 2 == 0) {
 #pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-                const int d0 = warp * (HD / 4) + 16 * mt + 2 * gid;
-                const uint32_t x0 = *reinterpret_cast<const uint16_t*>(vs + pr * RP + d0);
-                const uint32_t x1 = *reinterpret_cast<const uint16_t*>(vs + (pr + 1) * RP + d0);
-                const uint32_t x8 = *reinterpret_cast<const uint16_t*>(vs + (pr + 8) * RP + d0);
-                const uint32_t x9 = *reinterpret_cast<const uint16_t*>(vs + (pr + 9) * RP + d0);
-                const uint32_t lo = x0 | (x1 << 16), hi = x8 | (x9 << 16);
-                // (dim d0: positions pr, pr + 1), (d0 + 1: pr, pr + 1), then pr + 8, pr + 9
-                const uint32_t a0 = e4m3x2_to_f16x2((uint16_t)__byte_perm(lo, 0, 0x0020));
-                const uint32_t a1 = e4m3x2_to_f16x2((uint16_t)__byte_perm(lo, 0, 0x0031));
-                const uint32_t a2 = e4m3x2_to_f16x2((uint16_t)__byte_perm(hi, 0, 0x0020));
-                const uint32_t a3 = e4m3x2_to_f16x2((uint16_t)__byte_perm(hi, 0, 0x0031));
+                for (int mp = 0; mp < MT / 2; ++mp) {  // tiles 2 mp, 2 mp + 1: dims d4 .. d4 + 3
+                    const int d4 = warp * (HD / 4) + 32 * mp + 4 * gid;
+                    const uint32_t y0 = *reinterpret_cast<const uint32_t*>(vs + pr * RP + d4);
+                    const uint32_t y1 = *reinterpret_cast<const uint32_t*>(vs + (pr + 1) * RP + d4);
+                    const uint32_t y8 = *reinterpret_cast<const uint32_t*>(vs + (pr + 8) * RP + d4);
+                    const uint32_t y9 = *reinterpret_cast<const uint32_t*>(vs + (pr + 9) * RP + d4);
 #pragma unroll
-                for (int j = 0; j < NT; ++j) mma_f16_16816(acc[mt][j], a0, a1, a2, a3, b[j][0], b[j][1]);
+                    for (int u = 0; u < 2; ++u) {  // dims d4 + 2u (row g), d4 + 2u + 1 (row g + 8)
+                        const uint32_t s0 = 0x0040u + 0x0022u * u, s1 = s0 + 0x0011u;
+                        const uint32_t a0 = e4m3x2_to_f16x2((uint16_t)__byte_perm(y0, y1, s0));
+                        const uint32_t a1 = e4m3x2_to_f16x2((uint16_t)__byte_perm(y0, y1, s1));
+                        const uint32_t a2 = e4m3x2_to_f16x2((uint16_t)__byte_perm(y8, y9, s0));
+                        const uint32_t a3 = e4m3x2_to_f16x2((uint16_t)__byte_perm(y8, y9, s1));
+#pragma unroll
+                        for (int j = 0; j < NT; ++j)
+                            mma_f16_16816(acc[2 * mp + u][j], a0, a1, a2, a3, b[j][0], b[j][1]);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {  // dims d0 (row g), d0 + 1 (row g + 8)
+                    const int d0 = warp * (HD / 4) + 16 * mt + 2 * gid;
+                    const uint32_t x0 = *reinterpret_cast<const uint16_t*>(vs + pr * RP + d0);
+                    const uint32_t x1 = *reinterpret_cast<const uint16_t*>(vs + (pr + 1) * RP + d0);
+                    const uint32_t x8 = *reinterpret_cast<const uint16_t*>(vs + (pr + 8) * RP + d0);
+                    const uint32_t x9 = *reinterpret_cast<const uint16_t*>(vs + (pr + 9) * RP + d0);
+                    const uint32_t lo = x0 | (x1 << 16), hi = x8 | (x9 << 16);
+                    const uint32_t a0 = e4m3x2_to_f16x2((uint16_t)__byte_perm(lo, 0, 0x0020));
+                    const uint32_t a1 = e4m3x2_to_f16x2((uint16_t)__byte_perm(lo, 0, 0x0031));
+                    const uint32_t a2 = e4m3x2_to_f16x2((uint16_t)__byte_perm(hi, 0, 0x0020));
+                    const uint32_t a3 = e4m3x2_to_f16x2((uint16_t)__byte_perm(hi, 0, 0x0031));
+#pragma unroll
+                    for (int j = 0; j < NT; ++j) mma_f16_16816(acc[mt][j], a0, a1, a2, a3, b[j][0], b[j][1]);
+                }
             }
         }
     }
 
-    // this CTA's partials: (max, sum) per head, then its dims of the weighted V sums
+    // this CTA's partials: (max, sum) per head, then its dims of the weighted V sums; tile
+    // mt's row g holds dim vdim(mt), row g + 8 dim vdim(mt) + 1
+    auto vdim = [&](int mt) {
+        return MT % 2 == 0 ? warp * (HD / 4) + 32 * (mt / 2) + 4 * gid + 2 * (mt % 2)
+                           : warp * (HD / 4) + 16 * mt + 2 * gid;
+    };
     const int64_t rs = (int64_t)HD + 2;
 #pragma unroll
     for (int j = 0; j < NT; ++j)
@@ -322,7 +350,7 @@ __global__ void __launch_bounds__(kAThreads) attn_piece_kernel(const __grid_cons
             }
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
-                const int d0 = warp * (HD / 4) + 16 * mt + 2 * gid;
+                const int d0 = vdim(mt);
                 dst[2 + d0] = acc[mt][j][e];
                 dst[2 + d0 + 1] = acc[mt][j][2 + e];
             }
@@ -331,55 +359,64 @@ __global__ void __launch_bounds__(kAThreads) attn_piece_kernel(const __grid_cons
 
 // One CTA per query head: out = sum_s e^(m_s - M) acc_s / sum_s e^(m_s - M) l_s (zero
 // when no row was readable), as bf16. The pieces' (max, sum) pairs are loaded in parallel
-// and their factors folded in a fixed order; each thread then sums its dimension over the
-// pieces with many loads in flight.
+// and folded from shared memory in a fixed order; the dimensions' sums over the pieces
+// are split over 256 / hd thread groups (eight loads in flight each) and added in order.
 __global__ void __launch_bounds__(kAMaxHd) attn_merge_kernel(const __grid_constant__ AttnParams p) {
+    __shared__ float msm[kAMaxPieces];
+    __shared__ float lsm[kAMaxPieces];
     __shared__ float fac[kAMaxPieces];
+    __shared__ float accp[kAMaxHd];  // [parts][hd]
     __shared__ float red[kAMaxHd / 32];
     __shared__ float tot[2];
-    const int i = blockIdx.x, d = threadIdx.x, hd = p.hd;
-    const int lane = d & 31, warp = d >> 5;
+    const int i = blockIdx.x, t = threadIdx.x, hd = p.hd;
+    const int lane = t & 31, warp = t >> 5;
+    const int parts = kAMaxHd / hd, d = t % hd, part = t / hd;  // 1, 2 or 4 parts of the pieces
     pdl_wait();
     const int64_t rs = (int64_t)p.nq * (hd + 2);  // floats between a head's pieces
     const float* base = p.part + (int64_t)i * (hd + 2);
     float mloc = -INFINITY;
-    for (int s = d; s < p.pieces; s += kAMaxHd) mloc = fmaxf(mloc, base[s * rs]);
+    for (int s = t; s < p.pieces; s += kAMaxHd) {
+        msm[s] = base[s * rs];
+        lsm[s] = base[s * rs + 1];
+        mloc = fmaxf(mloc, msm[s]);
+    }
 #pragma unroll
     for (int o = 16; o; o >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, o));
     if (lane == 0) red[warp] = mloc;
     __syncthreads();
-    if (d == 0) {
-        float M = -INFINITY;
-        for (int w = 0; w < kAMaxHd / 32; ++w) M = fmaxf(M, red[w]);
-        tot[0] = M;
-    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kAMaxHd / 32; ++w) M = fmaxf(M, red[w]);
+    for (int s = t; s < p.pieces; s += kAMaxHd)
+        fac[s] = (M == -INFINITY || msm[s] == -INFINITY) ? 0.f : expf(msm[s] - M);
     __syncthreads();
-    const float M = tot[0];
-    for (int s = d; s < p.pieces; s += kAMaxHd) {
-        const float m = base[s * rs];
-        fac[s] = (M == -INFINITY || m == -INFINITY) ? 0.f : expf(m - M);
-    }
-    __syncthreads();
-    if (d == 0) {  // the denominator in piece order
+    if (warp == 0) {  // the denominator: lane-strided partial sums, then a fixed shuffle tree
         float L = 0.f;
-        for (int s = 0; s < p.pieces; ++s) L = fmaf(fac[s], base[s * rs + 1], L);
-        tot[1] = L;
+        for (int s = lane; s < p.pieces; s += 32) L = fmaf(fac[s], lsm[s], L);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        if (lane == 0) tot[1] = L;
     }
+    // the weighted V sums: thread (part, d) takes pieces part, part + parts, ..., eight
+    // loads in flight at a time; the parts are added in order afterwards
     float a = 0.f;
-    if (d < hd) {
-        int s = 0;
-        for (; s + 8 <= p.pieces; s += 8) {  // eight independent loads in flight
-            float v[8];
+    int s = part;
+    for (; s + 7 * parts < p.pieces; s += 8 * parts) {
+        float v[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) v[j] = base[(s + j) * rs + 2 + d];
+        for (int j = 0; j < 8; ++j) v[j] = base[(s + j * parts) * rs + 2 + d];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) a = fmaf(fac[s + j], v[j], a);
-        }
-        for (; s < p.pieces; ++s) a = fmaf(fac[s], base[s * rs + 2 + d], a);
+        for (int j = 0; j < 8; ++j) a = fmaf(fac[s + j * parts], v[j], a);
     }
+    for (; s < p.pieces; s += parts) a = fmaf(fac[s], base[s * rs + 2 + d], a);
+    accp[part * hd + d] = a;
     __syncthreads();
-    const float L = tot[1];
-    if (d < hd) p.out[(int64_t)i * hd + d] = f32_to_bf16(L > 0.f ? a / L * p.v_scale : 0.f);
+    if (part == 0) {
+        float sum = accp[d];
+        for (int q = 1; q < parts; ++q) sum += accp[q * hd + d];
+        const float L = tot[1];
+        p.out[(int64_t)i * hd + d] = f32_to_bf16(L > 0.f ? sum / L * p.v_scale : 0.f);
+    }
 }
 
 }  // namespace
