@@ -16,31 +16,39 @@
 //
 // Design (B200): rows are processed in chunks (the reference's PREFILL_CHUNK), whose
 // buffers (concat rows, fc output, RoPE table) live in the caller's workspace. The whole
-// call is ONE persistent kernel on the caller's stream: every CTA takes work items
-// ("tiles") from two counters, each in a fixed global order, so that the tiles of the
-// next chunk fill the SMs the current chunk leaves idle (a 2,048-row chunk's fc GEMM is
-// 320 output tiles, 2.16 waves on 148 SMs). Three kinds of tile:
+// call is ONE persistent kernel on the caller's stream, launched as CTA pairs (2-CTA
+// clusters, one CTA per SM): the pairs take GEMM work items ("tiles") from one counter and
+// every CTA's prologue warps take prologue tiles from another, each in a fixed global
+// order, so that the tiles of the next chunk fill the SMs the current chunk leaves idle (a
+// 2,048-row chunk's fc GEMM is 160 pair tiles, 2.16 waves on 74 pairs). Three kinds of
+// tile:
 //   P (chunk c, row block m, part n): the prologue of 8 rows, taken from its own counter
 //     by each CTA's two prologue warps whenever they are free: they read each row's
 //     embedding row and hidden row into registers, take the two RMSNorms, write the
 //     bf16 concat rows and the rows' RoPE table (the angle reduced in double, cos and
 //     sin in fp32), alongside the GEMM tiles, whose shared-memory ring they never use.
-//   F (c, m, n): a 128 x 256 tile of the fc GEMM, y = c . fc^T, bf16 out.
-//   V (c, m, n): a 128 x 256 tile of the k/v GEMM whose epilogue rotates k (RoPE),
+//   F (c, m, n): a 256 x 256 tile of the fc GEMM, y = c . fc^T, bf16 out (rows 256 m ..;
+//     the pair's CTA r holds row block 2 m + r).
+//   V (c, m, n): a 256 x 256 tile of the k/v GEMM whose epilogue rotates k (RoPE),
 //     encodes E4M3 and writes each row's 32-byte pieces at its paged slot.
 // GEMM order: for b = 0..chunks: F(b), then V(b - 1) (with a single lane V(b - 1) first).
-// Completion counters per chunk slot and row block (in the workspace header,
-// release/acquire at GPU scope) order the tiles: F(c, m, .) waits for P(c, m, .);
+// Completion counters per chunk slot and 128-row block (in the workspace header,
+// release/acquire at GPU scope; each CTA of a pair waits for and counts its own block)
+// order the tiles: F(c, m, .) waits for P(c, m, .);
 // V(c, m, .) for all of F(c, m, .); and a tile that overwrites a buffer another chunk
 // used (two lanes of concat and fc-output rows, three of RoPE rows) for that chunk's
 // readers. A GEMM tile only waits for GEMM tiles earlier in its order and for P tiles; a
 // P tile only for GEMM tiles of chunks two and three back, whose own P tiles were taken
 // earlier from the P counter. Tiles are claimed only by running CTAs, so every wait
-// ends. GEMM tiles run on the 5th-generation tensor cores: a 4-stage TMA ring
-// (128-byte swizzle, K-major A and B), tcgen05.mma from one thread into a double-
-// buffered 512-column TMEM accumulator, four epilogue warps reading it back with
-// tcgen05.ld while the next tile accumulates. A small FIFO in shared memory tells the
-// MMA and epilogue warps which tile comes next. Every wait is bounded (abort flag +
+// ends (every pair of the grid is resident at once). GEMM tiles run on the 5th-generation
+// tensor cores as cta_group::2 MMAs of 256 x 256 x 16: each CTA's 6-stage TMA ring (128-byte
+// swizzle, K-major) holds its 128 rows of A and 128 of the tile's 256 B rows, so each SM
+// stages and reads half the B it would alone; both CTAs' copies complete on rank 0's
+// barrier, rank 0's thread issues the MMAs into both SMs' double-buffered 512-column
+// TMEM accumulators and its commits free both CTAs' stages; each CTA's four epilogue
+// warps read back its own 128 rows with tcgen05.ld while the next tile accumulates. Rank
+// 0 announces each tile to both CTAs through a small FIFO in each one's shared memory
+// (remote stores and mbarrier arrivals). Every wait is bounded (abort flag +
 // MTP_DEVFLAG_TIMEOUT): nothing hangs.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -55,10 +63,14 @@
 namespace mtp {
 namespace {
 
+// A GEMM tile is 256 rows x BN columns, computed by a CTA pair (a 2-CTA cluster on one
+// TPC) with cta_group::2 MMAs of M = 256: each CTA stages its own 128 rows of A and half
+// of the tile's B rows, and holds its 128 rows x BN of the accumulator.
 constexpr int BM = 128, BN = 256, BK = 64;
-constexpr int kGStages = 4;
-constexpr int kAStageBytes = BM * BK * 2;  // 16 KB
-constexpr int kBStageBytes = BN * BK * 2;  // 32 KB
+constexpr int BNH = BN / 2;                 // B rows each CTA of the pair stages
+constexpr int kGStages = 6;
+constexpr int kAStageBytes = BM * BK * 2;   // 16 KB
+constexpr int kBStageBytes = BNH * BK * 2;  // 16 KB
 constexpr int kGStageBytes = kAStageBytes + kBStageBytes;
 // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue, warps 6-7 prologue
 constexpr int kGemmThreads = 256;
@@ -114,6 +126,8 @@ struct PrefillParams {
     int n_chunks;
     int mt_full;         // 128-row blocks of a full chunk
     int mt_last;         // of the last chunk
+    int mp_full;         // 256-row pair blocks (GEMM tile rows) of a full chunk
+    int mp_last;         // of the last chunk
     int nf;              // fc GEMM column tiles (h / 256)
     int nv;              // k/v GEMM column tiles (2 nkv hd / 256)
     int64_t total;       // GEMM tiles (the tile counter's range)
@@ -130,6 +144,8 @@ struct PrefillParams {
     int M, N, K;
 };
 
+// kind, chunk, rows, column tile. m is a pair block (rows 256 m ..) for GEMM tiles, whose
+// two 128-row blocks 2 m + r are those of the pair's CTA r; a 128-row block for P tiles.
 struct Tile {
     int kind, c, m, n;
 };
@@ -137,30 +153,38 @@ struct Tile {
 __device__ __forceinline__ int mt_of(const PrefillParams& p, int c) {
     return c == p.n_chunks - 1 ? p.mt_last : p.mt_full;
 }
+__device__ __forceinline__ int mp_of(const PrefillParams& p, int c) {
+    return c == p.n_chunks - 1 ? p.mp_last : p.mp_full;
+}
 
-// Row blocks of chunks 0 .. k - 1.
+// Row blocks (pair blocks) of chunks 0 .. k - 1.
 __device__ __forceinline__ int64_t cum_mt(const PrefillParams& p, int k) {
     k = max(0, min(k, p.n_chunks));
     return k <= p.n_chunks - 1 ? (int64_t)k * p.mt_full
                                : (int64_t)(p.n_chunks - 1) * p.mt_full + p.mt_last;
+}
+__device__ __forceinline__ int64_t cum_mp(const PrefillParams& p, int k) {
+    k = max(0, min(k, p.n_chunks));
+    return k <= p.n_chunks - 1 ? (int64_t)k * p.mp_full
+                               : (int64_t)(p.n_chunks - 1) * p.mp_full + p.mp_last;
 }
 
 // First GEMM tile of block b (b = 0 .. n_chunks + 1). With two lanes block b holds F(b),
 // then V(b - 1); with one lane V(b - 1), then F(b), since F(b) then reuses the fc-output
 // rows V(b - 1) reads.
 __device__ __forceinline__ int64_t block_start(const PrefillParams& p, int b) {
-    return p.nf * cum_mt(p, b) + p.nv * cum_mt(p, b - 1);
+    return p.nf * cum_mp(p, b) + p.nv * cum_mp(p, b - 1);
 }
 
 // GEMM tile t of the global order.
 __device__ Tile decode(const PrefillParams& p, int64_t t) {
     Tile r{};
     if (p.plain) {  // F tiles of one GEMM, M-fastest
-        const int mt = (p.M + BM - 1) / BM;
+        const int mp = (p.M + 2 * BM - 1) / (2 * BM);
         r.kind = TILE_F;
         r.c = 0;
-        r.m = (int)(t % mt);
-        r.n = (int)(t / mt);
+        r.m = (int)(t % mp);
+        r.n = (int)(t / mp);
         return r;
     }
     int lo = 0, hi = p.n_chunks;  // the last block starting at or before t
@@ -175,13 +199,13 @@ __device__ Tile decode(const PrefillParams& p, int64_t t) {
     bool found = false;
     auto seg = [&](int kind, int c) {
         if (found) return;
-        const int mt = mt_of(p, c);
-        const int64_t cnt = (int64_t)mt * (kind == TILE_F ? p.nf : p.nv);
+        const int mp = mp_of(p, c);
+        const int64_t cnt = (int64_t)mp * (kind == TILE_F ? p.nf : p.nv);
         if (off < cnt) {  // M-fastest
             r.kind = kind;
             r.c = c;
-            r.m = (int)(off % mt);
-            r.n = (int)(off / mt);
+            r.m = (int)(off % mp);
+            r.n = (int)(off / mp);
             found = true;
         } else {
             off -= cnt;
@@ -403,7 +427,7 @@ struct Maps {
     CUtensorMap b_wk, b_wv;
 };
 
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ Maps maps) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -415,7 +439,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint64_t* tempty = tfull + 2;          // [2]
     uint64_t* done = tempty + 2;           // MMA drain at exit
     uint64_t* qfull = done + 1;            // [kFifo] a tile index is in the FIFO slot
-    uint64_t* qempty = qfull + kFifo;      // [kFifo] both readers took it
+    uint64_t* qempty = qfull + kFifo;      // [kFifo] every reader took it
     int* fifo = reinterpret_cast<int*>(qempty + kFifo);          // [kFifo]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fifo + kFifo);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -426,27 +450,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int kvd = p.nkv * p.hd;
+    // The pair: rank 0 claims the GEMM tiles, announces each to both CTAs, and issues the
+    // MMAs; both CTAs stage their operands and run their own epilogue and prologue warps.
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    const int pair = (int)(blockIdx.x >> 1), npairs = (int)(gridDim.x >> 1);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kGStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&full[s], 1);   // rank 0's: its expect_tx; both CTAs' copies count on it
+            mbar_init(&empty[s], 1);  // the MMA commit, to both CTAs
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 1);  // one epilogue thread, after the epilogue warps sync
+            mbar_init(&tfull[b], 1);   // the MMA commit, to both CTAs
+            mbar_init(&tempty[b], 2);  // rank 0's: one epilogue thread of each CTA
         }
         for (int q = 0; q < kFifo; ++q) {
             mbar_init(&qfull[q], 1);
-            mbar_init(&qempty[q], 2);  // the MMA warp and the epilogue warps
+            mbar_init(&qempty[q], 4);  // rank 0's: its MMA and epilogue warps, rank 1's
+                                       // producer and epilogue warps
         }
         mbar_init(done, 1);
         *abort_flag = 0;
         mbar_fence_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, kTmemCols);
-        tmem_relinquish();
+        tmem_alloc_pair(tmem_slot, kTmemCols);
+        tmem_relinquish_pair();
     }
     const int half = p.hd / 2;
     if (!p.plain) {  // the rotation per position of each pair, in turns; norm weights
@@ -465,69 +495,96 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();  // both CTAs' barriers initialised, the pair's TMEM allocated
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    // stages of a tile in the ring: a GEMM tile's K blocks, or a P tile's row groups
+    // stages of a tile in the ring: a GEMM tile's K blocks
     auto tile_stages = [&](const Tile& tl) -> int {
-        if (tl.kind == TILE_P) return 0;  // read by the epilogue warps, not through the ring
         if (p.plain) return p.K / BK;
         return (tl.kind == TILE_F ? 2 * p.h : p.h) / BK;
     };
+    // this CTA's 128-row block of GEMM tile tl, and whether the chunk has it (the last pair
+    // block of a chunk with an odd number of row blocks has only rank 0's)
+    auto own_block = [&](const Tile& tl) -> int { return 2 * tl.m + (int)rank; };
+    auto has_block = [&](const Tile& tl) -> bool {
+        return own_block(tl) < (p.plain ? (p.M + BM - 1) / BM : mt_of(p, tl.c));
+    };
 
     if (warp == 0) {
-        // ---------------- producer: claims tiles, announces them, streams their stages
+        // ---------------- producer: (rank 0) claims tiles and announces them; both stage
+        // their operands
         int s = 0;
         uint32_t ph = 0;
         int q = 0;
         uint32_t qph = 0;
         int64_t issued = 0;
         bool stop = false;
-        // the plain GEMM (no dependencies) takes tiles b, b + grid, ...; the prefill claims
-        // every tile from the counter, so a claimed tile always belongs to a running CTA
-        int64_t t = blockIdx.x;
-        if (!p.plain && lane == 0) t = atomicAdd(p.ctr, 1u);
+        // the plain GEMM (no dependencies) takes tiles pair, pair + pairs, ...; the prefill
+        // claims every tile from the counter, so a claimed tile always belongs to a running
+        // pair
+        int64_t t = pair;
+        if (leader && !p.plain && lane == 0) t = atomicAdd(p.ctr, 1u);
         t = __shfl_sync(0xffffffffu, t, 0);
         while (!stop) {
-            const bool end = t >= p.total;
-            // announce the tile (or the end) to the MMA and epilogue warps
-            if (!mbar_wait_bounded(&qempty[q], qph ^ 1u, abort_flag)) break;
-            if (lane == 0) {
-                fifo[q] = end ? -1 : (int)t;
-                mbar_arrive(&qfull[q]);
+            bool end;
+            if (leader) {
+                // announce the tile (or the end) to both CTAs' readers
+                end = t >= p.total;
+                if (!mbar_wait_cluster_bounded(&qempty[q], qph ^ 1u, abort_flag)) break;
+                if (lane == 0) {
+                    const int v = end ? -1 : (int)t;
+                    fifo[q] = v;
+                    st_cluster_u32(map_rank(&fifo[q], 1), (uint32_t)v);
+                    mbar_arrive(&qfull[q]);
+                    mbar_arrive_cluster(map_rank(&qfull[q], 1));
+                }
+                __syncwarp();
+            } else {
+                // the tile rank 0 announced
+                if (!mbar_wait_cluster_bounded(&qfull[q], qph, abort_flag)) break;
+                const int v = fifo[q];
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(map_rank(&qempty[q], 0));
+                end = v < 0;
+                t = v;
             }
-            __syncwarp();
             if (++q == kFifo) {
                 q = 0;
                 qph ^= 1u;
             }
             if (end) break;
             const Tile tl = decode(p, t);
-            int64_t tn = t + gridDim.x;  // the next claim, issued early
-            if (!p.plain && lane == 0) tn = atomicAdd(p.ctr, 1u);
+            const int m = own_block(tl);
+            const bool has = has_block(tl);
+            int64_t tn = t + npairs;  // rank 0's next claim, issued early
+            if (leader && !p.plain && lane == 0) tn = atomicAdd(p.ctr, 1u);
             const int nst = tile_stages(tl);
             {
                 // operands: F reads the chunk's concat rows, V its fc output rows; each only
-                // once the tiles that write them are done
+                // once the tiles that write them are done. A block the chunk lacks stages
+                // rank 0's rows instead (its products are never stored).
                 const CUtensorMap* ma;
                 const CUtensorMap* mb;
-                int brow = tl.n * BN;
+                const int arow = (has ? m : m - 1) * BM;
+                int brow = tl.n * BN + (int)rank * BNH;
                 if (p.plain) {
                     ma = &maps.a_concat[0];
                     mb = &maps.b_fc;
                 } else if (tl.kind == TILE_F) {
                     ma = &maps.a_concat[tl.c % p.lanes];
                     mb = &maps.b_fc;
-                    if (lane == 0 && !wait_counter(counter(p, TILE_P, tl.c, tl.m),
-                                                   (uint32_t)((tl.c / kCtrSlots + 1) * kPParts), abort_flag))
+                    if (has && lane == 0 &&
+                        !wait_counter(counter(p, TILE_P, tl.c, m),
+                                      (uint32_t)((tl.c / kCtrSlots + 1) * kPParts), abort_flag))
                         stop = true;
                 } else {
                     ma = &maps.a_y[tl.c % p.lanes];
                     mb = brow < kvd ? &maps.b_wk : &maps.b_wv;
                     if (brow >= kvd) brow -= kvd;
-                    if (lane == 0 && !wait_counter(counter(p, TILE_F, tl.c, tl.m),
-                                                   (uint32_t)((tl.c / kCtrSlots + 1) * p.nf), abort_flag))
+                    if (has && lane == 0 &&
+                        !wait_counter(counter(p, TILE_F, tl.c, m),
+                                      (uint32_t)((tl.c / kCtrSlots + 1) * p.nf), abort_flag))
                         stop = true;
                 }
                 stop = __shfl_sync(0xffffffffu, (int)stop, 0) != 0;
@@ -539,9 +596,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                     if (lane == 0) {
                         uint8_t* st = stages + (size_t)s * kGStageBytes;
-                        mbar_arrive_expect_tx(&full[s], kGStageBytes);
-                        tma_load_2d_g(st, ma, kb * BK, tl.m * BM, &full[s]);
-                        tma_load_2d_g(st + kAStageBytes, mb, kb * BK, brow, &full[s]);
+                        const uint32_t fb = map_rank(&full[s], 0);
+                        if (leader) mbar_arrive_expect_tx(&full[s], 2 * kGStageBytes);
+                        tma_load_2d_pair(st, ma, kb * BK, arow, fb);
+                        tma_load_2d_pair(st + kAStageBytes, mb, kb * BK, brow, fb);
                     }
                     __syncwarp();
                     ++issued;
@@ -553,24 +611,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             t = __shfl_sync(0xffffffffu, tn, 0);
         }
-        // no copy left in flight
-        for (int64_t j = issued > kGStages ? issued - kGStages : 0; j < issued; ++j)
-            if (!mbar_wait_bounded(&full[j % kGStages], (uint32_t)((j / kGStages) & 1), nullptr)) break;
-        // if the loop stopped early, still tell the readers that no tile follows
-        if (stop && mbar_wait_bounded(&qempty[q], qph ^ 1u, nullptr) && lane == 0) {
+        // no copy left in flight: rank 0's full barriers count both CTAs' copies; rank 1's
+        // stages are free once the MMAs that read them completed
+        for (int64_t j = issued > kGStages ? issued - kGStages : 0; j < issued; ++j) {
+            const uint32_t par = (uint32_t)((j / kGStages) & 1);
+            if (!mbar_wait_bounded(leader ? &full[j % kGStages] : &empty[j % kGStages], par, nullptr))
+                break;
+        }
+        // if rank 0 stopped early, still tell every reader that no tile follows
+        if (leader && stop && mbar_wait_cluster_bounded(&qempty[q], qph ^ 1u, nullptr) && lane == 0) {
             fifo[q] = -1;
+            st_cluster_u32(map_rank(&fifo[q], 1), 0xFFFFFFFFu);
             mbar_arrive(&qfull[q]);
+            mbar_arrive_cluster(map_rank(&qfull[q], 1));
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------- MMA issuer (one thread)
-        constexpr uint32_t idesc = idesc_bf16(BM, BN);
+        // ---------------- MMA issuer: one thread of rank 0, for the pair
+        constexpr uint32_t idesc = idesc_bf16(2 * BM, BN);
         int s = 0;
         uint32_t ph = 0;
         int q = 0;
         uint32_t qph = 0;
         int local = 0;
-        bool stop = false;
+        bool stop = !leader;
         while (!stop) {
             if (!mbar_wait_bounded(&qfull[q], qph, abort_flag)) break;
             const int t = fifo[q];
@@ -585,7 +649,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int nst = tile_stages(tl);
             const int buf = local & 1;
             const uint32_t tph = (uint32_t)((local >> 1) & 1);
-            if (!mbar_wait_bounded(&tempty[buf], tph ^ 1u, abort_flag)) break;
+            // both CTAs' epilogues have read this accumulator's previous tile
+            if (!mbar_wait_cluster_bounded(&tempty[buf], tph ^ 1u, abort_flag)) break;
             tc_fence_after();
             const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
             for (int kb = 0; kb < nst; ++kb) {
@@ -599,9 +664,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const uint32_t b0 = a0 + kAStageBytes;
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k)
-                        umma_bf16(d_tmem, sdesc_k128(a0 + k * 32), sdesc_k128(b0 + k * 32), idesc,
-                                  (kb > 0 || k > 0) ? 1u : 0u);
-                    umma_commit(&empty[s]);  // frees the stage once these MMAs have read it
+                        umma_bf16_pair(d_tmem, sdesc_k128(a0 + k * 32), sdesc_k128(b0 + k * 32), idesc,
+                                       (kb > 0 || k > 0) ? 1u : 0u);
+                    umma_commit_pair(&empty[s], 3);  // frees both CTAs' stage once read
                 }
                 __syncwarp();
                 if (++s == kGStages) {
@@ -609,62 +674,62 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     ph ^= 1u;
                 }
             }
-            if (lane == 0) umma_commit(&tfull[buf]);  // accumulator ready for the epilogue
+            if (lane == 0) umma_commit_pair(&tfull[buf], 3);  // both accumulators ready
             __syncwarp();
             ++local;
         }
-        // every MMA this thread issued has completed before TMEM is released
-        if (lane == 0) umma_commit(done);
-        __syncwarp();
-        mbar_wait_bounded(done, 0u, nullptr);
+        if (leader) {
+            // every MMA this thread issued has completed before TMEM is released
+            if (lane == 0) umma_commit_pair(done, 1);
+            __syncwarp();
+            mbar_wait_bounded(done, 0u, nullptr);
+        }
     } else if (warp < 6) {
         // ---------------- epilogue warps 2..5: TMEM lane quarter = warp % 4
         const int qd = warp & 3;
         const int et = threadIdx.x - 64;  // 0..127
         const int ew = et >> 5;
-        int s = 0;
-        uint32_t ph = 0;
         int q = 0;
         uint32_t qph = 0;
         int local = 0;
         while (true) {
-            if (!mbar_wait_bounded(&qfull[q], qph, abort_flag)) break;
+            if (!mbar_wait_cluster_bounded(&qfull[q], qph, abort_flag)) break;
             const int t = fifo[q];
             named_sync(1, kEpiThreads);  // every epilogue thread has read the slot
-            if (et == 0) mbar_arrive(&qempty[q]);
+            if (et == 0) {
+                if (leader) mbar_arrive(&qempty[q]);
+                else mbar_arrive_cluster(map_rank(&qempty[q], 0));
+            }
             if (++q == kFifo) {
                 q = 0;
                 qph ^= 1u;
             }
             if (t < 0) break;
             const Tile tl = decode(p, t);
-            const int nst = tile_stages(tl);
+            const int m = own_block(tl);
+            const bool has = !p.plain && has_block(tl);  // its counters exist
             const int64_t crow0 = (int64_t)tl.c * p.chunk;  // prompt row of the chunk's row 0
             const int64_t rows_c = p.plain ? p.M : min(p.chunk, p.R - crow0);
-            // ---- GEMM tile: its stages are the MMA warp's
-            s += nst;
-            ph ^= (uint32_t)((s / kGStages) & 1);
-            s %= kGStages;
             const int buf = local & 1;
             const uint32_t tph = (uint32_t)((local >> 1) & 1);
             ++local;
             bool ok = mbar_wait_bounded(&tfull[buf], tph, abort_flag);
             // F writes the chunk lane's fc output rows: free once the chunk that used the
             // lane before has run its k/v tiles of these rows; V reads the RoPE rows
-            if (et == 0 && ok && !p.plain) {
+            if (et == 0 && ok && has) {
                 if (tl.kind == TILE_F && tl.c >= p.lanes) {
                     const int ca = tl.c - p.lanes;
-                    ok = wait_counter(counter(p, TILE_V, ca, tl.m),
+                    ok = wait_counter(counter(p, TILE_V, ca, m),
                                       (uint32_t)((ca / kCtrSlots + 1) * p.nv), abort_flag);
                 } else if (tl.kind == TILE_V) {
-                    ok = wait_counter(counter(p, TILE_P, tl.c, tl.m),
+                    ok = wait_counter(counter(p, TILE_P, tl.c, m),
                                       (uint32_t)((tl.c / kCtrSlots + 1) * kPParts), abort_flag);
                 }
             }
             named_sync(1, kEpiThreads);
             ok = ok && !*abort_flag;
             tc_fence_after();
-            const int row = tl.m * BM + qd * 32 + lane;  // row of the chunk (of A)
+            const int row = m * BM + qd * 32 + lane;  // row of the chunk (of A)
             const bool row_ok = ok && row < rows_c;
             const uint32_t tb = tmem_base + ((uint32_t)(qd * 32) << 16) + (uint32_t)(buf * BN);
             if (tl.kind == TILE_F) {
@@ -749,16 +814,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             tc_fence_before();
             named_sync(1, kEpiThreads);  // the accumulator is read, every store issued
-            const bool norm_y = tl.kind == TILE_F && !p.plain && p.in_norm != nullptr;
+            const bool norm_y = tl.kind == TILE_F && has && p.in_norm != nullptr;
             if (et == 0) {
-                mbar_arrive(&tempty[buf]);
-                if (!p.plain && !*abort_flag && !norm_y)
-                    counter_release_add(counter(p, tl.kind, tl.c, tl.m), 1u);
+                if (leader) mbar_arrive(&tempty[buf]);
+                else mbar_arrive_cluster(map_rank(&tempty[buf], 0));
+                if (has && !*abort_flag && !norm_y)
+                    counter_release_add(counter(p, tl.kind, tl.c, m), 1u);
                 if (norm_y) {
                     int last = 0;
                     if (!*abort_flag) {
                         fence_acq_rel_gpu();  // release this tile's y stores
-                        const uint32_t old = atomicAdd(counter(p, kArrivals, tl.c, tl.m), 1u);
+                        const uint32_t old = atomicAdd(counter(p, kArrivals, tl.c, m), 1u);
                         last = old + 1u == (uint32_t)((tl.c / kCtrSlots + 1) * p.nf);
                         fence_acq_rel_gpu();  // acquire the other tiles' stores
                     }
@@ -772,11 +838,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     // rows were written by other SMs)
                     uint16_t* Y = p.y[tl.c % p.lanes];
                     const int h = p.h, pieces = h / 8;
-                    const int nrow = (int)min((int64_t)BM, rows_c - (int64_t)tl.m * BM);
+                    const int nrow = (int)min((int64_t)BM, rows_c - (int64_t)m * BM);
                     const uint64_t wadd = f32x2_splat(p.norm_mode ? 1.f : 0.f);
                     const uint4* wn = p.w_in_smem ? w_s + 2 * pieces : reinterpret_cast<const uint4*>(p.in_norm);
                     for (int r = ew; r < nrow; r += kEpiThreads / 32) {
-                        uint4* yr = reinterpret_cast<uint4*>(Y + ((int64_t)tl.m * BM + r) * h);
+                        uint4* yr = reinterpret_cast<uint4*>(Y + ((int64_t)m * BM + r) * h);
                         uint64_t ss2 = 0;
 #pragma unroll 4
                         for (int j = lane; j < pieces; j += 32) ss2 = sumsq8(__ldcg(yr + j), ss2);
@@ -790,7 +856,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                     fence_proxy_async_global();  // read by the k/v tiles' TMA
                     named_sync(1, kEpiThreads);
-                    if (et == 0) counter_release_add(counter(p, TILE_F, tl.c, tl.m), (uint32_t)p.nf);
+                    if (et == 0) counter_release_add(counter(p, TILE_F, tl.c, m), (uint32_t)p.nf);
                 }
             }
         }
@@ -867,11 +933,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
         }
     }
-    __syncthreads();
+    tc_fence_before();
+    cluster_sync();  // neither CTA leaves while an MMA, a copy or an arrival may reach it
     if (*abort_flag && threadIdx.x == 0) raise_flag(p.dev_err, DEVFLAG_TIMEOUT);
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, kTmemCols);
+        tmem_dealloc_pair(tmem_base, kTmemCols);
     }
 }
 
@@ -941,6 +1008,41 @@ int weight_smem_bytes(const PrefillParams& p) {
     return p.plain ? 0 : (p.in_norm ? 3 : 2) * 2 * p.h;
 }
 
+// CTA pairs that can be resident at once with `smem` bytes each (every SM pair of a TPC
+// whose two SMs are both available), per device and size.
+cudaError_t resident_pairs(int dev, int smem, int* out) {
+    static std::mutex mu;
+    static int cached[64][2] = {};  // [device] {smem, pairs}
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev >= 0 && dev < 64 && cached[dev][0] == smem && cached[dev][1] > 0) {
+        *out = cached[dev][1];
+        return cudaSuccess;
+    }
+    int sms = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)(sms & ~1), 1, 1);
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if ((e = cudaOccupancyMaxActiveClusters(&n, prefill_kernel, &cfg)) != cudaSuccess) return e;
+    if (n < 1) return cudaErrorInvalidConfiguration;
+    if (dev >= 0 && dev < 64) {
+        cached[dev][0] = smem;
+        cached[dev][1] = n;
+    }
+    *out = n;
+    return cudaSuccess;
+}
+
 cudaError_t launch(PrefillParams p, const Maps& maps, cudaStream_t s) {
     if (p.total < 1) return cudaSuccess;
     const int wb = weight_smem_bytes(p);
@@ -949,13 +1051,14 @@ cudaError_t launch(PrefillParams p, const Maps& maps, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          smem);
     if (e != cudaSuccess) return e;
-    int dev = 0, sms = 148;
+    int dev = 0, pairs = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-        return e;
-    int64_t grid = sms;
+    if ((e = resident_pairs(dev, smem, &pairs)) != cudaSuccess) return e;
+    // every pair is resident at once: a tile claimed from the counter always belongs to a
+    // running pair, so every wait on another tile ends
+    int64_t grid = pairs;
     if (grid > p.total) grid = p.total;
-    prefill_kernel<<<(unsigned)grid, kGemmThreads, smem, s>>>(p, maps);
+    prefill_kernel<<<(unsigned)(2 * grid), kGemmThreads, smem, s>>>(p, maps);
     return cudaGetLastError();
 }
 
@@ -1028,6 +1131,8 @@ cudaError_t prefill_launch(const PrefillArgs& a, cudaStream_t s) {
     p.mt_full = (int)((a.chunk_rows + BM - 1) / BM);
     const int64_t last_rows = a.R - (int64_t)(p.n_chunks - 1) * a.chunk_rows;
     p.mt_last = (int)((last_rows + BM - 1) / BM);
+    p.mp_full = (p.mt_full + 1) / 2;
+    p.mp_last = (p.mt_last + 1) / 2;
     p.nf = a.h / BN;
     p.nv = 2 * kvd / BN;
     p.lanes = (a.R > a.chunk_rows && a.ws_bytes >= prefill_ws_bytes_lanes(a.chunk_rows, a.h, a.hd, 2))
@@ -1036,7 +1141,8 @@ cudaError_t prefill_launch(const PrefillArgs& a, cudaStream_t s) {
     p.p_total = 0;
     for (int c = 0; c < p.n_chunks; ++c) {
         const int mt = c == p.n_chunks - 1 ? p.mt_last : p.mt_full;
-        p.total += (int64_t)mt * (p.nf + p.nv);
+        const int mp = c == p.n_chunks - 1 ? p.mp_last : p.mp_full;
+        p.total += (int64_t)mp * (p.nf + p.nv);
         p.p_total += (int64_t)mt * kPParts;
     }
     if (a.hd / 2 > 128) return cudaErrorInvalidValue;
@@ -1062,9 +1168,9 @@ cudaError_t prefill_launch(const PrefillArgs& a, cudaStream_t s) {
             return e;
         if ((e = make_operand_map(&maps.a_y[l], p.y[l], a.chunk_rows, a.h, BM)) != cudaSuccess) return e;
     }
-    if ((e = make_operand_map(&maps.b_fc, a.fc, a.h, 2 * (int64_t)a.h, BN)) != cudaSuccess) return e;
-    if ((e = make_operand_map(&maps.b_wk, a.wk, kvd, a.h, BN)) != cudaSuccess) return e;
-    if ((e = make_operand_map(&maps.b_wv, a.wv, kvd, a.h, BN)) != cudaSuccess) return e;
+    if ((e = make_operand_map(&maps.b_fc, a.fc, a.h, 2 * (int64_t)a.h, BNH)) != cudaSuccess) return e;
+    if ((e = make_operand_map(&maps.b_wk, a.wk, kvd, a.h, BNH)) != cudaSuccess) return e;
+    if ((e = make_operand_map(&maps.b_wv, a.wv, kvd, a.h, BNH)) != cudaSuccess) return e;
     // the counters start at zero on every call (a memset node in the caller's stream)
     if ((e = cudaMemsetAsync(p.ctr, 0, header_bytes(a.chunk_rows), s)) != cudaSuccess) return e;
     return launch(p, maps, s);
@@ -1083,12 +1189,12 @@ cudaError_t gemm_bf16_launch(const uint16_t* A, const uint16_t* B, uint16_t* C, 
     p.n_chunks = 1;
     p.lanes = 1;
     p.nf = N / BN;
-    p.total = (int64_t)((M + BM - 1) / BM) * (N / BN);
+    p.total = (int64_t)((M + 2 * BM - 1) / (2 * BM)) * (N / BN);
     p.dev_err = dev_err;
     Maps maps{};
     cudaError_t e;
     if ((e = make_operand_map(&maps.a_concat[0], A, M, K, BM)) != cudaSuccess) return e;
-    if ((e = make_operand_map(&maps.b_fc, B, N, K, BN)) != cudaSuccess) return e;
+    if ((e = make_operand_map(&maps.b_fc, B, N, K, BNH)) != cudaSuccess) return e;
     return launch(p, maps, s);
 }
 

@@ -1,7 +1,7 @@
 // Thin wrappers over the sm_100a tensor-memory MMA instructions (tcgen05) and
 // tensor-map TMA loads used by the prefill GEMM and the many-input lm_head sweep.
-// cta_group::1 throughout: one CTA owns a 128-lane accumulator in its SM's tensor
-// memory.
+// cta_group::1 (one CTA owns a 128-lane accumulator in its SM's tensor memory) for the
+// sweeps, cta_group::2 (a CTA pair shares each MMA) for the prefill GEMM.
 #pragma once
 
 #include <cuda.h>
@@ -176,6 +176,66 @@ __device__ __forceinline__ void tma_load_2d_g(void* dst, const CUtensorMap* map,
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
         "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// ---------------------------------------------------------------- CTA pairs (cta_group::2)
+// The two CTAs of a 2-CTA cluster (ranks 0 and 1, on the two SMs of one TPC) share one MMA
+// of M = 256: A is 128 rows from each CTA's shared memory, B is N / 2 rows from each (the
+// same shared-memory offsets in both), D is each CTA's 128 rows x N in its own tensor
+// memory. Rank 0 issues the MMAs. A kernel uses either these forms or the cta_group::1
+// ones above, never both.
+
+// Warp-wide, in the same warp of both CTAs with the same `dst`: allocate `ncols` TMEM
+// columns in both SMs; the base address (the same in both) is written to each CTA's `dst`.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(dst)),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+// Warp-wide, in the allocating warp of both CTAs.
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+// D[tmem of both CTAs] (+)= A * B^T over the pair, bf16 inputs, fp32 accumulate. Issued by
+// one thread of rank 0; the descriptors' addresses apply to both CTAs' shared memory.
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive (once) on the mbarrier at `bar`'s offset in every CTA of `cta_mask` (bit r: rank r)
+// when every MMA issued so far by this thread has completed.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t cta_mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(smem_u32(bar)),
+        "h"(cta_mask)
+        : "memory");
+}
+
+// 2-D tile load into this CTA's shared memory whose completion (bytes) is counted on the
+// mbarrier at shared::cluster address `bar_cl`, which may be the other CTA's of the pair.
+// No multicast: each CTA loads its own tile.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, int x, int y,
+                                                 uint32_t bar_cl) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(bar_cl)
         : "memory");
 }
 

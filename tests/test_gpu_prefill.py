@@ -38,7 +38,8 @@ def gemm(A, B):
 
 
 @pytest.mark.parametrize("M,N,K", [(128, 256, 64), (300, 512, 640), (1000, 1024, 4096),
-                                   (2048, 4096, 256)])  # the last: several tiles per SM
+                                   (1400, 768, 512),    # 11 row blocks: the last pair has one
+                                   (2048, 4096, 256)])  # the last: several tiles per SM pair
 def test_gemm_matches_numpy(orc, M, N, K):
     A = synth.as_u16(synth.normal_bf16(synth._gen(M + N), (M, K), 1.0))
     B = synth.as_u16(synth.normal_bf16(synth._gen(K + 3), (N, K), 0.02))
@@ -287,6 +288,15 @@ def test_prefill_many_tiles_per_sm(orc):
     rows = np.unique(np.concatenate([[0, 255, 256, 2047],
                                      np.random.default_rng(6).choice(2048, 40, replace=False)]))
     check_rows(orc, d, outs[0][0], outs[0][1], rows)
+
+
+def test_prefill_odd_row_blocks(orc):
+    """Chunks of three 128-row blocks (384 rows; the last chunk 232 rows, two blocks): the
+    last 256-row pair block of a full chunk has rows for one CTA of the pair only."""
+    d = synth.prefill_inputs(seed=95, R=1000, vocab=400, h=512, nkv=2, hd=128)
+    kc, vc, err = run_prefill(d, chunk=384)
+    assert err == 0
+    check_rows(orc, d, kc, vc, np.arange(1000))
 
 
 def test_prefill_ragged_chunks_and_one_row(orc):
