@@ -434,11 +434,12 @@ mtp_status mtp_debug_kv_write(const uint16_t* k_rot, const uint16_t* v, int64_t 
  * code that must not risk the device synchronisation cudaMalloc/cudaFree can cause).
  * Inputs and outputs are the caller's, exactly as for mtp_lm_head_argmax; the scratch
  * is a static device array inside the library, mtp_noalloc_scratch_bytes() bytes
- * (524,544: a 256-byte header + 16-byte partials of up to 1,024 CTAs x 32 input rows)
- * held on every GPU that loads the library until the process exits. It has no room
- * for x in the form the many-input sweeps read it (FP8 tables from M = 7, NVFP4 from
- * M = 9), so those calls return MTP_ERR_WORKSPACE here; BF16 tables run at every M up
- * to 32.
+ * (983,296: a 256-byte header, 16-byte partials of up to 1,024 CTAs x 32 input rows and
+ * 448 KB for x in the form the quantized tables' sweeps read it) held on every GPU that
+ * loads the library until the process exits. Calls whose mtp_lm_head_ws_bytes exceeds
+ * it return MTP_ERR_WORKSPACE: BF16 tables run at every M up to 32; FP8 and NVFP4
+ * tables at every M up to 32 with k <= 7,152, NVFP4 with up to 16 inputs and
+ * k <= 8,448.
  *  - The first call made with a device current looks up that array's device address.
  *    Under the CUDA runtime's lazy module loading (the default since CUDA 12.2) that
  *    look-up is also when the array is committed on the device, so make the first call

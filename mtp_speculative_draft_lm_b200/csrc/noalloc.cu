@@ -6,8 +6,8 @@
 // back, an engine that reserves all free device memory for its KV cache at start-up
 // and treats any later allocation as an error, or code that must not risk the device
 // synchronisation that cudaMalloc/cudaFree can cause. They still pass their own
-// inputs and outputs; only the sweep's scratch (the CTA partials and the last-CTA
-// counter) comes from here.
+// inputs and outputs; only the sweep's scratch (the CTA partials, the last-CTA counter
+// and x in the form the quantized tables' sweeps read it) comes from here.
 //
 // The scratch is the file-scope device array below: every GPU that loads this library
 // holds it (kScratchBytes) until the process exits, and every call on that GPU shares
@@ -32,7 +32,10 @@
 namespace {
 
 constexpr size_t kTicketBytes = 256;
-constexpr size_t kScratchBytes = kTicketBytes + 16 * 32 * 1024;  // header + 1024 CTAs x 32 partials
+// header + 1024 CTAs x 32 partials + 448 KB for x in the form the quantized tables' sweeps
+// read it (NVFP4: its E2M1 terms and their scales; FP8 from 7 inputs: two E4M3 planes)
+constexpr size_t kXBytes = 448 * 1024;
+constexpr size_t kScratchBytes = kTicketBytes + 16 * 32 * 1024 + kXBytes;
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) uint8_t g_sweep_scratch[kScratchBytes];

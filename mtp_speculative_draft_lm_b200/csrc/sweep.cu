@@ -2187,6 +2187,484 @@ __global__ void __launch_bounds__(kQThreads, 1)
     }
 }
 
+// ---------------------------------------------------------------- NVFP4 block-scaled sweep
+// NVFP4 tables run the contraction on tcgen05 block-scaled FP4 MMAs (kind::mxf4nvf4, one
+// E4M3 scale per 16 elements on each operand, K = 64 per instruction): the table's E2M1
+// codes and E4M3 block scales are the A operand and its scale factors as stored, so
+// nothing is decoded. The B operand must be FP4 too, so each input is written as six
+// E2M1 terms (q4_xterms_kernel): per 16-element block a power-of-two scale s and balanced
+// base-8 digits d_t in [-4, 4], x 2^e = sum_t d_t s 8^-t + r; term t is B row t MP + m with
+// codes d_t / 2 and block scale 2 s, and the epilogue weighs accumulator column t MP + m
+// by 8^-t in fp32. Every element whose binary exponent is within 9 of its block's
+// largest |x| is represented exactly (a bf16 value has 8 significant bits and the last
+// digit's unit is s 8^-5 < 2^-16 of the block's largest), the rest within s 8^-5 / 2, i.e.
+// 2^-17 of the block's largest |x|; s is at least 2^-10 (x 2^e units, the input's largest
+// |x 2^e| in [128, 256)), so blocks below 2^-8 there are represented within 2^-26.
+// Products and sums are fp32 in the tensor core.
+// Roles: warp 0 streams stages (128 table rows x segs 128-byte code segments and their
+// block scales, the x terms' codes and block scales for the same K range); warps 6-9
+// write the stage's scale factors into the ring slot's tensor-memory columns with
+// tcgen05.st, in the layout the MMA reads (in every lane quarter, lane l and columns
+// 4 j + c hold K block j's scales of row l + 32 c, four per 32-bit column); warp 1 issues
+// the MMAs from one thread; warps 2-5 sum the six term columns per input, scale, mask
+// and keep per input a running (max, lowest row, sum of exp). Tiles of 128 rows are
+// handed out at run time; the last CTA folds the CTA partials.
+constexpr int kQ4Terms = 6;
+constexpr int kQ4Threads = 320;  // warp 0 TMA, 1 MMA, 2-5 epilogue, 6-9 scale factors
+constexpr int kQ4Epi = 4;
+constexpr int kQ4Head = 3072;    // barriers, misc, factors, fold; then the ring
+constexpr int kQ4MaxM = 16;      // N = 6 MP <= 128: one group of scale rows
+
+__host__ __device__ constexpr int q4_mp(int M) { return M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16; }
+__host__ __device__ constexpr int q4_n(int MP) { return (kQ4Terms * MP + 15) / 16 * 16; }
+inline size_t q4_code_bytes(int N, int64_t k) { return ((size_t)N * (size_t)(k / 2) + 1023) & ~(size_t)1023; }
+inline size_t q4_scale_bytes(int N, int64_t k) { return ((size_t)N * (size_t)(k / 16) + 1023) & ~(size_t)1023; }
+__host__ __device__ inline int q4_stage_bytes(int N, int segs) {
+    const int b = segs * (16384 + N * 128 + N * 16 + 2048);
+    return (b + 1023) & ~1023;
+}
+// tensor-memory columns: the two accumulators, then per ring slot 16 segs for the table's
+// scale factors and 16 segs for x's
+__host__ __device__ inline int q4_max_slots(int N, int segs) { return (512 - 2 * N) / (32 * segs); }
+
+// The E4M3 code of 2^e, e in [-9, 8] (normal from 2^-6, subnormal below).
+__device__ __forceinline__ uint32_t e4m3_pow2(int e) {
+    return e >= -6 ? (uint32_t)(e + 7) << 3 : 1u << (e + 9);
+}
+
+// x [M, k] bf16 -> the block-scaled sweep's B operand. CTA m < M: input m scaled by 2^e_m
+// (its largest |x| lands in [128, 256)), then per 16-element block b: s = 2^ceil(log2(a /
+// 4)) for the block's largest |x 2^e| = a (s >= 2^-10), digits d_t = rint(r_t / (s 8^-t))
+// with r_0 = x 2^e, r_{t+1} = r_t - d_t s 8^-t (all exact in fp32; |d_t| <= 4 since
+// |r_t| <= 4 s 8^-t); row t MP + m gets the E2M1 codes of d_t / 2 (magnitude |d_t|, sign
+// bit 3) and the block scale E4M3(2 s). CTAs M .. MP - 1 zero their rows and CTA MP the
+// rows past 6 MP. codes [N][k / 2], scales [N][k / 16].
+__global__ void __launch_bounds__(256) q4_xterms_kernel(const uint16_t* __restrict__ x, int M, int k,
+                                                        int MP, int N, uint8_t* __restrict__ codes,
+                                                        uint8_t* __restrict__ scales,
+                                                        int32_t* __restrict__ xexp) {
+    __shared__ float red[8];
+    const int m = blockIdx.x, tid = threadIdx.x;
+    const int64_t rb = k / 2, sp = k / 16;
+    if (m >= M) {  // zero rows: inputs past M (their six rows), or the rows past 6 MP
+        const int n0 = m < MP ? m : kQ4Terms * MP;
+        const int step = m < MP ? MP : 1;
+        const int n1 = m < MP ? kQ4Terms * MP : N;
+        for (int n = n0; n < n1; n += step) {
+            for (int64_t j = tid; j < rb; j += 256) codes[(int64_t)n * rb + j] = 0;
+            for (int64_t j = tid; j < sp; j += 256) scales[(int64_t)n * sp + j] = 0;
+        }
+        return;
+    }
+    const uint16_t* row = x + (int64_t)m * k;
+    float a = 0.f;
+    for (int j = tid; j < k; j += 256) a = fmaxf(a, fabsf(bf16_to_f32(row[j])));
+    for (int o = 16; o; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if ((tid & 31) == 0) red[tid >> 5] = a;
+    __syncthreads();
+    a = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) a = fmaxf(a, red[w]);
+    int ex = 0;
+    if (a > 0.f) frexpf(a, &ex);  // a in [2^(ex-1), 2^ex)
+    const int e = (a > 0.f) ? 8 - ex : 0;
+    if (tid == 0) xexp[m] = e;
+    const float f1 = ldexpf(1.f, e / 2), f2 = ldexpf(1.f, e - e / 2);
+    for (int b = tid; b < k / 16; b += 256) {
+        float v[16];
+        float bm = 0.f;
+        const uint4* src = reinterpret_cast<const uint4*>(row + 16 * b);
+        const uint4 u0 = __ldg(src), u1 = __ldg(src + 1);
+        const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            v[2 * i] = (bf16_lo(w[i]) * f1) * f2;
+            v[2 * i + 1] = (bf16_hi(w[i]) * f1) * f2;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) bm = fmaxf(bm, fabsf(v[i]));
+        int se = -10;  // s = 2^se
+        if (bm > 0.f) {
+            int be = 0;
+            const float fr = frexpf(bm, &be);  // bm = fr 2^be, fr in [1/2, 1)
+            se = max(fr == 0.5f ? be - 3 : be - 2, -10);
+        }
+        const uint8_t sc = (uint8_t)e4m3_pow2(se + 1);
+#pragma unroll
+        for (int t = 0; t < kQ4Terms; ++t) {
+            const float u = ldexpf(1.f, se - 3 * t), iu = ldexpf(1.f, 3 * t - se);
+            uint32_t lo = 0, hi = 0;  // 16 codes, element i in nibble i
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                float d = rintf(v[i] * iu);
+                d = fminf(fmaxf(d, -4.f), 4.f);
+                v[i] = fmaf(-d, u, v[i]);
+                const uint32_t c = (d < 0.f ? 8u : 0u) | (uint32_t)fabsf(d);
+                if (i < 8) lo |= c << (4 * i);
+                else hi |= c << (4 * (i - 8));
+            }
+            const int n = t * MP + m;
+            *reinterpret_cast<uint2*>(codes + (int64_t)n * rb + 8 * b) = make_uint2(lo, hi);
+            scales[(int64_t)n * sp + b] = sc;
+        }
+    }
+}
+
+// D[tmem] (+)= (A sfa) . (B sfb)^T, E2M1 operands from shared memory, E4M3 scales per 16
+// elements from tensor memory, K = 64. One thread.
+__device__ __forceinline__ void umma_q4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
+// Warp-wide: this warp's 32 TMEM lanes, 4 consecutive 32-bit columns from `taddr` (a
+// multiple of 4) written.
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(a), "r"(b),
+                 "r"(c), "r"(d)
+                 : "memory");
+}
+
+template <int MP>
+__global__ void __launch_bounds__(kQ4Threads, 1)
+    sweep_q4_kernel(const __grid_constant__ SweepParams p, const __grid_constant__ CUtensorMap map_codes,
+                    const __grid_constant__ CUtensorMap map_scales, const __grid_constant__ CUtensorMap map_x,
+                    const __grid_constant__ CUtensorMap map_xs) {
+    constexpr int N = q4_n(MP);
+    static_assert(N <= 128, "one group of scale rows");
+    constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | (8u << 24);
+    constexpr uint32_t kSfCol = 2 * N;  // accumulators: columns [0, 2N)
+    constexpr uint32_t kTmemCols = 512;
+
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + kMaxStages;
+    uint64_t* sfull = empty + kMaxStages;  // the slot's scale factors are in tensor memory
+    uint64_t* tfull = sfull + kMaxStages;  // [2]
+    uint64_t* tempty = tfull + 2;          // [2]
+    uint64_t* done = tempty + 2;
+    int* misc = reinterpret_cast<int*>(done + 1);
+    volatile int* abort_flag = misc;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 1);
+    volatile int* slot_tile = misc + 2;              // [kMaxStages]
+    volatile int* acc_tile = misc + 2 + kMaxStages;  // [2]
+    float* sfac = reinterpret_cast<float*>(smem + 512);    // [2][32]: 2^-e_m as two factors
+    float4* fold = reinterpret_cast<float4*>(smem + 768);  // [4 warps][32 inputs]
+    uint8_t* ring = smem + kQ4Head;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int S = p.stages;
+    const int stage_bytes = p.stage_bytes;
+    const int segs = p.segs;
+    const int NC = p.stages_per_tile;
+    const int M = p.M;
+    const int64_t T = p.num_tiles;
+    // stage layout: table codes | x term codes | x term scales [N][16 segs] | table scales
+    // [128][16 segs]
+    const int a_bytes = 16384 * segs;
+    const int x_off = a_bytes, x_bytes = N * 128 * segs;
+    const int xs_off = x_off + x_bytes, xs_bytes = N * 16 * segs;
+    const int as_off = xs_off + xs_bytes, as_bytes = 2048 * segs;
+    const uint32_t tx = (uint32_t)(a_bytes + x_bytes + xs_bytes + as_bytes);
+    const uint32_t slot_cols = 32u * (uint32_t)segs;  // per ring slot: table's, then x's
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+            mbar_init(&sfull[s], 4);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 2);
+            mbar_init(&tempty[b], kQ4Epi);
+        }
+        mbar_init(done, 1);
+        misc[0] = 0;
+        mbar_fence_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    pdl_launch_dependents();
+
+    if (warp == 0) {
+        // ---------------- producer: the tiles' stages, each tagged with its tile
+        int slot = 0;
+        uint32_t phase = 0;
+        int64_t issued = 0;
+        bool stop = false;
+        pdl_wait();  // the x terms come from the previous grid
+        int64_t tile = blockIdx.x;
+        int64_t pending = 0;
+        if (lane == 0) pending = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
+        while (tile < T && !stop) {
+            for (int ch = 0; ch < NC; ++ch) {
+                if (!mbar_wait_bounded(&empty[slot], phase ^ 1u, abort_flag)) {
+                    stop = true;
+                    break;
+                }
+                if (lane == 0) {
+                    uint8_t* dst = ring + (size_t)slot * stage_bytes;
+                    slot_tile[slot] = (int)tile;
+                    mbar_arrive_expect_tx(&full[slot], tx);
+                    tma_load_3d(dst, &map_codes, 0, (int)(tile * 128), ch * segs, &full[slot]);
+                    tma_load_3d(dst + x_off, &map_x, 0, 0, ch * segs, &full[slot]);
+                    tma_load_2d(dst + xs_off, &map_xs, ch * 8 * segs, 0, &full[slot]);
+                    tma_load_2d(dst + as_off, &map_scales, ch * 8 * segs, (int)(tile * 128), &full[slot]);
+                }
+                __syncwarp();
+                ++issued;
+                if (++slot == S) {
+                    slot = 0;
+                    phase ^= 1u;
+                }
+            }
+            tile = __shfl_sync(0xffffffffu, pending, 0);
+            if (lane == 0 && tile < T) pending = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
+        }
+        for (int64_t j = issued > S ? issued - S : 0; j < issued; ++j)
+            if (!mbar_wait_bounded(&full[j % S], (uint32_t)((j / S) & 1), nullptr)) break;
+        if (!stop && mbar_wait_bounded(&empty[slot], phase ^ 1u, abort_flag) && lane == 0) {
+            slot_tile[slot] = -1;
+            mbar_arrive(&full[slot]);
+        }
+        __syncwarp();
+    } else if (warp >= 6) {
+        // ---------------- scale factors: warp 6 + q writes lane quarter q; its lane l holds,
+        // for K block j, the scale words (four 16-element blocks each) of table rows and x
+        // term rows l, l + 32, l + 64, l + 96 at columns 4 j .. 4 j + 3 of the slot's regions
+        const int q = warp - 6;
+        int slot = 0;
+        uint32_t phase = 0;
+        const uint32_t lq = tmem_base + ((uint32_t)(q * 32) << 16);
+        while (true) {
+            if (!mbar_wait_bounded(&full[slot], phase, abort_flag)) break;
+            if (slot_tile[slot] < 0) break;
+            const uint8_t* st = ring + (size_t)slot * stage_bytes;
+            const uint32_t ca = lq + kSfCol + (uint32_t)slot * slot_cols;  // table's
+            const uint32_t cx = ca + 16u * (uint32_t)segs;                  // x's
+            for (int sg = 0; sg < segs; ++sg) {
+                uint4 ra[4], rx[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int r = lane + 32 * c;
+                    ra[c] = lds128(st + as_off + r * 16 * segs + 16 * sg);
+                    rx[c] = r < N ? lds128(st + xs_off + r * 16 * segs + 16 * sg) : make_uint4(0, 0, 0, 0);
+                }
+                const uint32_t c0 = 16u * (uint32_t)sg;
+                tmem_st4(ca + c0 + 0, ra[0].x, ra[1].x, ra[2].x, ra[3].x);
+                tmem_st4(ca + c0 + 4, ra[0].y, ra[1].y, ra[2].y, ra[3].y);
+                tmem_st4(ca + c0 + 8, ra[0].z, ra[1].z, ra[2].z, ra[3].z);
+                tmem_st4(ca + c0 + 12, ra[0].w, ra[1].w, ra[2].w, ra[3].w);
+                tmem_st4(cx + c0 + 0, rx[0].x, rx[1].x, rx[2].x, rx[3].x);
+                tmem_st4(cx + c0 + 4, rx[0].y, rx[1].y, rx[2].y, rx[3].y);
+                tmem_st4(cx + c0 + 8, rx[0].z, rx[1].z, rx[2].z, rx[3].z);
+                tmem_st4(cx + c0 + 12, rx[0].w, rx[1].w, rx[2].w, rx[3].w);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sfull[slot]);
+            if (++slot == S) {
+                slot = 0;
+                phase ^= 1u;
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer (lane 0)
+        int slot = 0;
+        uint32_t phase = 0;
+        int local = 0;
+        while (true) {
+            if (!mbar_wait_bounded(&full[slot], phase, abort_flag)) break;
+            const int tile = slot_tile[slot];
+            const int buf = local & 1;
+            const uint32_t tph = (uint32_t)((local >> 1) & 1);
+            if (!mbar_wait_bounded(&tempty[buf], tph ^ 1u, abort_flag)) break;
+            if (lane == 0) {  // the tile index for the epilogue (its own arrival, release)
+                acc_tile[buf] = tile;
+                mbar_arrive(&tfull[buf]);
+                if (tile < 0) mbar_arrive(&tfull[buf]);  // no MMAs behind the end marker
+            }
+            __syncwarp();
+            if (tile < 0) break;
+            const uint32_t d_tmem = tmem_base + (uint32_t)(buf * N);
+            bool ok = true;
+            for (int ch = 0; ch < NC; ++ch) {
+                if ((ch > 0 && !mbar_wait_bounded(&full[slot], phase, abort_flag)) ||
+                    !mbar_wait_bounded(&sfull[slot], phase, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t st = smem_u32(ring + (size_t)slot * stage_bytes);
+                    const uint32_t ca = tmem_base + kSfCol + (uint32_t)slot * slot_cols;
+                    const uint32_t cx = ca + 16u * (uint32_t)segs;
+                    const int kbs = 4 * segs;
+                    for (int kb = 0; kb < kbs; ++kb) {
+                        const uint32_t as = st + (uint32_t)((kb >> 2) * 16384 + (kb & 3) * 32);
+                        const uint32_t xs = st + (uint32_t)(x_off + (kb >> 2) * (N * 128) + (kb & 3) * 32);
+                        umma_q4(d_tmem, sdesc_k128(as), sdesc_k128(xs), kIdesc, ca + 4u * (uint32_t)kb,
+                                cx + 4u * (uint32_t)kb, (ch > 0 || kb > 0) ? 1u : 0u);
+                    }
+                    umma_commit(&empty[slot]);  // frees the stage (and its scale columns) once read
+                }
+                __syncwarp();
+                if (++slot == S) {
+                    slot = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (lane == 0) umma_commit(&tfull[buf]);  // the accumulator, once complete
+            __syncwarp();
+            ++local;
+            if (!ok) break;
+        }
+        if (lane == 0) umma_commit(done);
+        __syncwarp();
+        mbar_wait_bounded(done, 0u, nullptr);
+    } else {
+        // ---------------- epilogue: warp w reads tensor memory lanes 32 (w % 4) + [0, 32)
+        const int q = warp & 3;
+        const int ew = warp - 2;  // 0..3
+        const bool lp = p.out_logprob != nullptr || p.out_partial != nullptr;
+        pdl_wait();
+        if (ew == 0) {
+            const int e = lane < M ? -__ldg(p.xexp + lane) : 0;
+            sfac[lane] = ldexpf(1.f, e / 2);
+            sfac[32 + lane] = ldexpf(1.f, e - e / 2);
+        }
+        const float gsc = __ldg(p.global_scale);
+        named_sync(1, kQ4Epi * 32);
+        float best_v[MP], se[MP];
+        int32_t best_i[MP];
+#pragma unroll
+        for (int m = 0; m < MP; ++m) {
+            best_v[m] = -INFINITY;
+            best_i[m] = INT_MAX;
+            se[m] = 0.f;
+        }
+        int local = 0;
+        while (true) {
+            const int buf = local & 1;
+            const uint32_t tph = (uint32_t)((local >> 1) & 1);
+            if (!mbar_wait_bounded(&tfull[buf], tph, abort_flag)) break;
+            const int tile = acc_tile[buf];
+            if (tile < 0) break;
+            tc_fence_after();
+            // per input, the six term columns t MP + m weighed by 8^-t, in order of t
+            float l[MP];
+#pragma unroll
+            for (int m = 0; m < MP; ++m) l[m] = 0.f;
+            const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * N);
+#pragma unroll
+            for (int c0 = 0; c0 < N; c0 += 32) {
+                uint32_t v[32];
+                if (c0 + 32 <= N) {
+                    tmem_ld32(ta + c0, v);
+                } else {
+                    uint32_t h[16];
+                    tmem_ld16(ta + c0, h);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = h[i];
+                }
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int n = c0 + i;
+                    if (n < N && n < kQ4Terms * MP)
+                        l[n % MP] = fmaf(__uint_as_float(v[i]), 1.0f / (float)(1 << (3 * (n / MP))), l[n % MP]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[buf]);  // the accumulator is free again
+            const int64_t row = (int64_t)tile * 128 + q * 32 + lane;
+            const bool rvalid = row < p.n;
+#pragma unroll
+            for (int m = 0; m < MP; ++m) {
+                if (m >= M) break;
+                const float lv = ((l[m] * sfac[m]) * sfac[32 + m]) * gsc;
+                const bool ok = rvalid && mask_allows(p, m, row);
+                if (rvalid && p.out_logits)
+                    p.out_logits[(int64_t)m * p.n + row] = ok ? f32_to_bf16(lv) : (uint16_t)0xFF80u;
+                if (lp && ok && lv > -INFINITY) {
+                    float bv = best_v[m];
+                    lse_merge(bv, se[m], lv, 1.f);
+                }
+                // each thread's rows arrive in increasing order: the lowest wins a tie
+                if (ok && (lv > best_v[m] || (lv == best_v[m] && best_i[m] == INT_MAX))) {
+                    best_v[m] = lv;
+                    best_i[m] = (int32_t)row;
+                }
+            }
+            ++local;
+        }
+        // per input: fold the 32 lanes, then the four warps in order; publish; ticket
+#pragma unroll
+        for (int m = 0; m < MP; ++m) {
+            if (m >= M) break;
+#pragma unroll
+            for (int o = 16; o; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, best_v[m], o);
+                const int32_t oi = __shfl_xor_sync(0xffffffffu, best_i[m], o);
+                const float os = __shfl_xor_sync(0xffffffffu, se[m], o);
+                if (lp) {
+                    float bv = best_v[m];
+                    lse_merge(bv, se[m], ov, os);
+                }
+                if (ov > best_v[m] || (ov == best_v[m] && oi < best_i[m])) {
+                    best_v[m] = ov;
+                    best_i[m] = oi;
+                }
+            }
+            if (lane == 0) fold[ew * 32 + m] = make_float4(best_v[m], __int_as_float(best_i[m]), se[m], 0.f);
+        }
+        named_sync(1, kQ4Epi * 32);
+        if (ew == 0) {
+            if (lane < M) {
+                float bv = -INFINITY, bs = 0.f;
+                int32_t bi = INT_MAX;
+                for (int w = 0; w < kQ4Epi; ++w) {
+                    const float4 f = fold[w * 32 + lane];
+                    const int32_t fi = __float_as_int(f.y);
+                    if (lp) {
+                        float t = bv;
+                        lse_merge(t, bs, f.x, f.z);
+                    }
+                    if (f.x > bv || (f.x == bv && fi < bi)) {
+                        bv = f.x;
+                        bi = fi;
+                    }
+                }
+                reinterpret_cast<Partial*>(p.partials)[(int64_t)blockIdx.x * kPartSlots + lane] =
+                    Partial{bv, bi, bs, 0.f};
+            }
+            __syncwarp();
+            fence_acq_rel_gpu();  // every publishing lane's store before lane 0's ticket
+            __syncwarp();
+            if (*abort_flag && lane == 0) raise_flag(p.dev_err, DEVFLAG_TIMEOUT);
+            ticket_and_fold(p, lane, lp);
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
 struct Geometry {
     int kpad;
     int segs;             // 128-byte segments per row per stage
@@ -2601,6 +3079,87 @@ cudaError_t launch_tc4(const SweepParams& p, cudaStream_t s, SweepLaunch* info) 
     return cudaGetLastError();
 }
 
+WideGeometry q4_geometry(int64_t k, int N) {
+    WideGeometry g{};
+    const int row_segs = (int)(k / 256);  // 128-byte code segments per row
+    const long avail = (long)kSmemLimit - (long)kQ4Head;
+    for (int segs = 2; segs >= 1 && g.stages == 0; --segs) {
+        if (segs > row_segs) continue;
+        const int sb = q4_stage_bytes(N, segs);
+        int stages = avail > 0 ? (int)(avail / sb) : 0;
+        stages = min(stages, min(kMaxStages, q4_max_slots(N, segs)));
+        if (stages >= (segs == 2 ? 3 : 2)) {
+            g.segs = segs;
+            g.stages_per_tile = (row_segs + segs - 1) / segs;
+            g.stage_bytes = sb;
+            g.stages = stages;
+        }
+    }
+    g.smem = (size_t)kQ4Head + (size_t)g.stages * g.stage_bytes;
+    return g;
+}
+
+template <int MP>
+cudaError_t launch_q4(const SweepParams& p, cudaStream_t s, SweepLaunch* info) {
+    constexpr int N = q4_n(MP);
+    auto kern = sweep_q4_kernel<MP>;
+    const WideGeometry geo = q4_geometry(p.k, N);
+    if (geo.stages < 2) return cudaErrorInvalidValue;
+    uint8_t* xcodes = reinterpret_cast<uint8_t*>(p.x16);
+    uint8_t* xscales = xcodes + q4_code_bytes(N, p.k);
+    CUtensorMap map_codes, map_scales, map_x, map_xs;
+    cudaError_t e = make_code_map(&map_codes, p.w, p.n, p.row_bytes, geo.segs, 128);
+    if (e != cudaSuccess) return e;
+    if ((e = make_scale_map(&map_scales, p.block_scale, p.n, p.scale_pitch, geo.segs, 128)) != cudaSuccess)
+        return e;
+    if ((e = make_code_map(&map_x, xcodes, N, p.k / 2, geo.segs, N)) != cudaSuccess) return e;
+    if ((e = make_scale_map(&map_xs, xscales, N, p.k / 16, geo.segs, N)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)geo.smem)) !=
+        cudaSuccess)
+        return e;
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    SweepParams q = p;
+    q.num_tiles = (p.n + 127) / 128;
+    q.stages = geo.stages;
+    q.stage_bytes = geo.stage_bytes;
+    q.segs = geo.segs;
+    q.stages_per_tile = geo.stages_per_tile;
+    int64_t grid = sms;
+    if (grid > q.num_tiles) grid = q.num_tiles;
+    if (grid > kMaxGrid) grid = kMaxGrid;
+    if (grid < 1) grid = 1;
+    q4_xterms_kernel<<<MP + 1, 256, 0, s>>>(p.x, p.M, (int)p.k, MP, N, xcodes, xscales, p.xexp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kQ4Threads);
+    cfg.dynamicSmemBytes = geo.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if ((e = cudaLaunchKernelEx(&cfg, kern, q, map_codes, map_scales, map_x, map_xs)) != cudaSuccess)
+        return e;
+    if (info) {
+        info->grid = (int)grid;
+        info->smem_bytes = (int)geo.smem;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_q4_any(const SweepParams& p, cudaStream_t s, SweepLaunch* info) {
+    switch (q4_mp(p.M)) {
+        case 2: return launch_q4<2>(p, s, info);
+        case 4: return launch_q4<4>(p, s, info);
+        case 8: return launch_q4<8>(p, s, info);
+        default: return launch_q4<16>(p, s, info);
+    }
+}
+
 // Argmax sweeps that stream x per K chunk -- the tcgen05 sweeps, and for NVFP4 the wide
 // mma.sync sweep -- take FP8 tables from 7 inputs on (measured faster than 16-row tiles
 // from there), BF16 and NVFP4 from 9. NVFP4 runs 9-16 inputs on the wide sweep and 17-32
@@ -2623,9 +3182,13 @@ size_t sweep_smem_bytes(int M, int64_t k, int fmt, int* kpad_out, int mode, bool
         if (kpad_out) *kpad_out = g.kpad;
         return g.stages >= 2 ? g.smem : (size_t)kSmemLimit + 1;
     }
-    if (mode == 0 && streams_x(M, fmt)) {  // the tcgen05 / wide sweeps stage x per K chunk
-        const WideGeometry w = fmt == 2 ? (nvfp4_tc4(M) ? tc4_geometry(k, 32, 2) : wide_geometry(k, 2, 16))
-                                        : tc_geometry(k, fmt, M > 16 ? 32 : 16);
+    if (mode == 0 && fmt == 2 && M <= kQ4MaxM) {  // the block-scaled sweep
+        const WideGeometry w = q4_geometry(k, q4_n(q4_mp(M)));
+        if (kpad_out) *kpad_out = (int)k;
+        return w.stages >= 2 ? w.smem : (size_t)kSmemLimit + 1;
+    }
+    if (mode == 0 && streams_x(M, fmt)) {  // the tcgen05 sweeps stage x per K chunk
+        const WideGeometry w = fmt == 2 ? tc4_geometry(k, 32, 2) : tc_geometry(k, fmt, M > 16 ? 32 : 16);
         if (kpad_out) *kpad_out = (int)k;
         return w.stages >= 2 ? w.smem : (size_t)kSmemLimit + 1;
     }
@@ -2637,9 +3200,13 @@ size_t sweep_smem_bytes(int M, int64_t k, int fmt, int* kpad_out, int mode, bool
 int sweep_max_grid() { return kMaxGrid; }
 
 size_t sweep_x16_bytes(int M, int64_t k, int fmt) {
+    if (fmt == 2 && M <= kQ4MaxM) {  // the block-scaled sweep's x terms: codes, scales, exponents
+        const int N = q4_n(q4_mp(M));
+        return q4_code_bytes(N, k) + q4_scale_bytes(N, k) + 1024;
+    }
     if (fmt == 0 || !streams_x(M, fmt)) return 0;
-    // FP8: x's two E4M3 planes of 16 or 32 rows; NVFP4: the f16 copy of x. Then 1 KB
-    // for the per-input exponents.
+    // FP8: x's two E4M3 planes of 16 or 32 rows; NVFP4 past the block-scaled sweep: the f16
+    // copy of x. Then 1 KB for the per-input exponents.
     const size_t body = fmt == 1 ? (size_t)2 * (M > 16 ? 32 : 16) * (size_t)k : (size_t)M * (size_t)k * 2;
     return ((body + 1023) & ~(size_t)1023) + 1024;
 }
@@ -2704,7 +3271,7 @@ cudaError_t sweep_launch(const SweepParams& p, int fmt, int mode, cudaStream_t s
         if (fmt == 2)
             return p.M <= 2 ? launch_one<2, 1, 0, 1, 1>(p, s, info) : launch_one<2, 1, 0, 0, 1>(p, s, info);
     }
-    if (fmt == 2 && mode == 0 && p.M <= 2) return launch_one<2, 1, 0, 1, 0>(p, s, info);
+    if (fmt == 2 && mode == 0 && p.M <= kQ4MaxM) return launch_q4_any(p, s, info);
     if (mode == 0 && streams_x(p.M, fmt)) {
         const bool four = p.M > 16;
         if (fmt == 0) return four ? launch_tc<0, 32>(p, s, info) : launch_tc<0, 16>(p, s, info);

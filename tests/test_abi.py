@@ -130,24 +130,30 @@ def test_lm_head_lp_rejects(lib):
     assert lp(OUT, x=B2 + 4) == L.MTP_ERR_INVALID_ARG  # the same checks as mtp_lm_head_argmax
     assert lp(OUT, n_eff=101) == L.MTP_ERR_INVALID_ARG
     # partials are 16 bytes (max, index, sum of exponentials) for up to 1,024 CTAs x 32 inputs
-    assert wsb == 256 + 16 * 32 * 1024 and L.mtp_noalloc_scratch_bytes() == wsb
-    # quantized tables with many inputs add x as those sweeps read it (+ 1 KB of
-    # exponents): FP8, two E4M3 planes of 16 or 32 rows; NVFP4, an f16 copy of the M rows
+    assert wsb == 256 + 16 * 32 * 1024
+    # the no-alloc array adds 448 KB for x in the quantized sweeps' forms
+    assert L.mtp_noalloc_scratch_bytes() == wsb + 448 * 1024
+    up = lambda b: (b + 1023) // 1024 * 1024
+    # quantized tables add x as their sweeps read it (+ 1 KB of exponents): FP8 from 7
+    # inputs, two E4M3 planes of 16 or 32 rows; NVFP4 up to 16 inputs, N = 6 MP rows of
+    # E2M1 terms (MP = 2, 4, 8, 16) and their E4M3 block scales, then an f16 copy of x
     fp8 = weight(fmt=1, k=128, rs=OUT)
     assert L.mtp_lm_head_ws_bytes(fp8, 100, 6) == wsb  # FP8 streams x from 7 inputs on
     assert L.mtp_lm_head_ws_bytes(fp8, 100, 7) == wsb + 2 * 16 * 128 + 1024
     assert L.mtp_lm_head_ws_bytes(fp8, 100, 9) == wsb + 2 * 16 * 128 + 1024
     assert L.mtp_lm_head_ws_bytes(fp8, 100, 17) == wsb + 2 * 32 * 128 + 1024
     nv = weight(fmt=2, k=256, bs=OUT, gs=OUT)
-    assert L.mtp_lm_head_ws_bytes(nv, 100, 8) == wsb  # NVFP4 reads its f16 x copy from 9 inputs
-    assert L.mtp_lm_head_ws_bytes(nv, 100, 9) == wsb + ((9 * 256 * 2 + 1023) // 1024) * 1024 + 1024
+    for M, N in ((1, 16), (2, 16), (3, 32), (8, 48), (9, 96), (16, 96)):
+        assert L.mtp_lm_head_ws_bytes(nv, 100, M) == wsb + up(N * 128) + up(N * 16) + 1024, M
+    assert L.mtp_lm_head_ws_bytes(nv, 100, 17) == wsb + up(17 * 256 * 2) + 1024
     assert L.mtp_lm_head_ws_bytes(weight(k=128), 100, 32) == wsb
-    # the no-alloc array has no room for that copy: rejected before any CUDA call
+    # calls past the no-alloc array are rejected before any CUDA call
     noalloc = lambda head, M: st("mtp_lm_head_argmax_noalloc", C.byref(head), 100, B2, M, None,
                                  0, 0, OUT, None, None, None, None)
-    assert noalloc(fp8, 7) == L.MTP_ERR_WORKSPACE
-    assert noalloc(weight(fmt=2, k=256, bs=OUT, gs=OUT), 12) == L.MTP_ERR_WORKSPACE
-    assert noalloc(weight(fmt=2, k=256, bs=OUT, gs=OUT), 9) == L.MTP_ERR_WORKSPACE
+    assert noalloc(weight(fmt=1, k=14336, rs=OUT), 7) == L.MTP_ERR_WORKSPACE
+    assert noalloc(weight(fmt=1, k=7168, rs=OUT), 17) == L.MTP_ERR_WORKSPACE
+    assert noalloc(weight(fmt=2, k=8704, bs=OUT, gs=OUT), 16) == L.MTP_ERR_WORKSPACE
+    assert noalloc(weight(fmt=2, k=7168, bs=OUT, gs=OUT), 32) == L.MTP_ERR_WORKSPACE
     # the table descriptor is checked before its size is looked at: a bad format, a bad k
     # or a missing scale is an argument error, not a workspace one
     assert noalloc(weight(fmt=7, k=128), 12) == L.MTP_ERR_INVALID_ARG

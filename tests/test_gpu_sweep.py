@@ -267,8 +267,9 @@ def test_full_tables(orc, cfg, fmt):
 
 
 # Inputs for which the masked sweep (which reads only allowed rows) and the unmasked one
-# run the same kernel, so that their logits must agree bit for bit.
-SAME_KERNEL_M = {0: 8, 1: 6, 2: 8}
+# run the same kernel, so that their logits must agree bit for bit (NVFP4: none, the
+# unmasked sweep runs on block-scaled FP4 MMAs, the gathered one on decoded f16 MMAs).
+SAME_KERNEL_M = {0: 8, 1: 6, 2: 0}
 
 
 @pytest.mark.parametrize("cfg,fmt", FULL, ids=["bf16", "fp8", "nvfp4"])

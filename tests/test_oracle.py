@@ -563,6 +563,73 @@ def test_fp8_x_two_term_split(orc):
     assert abs(hi[1] + lo[1] - xs[1]) == 2.0 ** -10
 
 
+def _six_terms(orc, xs):
+    """The six-term split of one scaled input row (per 16-element block: s = 2^se the
+    smallest power of two >= max|block| / 4, at least 2^-10; balanced base-8 digits
+    d_t = rint(r_t / (s 8^-t)), r_{t+1} = r_t - d_t s 8^-t), written independently of the
+    kernel with numpy; returns (digits [6, k], se per block, reconstruction)."""
+    k = xs.size
+    xb = xs.reshape(-1, 16)
+    a = np.abs(xb).max(axis=1)
+    se = np.full(a.shape, -10, dtype=np.int64)
+    nz = a > 0
+    se[nz] = np.maximum(np.ceil(np.log2(a[nz] / 4)).astype(np.int64), -10)
+    r = xb.copy()
+    digits = np.zeros((6,) + xb.shape)
+    rec = np.zeros_like(xb)
+    for t in range(6):
+        u = np.ldexp(1.0, se - 3 * t)[:, None]
+        d = np.rint(r / u)
+        digits[t] = d
+        rec += d * u
+        r = r - d * u
+    return digits.reshape(6, k), se, rec.reshape(k)
+
+
+def test_nvfp4_x_six_term_split(orc):
+    """The reading behind the block-scaled NVFP4 sweep: an input row scaled by 2^e (its
+    largest |x| in [128, 256)) and written per 16-element block as six E2M1 terms with one
+    power-of-two E4M3 scale: every digit d_t lies in [-4, 4] (so d_t / 2 is an E2M1 value),
+    the block scale 2 s is an E4M3 value, every element whose binary exponent is within 9
+    of its block's largest |x| is represented exactly (its 8 significant bits end at or
+    above the last digit's unit s 8^-5 < 2^-16 max), and the rest within 2^-17 of the
+    block's largest |x|; where s sits at its 2^-10 floor (blocks below 2^-8 in scaled units)
+    every element is within 2^-26 in scaled units instead."""
+    rng = np.random.default_rng(12)
+    for scale in (1.0, 3e-3, 7e5, 1e-20):
+        v = np.concatenate([rng.standard_normal(3008), rng.standard_normal(512) * 1e-3,
+                            rng.standard_normal(512) * 1e-6, rng.standard_normal(16) * 1e-30,
+                            np.zeros(16), [1.0, -1.0, 2.0 ** -9, 3.0] + [0.0] * 12])
+        xb = orc.f64_to_bf16(v * scale)
+        x = orc.bf16_to_f64(xb)
+        a = np.abs(x).max()
+        e = 8 - math.frexp(a)[1]
+        xs = x * 2.0 ** e
+        assert 128 <= np.abs(xs).max() < 256
+        digits, se, rec = _six_terms(orc, xs)
+        assert np.all(np.abs(digits) <= 4)
+        half = digits / 2
+        assert np.array_equal(orc.e2m1_value(orc.e2m1_encode(half)), half)
+        sc = np.ldexp(1.0, se + 1)
+        assert np.array_equal(orc.e4m3_value(orc.e4m3_encode(sc)), sc)
+        err = np.abs(rec - xs)
+        bmax = np.repeat(np.abs(xs.reshape(-1, 16)).max(axis=1), 16)
+        ex = np.frexp(np.abs(xs))[1]
+        bex = np.frexp(bmax)[1]
+        floor = np.repeat(se == -10, 16)
+        near = (xs != 0) & (bex - ex <= 9) & ~floor
+        assert near.sum() > 3500 and np.all(err[near] == 0.0)
+        assert np.any(err[(xs != 0) & (bex - ex > 9)] > 0)  # and not beyond
+        assert np.all(err[~floor] <= 2.0 ** -17 * bmax[~floor])
+        assert np.all(err[floor] <= 2.0 ** -26)
+    # the bound is reached: an element 2^-14 below its block's largest, halfway between
+    # two steps of the last term, keeps half a step
+    xs = np.zeros(16)
+    xs[0], xs[1] = 200.0, 2.0 ** -7 * 1.5 + 2.0 ** -12 * 1.5
+    _, se, rec = _six_terms(orc, xs)
+    assert se[0] == 6 and abs(rec[1] - xs[1]) <= 2.0 ** -17 * 200.0
+
+
 # ---------------------------------------------------------------- decode attention pins
 def _attn_case(orc, seed, nq=8, nkv=2, hd=64, seq=40, bs=16, extra_blocks=3):
     rng = np.random.default_rng(seed)
