@@ -2215,7 +2215,7 @@ constexpr int kQ4Epi = 4;
 constexpr int kQ4Head = 3072;    // barriers, misc, factors, fold; then the ring
 constexpr int kQ4MaxM = 16;      // N = 6 MP <= 128: one group of scale rows
 
-__host__ __device__ constexpr int q4_mp(int M) { return M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16; }
+__host__ __device__ constexpr int q4_mp(int M) { return M <= 4 ? 4 : M <= 8 ? 8 : 16; }
 __host__ __device__ constexpr int q4_n(int MP) { return (kQ4Terms * MP + 15) / 16 * 16; }
 inline size_t q4_code_bytes(int N, int64_t k) { return ((size_t)N * (size_t)(k / 2) + 1023) & ~(size_t)1023; }
 inline size_t q4_scale_bytes(int N, int64_t k) { return ((size_t)N * (size_t)(k / 16) + 1023) & ~(size_t)1023; }
@@ -3153,7 +3153,6 @@ cudaError_t launch_q4(const SweepParams& p, cudaStream_t s, SweepLaunch* info) {
 
 cudaError_t launch_q4_any(const SweepParams& p, cudaStream_t s, SweepLaunch* info) {
     switch (q4_mp(p.M)) {
-        case 2: return launch_q4<2>(p, s, info);
         case 4: return launch_q4<4>(p, s, info);
         case 8: return launch_q4<8>(p, s, info);
         default: return launch_q4<16>(p, s, info);
@@ -3182,7 +3181,7 @@ size_t sweep_smem_bytes(int M, int64_t k, int fmt, int* kpad_out, int mode, bool
         if (kpad_out) *kpad_out = g.kpad;
         return g.stages >= 2 ? g.smem : (size_t)kSmemLimit + 1;
     }
-    if (mode == 0 && fmt == 2 && M <= kQ4MaxM) {  // the block-scaled sweep
+    if (mode == 0 && fmt == 2 && M >= 3 && M <= kQ4MaxM) {  // the block-scaled sweep
         const WideGeometry w = q4_geometry(k, q4_n(q4_mp(M)));
         if (kpad_out) *kpad_out = (int)k;
         return w.stages >= 2 ? w.smem : (size_t)kSmemLimit + 1;
@@ -3200,6 +3199,7 @@ size_t sweep_smem_bytes(int M, int64_t k, int fmt, int* kpad_out, int mode, bool
 int sweep_max_grid() { return kMaxGrid; }
 
 size_t sweep_x16_bytes(int M, int64_t k, int fmt) {
+    if (fmt == 2 && M <= 2) return 0;
     if (fmt == 2 && M <= kQ4MaxM) {  // the block-scaled sweep's x terms: codes, scales, exponents
         const int N = q4_n(q4_mp(M));
         return q4_code_bytes(N, k) + q4_scale_bytes(N, k) + 1024;
@@ -3271,6 +3271,9 @@ cudaError_t sweep_launch(const SweepParams& p, int fmt, int mode, cudaStream_t s
         if (fmt == 2)
             return p.M <= 2 ? launch_one<2, 1, 0, 1, 1>(p, s, info) : launch_one<2, 1, 0, 0, 1>(p, s, info);
     }
+    // NVFP4 with one or two inputs: per-block fp32 sums of unscaled codes (measured faster
+    // than the block-scaled sweep there, 67.8 against 71.5 us on the 131,072 x 5,120 table)
+    if (fmt == 2 && mode == 0 && p.M <= 2) return launch_one<2, 1, 0, 1, 0>(p, s, info);
     if (fmt == 2 && mode == 0 && p.M <= kQ4MaxM) return launch_q4_any(p, s, info);
     if (mode == 0 && streams_x(p.M, fmt)) {
         const bool four = p.M > 16;

@@ -135,15 +135,17 @@ def test_lm_head_lp_rejects(lib):
     assert L.mtp_noalloc_scratch_bytes() == wsb + 448 * 1024
     up = lambda b: (b + 1023) // 1024 * 1024
     # quantized tables add x as their sweeps read it (+ 1 KB of exponents): FP8 from 7
-    # inputs, two E4M3 planes of 16 or 32 rows; NVFP4 up to 16 inputs, N = 6 MP rows of
-    # E2M1 terms (MP = 2, 4, 8, 16) and their E4M3 block scales, then an f16 copy of x
+    # inputs, two E4M3 planes of 16 or 32 rows; NVFP4 from 3 to 16 inputs, N = 6 MP rows of
+    # E2M1 terms (MP = 4, 8, 16, rounded up to 16 rows) and their E4M3 block scales, then
+    # an f16 copy of x
     fp8 = weight(fmt=1, k=128, rs=OUT)
     assert L.mtp_lm_head_ws_bytes(fp8, 100, 6) == wsb  # FP8 streams x from 7 inputs on
     assert L.mtp_lm_head_ws_bytes(fp8, 100, 7) == wsb + 2 * 16 * 128 + 1024
     assert L.mtp_lm_head_ws_bytes(fp8, 100, 9) == wsb + 2 * 16 * 128 + 1024
     assert L.mtp_lm_head_ws_bytes(fp8, 100, 17) == wsb + 2 * 32 * 128 + 1024
     nv = weight(fmt=2, k=256, bs=OUT, gs=OUT)
-    for M, N in ((1, 16), (2, 16), (3, 32), (8, 48), (9, 96), (16, 96)):
+    assert L.mtp_lm_head_ws_bytes(nv, 100, 1) == wsb and L.mtp_lm_head_ws_bytes(nv, 100, 2) == wsb
+    for M, N in ((3, 32), (4, 32), (8, 48), (9, 96), (16, 96)):
         assert L.mtp_lm_head_ws_bytes(nv, 100, M) == wsb + up(N * 128) + up(N * 16) + 1024, M
     assert L.mtp_lm_head_ws_bytes(nv, 100, 17) == wsb + up(17 * 256 * 2) + 1024
     assert L.mtp_lm_head_ws_bytes(weight(k=128), 100, 32) == wsb

@@ -23,8 +23,7 @@ def bits(t):
 
 @pytest.mark.parametrize("fmt", [0, 1, 2])
 def test_noalloc_matches_workspace_entry_point(fmt):
-    # four inputs: FP8 from seven and NVFP4 from nine read x in a form (E4M3 planes, an f16
-    # copy) the static array has no room for
+    # four inputs: NVFP4 then writes x as E2M1 terms into the static array's x area
     n, k, M = 5000, 1024, 4
     d = synth.head_table(21 + fmt, n, k, M)
     w = d["W"].cuda()
