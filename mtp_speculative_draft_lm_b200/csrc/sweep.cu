@@ -42,7 +42,8 @@
 // Every mbarrier wait is bounded: a wait that runs out sets an abort flag and
 // MTP_DEVFLAG_TIMEOUT, and the kernel runs to its end.
 // More inputs than this design serves well (BF16 from 9, FP8 from 7) go to the tcgen05
-// sweep further down; NVFP4 from 9 inputs to the 64-row-tile wide sweep.
+// sweep further down; NVFP4 from 3 inputs to the block-scaled FP4 sweep (3-16) and the
+// tcgen05 sweep with A in tensor memory (17-32).
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -1065,31 +1066,11 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
     }
 }
 
-// ------------------------------------------------------------------ many inputs (M > 8)
-// With more than eight inputs the staged x no longer fits beside a useful ring (16 inputs
-// x K 5,120 in f16 is 160 KB), so tiles are 64 rows tall and every stage carries, next to
-// the table's K chunk for those rows, the inputs' x chunk for the same K range, loaded by
-// TMA from global memory (L2): x is read once per 64 table rows instead of being held
-// whole. Four row groups of 16 rows; the 16 compute warps are 4 per row group, each
-// taking every fourth slab of its group's rows. Quantized tables read a f16 copy of x,
-// scaled per row by a power of two, written by wide_x16_kernel just before.
-constexpr int kWRows = 64;
-constexpr int kWCW = 16;                  // compute warps
-constexpr int kWThreads = (kWCW + 2) * 32;
-constexpr int kWRedBuffers = 2;           // reducer hand-off buffers (double-buffered)
-// inputs per sweep: 8 NT columns (NT = 2: up to 16 inputs, NT = 4: up to 32)
-
-__host__ __device__ inline int wide_seg_elems(int fmt) { return fmt == 0 ? 64 : fmt == 1 ? 128 : 256; }
-__host__ __device__ inline int wide_code_bytes(int segs) { return kWRows * 128 * segs; }
-__host__ __device__ inline int wide_scale_bytes(int fmt, int segs) { return fmt == 2 ? kWRows * 16 * segs : 0; }
-__host__ __device__ inline int wide_xsegs(int fmt, int segs) { return segs * wide_seg_elems(fmt) / 64; }
-__host__ __device__ inline int wide_x_bytes(int fmt, int segs, int cols) {
-    return wide_xsegs(fmt, segs) * cols * 128;
-}
-
+// ------------------------------------------------------------------ x as f16
 // x [M, k] bf16 -> f16 scaled by 2^e_m (the largest |x| of row m lands in [2^14, 2^15)),
-// as stage_to_f16 does in shared memory for the narrow sweep. One CTA per input row.
-__global__ void __launch_bounds__(256) wide_x16_kernel(const uint16_t* __restrict__ x, int k,
+// as stage_to_f16 does in shared memory for the narrow sweep; the copy the NVFP4 sweep
+// with A in tensor memory reads as its B operand. One CTA per input row.
+__global__ void __launch_bounds__(256) x16_kernel(const uint16_t* __restrict__ x, int k,
                                                         uint16_t* __restrict__ x16,
                                                         int32_t* __restrict__ xexp) {
     __shared__ float red[8];
@@ -1110,338 +1091,6 @@ __global__ void __launch_bounds__(256) wide_x16_kernel(const uint16_t* __restric
     const float f1 = ldexpf(1.f, e / 2), f2 = ldexpf(1.f, e - e / 2);
     for (int j = tid; j < k; j += 256)
         x16[(int64_t)m * k + j] = f32_to_f16((bf16_to_f32(row[j]) * f1) * f2);
-}
-
-// One slab of one row group for 16 inputs (two MMA column blocks). The codes are read as in
-// slab_mma; the lane's x elements [e, e + V) of inputs g and g + 8 come from the stage's
-// x chunk, [x segment of 64 elements][16 inputs][128 B] with the 128-byte swizzle.
-template <int FMT, int NT>
-__device__ __forceinline__ void slab_mma_wide(float (&acc)[2][NT][4], const uint8_t* cw,
-                                              const uint8_t* sw, uint32_t spitch8,
-                                              const uint8_t* xst, int e, int g) {
-    const uint4 ra = lds128(cw);
-    const uint4 rb = lds128(cw + 1024);
-    const uint8_t* x0 = xst + (e >> 6) * (8 * NT * 128) + g * 128;  // input g; t*8 + g below
-    const int cb = (e & 63) >> 3;                                     // first 16-byte chunk
-#define XQ(t, q) lds128(x0 + (t) * 1024 + ((((cb) + (q)) ^ g) << 4))
-    if (FMT == 0) {
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-            const uint4 xa = XQ(t, 0);
-            mma_bf16_16816(acc[0][t], ra.x, rb.x, ra.y, rb.y, xa.x, xa.y);
-            mma_bf16_16816(acc[1][t], ra.z, rb.z, ra.w, rb.w, xa.z, xa.w);
-        }
-    } else if (FMT == 1) {
-        const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w};
-        const uint32_t wb[4] = {rb.x, rb.y, rb.z, rb.w};
-        uint32_t a[4][4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            a[i][0] = e4m3x2_to_f16x2((uint16_t)(wa[i] & 0xFFFFu));
-            a[i][2] = e4m3x2_to_f16x2((uint16_t)(wa[i] >> 16));
-            a[i][1] = e4m3x2_to_f16x2((uint16_t)(wb[i] & 0xFFFFu));
-            a[i][3] = e4m3x2_to_f16x2((uint16_t)(wb[i] >> 16));
-        }
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-            const uint4 x_0 = XQ(t, 0), x_1 = XQ(t, 1);
-            const uint32_t xa[8] = {x_0.x, x_0.y, x_0.z, x_0.w, x_1.x, x_1.y, x_1.z, x_1.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                mma_f16_16816(acc[i & 1][t], a[i][0], a[i][1], a[i][2], a[i][3], xa[2 * i], xa[2 * i + 1]);
-        }
-    } else {
-        const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w};
-        const uint32_t wb[4] = {rb.x, rb.y, rb.z, rb.w};
-        const uint16_t s0v = *reinterpret_cast<const uint16_t*>(sw);
-        const uint16_t s1v = *reinterpret_cast<const uint16_t*>(sw + spitch8);
-        const uint32_t sa = e4m3x2_to_f16x2(s0v);
-        const uint32_t sb = e4m3x2_to_f16x2(s1v);
-        const uint32_t sa_lo = __byte_perm(sa, 0, 0x1010), sa_hi = __byte_perm(sa, 0, 0x3232);
-        const uint32_t sb_lo = __byte_perm(sb, 0, 0x1010), sb_hi = __byte_perm(sb, 0, 0x3232);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            uint32_t qa[4], qb[4];
-            e2m1x8_to_f16x2x4(wa[i], qa);
-            e2m1x8_to_f16x2x4(wb[i], qb);
-            const uint32_t s_a = i < 2 ? sa_lo : sa_hi;
-            const uint32_t s_b = i < 2 ? sb_lo : sb_hi;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                qa[q] = hmul2(qa[q], s_a);
-                qb[q] = hmul2(qb[q], s_b);
-            }
-#pragma unroll
-            for (int t = 0; t < NT; ++t) {
-                const uint4 xv = XQ(t, i);
-                mma_f16_16816(acc[0][t], qa[0], qb[0], qa[1], qb[1], xv.x, xv.y);
-                mma_f16_16816(acc[1][t], qa[2], qb[2], qa[3], qb[3], xv.z, xv.w);
-            }
-        }
-    }
-#undef XQ
-}
-
-template <int FMT, int NT>
-__global__ void __launch_bounds__(kWThreads, 1)
-    sweep_wide_kernel(const __grid_constant__ SweepParams p, const __grid_constant__ CUtensorMap map_codes,
-                      const __grid_constant__ CUtensorMap map_scales,
-                      const __grid_constant__ CUtensorMap map_x) {
-    constexpr int V = Fmt<FMT>::V;
-    constexpr int SLAB = 4 * V;
-    constexpr int CW = kWCW;
-    constexpr int REDUCER = CW, PRODUCER = CW + 1;
-    constexpr int COLS = 8 * NT;          // inputs per tile pass
-    constexpr int kWRedFloats = 16 * COLS;  // one warp's tile partial: 16 rows x COLS inputs
-    constexpr int LPI = 32 / COLS;        // reducer lanes per input (2 or 1)
-    constexpr int NB = kWRedBuffers;  // tile hand-off buffers (one measured slower)
-
-    extern __shared__ __align__(1024) uint8_t smem[];
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
-    uint64_t* empty = full + kMaxStages;
-    uint64_t* red_full = empty + kMaxStages;  // [2]
-    uint64_t* red_empty = red_full + 2;       // [2]
-    // misc: [0] abort, [18..29] tile of each ring slot, [30..31] tile of each reducer buffer
-    int* misc = reinterpret_cast<int*>(red_empty + 2);
-    volatile int* abort_flag = misc;
-    volatile int* slot_tile = misc + 18;
-    volatile int* red_tile = misc + 30;
-    float* red = reinterpret_cast<float*>(misc + 32);  // [NB][CW][16 rows][COLS inputs]
-    const uint32_t head_end = smem_u32(red + NB * CW * kWRedFloats);
-    uint8_t* ring = smem + (((head_end + 1023u) & ~1023u) - smem_u32(smem));
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t K = p.k;
-    const int S = p.stages;
-    const int stage_bytes = p.stage_bytes;
-    const int segs = p.segs;
-    const int NC = p.stages_per_tile;
-    const int M = p.M;
-    const int code_b = wide_code_bytes(segs);
-    const int scale_b = wide_scale_bytes(FMT, segs);
-    const int xsegs = wide_xsegs(FMT, segs);
-    const int64_t T = p.num_tiles;  // 64-row tiles
-
-    if (tid == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], CW);
-        }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&red_full[b], CW);
-            mbar_init(&red_empty[b], 1);
-        }
-        misc[0] = 0;
-        mbar_fence_init();
-    }
-    __syncthreads();
-    pdl_launch_dependents();
-
-    // ------------------------------------------------------------ producer warp
-    if (warp == PRODUCER) {
-        int slot = 0;
-        uint32_t phase = 0;
-        int64_t issued = 0;
-        const uint32_t tx = (uint32_t)(code_b + scale_b + wide_x_bytes(FMT, segs, COLS));
-        bool stop = false;
-        // every stage reads x, which the previous kernel (the f16 copy) may write
-        pdl_wait();
-        int64_t tile = blockIdx.x;
-        int64_t pending = 0;
-        if (lane == 0) pending = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
-        while (tile < T && !stop) {
-            for (int ch = 0; ch < NC; ++ch) {
-                if (!mbar_wait_bounded(&empty[slot], phase ^ 1u, abort_flag)) {
-                    stop = true;
-                    break;
-                }
-                if (lane == 0) {
-                    uint8_t* dst = ring + (size_t)slot * stage_bytes;
-                    slot_tile[slot] = (int)tile;
-                    mbar_arrive_expect_tx(&full[slot], tx);
-                    tma_load_3d(dst, &map_codes, 0, (int)(tile * kWRows), ch * segs, &full[slot]);
-                    if (FMT == 2)
-                        tma_load_2d(dst + code_b, &map_scales, ch * 8 * segs, (int)(tile * kWRows),
-                                    &full[slot]);
-                    tma_load_3d(dst + code_b + scale_b, &map_x, 0, 0, ch * xsegs, &full[slot]);
-                }
-                __syncwarp();
-                ++issued;
-                if (++slot == S) {
-                    slot = 0;
-                    phase ^= 1u;
-                }
-            }
-            tile = __shfl_sync(0xffffffffu, pending, 0);
-            if (lane == 0 && tile < T) pending = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
-        }
-        for (int64_t j = issued > S ? issued - S : 0; j < issued; ++j)
-            if (!mbar_wait_bounded(&full[j % S], (uint32_t)((j / S) & 1), nullptr)) break;
-        if (!stop && mbar_wait_bounded(&empty[slot], phase ^ 1u, abort_flag) && lane == 0) {
-            slot_tile[slot] = -1;
-            mbar_arrive(&full[slot]);
-        }
-        __syncwarp();
-        return;
-    }
-
-    // ------------------------------------------------------------ reducer warp
-    if (warp == REDUCER) {
-        // lane holds input m = lane % COLS and the rows r = h (mod LPI), h = lane / COLS,
-        // of each tile, with a running (max, lowest row) and sum of exp over them
-        const int m = lane % COLS, h = lane / COLS;
-        const bool lp = p.out_logprob != nullptr || p.out_partial != nullptr;
-        pdl_wait();
-        const float gsc = FMT == 2 ? __ldg(p.global_scale) : 1.f;
-        float fa = 1.f, fb = 1.f;  // 2^-xexp[m] as two factors
-        if (FMT != 0 && m < M) {
-            const int e = -__ldg(p.xexp + m);
-            fa = ldexpf(1.f, e / 2);
-            fb = ldexpf(1.f, e - e / 2);
-        }
-        if (lane == 0) {
-            if (FMT == 1) l2_prefetch_share(p.row_scale, p.n * 4);
-            if (p.mask) l2_prefetch_share(p.mask, ((p.M - 1) * p.mask_stride + p.mask_words) * 4);
-        }
-        float best_v = -INFINITY, se = 0.f;
-        int32_t best_i = INT_MAX;
-        int buf = 0;
-        uint32_t fph = 0u;
-        while (true) {
-            if (!mbar_wait_bounded(&red_full[buf], (fph >> buf) & 1u, abort_flag)) break;
-            fph ^= 1u << buf;
-            const int tile_id = red_tile[buf];
-            if (tile_id < 0) break;
-            const int64_t row0 = (int64_t)tile_id * kWRows;
-            float rs_a = 0.f, rs_b = 0.f;  // row scales of rows row0 + lane, row0 + 32 + lane
-            if (FMT == 1) {
-                if (row0 + lane < p.n) rs_a = __ldg(p.row_scale + row0 + lane);
-                if (row0 + 32 + lane < p.n) rs_b = __ldg(p.row_scale + row0 + 32 + lane);
-            }
-            const float* rb = red + (size_t)buf * CW * kWRedFloats;
-#pragma unroll 4
-            for (int j = 0; j < kWRows / LPI; ++j) {
-                const int r = LPI * j + h;  // row within the tile
-                const int rg = r >> 4, rr = r & 15;
-                // the four warps of the row group, in order
-                float a = rb[(rg + 0) * kWRedFloats + rr * COLS + m];
-                a += rb[(rg + 4) * kWRedFloats + rr * COLS + m];
-                a += rb[(rg + 8) * kWRedFloats + rr * COLS + m];
-                a += rb[(rg + 12) * kWRedFloats + rr * COLS + m];
-                float rs = 1.f;
-                if (FMT == 1) rs = __shfl_sync(0xffffffffu, LPI * j < 32 ? rs_a : rs_b, r & 31);
-                const int64_t row = row0 + r;
-                const bool valid = row < p.n && m < M;
-                float l = a;
-                if (FMT != 0) l = (l * fa) * fb;
-                if (FMT == 1) l *= rs;
-                if (FMT == 2) l *= gsc;
-                const bool ok = valid && mask_allows(p, m, row);
-                if (valid && p.out_logits)
-                    p.out_logits[(int64_t)m * p.n + row] = ok ? f32_to_bf16(l) : (uint16_t)0xFF80u;
-                if (lp && ok && l > -INFINITY) {
-                    float v = best_v;
-                    lse_merge(v, se, l, 1.f);
-                }
-                if (ok && (l > best_v || (l == best_v && best_i == INT_MAX))) {
-                    best_v = l;
-                    best_i = (int32_t)row;
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&red_empty[buf]);
-            buf = (buf + 1) % NB;
-        }
-        if (*abort_flag) raise_flag(p.dev_err, DEVFLAG_TIMEOUT);
-        // fold the row parities of each input (two lanes at 16 inputs), then lanes m < M publish
-        if (LPI == 2) {
-            const float ov = __shfl_xor_sync(0xffffffffu, best_v, 16);
-            const int32_t oi = __shfl_xor_sync(0xffffffffu, best_i, 16);
-            const float os = __shfl_xor_sync(0xffffffffu, se, 16);
-            if (lp) {
-                float v = best_v;
-                lse_merge(v, se, ov, os);
-            }
-            if (ov > best_v || (ov == best_v && oi < best_i)) {
-                best_v = ov;
-                best_i = oi;
-            }
-        }
-        Partial* parts = reinterpret_cast<Partial*>(p.partials);
-        if (h == 0 && m < M) parts[(int64_t)blockIdx.x * kPartSlots + m] = Partial{best_v, best_i, se, 0.f};
-        __syncwarp();
-        fence_acq_rel_gpu();  // every publishing lane's store before lane 0's ticket
-        __syncwarp();
-        ticket_and_fold(p, lane, lp);
-        return;
-    }
-
-    // ------------------------------------------------------------ compute warps
-    const int g = lane >> 2, c = lane & 3;
-    const int rg = warp & 3, sub = warp >> 2;
-    const int r0 = tile_row(g);
-    const int rowb = rg * 16 + r0;  // table row of MMA row g within the tile
-    const uint32_t xr = (uint32_t)(r0 & 7) << 4;
-    const uint32_t coff0 = (uint32_t)rowb * 128u + (((uint32_t)c * 16u) ^ xr);
-    const uint32_t coff1 = (uint32_t)rowb * 128u + ((64u + (uint32_t)c * 16u) ^ xr);
-    const uint32_t spitch = 16u * (uint32_t)segs;
-    const uint32_t soff = (uint32_t)code_b + (uint32_t)rowb * spitch + 2u * (uint32_t)c;
-    const int total_slabs = (int)(K / SLAB);
-    const int slabs_per_stage = 2 * segs;
-
-    float acc[2][NT][4];
-#pragma unroll
-    for (int a = 0; a < 2; ++a)
-#pragma unroll
-        for (int t = 0; t < NT; ++t)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[a][t][i] = 0.f;
-
-    int buf = 0;
-    uint32_t eph = 0u;
-    int slot = 0;
-    uint32_t phase = 0;
-    while (true) {
-        if (!mbar_wait_bounded(&full[slot], phase, abort_flag)) break;
-        const int tile = slot_tile[slot];
-        if (tile < 0) break;
-        for (int ch = 0; ch < NC; ++ch) {
-            if (ch > 0 && !mbar_wait_bounded(&full[slot], phase, abort_flag)) break;
-            const uint8_t* st = ring + (size_t)slot * stage_bytes;
-            const uint8_t* xst = st + code_b + scale_b;
-            const int a0 = ch * slabs_per_stage;
-            const int nv = min(slabs_per_stage, total_slabs - a0);
-            for (int l = sub; l < nv; l += 4)
-                slab_mma_wide<FMT, NT>(acc, st + (l >> 1) * (kWRows * 128) + ((l & 1) ? coff1 : coff0),
-                                   st + soff + l * 8, 8u * spitch, xst, l * SLAB + c * V, g);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[slot]);
-            if (++slot == S) {
-                slot = 0;
-                phase ^= 1u;
-            }
-        }
-        mbar_wait_bounded(&red_empty[buf], ((eph >> buf) & 1u) ^ 1u, abort_flag);
-        eph ^= 1u << buf;
-        float* rp = red + (size_t)buf * CW * kWRedFloats + warp * kWRedFloats;
-#pragma unroll
-        for (int t = 0; t < NT; ++t)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int row = (i < 2 ? r0 : r0 + 8);
-                rp[row * COLS + t * 8 + 2 * c + (i & 1)] = acc[0][t][i] + acc[1][t][i];
-                acc[0][t][i] = acc[1][t][i] = 0.f;
-            }
-        if (warp == 0 && lane == 0) red_tile[buf] = tile;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&red_full[buf]);
-        buf = (buf + 1) % NB;
-    }
-    if (mbar_wait_bounded(&red_empty[buf], ((eph >> buf) & 1u) ^ 1u, abort_flag)) {
-        if (warp == 0 && lane == 0) red_tile[buf] = -1;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&red_full[buf]);
-    }
 }
 
 // ---------------------------------------------------------------- tcgen05 sweep
@@ -1805,7 +1454,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
 // scale into f16 -- exact: a code has at most 2 significant bits and a scale 4, and every
 // product lies in [2^-10, 2688] -- and store them with tcgen05.st into tensor memory, one
 // table row per lane; one thread issues tcgen05.mma kind::f16 with A from tensor memory and
-// the f16 copy of x (scaled per input by a power of two, as the wide sweep reads it) as B
+// the f16 copy of x (x16_kernel: scaled per input by a power of two) as B
 // from shared memory, fp32 accumulator in tensor memory. Decoding into tensor memory keeps
 // the 4x larger f16 operand out of shared memory. A tile is H x 128 table rows (H MMA
 // halves sharing every x chunk, so x is read once per 128 H rows); each stage carries the
@@ -2783,91 +2432,6 @@ struct WideGeometry {
     size_t smem;
 };
 
-WideGeometry wide_geometry(int64_t k, int fmt, int cols) {
-    WideGeometry g{};
-    size_t head = (size_t)(2 * kMaxStages + 4) * 8 + 32 * sizeof(int) +
-                  (size_t)kWRedBuffers * kWCW * 16 * cols * sizeof(float);
-    head = ((head + 1023) & ~(size_t)1023) + 1024;
-    const int64_t row_bytes = fmt == 0 ? k * 2 : fmt == 1 ? k : k / 2;
-    const int row_segs = (int)(row_bytes / 128);
-    const long avail = (long)kSmemLimit - (long)head;
-    for (int want = 3; want >= 2 && g.stages < 2; --want) {
-        for (int max_segs = 32; max_segs >= 1; --max_segs) {
-            const int nc = (row_segs + max_segs - 1) / max_segs;
-            const int segs = (row_segs + nc - 1) / nc;
-            const int sb = wide_code_bytes(segs) + wide_scale_bytes(fmt, segs) + wide_x_bytes(fmt, segs, cols);
-            int stages = avail > 0 ? (int)(avail / sb) : 0;
-            if (stages > kMaxStages) stages = kMaxStages;
-            if (stages >= want) {
-                g.segs = segs;
-                g.stages_per_tile = nc;
-                g.stage_bytes = sb;
-                g.stages = stages;
-                break;
-            }
-        }
-    }
-    g.smem = head + (size_t)g.stages * g.stage_bytes;
-    return g;
-}
-
-template <int FMT, int NT>
-cudaError_t launch_wide(const SweepParams& p, cudaStream_t s, SweepLaunch* info) {
-    auto kern = sweep_wide_kernel<FMT, NT>;
-    const WideGeometry geo = wide_geometry(p.k, FMT, 8 * NT);
-    if (geo.stages < 2) return cudaErrorInvalidValue;
-    const int xsegs = wide_xsegs(FMT, geo.segs);
-    CUtensorMap map_codes, map_scales, map_x;
-    cudaError_t e = make_code_map(&map_codes, p.w, p.n, p.row_bytes, geo.segs, kWRows);
-    if (e != cudaSuccess) return e;
-    if (FMT == 2) {
-        if ((e = make_scale_map(&map_scales, p.block_scale, p.n, p.scale_pitch, geo.segs, kWRows)) !=
-            cudaSuccess)
-            return e;
-    } else {
-        map_scales = map_codes;  // unused
-    }
-    const void* xsrc = FMT == 0 ? static_cast<const void*>(p.x) : static_cast<const void*>(p.x16);
-    if ((e = make_x_map(&map_x, xsrc, p.M, p.k, xsegs, 8 * NT)) != cudaSuccess) return e;
-    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)geo.smem)) != cudaSuccess)
-        return e;
-    int dev = 0, sms = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-        return e;
-    SweepParams q = p;
-    q.num_tiles = (p.n + kWRows - 1) / kWRows;
-    q.stages = geo.stages;
-    q.stage_bytes = geo.stage_bytes;
-    q.segs = geo.segs;
-    q.stages_per_tile = geo.stages_per_tile;
-    int64_t grid = sms;
-    if (grid > q.num_tiles) grid = q.num_tiles;
-    if (grid > kMaxGrid) grid = kMaxGrid;
-    if (grid < 1) grid = 1;
-    if (FMT != 0) {  // the f16 copy of x the stages read
-        wide_x16_kernel<<<p.M, 256, 0, s>>>(p.x, (int)p.k, p.x16, p.xexp);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(kWThreads);
-    cfg.dynamicSmemBytes = geo.smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if ((e = cudaLaunchKernelEx(&cfg, kern, q, map_codes, map_scales, map_x)) != cudaSuccess) return e;
-    if (info) {
-        info->grid = (int)grid;
-        info->smem_bytes = (int)geo.smem;
-    }
-    return cudaGetLastError();
-}
-
 template <int FMT, int NT, int MODE, int BD, int G>
 cudaError_t launch_one(const SweepParams& p, cudaStream_t s, SweepLaunch* info) {
     auto kern = sweep_kernel<FMT, NT, MODE, BD, G>;
@@ -3059,7 +2623,7 @@ cudaError_t launch_tc4(const SweepParams& p, cudaStream_t s, SweepLaunch* info) 
     if (grid > q.num_tiles) grid = q.num_tiles;
     if (grid > kMaxGrid) grid = kMaxGrid;
     if (grid < 1) grid = 1;
-    wide_x16_kernel<<<p.M, 256, 0, s>>>(p.x, (int)p.k, p.x16, p.xexp);  // x as f16, per-input 2^e
+    x16_kernel<<<p.M, 256, 0, s>>>(p.x, (int)p.k, p.x16, p.xexp);  // x as f16, per-input 2^e
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)grid);
@@ -3159,15 +2723,13 @@ cudaError_t launch_q4_any(const SweepParams& p, cudaStream_t s, SweepLaunch* inf
     }
 }
 
-// Argmax sweeps that stream x per K chunk -- the tcgen05 sweeps, and for NVFP4 the wide
-// mma.sync sweep -- take FP8 tables from 7 inputs on (measured faster than 16-row tiles
-// from there), BF16 and NVFP4 from 9. NVFP4 runs 9-16 inputs on the wide sweep and 17-32
-// on the tcgen05 sweep with A in tensor memory: measured on a B200, M = 4 / 16 / 32 took
-// 86 / 134 / 258 us on the narrow / wide / wide sweeps and 152 / 186 / 221 us on the
-// tensor-memory sweep, whose decode -> tensor memory -> MMA round trip per 128-column
-// slot (three slots) bounds it.
+// Argmax sweeps that stream x per K chunk -- the tcgen05 sweeps -- take FP8 tables from 7
+// inputs on (measured faster than 16-row tiles from there), BF16 from 9; NVFP4 tables from
+// 17 (3-16 run on the block-scaled sweep, which streams its x terms the same way). The
+// NVFP4 sweep with A in tensor memory (17-32) is bound by its MMA issue: sixteen 128 x 32
+// x 16 MMAs per 256-element slot at ~50 cycles each, with the decode warps waiting on
+// them (221 us at M = 32 on the 131,072 x 5,120 table).
 inline bool streams_x(int M, int fmt) { return fmt == 1 ? M >= 7 : M > 8; }
-inline bool nvfp4_tc4(int M) { return M > 16; }
 
 }  // namespace
 
@@ -3279,12 +2841,13 @@ cudaError_t sweep_launch(const SweepParams& p, int fmt, int mode, cudaStream_t s
         const bool four = p.M > 16;
         if (fmt == 0) return four ? launch_tc<0, 32>(p, s, info) : launch_tc<0, 16>(p, s, info);
         if (fmt == 1) return four ? launch_tc<1, 32>(p, s, info) : launch_tc<1, 16>(p, s, info);
-        if (fmt == 2) return nvfp4_tc4(p.M) ? launch_tc4<32, 2>(p, s, info) : launch_wide<2, 2>(p, s, info);
+        if (fmt == 2) return launch_tc4<32, 2>(p, s, info);  // 17-32 inputs
     }
 #define MTP_SWEEP_CASE(F, NTV, MD) \
     if (fmt == F && (NTV == 2) == two && mode == MD) return launch_one<F, NTV, MD, 0, 0>(p, s, info);
-    // (mode 0 inputs past streams_x went to the tcgen05 / wide sweeps above)
-    MTP_SWEEP_CASE(0, 1, 0) MTP_SWEEP_CASE(1, 1, 0) MTP_SWEEP_CASE(2, 1, 0)
+    // (mode 0 inputs past streams_x went to the tcgen05 sweeps above, NVFP4 ones to the
+    // block-scaled and block-diagonal sweeps)
+    MTP_SWEEP_CASE(0, 1, 0) MTP_SWEEP_CASE(1, 1, 0)
     MTP_SWEEP_CASE(0, 1, 1) MTP_SWEEP_CASE(0, 2, 1)
     MTP_SWEEP_CASE(1, 1, 1) MTP_SWEEP_CASE(1, 2, 1)
     MTP_SWEEP_CASE(2, 1, 1) MTP_SWEEP_CASE(2, 2, 1)
