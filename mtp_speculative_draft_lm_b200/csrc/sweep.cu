@@ -1066,33 +1066,6 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
     }
 }
 
-// ------------------------------------------------------------------ x as f16
-// x [M, k] bf16 -> f16 scaled by 2^e_m (the largest |x| of row m lands in [2^14, 2^15)),
-// as stage_to_f16 does in shared memory for the narrow sweep; the copy the NVFP4 sweep
-// with A in tensor memory reads as its B operand. One CTA per input row.
-__global__ void __launch_bounds__(256) x16_kernel(const uint16_t* __restrict__ x, int k,
-                                                        uint16_t* __restrict__ x16,
-                                                        int32_t* __restrict__ xexp) {
-    __shared__ float red[8];
-    const int m = blockIdx.x, tid = threadIdx.x;
-    const uint16_t* row = x + (int64_t)m * k;
-    float a = 0.f;
-    for (int j = tid; j < k; j += 256) a = fmaxf(a, fabsf(bf16_to_f32(row[j])));
-    for (int o = 16; o; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-    if ((tid & 31) == 0) red[tid >> 5] = a;
-    __syncthreads();
-    a = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) a = fmaxf(a, red[w]);
-    int ex = 0;
-    if (a > 0.f) frexpf(a, &ex);
-    const int e = (a > 0.f) ? 15 - ex : 0;
-    if (tid == 0) xexp[m] = e;
-    const float f1 = ldexpf(1.f, e / 2), f2 = ldexpf(1.f, e - e / 2);
-    for (int j = tid; j < k; j += 256)
-        x16[(int64_t)m * k + j] = f32_to_f16((bf16_to_f32(row[j]) * f1) * f2);
-}
-
 // ---------------------------------------------------------------- tcgen05 sweep
 // BF16 and FP8 tables with 9-32 inputs run the contraction on the tcgen05 tensor cores:
 // one 128 x N x k MMA per 16 (BF16) or 32 (FP8) elements of K, with 128 table rows as A
@@ -1419,395 +1392,6 @@ __global__ void __launch_bounds__(kTThreads, 1)
                 float bv = -INFINITY, bs = 0.f;
                 int32_t bi = INT_MAX;
                 for (int w = 0; w < kTEpiWarps; ++w) {
-                    const float4 f = fold[w * 32 + lane];
-                    const int32_t fi = __float_as_int(f.y);
-                    if (lp) {
-                        float t = bv;
-                        lse_merge(t, bs, f.x, f.z);
-                    }
-                    if (f.x > bv || (f.x == bv && fi < bi)) {
-                        bv = f.x;
-                        bi = fi;
-                    }
-                }
-                reinterpret_cast<Partial*>(p.partials)[(int64_t)blockIdx.x * kPartSlots + lane] =
-                    Partial{bv, bi, bs, 0.f};
-            }
-            __syncwarp();
-            fence_acq_rel_gpu();  // every publishing lane's store before lane 0's ticket
-            __syncwarp();
-            if (*abort_flag && lane == 0) raise_flag(p.dev_err, DEVFLAG_TIMEOUT);
-            ticket_and_fold(p, lane, lp);
-        }
-    }
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem_base, kTmemCols);
-    }
-}
-
-// ---------------------------------------------------------------- NVFP4 tcgen05 sweep
-// NVFP4 tables with 17-32 inputs run the contraction on the tcgen05 tensor cores with A in
-// tensor memory. Eight decode warps (two per lane quarter, each half of every segment)
-// turn each table row's E2M1 codes times their E4M3 block
-// scale into f16 -- exact: a code has at most 2 significant bits and a scale 4, and every
-// product lies in [2^-10, 2688] -- and store them with tcgen05.st into tensor memory, one
-// table row per lane; one thread issues tcgen05.mma kind::f16 with A from tensor memory and
-// the f16 copy of x (x16_kernel: scaled per input by a power of two) as B
-// from shared memory, fp32 accumulator in tensor memory. Decoding into tensor memory keeps
-// the 4x larger f16 operand out of shared memory. A tile is H x 128 table rows (H MMA
-// halves sharing every x chunk, so x is read once per 128 H rows); each stage carries the
-// tile's code segments, their block scales and x's same K range (one TMA box each, 128-byte
-// swizzle for codes and x). A segment (256 elements) of one half fills one of three
-// 128-column A slots, so decoding runs a slot ahead of the MMAs. Four epilogue warps drain
-// the double-buffered accumulators as the tcgen05 sweep does (per input a running max,
-// lowest row, sum of exp), and the CTA partials go through the shared last-CTA fold.
-constexpr int kQDecWarps = 8;    // two per tensor-memory lane quarter, each half of a segment
-constexpr int kQThreads = (2 + kQDecWarps + 4) * 32;  // TMA, MMA, decode, four epilogue warps
-constexpr int kQSlots = 3;      // tensor-memory A slots (one half's segment each)
-constexpr int kQAcol = 128;     // first A column; the accumulators use columns [0, 4N)
-constexpr int kQHead = 3072;    // barriers, misc, factors, fold; then the ring
-
-__host__ __device__ inline int tc4_code_bytes(int H, int segs) { return H * 128 * 128 * segs; }
-__host__ __device__ inline int tc4_scale_bytes(int H, int segs) { return H * 128 * 16 * segs; }
-__host__ __device__ inline int tc4_x_bytes(int N, int segs) { return 4 * segs * N * 128; }
-__host__ __device__ inline int tc4_stage_bytes(int N, int H, int segs) {
-    return tc4_code_bytes(H, segs) + tc4_scale_bytes(H, segs) + tc4_x_bytes(N, segs);
-}
-
-template <int N, int H>
-__global__ void __launch_bounds__(kQThreads, 1)
-    sweep_tc4_kernel(const __grid_constant__ SweepParams p, const __grid_constant__ CUtensorMap map_codes,
-                     const __grid_constant__ CUtensorMap map_scales,
-                     const __grid_constant__ CUtensorMap map_x) {
-    static_assert(N == 16 || N == 32, "16 or 32 input columns");
-    static_assert(H == 1 || H == 2, "one or two 128-row halves");
-    constexpr uint32_t kTmemCols = 512;
-    constexpr int TR = 128 * H;  // table rows per tile
-    extern __shared__ __align__(1024) uint8_t smem[];
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
-    uint64_t* empty = full + kMaxStages;   // the decode warps + the MMA commit
-    uint64_t* afull = empty + kMaxStages;  // [kQSlots] the decode warps
-    uint64_t* aempty = afull + kQSlots;    // [kQSlots] the MMA commit
-    uint64_t* tfull = aempty + kQSlots;    // [2] the tile index posted + the MMA commit
-    uint64_t* tempty = tfull + 2;          // [2] 4 epilogue warps
-    uint64_t* done = tempty + 2;
-    int* misc = reinterpret_cast<int*>(done + 1);
-    volatile int* abort_flag = misc;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 1);
-    volatile int* slot_tile = misc + 2;             // [kMaxStages]
-    volatile int* acc_tile = misc + 2 + kMaxStages;  // [2]
-    float* sfac = reinterpret_cast<float*>(smem + 512);    // [2][32]: 2^-e_m as two factors
-    float4* fold = reinterpret_cast<float4*>(smem + 768);  // [4 warps][32 inputs]
-    uint8_t* ring = smem + kQHead;
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int S = p.stages;
-    const int stage_bytes = p.stage_bytes;
-    const int segs = p.segs;
-    const int NC = p.stages_per_tile;
-    const int M = p.M;
-    const int64_t T = p.num_tiles;
-    const int row_segs = (int)(p.row_bytes / 128);
-    const int code_b = tc4_code_bytes(H, segs), scale_b = tc4_scale_bytes(H, segs);
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kQDecWarps + 1);
-        }
-        for (int k = 0; k < kQSlots; ++k) {
-            mbar_init(&afull[k], kQDecWarps);
-            mbar_init(&aempty[k], 1);
-        }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&tfull[b], 2);
-            mbar_init(&tempty[b], 4);
-        }
-        mbar_init(done, 1);
-        misc[0] = 0;
-        mbar_fence_init();
-    }
-    if (warp == 1) {
-        tmem_alloc(tmem_slot, kTmemCols);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem_base = *tmem_slot;
-    pdl_launch_dependents();
-
-    if (warp == 0) {
-        // ---------------- producer: the tiles' stages, each tagged with its tile
-        int slot = 0;
-        uint32_t phase = 0;
-        int64_t issued = 0;
-        bool stop = false;
-        pdl_wait();  // x's f16 copy comes from the previous grid
-        int64_t tile = blockIdx.x;
-        int64_t pending = 0;
-        if (lane == 0) pending = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
-        while (tile < T && !stop) {
-            for (int ch = 0; ch < NC; ++ch) {
-                if (!mbar_wait_bounded(&empty[slot], phase ^ 1u, abort_flag)) {
-                    stop = true;
-                    break;
-                }
-                if (lane == 0) {
-                    uint8_t* dst = ring + (size_t)slot * stage_bytes;
-                    slot_tile[slot] = (int)tile;
-                    mbar_arrive_expect_tx(&full[slot], (uint32_t)stage_bytes);
-                    tma_load_3d(dst, &map_codes, 0, (int)(tile * TR), ch * segs, &full[slot]);
-                    tma_load_2d(dst + code_b, &map_scales, ch * 8 * segs, (int)(tile * TR), &full[slot]);
-                    tma_load_3d(dst + code_b + scale_b, &map_x, 0, 0, ch * 4 * segs, &full[slot]);
-                }
-                __syncwarp();
-                ++issued;
-                if (++slot == S) {
-                    slot = 0;
-                    phase ^= 1u;
-                }
-            }
-            tile = __shfl_sync(0xffffffffu, pending, 0);
-            if (lane == 0 && tile < T) pending = (int64_t)gridDim.x + atomicAdd(p.ticket + 1, 1u);
-        }
-        for (int64_t j = issued > S ? issued - S : 0; j < issued; ++j)
-            if (!mbar_wait_bounded(&full[j % S], (uint32_t)((j / S) & 1), nullptr)) break;
-        if (!stop && mbar_wait_bounded(&empty[slot], phase ^ 1u, abort_flag) && lane == 0) {
-            slot_tile[slot] = -1;
-            mbar_arrive(&full[slot]);
-        }
-        __syncwarp();
-    } else if (warp == 1) {
-        // ---------------- MMA issuer (lane 0)
-        constexpr uint32_t idesc = idesc_f16(128, N);
-        int slot = 0, aslot = 0, local = 0;
-        uint32_t phase = 0, aphase = 0;
-        while (true) {
-            if (!mbar_wait_bounded(&full[slot], phase, abort_flag)) break;
-            const int tile = slot_tile[slot];
-            const int buf = local & 1;
-            const uint32_t tph = (uint32_t)((local >> 1) & 1);
-            if (!mbar_wait_bounded(&tempty[buf], tph ^ 1u, abort_flag)) break;
-            if (lane == 0) {  // the tile index for the epilogue (its own arrival, release)
-                acc_tile[buf] = tile;
-                mbar_arrive(&tfull[buf]);
-                if (tile < 0) mbar_arrive(&tfull[buf]);  // no MMAs behind the end marker
-            }
-            __syncwarp();
-            if (tile < 0) break;
-            const uint32_t d0 = tmem_base + (uint32_t)(buf * H * N);
-            bool ok = true;
-            for (int ch = 0; ch < NC && ok; ++ch) {
-                if (ch > 0 && !mbar_wait_bounded(&full[slot], phase, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                const uint32_t x0 = smem_u32(ring + (size_t)slot * stage_bytes) + (uint32_t)(code_b + scale_b);
-                const int nseg = min(segs, row_segs - ch * segs);
-                for (int sg = 0; sg < nseg && ok; ++sg) {
-                    for (int h = 0; h < H; ++h) {
-                        if (!mbar_wait_bounded(&afull[aslot], aphase, abort_flag)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        if (lane == 0) {
-                            const uint32_t a0 = tmem_base + (uint32_t)(kQAcol + aslot * 128);
-#pragma unroll
-                            for (int kk = 0; kk < 16; ++kk) {
-                                const uint32_t xa = x0 + (uint32_t)((4 * sg + (kk >> 2)) * (N * 128) + (kk & 3) * 32);
-                                umma_f16_ta(d0 + (uint32_t)(h * N), a0 + (uint32_t)(kk * 8), sdesc_k128(xa), idesc,
-                                            (ch > 0 || sg > 0 || kk > 0) ? 1u : 0u);
-                            }
-                            umma_commit(&aempty[aslot]);  // the slot is free once these have read it
-                        }
-                        __syncwarp();
-                        if (++aslot == kQSlots) {
-                            aslot = 0;
-                            aphase ^= 1u;
-                        }
-                    }
-                }
-                if (lane == 0) umma_commit(&empty[slot]);  // x of the stage is read
-                __syncwarp();
-                if (++slot == S) {
-                    slot = 0;
-                    phase ^= 1u;
-                }
-            }
-            if (lane == 0) umma_commit(&tfull[buf]);  // the accumulators, once complete
-            __syncwarp();
-            ++local;
-            if (!ok) break;
-        }
-        if (lane == 0) umma_commit(done);
-        __syncwarp();
-        mbar_wait_bounded(done, 0u, nullptr);
-    } else if (warp < 2 + kQDecWarps) {
-        // ---------------- decode warps: tensor-memory lane quarter q = warp % 4, one table
-        // row per thread and half (row h * 128 + 32 q + lane of the tile); warp pair
-        // (q, part) splits each segment's four 64-element pieces two and two
-        const int q = warp & 3;
-        const int part = (warp - 2) >> 2;  // 0 or 1
-        int slot = 0, aslot = 0;
-        uint32_t phase = 0, aphase = 0;
-        while (true) {
-            if (!mbar_wait_bounded(&full[slot], phase, abort_flag)) break;
-            if (slot_tile[slot] < 0) break;
-            bool ok = true;
-            for (int ch = 0; ch < NC && ok; ++ch) {
-                if (ch > 0 && !mbar_wait_bounded(&full[slot], phase, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                const uint8_t* st = ring + (size_t)slot * stage_bytes;
-                const int nseg = min(segs, row_segs - ch * segs);
-                for (int sg = 0; sg < nseg && ok; ++sg) {
-                    for (int h = 0; h < H; ++h) {
-                        const int r = h * 128 + q * 32 + lane;  // row of the tile
-                        if (!mbar_wait_bounded(&aempty[aslot], aphase ^ 1u, abort_flag)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        // the row's 128 code bytes (8 chunks, 128-byte swizzle) and 16 scales
-                        const uint8_t* crow = st + (size_t)sg * (TR * 128) + (size_t)r * 128;
-                        // this warp's eight block scales (blocks 8 part .. 8 part + 7)
-                        const uint2 sc = *reinterpret_cast<const uint2*>(
-                            st + code_b + (size_t)r * 16 * segs + sg * 16 + 8 * part);
-                        const uint32_t scw[2] = {sc.x, sc.y};
-                        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) +
-                                               (uint32_t)(kQAcol + aslot * 128);
-#pragma unroll
-                        for (int jj = 0; jj < 2; ++jj) {  // 64 elements (two chunks, four blocks)
-                            const int j = 2 * part + jj;
-                            const uint4 c0 = lds128(crow + (((2 * j) ^ (r & 7)) << 4));
-                            const uint4 c1 = lds128(crow + (((2 * j + 1) ^ (r & 7)) << 4));
-                            const uint32_t wd[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                            // the four blocks' E4M3 scales as f16, each in both halves
-                            const uint32_t s01 = e4m3x2_to_f16x2((uint16_t)(scw[jj] & 0xFFFFu));
-                            const uint32_t s23 = e4m3x2_to_f16x2((uint16_t)(scw[jj] >> 16));
-                            const uint32_t bs[4] = {__byte_perm(s01, 0, 0x1010), __byte_perm(s01, 0, 0x3232),
-                                                    __byte_perm(s23, 0, 0x1010), __byte_perm(s23, 0, 0x3232)};
-                            uint32_t out[32];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                uint32_t o[4];
-                                e2m1x8_to_f16x2x4(wd[i], o);
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) out[4 * i + e] = hmul2(o[e], bs[i >> 1]);
-                            }
-                            tmem_st32(taddr + (uint32_t)(j * 32), out);
-                        }
-                        tmem_st_wait();
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&afull[aslot]);
-                        if (++aslot == kQSlots) {
-                            aslot = 0;
-                            aphase ^= 1u;
-                        }
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[slot]);  // codes and scales of the stage read
-                if (++slot == S) {
-                    slot = 0;
-                    phase ^= 1u;
-                }
-            }
-            if (!ok) break;
-        }
-    } else {
-        // ---------------- epilogue: warp w reads tensor memory lanes 32 (w % 4) + [0, 32)
-        // (one table row per lane); per tile and input the warp folds its 32 rows with
-        // shuffles and lane m keeps input m's running (max, lowest row, sum of exp)
-        const int q = warp & 3;
-        const int ew = warp - (2 + kQDecWarps);  // 0..3
-        const bool lp = p.out_logprob != nullptr || p.out_partial != nullptr;
-        pdl_wait();
-        if (ew == 0) {
-            const int e = lane < M ? -__ldg(p.xexp + lane) : 0;
-            sfac[lane] = ldexpf(1.f, e / 2);
-            sfac[32 + lane] = ldexpf(1.f, e - e / 2);
-        }
-        const float gsc = __ldg(p.global_scale);
-        named_sync(1, 4 * 32);
-        float my_v = -INFINITY, my_s = 0.f;  // input `lane`'s state
-        int32_t my_i = INT_MAX;
-        int local = 0;
-        while (true) {
-            const int buf = local & 1;
-            const uint32_t tph = (uint32_t)((local >> 1) & 1);
-            if (!mbar_wait_bounded(&tfull[buf], tph, abort_flag)) break;
-            const int tile = acc_tile[buf];
-            if (tile < 0) break;
-            tc_fence_after();
-            // one half at a time (registers); the accumulators are released after the last
-#pragma unroll 1
-            for (int h = 0; h < H; ++h) {
-                uint32_t v[N];
-                const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)((buf * H + h) * N);
-                if constexpr (N == 32)
-                    tmem_ld32(ta, v);
-                else
-                    tmem_ld16(ta, v);
-                tmem_ld_wait();
-                if (h == H - 1) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&tempty[buf]);  // the accumulators are free again
-                }
-                const int64_t row = (int64_t)tile * TR + h * 128 + q * 32 + lane;
-                const bool rvalid = row < p.n;
-#pragma unroll
-                for (int m = 0; m < N; ++m) {
-                    if (m >= M) break;  // warp-uniform
-                    const float l = (((__uint_as_float(v[m]) * sfac[m]) * sfac[32 + m])) * gsc;
-                    const bool ok = rvalid && mask_allows(p, m, row);
-                    if (rvalid && p.out_logits)
-                        p.out_logits[(int64_t)m * p.n + row] = ok ? f32_to_bf16(l) : (uint16_t)0xFF80u;
-                    // the 32 rows' (max, lowest row, sum of exp), lanes in a fixed tree
-                    float bv = ok ? l : -INFINITY, bs = (ok && l > -INFINITY) ? 1.f : 0.f;
-                    int32_t bi = ok ? (int32_t)row : INT_MAX;
-#pragma unroll
-                    for (int o = 16; o; o >>= 1) {
-                        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                        const int32_t oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                        const float os = __shfl_xor_sync(0xffffffffu, bs, o);
-                        if (lp) {
-                            float t = bv;
-                            lse_merge(t, bs, ov, os);
-                        }
-                        if (ov > bv || (ov == bv && oi < bi)) {
-                            bv = ov;
-                            bi = oi;
-                        }
-                    }
-                    if (lane == m) {  // rows arrive in increasing order: the earlier wins a tie
-                        if (lp) {
-                            float t = my_v;
-                            lse_merge(t, my_s, bv, bs);
-                        }
-                        if (bv > my_v || (bv == my_v && bi < my_i)) {
-                            my_v = bv;
-                            my_i = bi;
-                        }
-                    }
-                }
-            }
-            ++local;
-        }
-        if (lane < M) fold[ew * 32 + lane] = make_float4(my_v, __int_as_float(my_i), my_s, 0.f);
-        named_sync(1, 4 * 32);
-        if (ew == 0) {
-            if (lane < M) {
-                float bv = -INFINITY, bs = 0.f;
-                int32_t bi = INT_MAX;
-                for (int w = 0; w < 4; ++w) {
                     const float4 f = fold[w * 32 + lane];
                     const int32_t fi = __float_as_int(f.y);
                     if (lp) {
@@ -2314,6 +1898,445 @@ __global__ void __launch_bounds__(kQ4Threads, 1)
     }
 }
 
+// The same contraction for 17-32 inputs (N = 192 term rows) on CTA pairs (2-CTA clusters,
+// cta_group::2): a tile is 256 table rows and one MMA of M = 256 covers both CTAs' 128 rows.
+// The B operand (x's terms) is split between the pair, so each CTA stages half of x's term
+// rows next to its table rows -- 66 KB stages, three deep, where one CTA alone would have
+// room for two. (A paired MMA keeps each SM's tensor pipe as long as a single-CTA one of
+// its 128 rows, so pairs only pay where the x stages are this large.) Roles per CTA: warp 0
+// streams stages (its 128 rows x 2 code segments and its half of x's term codes, both
+// completing on rank 0's barrier; on its own barrier its rows' block scales and all of x's
+// term scales); warps 6-9 write the stage's scale factors into its tensor memory (table
+// rows at columns 4 j + c, x term rows 128 .. at 4 j + 4 + c, K blocks 8 columns apart)
+// and tell rank 0; rank 0's warp 1 issues the MMAs once both CTAs' scale warps are done;
+// warps 2-5 of each CTA drain its 128 rows. Rank 0 claims the tiles at run time and
+// announces each to both CTAs through a small FIFO in each one's shared memory.
+constexpr int kQ4Fifo = 8;  // tiles announced ahead
+__host__ __device__ inline int q4p_stage_bytes(int segs) {  // per CTA, N = 192
+    return ((segs * (16384 + 96 * 128 + 192 * 16 + 2048)) + 1023) & ~1023;
+}
+__host__ __device__ inline int q4p_max_slots(int segs) { return (512 - 192) / (16 * segs * 3); }
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kQ4Threads, 1)
+    sweep_q4p_kernel(const __grid_constant__ SweepParams p, const __grid_constant__ CUtensorMap map_codes,
+                    const __grid_constant__ CUtensorMap map_scales, const __grid_constant__ CUtensorMap map_x,
+                    const __grid_constant__ CUtensorMap map_xs) {
+    constexpr int MP = 32;
+    constexpr int N = q4_n(MP);          // 192
+    constexpr int NH = N / 2;            // x term rows this CTA stages
+    constexpr int G = 2;                 // groups of 128 B rows (scale-factor column blocks)
+    constexpr int NBUF = 1;              // one accumulator (2 N columns would leave no room)
+    constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | (16u << 24);  // M 256
+    constexpr uint32_t kSfCol = NBUF * N;  // accumulators: columns [0, NBUF N)
+    constexpr uint32_t kTmemCols = 512;
+
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);  // rank 0's: both CTAs' codes
+    uint64_t* empty = full + kMaxStages;                 // the MMA commit, to both CTAs
+    uint64_t* sraw = empty + kMaxStages;                 // this CTA's scale bytes landed
+    uint64_t* sfull = sraw + kMaxStages;                 // rank 0's: both CTAs' scale factors written
+    uint64_t* tfull = sfull + kMaxStages;                // [2] the MMA commit, to both CTAs
+    uint64_t* tempty = tfull + 2;                        // [2] rank 0's: both CTAs' epilogues
+    uint64_t* qfull = tempty + 2;                        // [kQ4Fifo]
+    uint64_t* qempty = qfull + kQ4Fifo;                  // [kQ4Fifo] rank 0's
+    uint64_t* done = qempty + kQ4Fifo;
+    int* misc = reinterpret_cast<int*>(done + 1);
+    volatile int* abort_flag = misc;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 1);
+    volatile int* slot_tile = misc + 2;              // [kMaxStages]
+    int* fifo = misc + 2 + kMaxStages;               // [kQ4Fifo]
+    float* sfac = reinterpret_cast<float*>(smem + 768);     // [2][32]: 2^-e_m as two factors
+    float4* fold = reinterpret_cast<float4*>(smem + 1024);  // [4 warps][32 inputs]
+    uint8_t* ring = smem + kQ4Head;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    const int pair = (int)(blockIdx.x >> 1), npairs = (int)(gridDim.x >> 1);
+    const int S = p.stages;
+    const int stage_bytes = p.stage_bytes;
+    const int segs = p.segs;
+    const int NC = p.stages_per_tile;
+    const int M = p.M;
+    const int64_t T = p.num_tiles;  // 256-row tiles
+    // stage layout: table codes (this CTA's 128 rows) | x term codes (its N / 2 rows) |
+    // x term scales [N][16 segs] | table scales [128][16 segs]
+    const int a_bytes = 16384 * segs;
+    const int x_off = a_bytes, x_bytes = NH * 128 * segs;
+    const int xs_off = x_off + x_bytes, xs_bytes = N * 16 * segs;
+    const int as_off = xs_off + xs_bytes, as_bytes = 2048 * segs;
+    const uint32_t code_tx = (uint32_t)(2 * (a_bytes + x_bytes));  // both CTAs', on rank 0's barrier
+    const uint32_t scale_tx = (uint32_t)(xs_bytes + as_bytes);
+    const uint32_t sfa_cols = 16u * (uint32_t)segs;                  // per ring slot
+    const uint32_t slot_cols = sfa_cols * (1u + (uint32_t)G);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+            mbar_init(&sraw[s], 1);
+            mbar_init(&sfull[s], 8);  // four scale warps of each CTA
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 2 * kQ4Epi);
+        }
+        for (int q = 0; q < kQ4Fifo; ++q) {
+            mbar_init(&qfull[q], 1);
+            mbar_init(&qempty[q], 3);  // rank 0's epilogue, rank 1's producer and epilogue
+        }
+        mbar_init(done, 1);
+        misc[0] = 0;
+        mbar_fence_init();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();  // both CTAs' barriers initialised, the pair's tensor memory allocated
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    pdl_launch_dependents();
+
+    if (warp == 0) {
+        // ---------------- producer: rank 0 claims tiles and announces them; both CTAs stream
+        int slot = 0;
+        uint32_t phase = 0;
+        int q = 0;
+        uint32_t qph = 0;
+        int64_t issued = 0;
+        bool stop = false;
+        pdl_wait();  // the x terms come from the previous grid
+        int64_t tile = pair;
+        int64_t pending = 0;
+        if (leader && lane == 0) pending = (int64_t)npairs + atomicAdd(p.ticket + 1, 1u);
+        while (!stop) {
+            bool end;
+            if (leader) {
+                end = tile >= T;
+                if (!mbar_wait_cluster_bounded(&qempty[q], qph ^ 1u, abort_flag)) break;
+                if (lane == 0) {
+                    const int v = end ? -1 : (int)tile;
+                    fifo[q] = v;
+                    st_cluster_u32(map_rank(&fifo[q], 1), (uint32_t)v);
+                    mbar_arrive(&qfull[q]);
+                    mbar_arrive_cluster(map_rank(&qfull[q], 1));
+                }
+                __syncwarp();
+            } else {
+                if (!mbar_wait_cluster_bounded(&qfull[q], qph, abort_flag)) break;
+                const int v = fifo[q];
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(map_rank(&qempty[q], 0));
+                end = v < 0;
+                tile = v;
+            }
+            if (++q == kQ4Fifo) {
+                q = 0;
+                qph ^= 1u;
+            }
+            if (end) break;
+            const int arow = (int)(tile * 256 + rank * 128);
+            for (int ch = 0; ch < NC; ++ch) {
+                if (!mbar_wait_bounded(&empty[slot], phase ^ 1u, abort_flag)) {
+                    stop = true;
+                    break;
+                }
+                if (lane == 0) {
+                    uint8_t* dst = ring + (size_t)slot * stage_bytes;
+                    slot_tile[slot] = (int)tile;
+                    const uint32_t fb = map_rank(&full[slot], 0);
+                    if (leader) mbar_arrive_expect_tx(&full[slot], code_tx);
+                    tma_load_3d_pair(dst, &map_codes, 0, arow, ch * segs, fb);
+                    tma_load_3d_pair(dst + x_off, &map_x, 0, (int)rank * NH, ch * segs, fb);
+                    mbar_arrive_expect_tx(&sraw[slot], scale_tx);
+                    tma_load_2d(dst + xs_off, &map_xs, ch * 8 * segs, 0, &sraw[slot]);
+                    tma_load_2d(dst + as_off, &map_scales, ch * 8 * segs, arow, &sraw[slot]);
+                }
+                __syncwarp();
+                ++issued;
+                if (++slot == S) {
+                    slot = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (leader) {
+                tile = __shfl_sync(0xffffffffu, pending, 0);
+                if (lane == 0 && tile < T) pending = (int64_t)npairs + atomicAdd(p.ticket + 1, 1u);
+            }
+        }
+        // no copy left in flight: rank 0's full barriers count both CTAs' codes; rank 1's
+        // stages are free once the MMAs that read them completed; each CTA's scale bytes
+        for (int64_t j = issued > S ? issued - S : 0; j < issued; ++j) {
+            const uint32_t par = (uint32_t)((j / S) & 1);
+            if (!mbar_wait_bounded(leader ? &full[j % S] : &empty[j % S], par, nullptr)) break;
+            if (!mbar_wait_bounded(&sraw[j % S], par, nullptr)) break;
+        }
+        // the end marker for this CTA's scale warps (and rank 0's MMA thread): a stage tagged
+        // -1, no copy; if rank 0 stopped early, still tell every FIFO reader
+        if (!stop && mbar_wait_bounded(&empty[slot], phase ^ 1u, abort_flag) && lane == 0) {
+            slot_tile[slot] = -1;
+            mbar_arrive(&sraw[slot]);
+            if (leader) mbar_arrive(&full[slot]);
+        }
+        if (leader && stop && mbar_wait_cluster_bounded(&qempty[q], qph ^ 1u, nullptr) && lane == 0) {
+            fifo[q] = -1;
+            st_cluster_u32(map_rank(&fifo[q], 1), 0xFFFFFFFFu);
+            mbar_arrive(&qfull[q]);
+            mbar_arrive_cluster(map_rank(&qfull[q], 1));
+        }
+        __syncwarp();
+    } else if (warp >= 6) {
+        // ---------------- scale factors: warp 6 + q writes lane quarter q of this CTA's tensor
+        // memory -- its table rows' scale words and all x term rows' -- for each stage, then
+        // tells rank 0's MMA thread
+        const int qd = warp - 6;
+        int slot = 0;
+        uint32_t phase = 0;
+        const uint32_t lq = tmem_base + ((uint32_t)(qd * 32) << 16);
+                while (true) {
+            if (!mbar_wait_bounded(&sraw[slot], phase, abort_flag)) break;
+            if (slot_tile[slot] < 0) break;
+            const uint8_t* st = ring + (size_t)slot * stage_bytes;
+            const uint32_t ca = lq + kSfCol + (uint32_t)slot * slot_cols;  // table rows'
+            const uint32_t cx = ca + sfa_cols;                              // x term rows'
+            for (int sg = 0; sg < segs; ++sg) {
+                uint4 ra[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) ra[c] = lds128(st + as_off + (lane + 32 * c) * 16 * segs + 16 * sg);
+                const uint32_t c0 = 16u * (uint32_t)sg;
+                tmem_st4(ca + c0 + 0, ra[0].x, ra[1].x, ra[2].x, ra[3].x);
+                tmem_st4(ca + c0 + 4, ra[0].y, ra[1].y, ra[2].y, ra[3].y);
+                tmem_st4(ca + c0 + 8, ra[0].z, ra[1].z, ra[2].z, ra[3].z);
+                tmem_st4(ca + c0 + 12, ra[0].w, ra[1].w, ra[2].w, ra[3].w);
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    uint4 rx[4];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int r = 128 * g + lane + 32 * c;
+                        rx[c] = r < N ? lds128(st + xs_off + r * 16 * segs + 16 * sg) : make_uint4(0, 0, 0, 0);
+                    }
+                    // K block 4 sg + j at columns 4 G (4 sg + j) + 4 g
+                    const uint32_t b0 = cx + 4u * (uint32_t)G * (4u * (uint32_t)sg) + 4u * (uint32_t)g;
+                    tmem_st4(b0 + 0u * 4u * G, rx[0].x, rx[1].x, rx[2].x, rx[3].x);
+                    tmem_st4(b0 + 1u * 4u * G, rx[0].y, rx[1].y, rx[2].y, rx[3].y);
+                    tmem_st4(b0 + 2u * 4u * G, rx[0].z, rx[1].z, rx[2].z, rx[3].z);
+                    tmem_st4(b0 + 3u * 4u * G, rx[0].w, rx[1].w, rx[2].w, rx[3].w);
+                }
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (leader) mbar_arrive(&sfull[slot]);
+                else mbar_arrive_cluster(map_rank(&sfull[slot], 0));
+            }
+            if (++slot == S) {
+                slot = 0;
+                phase ^= 1u;
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer: one thread of rank 0, for the pair
+        int slot = 0;
+        uint32_t phase = 0;
+        int local = 0;
+        bool stop = !leader;
+        while (!stop) {
+            if (!mbar_wait_bounded(&full[slot], phase, abort_flag)) break;
+            const int tile = slot_tile[slot];
+            if (tile < 0) break;
+            const int buf = NBUF == 2 ? (local & 1) : 0;
+            const uint32_t tph = (uint32_t)((NBUF == 2 ? (local >> 1) : local) & 1);
+            // both CTAs' epilogues have read this accumulator's previous tile
+            if (!mbar_wait_cluster_bounded(&tempty[buf], tph ^ 1u, abort_flag)) break;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + (uint32_t)(buf * N);
+            for (int ch = 0; ch < NC; ++ch) {
+                if ((ch > 0 && !mbar_wait_bounded(&full[slot], phase, abort_flag)) ||
+                    !mbar_wait_cluster_bounded(&sfull[slot], phase, abort_flag)) {
+                    stop = true;
+                    break;
+                }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t st = smem_u32(ring + (size_t)slot * stage_bytes);
+                    const uint32_t ca = tmem_base + kSfCol + (uint32_t)slot * slot_cols;
+                    const uint32_t cx = ca + sfa_cols;
+                    const int kbs = 4 * segs;
+                    for (int kb = 0; kb < kbs; ++kb) {
+                        const uint32_t as = st + (uint32_t)((kb >> 2) * 16384 + (kb & 3) * 32);
+                        const uint32_t xs = st + (uint32_t)(x_off + (kb >> 2) * (NH * 128) + (kb & 3) * 32);
+                        umma_q4_pair(d_tmem, sdesc_k128(as), sdesc_k128(xs), kIdesc, ca + 4u * (uint32_t)kb,
+                                     cx + 4u * (uint32_t)G * (uint32_t)kb, (ch > 0 || kb > 0) ? 1u : 0u);
+                    }
+                    umma_commit_pair(&empty[slot], 3);  // frees both CTAs' stage and scale columns
+                }
+                __syncwarp();
+                if (++slot == S) {
+                    slot = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (lane == 0 && !stop) umma_commit_pair(&tfull[buf], 3);  // both CTAs' accumulators
+            __syncwarp();
+            ++local;
+        }
+        if (leader) {
+            if (lane == 0) umma_commit_pair(done, 1);
+            __syncwarp();
+            mbar_wait_bounded(done, 0u, nullptr);
+        }
+    } else {
+        // ---------------- epilogue: warp w reads tensor memory lanes 32 (w % 4) + [0, 32) of
+        // this CTA (its 128 rows of the tile); the tiles come from the FIFO
+        const int q = warp & 3;
+        const int ew = warp - 2;  // 0..3
+        const int et = threadIdx.x - 64;
+        const bool lp = p.out_logprob != nullptr || p.out_partial != nullptr;
+        pdl_wait();
+        if (ew == 0) {
+            const int e = lane < M ? -__ldg(p.xexp + lane) : 0;
+            sfac[lane] = ldexpf(1.f, e / 2);
+            sfac[32 + lane] = ldexpf(1.f, e - e / 2);
+        }
+        const float gsc = __ldg(p.global_scale);
+        named_sync(1, kQ4Epi * 32);
+        float best_v[MP], se[MP];
+        int32_t best_i[MP];
+#pragma unroll
+        for (int m = 0; m < MP; ++m) {
+            best_v[m] = -INFINITY;
+            best_i[m] = INT_MAX;
+            se[m] = 0.f;
+        }
+        int fq = 0;
+        uint32_t fph = 0;
+        int local = 0;
+        while (true) {
+            if (!mbar_wait_cluster_bounded(&qfull[fq], fph, abort_flag)) break;
+            const int tile = fifo[fq];
+            named_sync(1, kQ4Epi * 32);  // every epilogue thread has read the slot
+            if (et == 0) {
+                if (leader) mbar_arrive(&qempty[fq]);
+                else mbar_arrive_cluster(map_rank(&qempty[fq], 0));
+            }
+            if (++fq == kQ4Fifo) {
+                fq = 0;
+                fph ^= 1u;
+            }
+            if (tile < 0) break;
+            const int buf = NBUF == 2 ? (local & 1) : 0;
+            const uint32_t tph = (uint32_t)((NBUF == 2 ? (local >> 1) : local) & 1);
+            ++local;
+            if (!mbar_wait_bounded(&tfull[buf], tph, abort_flag)) break;
+            tc_fence_after();
+            const int64_t row = (int64_t)tile * 256 + rank * 128 + q * 32 + lane;
+            const bool rvalid = row < p.n;
+            const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * N);
+            // per input, the six term columns 32 t + m weighed by 8^-t, in order of t; 16
+            // inputs at a time (registers)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                float l[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) l[i] = 0.f;
+#pragma unroll
+                for (int t = 0; t < kQ4Terms; ++t) {
+                    uint32_t v[16];
+                    tmem_ld16(ta + (uint32_t)(32 * t + 16 * hh), v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) l[i] = fmaf(__uint_as_float(v[i]), 1.0f / (float)(1 << (3 * t)), l[i]);
+                }
+                if (hh == 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {  // the accumulator is free again (for this CTA)
+                        if (leader) mbar_arrive(&tempty[buf]);
+                        else mbar_arrive_cluster(map_rank(&tempty[buf], 0));
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int m = 16 * hh + i;
+                    if (m >= M) break;
+                    const float lv = ((l[i] * sfac[m]) * sfac[32 + m]) * gsc;
+                    const bool ok = rvalid && mask_allows(p, m, row);
+                    if (rvalid && p.out_logits)
+                        p.out_logits[(int64_t)m * p.n + row] = ok ? f32_to_bf16(lv) : (uint16_t)0xFF80u;
+                    if (lp && ok && lv > -INFINITY) {
+                        float bv = best_v[m];
+                        lse_merge(bv, se[m], lv, 1.f);
+                    }
+                    // each thread's rows arrive in increasing order: the lowest wins a tie
+                    if (ok && (lv > best_v[m] || (lv == best_v[m] && best_i[m] == INT_MAX))) {
+                        best_v[m] = lv;
+                        best_i[m] = (int32_t)row;
+                    }
+                }
+            }
+        }
+        // per input: fold the 32 lanes, then the four warps in order; publish; ticket
+#pragma unroll
+        for (int m = 0; m < MP; ++m) {
+            if (m >= M) break;
+            int32_t bi = best_i[m];
+#pragma unroll
+            for (int o = 16; o; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, best_v[m], o);
+                const int32_t oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                const float os = __shfl_xor_sync(0xffffffffu, se[m], o);
+                if (lp) {
+                    float bv = best_v[m];
+                    lse_merge(bv, se[m], ov, os);
+                }
+                if (ov > best_v[m] || (ov == best_v[m] && oi < bi)) {
+                    best_v[m] = ov;
+                    bi = oi;
+                }
+            }
+            if (lane == 0) fold[ew * 32 + m] = make_float4(best_v[m], __int_as_float(bi), se[m], 0.f);
+        }
+        named_sync(1, kQ4Epi * 32);
+        if (ew == 0) {
+            if (lane < M) {
+                float bv = -INFINITY, bs = 0.f;
+                int32_t bi = INT_MAX;
+                for (int w = 0; w < kQ4Epi; ++w) {
+                    const float4 f = fold[w * 32 + lane];
+                    const int32_t fi = __float_as_int(f.y);
+                    if (lp) {
+                        float t = bv;
+                        lse_merge(t, bs, f.x, f.z);
+                    }
+                    if (f.x > bv || (f.x == bv && fi < bi)) {
+                        bv = f.x;
+                        bi = fi;
+                    }
+                }
+                reinterpret_cast<Partial*>(p.partials)[(int64_t)blockIdx.x * kPartSlots + lane] =
+                    Partial{bv, bi, bs, 0.f};
+            }
+            __syncwarp();
+            fence_acq_rel_gpu();  // every publishing lane's store before lane 0's ticket
+            __syncwarp();
+            if (*abort_flag && lane == 0) raise_flag(p.dev_err, DEVFLAG_TIMEOUT);
+            ticket_and_fold(p, lane, lp);
+        }
+    }
+    tc_fence_before();
+    cluster_sync();  // neither CTA leaves while an MMA, a copy or an arrival may reach it
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, kTmemCols);
+    }
+}
+
+
+
 struct Geometry {
     int kpad;
     int segs;             // 128-byte segments per row per stage
@@ -2571,77 +2594,6 @@ cudaError_t launch_tc(const SweepParams& p, cudaStream_t s, SweepLaunch* info) {
 
 // Stage geometry of the NVFP4 tcgen05 sweep: two 128-byte segments per row per stage when
 // that leaves at least three stages, else one segment (at least two stages).
-WideGeometry tc4_geometry(int64_t k, int N, int H) {
-    WideGeometry g{};
-    const int row_segs = (int)(k / 2 / 128);
-    const long avail = (long)kSmemLimit - (long)kQHead;
-    for (int want = 3; want >= 2 && g.stages < 2; --want) {
-        for (int segs = 2; segs >= 1; --segs) {
-            if (segs > row_segs) continue;
-            const int sb = tc4_stage_bytes(N, H, segs);
-            int stages = avail > 0 ? (int)(avail / sb) : 0;
-            if (stages > kMaxStages) stages = kMaxStages;
-            if (stages >= want) {
-                g.segs = segs;
-                g.stages_per_tile = (row_segs + segs - 1) / segs;
-                g.stage_bytes = sb;
-                g.stages = stages;
-                break;
-            }
-        }
-    }
-    g.smem = (size_t)kQHead + (size_t)g.stages * g.stage_bytes;
-    return g;
-}
-
-template <int N, int H>
-cudaError_t launch_tc4(const SweepParams& p, cudaStream_t s, SweepLaunch* info) {
-    auto kern = sweep_tc4_kernel<N, H>;
-    const WideGeometry geo = tc4_geometry(p.k, N, H);
-    if (geo.stages < 2) return cudaErrorInvalidValue;
-    CUtensorMap map_codes, map_scales, map_x;
-    cudaError_t e = make_code_map(&map_codes, p.w, p.n, p.row_bytes, geo.segs, 128 * H);
-    if (e != cudaSuccess) return e;
-    if ((e = make_scale_map(&map_scales, p.block_scale, p.n, p.scale_pitch, geo.segs, 128 * H)) !=
-        cudaSuccess)
-        return e;
-    if ((e = make_x_map(&map_x, p.x16, p.M, p.k, 4 * geo.segs, N)) != cudaSuccess) return e;
-    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)geo.smem)) != cudaSuccess)
-        return e;
-    int dev = 0, sms = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-        return e;
-    SweepParams q = p;
-    q.num_tiles = (p.n + 128 * H - 1) / (128 * H);
-    q.stages = geo.stages;
-    q.stage_bytes = geo.stage_bytes;
-    q.segs = geo.segs;
-    q.stages_per_tile = geo.stages_per_tile;
-    int64_t grid = sms;
-    if (grid > q.num_tiles) grid = q.num_tiles;
-    if (grid > kMaxGrid) grid = kMaxGrid;
-    if (grid < 1) grid = 1;
-    x16_kernel<<<p.M, 256, 0, s>>>(p.x, (int)p.k, p.x16, p.xexp);  // x as f16, per-input 2^e
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(kQThreads);
-    cfg.dynamicSmemBytes = geo.smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if ((e = cudaLaunchKernelEx(&cfg, kern, q, map_codes, map_scales, map_x)) != cudaSuccess) return e;
-    if (info) {
-        info->grid = (int)grid;
-        info->smem_bytes = (int)geo.smem;
-    }
-    return cudaGetLastError();
-}
 
 WideGeometry q4_geometry(int64_t k, int N) {
     WideGeometry g{};
@@ -2723,6 +2675,79 @@ cudaError_t launch_q4_any(const SweepParams& p, cudaStream_t s, SweepLaunch* inf
     }
 }
 
+WideGeometry q4p_geometry(int64_t k) {
+    WideGeometry g{};
+    const int row_segs = (int)(k / 256);  // 128-byte code segments per row
+    const long avail = (long)kSmemLimit - (long)kQ4Head;
+    for (int segs = 2; segs >= 1 && g.stages == 0; --segs) {
+        if (segs > row_segs) continue;
+        const int sb = q4p_stage_bytes(segs);
+        int stages = avail > 0 ? (int)(avail / sb) : 0;
+        stages = min(stages, min(kMaxStages, q4p_max_slots(segs)));
+        if (stages >= (segs == 2 ? 3 : 2)) {
+            g.segs = segs;
+            g.stages_per_tile = (row_segs + segs - 1) / segs;
+            g.stage_bytes = sb;
+            g.stages = stages;
+        }
+    }
+    g.smem = (size_t)kQ4Head + (size_t)g.stages * g.stage_bytes;
+    return g;
+}
+
+cudaError_t launch_q4p(const SweepParams& p, cudaStream_t s, SweepLaunch* info) {
+    constexpr int MP = 32, N = q4_n(MP);
+    auto kern = sweep_q4p_kernel;
+    const WideGeometry geo = q4p_geometry(p.k);
+    if (geo.stages < 2) return cudaErrorInvalidValue;
+    uint8_t* xcodes = reinterpret_cast<uint8_t*>(p.x16);
+    uint8_t* xscales = xcodes + q4_code_bytes(N, p.k);
+    CUtensorMap map_codes, map_scales, map_x, map_xs;
+    cudaError_t e = make_code_map(&map_codes, p.w, p.n, p.row_bytes, geo.segs, 128);
+    if (e != cudaSuccess) return e;
+    if ((e = make_scale_map(&map_scales, p.block_scale, p.n, p.scale_pitch, geo.segs, 128)) != cudaSuccess)
+        return e;
+    if ((e = make_code_map(&map_x, xcodes, N, p.k / 2, geo.segs, N / 2)) != cudaSuccess) return e;
+    if ((e = make_scale_map(&map_xs, xscales, N, p.k / 16, geo.segs, N)) != cudaSuccess) return e;
+    const size_t smem = geo.smem;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+        cudaSuccess)
+        return e;
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    SweepParams q = p;
+    q.num_tiles = (p.n + 255) / 256;  // pair tiles
+    q.stages = geo.stages;
+    q.stage_bytes = geo.stage_bytes;
+    q.segs = geo.segs;
+    q.stages_per_tile = geo.stages_per_tile;
+    int64_t pairs = sms / 2;
+    if (pairs > q.num_tiles) pairs = q.num_tiles;
+    if (pairs > kMaxGrid / 2) pairs = kMaxGrid / 2;
+    if (pairs < 1) pairs = 1;
+    q4_xterms_kernel<<<MP + 1, 256, 0, s>>>(p.x, p.M, (int)p.k, MP, N, xcodes, xscales, p.xexp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)(2 * pairs));
+    cfg.blockDim = dim3(kQ4Threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if ((e = cudaLaunchKernelEx(&cfg, kern, q, map_codes, map_scales, map_x, map_xs)) != cudaSuccess)
+        return e;
+    if (info) {
+        info->grid = (int)(2 * pairs);
+        info->smem_bytes = (int)smem;
+    }
+    return cudaGetLastError();
+}
+
+
 // Argmax sweeps that stream x per K chunk -- the tcgen05 sweeps -- take FP8 tables from 7
 // inputs on (measured faster than 16-row tiles from there), BF16 from 9; NVFP4 tables from
 // 17 (3-16 run on the block-scaled sweep, which streams its x terms the same way). The
@@ -2743,13 +2768,13 @@ size_t sweep_smem_bytes(int M, int64_t k, int fmt, int* kpad_out, int mode, bool
         if (kpad_out) *kpad_out = g.kpad;
         return g.stages >= 2 ? g.smem : (size_t)kSmemLimit + 1;
     }
-    if (mode == 0 && fmt == 2 && M >= 3 && M <= kQ4MaxM) {  // the block-scaled sweep
-        const WideGeometry w = q4_geometry(k, q4_n(q4_mp(M)));
+    if (mode == 0 && fmt == 2 && M >= 3) {  // the block-scaled sweeps
+        const WideGeometry w = M <= kQ4MaxM ? q4_geometry(k, q4_n(q4_mp(M))) : q4p_geometry(k);
         if (kpad_out) *kpad_out = (int)k;
         return w.stages >= 2 ? w.smem : (size_t)kSmemLimit + 1;
     }
     if (mode == 0 && streams_x(M, fmt)) {  // the tcgen05 sweeps stage x per K chunk
-        const WideGeometry w = fmt == 2 ? tc4_geometry(k, 32, 2) : tc_geometry(k, fmt, M > 16 ? 32 : 16);
+        const WideGeometry w = tc_geometry(k, fmt, M > 16 ? 32 : 16);
         if (kpad_out) *kpad_out = (int)k;
         return w.stages >= 2 ? w.smem : (size_t)kSmemLimit + 1;
     }
@@ -2762,14 +2787,13 @@ int sweep_max_grid() { return kMaxGrid; }
 
 size_t sweep_x16_bytes(int M, int64_t k, int fmt) {
     if (fmt == 2 && M <= 2) return 0;
-    if (fmt == 2 && M <= kQ4MaxM) {  // the block-scaled sweep's x terms: codes, scales, exponents
-        const int N = q4_n(q4_mp(M));
+    if (fmt == 2) {  // the block-scaled sweeps' x terms: codes, scales, exponents
+        const int N = M <= kQ4MaxM ? q4_n(q4_mp(M)) : q4_n(32);
         return q4_code_bytes(N, k) + q4_scale_bytes(N, k) + 1024;
     }
     if (fmt == 0 || !streams_x(M, fmt)) return 0;
-    // FP8: x's two E4M3 planes of 16 or 32 rows; NVFP4 past the block-scaled sweep: the f16
-    // copy of x. Then 1 KB for the per-input exponents.
-    const size_t body = fmt == 1 ? (size_t)2 * (M > 16 ? 32 : 16) * (size_t)k : (size_t)M * (size_t)k * 2;
+    // FP8: x's two E4M3 planes of 16 or 32 rows. Then 1 KB for the per-input exponents.
+    const size_t body = (size_t)2 * (M > 16 ? 32 : 16) * (size_t)k;
     return ((body + 1023) & ~(size_t)1023) + 1024;
 }
 
@@ -2837,11 +2861,11 @@ cudaError_t sweep_launch(const SweepParams& p, int fmt, int mode, cudaStream_t s
     // than the block-scaled sweep there, 67.8 against 71.5 us on the 131,072 x 5,120 table)
     if (fmt == 2 && mode == 0 && p.M <= 2) return launch_one<2, 1, 0, 1, 0>(p, s, info);
     if (fmt == 2 && mode == 0 && p.M <= kQ4MaxM) return launch_q4_any(p, s, info);
+    if (fmt == 2 && mode == 0) return launch_q4p(p, s, info);  // 17-32 inputs, CTA pairs
     if (mode == 0 && streams_x(p.M, fmt)) {
         const bool four = p.M > 16;
         if (fmt == 0) return four ? launch_tc<0, 32>(p, s, info) : launch_tc<0, 16>(p, s, info);
         if (fmt == 1) return four ? launch_tc<1, 32>(p, s, info) : launch_tc<1, 16>(p, s, info);
-        if (fmt == 2) return launch_tc4<32, 2>(p, s, info);  // 17-32 inputs
     }
 #define MTP_SWEEP_CASE(F, NTV, MD) \
     if (fmt == F && (NTV == 2) == two && mode == MD) return launch_one<F, NTV, MD, 0, 0>(p, s, info);

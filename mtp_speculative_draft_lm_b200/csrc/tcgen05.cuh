@@ -239,4 +239,29 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
         : "memory");
 }
 
+// 3-D tile load into this CTA's shared memory completing on the mbarrier at shared::cluster
+// address `bar_cl` (which may be the other CTA's of the pair). No multicast.
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, int x, int y, int z,
+                                                 uint32_t bar_cl) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(z), "r"(bar_cl)
+        : "memory");
+}
+
+// D[tmem of both CTAs] (+)= (A sfa) . (B sfb)^T over the pair: E2M1 operands from both CTAs'
+// shared memory (A: 128 rows each, B: N / 2 rows each), E4M3 scales per 16 elements from
+// each CTA's tensor memory (its A rows', and all N B rows'), K = 64. One thread of rank 0.
+__device__ __forceinline__ void umma_q4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
 }  // namespace mtp

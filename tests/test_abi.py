@@ -135,9 +135,8 @@ def test_lm_head_lp_rejects(lib):
     assert L.mtp_noalloc_scratch_bytes() == wsb + 448 * 1024
     up = lambda b: (b + 1023) // 1024 * 1024
     # quantized tables add x as their sweeps read it (+ 1 KB of exponents): FP8 from 7
-    # inputs, two E4M3 planes of 16 or 32 rows; NVFP4 from 3 to 16 inputs, N = 6 MP rows of
-    # E2M1 terms (MP = 4, 8, 16, rounded up to 16 rows) and their E4M3 block scales, then
-    # an f16 copy of x
+    # inputs, two E4M3 planes of 16 or 32 rows; NVFP4 from 3 inputs, N = 6 MP rows of E2M1
+    # terms (MP = 4, 8, 16, 32, rounded up to 16 rows) and their E4M3 block scales
     fp8 = weight(fmt=1, k=128, rs=OUT)
     assert L.mtp_lm_head_ws_bytes(fp8, 100, 6) == wsb  # FP8 streams x from 7 inputs on
     assert L.mtp_lm_head_ws_bytes(fp8, 100, 7) == wsb + 2 * 16 * 128 + 1024
@@ -145,9 +144,8 @@ def test_lm_head_lp_rejects(lib):
     assert L.mtp_lm_head_ws_bytes(fp8, 100, 17) == wsb + 2 * 32 * 128 + 1024
     nv = weight(fmt=2, k=256, bs=OUT, gs=OUT)
     assert L.mtp_lm_head_ws_bytes(nv, 100, 1) == wsb and L.mtp_lm_head_ws_bytes(nv, 100, 2) == wsb
-    for M, N in ((3, 32), (4, 32), (8, 48), (9, 96), (16, 96)):
+    for M, N in ((3, 32), (4, 32), (8, 48), (9, 96), (16, 96), (17, 192), (32, 192)):
         assert L.mtp_lm_head_ws_bytes(nv, 100, M) == wsb + up(N * 128) + up(N * 16) + 1024, M
-    assert L.mtp_lm_head_ws_bytes(nv, 100, 17) == wsb + up(17 * 256 * 2) + 1024
     assert L.mtp_lm_head_ws_bytes(weight(k=128), 100, 32) == wsb
     # calls past the no-alloc array are rejected before any CUDA call
     noalloc = lambda head, M: st("mtp_lm_head_argmax_noalloc", C.byref(head), 100, B2, M, None,
@@ -155,7 +153,7 @@ def test_lm_head_lp_rejects(lib):
     assert noalloc(weight(fmt=1, k=14336, rs=OUT), 7) == L.MTP_ERR_WORKSPACE
     assert noalloc(weight(fmt=1, k=7168, rs=OUT), 17) == L.MTP_ERR_WORKSPACE
     assert noalloc(weight(fmt=2, k=8704, bs=OUT, gs=OUT), 16) == L.MTP_ERR_WORKSPACE
-    assert noalloc(weight(fmt=2, k=7168, bs=OUT, gs=OUT), 32) == L.MTP_ERR_WORKSPACE
+    assert noalloc(weight(fmt=2, k=4352, bs=OUT, gs=OUT), 32) == L.MTP_ERR_WORKSPACE
     # the table descriptor is checked before its size is looked at: a bad format, a bad k
     # or a missing scale is an argument error, not a workspace one
     assert noalloc(weight(fmt=7, k=128), 12) == L.MTP_ERR_INVALID_ARG
