@@ -184,22 +184,26 @@ mtp_status mtp_combine(const uint16_t* embed, int64_t vocab, const int32_t* toke
  *   dev_err       (device) i32 [1] or NULL
  *   ws            (device) >= mtp_lm_head_ws_bytes(head, n_eff, M) bytes, 16-byte
  *                 aligned, ALL ZERO before the first call; each call leaves its
- *                 counter zero again. It also holds x as the many-input sweeps read
- *                 it, rewritten by each call: for FP8 tables with M >= 7 two E4M3
+ *                 counter zero again. It also holds x as the quantized tables' sweeps
+ *                 read it, rewritten by each call: for FP8 tables with M >= 7 two E4M3
  *                 planes of 16 or 32 rows (2 * 16 * k or 2 * 32 * k bytes), for NVFP4
- *                 with M >= 9 an f16 copy (M * k * 2 bytes).
+ *                 with M >= 3 six E2M1 terms per input (N = 32, 48, 96 or 192 rows of
+ *                 k / 2 code bytes and k / 16 scale bytes).
  * Requires 1 <= M <= 32, 1 <= n_eff <= n; table rows a multiple of 128 bytes (k % 64
  * for BF16, % 128 for FP8, % 256 for NVFP4; the sweep streams 128-byte segments); for
  * M <= 8 (FP8: M <= 6) the staged inputs (M * k * 2 bytes) must leave shared memory for
  * the stream (MTP_ERR_UNSUPPORTED otherwise; more inputs stream x per K chunk instead).
  * Results are bit-identical for every M within BF16 1-8, 9-16, 17-32; FP8 1-6, 7-16,
- * 17-32; NVFP4 1-2, 3-8, 9-16, 17-32, whose sweeps sum the same products in different
- * fixed orders. BF16 tables from 9 inputs, FP8 from 7 and NVFP4 from 17 run on the
- * tcgen05 tensor cores (NVFP4 9-16 on legacy MMAs with x streamed per K chunk, decoding
- * to f16 in registers); there x enters FP8 products as two E4M3 terms whose sum is x
- * exactly except for elements below 2^-9 of the input's largest |x|, which keep an
- * absolute error of at most 2^-17 of that largest |x|. With a grammar mask and up to 8
- * inputs only the table rows that some input's mask allows are read.
+ * 17-32; NVFP4 1-2, 3-16, 17-32, whose sweeps sum the same products in different fixed
+ * orders. BF16 tables from 9 inputs, FP8 from 7 and NVFP4 from 3 run on the tcgen05
+ * tensor cores. There x enters FP8 products as two E4M3 terms whose sum is x exactly
+ * except for elements below 2^-9 of the input's largest |x|, which keep an absolute error
+ * of at most 2^-17 of that largest |x|; NVFP4 products take the table's E2M1 codes and
+ * E4M3 block scales as stored (block-scaled FP4 MMAs) and x as six E2M1 terms per
+ * 16-element block with a power-of-two scale, whose sum is x exactly for every element
+ * within 9 binades of its block's largest |x| and within 2^-17 of that largest |x|
+ * otherwise. With a grammar mask and up to 8 inputs only the table rows that some
+ * input's mask allows are read.
  * ------------------------------------------------------------------------------ */
 size_t mtp_lm_head_ws_bytes(const mtp_weight* head, int64_t n_eff, int32_t M);
 mtp_status mtp_lm_head_argmax(const mtp_weight* head, int64_t n_eff, const uint16_t* x,
@@ -437,9 +441,9 @@ mtp_status mtp_debug_kv_write(const uint16_t* k_rot, const uint16_t* v, int64_t 
  * (983,296: a 256-byte header, 16-byte partials of up to 1,024 CTAs x 32 input rows and
  * 448 KB for x in the form the quantized tables' sweeps read it) held on every GPU that
  * loads the library until the process exits. Calls whose mtp_lm_head_ws_bytes exceeds
- * it return MTP_ERR_WORKSPACE: BF16 tables run at every M up to 32; FP8 and NVFP4
- * tables at every M up to 32 with k <= 7,152, NVFP4 with up to 16 inputs and
- * k <= 8,448.
+ * it return MTP_ERR_WORKSPACE: BF16 tables run at every M up to 32; FP8 tables at every
+ * M up to 32 with k <= 7,152; NVFP4 tables with up to 16 inputs and k <= 8,448, with
+ * 17-32 inputs and k <= 4,096.
  *  - The first call made with a device current looks up that array's device address.
  *    Under the CUDA runtime's lazy module loading (the default since CUDA 12.2) that
  *    look-up is also when the array is committed on the device, so make the first call
