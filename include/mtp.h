@@ -273,7 +273,8 @@ mtp_status mtp_lm_head_argmax_lp(const mtp_weight* head, int64_t n_eff, const ui
  *   embed (device) bf16 [vocab, h]; token_ids (device) i32 [M] (a bad id reads as a zero row
  *   and sets MTP_DEVFLAG_BAD_TOKEN); hidden (device) bf16 [M, h]; w_norm_* (device) bf16 [h];
  *   fc (device) bf16 [h, 2h]; head (device) bf16 [>= n_eff, h], rows packed at h;
- *   out_y (device) bf16 [M, h] or NULL: y, for instance the next step's hidden rows;
+ *   out_y (device) bf16 [M, h] or NULL: y, for instance the next step's hidden rows (it
+ *   must not overlap hidden: MTP_ERR_INVALID_ARG);
  *   out_idx (device) i32 [M]; out_val (device) f32 [M] or NULL; dev_err i32 [1] or NULL.
  * One thread-block cluster does the whole step (no workspace), so it suits heads that sit
  * in L2 (a few MB, as the tiny draft head's 2 MB); a large head belongs to

@@ -332,6 +332,11 @@ mtp_status mtp_draft_step(const uint16_t* embed, int64_t vocab, const int32_t* t
         !aligned(out_y, 2) || !aligned(out_idx, 4) || !aligned(out_val, 4) || !aligned(mask, 4) ||
         !aligned(dev_err, 4))
         return MTP_ERR_INVALID_ARG;
+    if (out_y) {  // each CTA writes its slice of y while others may still read hidden
+        const uintptr_t y0 = reinterpret_cast<uintptr_t>(out_y), x0 = reinterpret_cast<uintptr_t>(hidden);
+        const uintptr_t bytes = (uintptr_t)M * (uintptr_t)h * 2u;
+        if (y0 < x0 + bytes && x0 < y0 + bytes) return MTP_ERR_INVALID_ARG;
+    }
     return from_cuda(mtp::draft_step_launch(embed, vocab, token_ids, hidden, M, h, w_norm_embed,
                                             w_norm_hidden, eps, norm_mode, fc, head, n_eff, mask,
                                             mask_words,

@@ -307,9 +307,10 @@ def test_wait_timeout_rejects(lib):
 
 
 def test_draft_step_rejects(lib):
-    def ds(M=1, h=256, embed=A, head=B2, mask=None, mw=0, ms=0, idx=OUT, n=100, mode=0):
-        return st("mtp_draft_step", embed, 100, OUT, A, M, h, A, A, 1e-6, mode, A, head, n, mask,
-                  mw, ms, None, idx, None, None, None)
+    def ds(M=1, h=256, embed=A, head=B2, mask=None, mw=0, ms=0, idx=OUT, n=100, mode=0, y=None,
+           hid=A):
+        return st("mtp_draft_step", embed, 100, OUT, hid, M, h, A, A, 1e-6, mode, A, head, n, mask,
+                  mw, ms, y, idx, None, None, None)
     assert ds(embed=None) == L.MTP_ERR_INVALID_ARG
     assert ds(idx=None) == L.MTP_ERR_INVALID_ARG
     assert ds(h=260) == L.MTP_ERR_INVALID_ARG       # h % 8
@@ -319,6 +320,9 @@ def test_draft_step_rejects(lib):
     assert ds(M=5) == L.MTP_ERR_UNSUPPORTED         # up to 4 inputs
     assert ds(h=2048) == L.MTP_ERR_UNSUPPORTED      # up to hidden 1024
     assert ds(head=B2 + 8) == L.MTP_ERR_INVALID_ARG  # 16-byte aligned head
+    assert ds(y=A) == L.MTP_ERR_INVALID_ARG          # out_y must not overlap hidden
+    assert ds(y=A + 510, h=256) == L.MTP_ERR_INVALID_ARG
+    assert ds(y=A - 510, h=256) == L.MTP_ERR_INVALID_ARG
 
 
 def test_paged_decode_attn_rejects(lib):

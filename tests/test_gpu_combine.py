@@ -211,17 +211,24 @@ def test_draft_step_one_plus_w(orc, M):
         assert_argmax(int(idx[m]), ref_l[m])
 
 
-@pytest.mark.parametrize("h,vocab", [(64, 1000), (512, 3333), (1024, 5000)])
-def test_draft_step_other_widths(orc, h, vocab):
-    d = draft(2, seed=31 + h, h=h, vocab=vocab)
+# One input with h <= 256 and at most 256 head rows per CTA takes the register form (the
+# weights held as MMA fragments); the rest, and every M > 1, the staged form (h 512:
+# staged in shared memory; h 1024 with 5000 rows: read through L1). h 8 and 24 leave lanes
+# without a k piece; 1000 rows leave a ragged last tile; 5000 rows at h 256 go staged.
+@pytest.mark.parametrize("h,vocab,M", [(64, 1000, 1), (64, 1000, 2), (512, 3333, 1), (512, 3333, 2),
+                                       (1024, 5000, 1), (1024, 5000, 2), (8, 300, 1), (24, 777, 1),
+                                       (24, 777, 3), (256, 5000, 1), (256, 4000, 1)])
+def test_draft_step_other_widths(orc, h, vocab, M):
+    d = draft(M, seed=31 + h + vocab, h=h, vocab=vocab)
     idx, val, y, err = gpu_draft_step(d)
     assert err == 0
     ref_y, _, _ = orc.combine(d["embed"], d["tokens"].numpy(), d["hidden"], d["w_norm_embed"],
                               d["w_norm_hidden"], d["eps"], d["fc"])
     assert_close(bf16_bits_to_f64(y), bf16_bits_to_f64(ref_y), "y")
     ref_l, _, _, _ = orc.lm_head_argmax(0, d["lm_head"], d["h"], y)
-    for m in range(2):
+    for m in range(M):
         assert_argmax(int(idx[m]), ref_l[m])
+        assert_close([val[m]], [ref_l[m].max()], "out_val")
 
 
 def test_draft_step_mask_and_flags(orc):
@@ -243,6 +250,57 @@ def test_draft_step_mask_and_flags(orc):
     assert idx[1] == 0 and val[1] == -np.inf
     for m in (0, 2):
         assert_argmax(int(idx[m]), ref_l[m], allowed[m])
+
+
+@pytest.mark.parametrize("keep", [0.1, 0.0])
+def test_draft_step_mask_one_input(orc, keep):
+    """One input (the register form) under a sparse mask, and under a mask allowing nothing
+    (index 0, -inf, the empty-mask flag)."""
+    d = draft(1, seed=91)
+    allowed, words = synth.keep_mask(23, 1, d["vocab"], keep)
+    W = words.shape[1]
+    idx, val, y, err = gpu_draft_step(d, mask=words.reshape(-1), mask_words=W, stride=W)
+    ref_l, _, _, _ = orc.lm_head_argmax(0, d["lm_head"], d["h"], y)
+    if allowed[0].any():
+        assert err == 0
+        assert_argmax(int(idx[0]), ref_l[0], allowed[0])
+    else:
+        assert err == L.MTP_DEVFLAG_EMPTY_MASK
+        assert idx[0] == 0 and val[0] == -np.inf
+
+
+def test_draft_step_bad_token_one_input(orc):
+    """One input (the register form) with a token id outside the vocabulary: a zero
+    embedding row and the bad-token flag."""
+    d = draft(1, seed=92)
+    toks = np.asarray([d["vocab"] + 5], np.int32)
+    idx, val, y, err = gpu_draft_step(d, tokens=toks)
+    assert err == L.MTP_DEVFLAG_BAD_TOKEN
+    ref_y, _, _ = orc.combine(d["embed"], toks, d["hidden"], d["w_norm_embed"], d["w_norm_hidden"],
+                              d["eps"], d["fc"])
+    assert_close(bf16_bits_to_f64(y), bf16_bits_to_f64(ref_y), "y")
+    ref_l, _, _, _ = orc.lm_head_argmax(0, d["lm_head"], d["h"], y)
+    assert_argmax(int(idx[0]), ref_l[0])
+
+
+def test_draft_step_unaligned_norm_weights(orc):
+    """Norm weights only 2-byte aligned (a view one element into a buffer): one input then
+    takes the staged form, with the same results as the oracle."""
+    d = draft(1, seed=93)
+    dd = {k: (to_dev_u16(v) if isinstance(v, np.ndarray) and v.dtype == np.uint16 else v)
+          for k, v in d.items()}
+    for key in ("w_norm_embed", "w_norm_hidden"):
+        buf = torch.empty((d["h"] + 1,), dtype=dd[key].dtype, device="cuda")
+        buf[1:] = dd[key]
+        dd[key] = buf[1:]
+        assert dd[key].data_ptr() % 16 == 2
+    idx, val, y, err = gpu_draft_step(d, dd=dd)
+    assert err == 0
+    ref_y, _, _ = orc.combine(d["embed"], d["tokens"].numpy(), d["hidden"], d["w_norm_embed"],
+                              d["w_norm_hidden"], d["eps"], d["fc"])
+    assert_close(bf16_bits_to_f64(y), bf16_bits_to_f64(ref_y), "y")
+    ref_l, _, _, _ = orc.lm_head_argmax(0, d["lm_head"], d["h"], y)
+    assert_argmax(int(idx[0]), ref_l[0])
 
 
 def test_draft_step_chain_eager_and_graph(orc):
