@@ -13,17 +13,24 @@
 // Design (B200, HBM-bound: every cached K and V byte is read once): CTA (g, piece) takes
 // kv head g over a contiguous range of positions (as many CTAs as the SMs hold at once), in
 // sub-pieces of 64 positions that a three-stage ring of 16-byte asynchronous copies
-// brings into shared memory (rows of a missing block zero-filled). Both contractions run
-// on the tensor cores (mma.sync m16n8k16, f16 operands, fp32 accumulators): the scores as
-// K[64 positions, hd] . Q^T, with E4M3 K decoded exactly to f16 and each query head in
-// f16 scaled by a power of two (exact), then an online softmax over the sub-pieces (fp32
-// running maximum and sum) and the weighted V sum as V^T . W^T, the weights
-// exp(s - max) in (0, 1] rounded to f16 (the same rounded weights in the sum of exps).
-// Each CTA writes its heads' (max, sum, weighted V sum); a second kernel merges the pieces
-// of each head in a fixed order (deterministic) and writes bf16. Rows whose block is
-// missing or out of range are skipped and set MTP_DEVFLAG_BAD_SLOT.
+// brings into shared memory (rows of a missing block zero-filled). Warp w owns positions
+// 16 w + [0, 16) of every sub-piece and runs its own online softmax (fp32 running maximum
+// and sum per query head) and its own weighted V sum over all head dims, so the warps
+// meet once per sub-piece (the ring) and once at the end. Both contractions run on the
+// tensor cores (mma.sync m16n8k16, f16 operands, fp32 accumulators): the scores as
+// K[16 positions, hd] . Q^T, with E4M3 K decoded exactly to f16 and each query head in
+// f16 scaled by a power of two (exact); the weights exp(s - max) in (0, 1] rounded to f16
+// (the same rounded weights in the sum of exps) go from the score accumulators to the B
+// operand of V^T . W^T in registers (an 8 x 8 transpose, movmatrix). At the end the four
+// warps' states merge in a fixed order into the CTA's (max, sum, weighted V sum) per head;
+// a second kernel merges the pieces of each head in a fixed order (deterministic) and
+// writes bf16. Rows whose block is missing or out of range are skipped and set
+// MTP_DEVFLAG_BAD_SLOT.
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -37,7 +44,6 @@ constexpr int kAStages = 3;
 constexpr int kAMaxGroup = 16;  // query heads per kv head
 constexpr int kAMaxHd = 256;
 constexpr int kAMaxPieces = 1024;  // pieces per kv head (the merge keeps a factor per piece)
-constexpr int kWPitch = kSP + 8;   // f16 weights per head row in shared memory
 
 struct AttnParams {
     const uint16_t* q;  // [nq, hd] bf16
@@ -69,43 +75,74 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// Transpose of an 8 x 8 matrix of 16-bit values in the mma fragment layout (lane holds
+// row lane / 4, columns 2 (lane % 4) + {0, 1}).
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t v) {
+    uint32_t r;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(v));
+    return r;
+}
+
 __device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.f16x2.f32 %0, %2, %1;" : "=r"(r) : "f"(lo), "f"(hi));
     return r;
 }
 
-template <int HD>
-__host__ __device__ constexpr int attn_row_pitch() { return HD + 16; }  // bank-conflict-free
+// Row pitch of a staged cache row: HD + 16 bytes with the 16-byte copies (bank-conflict
+// free); HD = 128 bytes, 128-byte swizzled, with the tensor copies.
+template <int HD, bool TMA>
+__host__ __device__ constexpr int attn_row_pitch() { return TMA ? HD : HD + 16; }
 template <int HD>
 __host__ __device__ constexpr int attn_q_pitch() { return HD + 8; }     // f16 elements
 
-template <int HD>
+template <int HD, bool TMA>
 __host__ __device__ constexpr size_t attn_smem_bytes() {
-    return (size_t)kAStages * 2 * kSP * attn_row_pitch<HD>()  // K and V rings
+    return (size_t)kAStages * 2 * kSP * attn_row_pitch<HD, TMA>()  // K and V rings
            + (size_t)kAMaxGroup * attn_q_pitch<HD>() * 2         // q in f16
-           + (size_t)kAMaxGroup * kWPitch * 2                    // weights in f16
            + (size_t)kAStages * kSP * 4                          // row valid flags
            + (size_t)2 * 4 * kAMaxGroup * 4                      // per-warp max and sum
-           + (size_t)kAMaxGroup * 4;                             // per-head score factor
+           + (size_t)kAMaxGroup * 4                              // per-head score factor
+           + (TMA ? (size_t)kAStages * 8 + 1024 : 0);            // stage barriers, alignment
 }
 
-template <int HD, int NT>
-__global__ void __launch_bounds__(kAThreads) attn_piece_kernel(const __grid_constant__ AttnParams p) {
-    extern __shared__ __align__(16) uint8_t smem[];
-    constexpr int RP = attn_row_pitch<HD>();
+__device__ __forceinline__ void tma_load_3d_attn(void* dst, const CUtensorMap* map, int x, int y, int z,
+                                                 uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// TMA (HD = 128, block size a multiple of 16): warp 0 brings each sub-piece in as four
+// tensor copies of 16 cache rows (one per 16 positions, each inside one block) per K and
+// V, completing on the stage's barrier; rows of a missing block and past the sequence are
+// zero-filled by the warp (a group cut by the sequence's end is copied row by row).
+template <int HD, int NT, bool TMA>
+__global__ void __launch_bounds__(kAThreads) attn_piece_kernel(const __grid_constant__ AttnParams p,
+                                                               const __grid_constant__ CUtensorMap kmap,
+                                                               const __grid_constant__ CUtensorMap vmap) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    static_assert(!TMA || HD == 128, "tensor copies: 128-byte rows");
+    // (the tensor copies' 128-byte swizzle wants 1024-byte aligned stages)
+    uint8_t* smem = TMA ? smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u) : smem_raw;
+    constexpr int RP = attn_row_pitch<HD, TMA>();
     constexpr int QP = attn_q_pitch<HD>();
     constexpr int KC = HD / 16;          // 16-byte pieces of a row, and MMA K chunks
-    constexpr int MT = HD / 64;          // 16-dim tiles of the V sum per warp
     uint8_t* kring = smem;                                          // [stages][kSP][RP]
     uint8_t* vring = kring + kAStages * kSP * RP;                   // [stages][kSP][RP]
     uint16_t* qh = reinterpret_cast<uint16_t*>(vring + kAStages * kSP * RP);  // [16][QP] f16
-    uint16_t* wsm = qh + kAMaxGroup * QP;                           // [16][kWPitch] f16
-    int* valid = reinterpret_cast<int*>(wsm + kAMaxGroup * kWPitch);  // [stages][kSP]
+    int* valid = reinterpret_cast<int*>(qh + kAMaxGroup * QP);       // [stages][kSP]
     float* redm = reinterpret_cast<float*>(valid + kAStages * kSP);   // [4][16]
     float* redl = redm + 4 * kAMaxGroup;                               // [4][16]
     float* hfac = redl + 4 * kAMaxGroup;                               // [16]
+    uint64_t* fullb = reinterpret_cast<uint64_t*>(hfac + kAMaxGroup);  // [stages] (TMA)
+    // byte offset of 16-byte chunk c of staged row r (the swizzle of the tensor copies)
+    auto chunk_at = [](int r, int c) -> int { return TMA ? r * RP + ((c ^ (r & 7)) << 4) : r * RP + (c << 4); };
 
+    static_assert((size_t)kAStages * 2 * kSP * RP >= (size_t)4 * kAMaxGroup * HD * 4,
+                  "the ring holds the warps' sums at the end");
     const int g = blockIdx.x, piece = blockIdx.y, tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31, gid = lane >> 2, tig = lane & 3;
     const int G = p.group;
@@ -117,9 +154,20 @@ __global__ void __launch_bounds__(kAThreads) attn_piece_kernel(const __grid_cons
     // copies of sub-piece i into ring stage i % 3 (positions past the piece: invalid)
     // 32-bit position arithmetic (seq_len <= 2^21); a power-of-two block size shifts
     const int pend32 = (int)pend;
-    // copies of sub-piece i: thread t takes half of row t / 2 (its slot looked up once)
+    // copies of sub-piece i: thread t takes half of row t / 2 (its slot looked up once).
+    // The block-table entry of the thread's row in the next sub-piece is loaded one issue
+    // ahead, so that its latency is not paid in front of the copies.
     static_assert(kAThreads == 2 * kSP, "two threads per row of a sub-piece");
-    auto issue = [&](int i) {
+    auto load_blk = [&](int i) -> int32_t {  // -1: no readable block (or past the piece)
+        const int pos = (int)pbeg + i * kSP + (tid >> 1);
+        if (i >= nsub || pos >= pend32) return -1;
+        const int b = p.bs_shift >= 0 ? pos >> p.bs_shift : pos / p.block_size;
+        return b < p.n_table ? __ldg(p.block_table + b) : -1;
+    };
+    int32_t blk_next = load_blk(0);
+    auto issue_cp = [&](int i) {
+        const int32_t blk = blk_next;
+        blk_next = load_blk(i + 1);
         if (i < nsub) {
             const int st = i % kAStages;
             const int r = tid >> 1, hf = tid & 1;
@@ -127,11 +175,8 @@ __global__ void __launch_bounds__(kAThreads) attn_piece_kernel(const __grid_cons
             int64_t slot = -1;
             if (pos < pend32) {
                 const int b = p.bs_shift >= 0 ? pos >> p.bs_shift : pos / p.block_size;
-                if (b < p.n_table) {
-                    const int32_t blk = __ldg(p.block_table + b);
-                    if (blk >= 0 && blk < p.num_blocks)
-                        slot = (int64_t)blk * p.block_size + (pos - b * p.block_size);
-                }
+                if (b < p.n_table && blk >= 0 && blk < p.num_blocks)
+                    slot = (int64_t)blk * p.block_size + (pos - b * p.block_size);
                 if (slot < 0 && hf == 0) raise_flag(p.dev_err, DEVFLAG_BAD_SLOT);
             }
             if (hf == 0) valid[st * kSP + r] = slot >= 0;
@@ -152,8 +197,72 @@ __global__ void __launch_bounds__(kAThreads) attn_piece_kernel(const __grid_cons
         }
         cp_async_commit();  // one group per sub-piece, empty past the end
     };
-    issue(0);
-    issue(1);
+    if (TMA && tid == 0) {
+        for (int b = 0; b < kAStages; ++b) mbar_init(&fullb[b], 1);
+        mbar_fence_init();
+    }
+    if (TMA) __syncthreads();
+    // tensor copies of sub-piece i (warp 0): lane q < 4 takes positions 16 q + [0, 16)
+    auto issue_tma = [&](int i) {
+        if (i >= nsub) return;
+        const int st = i % kAStages;
+        const int pos0 = (int)pbeg + i * kSP + 16 * (lane & 3);
+        const int nv = lane < 4 ? max(0, min(16, pend32 - pos0)) : 0;  // rows before the end
+        int row0 = -1;                                                  // first cache row
+        if (nv > 0) {
+            const int b = p.bs_shift >= 0 ? pos0 >> p.bs_shift : pos0 / p.block_size;
+            const int32_t blk = b < p.n_table ? __ldg(p.block_table + b) : -1;
+            if (blk >= 0 && blk < p.num_blocks) row0 = blk * p.block_size + (pos0 - b * p.block_size);
+            else raise_flag(p.dev_err, DEVFLAG_BAD_SLOT);
+        }
+        const uint32_t whole = __ballot_sync(0xffffffffu, nv == 16 && row0 >= 0);  // groups by tensor copy
+        uint8_t* kst = kring + st * kSP * RP;
+        uint8_t* vst = vring + st * kSP * RP;
+        // the other groups: zeros, and the readable rows of a group cut by the end
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+            if ((whole >> q) & 1u) continue;
+            const int qnv = __shfl_sync(0xffffffffu, nv, q);
+            const int qrow = __shfl_sync(0xffffffffu, row0, q);
+            for (int u = lane; u < 16 * KC; u += 32) {  // 16 rows x KC chunks
+                const int r = u / KC, c = u - r * KC;
+                uint4 kv = make_uint4(0, 0, 0, 0), vv = kv;
+                if (qrow >= 0 && r < qnv) {
+                    const int64_t off = ((int64_t)(qrow + r) * p.nkv + g) * HD + 16 * c;
+                    kv = *reinterpret_cast<const uint4*>(p.k_cache + off);
+                    vv = *reinterpret_cast<const uint4*>(p.v_cache + off);
+                }
+                *reinterpret_cast<uint4*>(kst + chunk_at(16 * q + r, c)) = kv;
+                *reinterpret_cast<uint4*>(vst + chunk_at(16 * q + r, c)) = vv;
+            }
+        }
+        // row valid flags: row 16 q + j of the sub-piece
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int r = lane + 32 * h, q = r >> 4;
+            const int qnv = __shfl_sync(0xffffffffu, nv, q);
+            const int qrow = __shfl_sync(0xffffffffu, row0, q);
+            valid[st * kSP + r] = qrow >= 0 && (r & 15) < qnv;
+        }
+        __syncwarp();  // the warp's stores above, before the barrier's arrival below
+        // (and every earlier access to the stage through plain loads and stores ordered
+        // before the tensor copies rewrite it)
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        if (lane == 0) mbar_arrive_expect_tx(&fullb[st], (uint32_t)__popc(whole) * 2u * 16u * HD);
+        __syncwarp();
+        if ((whole >> lane) & 1u) {
+            tma_load_3d_attn(kst + 16 * lane * RP, &kmap, 0, g, row0, &fullb[st]);
+            tma_load_3d_attn(vst + 16 * lane * RP, &vmap, 0, g, row0, &fullb[st]);
+        }
+    };
+    auto issue = [&](int i) {
+        if constexpr (TMA) {
+            if (warp == 0) issue_tma(i);
+        } else {
+            issue_cp(i);
+        }
+    };
+    for (int i = 0; i < kAStages - 1; ++i) issue(i);
 
     // the group's query heads in f16, each scaled by 2^e so its largest |q| lies in
     // [2^14, 2^15) (exact: a bf16 value has 8 significant bits); heads past G are zero
@@ -173,21 +282,30 @@ __global__ void __launch_bounds__(kAThreads) attn_piece_kernel(const __grid_cons
         if (lane == 0) hfac[h] = ldexpf(p.qk_scale, -e);
     }
 
-    float m_run[NT][2], l_run[NT][2], acc[MT][NT][4];
+    // Each warp runs its own online softmax over its 16 positions of every sub-piece
+    // (positions 16 warp + [0, 16)) and its own weighted V sum over all hd dims; the four
+    // warps' states merge once, at the end. Lane (gid, tig) holds heads 8 j + 2 tig + e.
+    constexpr int DT = HD / 16;  // 16-dim tiles of the weighted V sum
+    float m_run[NT][2], l_run[NT][2], acc[DT][NT][4];
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
         m_run[j][0] = m_run[j][1] = -INFINITY;
-        l_run[j][0] = l_run[j][1] = 0.f;
+        l_run[j][0] = l_run[j][1] = 0.f;  // this lane's positions' weights (summed at the end)
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
+        for (int dt = 0; dt < DT; ++dt)
 #pragma unroll
-            for (int k = 0; k < 4; ++k) acc[mt][j][k] = 0.f;
+            for (int k = 0; k < 4; ++k) acc[dt][j][k] = 0.f;
     }
 
     for (int i = 0; i < nsub; ++i) {
-        cp_async_wait<1>();  // this thread's copies of sub-piece i have landed
-        __syncthreads();     // everyone's; and sub-piece i - 1 is fully consumed
-        issue(i + 2);
+        if constexpr (TMA) {
+            if (!mbar_wait_bounded(&fullb[i % kAStages], (uint32_t)((i / kAStages) & 1), nullptr) && tid == 0)
+                raise_flag(p.dev_err, DEVFLAG_TIMEOUT);
+        } else {
+            cp_async_wait<kAStages - 2>();  // this thread's copies of sub-piece i have landed
+        }
+        __syncthreads();  // everyone's; and sub-piece i - 1 is fully consumed
+        issue(i + kAStages - 1);
         const int st = i % kAStages;
         const uint8_t* ks = kring + st * kSP * RP;
         const uint8_t* vs = vring + st * kSP * RP;
@@ -200,11 +318,11 @@ __global__ void __launch_bounds__(kAThreads) attn_piece_kernel(const __grid_cons
         for (int j = 0; j < NT; ++j)
 #pragma unroll
             for (int k = 0; k < 4; ++k) sc[j][k] = 0.f;
-        const uint8_t* kr0 = ks + (16 * warp + gid) * RP + 4 * tig;
+        const int kr = 16 * warp + gid;
 #pragma unroll
         for (int c = 0; c < KC; ++c) {
-            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(kr0 + 16 * c);
-            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(kr0 + 8 * RP + 16 * c);
+            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(ks + chunk_at(kr, c) + 4 * tig);
+            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(ks + chunk_at(kr + 8, c) + 4 * tig);
             const uint32_t a0 = e4m3x2_to_f16x2((uint16_t)(w0 & 0xFFFFu));
             const uint32_t a2 = e4m3x2_to_f16x2((uint16_t)(w0 >> 16));
             const uint32_t a1 = e4m3x2_to_f16x2((uint16_t)(w1 & 0xFFFFu));
@@ -215,146 +333,125 @@ __global__ void __launch_bounds__(kAThreads) attn_piece_kernel(const __grid_cons
                 mma_f16_16816(sc[j], a0, a1, a2, a3, b.x, b.y);
             }
         }
-        // scale per head; rows that are not readable score -inf
+        // scale per head; rows that are not readable score -inf. The warp's running
+        // maximum per head; weights exp(s - max) rounded to f16 (the same rounded weights
+        // in the sum of exps), packed per position as (head 2 tig, head 2 tig + 1) and
+        // transposed (movmatrix) into the B fragments of the V sum: (positions, head gid)
         const bool v0 = valid[st * kSP + 16 * warp + gid] != 0;
         const bool v1 = valid[st * kSP + 16 * warp + gid + 8] != 0;
-        float mloc[NT][2];
+        uint32_t bp[NT][2];
 #pragma unroll
-        for (int j = 0; j < NT; ++j)
+        for (int j = 0; j < NT; ++j) {
+            uint16_t wl[2], wh[2];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const float f = hfac[8 * j + 2 * tig + e];
-                sc[j][e] = v0 ? sc[j][e] * f : -INFINITY;
-                sc[j][2 + e] = v1 ? sc[j][2 + e] * f : -INFINITY;
-                float m = fmaxf(sc[j][e], sc[j][2 + e]);
+                const float s0 = v0 ? sc[j][e] * f : -INFINITY;
+                const float s1 = v1 ? sc[j][2 + e] * f : -INFINITY;
+                float m = fmaxf(s0, s1);
 #pragma unroll
                 for (int o = 4; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                mloc[j][e] = m;
-            }
-        if (gid == 0)
-#pragma unroll
-            for (int j = 0; j < NT; ++j)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) redm[warp * kAMaxGroup + 8 * j + 2 * tig + e] = mloc[j][e];
-        __syncthreads();
-        // the new running maximum; weights exp(s - max) as f16 into shared memory
-        // ([head][position]); their sum per warp
-        float alpha[NT][2];
-#pragma unroll
-        for (int j = 0; j < NT; ++j)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int h = 8 * j + 2 * tig + e;
-                const float msub = fmaxf(fmaxf(redm[h], redm[kAMaxGroup + h]),
-                                         fmaxf(redm[2 * kAMaxGroup + h], redm[3 * kAMaxGroup + h]));
-                const float mnew = fmaxf(m_run[j][e], msub);
-                alpha[j][e] = (m_run[j][e] == -INFINITY) ? 0.f : expf(m_run[j][e] - mnew);
+                const float mnew = fmaxf(m_run[j][e], m);
+                const float alpha = (m_run[j][e] == -INFINITY) ? 0.f : expf(m_run[j][e] - mnew);
                 m_run[j][e] = mnew;
-                float lsum = 0.f;
+                const float w0 = (s0 == -INFINITY) ? 0.f : expf(s0 - mnew);
+                const float w1 = (s1 == -INFINITY) ? 0.f : expf(s1 - mnew);
+                const uint32_t hw = f32x2_to_f16x2(w0, w1);  // (position gid, position gid + 8)
+                wl[e] = (uint16_t)(hw & 0xFFFFu);
+                wh[e] = (uint16_t)(hw >> 16);
+                const float2 wf = f16x2_to_f32x2(hw);
+                l_run[j][e] = l_run[j][e] * alpha + (wf.x + wf.y);
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const float s = sc[j][2 * half + e];
-                    const float w = (s == -INFINITY) ? 0.f : expf(s - mnew);
-                    const uint16_t wh = (uint16_t)(f32x2_to_f16x2(w, 0.f) & 0xFFFFu);
-                    wsm[h * kWPitch + 16 * warp + gid + 8 * half] = wh;
-                    lsum += f16x2_to_f32x2((uint32_t)wh).x;
-                }
-#pragma unroll
-                for (int o = 4; o < 32; o <<= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-                if (gid == 0) redl[warp * kAMaxGroup + h] = lsum;
-            }
-        __syncthreads();
-#pragma unroll
-        for (int j = 0; j < NT; ++j)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int h = 8 * j + 2 * tig + e;
-                const float ls = (redl[h] + redl[kAMaxGroup + h]) + (redl[2 * kAMaxGroup + h] + redl[3 * kAMaxGroup + h]);
-                l_run[j][e] = l_run[j][e] * alpha[j][e] + ls;
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-                    acc[mt][j][e] *= alpha[j][e];
-                    acc[mt][j][2 + e] *= alpha[j][e];
+                for (int dt = 0; dt < DT; ++dt) {
+                    acc[dt][j][e] *= alpha;
+                    acc[dt][j][2 + e] *= alpha;
                 }
             }
-        // the weighted V sum of dims warp * HD/4 + [0, HD/4): V^T (A) . W^T (B). The M
-        // dimension is permuted (vdim below gives the dim of each tile row), so that a
-        // thread's dims are one 16-bit load (one 16-dim tile) or one 32-bit load (a pair
-        // of tiles) per position
+            bp[j][0] = movmatrix_trans((uint32_t)wl[0] | ((uint32_t)wl[1] << 16));
+            bp[j][1] = movmatrix_trans((uint32_t)wh[0] | ((uint32_t)wh[1] << 16));
+        }
+        // the weighted V sum over the warp's 16 positions, all dims: V^T (A) . W^T (B). The
+        // M dimension is permuted: tile 2 mp + u has dim 32 mp + 4 gid + 2 u in row gid and
+        // the next dim in row gid + 8, so a thread's dims are one 32-bit load per position
+        const int pr = 16 * warp + 2 * tig;  // positions pr, pr + 1, pr + 8, pr + 9
 #pragma unroll
-        for (int kk = 0; kk < kSP / 16; ++kk) {
-            const int pr = 16 * kk + 2 * tig;  // positions pr, pr + 1, pr + 8, pr + 9
-            uint32_t b[NT][2];
+        for (int mp = 0; mp < HD / 32; ++mp) {
+            const int vc = 2 * mp + (gid >> 2), vo = 4 * (gid & 3);  // chunk, byte in it
+            const uint32_t y0 = *reinterpret_cast<const uint32_t*>(vs + chunk_at(pr, vc) + vo);
+            const uint32_t y1 = *reinterpret_cast<const uint32_t*>(vs + chunk_at(pr + 1, vc) + vo);
+            const uint32_t y8 = *reinterpret_cast<const uint32_t*>(vs + chunk_at(pr + 8, vc) + vo);
+            const uint32_t y9 = *reinterpret_cast<const uint32_t*>(vs + chunk_at(pr + 9, vc) + vo);
 #pragma unroll
-            for (int j = 0; j < NT; ++j) {
-                b[j][0] = *reinterpret_cast<const uint32_t*>(wsm + (8 * j + gid) * kWPitch + pr);
-                b[j][1] = *reinterpret_cast<const uint32_t*>(wsm + (8 * j + gid) * kWPitch + pr + 8);
-            }
-            if constexpr (MT % 2 == 0) {
+            for (int u = 0; u < 2; ++u) {
+                const uint32_t s0 = 0x0040u + 0x0022u * u, s1 = s0 + 0x0011u;
+                const uint32_t a0 = e4m3x2_to_f16x2((uint16_t)__byte_perm(y0, y1, s0));
+                const uint32_t a1 = e4m3x2_to_f16x2((uint16_t)__byte_perm(y0, y1, s1));
+                const uint32_t a2 = e4m3x2_to_f16x2((uint16_t)__byte_perm(y8, y9, s0));
+                const uint32_t a3 = e4m3x2_to_f16x2((uint16_t)__byte_perm(y8, y9, s1));
 #pragma unroll
-                for (int mp = 0; mp < MT / 2; ++mp) {  // tiles 2 mp, 2 mp + 1: dims d4 .. d4 + 3
-                    const int d4 = warp * (HD / 4) + 32 * mp + 4 * gid;
-                    const uint32_t y0 = *reinterpret_cast<const uint32_t*>(vs + pr * RP + d4);
-                    const uint32_t y1 = *reinterpret_cast<const uint32_t*>(vs + (pr + 1) * RP + d4);
-                    const uint32_t y8 = *reinterpret_cast<const uint32_t*>(vs + (pr + 8) * RP + d4);
-                    const uint32_t y9 = *reinterpret_cast<const uint32_t*>(vs + (pr + 9) * RP + d4);
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {  // dims d4 + 2u (row g), d4 + 2u + 1 (row g + 8)
-                        const uint32_t s0 = 0x0040u + 0x0022u * u, s1 = s0 + 0x0011u;
-                        const uint32_t a0 = e4m3x2_to_f16x2((uint16_t)__byte_perm(y0, y1, s0));
-                        const uint32_t a1 = e4m3x2_to_f16x2((uint16_t)__byte_perm(y0, y1, s1));
-                        const uint32_t a2 = e4m3x2_to_f16x2((uint16_t)__byte_perm(y8, y9, s0));
-                        const uint32_t a3 = e4m3x2_to_f16x2((uint16_t)__byte_perm(y8, y9, s1));
-#pragma unroll
-                        for (int j = 0; j < NT; ++j)
-                            mma_f16_16816(acc[2 * mp + u][j], a0, a1, a2, a3, b[j][0], b[j][1]);
-                    }
-                }
-            } else {
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {  // dims d0 (row g), d0 + 1 (row g + 8)
-                    const int d0 = warp * (HD / 4) + 16 * mt + 2 * gid;
-                    const uint32_t x0 = *reinterpret_cast<const uint16_t*>(vs + pr * RP + d0);
-                    const uint32_t x1 = *reinterpret_cast<const uint16_t*>(vs + (pr + 1) * RP + d0);
-                    const uint32_t x8 = *reinterpret_cast<const uint16_t*>(vs + (pr + 8) * RP + d0);
-                    const uint32_t x9 = *reinterpret_cast<const uint16_t*>(vs + (pr + 9) * RP + d0);
-                    const uint32_t lo = x0 | (x1 << 16), hi = x8 | (x9 << 16);
-                    const uint32_t a0 = e4m3x2_to_f16x2((uint16_t)__byte_perm(lo, 0, 0x0020));
-                    const uint32_t a1 = e4m3x2_to_f16x2((uint16_t)__byte_perm(lo, 0, 0x0031));
-                    const uint32_t a2 = e4m3x2_to_f16x2((uint16_t)__byte_perm(hi, 0, 0x0020));
-                    const uint32_t a3 = e4m3x2_to_f16x2((uint16_t)__byte_perm(hi, 0, 0x0031));
-#pragma unroll
-                    for (int j = 0; j < NT; ++j) mma_f16_16816(acc[mt][j], a0, a1, a2, a3, b[j][0], b[j][1]);
-                }
+                for (int j = 0; j < NT; ++j) mma_f16_16816(acc[2 * mp + u][j], a0, a1, a2, a3, bp[j][0], bp[j][1]);
             }
         }
     }
 
-    // this CTA's partials: (max, sum) per head, then its dims of the weighted V sums; tile
-    // mt's row g holds dim vdim(mt), row g + 8 dim vdim(mt) + 1
-    auto vdim = [&](int mt) {
-        return MT % 2 == 0 ? warp * (HD / 4) + 32 * (mt / 2) + 4 * gid + 2 * (mt % 2)
-                           : warp * (HD / 4) + 16 * mt + 2 * gid;
-    };
-    const int64_t rs = (int64_t)HD + 2;
+    // merge the four warps (fixed order) into this CTA's partials: per head the largest
+    // warp maximum M, sum_w e^(m_w - M) l_w and sum_w e^(m_w - M) acc_w; tile dt's row gid
+    // holds dim vdim(dt), row gid + 8 dim vdim(dt) + 1
+    auto vdim = [&](int dt) { return 32 * (dt / 2) + 4 * gid + 2 * (dt % 2); };
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) l_run[j][e] += __shfl_xor_sync(0xffffffffu, l_run[j][e], o);
+    __syncthreads();  // every warp is past the ring: it holds the warps' sums from here
+    float* accs = reinterpret_cast<float*>(kring);  // [4 warps][kAMaxGroup heads][HD]
+    if (gid == 0)
+#pragma unroll
+        for (int j = 0; j < NT; ++j)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                redm[warp * kAMaxGroup + 8 * j + 2 * tig + e] = m_run[j][e];
+                redl[warp * kAMaxGroup + 8 * j + 2 * tig + e] = l_run[j][e];
+            }
+    __syncthreads();
 #pragma unroll
     for (int j = 0; j < NT; ++j)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const int h = 8 * j + 2 * tig + e;
-            if (h >= G) continue;
-            float* dst = p.part + ((int64_t)piece * p.nq + g * G + h) * rs;
-            if (warp == 0 && gid == 0) {
-                dst[0] = m_run[j][e];
-                dst[1] = l_run[j][e];
-            }
+            const float M = fmaxf(fmaxf(redm[h], redm[kAMaxGroup + h]),
+                                  fmaxf(redm[2 * kAMaxGroup + h], redm[3 * kAMaxGroup + h]));
+            const float f = (m_run[j][e] == -INFINITY) ? 0.f : expf(m_run[j][e] - M);
+            float* dst = accs + (warp * kAMaxGroup + h) * HD;
 #pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-                const int d0 = vdim(mt);
-                dst[2 + d0] = acc[mt][j][e];
-                dst[2 + d0 + 1] = acc[mt][j][2 + e];
+            for (int dt = 0; dt < DT; ++dt) {
+                const int d0 = vdim(dt);
+                dst[d0] = acc[dt][j][e] * f;
+                dst[d0 + 1] = acc[dt][j][2 + e] * f;
             }
         }
+    __syncthreads();
+    const int64_t rs = (int64_t)HD + 2;
+    for (int idx = tid; idx < G * HD; idx += kAThreads) {
+        const int h = idx / HD, d = idx - h * HD;
+        const float v = ((accs[h * HD + d] + accs[(kAMaxGroup + h) * HD + d]) +
+                         accs[(2 * kAMaxGroup + h) * HD + d]) +
+                        accs[(3 * kAMaxGroup + h) * HD + d];
+        p.part[((int64_t)piece * p.nq + g * G + h) * rs + 2 + d] = v;
+    }
+    for (int h = tid; h < G; h += kAThreads) {
+        float M = -INFINITY;
+        for (int w = 0; w < 4; ++w) M = fmaxf(M, redm[w * kAMaxGroup + h]);
+        float L = 0.f;
+        for (int w = 0; w < 4; ++w) {
+            const float mw = redm[w * kAMaxGroup + h];
+            L += (mw == -INFINITY) ? 0.f : expf(mw - M) * redl[w * kAMaxGroup + h];
+        }
+        float* dst = p.part + ((int64_t)piece * p.nq + g * G + h) * rs;
+        dst[0] = M;
+        dst[1] = L;
+    }
 }
 
 // One CTA per query head: out = sum_s e^(m_s - M) acc_s / sum_s e^(m_s - M) l_s (zero
@@ -435,14 +532,47 @@ size_t attn_ws_bytes(int nq, int hd, int64_t seq_len) {
     return (size_t)(pieces < 1 ? 1 : pieces) * (size_t)nq * (size_t)(hd + 2) * sizeof(float);
 }
 
-template <int HD, int NT>
-cudaError_t launch_pieces(const AttnParams& p, cudaStream_t s) {
-    constexpr size_t smem = attn_smem_bytes<HD>();
-    auto kern = attn_piece_kernel<HD, NT>;
+template <int HD, int NT, bool TMA>
+cudaError_t launch_pieces(const AttnParams& p, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                          cudaStream_t s) {
+    constexpr size_t smem = attn_smem_bytes<HD, TMA>();
+    auto kern = attn_piece_kernel<HD, NT, TMA>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<dim3((unsigned)p.nkv, (unsigned)p.pieces), kAThreads, smem, s>>>(p);
+    kern<<<dim3((unsigned)p.nkv, (unsigned)p.pieces), kAThreads, smem, s>>>(p, kmap, vmap);
     return cudaGetLastError();
+}
+
+typedef CUresult (*AttnEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                 CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                 CUtensorMapFloatOOBfill);
+
+AttnEncodeFn attn_encode_fn() {
+    static AttnEncodeFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<AttnEncodeFn>(f);
+    });
+    return fn;
+}
+
+// A cache [num_blocks * block_size rows][nkv][128] E4M3 as a 3-D tensor (byte of the head
+// row, kv head, cache row); boxes of 128 bytes x 1 head x 16 rows, 128-byte swizzle.
+bool attn_cache_map(CUtensorMap* m, const uint8_t* base, int nkv, int64_t rows) {
+    AttnEncodeFn fn = attn_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {128, (cuuint64_t)nkv, (cuuint64_t)rows};
+    cuuint64_t strides[2] = {128, (cuuint64_t)nkv * 128};
+    cuuint32_t box[3] = {128, 1, 16};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 cudaError_t attn_launch(const uint16_t* q, int nq, int nkv, int hd, const uint8_t* k_cache,
@@ -473,9 +603,19 @@ cudaError_t attn_launch(const uint16_t* q, int nq, int nkv, int hd, const uint8_
     cudaError_t e;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    // tensor copies for 128-dim heads in blocks of a multiple of 16 rows (16-byte aligned
+    // caches, cache rows addressable as 32-bit coordinates); 16-byte copies otherwise
+    CUtensorMap kmap{}, vmap{};
+    const int64_t cache_rows = num_blocks * (int64_t)block_size;
+    const bool tma = hd == 128 && block_size % 16 == 0 && cache_rows < ((int64_t)1 << 31) &&
+                     (reinterpret_cast<uintptr_t>(k_cache) & 15) == 0 &&
+                     (reinterpret_cast<uintptr_t>(v_cache) & 15) == 0 &&
+                     attn_cache_map(&kmap, k_cache, nkv, cache_rows) &&
+                     attn_cache_map(&vmap, v_cache, nkv, cache_rows);
     // as many CTAs as fit on the SMs at once (shared memory bound, at most four per SM)
-    const size_t smem = hd == 64 ? attn_smem_bytes<64>() : hd == 128 ? attn_smem_bytes<128>()
-                                                                      : attn_smem_bytes<256>();
+    const size_t smem = tma ? attn_smem_bytes<128, true>()
+                            : hd == 64 ? attn_smem_bytes<64, false>()
+                                       : hd == 128 ? attn_smem_bytes<128, false>() : attn_smem_bytes<256, false>();
     int per_sm = (int)((size_t)227 * 1024 / smem);
     per_sm = per_sm < 1 ? 1 : per_sm > 4 ? 4 : per_sm;
     int64_t pieces = ((int64_t)per_sm * sms + nkv - 1) / nkv;
@@ -485,9 +625,10 @@ cudaError_t attn_launch(const uint16_t* q, int nq, int nkv, int hd, const uint8_
     p.per_piece = (int64_t)kSP * ((subs + pieces - 1) / pieces);
     p.pieces = (int)((seq_len + p.per_piece - 1) / p.per_piece);
     const bool two = p.group > 8;
-    if (hd == 64) e = two ? launch_pieces<64, 2>(p, s) : launch_pieces<64, 1>(p, s);
-    else if (hd == 128) e = two ? launch_pieces<128, 2>(p, s) : launch_pieces<128, 1>(p, s);
-    else e = two ? launch_pieces<256, 2>(p, s) : launch_pieces<256, 1>(p, s);
+    if (tma) e = two ? launch_pieces<128, 2, true>(p, kmap, vmap, s) : launch_pieces<128, 1, true>(p, kmap, vmap, s);
+    else if (hd == 64) e = two ? launch_pieces<64, 2, false>(p, kmap, vmap, s) : launch_pieces<64, 1, false>(p, kmap, vmap, s);
+    else if (hd == 128) e = two ? launch_pieces<128, 2, false>(p, kmap, vmap, s) : launch_pieces<128, 1, false>(p, kmap, vmap, s);
+    else e = two ? launch_pieces<256, 2, false>(p, kmap, vmap, s) : launch_pieces<256, 1, false>(p, kmap, vmap, s);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)nq);

@@ -71,3 +71,29 @@ def test_attention_over_the_prefill_cache(orc):
     ref, _ = orc.paged_decode_attn(q, 4, kcn, vcn, bt, 16, nb, 1000)
     assert err == 0
     assert_close(got, ref, "prefill cache")
+
+
+@pytest.mark.parametrize("bs,seq", [(32, 777), (64, 1000), (8, 333)])
+def test_attention_block_sizes(orc, bs, seq):
+    """Blocks of 32 and 64 rows (several 16-row copies inside one block) and of 8 rows (the
+    16-byte copy path)."""
+    q, kc, vc, bt, nb = case(orc, 11 + bs, 16, 2, 128, seq, bs=bs)
+    got, err = run(q, 2, kc, vc, bt, seq)
+    ref, flags = orc.paged_decode_attn(q, 2, kc, vc, bt, bs, nb, seq)
+    assert err == 0 and flags == 0
+    assert_close(got, ref, f"block size {bs}")
+
+
+def test_attention_nan_past_the_end(orc):
+    """Rows past the sequence inside its last block hold the E4M3 NaN code in K and V: they
+    are never read (a finite output equal to the oracle's, which reads rows < seq_len)."""
+    seq = 70  # the last block holds rows 64 .. 69 of the sequence and 10 more
+    q, kc, vc, bt, nb = case(orc, 5, 16, 2, 128, seq)
+    for pos in range(seq, (seq // 16 + 1) * 16):
+        kc[bt[pos // 16], pos % 16] = 0x7F
+        vc[bt[pos // 16], pos % 16] = 0x7F
+    got, err = run(q, 2, kc, vc, bt, seq)
+    ref, _ = orc.paged_decode_attn(q, 2, kc, vc, bt, 16, nb, seq)
+    assert err == 0
+    assert np.all(np.isfinite(got))
+    assert_close(got, ref, "NaN rows past the end")
