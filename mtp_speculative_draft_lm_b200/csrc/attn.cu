@@ -12,20 +12,21 @@
 //
 // Design (B200, HBM-bound: every cached K and V byte is read once): CTA (g, piece) takes
 // kv head g over a contiguous range of positions (as many CTAs as the SMs hold at once), in
-// sub-pieces of 64 positions that a three-stage ring of 16-byte asynchronous copies
-// brings into shared memory (rows of a missing block zero-filled). Warp w owns positions
+// sub-pieces of 64 positions that a three-stage ring brings into shared memory: tensor
+// copies of 16 cache rows (128-dim heads, blocks of a multiple of 16 rows), else 16-byte
+// asynchronous copies; rows of a missing block are zero-filled. Warp w owns positions
 // 16 w + [0, 16) of every sub-piece and runs its own online softmax (fp32 running maximum
 // and sum per query head) and its own weighted V sum over all head dims, so the warps
 // meet once per sub-piece (the ring) and once at the end. Both contractions run on the
 // tensor cores (mma.sync m16n8k16, f16 operands, fp32 accumulators): the scores as
 // K[16 positions, hd] . Q^T, with E4M3 K decoded exactly to f16 and each query head in
-// f16 scaled by a power of two (exact); the weights exp(s - max) in (0, 1] rounded to f16
-// (the same rounded weights in the sum of exps) go from the score accumulators to the B
-// operand of V^T . W^T in registers (an 8 x 8 transpose, movmatrix). At the end the four
-// warps' states merge in a fixed order into the CTA's (max, sum, weighted V sum) per head;
-// a second kernel merges the pieces of each head in a fixed order (deterministic) and
-// writes bf16. Rows whose block is missing or out of range are skipped and set
-// MTP_DEVFLAG_BAD_SLOT.
+// f16 scaled by a power of two (exact); the weights exp(s - max) in (0, 1] (the hardware
+// exponential) rounded to f16 (the same rounded weights in the sum of exps) go from the
+// score accumulators to the B operand of V^T . W^T in registers (an 8 x 8 transpose,
+// movmatrix). At the end the four warps' states merge in a fixed order into the CTA's
+// (max, sum, weighted V sum) per head; a second kernel merges the pieces of each head in a
+// fixed order (deterministic) and writes bf16. Rows whose block is missing or out of range
+// are skipped and set MTP_DEVFLAG_BAD_SLOT.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -352,10 +353,12 @@ __global__ void __launch_bounds__(kAThreads) attn_piece_kernel(const __grid_cons
 #pragma unroll
                 for (int o = 4; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
                 const float mnew = fmaxf(m_run[j][e], m);
-                const float alpha = (m_run[j][e] == -INFINITY) ? 0.f : expf(m_run[j][e] - mnew);
+                // (the hardware exponential: its ~1e-6 relative error is far below the f16
+                // rounding of the weights)
+                const float alpha = (m_run[j][e] == -INFINITY) ? 0.f : __expf(m_run[j][e] - mnew);
                 m_run[j][e] = mnew;
-                const float w0 = (s0 == -INFINITY) ? 0.f : expf(s0 - mnew);
-                const float w1 = (s1 == -INFINITY) ? 0.f : expf(s1 - mnew);
+                const float w0 = (s0 == -INFINITY) ? 0.f : __expf(s0 - mnew);
+                const float w1 = (s1 == -INFINITY) ? 0.f : __expf(s1 - mnew);
                 const uint32_t hw = f32x2_to_f16x2(w0, w1);  // (position gid, position gid + 8)
                 wl[e] = (uint16_t)(hw & 0xFFFFu);
                 wh[e] = (uint16_t)(hw >> 16);
