@@ -457,25 +457,27 @@ __global__ void __launch_bounds__(kAThreads) attn_piece_kernel(const __grid_cons
     }
 }
 
+constexpr int kMThreads = 1024;  // merge: hd-thread groups, each a share of the pieces
+
 // One CTA per query head: out = sum_s e^(m_s - M) acc_s / sum_s e^(m_s - M) l_s (zero
 // when no row was readable), as bf16. The pieces' (max, sum) pairs are loaded in parallel
 // and folded from shared memory in a fixed order; the dimensions' sums over the pieces
-// are split over 256 / hd thread groups (eight loads in flight each) and added in order.
-__global__ void __launch_bounds__(kAMaxHd) attn_merge_kernel(const __grid_constant__ AttnParams p) {
+// are split over 1024 / hd thread groups (eight loads in flight each) and added in order.
+__global__ void __launch_bounds__(kMThreads) attn_merge_kernel(const __grid_constant__ AttnParams p) {
     __shared__ float msm[kAMaxPieces];
     __shared__ float lsm[kAMaxPieces];
     __shared__ float fac[kAMaxPieces];
-    __shared__ float accp[kAMaxHd];  // [parts][hd]
-    __shared__ float red[kAMaxHd / 32];
+    __shared__ float accp[kMThreads];  // [parts][hd]
+    __shared__ float red[kMThreads / 32];
     __shared__ float tot[2];
     const int i = blockIdx.x, t = threadIdx.x, hd = p.hd;
     const int lane = t & 31, warp = t >> 5;
-    const int parts = kAMaxHd / hd, d = t % hd, part = t / hd;  // 1, 2 or 4 parts of the pieces
+    const int parts = kMThreads / hd, d = t % hd, part = t / hd;  // 4, 8 or 16 parts of the pieces
     pdl_wait();
     const int64_t rs = (int64_t)p.nq * (hd + 2);  // floats between a head's pieces
     const float* base = p.part + (int64_t)i * (hd + 2);
     float mloc = -INFINITY;
-    for (int s = t; s < p.pieces; s += kAMaxHd) {
+    for (int s = t; s < p.pieces; s += kMThreads) {
         msm[s] = base[s * rs];
         lsm[s] = base[s * rs + 1];
         mloc = fmaxf(mloc, msm[s]);
@@ -486,8 +488,8 @@ __global__ void __launch_bounds__(kAMaxHd) attn_merge_kernel(const __grid_consta
     __syncthreads();
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kAMaxHd / 32; ++w) M = fmaxf(M, red[w]);
-    for (int s = t; s < p.pieces; s += kAMaxHd)
+    for (int w = 0; w < kMThreads / 32; ++w) M = fmaxf(M, red[w]);
+    for (int s = t; s < p.pieces; s += kMThreads)
         fac[s] = (M == -INFINITY || msm[s] == -INFINITY) ? 0.f : expf(msm[s] - M);
     __syncthreads();
     if (warp == 0) {  // the denominator: lane-strided partial sums, then a fixed shuffle tree
@@ -635,7 +637,7 @@ cudaError_t attn_launch(const uint16_t* q, int nq, int nkv, int hd, const uint8_
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)nq);
-    cfg.blockDim = dim3(kAMaxHd);
+    cfg.blockDim = dim3(kMThreads);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
