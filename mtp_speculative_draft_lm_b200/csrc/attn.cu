@@ -266,21 +266,55 @@ __global__ void __launch_bounds__(kAThreads) attn_piece_kernel(const __grid_cons
     for (int i = 0; i < kAStages - 1; ++i) issue(i);
 
     // the group's query heads in f16, each scaled by 2^e so its largest |q| lies in
-    // [2^14, 2^15) (exact: a bf16 value has 8 significant bits); heads past G are zero
-    for (int h = warp; h < kAMaxGroup; h += kAThreads / 32) {
-        float mx = 0.f;
-        if (h < G)
-            for (int d = lane; d < HD; d += 32)
-                mx = fmaxf(mx, fabsf(bf16_to_f32(p.q[(int64_t)(g * G + h) * HD + d])));
+    // [2^14, 2^15) (exact: a bf16 value has 8 significant bits); heads past G are zero.
+    // Warp w takes heads 4 w .. 4 w + 3: lane l holds 8 dims of head 4 w + k HPL + l / LH,
+    // all loads issued at once, each head's maximum folded over its LH lanes (q 16-byte
+    // aligned; else one head at a time)
+    if ((reinterpret_cast<uintptr_t>(p.q) & 15u) == 0) {
+        constexpr int LH = HD / 8, HPL = 32 / LH, NL = 4 / HPL;
+        static_assert(kAMaxGroup == 4 * (kAThreads / 32) && 4 % HPL == 0, "four heads per warp");
+        uint4 qr[NL];
 #pragma unroll
-        for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        int e = 0;
-        if (mx > 0.f) e = 14 - ilogbf(mx);
-        for (int d = lane; d < HD; d += 32) {
-            const float v = h < G ? ldexpf(bf16_to_f32(p.q[(int64_t)(g * G + h) * HD + d]), e) : 0.f;
-            qh[h * QP + d] = (uint16_t)(f32x2_to_f16x2(v, 0.f) & 0xFFFFu);
+        for (int k = 0; k < NL; ++k) {
+            const int h = 4 * warp + k * HPL + lane / LH;
+            qr[k] = h < G ? *reinterpret_cast<const uint4*>(p.q + (int64_t)(g * G + h) * HD + 8 * (lane % LH))
+                          : make_uint4(0, 0, 0, 0);
         }
-        if (lane == 0) hfac[h] = ldexpf(p.qk_scale, -e);
+#pragma unroll
+        for (int k = 0; k < NL; ++k) {
+            const int h = 4 * warp + k * HPL + lane / LH;
+            const uint32_t w[4] = {qr[k].x, qr[k].y, qr[k].z, qr[k].w};
+            float mx = 0.f;
+#pragma unroll
+            for (int t = 0; t < 4; ++t) mx = fmaxf(mx, fmaxf(fabsf(bf16_lo(w[t])), fabsf(bf16_hi(w[t]))));
+#pragma unroll
+            for (int o = LH / 2; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            int e = 0;
+            if (mx > 0.f) e = 14 - ilogbf(mx);
+            uint4 o4;
+            o4.x = f32x2_to_f16x2(ldexpf(bf16_lo(w[0]), e), ldexpf(bf16_hi(w[0]), e));
+            o4.y = f32x2_to_f16x2(ldexpf(bf16_lo(w[1]), e), ldexpf(bf16_hi(w[1]), e));
+            o4.z = f32x2_to_f16x2(ldexpf(bf16_lo(w[2]), e), ldexpf(bf16_hi(w[2]), e));
+            o4.w = f32x2_to_f16x2(ldexpf(bf16_lo(w[3]), e), ldexpf(bf16_hi(w[3]), e));
+            *reinterpret_cast<uint4*>(qh + h * QP + 8 * (lane % LH)) = o4;
+            if (lane % LH == 0) hfac[h] = ldexpf(p.qk_scale, -e);
+        }
+    } else {
+        for (int h = warp; h < kAMaxGroup; h += kAThreads / 32) {
+            float mx = 0.f;
+            if (h < G)
+                for (int d = lane; d < HD; d += 32)
+                    mx = fmaxf(mx, fabsf(bf16_to_f32(p.q[(int64_t)(g * G + h) * HD + d])));
+#pragma unroll
+            for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            int e = 0;
+            if (mx > 0.f) e = 14 - ilogbf(mx);
+            for (int d = lane; d < HD; d += 32) {
+                const float v = h < G ? ldexpf(bf16_to_f32(p.q[(int64_t)(g * G + h) * HD + d]), e) : 0.f;
+                qh[h * QP + d] = (uint16_t)(f32x2_to_f16x2(v, 0.f) & 0xFFFFu);
+            }
+            if (lane == 0) hfac[h] = ldexpf(p.qk_scale, -e);
+        }
     }
 
     // Each warp runs its own online softmax over its 16 positions of every sub-piece

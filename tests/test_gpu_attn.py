@@ -97,3 +97,18 @@ def test_attention_nan_past_the_end(orc):
     assert err == 0
     assert np.all(np.isfinite(got))
     assert_close(got, ref, "NaN rows past the end")
+
+
+def test_attention_unaligned_query(orc):
+    """q only 2-byte aligned (a view one element into a buffer): the per-head staging."""
+    q, kc, vc, bt, nb = case(orc, 9, 16, 2, 128, 300)
+    buf = torch.empty((q.size + 1,), dtype=torch.bfloat16, device="cuda")
+    buf[1:] = to_dev_u16(q).reshape(-1)
+    qd = buf[1:].reshape(q.shape)
+    assert qd.data_ptr() % 16 == 2
+    err = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    out, _ = api.paged_decode_attn(qd, 2, to_dev(kc), to_dev(vc), to_dev(bt), 300, dev_err=err)
+    torch.cuda.synchronize()
+    ref, _ = orc.paged_decode_attn(q, 2, kc, vc, bt, 16, nb, 300)
+    assert int(err.item()) == 0
+    assert_close(bf16_bits_to_f64(u16_of(out)), ref, "unaligned q")
