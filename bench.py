@@ -34,7 +34,7 @@ FALLBACK_HBM_GBS = 6650.0
 # the sha256 of sweep.cu when it was captured; reported as null once the source changed.
 # bf16_M1: a full-size capture (one-pass metrics) of the headline sweep, the mean of two
 # launches: 1,268,870,144 + 128,256 and 1,268,873,728 + 133,632 B.
-NCU_TRAFFIC = {"bf16_M1": (1269002880, "e2d56e5da49d5793")}
+NCU_TRAFFIC = {"bf16_M1": (1269123712, "5ffd0495da62c93b")}
 
 
 def sweep_source_hash() -> str:
