@@ -43,7 +43,6 @@ constexpr int kSP = 64;          // positions per sub-piece (four warps x 16)
 constexpr int kAThreads = 128;
 constexpr int kAStages = 3;
 constexpr int kAMaxGroup = 16;  // query heads per kv head
-constexpr int kAMaxHd = 256;
 constexpr int kAMaxPieces = 1024;  // pieces per kv head (the merge keeps a factor per piece)
 
 struct AttnParams {
